@@ -1,0 +1,386 @@
+#!/usr/bin/env python
+"""Benchmark of the chunkwise gated-linear-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c3] [--impl ours|reference]
+
+One step = one pass of the whole path over one batch of synthetic input: gla_fwd then
+gla_bwd (workloads with a backward) through the library's C ABI. Default workload c3:
+GLA forward+backward, B=4 H=16 L=4096 Dk=128 Dv=256, bf16 I/O, per-key log-gate
+logsigmoid(N(0,1))/16, dO ~ N(0,1), chunk 64.
+
+Prints one JSON line on rank 0. `value` is whole-job tokens/s with inputs resident in
+HBM (CUDA events per step on the launching stream; the 256 MiB L2 flush between steps is
+outside the events); `e2e` is the same metric through the public Python API with host
+(pinned) tensors, host<->device copies inside the timed region. Under torchrun each rank
+runs its own batch (weak scaling, no data-path collective); the step time is the max over
+ranks. `--impl reference` times the float64 CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from linear_rnn_b200 import inputs as I  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ accounting
+def io_bytes(w):
+    return 2 if w.dtype == "bf16" else 4
+
+
+def gate_elems(w):
+    return {I.GATE_NONE: 0, I.GATE_PER_KEY: w.Dk, I.GATE_PER_HEAD: 1}[w.gate]
+
+
+def flops(w, backward):
+    """Algorithmic FLOPs: per token-head C*Dk + C*Dv + 4*Dk*Dv forward (causal-half intra
+    products, inter q~S, state K^T V) and C*(3Dk+2Dv) + 8*Dk*Dv backward."""
+    th = w.B * w.H * w.L
+    f = th * (w.chunk * w.Dk + w.chunk * w.Dv + 4 * w.Dk * w.Dv)
+    if backward:
+        f += th * (w.chunk * (3 * w.Dk + 2 * w.Dv) + 8 * w.Dk * w.Dv)
+    return float(f)
+
+
+def compulsory_bytes(w, backward):
+    """Read every input once and write every output once (chunk states are not compulsory)."""
+    th = w.B * w.H * w.L
+    e = io_bytes(w)
+    st = 4 * w.B * w.H * w.Dk * w.Dv
+    ig = 4 * th if w.input_gate else 0
+    fwd = th * (2 * w.Dk + w.Dv) * e + 4 * th * gate_elems(w) + ig + th * w.Dv * e + st
+    fwd += st if w.h0_std > 0 else 0
+    if not backward:
+        return float(fwd)
+    bwd = th * (2 * w.Dk + 2 * w.Dv) * e + 4 * th * gate_elems(w) + ig          # q k v dO g (i)
+    bwd += th * (2 * w.Dk + w.Dv) * e + 4 * th * gate_elems(w) + ig              # dq dk dv dg (di)
+    bwd += 2 * st if w.h0_std > 0 else 0                                         # h0, dh0
+    return float(fwd + bwd)
+
+
+def kernel_bytes(name, w):
+    """Algorithmic bytes of one launch of each kernel: its own inputs read once and its
+    outputs written once (workspace tensors it exchanges with other kernels included)."""
+    th = w.B * w.H * w.L
+    e = io_bytes(w)
+    ge = 4 * th * gate_elems(w)
+    N = math.ceil(w.L / w.chunk)
+    states = 4.0 * w.B * w.H * N * w.Dk * w.Dv
+    q = k = th * w.Dk * e
+    v = o = th * w.Dv * e
+    table = {
+        "simt_cumsum": 2 * ge,
+        "simt_state": k + v + ge + states,
+        "simt_out": q + k + v + ge + states + o,
+        "simt_dstate": q + o + ge + states,
+        "simt_dq": q + k + v + o + ge + states + q + 4 * th * w.Dk,
+        "simt_dk": q + k + v + o + ge + states + k + 2 * 4 * th * w.Dk,
+        "simt_dv": q + k + o + ge + states + v,
+        "simt_dg_key": 2 * 4 * th * w.Dk,
+        "tc_fwd": q + k + v + ge + o + 4 * w.B * w.H * w.Dk * w.Dv * (2 if w.h0_std > 0 else 1),
+    }
+    return float(table.get(name, 0.0))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons with nvidia-smi every 200 ms."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.error = None
+
+    def start(self):
+        try:
+            uuid = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+                uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            except Exception:
+                pass
+            sel = ["--id=" + uuid] if uuid else ["-i", str(self.dev)]
+            self.proc = subprocess.Popen(["nvidia-smi", *sel, "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception as ex:  # nvidia-smi missing
+            self.error = str(ex)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": self.error or "no sampler"}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[3:7]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle baseline
+def oracle_sample(w, seed, heads):
+    """Times the float64 oracle on `heads` whole heads (full L) of the workload.
+    Returns (tokens_equivalent, seconds, threads)."""
+    import oracle
+    sub = w.replace(B=1, H=heads)
+    x = I.make_inputs(sub, seed=seed)
+    t0 = time.perf_counter()
+    oracle.gla_fwd(x["q"], x["k"], x["v"], x["g"], x["igate"], x["h0"], w.scale)
+    if w.backward:
+        oracle.gla_bwd(x["q"], x["k"], x["v"], x["g"], x["igate"], x["h0"], x["dO"], None, w.scale)
+    dt = time.perf_counter() - t0
+    return w.L * heads / w.H, dt, oracle.num_threads()
+
+
+def oracle_heads(w):
+    # about 10-30 s of host work on a multi-core box; heads are the unit of parallelism
+    return max(1, min(w.B * w.H, 4 * (os.cpu_count() or 8)))
+
+
+# ------------------------------------------------------------------ main
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group(
+            "nccl" if torch.cuda.is_available() else "gloo", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def base_line(w, args, world):
+    return {"metric": "GLA chunkwise fwd/bwd tokens/s", "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded; workload recipe in DESIGN.md)",
+            "config": {"workload": f"{w.name}: {'GLA forward+backward' if w.backward else 'GLA forward'}, "
+                                   f"B={w.B} H={w.H} L={w.L} Dk={w.Dk} Dv={w.Dv} chunk={w.chunk} {w.dtype}",
+                       "global_batch": w.B * world, "seq_len": w.L, "parallelism": f"replicas x{world}",
+                       "l2": "256 MiB L2 flush between steps, outside the per-step events; inputs > L2"}}
+
+
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return
+    heads = max(1, oracle_heads(w) // 2)
+    for _ in range(args.warmup):
+        oracle_sample(w, 0, heads)
+    tok = 0.0
+    tot = 0.0
+    thr = 1
+    for i in range(args.steps):
+        t, dt, thr = oracle_sample(w, i, heads)
+        tok += t
+        tot += dt
+    val = tok / tot
+    line = base_line(w, args, 1)
+    line.update({"impl": "reference", "value": val, "ms_per_step": 1e3 * tot / args.steps, "dtype": "f64",
+                 "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                                  "sample": f"{heads} of {w.B * w.H} heads, full L={w.L}, "
+                                            f"{'fwd+bwd' if w.backward else 'fwd'} per step"},
+                 "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+                 "gpu_launches": 0})
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="c3", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--plan", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = I.WORKLOADS[args.workload]
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, w, world, rank)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    from linear_rnn_b200 import _lib, ops
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    x = I.make_inputs(w, seed=rank)
+    xd = {k: (None if v is None else v.to(dev)) for k, v in x.items()}
+    kw = dict(scale=w.scale, chunk=w.chunk, plan=args.plan)
+    prob = ops.make_problem(xd["q"], xd["v"], xd["g"], **kw)
+    ws = torch.empty(max(ops.gla_workspace_bytes(prob, False), ops.gla_workspace_bytes(prob, True) if w.backward
+                         else 0), dtype=torch.uint8, device=dev)
+
+    def step():
+        ops.gla_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["igate"], xd["h0"], workspace=ws, **kw)
+        if w.backward:
+            ops.gla_bwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["igate"], xd["h0"], xd["dO"], None, workspace=ws,
+                        **kw)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    n0 = _lib.launch_count()
+    _lib.profiler_enable(True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    _lib.profiler_enable(False)
+    launches = _lib.launch_count() - n0
+    kprof = _lib.profiler_read()
+    clocks = sampler.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    tokens = w.B * w.L * args.steps * world
+    value = tokens / (total_ms / 1e3)
+
+    # ------- end to end: host (pinned) tensors through the public API
+    e2e = None
+    if not args.no_e2e:
+        xh = {k: (None if v is None else v.pin_memory()) for k, v in x.items()}
+        h2d = sum(t.numel() * t.element_size() for n, t in xh.items()
+                  if t is not None and n in ("q", "k", "v", "g", "igate", "h0"))
+        d2h = 0
+
+        def e2e_step():
+            nonlocal d2h
+            o, hT = ops.gla_fwd(xh["q"], xh["k"], xh["v"], xh["g"], xh["igate"], xh["h0"], **kw)
+            nb = o.numel() * o.element_size() + hT.numel() * hT.element_size()
+            if w.backward:
+                r = ops.gla_bwd(xh["q"], xh["k"], xh["v"], xh["g"], xh["igate"], xh["h0"], xh["dO"], None, **kw)
+                nb += sum(t.numel() * t.element_size() for t in r.values() if t is not None)
+            d2h = nb
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(args.steps):
+            e2e_step()
+        s1.record()
+        torch.cuda.synchronize()
+        e_ms = s0.elapsed_time(s1)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(t.item())
+        h2d_step = h2d * (2 if w.backward else 1) + (sum(xh[n].numel() * xh[n].element_size() for n in ("dO",))
+                                                     if w.backward else 0)
+        e2e = {"value": tokens / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d_step),
+               "d2h_bytes_per_step": int(d2h)}
+
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    peaks, peak_src = load_peaks()
+    fl = flops(w, w.backward)
+    by = compulsory_bytes(w, w.backward)
+    t_step = total_ms / args.steps / 1e3
+    roof_t = max(fl / (peaks["bf16_tflops"] * 1e12), by / (peaks["hbm_gbs"] * 1e9))
+    dom = max(kprof.items(), key=lambda kv: kv[1][1]) if kprof else None
+    roofline = None
+    if dom:
+        name, (cnt, ms) = dom
+        avg_s = ms / cnt / 1e3
+        kb = kernel_bytes(name, w)
+        ach = kb / avg_s / 1e9
+        share = ms / sum(v[1] for v in kprof.values())
+        roofline = {"bound": "hbm", "kernel": name, "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": ach / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
+                    "algorithmic_bytes_per_launch": kb, "avg_launch_us": avg_s * 1e6, "share_of_step": share}
+    line = base_line(w, args, world)
+    line.update({"value": value, "ms_per_step": total_ms / args.steps, "e2e": e2e, "gpu_launches": int(launches),
+                 "roofline": roofline, "clocks": clocks,
+                 "step_roofline": {"tflops": fl / t_step / 1e12, "gbs_compulsory": by / t_step / 1e9,
+                                   "roofline_us": roof_t * 1e6, "frac": roof_t / t_step, "peak_source": peak_src},
+                 "kernels": {n: {"launches": c, "avg_us": 1e3 * m / c} for n, (c, m) in sorted(kprof.items())},
+                 "plan": args.plan})
+    if world == 1 and not args.no_cpu_baseline:
+        heads = oracle_heads(w)
+        tk, dt, thr = oracle_sample(w, 0, heads)
+        line["cpu_baseline"] = {"value": tk / dt, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                                "sample": f"{heads} of {w.B * w.H} heads, full L={w.L}, "
+                                          f"{'fwd+bwd' if w.backward else 'fwd'}, float64, {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,146 @@
+/*
+ * gla.h -- C ABI of the B200 (sm_100a) chunkwise gated linear attention library.
+ *
+ * The operation (recurrent form; talk summary "Hardware-Efficient Training of Linear
+ * Attention Models", sections 4:04 and 7:36; data-dependent gates from the GLA
+ * abstract, Yang et al.): per (batch b, head h), with a Dk x Dv matrix state S,
+ *
+ *     S_t = diag(alpha_t) S_{t-1} + k'_t^T v_t,    o_t = scale * q_t S_t,
+ *     alpha_t = exp(g_t),  k'_t = i_t k_t (input gate, optional, else k'_t = k_t),
+ *     S_{-1} = h0 (or 0),  hT = S_{L-1}.
+ *
+ * The readout uses the updated state S_t. The library evaluates it with the chunkwise
+ * ("trunk-wise") algorithm of the same talk, section 11:58: the sequence is cut into
+ * chunks of C tokens, states are formed only at chunk boundaries with K^T V matrix
+ * products, and each chunk's output is the inter-chunk term (q_t decayed) S plus a
+ * masked intra-chunk product. Large chunks are tiled inside the chunk (Tiled Flash
+ * Linear Attention abstract).
+ *
+ * Conventions for every entry point:
+ *  - Layout BHLD, contiguous: q,k [B,H,L,Dk]; v,o,dO [B,H,L,Dv]; per-key gates
+ *    g,dg [B,H,L,Dk]; per-head gates g,dg [B,H,L]; input gate i,di [B,H,L];
+ *    states h0,hT,dhT,dh0 [B,H,Dk,Dv] (row = key dim).
+ *  - q,k,v,o,dO,dq,dk,dv have the I/O dtype of the problem (GLA_F32 or GLA_BF16);
+ *    g, i, h0, hT and all their gradients are always float32. Accumulation is fp32.
+ *  - g is the log of the decay (g <= 0 for a decay in (0,1]); the library applies no
+ *    activation to it. It must be finite; within any 64-token tile the decay of one key
+ *    dim should span less than about 80 nats (exp stays inside fp32 range), otherwise
+ *    results lose accuracy (no fault, no error code).
+ *  - Every pointer is a DEVICE pointer owned by the caller, 16-byte aligned. The
+ *    library allocates nothing; scratch memory is the caller's workspace `ws` of at
+ *    least gla_workspace_bytes() bytes (16-byte aligned, contents need not be zeroed).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL means
+ *    the legacy default stream). Argument errors are detected on the host before any
+ *    launch; launch failures map to GLA_ERR_CUDA. No exception crosses the ABI.
+ *  - Thread safety: concurrent calls are safe when they use distinct workspaces.
+ */
+#ifndef GLA_B200_H
+#define GLA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GLA_API __attribute__((visibility("default")))
+#else
+#define GLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GLA_OK = 0,
+    GLA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, bad enum */
+    GLA_ERR_UNSUPPORTED = 2,  /* valid request this build cannot run (shape, plan) */
+    GLA_ERR_WORKSPACE = 3,    /* ws_bytes smaller than gla_workspace_bytes() */
+    GLA_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
+    GLA_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up (see below) */
+} gla_status;
+
+typedef enum { GLA_F32 = 0, GLA_BF16 = 1 } gla_dtype;
+
+typedef enum {
+    GLA_GATE_NONE = 0,     /* alpha = 1: plain causal linear attention */
+    GLA_GATE_PER_KEY = 1,  /* g [B,H,L,Dk]: one log-decay per key dim (GLA) */
+    GLA_GATE_PER_HEAD = 2  /* g [B,H,L]: one scalar log-decay per head (mLSTM-style) */
+} gla_gate_mode;
+
+typedef enum {
+    GLA_PLAN_AUTO = 0,     /* library picks from shape, dtype and SM count */
+    GLA_PLAN_SIMT = 1,     /* CUDA-core chunk-parallel kernels: any supported shape,
+                              fp32 or bf16 I/O; the only plan for fp32 I/O */
+    GLA_PLAN_TC = 2        /* tcgen05/TMEM tensor-core kernels; bf16 I/O only */
+} gla_plan;
+
+typedef struct {
+    int B, H, L;          /* batch, heads, tokens (L >= 0; L = 0 gives hT = h0) */
+    int Dk, Dv;           /* head dims: each one of 64, 128, 256 */
+    int chunk;            /* chunk size C: a multiple of 16 in [16, 1024] */
+    float scale;          /* output scale (typically Dk^-1/2) */
+    gla_dtype io;         /* dtype of q, k, v, o, dO, dq, dk, dv */
+    gla_gate_mode gate;
+    int plan;             /* a gla_plan value */
+} gla_problem;
+
+/* Bytes of caller-provided workspace needed by gla_fwd (for_backward = 0) or gla_bwd
+ * (for_backward = 1) for this problem; 0 when the problem is invalid. The size depends
+ * only on the problem (sizes, dtype, gate mode, plan), never on the data. */
+GLA_API size_t gla_workspace_bytes(const gla_problem* p, int for_backward);
+
+/* Forward pass.
+ *   q,k,v  : inputs (I/O dtype);  g: log-decays (NULL iff gate == GLA_GATE_NONE)
+ *   igate  : input gate [B,H,L] f32 or NULL;  h0: initial state f32 or NULL (= 0)
+ *   o      : output [B,H,L,Dv] (I/O dtype), written completely
+ *   hT     : final state f32 or NULL (not written)
+ *   ws     : workspace, ws_bytes >= gla_workspace_bytes(p, 0)
+ * Errors: GLA_ERR_INVALID_ARG, GLA_ERR_UNSUPPORTED, GLA_ERR_WORKSPACE, GLA_ERR_CUDA. */
+GLA_API gla_status gla_fwd(const gla_problem* p, const void* q, const void* k, const void* v,
+                   const float* g, const float* igate, const float* h0,
+                   void* o, float* hT, void* ws, size_t ws_bytes, void* stream);
+
+/* Backward pass. Recomputes the chunk states from its inputs (it does not need the
+ * forward's workspace). Inputs as for gla_fwd plus
+ *   dO  : upstream gradient of o (I/O dtype);  dhT: upstream gradient of hT or NULL (= 0)
+ * Outputs (written completely):
+ *   dq, dk, dv (I/O dtype);  dg (like g, f32; must be NULL iff gate == GLA_GATE_NONE)
+ *   di [B,H,L] f32 (non-NULL only with igate);  dh0 f32 or NULL (not written)
+ * dg is the reverse cumulative sum over the whole sequence of q*dq - k'*dk' (plus the
+ * final-state term sum_e dhT*hT); for GLA_GATE_PER_HEAD it is summed over key dims.
+ * Errors as for gla_fwd. */
+GLA_API gla_status gla_bwd(const gla_problem* p, const void* q, const void* k, const void* v,
+                   const float* g, const float* igate, const float* h0,
+                   const void* dO, const float* dhT,
+                   void* dq, void* dk, void* dv, float* dg, float* di, float* dh0,
+                   void* ws, size_t ws_bytes, void* stream);
+
+/* Static description of a status code (never NULL). */
+GLA_API const char* gla_status_string(gla_status s);
+
+/* Synchronises `stream`, then reads the device status word kept at the start of the
+ * workspace of the last call that used `ws`: GLA_OK, or GLA_ERR_TIMEOUT when a bounded
+ * device-side wait gave up; GLA_ERR_CUDA if the synchronisation itself failed. */
+GLA_API gla_status gla_check_device_status(void* ws, void* stream);
+
+/* Library version as 10000*major + 100*minor + patch. */
+GLA_API int gla_version(void);
+
+/* Measurement support (not needed for computing).
+ * gla_launch_count: number of kernels this process has launched through the library.
+ * gla_profiler_enable(1): from now on every kernel launch is bracketed by two CUDA events
+ *   recorded on the launching stream (host cost: a few microseconds per launch).
+ * gla_profiler_read: synchronises on the recorded events, aggregates them by kernel name
+ *   into up to max_kernels entries (name copied into names + i*name_stride, NUL-terminated;
+ *   launches[i]; total_ms[i] = summed event time), forgets them, and returns the number of
+ *   distinct kernels seen (-1 on a CUDA error). Any output pointer may be NULL.
+ * Not meant for concurrent use from several host threads while enabled. */
+GLA_API unsigned long long gla_launch_count(void);
+GLA_API gla_status gla_profiler_enable(int enable);
+GLA_API int gla_profiler_read(char* names, int name_stride, int* launches, double* total_ms, int max_kernels);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GLA_B200_H */

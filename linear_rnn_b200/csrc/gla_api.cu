@@ -1,0 +1,216 @@
+// C ABI of the library: argument validation, plan choice, workspace accounting and
+// error mapping. Every numerical step runs in the plans' CUDA kernels.
+#include <string.h>
+
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "gla_common.cuh"
+#include "gla_plans.h"
+
+using namespace gla;
+
+// ------------------------------------------------------------ launch accounting
+namespace {
+struct ProfRecord {
+    std::string name;
+    cudaEvent_t start, stop;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+unsigned long long g_launches = 0;
+std::vector<ProfRecord> g_prof_open;  // recorded, not yet read
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+}  // namespace
+
+namespace gla {
+void prof_begin(const char* name, cudaStream_t st) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    ++g_launches;
+    if (!g_prof_on) return;
+    ProfRecord r{name, take_event(), take_event()};
+    cudaEventRecord(r.start, st);
+    g_prof_open.push_back(r);
+}
+void prof_end(cudaStream_t st) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (!g_prof_on || g_prof_open.empty()) return;
+    cudaEventRecord(g_prof_open.back().stop, st);
+}
+}  // namespace gla
+
+namespace {
+
+bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool dim_ok(int d) { return d == 64 || d == 128 || d == 256; }
+
+// Validates the problem; fills Dims and the resolved plan.
+gla_status check_problem(const gla_problem* p, Dims* P, int* plan) {
+    if (!p) return GLA_ERR_INVALID_ARG;
+    if (p->B < 0 || p->H < 0 || p->L < 0) return GLA_ERR_INVALID_ARG;
+    if (p->io != GLA_F32 && p->io != GLA_BF16) return GLA_ERR_INVALID_ARG;
+    if (p->gate != GLA_GATE_NONE && p->gate != GLA_GATE_PER_KEY && p->gate != GLA_GATE_PER_HEAD)
+        return GLA_ERR_INVALID_ARG;
+    if (p->plan < GLA_PLAN_AUTO || p->plan > GLA_PLAN_TC) return GLA_ERR_INVALID_ARG;
+    if (p->chunk < 16 || p->chunk > 1024 || p->chunk % 16 != 0) return GLA_ERR_UNSUPPORTED;
+    if (!dim_ok(p->Dk) || !dim_ok(p->Dv)) return GLA_ERR_UNSUPPORTED;
+    if ((long long)p->B * p->H > 65535LL) return GLA_ERR_UNSUPPORTED;  // grid z extent
+    int pl = p->plan;
+    if (pl == GLA_PLAN_AUTO) pl = GLA_PLAN_SIMT;
+    if (pl == GLA_PLAN_TC) return GLA_ERR_UNSUPPORTED;
+    P->B = p->B; P->H = p->H; P->L = p->L; P->Dk = p->Dk; P->Dv = p->Dv; P->C = p->chunk;
+    P->N = cdiv(p->L, p->chunk);
+    P->gate = p->gate;
+    P->scale = p->scale;
+    *plan = pl;
+    return GLA_OK;
+}
+
+gla_status map_cuda(cudaError_t e) { return e == cudaSuccess ? GLA_OK : GLA_ERR_CUDA; }
+
+size_t ws_bytes(const Dims& P, int plan, bool bwd) {
+    (void)plan;
+    return simt::workspace_bytes(P, bwd);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gla_workspace_bytes(const gla_problem* p, int for_backward) {
+    Dims P;
+    int plan;
+    if (check_problem(p, &P, &plan) != GLA_OK) return 0;
+    return ws_bytes(P, plan, for_backward != 0);
+}
+
+gla_status gla_fwd(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
+                   const float* igate, const float* h0, void* o, float* hT, void* ws, size_t ws_bytes_given,
+                   void* stream) {
+    Dims P;
+    int plan;
+    gla_status s = check_problem(p, &P, &plan);
+    if (s != GLA_OK) return s;
+    const bool empty = (size_t)P.B * P.H * P.L == 0;
+    if (!empty && (!q || !k || !v || !o)) return GLA_ERR_INVALID_ARG;
+    if ((p->gate == GLA_GATE_NONE) != (g == nullptr) && !empty) return GLA_ERR_INVALID_ARG;
+    if (!ws) return GLA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, g, igate, h0, o, hT, ws};
+    for (const void* x : ptrs)
+        if (!aligned16(x)) return GLA_ERR_INVALID_ARG;
+    if (ws_bytes_given < ws_bytes(P, plan, false)) return GLA_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, st);
+    if (e != cudaSuccess) return GLA_ERR_CUDA;
+    if ((size_t)P.B * P.H == 0) return GLA_OK;
+    e = simt::fwd(P, p->io, q, k, v, g, igate, h0, o, hT, ws, st);
+    return map_cuda(e);
+}
+
+gla_status gla_bwd(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
+                   const float* igate, const float* h0, const void* dO, const float* dhT, void* dq, void* dk,
+                   void* dv, float* dg, float* di, float* dh0, void* ws, size_t ws_bytes_given, void* stream) {
+    Dims P;
+    int plan;
+    gla_status s = check_problem(p, &P, &plan);
+    if (s != GLA_OK) return s;
+    const bool empty = (size_t)P.B * P.H * P.L == 0;
+    if (!empty && (!q || !k || !v || !dO || !dq || !dk || !dv)) return GLA_ERR_INVALID_ARG;
+    if (!empty && (p->gate == GLA_GATE_NONE) != (g == nullptr)) return GLA_ERR_INVALID_ARG;
+    if (!empty && (p->gate == GLA_GATE_NONE) != (dg == nullptr)) return GLA_ERR_INVALID_ARG;
+    if (di && !igate) return GLA_ERR_INVALID_ARG;
+    if (!ws) return GLA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, g, igate, h0, dO, dhT, dq, dk, dv, dg, di, dh0, ws};
+    for (const void* x : ptrs)
+        if (!aligned16(x)) return GLA_ERR_INVALID_ARG;
+    if (ws_bytes_given < ws_bytes(P, plan, true)) return GLA_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, st);
+    if (e != cudaSuccess) return GLA_ERR_CUDA;
+    if ((size_t)P.B * P.H == 0) return GLA_OK;
+    e = simt::bwd(P, p->io, q, k, v, g, igate, h0, dO, dhT, dq, dk, dv, dg, di, dh0, ws, st);
+    return map_cuda(e);
+}
+
+const char* gla_status_string(gla_status status) {
+    const int s = static_cast<int>(status);  // any int may arrive through the ABI
+    switch (s) {
+        case GLA_OK: return "ok";
+        case GLA_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, bad size or enum)";
+        case GLA_ERR_UNSUPPORTED: return "unsupported problem (head dims, chunk size or plan)";
+        case GLA_ERR_WORKSPACE: return "workspace too small";
+        case GLA_ERR_CUDA: return "CUDA runtime error";
+        case GLA_ERR_TIMEOUT: return "bounded device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+gla_status gla_check_device_status(void* ws, void* stream) {
+    if (!ws) return GLA_ERR_INVALID_ARG;
+    int word = 0;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(&word, ws, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return GLA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return GLA_ERR_CUDA;
+    return word == kDevStatusOk ? GLA_OK : GLA_ERR_TIMEOUT;
+}
+
+int gla_version(void) { return 100; }
+
+unsigned long long gla_launch_count(void) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    return g_launches;
+}
+
+gla_status gla_profiler_enable(int enable) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_on = enable != 0;
+    return GLA_OK;
+}
+
+int gla_profiler_read(char* names, int name_stride, int* launches, double* total_ms, int max_kernels) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    std::vector<std::string> keys;
+    std::vector<int> cnt;
+    std::vector<double> ms;
+    for (ProfRecord& r : g_prof_open) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess)
+            return -1;
+        size_t i = 0;
+        while (i < keys.size() && keys[i] != r.name) ++i;
+        if (i == keys.size()) {
+            keys.push_back(r.name);
+            cnt.push_back(0);
+            ms.push_back(0.0);
+        }
+        cnt[i] += 1;
+        ms[i] += t;
+        g_event_pool.push_back(r.start);
+        g_event_pool.push_back(r.stop);
+    }
+    g_prof_open.clear();
+    const int n = (int)keys.size();
+    for (int i = 0; i < n && i < max_kernels; ++i) {
+        if (names && name_stride > 0) {
+            strncpy(names + (size_t)i * name_stride, keys[i].c_str(), name_stride - 1);
+            names[(size_t)i * name_stride + name_stride - 1] = 0;
+        }
+        if (launches) launches[i] = cnt[i];
+        if (total_ms) total_ms[i] = ms[i];
+    }
+    return n;
+}
+
+}  // extern "C"

@@ -1,0 +1,45 @@
+// Shared device/host helpers of the CUDA library (not of the oracle).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gla.h"
+
+namespace gla {
+
+// Kernel-side view of one problem. Pointers are device pointers.
+struct Dims {
+    int B, H, L, Dk, Dv, C, N;  // N = number of chunks = ceil(L / C)
+    int gate;                    // gla_gate_mode
+    float scale;
+};
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+__host__ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
+__host__ __device__ __forceinline__ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Device status word at the start of every workspace (first 256 bytes).
+constexpr size_t kStatusBytes = 256;
+constexpr int kDevStatusOk = 0;
+constexpr int kDevStatusTimeout = 1;
+
+// Launch accounting (gla_api.cu): every kernel launch of the library goes through
+// GLA_LAUNCH, which counts it and, while the profiler is enabled, brackets it with CUDA
+// events recorded on the launching stream.
+void prof_begin(const char* name, cudaStream_t st);
+void prof_end(cudaStream_t st);
+
+}  // namespace gla
+
+#define GLA_LAUNCH(name, stream, ...)      \
+    do {                                   \
+        ::gla::prof_begin(name, stream);   \
+        __VA_ARGS__;                       \
+        ::gla::prof_end(stream);           \
+    } while (0)

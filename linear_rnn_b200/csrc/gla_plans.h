@@ -1,0 +1,16 @@
+// Internal interface between the C-ABI layer (gla_api.cu) and the kernel plans.
+#pragma once
+#include <cuda_runtime.h>
+
+#include "gla_common.cuh"
+
+namespace gla {
+namespace simt {
+size_t workspace_bytes(const Dims& P, bool bwd);
+cudaError_t fwd(const Dims& P, gla_dtype io, const void* q, const void* k, const void* v, const float* g,
+                const float* ig, const float* h0, void* o, float* hT, void* ws, cudaStream_t st);
+cudaError_t bwd(const Dims& P, gla_dtype io, const void* q, const void* k, const void* v, const float* g,
+                const float* ig, const float* h0, const void* dO, const float* dhT, void* dq, void* dk, void* dv,
+                float* dg, float* di, float* dh0, void* ws, cudaStream_t st);
+}  // namespace simt
+}  // namespace gla

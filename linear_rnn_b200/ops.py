@@ -1,0 +1,143 @@
+"""Python entry points with the names of the C ABI (include/gla.h): gla_fwd, gla_bwd,
+gla_workspace_bytes, gla_check_device_status.
+
+They marshal torch tensors into the C calls: shape/dtype checks, the gate mode read
+from g's rank, a workspace allocated with torch (the library itself allocates nothing),
+and the current torch CUDA stream. Tensors on the host are copied to the current CUDA
+device and results copied back (the end-to-end call of a host-side user); tensors
+already on the device are used in place.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import Dict, Optional, Tuple
+
+import torch
+
+from . import _lib
+from ._lib import GlaError, GlaProblem
+
+_PLANS = {"auto": _lib.GLA_PLAN_AUTO, "simt": _lib.GLA_PLAN_SIMT, "tc": _lib.GLA_PLAN_TC}
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _io_dtype(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return _lib.GLA_F32
+    if dt == torch.bfloat16:
+        return _lib.GLA_BF16
+    raise TypeError(f"q/k/v must be float32 or bfloat16, got {dt}")
+
+
+def make_problem(q: torch.Tensor, v: torch.Tensor, g: Optional[torch.Tensor], *, scale: Optional[float],
+                 chunk: int, plan: str) -> GlaProblem:
+    if q.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be [B, H, L, D]")
+    B, H, L, Dk = q.shape
+    Dv = v.shape[-1]
+    if g is None:
+        gate = _lib.GLA_GATE_NONE
+    elif g.dim() == 4:
+        gate = _lib.GLA_GATE_PER_KEY
+    elif g.dim() == 3:
+        gate = _lib.GLA_GATE_PER_HEAD
+    else:
+        raise ValueError("g must be [B,H,L,Dk] (per key dim) or [B,H,L] (per head)")
+    if plan not in _PLANS:
+        raise ValueError(f"plan must be one of {sorted(_PLANS)}")
+    return GlaProblem(B, H, L, Dk, Dv, int(chunk), float(1.0 / math.sqrt(Dk) if scale is None else scale),
+                      _io_dtype(q.dtype), gate, _PLANS[plan])
+
+
+def gla_workspace_bytes(problem: GlaProblem, for_backward: bool) -> int:
+    return int(_lib.lib.gla_workspace_bytes(ctypes.byref(problem), int(for_backward)))
+
+
+def _stream_handle(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _to_dev(t: Optional[torch.Tensor], device: torch.device) -> Optional[torch.Tensor]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("inputs must be contiguous (BHLD)")
+    if t.device.type == "cuda":
+        return t
+    return t.to(device, non_blocking=True)
+
+
+def _check(status: int, where: str):
+    if status != _lib.GLA_OK:
+        raise GlaError(status, where)
+
+
+def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.Tensor:
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise GlaError(_lib.GLA_ERR_WORKSPACE, "workspace")
+        return workspace
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def gla_fwd(q, k, v, g=None, igate=None, h0=None, *, scale: Optional[float] = None, chunk: int = 64,
+            plan: str = "auto", output_final_state: bool = True,
+            workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Forward pass. Returns (o, hT); hT is None when output_final_state is False."""
+    host = q.device.type != "cuda"
+    device = torch.device("cuda", torch.cuda.current_device()) if host else q.device
+    q, k, v, g, igate, h0 = (_to_dev(t, device) for t in (q, k, v, g, igate, h0))
+    prob = make_problem(q, v, g, scale=scale, chunk=chunk, plan=plan)
+    o = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=device)
+    hT = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
+                     device=device) if output_final_state else None
+    nbytes = gla_workspace_bytes(prob, False)
+    if nbytes == 0:
+        raise GlaError(_lib.GLA_ERR_UNSUPPORTED, "gla_workspace_bytes")
+    ws = _workspace(nbytes, device, workspace)
+    st = _lib.lib.gla_fwd(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(igate), _ptr(h0),
+                          _ptr(o), _ptr(hT), _ptr(ws), ws.numel() * ws.element_size(), _stream_handle(device))
+    _check(st, "gla_fwd")
+    if host:
+        o = o.cpu()
+        hT = hT.cpu() if hT is not None else None
+    return o, hT
+
+
+def gla_bwd(q, k, v, g, igate, h0, dO, dhT=None, *, scale: Optional[float] = None, chunk: int = 64,
+            plan: str = "auto", output_dh0: bool = True,
+            workspace: Optional[torch.Tensor] = None) -> Dict[str, Optional[torch.Tensor]]:
+    """Backward pass. Returns dict dq, dk, dv, dg (None if ungated), di (None without an
+    input gate), dh0 (None when output_dh0 is False)."""
+    host = q.device.type != "cuda"
+    device = torch.device("cuda", torch.cuda.current_device()) if host else q.device
+    q, k, v, g, igate, h0, dO, dhT = (_to_dev(t, device) for t in (q, k, v, g, igate, h0, dO, dhT))
+    prob = make_problem(q, v, g, scale=scale, chunk=chunk, plan=plan)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    dg = torch.empty_like(g) if g is not None else None
+    di = torch.empty_like(igate) if igate is not None else None
+    dh0 = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
+                      device=device) if output_dh0 else None
+    nbytes = gla_workspace_bytes(prob, True)
+    if nbytes == 0:
+        raise GlaError(_lib.GLA_ERR_UNSUPPORTED, "gla_workspace_bytes")
+    ws = _workspace(nbytes, device, workspace)
+    st = _lib.lib.gla_bwd(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(igate), _ptr(h0),
+                          _ptr(dO), _ptr(dhT), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(di), _ptr(dh0),
+                          _ptr(ws), ws.numel() * ws.element_size(), _stream_handle(device))
+    _check(st, "gla_bwd")
+    out = {"dq": dq, "dk": dk, "dv": dv, "dg": dg, "di": di, "dh0": dh0}
+    if host:
+        out = {n: (t.cpu() if t is not None else None) for n, t in out.items()}
+    return out
+
+
+def gla_check_device_status(workspace: torch.Tensor) -> int:
+    device = workspace.device
+    return int(_lib.lib.gla_check_device_status(_ptr(workspace), _stream_handle(device)))

@@ -1,0 +1,124 @@
+"""Host-only checks of the C ABI: the library loads, exports every symbol that
+include/gla.h declares, and validates arguments on the host (no GPU needed: every call
+here fails validation before any CUDA call)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from linear_rnn_b200 import _lib, build
+from linear_rnn_b200._lib import GlaProblem
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    syms = set()
+    for name in os.listdir(os.path.join(ROOT, "include")):
+        if name.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", name)).read()
+            syms |= set(re.findall(r"GLA_API\s+[\w\s\*]+?\b(gla_\w+)\s*\(", text))
+    return syms
+
+
+def test_library_exports_every_declared_symbol():
+    syms = declared_symbols()
+    assert {"gla_fwd", "gla_bwd", "gla_workspace_bytes"} <= syms
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (gla_\w+)", out))
+    assert syms <= exported, syms - exported
+    assert set(_lib.EXPORTED) == syms
+    for s in syms:
+        assert hasattr(_lib.lib, s)
+
+
+def test_library_is_built_for_sm100a_only():
+    out = subprocess.run(["cuobjdump", "--list-elf", build.LIB], capture_output=True, text=True)
+    if out.returncode != 0:
+        pytest.skip("cuobjdump unavailable")
+    archs = set(re.findall(r"sm_\w+", out.stdout))
+    assert archs == {"sm_100a"}, archs
+
+
+def prob(**kw):
+    base = dict(B=2, H=3, L=300, Dk=128, Dv=64, chunk=64, scale=0.1, io=_lib.GLA_BF16,
+                gate=_lib.GLA_GATE_PER_KEY, plan=_lib.GLA_PLAN_SIMT)
+    base.update(kw)
+    return GlaProblem(*[base[f] for f, _ in GlaProblem._fields_])
+
+
+def ws_bytes(**kw):
+    p = prob(**kw)
+    return _lib.lib.gla_workspace_bytes(ctypes.byref(p), 0), _lib.lib.gla_workspace_bytes(ctypes.byref(p), 1)
+
+
+def test_workspace_sizes():
+    f, b = ws_bytes()
+    assert 0 < f < b
+    # states at chunk boundaries only: ceil(300/64) = 5 states of 128x64 fp32 per head
+    assert f >= 2 * 3 * 5 * 128 * 64 * 4
+    assert ws_bytes(Dk=96) == (0, 0)
+    assert ws_bytes(chunk=24) == (0, 0)
+    assert ws_bytes(chunk=2048) == (0, 0)
+    assert ws_bytes(L=-1) == (0, 0)
+    assert ws_bytes(io=7) == (0, 0)
+    assert ws_bytes(gate=9) == (0, 0)
+    # larger chunks materialise fewer states
+    assert ws_bytes(chunk=256)[0] < ws_bytes(chunk=64)[0]
+
+
+def test_status_strings():
+    for s in range(6):
+        assert len(_lib.status_string(s)) >= 2
+    assert "unknown" in _lib.status_string(99)
+
+
+def _fwd(p, **ptrs):
+    args = dict(q=16, k=16, v=16, g=16, ig=None, h0=None, o=16, hT=None, ws=16, nbytes=1 << 30)
+    args.update(ptrs)
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    return _lib.lib.gla_fwd(ctypes.byref(p), vp(args["q"]), vp(args["k"]), vp(args["v"]), vp(args["g"]),
+                            vp(args["ig"]), vp(args["h0"]), vp(args["o"]), vp(args["hT"]), vp(args["ws"]),
+                            args["nbytes"], None)
+
+
+def test_fwd_argument_validation_happens_before_launch():
+    p = prob()
+    assert _fwd(p, q=None) == _lib.GLA_ERR_INVALID_ARG
+    assert _fwd(p, g=None) == _lib.GLA_ERR_INVALID_ARG           # gate mode says per-key
+    assert _fwd(prob(gate=_lib.GLA_GATE_NONE)) == _lib.GLA_ERR_INVALID_ARG  # g given, no gate
+    assert _fwd(p, k=24) == _lib.GLA_ERR_INVALID_ARG              # misaligned
+    assert _fwd(p, ws=None) == _lib.GLA_ERR_INVALID_ARG
+    assert _fwd(p, nbytes=100) == _lib.GLA_ERR_WORKSPACE
+    assert _fwd(prob(Dv=32)) == _lib.GLA_ERR_UNSUPPORTED
+    assert _fwd(prob(chunk=40)) == _lib.GLA_ERR_UNSUPPORTED
+    assert _lib.lib.gla_fwd(None, None, None, None, None, None, None, None, None, None, 0, None) == \
+        _lib.GLA_ERR_INVALID_ARG
+
+
+def test_bwd_argument_validation_happens_before_launch():
+    p = prob()
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+
+    def call(**kw):
+        a = dict(q=16, k=16, v=16, g=16, ig=None, h0=None, dO=16, dhT=None, dq=16, dk=16, dv=16, dg=16,
+                 di=None, dh0=None, ws=16, nbytes=1 << 30, p=p)
+        a.update(kw)
+        return _lib.lib.gla_bwd(ctypes.byref(a["p"]), *(vp(a[n]) for n in
+                                ("q", "k", "v", "g", "ig", "h0", "dO", "dhT", "dq", "dk", "dv", "dg", "di", "dh0",
+                                 "ws")), a["nbytes"], None)
+    assert call(dO=None) == _lib.GLA_ERR_INVALID_ARG
+    assert call(dg=None) == _lib.GLA_ERR_INVALID_ARG
+    assert call(di=16) == _lib.GLA_ERR_INVALID_ARG       # di without an input gate
+    assert call(dq=8) == _lib.GLA_ERR_INVALID_ARG
+    assert call(nbytes=4096) == _lib.GLA_ERR_WORKSPACE
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    import importlib
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError, match="no CPU fallback"):
+        _lib._load()
+    importlib.reload(_lib)

@@ -1,0 +1,221 @@
+"""GPU parity: the CUDA library against the float64 oracle on the same seeded inputs.
+
+Error metric per output tensor: max|x - x_ref| / max|x_ref| over the compared
+elements; bound 1e-2 for bf16 I/O and 1e-4 for fp32 I/O (o, hT, dq, dk, dv, dg, di,
+dh0). Small cases compare every element; the full-size workloads run the whole batch on
+the GPU (in the launch configuration the benchmark times) and compare whole heads that
+the oracle recomputes independently.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_rnn_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 1e-2}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def ops():
+    from linear_rnn_b200 import ops as _ops
+    return _ops
+
+
+def f64(t):
+    return None if t is None else t.detach().to("cpu", torch.float64).numpy()
+
+
+def err(got, ref):
+    return float(np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-30))
+
+
+def to_cuda(x):
+    return {k: (None if v is None else v.cuda()) for k, v in x.items()}
+
+
+def gpu_fwd(x, w, plan="auto", chunk=None):
+    xd = to_cuda(x)
+    o, hT = ops().gla_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["igate"], xd["h0"], scale=w.scale,
+                          chunk=chunk or w.chunk, plan=plan)
+    return f64(o), f64(hT)
+
+
+def gpu_bwd(x, w, plan="auto", chunk=None):
+    xd = to_cuda(x)
+    r = ops().gla_bwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["igate"], xd["h0"], xd["dO"], xd.get("dhT"),
+                      scale=w.scale, chunk=chunk or w.chunk, plan=plan)
+    return {k: f64(v) for k, v in r.items()}
+
+
+def flat_heads(t, heads):
+    """[B,H,...] -> [1, len(heads), ...] picking flat head indices b*H + h."""
+    if t is None:
+        return None
+    B, H = t.shape[0], t.shape[1]
+    return t.reshape((B * H,) + tuple(t.shape[2:]))[heads].unsqueeze(0)
+
+
+def check_fwd(x, w, plan="auto", chunk=None, heads=None):
+    o, hT = gpu_fwd(x, w, plan, chunk)
+    xs = x if heads is None else {k: flat_heads(v, heads) for k, v in x.items()}
+    ro, rhT = oracle.gla_fwd(xs["q"], xs["k"], xs["v"], xs["g"], xs["igate"], xs["h0"], w.scale)
+    if heads is not None:
+        o, hT = flat_heads(o, heads), flat_heads(hT, heads)
+    tol = TOL[w.dtype]
+    assert err(o, ro) <= tol, ("o", err(o, ro))
+    assert err(hT, rhT) <= tol, ("hT", err(hT, rhT))
+    return err(o, ro), err(hT, rhT)
+
+
+def check_bwd(x, w, plan="auto", chunk=None, heads=None):
+    r = gpu_bwd(x, w, plan, chunk)
+    xs = x if heads is None else {k: flat_heads(v, heads) for k, v in x.items()}
+    ref = oracle.gla_bwd(xs["q"], xs["k"], xs["v"], xs["g"], xs["igate"], xs["h0"], xs["dO"], xs.get("dhT"),
+                         w.scale)
+    tol = TOL[w.dtype]
+    errs = {}
+    for name in ("dq", "dk", "dv", "dg", "di", "dh0"):
+        if ref[name] is None:
+            assert r[name] is None, name
+            continue
+        got = r[name] if heads is None else flat_heads(r[name], heads)
+        errs[name] = err(got, ref[name])
+        assert errs[name] <= tol, (name, errs[name])
+    return errs
+
+
+def with_dhT(x, w, seed=0):
+    x = dict(x)
+    x["dhT"] = I.make_dhT(w, seed)
+    return x
+
+
+# ---------------------------------------------------------------- small workloads
+
+@pytest.mark.parametrize("name", ["c1", "c2", "c3", "c4", "c5"])
+def test_small_workloads_full_compare(name):
+    w = I.small(I.WORKLOADS[name])
+    x = I.make_inputs(w, seed=1)
+    check_fwd(x, w)
+    if w.backward:
+        check_bwd(x, w)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("L", [1, 15, 16, 63, 64, 65, 200])
+def test_ragged_lengths(dtype, L):
+    w = I.WORKLOADS["c3"].replace(B=1, H=2, L=L, Dk=64, Dv=64, dtype=dtype, h0_std=0.5, backward=True)
+    x = with_dhT(I.make_inputs(w, seed=2), w)
+    check_fwd(x, w)
+    check_bwd(x, w)
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 48, 128, 256, 1024])
+def test_chunk_sizes(chunk):
+    w = I.WORKLOADS["c3"].replace(B=1, H=2, L=300, Dk=64, Dv=128, dtype="f32", chunk=chunk, h0_std=0.3,
+                                  backward=True)
+    x = with_dhT(I.make_inputs(w, seed=3), w)
+    check_fwd(x, w)
+    check_bwd(x, w)
+
+
+@pytest.mark.parametrize("Dk,Dv", [(64, 128), (128, 64), (256, 64), (64, 256), (128, 128)])
+def test_head_dims(Dk, Dv):
+    w = I.WORKLOADS["c3"].replace(B=2, H=1, L=150, Dk=Dk, Dv=Dv, dtype="bf16", h0_std=0.2)
+    x = with_dhT(I.make_inputs(w, seed=4), w)
+    check_fwd(x, w)
+    check_bwd(x, w)
+
+
+@pytest.mark.parametrize("gate,ig", [(I.GATE_NONE, False), (I.GATE_PER_HEAD, False), (I.GATE_PER_KEY, True),
+                                     (I.GATE_NONE, True)])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_gate_modes(gate, ig, dtype):
+    w = I.WORKLOADS["c3"].replace(B=1, H=2, L=190, Dk=64, Dv=64, dtype=dtype, gate=gate, input_gate=ig,
+                                  h0_std=0.4)
+    x = with_dhT(I.make_inputs(w, seed=5), w)
+    check_fwd(x, w)
+    check_bwd(x, w)
+
+
+def test_initial_state_is_carried():
+    """Weak decay (g ~ -0.001) so h0 matters over the whole sequence."""
+    w = I.WORKLOADS["c4"].replace(B=1, H=2, L=256, Dk=64, Dv=64, dtype="f32", gate_div=800.0, chunk=64)
+    x = I.make_inputs(w, seed=6)
+    ro, _ = oracle.gla_fwd(x["q"], x["k"], x["v"], x["g"], None, None, w.scale)
+    rh, _ = oracle.gla_fwd(x["q"], x["k"], x["v"], x["g"], None, x["h0"], w.scale)
+    assert err(ro, rh) > 0.05  # the initial state is visible in the output
+    check_fwd(x, w)
+
+
+def test_empty_sequence():
+    w = I.WORKLOADS["c3"].replace(B=1, H=2, L=0, Dk=64, Dv=64, dtype="f32", h0_std=1.0, backward=True)
+    x = with_dhT(I.make_inputs(w, seed=7), w)
+    o, hT = gpu_fwd(x, w)
+    assert o.shape == (1, 2, 0, 64)
+    assert np.array_equal(hT, f64(x["h0"]))
+    r = gpu_bwd(x, w)
+    assert np.array_equal(r["dh0"], f64(x["dhT"]))
+
+
+def test_deterministic():
+    w = I.small(I.WORKLOADS["c3"])
+    x = with_dhT(I.make_inputs(w, seed=8), w)
+    a, b = gpu_bwd(x, w), gpu_bwd(x, w)
+    for k in a:
+        if a[k] is not None:
+            assert np.array_equal(a[k], b[k]), k
+    assert np.array_equal(gpu_fwd(x, w)[0], gpu_fwd(x, w)[0])
+
+
+def test_outputs_fully_written_over_nan_poison():
+    """Call the C ABI directly with NaN-filled output buffers."""
+    from linear_rnn_b200 import _lib
+    w = I.WORKLOADS["c3"].replace(B=1, H=2, L=130, Dk=64, Dv=128, dtype="bf16")
+    x = to_cuda(I.make_inputs(w, seed=9))
+    p = ops().make_problem(x["q"], x["v"], x["g"], scale=w.scale, chunk=64, plan="auto")
+    o = torch.full((1, 2, 130, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    hT = torch.full((1, 2, 64, 128), float("nan"), device="cuda")
+    nb = _lib.lib.gla_workspace_bytes(ctypes.byref(p), 0)
+    ws = torch.full((nb,), 255, dtype=torch.uint8, device="cuda")
+    P = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    st = _lib.lib.gla_fwd(ctypes.byref(p), P(x["q"]), P(x["k"]), P(x["v"]), P(x["g"]), None, None, P(o), P(hT),
+                          P(ws), nb, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    assert _lib.lib.gla_check_device_status(P(ws), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)) == 0
+    assert not torch.isnan(o).any() and not torch.isnan(hT).any()
+
+
+def test_host_tensors_round_trip():
+    """The end-to-end call with host tensors (copies in, compute, copies out)."""
+    w = I.small(I.WORKLOADS["c2"])
+    x = I.make_inputs(w, seed=10)
+    o, hT = ops().gla_fwd(x["q"], x["k"], x["v"], x["g"], scale=w.scale, chunk=w.chunk)
+    assert o.device.type == "cpu"
+    ro, rhT = oracle.gla_fwd(x["q"], x["k"], x["v"], x["g"], None, None, w.scale)
+    assert err(f64(o), ro) <= TOL["bf16"] and err(f64(hT), rhT) <= TOL["bf16"]
+
+
+# --------------------------------------------------------- full-size workloads
+
+FULL_HEADS = {"c1": None, "c2": [0, 77], "c3": [3, 40], "c4": [0, 5], "c5": [1, 14]}
+
+
+@pytest.mark.parametrize("name", ["c1", "c2", "c3", "c4", "c5"])
+def test_full_size_workload(name):
+    w = I.WORKLOADS[name]
+    x = I.make_inputs(w, seed=0)
+    heads = FULL_HEADS[name]
+    check_fwd(x, w, heads=heads)
+    if w.backward:
+        check_bwd(x, w, heads=heads)
