@@ -67,13 +67,22 @@ gla_status check_problem(const gla_problem* p, Dims* P, int* plan) {
     if (p->chunk < 16 || p->chunk > 1024 || p->chunk % 16 != 0) return GLA_ERR_UNSUPPORTED;
     if (!dim_ok(p->Dk) || !dim_ok(p->Dv)) return GLA_ERR_UNSUPPORTED;
     if ((long long)p->B * p->H > 65535LL) return GLA_ERR_UNSUPPORTED;  // grid z extent
-    int pl = p->plan;
-    if (pl == GLA_PLAN_AUTO) pl = GLA_PLAN_SIMT;
-    if (pl == GLA_PLAN_TC) return GLA_ERR_UNSUPPORTED;
     P->B = p->B; P->H = p->H; P->L = p->L; P->Dk = p->Dk; P->Dv = p->Dv; P->C = p->chunk;
     P->N = cdiv(p->L, p->chunk);
     P->gate = p->gate;
     P->scale = p->scale;
+    *plan = p->plan;
+    return GLA_OK;
+}
+
+// The tensor-core plan runs bf16 I/O with chunks that are whole 64-token tiles.
+bool tc_ok(const gla_problem* p, const Dims& P) { return p->io == GLA_BF16 && tc::supports(P); }
+
+// Plan of the forward / backward: AUTO prefers the tensor-core plan where it applies.
+gla_status resolve(const gla_problem* p, const Dims& P, bool bwd, int* plan) {
+    int pl = p->plan;
+    if (pl == GLA_PLAN_AUTO) pl = (!bwd && tc_ok(p, P)) ? GLA_PLAN_TC : GLA_PLAN_SIMT;
+    if (pl == GLA_PLAN_TC && (bwd || !tc_ok(p, P))) return GLA_ERR_UNSUPPORTED;
     *plan = pl;
     return GLA_OK;
 }
@@ -81,7 +90,7 @@ gla_status check_problem(const gla_problem* p, Dims* P, int* plan) {
 gla_status map_cuda(cudaError_t e) { return e == cudaSuccess ? GLA_OK : GLA_ERR_CUDA; }
 
 size_t ws_bytes(const Dims& P, int plan, bool bwd) {
-    (void)plan;
+    if (plan == GLA_PLAN_TC && !bwd) return tc::fwd_workspace_bytes(P);
     return simt::workspace_bytes(P, bwd);
 }
 
@@ -93,6 +102,7 @@ size_t gla_workspace_bytes(const gla_problem* p, int for_backward) {
     Dims P;
     int plan;
     if (check_problem(p, &P, &plan) != GLA_OK) return 0;
+    if (resolve(p, P, for_backward != 0, &plan) != GLA_OK) return 0;
     return ws_bytes(P, plan, for_backward != 0);
 }
 
@@ -102,6 +112,8 @@ gla_status gla_fwd(const gla_problem* p, const void* q, const void* k, const voi
     Dims P;
     int plan;
     gla_status s = check_problem(p, &P, &plan);
+    if (s != GLA_OK) return s;
+    s = resolve(p, P, false, &plan);
     if (s != GLA_OK) return s;
     const bool empty = (size_t)P.B * P.H * P.L == 0;
     if (!empty && (!q || !k || !v || !o)) return GLA_ERR_INVALID_ARG;
@@ -115,7 +127,10 @@ gla_status gla_fwd(const gla_problem* p, const void* q, const void* k, const voi
     cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, st);
     if (e != cudaSuccess) return GLA_ERR_CUDA;
     if ((size_t)P.B * P.H == 0) return GLA_OK;
-    e = simt::fwd(P, p->io, q, k, v, g, igate, h0, o, hT, ws, st);
+    if (plan == GLA_PLAN_TC && P.L > 0)
+        e = tc::fwd(P, q, k, v, g, igate, h0, o, hT, ws, st);
+    else
+        e = simt::fwd(P, p->io, q, k, v, g, igate, h0, o, hT, ws, st);
     return map_cuda(e);
 }
 
@@ -125,6 +140,8 @@ gla_status gla_bwd(const gla_problem* p, const void* q, const void* k, const voi
     Dims P;
     int plan;
     gla_status s = check_problem(p, &P, &plan);
+    if (s != GLA_OK) return s;
+    s = resolve(p, P, true, &plan);
     if (s != GLA_OK) return s;
     const bool empty = (size_t)P.B * P.H * P.L == 0;
     if (!empty && (!q || !k || !v || !dO || !dq || !dk || !dv)) return GLA_ERR_INVALID_ARG;

@@ -1,0 +1,632 @@
+// Tensor-core (tcgen05 / TMEM / TMA) forward of chunkwise gated linear attention, bf16 I/O.
+//
+// One CTA owns a (batch*head, Dv tile, sequence segment) and walks its segment in tiles
+// of 64 tokens, keeping the Dk x DVT state on chip: fp32 in registers (each thread owns
+// key-dim rows of it, the layout a tcgen05.ld of an M=128 accumulator delivers) and a
+// bf16 copy in shared memory as the B operand of the inter-chunk product. Per tile
+// (the chunk ("trunk") step of the talk summary "Hardware-Efficient Training of Linear
+// Attention Models", section 11:58, with the gates of the GLA abstract):
+//   b      = in-tile inclusive cumsum of the log-gate (fp32), Gamma = b at the last row
+//   q~     = q * e^b,   k~ = i * k * e^-b            (bf16, in place in the TMA tile)
+//   A      = q~ k~^T                (tcgen05, M=64 N=64 K=Dk, TMEM lanes 0-15 of each quadrant)
+//   O      = q~ S_prev              (tcgen05, M=64 N=DVT K=Dk, TMEM lanes 16-31)
+//   dS'    = k~^T V                 (tcgen05, M=128 (or 64) N=DVT K=64)
+//   P      = causal mask of A (bf16 in shared memory);  O += P V   (tcgen05)
+//   S      = diag(e^Gamma) (S_prev + dS')      (registers; bf16 copy for the next tile)
+//   o      = scale * O
+// q~ k~^T equals sum_d q_td k_sd e^(b_td - b_sd): the single in-tile reference point keeps
+// every exponent inside the tile's span. The state update uses k~ (not k e^(Gamma-b))
+// and applies e^Gamma to the rows afterwards, so one bf16 key tile serves both products.
+//
+// Plans: a single pass per (bh, Dv tile) when that fills the GPU; otherwise the
+// sequence is cut into segments (a multiple of the chunk size) processed in parallel:
+// a state-only pass gives each segment's local end state and total log-decay, a small
+// scan turns them into each segment's initial state, and the output pass starts every
+// segment from its initial state -- the two-level chunking of the Tiled Flash Linear
+// Attention abstract (large chunks, tiled inside, few materialised states).
+#include <cudaTypedefs.h>
+
+#include "gla_common.cuh"
+#include "gla_plans.h"
+#include "sm100.cuh"
+
+namespace gla {
+namespace tc {
+
+using namespace sm100;
+
+constexpr int TR = 64;        // tokens per tile
+constexpr int NTHR = 256;     // two warpgroups
+constexpr uint32_t BLK = 8192;  // one 64-column bf16 block of a 64-row tile (64 x 128 B)
+
+template <int DK, int DVT, int GATE, int MODE>
+struct Cfg {
+    // MODE 0: output pass (q, k, g, v). MODE 1: state-only pass (k, g, v).
+    static constexpr uint32_t QB = MODE == 0 ? TR * DK * 2 : 0;
+    static constexpr uint32_t KB = TR * DK * 2;
+    static constexpr uint32_t GB = GATE == 1 ? TR * DK * 4 : 0;
+    static constexpr uint32_t VB = TR * DVT * 2;
+    static constexpr uint32_t STAGE = QB + KB + GB + VB;
+    static constexpr uint32_t PB = MODE == 0 ? TR * TR * 2 : 0;
+    static constexpr uint32_t SB = MODE == 0 ? DK * DVT * 2 : 0;
+    static constexpr uint32_t SMALL = 4096 + 2 * DK * 4 + 4 * TR * 4 + 64;
+    static constexpr int NS = (2 * STAGE + PB + SB + SMALL + 1024 <= 227 * 1024) ? 2 : 1;
+    static constexpr uint32_t SMEM = NS * STAGE + PB + SB + SMALL + 1024;
+    static constexpr int NH = DK == 256 ? 2 : 1;            // M=128 halves of the state
+    static constexpr int MS = DK == 64 ? 64 : 128;           // M of the state MMA
+    static constexpr uint32_t COL_S = (MODE == 0) ? (DVT > 64 ? DVT : 64) : 0;
+    static constexpr uint32_t NCOL_USED = COL_S + NH * DVT;
+    static constexpr uint32_t NCOL = NCOL_USED <= 32 ? 32 : NCOL_USED <= 64 ? 64 : NCOL_USED <= 128 ? 128
+                                     : NCOL_USED <= 256 ? 256 : 512;
+    static constexpr int HALF = DVT / 2;                     // state columns per warpgroup
+    static_assert(STAGE % 1024 == 0, "stage alignment");
+    static_assert(SMEM <= 227 * 1024, "shared memory");
+    static_assert(HALF % 32 == 0, "column chunks");
+};
+
+struct FwdArgs {
+    const float* gh;      // per-head log-gate [BH*L] (GATE == 2)
+    const float* ig;      // input gate [BH*L] or null
+    const float* h0;      // [BH, Dk, Dv] or null
+    const float* sinit;   // [BH, nseg, Dk, Dv] initial states of segments z > 0 (output pass)
+    __nv_bfloat16* o;     // [BH, L, Dv]
+    float* hT;            // [BH, Dk, Dv] or null
+    float* seg_state;     // state-only pass: [BH, nseg, Dk, Dv] local end states
+    float* seg_gamma;     // state-only pass: [BH, nseg, Dk] total log-decay of the segment
+    int* status;
+    int tiles_per_seg;
+    int nseg;
+};
+
+__device__ __forceinline__ void store8_bf16(uint8_t* base, uint32_t off, const float* v) {
+    uint32_t w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        __nv_bfloat162 p = __floats2bfloat162_rn(v[2 * u], v[2 * u + 1]);
+        w[u] = *reinterpret_cast<uint32_t*>(&p);
+    }
+    *reinterpret_cast<uint4*>(base + off) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <int DK, int DVT, int GATE, int MODE>
+__global__ void __launch_bounds__(NTHR, 1)
+    k_tc_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+             const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg, FwdArgs A, Dims P) {
+    using C = Cfg<DK, DVT, GATE, MODE>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sP = sm + C::NS * C::STAGE;
+    uint8_t* sS = sP + C::PB;
+    uint8_t* small = sS + C::SB;
+    uint64_t* bar_full = reinterpret_cast<uint64_t*>(small);        // [2]
+    uint64_t* bar_mma1 = bar_full + 2;
+    uint64_t* bar_mma2 = bar_full + 3;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_full + 4);
+    float* tot = reinterpret_cast<float*>(small + 64);               // [512] cumsum group totals
+    float* gam = tot + 512 + 512;                                    // [DK] e^Gamma of the tile
+    float* gaml = gam + DK;                                          // [DK] Gamma of the tile
+    float* rowE = gaml + DK;                                         // [64] e^b   (per-head gate)
+    float* rowEi = rowE + TR;                                        // [64] e^-b
+    float* igs = rowEi + TR;                                         // [64] input gate
+    float* ghs = igs + TR;                                           // [64] per-head gate
+
+    const int bh = blockIdx.x, vt = blockIdx.y, z = blockIdx.z;
+    const int e0 = vt * DVT;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2, qd = warp & 3;
+    const int ntiles_all = cdiv(P.L, TR);
+    const int tile0 = z * A.tiles_per_seg;
+    const int tile1 = min(ntiles_all, tile0 + A.tiles_per_seg);
+    const int ntiles = tile1 - tile0;
+    const long rowbase = (long)bh * P.L;
+
+    if (tid == 0) {
+        mbar_init(&bar_full[0], 1);
+        mbar_init(&bar_full[1], 1);
+        mbar_init(bar_mma1, 1);
+        mbar_init(bar_mma2, 1);
+        mbar_fence_init();
+        if (MODE == 0) tma_prefetch_desc(&tq);
+        tma_prefetch_desc(&tk);
+        tma_prefetch_desc(&tv);
+        if (GATE == 1) tma_prefetch_desc(&tg);
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, C::NCOL);
+
+    // ---- state registers: thread owns rows d (per half) and HALF columns of the Dv tile
+    // M=128 layout: row d = 32*qd + lane. M=64 layout (DK == 64): row d = 16*qd + lane, lane < 16.
+    const bool srow_ok = (DK != 64) || (lane < 16);
+    float Sreg[C::NH][C::HALF];
+    float glog[C::NH];
+#pragma unroll
+    for (int h = 0; h < C::NH; ++h) {
+        const int d = (DK == 64 ? 16 * qd + (lane & 15) : 32 * qd + lane) + 128 * h;
+        glog[h] = 0.f;
+        const float* src = nullptr;
+        if (MODE == 0) {
+            if (z == 0) src = A.h0 ? A.h0 + ((long)bh * DK + d) * P.Dv : nullptr;
+            else src = A.sinit + (((long)bh * A.nseg + z) * DK + d) * P.Dv;
+        }
+#pragma unroll
+        for (int j = 0; j < C::HALF; ++j) Sreg[h][j] = (src && srow_ok) ? src[e0 + wg * C::HALF + j] : 0.f;
+    }
+    if (MODE == 0 && srow_ok) {
+#pragma unroll
+        for (int h = 0; h < C::NH; ++h) {
+            const int d = (DK == 64 ? 16 * qd + lane : 32 * qd + lane) + 128 * h;
+#pragma unroll
+            for (int j = 0; j < C::HALF; j += 8)
+                store8_bf16(sS, sw128_off(d, wg * C::HALF + j, DK * 128), &Sreg[h][j]);
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+
+    auto issue_loads = [&](int i, int s) {
+        uint8_t* st = sm + s * C::STAGE;
+        const int t0 = (tile0 + i) * TR;
+        mbar_arrive_expect_tx(&bar_full[s], C::STAGE);
+        if (MODE == 0)
+            for (int cb = 0; cb < DK / 64; ++cb) tma_load_3d(st + cb * BLK, &tq, cb * 64, t0, bh, &bar_full[s]);
+        for (int cb = 0; cb < DK / 64; ++cb) tma_load_3d(st + C::QB + cb * BLK, &tk, cb * 64, t0, bh, &bar_full[s]);
+        if (GATE == 1) tma_load_3d(st + C::QB + C::KB, &tg, 0, t0, bh, &bar_full[s]);
+        for (int vb = 0; vb < DVT / 64; ++vb)
+            tma_load_3d(st + C::QB + C::KB + C::GB + vb * BLK, &tv, e0 + vb * 64, t0, bh, &bar_full[s]);
+    };
+    if (tid == 0)
+        for (int i = 0; i < C::NS && i < ntiles; ++i) issue_loads(i, i);
+
+    int err = 0;
+    int issued_mma1 = 0, issued_mma2 = 0, consumed = 0;
+    for (int i = 0; i < ntiles; ++i) {
+        const int s = i % C::NS;
+        uint8_t* st = sm + s * C::STAGE;
+        uint8_t* sq = st;
+        uint8_t* sk = st + C::QB;
+        const float* sg = reinterpret_cast<const float*>(st + C::QB + C::KB);
+        uint8_t* sv = st + C::QB + C::KB + C::GB;
+        const int t0 = (tile0 + i) * TR;
+
+        // per-row scalars of this tile (plain loads, independent of the TMA stage)
+        if (tid < TR) {
+            const int t = t0 + tid;
+            igs[tid] = (A.ig && t < P.L) ? A.ig[rowbase + t] : 1.f;
+            if (GATE == 2) ghs[tid] = (t < P.L) ? A.gh[rowbase + t] : 0.f;
+        }
+        const bool ok = mbar_wait(&bar_full[s], (i / C::NS) & 1);
+        if (__syncthreads_or(!ok)) { err = 1; break; }
+        consumed = i + 1;
+
+        // ------------------------------------------------ transform (in place)
+        constexpr int NP = DK / 2, RG = NTHR / NP, RPG = TR / RG;
+        const int cp = tid % NP, rg = tid / NP, d = 2 * cp;
+        if (GATE == 1) {
+            float ax = 0.f, ay = 0.f;
+            for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
+                const float2 gv = *reinterpret_cast<const float2*>(sg + r * DK + d);
+                ax += gv.x;
+                ay += gv.y;
+            }
+            tot[rg * DK + d] = ax;
+            tot[rg * DK + d + 1] = ay;
+        } else if (GATE == 2) {
+            if (warp == 0) {   // warp scan over 64 rows, two rows per lane
+                const float g0 = ghs[2 * lane], g1 = ghs[2 * lane + 1];
+                float v = g0 + g1;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float n = __shfl_up_sync(0xffffffffu, v, off);
+                    if (lane >= off) v += n;
+                }
+                const float b1 = v, b0 = v - g1;
+                rowE[2 * lane] = __expf(b0);
+                rowE[2 * lane + 1] = __expf(b1);
+                rowEi[2 * lane] = __expf(-b0);
+                rowEi[2 * lane + 1] = __expf(-b1);
+                const float G = __shfl_sync(0xffffffffu, b1, 31);
+                if (lane == 0) { gam[0] = __expf(G); gaml[0] = G; }
+            }
+        }
+        __syncthreads();
+        {
+            float bx = 0.f, by = 0.f;
+            if (GATE == 1) {
+                float Gx = 0.f, Gy = 0.f;
+                for (int r2 = 0; r2 < RG; ++r2) {
+                    const float tx = tot[r2 * DK + d], ty = tot[r2 * DK + d + 1];
+                    if (r2 < rg) { bx += tx; by += ty; }
+                    Gx += tx;
+                    Gy += ty;
+                }
+                if (rg == 0) {
+                    gam[d] = __expf(Gx); gam[d + 1] = __expf(Gy);
+                    gaml[d] = Gx; gaml[d + 1] = Gy;
+                }
+            }
+            for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
+                float eqx = 1.f, eqy = 1.f, ekx = 1.f, eky = 1.f;
+                if (GATE == 1) {
+                    const float2 gv = *reinterpret_cast<const float2*>(sg + r * DK + d);
+                    bx += gv.x;
+                    by += gv.y;
+                    eqx = __expf(bx); eqy = __expf(by);
+                    ekx = __expf(-bx); eky = __expf(-by);
+                } else if (GATE == 2) {
+                    eqx = eqy = rowE[r];
+                    ekx = eky = rowEi[r];
+                }
+                const float iv = igs[r];
+                const uint32_t off = sw128_off(r, d, BLK);
+                if (MODE == 0) {
+                    __nv_bfloat162* pq = reinterpret_cast<__nv_bfloat162*>(sq + off);
+                    const float2 qf = __bfloat1622float2(*pq);
+                    *pq = __floats2bfloat162_rn(qf.x * eqx, qf.y * eqy);
+                }
+                __nv_bfloat162* pk = reinterpret_cast<__nv_bfloat162*>(sk + off);
+                const float2 kf = __bfloat1622float2(*pk);
+                *pk = __floats2bfloat162_rn(kf.x * iv * ekx, kf.y * iv * eky);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ------------------------------------------------ MMAs, group 1
+        if (tid == 0) {
+            const uint32_t qa = smem_u32(sq), ka = smem_u32(sk), va = smem_u32(sv);
+            if (MODE == 0) {
+                const uint32_t sa = smem_u32(sS);
+                const uint32_t idA = idesc_bf16(64, 64, 0, 0), idO = idesc_bf16(64, DVT, 0, 1);
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+                    mma_bf16(tbase, sw128_desc(qa + koff, 16, 1024), sw128_desc(ka + koff, 16, 1024), idA, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+                    mma_bf16(tbase + (16u << 16), sw128_desc(qa + koff, 16, 1024),
+                             sw128_desc(sa + kk * 2048, DK * 128, 1024), idO, kk > 0);
+                }
+            }
+            const uint32_t idS = idesc_bf16(C::MS, DVT, 1, 1);
+#pragma unroll
+            for (int h = 0; h < C::NH; ++h)
+#pragma unroll
+                for (int ks = 0; ks < TR / 16; ++ks)
+                    mma_bf16(tbase + C::COL_S + h * DVT, sw128_desc(ka + h * 2 * BLK + ks * 2048, BLK, 1024),
+                             sw128_desc(va + ks * 2048, BLK, 1024), idS, ks > 0);
+            mma_commit(bar_mma1);
+        }
+        ++issued_mma1;
+        {
+            const bool ok1 = mbar_wait(bar_mma1, i & 1);
+            if (__syncthreads_or(!ok1)) { err = 1; break; }
+        }
+        tc_fence_after();
+
+        // ------------------------------------------------ P = mask(A) -> shared
+        if (MODE == 0) {
+            uint32_t r[32];
+            tmem_ld32(tbase + ((uint32_t)(32 * qd) << 16) + 32 * wg, r);
+            tmem_wait_ld();
+            if (lane < 16) {
+                const int t = 16 * qd + lane;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    float f[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int sidx = 32 * wg + 8 * u + j;
+                        f[j] = (sidx <= t) ? __uint_as_float(r[8 * u + j]) : 0.f;
+                    }
+                    store8_bf16(sP, sw128_off(t, 32 * wg + 8 * u, BLK), f);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            if (tid == 0) {
+                const uint32_t pa = smem_u32(sP), va = smem_u32(sv);
+                const uint32_t idO = idesc_bf16(64, DVT, 0, 1);
+#pragma unroll
+                for (int ks = 0; ks < TR / 16; ++ks)
+                    mma_bf16(tbase + (16u << 16), sw128_desc(pa + ks * 32, 16, 1024),
+                             sw128_desc(va + ks * 2048, BLK, 1024), idO, 1);
+                mma_commit(bar_mma2);
+            }
+            ++issued_mma2;
+        }
+
+        // ------------------------------------------------ state update (overlaps P V)
+#pragma unroll
+        for (int h = 0; h < C::NH; ++h) {
+            const int d = (DK == 64 ? 16 * qd + (lane & 15) : 32 * qd + lane) + 128 * h;
+            const float eg = gam[GATE == 2 ? 0 : (GATE == 1 ? d : 0)];
+            const float gl = gaml[GATE == 2 ? 0 : (GATE == 1 ? d : 0)];
+            const float egv = GATE == 0 ? 1.f : eg;
+            if (GATE != 0) glog[h] += gl;
+#pragma unroll
+            for (int c = 0; c < C::HALF; c += 32) {
+                uint32_t r[32];
+                tmem_ld32(tbase + ((uint32_t)(32 * qd) << 16) + C::COL_S + h * DVT + wg * C::HALF + c, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) Sreg[h][c + j] = egv * (Sreg[h][c + j] + __uint_as_float(r[j]));
+            }
+            if (MODE == 0 && srow_ok) {
+#pragma unroll
+                for (int j = 0; j < C::HALF; j += 8)
+                    store8_bf16(sS, sw128_off(d, wg * C::HALF + j, DK * 128), &Sreg[h][j]);
+            }
+        }
+
+        // ------------------------------------------------ output
+        if (MODE == 0) {
+            const bool ok2 = mbar_wait(bar_mma2, i & 1);
+            if (__syncthreads_or(!ok2)) { err = 1; break; }
+            tc_fence_after();
+            const int t = 16 * qd + (lane & 15);
+            const bool row_ok = (lane >= 16) && (t0 + t < P.L);
+            __nv_bfloat16* orow = A.o + (rowbase + t0 + t) * P.Dv + e0 + wg * C::HALF;
+#pragma unroll
+            for (int c = 0; c < C::HALF; c += 32) {
+                uint32_t r[32];
+                tmem_ld32(tbase + ((uint32_t)(32 * qd) << 16) + wg * C::HALF + c, r);
+                tmem_wait_ld();
+                if (row_ok) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) {
+                            __nv_bfloat162 b2 = __floats2bfloat162_rn(P.scale * __uint_as_float(r[8 * u + 2 * p]),
+                                                                      P.scale * __uint_as_float(r[8 * u + 2 * p + 1]));
+                            w[p] = *reinterpret_cast<uint32_t*>(&b2);
+                        }
+                        *reinterpret_cast<uint4*>(orow + c + 8 * u) = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0 && i + C::NS < ntiles) issue_loads(i + C::NS, s);
+    }
+
+    if (err) {
+        if (tid == 0) {
+            atomicExch(A.status, kDevStatusTimeout);
+            // let every issued copy and product land before the shared memory and TMEM go away
+            for (int i = consumed; i < ntiles && i < consumed + C::NS; ++i)
+                mbar_wait(&bar_full[i % C::NS], (i / C::NS) & 1, 1u << 20);
+            if (issued_mma1) mbar_wait(bar_mma1, (issued_mma1 - 1) & 1, 1u << 20);
+            if (issued_mma2) mbar_wait(bar_mma2, (issued_mma2 - 1) & 1, 1u << 20);
+        }
+    } else if (srow_ok) {
+        // final state of the segment
+#pragma unroll
+        for (int h = 0; h < C::NH; ++h) {
+            const int d = (DK == 64 ? 16 * qd + lane : 32 * qd + lane) + 128 * h;
+            float* dst = nullptr;
+            if (MODE == 0) {
+                if (z == A.nseg - 1 && A.hT) dst = A.hT + ((long)bh * DK + d) * P.Dv;
+            } else {
+                dst = A.seg_state + (((long)bh * A.nseg + z) * DK + d) * P.Dv;
+                if (vt == 0 && wg == 0) A.seg_gamma[((long)bh * A.nseg + z) * DK + d] = glog[h];
+            }
+            if (dst)
+#pragma unroll
+                for (int j = 0; j < C::HALF; j += 4)
+                    *reinterpret_cast<float4*>(dst + e0 + wg * C::HALF + j) =
+                        make_float4(Sreg[h][j], Sreg[h][j + 1], Sreg[h][j + 2], Sreg[h][j + 3]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, C::NCOL);
+}
+
+// Segment scan: sinit[z] = e^{Gamma_{z-1}} sinit[z-1] + dS_{z-1}, sinit[0] = h0 (or 0).
+// One thread per (bh, d, e) element; loads a batch of segment values before the chain.
+__global__ void k_seg_scan(const float* __restrict__ seg_state, const float* __restrict__ seg_gamma,
+                           const float* __restrict__ h0, float* __restrict__ sinit, int BH, int Dk, int Dv, int nseg) {
+    const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long per = (long)Dk * Dv;
+    if (idx >= (long)BH * per) return;
+    const long bh = idx / per, de = idx % per;
+    const int d = (int)(de / Dv);
+    float S = h0 ? h0[idx] : 0.f;
+    constexpr int BATCH = 16;
+    for (int z0 = 0; z0 < nseg - 1; z0 += BATCH) {
+        float ds[BATCH], gl[BATCH];
+#pragma unroll
+        for (int u = 0; u < BATCH; ++u) {
+            const int z = z0 + u;
+            if (z < nseg - 1) {
+                ds[u] = seg_state[((bh * nseg + z) * per) + de];
+                gl[u] = seg_gamma[(bh * nseg + z) * Dk + d];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < BATCH; ++u) {
+            const int z = z0 + u;
+            if (z < nseg - 1) {
+                S = __expf(gl[u]) * S + ds[u];
+                sinit[((bh * nseg + z + 1) * per) + de] = S;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ host side
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 3D map over [BH][L][D] (D innermost) with a box of {box0, 64, 1}.
+static bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int D, int L, int BH,
+                     int box0, bool swz) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)L, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * esize, (cuuint64_t)D * esize * L};
+    cuuint32_t box[3] = {(cuuint32_t)box0, (cuuint32_t)TR, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int DK, int DVT, int GATE, int MODE>
+static cudaError_t launch_one(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                              const CUtensorMap& mg, const FwdArgs& a, const Dims& P, int nseg, cudaStream_t st) {
+    using C = Cfg<DK, DVT, GATE, MODE>;
+    auto kern = k_tc_fwd<DK, DVT, GATE, MODE>;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    dim3 grid(P.B * P.H, P.Dv / DVT, nseg);
+    GLA_LAUNCH(MODE == 0 ? "tc_fwd" : "tc_fwd_state", st, kern<<<grid, NTHR, C::SMEM, st>>>(mq, mk, mv, mg, a, P));
+    return cudaGetLastError();
+}
+
+int pick_dvt(const Dims& P) { return (P.Dk == 256 || P.Dv % 128 != 0) ? 64 : 128; }
+
+static int num_sms() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+FwdPlan plan_fwd(const Dims& P) {
+    FwdPlan pl{};
+    pl.dvt = pick_dvt(P);
+    const int ntiles = cdiv(P.L, TR);
+    const long base = (long)P.B * P.H * (P.Dv / pl.dvt);
+    const int sms = num_sms();
+    int nseg = 1;
+    if (base * 4 < (long)sms * 3 && ntiles > 1) nseg = (int)((long)sms / base);
+    if (nseg < 1) nseg = 1;
+    // segments are whole chunks (the chunk is a multiple of the 64-token tile)
+    const int tiles_per_chunk = P.C / TR;
+    const int nchunks = cdiv(P.L, P.C);
+    if (nseg > nchunks) nseg = nchunks;
+    int chunks_per_seg = cdiv(nchunks, nseg);
+    pl.tiles_per_seg = chunks_per_seg * tiles_per_chunk;
+    pl.nseg = cdiv(ntiles, pl.tiles_per_seg);
+    if (pl.nseg < 1) pl.nseg = 1;
+    return pl;
+}
+
+size_t fwd_workspace_bytes(const Dims& P) {
+    const FwdPlan pl = plan_fwd(P);
+    if (pl.nseg <= 1) return kStatusBytes;
+    const size_t BH = (size_t)P.B * P.H;
+    size_t off = kStatusBytes;
+    off = align_up(off + 4 * BH * pl.nseg * P.Dk * P.Dv, 256);   // local end states
+    off = align_up(off + 4 * BH * pl.nseg * P.Dk, 256);          // log-decay totals
+    off = align_up(off + 4 * BH * pl.nseg * P.Dk * P.Dv, 256);   // initial states
+    return off;
+}
+
+bool supports(const Dims& P) {
+    return P.C % TR == 0 && (P.Dk == 64 || P.Dk == 128 || P.Dk == 256) && P.Dv % 64 == 0;
+}
+
+template <int DK, int DVT, int GATE>
+static cudaError_t run(const Dims& P, const void* q, const void* k, const void* v, const float* g,
+                       const float* ig, const float* h0, void* o, float* hT, void* ws, cudaStream_t st) {
+    const FwdPlan pl = plan_fwd(P);
+    CUtensorMap mq, mk, mv, mg;
+    const int BH = P.B * P.H;
+    if (!make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dk, P.L, BH, 64, true) ||
+        !make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dk, P.L, BH, 64, true) ||
+        !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dv, P.L, BH, 64, true))
+        return cudaErrorInvalidValue;
+    if (GATE == 1) {
+        if (!make_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, P.Dk, P.L, BH, P.Dk, false))
+            return cudaErrorInvalidValue;
+    } else {
+        mg = mk;  // unused
+    }
+    FwdArgs a{};
+    a.gh = GATE == 2 ? g : nullptr;
+    a.ig = ig;
+    a.h0 = h0;
+    a.o = static_cast<__nv_bfloat16*>(o);
+    a.hT = hT;
+    a.status = static_cast<int*>(ws);
+    a.tiles_per_seg = pl.tiles_per_seg;
+    a.nseg = pl.nseg;
+    if (pl.nseg > 1) {
+        char* w = static_cast<char*>(ws);
+        size_t off = kStatusBytes;
+        a.seg_state = reinterpret_cast<float*>(w + off);
+        off = align_up(off + 4 * (size_t)BH * pl.nseg * P.Dk * P.Dv, 256);
+        a.seg_gamma = reinterpret_cast<float*>(w + off);
+        off = align_up(off + 4 * (size_t)BH * pl.nseg * P.Dk, 256);
+        a.sinit = reinterpret_cast<float*>(w + off);
+        // local end states of every segment but the last
+        Dims Ps = P;
+        cudaError_t e = launch_one<DK, DVT, GATE, 1>(mq, mk, mv, mg, a, Ps, pl.nseg - 1, st);
+        if (e != cudaSuccess) return e;
+        const long n = (long)BH * P.Dk * P.Dv;
+        GLA_LAUNCH("tc_seg_scan", st,
+                   k_seg_scan<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+                       a.seg_state, a.seg_gamma, h0, const_cast<float*>(a.sinit), BH, P.Dk, P.Dv, pl.nseg));
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return launch_one<DK, DVT, GATE, 0>(mq, mk, mv, mg, a, P, pl.nseg, st);
+}
+
+template <int DK, int DVT>
+static cudaError_t run_gate(const Dims& P, const void* q, const void* k, const void* v, const float* g,
+                            const float* ig, const float* h0, void* o, float* hT, void* ws, cudaStream_t st) {
+    switch (P.gate) {
+        case GLA_GATE_NONE: return run<DK, DVT, 0>(P, q, k, v, g, ig, h0, o, hT, ws, st);
+        case GLA_GATE_PER_KEY: return run<DK, DVT, 1>(P, q, k, v, g, ig, h0, o, hT, ws, st);
+        default: return run<DK, DVT, 2>(P, q, k, v, g, ig, h0, o, hT, ws, st);
+    }
+}
+
+cudaError_t fwd(const Dims& P, const void* q, const void* k, const void* v, const float* g, const float* ig,
+                const float* h0, void* o, float* hT, void* ws, cudaStream_t st) {
+    const int dvt = pick_dvt(P);
+    if (P.Dk == 64) {
+        if (dvt == 128) return run_gate<64, 128>(P, q, k, v, g, ig, h0, o, hT, ws, st);
+        return run_gate<64, 64>(P, q, k, v, g, ig, h0, o, hT, ws, st);
+    }
+    if (P.Dk == 128) {
+        if (dvt == 128) return run_gate<128, 128>(P, q, k, v, g, ig, h0, o, hT, ws, st);
+        return run_gate<128, 64>(P, q, k, v, g, ig, h0, o, hT, ws, st);
+    }
+    return run_gate<256, 64>(P, q, k, v, g, ig, h0, o, hT, ws, st);
+}
+
+}  // namespace tc
+}  // namespace gla

@@ -150,7 +150,8 @@ def test_gate_modes(gate, ig, dtype):
 
 def test_initial_state_is_carried():
     """Weak decay (g ~ -0.001) so h0 matters over the whole sequence."""
-    w = I.WORKLOADS["c4"].replace(B=1, H=2, L=256, Dk=64, Dv=64, dtype="f32", gate_div=800.0, chunk=64)
+    w = I.WORKLOADS["c4"].replace(B=1, H=2, L=256, Dk=64, Dv=64, dtype="f32", gate_div=800.0, chunk=64,
+                                  h0_std=3.0)
     x = I.make_inputs(w, seed=6)
     ro, _ = oracle.gla_fwd(x["q"], x["k"], x["v"], x["g"], None, None, w.scale)
     rh, _ = oracle.gla_fwd(x["q"], x["k"], x["v"], x["g"], None, x["h0"], w.scale)

@@ -1,0 +1,116 @@
+"""GPU parity of the tensor-core (tcgen05) plan against the float64 oracle.
+
+Covers the single-pass plan (enough (batch*head, Dv tile) pairs to fill the GPU) and
+the segmented plan (few heads: segment states, scan, output pass), ragged tails, head
+dims, gate modes, the input gate, initial and final states. bf16 I/O, bound 1e-2 on the
+max-normalised error of every output.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_rnn_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def f64(t):
+    return None if t is None else t.detach().to("cpu", torch.float64).numpy()
+
+
+def err(got, ref):
+    return float(np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-30))
+
+
+def run_tc_fwd(w, seed, plan="tc"):
+    from linear_rnn_b200 import ops
+    x = I.make_inputs(w, seed=seed)
+    xd = {k: (None if v is None else v.cuda()) for k, v in x.items()}
+    o, hT = ops.gla_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["igate"], xd["h0"], scale=w.scale, chunk=w.chunk,
+                        plan=plan)
+    ro, rhT = oracle.gla_fwd(x["q"], x["k"], x["v"], x["g"], x["igate"], x["h0"], w.scale)
+    return err(f64(o), ro), err(f64(hT), rhT)
+
+
+def base(**kw):
+    w = I.WORKLOADS["c3"].replace(dtype="bf16", backward=False, chunk=64)
+    return w.replace(**kw)
+
+
+@pytest.mark.parametrize("L", [1, 40, 64, 65, 200, 1000])
+def test_tc_segmented_ragged(L):
+    w = base(B=1, H=2, L=L, Dk=128, Dv=128, h0_std=0.5)
+    eo, eh = run_tc_fwd(w, 11)
+    assert eo <= TOL and eh <= TOL, (eo, eh)
+
+
+@pytest.mark.parametrize("L", [64, 130, 700])
+def test_tc_single_pass(L):
+    # 4*32 heads x 1 Dv tile = 128 CTAs: one pass per (head, Dv tile)
+    w = base(B=4, H=32, L=L, Dk=64, Dv=64, h0_std=0.3)
+    eo, eh = run_tc_fwd(w, 12)
+    assert eo <= TOL and eh <= TOL, (eo, eh)
+
+
+@pytest.mark.parametrize("Dk,Dv", [(64, 64), (64, 128), (128, 64), (128, 128), (128, 256), (256, 64), (256, 256),
+                                   (64, 256)])
+def test_tc_head_dims(Dk, Dv):
+    w = base(B=1, H=3, L=333, Dk=Dk, Dv=Dv, h0_std=0.2)
+    eo, eh = run_tc_fwd(w, 13)
+    assert eo <= TOL and eh <= TOL, (eo, eh)
+
+
+@pytest.mark.parametrize("gate,ig", [(I.GATE_NONE, False), (I.GATE_PER_HEAD, False), (I.GATE_PER_HEAD, True),
+                                     (I.GATE_PER_KEY, True), (I.GATE_NONE, True)])
+def test_tc_gate_modes(gate, ig):
+    w = base(B=2, H=2, L=300, Dk=128, Dv=128, gate=gate, input_gate=ig, h0_std=0.4,
+             gate_mean=3.0 if gate == I.GATE_PER_HEAD else 0.0, gate_div=1.0 if gate == I.GATE_PER_HEAD else 16.0)
+    eo, eh = run_tc_fwd(w, 14)
+    assert eo <= TOL and eh <= TOL, (eo, eh)
+
+
+@pytest.mark.parametrize("chunk", [64, 128, 256, 1024])
+def test_tc_chunk_sizes(chunk):
+    w = base(B=1, H=2, L=2500, Dk=128, Dv=128, chunk=chunk, h0_std=0.3)
+    eo, eh = run_tc_fwd(w, 15)
+    assert eo <= TOL and eh <= TOL, (eo, eh)
+
+
+def test_tc_rejects_fp32_and_odd_chunks():
+    from linear_rnn_b200 import ops
+    from linear_rnn_b200._lib import GlaError
+    q = torch.zeros(1, 1, 64, 64, device="cuda")
+    with pytest.raises(GlaError):
+        ops.gla_fwd(q, q, q, None, scale=1.0, chunk=64, plan="tc")
+    qb = q.bfloat16()
+    with pytest.raises(GlaError):
+        ops.gla_fwd(qb, qb, qb, None, scale=1.0, chunk=48, plan="tc")
+
+
+def test_tc_matches_simt_plan():
+    """Both GPU plans against each other (bf16 outputs; they round differently)."""
+    from linear_rnn_b200 import ops
+    w = base(B=2, H=4, L=513, Dk=128, Dv=128, h0_std=0.2)
+    x = {k: (None if v is None else v.cuda()) for k, v in I.make_inputs(w, seed=16).items()}
+    a = ops.gla_fwd(x["q"], x["k"], x["v"], x["g"], None, x["h0"], scale=w.scale, plan="tc")
+    b = ops.gla_fwd(x["q"], x["k"], x["v"], x["g"], None, x["h0"], scale=w.scale, plan="simt")
+    assert err(f64(a[0]), f64(b[0])) < 1e-2
+    assert err(f64(a[1]), f64(b[1])) < 1e-2
+
+
+def test_tc_deterministic():
+    from linear_rnn_b200 import ops
+    w = base(B=1, H=2, L=900, Dk=128, Dv=128)
+    x = {k: (None if v is None else v.cuda()) for k, v in I.make_inputs(w, seed=17).items()}
+    a = ops.gla_fwd(x["q"], x["k"], x["v"], x["g"], scale=w.scale, plan="tc")
+    b = ops.gla_fwd(x["q"], x["k"], x["v"], x["g"], scale=w.scale, plan="tc")
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
