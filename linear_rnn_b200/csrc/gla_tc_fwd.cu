@@ -36,7 +36,6 @@ namespace tc {
 using namespace sm100;
 
 constexpr int TR = 64;        // tokens per tile
-constexpr int NTHR = 256;     // two warpgroups
 constexpr uint32_t BLK = 8192;  // one 64-column bf16 block of a 64-row tile (64 x 128 B)
 
 template <int DK, int DVT, int GATE, int MODE>
@@ -47,21 +46,22 @@ struct Cfg {
     static constexpr uint32_t GB = GATE == 1 ? TR * DK * 4 : 0;
     static constexpr uint32_t VB = TR * DVT * 2;
     static constexpr uint32_t STAGE = QB + KB + GB + VB;
-    static constexpr uint32_t PB = MODE == 0 ? TR * TR * 2 : 0;
-    static constexpr uint32_t SB = MODE == 0 ? DK * DVT * 2 : 0;
-    static constexpr uint32_t SMALL = 4096 + 2 * DK * 4 + 4 * TR * 4 + 64;
+    static constexpr uint32_t PB = MODE == 0 ? 2 * TR * TR * 2 : 0;   // P, double-buffered
+    static constexpr uint32_t SB = MODE == 0 ? DK * DVT * 2 : 0;      // bf16 state
+    static constexpr uint32_t SMALL = 256 + 4096 + 16 * DK + 1024;
     static constexpr int NS = (2 * STAGE + PB + SB + SMALL + 1024 <= 227 * 1024) ? 2 : 1;
     static constexpr uint32_t SMEM = NS * STAGE + PB + SB + SMALL + 1024;
     static constexpr int NH = DK == 256 ? 2 : 1;            // M=128 halves of the state
     static constexpr int MS = DK == 64 ? 64 : 128;           // M of the state MMA
     static constexpr uint32_t COL_S = (MODE == 0) ? (DVT > 64 ? DVT : 64) : 0;
-    static constexpr uint32_t NCOL_USED = COL_S + NH * DVT;
-    static constexpr uint32_t NCOL = NCOL_USED <= 32 ? 32 : NCOL_USED <= 64 ? 64 : NCOL_USED <= 128 ? 128
-                                     : NCOL_USED <= 256 ? 256 : 512;
+    static constexpr uint32_t BUF_USED = COL_S + NH * DVT;
+    static constexpr uint32_t BUFCOLS = BUF_USED <= 32 ? 32 : BUF_USED <= 64 ? 64 : BUF_USED <= 128 ? 128 : 256;
+    static constexpr uint32_t NCOL = 2 * BUFCOLS;            // two accumulator buffers
     static constexpr int HALF = DVT / 2;                     // state columns per warpgroup
     static_assert(STAGE % 1024 == 0, "stage alignment");
     static_assert(SMEM <= 227 * 1024, "shared memory");
     static_assert(HALF % 32 == 0, "column chunks");
+    static_assert(BUF_USED <= 256 && NCOL <= 512, "tensor memory");
 };
 
 struct FwdArgs {
@@ -88,74 +88,86 @@ __device__ __forceinline__ void store8_bf16(uint8_t* base, uint32_t off, const f
     *reinterpret_cast<uint4*>(base + off) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// Thread roles: warps 0-7 (two warpgroups) transform tiles and run the epilogues; warp 8
+// issues the tcgen05 MMAs; warp 9 issues the TMA loads. They hand tiles to each other
+// through mbarriers, so the transform of tile i+1 runs while the tensor core works on
+// tile i, and the epilogues of tile i overlap the MMAs of tile i+1 (two TMEM buffers).
+constexpr int NCOMP = 256;
+constexpr int NTHR_WS = NCOMP + 64;
+constexpr int BAR_COMP = 1;   // named barrier of the 256 compute threads
+
 template <int DK, int DVT, int GATE, int MODE>
-__global__ void __launch_bounds__(NTHR, 1)
+__global__ void __launch_bounds__(NTHR_WS, 1)
     k_tc_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
              const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg, FwdArgs A, Dims P) {
     using C = Cfg<DK, DVT, GATE, MODE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sP = sm + C::NS * C::STAGE;
-    uint8_t* sS = sP + C::PB;
+    uint8_t* sPb = sm + C::NS * C::STAGE;
+    uint8_t* sS = sPb + C::PB;
     uint8_t* small = sS + C::SB;
-    uint64_t* bar_full = reinterpret_cast<uint64_t*>(small);        // [2]
-    uint64_t* bar_mma1 = bar_full + 2;
-    uint64_t* bar_mma2 = bar_full + 3;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_full + 4);
-    float* tot = reinterpret_cast<float*>(small + 64);               // [512] cumsum group totals
-    float* gam = tot + 512 + 512;                                    // [DK] e^Gamma of the tile
-    float* gaml = gam + DK;                                          // [DK] Gamma of the tile
-    float* rowE = gaml + DK;                                         // [64] e^b   (per-head gate)
-    float* rowEi = rowE + TR;                                        // [64] e^-b
-    float* igs = rowEi + TR;                                         // [64] input gate
-    float* ghs = igs + TR;                                           // [64] per-head gate
+    uint64_t* bars = reinterpret_cast<uint64_t*>(small);
+    uint64_t* bar_full = bars + 0;     // [2] TMA landed
+    uint64_t* bar_empty = bars + 2;    // [2] stage's MMAs done
+    uint64_t* bar_trans = bars + 4;    // [2] stage transformed
+    uint64_t* bar_mma1 = bars + 6;     // [2] A, dS', O_inter of the buffer done
+    uint64_t* bar_mma2 = bars + 8;     // [2] P V done
+    uint64_t* bar_pready = bars + 10;  // [2] P written
+    uint64_t* bar_tfree = bars + 12;   // [2] TMEM buffer read out
+    uint64_t* bar_sready = bars + 14;  // bf16 state of the last tile written
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 128);
+    volatile int* abortp = reinterpret_cast<volatile int*>(small + 132);
+    int* n_issued = reinterpret_cast<int*>(small + 136);
+    int* n_consumed = reinterpret_cast<int*>(small + 140);
+    int* n_mma1 = reinterpret_cast<int*>(small + 144);
+    int* n_mma2 = reinterpret_cast<int*>(small + 148);
+    float* tot = reinterpret_cast<float*>(small + 256);      // [1024] cumsum group totals
+    float* gamb = tot + 1024;                                // [2][DK] e^Gamma per buffer
+    float* gamlb = gamb + 2 * DK;                            // [2][DK] Gamma per buffer
+    float* rowE = gamlb + 2 * DK;                            // [64] e^b   (per-head gate)
+    float* rowEi = rowE + TR;                                // [64] e^-b
+    float* igs = rowEi + TR;                                 // [64] input gate
+    float* ghs = igs + TR;                                   // [64] per-head gate
 
     const int bh = blockIdx.x, vt = blockIdx.y, z = blockIdx.z;
     const int e0 = vt * DVT;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2, qd = warp & 3;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = (warp >> 2) & 1, qd = warp & 3;
     const int ntiles_all = cdiv(P.L, TR);
     const int tile0 = z * A.tiles_per_seg;
-    const int tile1 = min(ntiles_all, tile0 + A.tiles_per_seg);
-    const int ntiles = tile1 - tile0;
+    const int ntiles = min(ntiles_all, tile0 + A.tiles_per_seg) - tile0;
     const long rowbase = (long)bh * P.L;
 
     if (tid == 0) {
-        mbar_init(&bar_full[0], 1);
-        mbar_init(&bar_full[1], 1);
-        mbar_init(bar_mma1, 1);
-        mbar_init(bar_mma2, 1);
+        for (int j = 0; j < 15; ++j) mbar_init(&bars[j], 1);
+        *abortp = 0;
+        *n_issued = 0;
+        *n_consumed = 0;
+        *n_mma1 = 0;
+        *n_mma2 = 0;
         mbar_fence_init();
-        if (MODE == 0) tma_prefetch_desc(&tq);
-        tma_prefetch_desc(&tk);
-        tma_prefetch_desc(&tv);
-        if (GATE == 1) tma_prefetch_desc(&tg);
     }
     if (warp == 0) tmem_alloc(tmem_slot, C::NCOL);
 
-    // ---- state registers: thread owns rows d (per half) and HALF columns of the Dv tile
-    // M=128 layout: row d = 32*qd + lane. M=64 layout (DK == 64): row d = 16*qd + lane, lane < 16.
+    // ---- compute threads: state registers (rows d, HALF columns of the Dv tile)
     const bool srow_ok = (DK != 64) || (lane < 16);
     float Sreg[C::NH][C::HALF];
     float glog[C::NH];
-#pragma unroll
-    for (int h = 0; h < C::NH; ++h) {
-        const int d = (DK == 64 ? 16 * qd + (lane & 15) : 32 * qd + lane) + 128 * h;
-        glog[h] = 0.f;
-        const float* src = nullptr;
-        if (MODE == 0) {
-            if (z == 0) src = A.h0 ? A.h0 + ((long)bh * DK + d) * P.Dv : nullptr;
-            else src = A.sinit + (((long)bh * A.nseg + z) * DK + d) * P.Dv;
-        }
-#pragma unroll
-        for (int j = 0; j < C::HALF; ++j) Sreg[h][j] = (src && srow_ok) ? src[e0 + wg * C::HALF + j] : 0.f;
-    }
-    if (MODE == 0 && srow_ok) {
+    if (tid < NCOMP) {
 #pragma unroll
         for (int h = 0; h < C::NH; ++h) {
-            const int d = (DK == 64 ? 16 * qd + lane : 32 * qd + lane) + 128 * h;
+            const int d = (DK == 64 ? 16 * qd + (lane & 15) : 32 * qd + lane) + 128 * h;
+            glog[h] = 0.f;
+            const float* src = nullptr;
+            if (MODE == 0) {
+                if (z == 0) src = A.h0 ? A.h0 + ((long)bh * DK + d) * P.Dv : nullptr;
+                else src = A.sinit + (((long)bh * A.nseg + z) * DK + d) * P.Dv;
+            }
 #pragma unroll
-            for (int j = 0; j < C::HALF; j += 8)
-                store8_bf16(sS, sw128_off(d, wg * C::HALF + j, DK * 128), &Sreg[h][j]);
+            for (int j = 0; j < C::HALF; ++j) Sreg[h][j] = (src && srow_ok) ? src[e0 + wg * C::HALF + j] : 0.f;
+            if (MODE == 0 && srow_ok)
+#pragma unroll
+                for (int j = 0; j < C::HALF; j += 8)
+                    store8_bf16(sS, sw128_off(d, wg * C::HALF + j, DK * 128), &Sreg[h][j]);
         }
     }
     fence_proxy_async_smem();
@@ -164,85 +176,158 @@ __global__ void __launch_bounds__(NTHR, 1)
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
 
-    auto issue_loads = [&](int i, int s) {
-        uint8_t* st = sm + s * C::STAGE;
-        const int t0 = (tile0 + i) * TR;
-        mbar_arrive_expect_tx(&bar_full[s], C::STAGE);
-        if (MODE == 0)
-            for (int cb = 0; cb < DK / 64; ++cb) tma_load_3d(st + cb * BLK, &tq, cb * 64, t0, bh, &bar_full[s]);
-        for (int cb = 0; cb < DK / 64; ++cb) tma_load_3d(st + C::QB + cb * BLK, &tk, cb * 64, t0, bh, &bar_full[s]);
-        if (GATE == 1) tma_load_3d(st + C::QB + C::KB, &tg, 0, t0, bh, &bar_full[s]);
-        for (int vb = 0; vb < DVT / 64; ++vb)
-            tma_load_3d(st + C::QB + C::KB + C::GB + vb * BLK, &tv, e0 + vb * 64, t0, bh, &bar_full[s]);
-    };
-    if (tid == 0)
-        for (int i = 0; i < C::NS && i < ntiles; ++i) issue_loads(i, i);
-
-    int err = 0;
-    int issued_mma1 = 0, issued_mma2 = 0, consumed = 0;
-    for (int i = 0; i < ntiles; ++i) {
-        const int s = i % C::NS;
-        uint8_t* st = sm + s * C::STAGE;
-        uint8_t* sq = st;
-        uint8_t* sk = st + C::QB;
-        const float* sg = reinterpret_cast<const float*>(st + C::QB + C::KB);
-        uint8_t* sv = st + C::QB + C::KB + C::GB;
-        const int t0 = (tile0 + i) * TR;
-
-        // per-row scalars of this tile (plain loads, independent of the TMA stage)
-        if (tid < TR) {
-            const int t = t0 + tid;
-            igs[tid] = (A.ig && t < P.L) ? A.ig[rowbase + t] : 1.f;
-            if (GATE == 2) ghs[tid] = (t < P.L) ? A.gh[rowbase + t] : 0.f;
-        }
-        const bool ok = mbar_wait(&bar_full[s], (i / C::NS) & 1);
-        if (__syncthreads_or(!ok)) { err = 1; break; }
-        consumed = i + 1;
-
-        // ------------------------------------------------ transform (in place)
-        constexpr int NP = DK / 2, RG = NTHR / NP, RPG = TR / RG;
-        const int cp = tid % NP, rg = tid / NP, d = 2 * cp;
-        if (GATE == 1) {
-            float ax = 0.f, ay = 0.f;
-            for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
-                const float2 gv = *reinterpret_cast<const float2*>(sg + r * DK + d);
-                ax += gv.x;
-                ay += gv.y;
+    if (warp == 9) {
+        // ================================================================ TMA producer
+        if (lane == 0) {
+            if (MODE == 0) tma_prefetch_desc(&tq);
+            tma_prefetch_desc(&tk);
+            tma_prefetch_desc(&tv);
+            if (GATE == 1) tma_prefetch_desc(&tg);
+            for (int j = 0; j < ntiles; ++j) {
+                const int s = j % C::NS;
+                if (j >= C::NS && !mbar_wait_abort(&bar_empty[s], ((j / C::NS) - 1) & 1, abortp)) break;
+                uint8_t* st = sm + s * C::STAGE;
+                const int t0 = (tile0 + j) * TR;
+                mbar_arrive_expect_tx(&bar_full[s], C::STAGE);
+                if (MODE == 0)
+                    for (int cb = 0; cb < DK / 64; ++cb)
+                        tma_load_3d(st + cb * BLK, &tq, cb * 64, t0, bh, &bar_full[s]);
+                for (int cb = 0; cb < DK / 64; ++cb)
+                    tma_load_3d(st + C::QB + cb * BLK, &tk, cb * 64, t0, bh, &bar_full[s]);
+                if (GATE == 1) tma_load_3d(st + C::QB + C::KB, &tg, 0, t0, bh, &bar_full[s]);
+                for (int vb = 0; vb < DVT / 64; ++vb)
+                    tma_load_3d(st + C::QB + C::KB + C::GB + vb * BLK, &tv, e0 + vb * 64, t0, bh, &bar_full[s]);
+                *n_issued = j + 1;
             }
-            tot[rg * DK + d] = ax;
-            tot[rg * DK + d + 1] = ay;
-        } else if (GATE == 2) {
-            if (warp == 0) {   // warp scan over 64 rows, two rows per lane
-                const float g0 = ghs[2 * lane], g1 = ghs[2 * lane + 1];
-                float v = g0 + g1;
+        }
+    } else if (warp == 8) {
+        // ================================================================ MMA issuer
+        if (lane == 0) {
+            for (int i = 0; i < ntiles; ++i) {
+                const int s = i % C::NS, b = i & 1;
+                if (!mbar_wait_abort(&bar_trans[s], (i / C::NS) & 1, abortp)) break;
+                if (i >= 2 && !mbar_wait_abort(&bar_tfree[b], ((i >> 1) - 1) & 1, abortp)) break;
+                tc_fence_after();
+                uint8_t* st = sm + s * C::STAGE;
+                const uint32_t qa = smem_u32(st), ka = smem_u32(st + C::QB), va = smem_u32(st + C::QB + C::KB + C::GB);
+                const uint32_t tb = tbase + b * C::BUFCOLS;
+                if (MODE == 0) {
+                    const uint32_t idA = idesc_bf16(64, 64, 0, 0);
 #pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float n = __shfl_up_sync(0xffffffffu, v, off);
-                    if (lane >= off) v += n;
+                    for (int kk = 0; kk < DK / 16; ++kk) {
+                        const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+                        mma_bf16(tb, sw128_desc(qa + koff, 16, 1024), sw128_desc(ka + koff, 16, 1024), idA, kk > 0);
+                    }
                 }
-                const float b1 = v, b0 = v - g1;
-                rowE[2 * lane] = __expf(b0);
-                rowE[2 * lane + 1] = __expf(b1);
-                rowEi[2 * lane] = __expf(-b0);
-                rowEi[2 * lane + 1] = __expf(-b1);
-                const float G = __shfl_sync(0xffffffffu, b1, 31);
-                if (lane == 0) { gam[0] = __expf(G); gaml[0] = G; }
+                const uint32_t idS = idesc_bf16(C::MS, DVT, 1, 1);
+#pragma unroll
+                for (int h = 0; h < C::NH; ++h)
+#pragma unroll
+                    for (int ks = 0; ks < TR / 16; ++ks)
+                        mma_bf16(tb + C::COL_S + h * DVT, sw128_desc(ka + h * 2 * BLK + ks * 2048, BLK, 1024),
+                                 sw128_desc(va + ks * 2048, BLK, 1024), idS, ks > 0);
+                if (MODE == 0) {
+                    if (i >= 1) {
+                        if (!mbar_wait_abort(bar_sready, (i - 1) & 1, abortp)) break;
+                        tc_fence_after();
+                    }
+                    const uint32_t sa = smem_u32(sS);
+                    const uint32_t idO = idesc_bf16(64, DVT, 0, 1);
+#pragma unroll
+                    for (int kk = 0; kk < DK / 16; ++kk) {
+                        const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+                        mma_bf16(tb + (16u << 16), sw128_desc(qa + koff, 16, 1024),
+                                 sw128_desc(sa + kk * 2048, DK * 128, 1024), idO, kk > 0);
+                    }
+                }
+                mma_commit(&bar_mma1[b]);
+                *n_mma1 = i + 1;
+                if (MODE == 0) {
+                    if (!mbar_wait_abort(&bar_pready[b], (i >> 1) & 1, abortp)) break;
+                    tc_fence_after();
+                    const uint32_t pa = smem_u32(sPb + b * (TR * TR * 2));
+                    const uint32_t idO = idesc_bf16(64, DVT, 0, 1);
+#pragma unroll
+                    for (int ks = 0; ks < TR / 16; ++ks)
+                        mma_bf16(tb + (16u << 16), sw128_desc(pa + ks * 32, 16, 1024),
+                                 sw128_desc(va + ks * 2048, BLK, 1024), idO, 1);
+                    mma_commit(&bar_mma2[b]);
+                    *n_mma2 = i + 1;
+                }
+                if (i + C::NS < ntiles) mma_commit(&bar_empty[s]);
             }
         }
-        __syncthreads();
-        {
+    } else {
+        // ================================================================ compute warpgroups
+        const int ctid = tid;  // 0..255
+        // Transform tile j in place: q~ = q e^b, k~ = i k e^-b; e^Gamma into buffer j&1.
+        auto transform = [&](int j) -> bool {
+            const int s = j % C::NS, b = j & 1;
+            uint8_t* st = sm + s * C::STAGE;
+            uint8_t* sq = st;
+            uint8_t* sk = st + C::QB;
+            const float* sg = reinterpret_cast<const float*>(st + C::QB + C::KB);
+            float* gam = gamb + b * DK;
+            float* gaml = gamlb + b * DK;
+            const int t0 = (tile0 + j) * TR;
+            if (ctid < TR) {
+                const int t = t0 + ctid;
+                igs[ctid] = (A.ig && t < P.L) ? A.ig[rowbase + t] : 1.f;
+                if (GATE == 2) ghs[ctid] = (t < P.L) ? A.gh[rowbase + t] : 0.f;
+            }
+            const bool ok = mbar_wait_abort(&bar_full[s], (j / C::NS) & 1, abortp);
+            if (!named_bar_and(BAR_COMP, NCOMP, ok)) return false;
+            if (ctid == 0) *n_consumed = j + 1;
+            constexpr int NP = DK / 2, RG = NCOMP / NP, RPG = TR / RG;
+            const int cp = ctid % NP, rg = ctid / NP, d = 2 * cp;
+            if (GATE == 1) {
+                float ax = 0.f, ay = 0.f;
+                for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
+                    const float2 gv = *reinterpret_cast<const float2*>(sg + r * DK + d);
+                    ax += gv.x;
+                    ay += gv.y;
+                }
+                tot[rg * DK + d] = ax;
+                tot[rg * DK + d + 1] = ay;
+            } else if (GATE == 2) {
+                if (warp == 0) {  // warp scan over 64 rows, two rows per lane
+                    const float g0 = ghs[2 * lane], g1 = ghs[2 * lane + 1];
+                    float v = g0 + g1;
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const float n = __shfl_up_sync(0xffffffffu, v, off);
+                        if (lane >= off) v += n;
+                    }
+                    const float b1 = v, b0 = v - g1;
+                    rowE[2 * lane] = __expf(b0);
+                    rowE[2 * lane + 1] = __expf(b1);
+                    rowEi[2 * lane] = __expf(-b0);
+                    rowEi[2 * lane + 1] = __expf(-b1);
+                    const float G = __shfl_sync(0xffffffffu, b1, 31);
+                    if (lane == 0) {
+                        gam[0] = __expf(G);
+                        gaml[0] = G;
+                    }
+                }
+            }
+            named_bar_sync(BAR_COMP, NCOMP);
             float bx = 0.f, by = 0.f;
             if (GATE == 1) {
                 float Gx = 0.f, Gy = 0.f;
                 for (int r2 = 0; r2 < RG; ++r2) {
                     const float tx = tot[r2 * DK + d], ty = tot[r2 * DK + d + 1];
-                    if (r2 < rg) { bx += tx; by += ty; }
+                    if (r2 < rg) {
+                        bx += tx;
+                        by += ty;
+                    }
                     Gx += tx;
                     Gy += ty;
                 }
                 if (rg == 0) {
-                    gam[d] = __expf(Gx); gam[d + 1] = __expf(Gy);
-                    gaml[d] = Gx; gaml[d + 1] = Gy;
+                    gam[d] = __expf(Gx);
+                    gam[d + 1] = __expf(Gy);
+                    gaml[d] = Gx;
+                    gaml[d + 1] = Gy;
                 }
             }
             for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
@@ -251,8 +336,10 @@ __global__ void __launch_bounds__(NTHR, 1)
                     const float2 gv = *reinterpret_cast<const float2*>(sg + r * DK + d);
                     bx += gv.x;
                     by += gv.y;
-                    eqx = __expf(bx); eqy = __expf(by);
-                    ekx = __expf(-bx); eky = __expf(-by);
+                    eqx = __expf(bx);
+                    eqy = __expf(by);
+                    ekx = __expf(-bx);
+                    eky = __expf(-by);
                 } else if (GATE == 2) {
                     eqx = eqy = rowE[r];
                     ekx = eky = rowEi[r];
@@ -268,148 +355,123 @@ __global__ void __launch_bounds__(NTHR, 1)
                 const float2 kf = __bfloat1622float2(*pk);
                 *pk = __floats2bfloat162_rn(kf.x * iv * ekx, kf.y * iv * eky);
             }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-
-        // ------------------------------------------------ MMAs, group 1
-        if (tid == 0) {
-            const uint32_t qa = smem_u32(sq), ka = smem_u32(sk), va = smem_u32(sv);
-            if (MODE == 0) {
-                const uint32_t sa = smem_u32(sS);
-                const uint32_t idA = idesc_bf16(64, 64, 0, 0), idO = idesc_bf16(64, DVT, 0, 1);
-#pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk) {
-                    const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
-                    mma_bf16(tbase, sw128_desc(qa + koff, 16, 1024), sw128_desc(ka + koff, 16, 1024), idA, kk > 0);
-                }
-#pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk) {
-                    const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
-                    mma_bf16(tbase + (16u << 16), sw128_desc(qa + koff, 16, 1024),
-                             sw128_desc(sa + kk * 2048, DK * 128, 1024), idO, kk > 0);
-                }
-            }
-            const uint32_t idS = idesc_bf16(C::MS, DVT, 1, 1);
-#pragma unroll
-            for (int h = 0; h < C::NH; ++h)
-#pragma unroll
-                for (int ks = 0; ks < TR / 16; ++ks)
-                    mma_bf16(tbase + C::COL_S + h * DVT, sw128_desc(ka + h * 2 * BLK + ks * 2048, BLK, 1024),
-                             sw128_desc(va + ks * 2048, BLK, 1024), idS, ks > 0);
-            mma_commit(bar_mma1);
-        }
-        ++issued_mma1;
-        {
-            const bool ok1 = mbar_wait(bar_mma1, i & 1);
-            if (__syncthreads_or(!ok1)) { err = 1; break; }
-        }
-        tc_fence_after();
-
-        // ------------------------------------------------ P = mask(A) -> shared
-        if (MODE == 0) {
-            uint32_t r[32];
-            tmem_ld32(tbase + ((uint32_t)(32 * qd) << 16) + 32 * wg, r);
-            tmem_wait_ld();
-            if (lane < 16) {
-                const int t = 16 * qd + lane;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    float f[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int sidx = 32 * wg + 8 * u + j;
-                        f[j] = (sidx <= t) ? __uint_as_float(r[8 * u + j]) : 0.f;
-                    }
-                    store8_bf16(sP, sw128_off(t, 32 * wg + 8 * u, BLK), f);
-                }
-            }
             fence_proxy_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            tc_fence_after();
-            if (tid == 0) {
-                const uint32_t pa = smem_u32(sP), va = smem_u32(sv);
-                const uint32_t idO = idesc_bf16(64, DVT, 0, 1);
-#pragma unroll
-                for (int ks = 0; ks < TR / 16; ++ks)
-                    mma_bf16(tbase + (16u << 16), sw128_desc(pa + ks * 32, 16, 1024),
-                             sw128_desc(va + ks * 2048, BLK, 1024), idO, 1);
-                mma_commit(bar_mma2);
-            }
-            ++issued_mma2;
-        }
+            named_bar_sync(BAR_COMP, NCOMP);
+            if (ctid == 0) mbar_arrive(&bar_trans[s]);
+            return true;
+        };
 
-        // ------------------------------------------------ state update (overlaps P V)
-#pragma unroll
-        for (int h = 0; h < C::NH; ++h) {
-            const int d = (DK == 64 ? 16 * qd + (lane & 15) : 32 * qd + lane) + 128 * h;
-            const float eg = gam[GATE == 2 ? 0 : (GATE == 1 ? d : 0)];
-            const float gl = gaml[GATE == 2 ? 0 : (GATE == 1 ? d : 0)];
-            const float egv = GATE == 0 ? 1.f : eg;
-            if (GATE != 0) glog[h] += gl;
-#pragma unroll
-            for (int c = 0; c < C::HALF; c += 32) {
-                uint32_t r[32];
-                tmem_ld32(tbase + ((uint32_t)(32 * qd) << 16) + C::COL_S + h * DVT + wg * C::HALF + c, r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) Sreg[h][c + j] = egv * (Sreg[h][c + j] + __uint_as_float(r[j]));
+        bool alive = ntiles > 0 ? transform(0) : true;
+        for (int i = 0; alive && i < ntiles; ++i) {
+            const int b = i & 1;
+            const uint32_t tb = tbase + b * C::BUFCOLS;
+            if (C::NS == 2 && i + 1 < ntiles && !transform(i + 1)) break;
+            {
+                const bool ok = mbar_wait_abort(&bar_mma1[b], (i >> 1) & 1, abortp);
+                if (!named_bar_and(BAR_COMP, NCOMP, ok)) break;
             }
-            if (MODE == 0 && srow_ok) {
-#pragma unroll
-                for (int j = 0; j < C::HALF; j += 8)
-                    store8_bf16(sS, sw128_off(d, wg * C::HALF + j, DK * 128), &Sreg[h][j]);
-            }
-        }
-
-        // ------------------------------------------------ output
-        if (MODE == 0) {
-            const bool ok2 = mbar_wait(bar_mma2, i & 1);
-            if (__syncthreads_or(!ok2)) { err = 1; break; }
             tc_fence_after();
-            const int t = 16 * qd + (lane & 15);
-            const bool row_ok = (lane >= 16) && (t0 + t < P.L);
-            __nv_bfloat16* orow = A.o + (rowbase + t0 + t) * P.Dv + e0 + wg * C::HALF;
-#pragma unroll
-            for (int c = 0; c < C::HALF; c += 32) {
+            const int t0 = (tile0 + i) * TR;
+            // ---- P = causal mask of A -> shared (double-buffered)
+            if (MODE == 0) {
+                uint8_t* sP = sPb + b * (TR * TR * 2);
                 uint32_t r[32];
-                tmem_ld32(tbase + ((uint32_t)(32 * qd) << 16) + wg * C::HALF + c, r);
+                tmem_ld32(tb + ((uint32_t)(32 * qd) << 16) + 32 * wg, r);
                 tmem_wait_ld();
-                if (row_ok) {
+                if (lane < 16) {
+                    const int t = 16 * qd + lane;
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        uint32_t w[4];
+                        float f[8];
 #pragma unroll
-                        for (int p = 0; p < 4; ++p) {
-                            __nv_bfloat162 b2 = __floats2bfloat162_rn(P.scale * __uint_as_float(r[8 * u + 2 * p]),
-                                                                      P.scale * __uint_as_float(r[8 * u + 2 * p + 1]));
-                            w[p] = *reinterpret_cast<uint32_t*>(&b2);
+                        for (int j = 0; j < 8; ++j) {
+                            const int sidx = 32 * wg + 8 * u + j;
+                            f[j] = (sidx <= t) ? __uint_as_float(r[8 * u + j]) : 0.f;
                         }
-                        *reinterpret_cast<uint4*>(orow + c + 8 * u) = make_uint4(w[0], w[1], w[2], w[3]);
+                        store8_bf16(sP, sw128_off(t, 32 * wg + 8 * u, BLK), f);
+                    }
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(BAR_COMP, NCOMP);
+                if (ctid == 0) mbar_arrive(&bar_pready[b]);
+            }
+            // ---- state: S = e^Gamma (S + dS'); bf16 copy for the next tile's inter product
+            {
+                const float* gam = gamb + b * DK;
+                const float* gaml = gamlb + b * DK;
+#pragma unroll
+                for (int h = 0; h < C::NH; ++h) {
+                    const int d = (DK == 64 ? 16 * qd + (lane & 15) : 32 * qd + lane) + 128 * h;
+                    const int gi = GATE == 1 ? d : 0;
+                    const float egv = GATE == 0 ? 1.f : gam[gi];
+                    if (GATE != 0) glog[h] += gaml[gi];
+#pragma unroll
+                    for (int c = 0; c < C::HALF; c += 32) {
+                        uint32_t r[32];
+                        tmem_ld32(tb + ((uint32_t)(32 * qd) << 16) + C::COL_S + h * DVT + wg * C::HALF + c, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) Sreg[h][c + j] = egv * (Sreg[h][c + j] + __uint_as_float(r[j]));
+                    }
+                    if (MODE == 0 && srow_ok) {
+#pragma unroll
+                        for (int j = 0; j < C::HALF; j += 8)
+                            store8_bf16(sS, sw128_off(d, wg * C::HALF + j, DK * 128), &Sreg[h][j]);
+                    }
+                }
+                if (MODE == 0) {
+                    fence_proxy_async_smem();
+                    named_bar_sync(BAR_COMP, NCOMP);
+                    if (ctid == 0) mbar_arrive(bar_sready);
+                }
+            }
+            // ---- output tile
+            if (MODE == 0) {
+                const bool ok = mbar_wait_abort(&bar_mma2[b], (i >> 1) & 1, abortp);
+                if (!named_bar_and(BAR_COMP, NCOMP, ok)) break;
+                tc_fence_after();
+                const int t = 16 * qd + (lane & 15);
+                const bool row_ok = (lane >= 16) && (t0 + t < P.L);
+                __nv_bfloat16* orow = A.o + (rowbase + t0 + t) * P.Dv + e0 + wg * C::HALF;
+#pragma unroll
+                for (int c = 0; c < C::HALF; c += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tb + ((uint32_t)(32 * qd) << 16) + wg * C::HALF + c, r);
+                    tmem_wait_ld();
+                    if (row_ok) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int p2 = 0; p2 < 4; ++p2) {
+                                __nv_bfloat162 b2 =
+                                    __floats2bfloat162_rn(P.scale * __uint_as_float(r[8 * u + 2 * p2]),
+                                                          P.scale * __uint_as_float(r[8 * u + 2 * p2 + 1]));
+                                w[p2] = *reinterpret_cast<uint32_t*>(&b2);
+                            }
+                            *reinterpret_cast<uint4*>(orow + c + 8 * u) = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
                     }
                 }
             }
+            tc_fence_before();
+            named_bar_sync(BAR_COMP, NCOMP);
+            if (ctid == 0) mbar_arrive(&bar_tfree[b]);
+            if (C::NS == 1 && i + 1 < ntiles && !transform(i + 1)) break;
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (tid == 0 && i + C::NS < ntiles) issue_loads(i + C::NS, s);
     }
 
-    if (err) {
+    __syncthreads();
+    if (*abortp) {
         if (tid == 0) {
             atomicExch(A.status, kDevStatusTimeout);
-            // let every issued copy and product land before the shared memory and TMEM go away
-            for (int i = consumed; i < ntiles && i < consumed + C::NS; ++i)
-                mbar_wait(&bar_full[i % C::NS], (i / C::NS) & 1, 1u << 20);
-            if (issued_mma1) mbar_wait(bar_mma1, (issued_mma1 - 1) & 1, 1u << 20);
-            if (issued_mma2) mbar_wait(bar_mma2, (issued_mma2 - 1) & 1, 1u << 20);
+            // let every issued copy and product land before shared memory and TMEM go away
+            for (int j = *n_consumed; j < *n_issued; ++j)
+                mbar_wait(&bar_full[j % C::NS], (j / C::NS) & 1, 1u << 20);
+            if (*n_mma1) mbar_wait(&bar_mma1[(*n_mma1 - 1) & 1], ((*n_mma1 - 1) >> 1) & 1, 1u << 20);
+            if (*n_mma2) mbar_wait(&bar_mma2[(*n_mma2 - 1) & 1], ((*n_mma2 - 1) >> 1) & 1, 1u << 20);
         }
-    } else if (srow_ok) {
+    } else if (tid < NCOMP && srow_ok) {
         // final state of the segment
 #pragma unroll
         for (int h = 0; h < C::NH; ++h) {
@@ -505,7 +567,7 @@ static cudaError_t launch_one(const CUtensorMap& mq, const CUtensorMap& mk, cons
         attr = true;
     }
     dim3 grid(P.B * P.H, P.Dv / DVT, nseg);
-    GLA_LAUNCH(MODE == 0 ? "tc_fwd" : "tc_fwd_state", st, kern<<<grid, NTHR, C::SMEM, st>>>(mq, mk, mv, mg, a, P));
+    GLA_LAUNCH(MODE == 0 ? "tc_fwd" : "tc_fwd_state", st, kern<<<grid, NTHR_WS, C::SMEM, st>>>(mq, mk, mv, mg, a, P));
     return cudaGetLastError();
 }
 

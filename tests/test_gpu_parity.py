@@ -62,7 +62,7 @@ def flat_heads(t, heads):
     if t is None:
         return None
     B, H = t.shape[0], t.shape[1]
-    return t.reshape((B * H,) + tuple(t.shape[2:]))[heads].unsqueeze(0)
+    return t.reshape((B * H,) + tuple(t.shape[2:]))[heads][None]
 
 
 def check_fwd(x, w, plan="auto", chunk=None, heads=None):
