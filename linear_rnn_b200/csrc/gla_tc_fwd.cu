@@ -57,10 +57,10 @@ struct Cfg {
     static constexpr uint32_t BUF_USED = COL_S + NH * DVT;
     static constexpr uint32_t BUFCOLS = BUF_USED <= 32 ? 32 : BUF_USED <= 64 ? 64 : BUF_USED <= 128 ? 128 : 256;
     static constexpr uint32_t NCOL = 2 * BUFCOLS;            // two accumulator buffers
-    static constexpr int HALF = DVT / 2;                     // state columns per warpgroup
+    static constexpr int HALF = DVT / 4;                     // state columns per compute warpgroup
     static_assert(STAGE % 1024 == 0, "stage alignment");
     static_assert(SMEM <= 227 * 1024, "shared memory");
-    static_assert(HALF % 32 == 0, "column chunks");
+    static_assert(HALF % 16 == 0, "column chunks");
     static_assert(BUF_USED <= 256 && NCOL <= 512, "tensor memory");
 };
 
@@ -88,11 +88,14 @@ __device__ __forceinline__ void store8_bf16(uint8_t* base, uint32_t off, const f
     *reinterpret_cast<uint4*>(base + off) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// Thread roles: warps 0-7 (two warpgroups) transform tiles and run the epilogues; warp 8
-// issues the tcgen05 MMAs; warp 9 issues the TMA loads. They hand tiles to each other
+// Thread roles: warps 0-15 (four warpgroups) transform tiles and run the epilogues; warp 16
+// issues the tcgen05 MMAs; warp 17 issues the TMA loads. They hand tiles to each other
 // through mbarriers, so the transform of tile i+1 runs while the tensor core works on
 // tile i, and the epilogues of tile i overlap the MMAs of tile i+1 (two TMEM buffers).
-constexpr int NCOMP = 256;
+// Each compute warpgroup owns a quarter of the state columns; warp w reads TMEM lane
+// quadrant w % 4.
+constexpr int NCOMP = 512;
+constexpr int NCWG = NCOMP / 128;
 constexpr int NTHR_WS = NCOMP + 64;
 constexpr int BAR_COMP = 1;   // named barrier of the 256 compute threads
 
@@ -131,7 +134,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
 
     const int bh = blockIdx.x, vt = blockIdx.y, z = blockIdx.z;
     const int e0 = vt * DVT;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = (warp >> 2) & 1, qd = warp & 3;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = (warp >> 2) & 3, qd = warp & 3;
     const int ntiles_all = cdiv(P.L, TR);
     const int tile0 = z * A.tiles_per_seg;
     const int ntiles = min(ntiles_all, tile0 + A.tiles_per_seg) - tile0;
@@ -176,7 +179,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
 
-    if (warp == 9) {
+    if (warp == NCOMP / 32 + 1) {
         // ================================================================ TMA producer
         if (lane == 0) {
             if (MODE == 0) tma_prefetch_desc(&tq);
@@ -200,7 +203,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 *n_issued = j + 1;
             }
         }
-    } else if (warp == 8) {
+    } else if (warp == NCOMP / 32) {
         // ================================================================ MMA issuer
         if (lane == 0) {
             for (int i = 0; i < ntiles; ++i) {
@@ -259,7 +262,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
         }
     } else {
         // ================================================================ compute warpgroups
-        const int ctid = tid;  // 0..255
+        const int ctid = tid;  // 0..NCOMP-1
         // Transform tile j in place: q~ = q e^b, k~ = i k e^-b; e^Gamma into buffer j&1.
         auto transform = [&](int j) -> bool {
             const int s = j % C::NS, b = j & 1;
@@ -365,7 +368,6 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
         for (int i = 0; alive && i < ntiles; ++i) {
             const int b = i & 1;
             const uint32_t tb = tbase + b * C::BUFCOLS;
-            if (C::NS == 2 && i + 1 < ntiles && !transform(i + 1)) break;
             {
                 const bool ok = mbar_wait_abort(&bar_mma1[b], (i >> 1) & 1, abortp);
                 if (!named_bar_and(BAR_COMP, NCOMP, ok)) break;
@@ -375,20 +377,20 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
             // ---- P = causal mask of A -> shared (double-buffered)
             if (MODE == 0) {
                 uint8_t* sP = sPb + b * (TR * TR * 2);
-                uint32_t r[32];
-                tmem_ld32(tb + ((uint32_t)(32 * qd) << 16) + 32 * wg, r);
+                uint32_t r[16];
+                tmem_ld16(tb + ((uint32_t)(32 * qd) << 16) + 16 * wg, r);
                 tmem_wait_ld();
                 if (lane < 16) {
                     const int t = 16 * qd + lane;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < 2; ++u) {
                         float f[8];
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
-                            const int sidx = 32 * wg + 8 * u + j;
+                            const int sidx = 16 * wg + 8 * u + j;
                             f[j] = (sidx <= t) ? __uint_as_float(r[8 * u + j]) : 0.f;
                         }
-                        store8_bf16(sP, sw128_off(t, 32 * wg + 8 * u, BLK), f);
+                        store8_bf16(sP, sw128_off(t, 16 * wg + 8 * u, BLK), f);
                     }
                 }
                 fence_proxy_async_smem();
@@ -406,12 +408,12 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     const float egv = GATE == 0 ? 1.f : gam[gi];
                     if (GATE != 0) glog[h] += gaml[gi];
 #pragma unroll
-                    for (int c = 0; c < C::HALF; c += 32) {
-                        uint32_t r[32];
-                        tmem_ld32(tb + ((uint32_t)(32 * qd) << 16) + C::COL_S + h * DVT + wg * C::HALF + c, r);
+                    for (int c = 0; c < C::HALF; c += 16) {
+                        uint32_t r[16];
+                        tmem_ld16(tb + ((uint32_t)(32 * qd) << 16) + C::COL_S + h * DVT + wg * C::HALF + c, r);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) Sreg[h][c + j] = egv * (Sreg[h][c + j] + __uint_as_float(r[j]));
+                        for (int j = 0; j < 16; ++j) Sreg[h][c + j] = egv * (Sreg[h][c + j] + __uint_as_float(r[j]));
                     }
                     if (MODE == 0 && srow_ok) {
 #pragma unroll
@@ -425,6 +427,8 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     if (ctid == 0) mbar_arrive(bar_sready);
                 }
             }
+            // ---- next tile's transform overlaps this tile's P V product
+            if (C::NS == 2 && i + 1 < ntiles && !transform(i + 1)) break;
             // ---- output tile
             if (MODE == 0) {
                 const bool ok = mbar_wait_abort(&bar_mma2[b], (i >> 1) & 1, abortp);
@@ -434,13 +438,13 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 const bool row_ok = (lane >= 16) && (t0 + t < P.L);
                 __nv_bfloat16* orow = A.o + (rowbase + t0 + t) * P.Dv + e0 + wg * C::HALF;
 #pragma unroll
-                for (int c = 0; c < C::HALF; c += 32) {
-                    uint32_t r[32];
-                    tmem_ld32(tb + ((uint32_t)(32 * qd) << 16) + wg * C::HALF + c, r);
+                for (int c = 0; c < C::HALF; c += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tb + ((uint32_t)(32 * qd) << 16) + wg * C::HALF + c, r);
                     tmem_wait_ld();
                     if (row_ok) {
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
+                        for (int u = 0; u < 2; ++u) {
                             uint32_t w[4];
 #pragma unroll
                             for (int p2 = 0; p2 < 4; ++p2) {
