@@ -75,14 +75,17 @@ gla_status check_problem(const gla_problem* p, Dims* P, int* plan) {
     return GLA_OK;
 }
 
-// The tensor-core plan runs bf16 I/O with chunks that are whole 64-token tiles.
-bool tc_ok(const gla_problem* p, const Dims& P) { return p->io == GLA_BF16 && tc::supports(P); }
+// The tensor-core plan runs bf16 I/O with chunks that are whole 64-token tiles; its
+// backward holds the Dk x Dv state gradient in tensor memory (Dk <= 128).
+bool tc_ok(const gla_problem* p, const Dims& P, bool bwd) {
+    return p->io == GLA_BF16 && (bwd ? tc::bwd_supports(P) : tc::supports(P));
+}
 
 // Plan of the forward / backward: AUTO prefers the tensor-core plan where it applies.
 gla_status resolve(const gla_problem* p, const Dims& P, bool bwd, int* plan) {
     int pl = p->plan;
-    if (pl == GLA_PLAN_AUTO) pl = (!bwd && tc_ok(p, P)) ? GLA_PLAN_TC : GLA_PLAN_SIMT;
-    if (pl == GLA_PLAN_TC && (bwd || !tc_ok(p, P))) return GLA_ERR_UNSUPPORTED;
+    if (pl == GLA_PLAN_AUTO) pl = tc_ok(p, P, bwd) ? GLA_PLAN_TC : GLA_PLAN_SIMT;
+    if (pl == GLA_PLAN_TC && !tc_ok(p, P, bwd)) return GLA_ERR_UNSUPPORTED;
     *plan = pl;
     return GLA_OK;
 }
@@ -90,7 +93,7 @@ gla_status resolve(const gla_problem* p, const Dims& P, bool bwd, int* plan) {
 gla_status map_cuda(cudaError_t e) { return e == cudaSuccess ? GLA_OK : GLA_ERR_CUDA; }
 
 size_t ws_bytes(const Dims& P, int plan, bool bwd) {
-    if (plan == GLA_PLAN_TC && !bwd) return tc::fwd_workspace_bytes(P);
+    if (plan == GLA_PLAN_TC) return bwd ? tc::bwd_workspace_bytes(P) : tc::fwd_workspace_bytes(P);
     return simt::workspace_bytes(P, bwd);
 }
 
@@ -157,7 +160,10 @@ gla_status gla_bwd(const gla_problem* p, const void* q, const void* k, const voi
     cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, st);
     if (e != cudaSuccess) return GLA_ERR_CUDA;
     if ((size_t)P.B * P.H == 0) return GLA_OK;
-    e = simt::bwd(P, p->io, q, k, v, g, igate, h0, dO, dhT, dq, dk, dv, dg, di, dh0, ws, st);
+    if (plan == GLA_PLAN_TC && P.L > 0)
+        e = tc::bwd(P, q, k, v, g, igate, h0, dO, dhT, dq, dk, dv, dg, di, dh0, ws, st);
+    else
+        e = simt::bwd(P, p->io, q, k, v, g, igate, h0, dO, dhT, dq, dk, dv, dg, di, dh0, ws, st);
     return map_cuda(e);
 }
 

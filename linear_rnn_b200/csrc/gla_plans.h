@@ -25,5 +25,22 @@ bool supports(const Dims& P);
 size_t fwd_workspace_bytes(const Dims& P);
 cudaError_t fwd(const Dims& P, const void* q, const void* k, const void* v, const float* g, const float* ig,
                 const float* h0, void* o, float* hT, void* ws, cudaStream_t st);
+// Segment state passes and scans shared by the forward and the backward.
+//   mode 1: forward local end states of segments 0..nseg-2 (a = k, b = v)
+//   mode 2: reverse local state gradients of segments 1..nseg-1 (a = q, b = dO)
+cudaError_t state_pass(const Dims& P, int mode, const void* a_src, const void* b_src, const float* g,
+                       const float* ig, int nseg, int tiles_per_seg, float* seg_state, float* seg_gamma, int* status,
+                       cudaStream_t st);
+cudaError_t seg_scan(const Dims& P, int nseg, const float* seg_state, const float* seg_gamma, const float* h0,
+                     float* sinit, cudaStream_t st);
+cudaError_t seg_rscan(const Dims& P, int nseg, const float* seg_state, const float* seg_gamma, const float* dhT,
+                      float* gend, cudaStream_t st);
+int num_sms();
+// Backward (gla_tc_bwd.cu)
+bool bwd_supports(const Dims& P);
+size_t bwd_workspace_bytes(const Dims& P);
+cudaError_t bwd(const Dims& P, const void* q, const void* k, const void* v, const float* g, const float* ig,
+                const float* h0, const void* dO, const float* dhT, void* dq, void* dk, void* dv, float* dg, float* di,
+                float* dh0, void* ws, cudaStream_t st);
 }  // namespace tc
 }  // namespace gla

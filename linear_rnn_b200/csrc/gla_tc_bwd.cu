@@ -1,0 +1,1064 @@
+// Tensor-core (tcgen05 / TMEM / TMA) backward of chunkwise gated linear attention, bf16 I/O.
+//
+// Per 64-token tile, with b the in-tile cumulative log-gate, Gamma its total, k' = i k,
+// q~ = q e^b, k~ = k' e^-b, S the state before the tile and G = dL/dS after it (the
+// chunkwise backward restated from the forward of the talk summary "Hardware-Efficient
+// Training of Linear Attention Models", section 11:58, with the GLA abstract's gates):
+//   dq   = scale e^b * ( dO S^T + mask(dO V^T) k~ )
+//   G~   = diag(e^Gamma) G
+//   dk'  = e^-b * ( mask(dO V^T)^T (scale q~) + V G~^T ),   dk = i dk'
+//   dv   = mask(scale q~ k~^T)^T dO + k~ G~
+//   G_prev = G~ + (scale q~)^T dO
+//   dg   = reverse cumulative sum over the whole sequence of q*dq - k*dk (+ sum_e dhT*hT),
+//          (k*dk = k'*dk' because dk = i dk')
+// Kernels:
+//   tc_bwd_dq    forward tile walk per (b*h, key-dim block, segment); S in TMEM (fp32, the
+//                state MMA accumulates onto it, a TMEM pass applies e^Gamma) and bf16 in
+//                shared memory as the B operand of dO S^T.
+//   tc_bwd_dkdv  reverse tile walk per (b*h, segment); G in TMEM, bf16 G~ in shared memory.
+//   tc_bwd_dg    reverse cumulative sum of q*dq - k*dk, fp32.
+// Segment boundary states come from the forward state pass + scan; segment boundary
+// state gradients from the reverse state pass (gla_tc_fwd.cu, mode 2) + reverse scan.
+#include "gla_plans.h"
+#include "gla_tc_common.cuh"
+
+namespace gla {
+namespace tc {
+
+using namespace sm100;
+
+constexpr int NT_B = 256;  // 8 warps: two warpgroups; thread 0 also issues TMA and MMA
+
+struct BwdArgs {
+    const float* gh;      // per-head log-gate [BH*L]
+    const float* ig;      // input gate [BH*L] or null
+    const float* sinit;   // initial state per (bh, segment) [BH, nseg, Dk, Dv] or null (then h0 / 0)
+    const float* h0;
+    const float* gend;    // state gradient at the end of each segment [BH, nseg, Dk, Dv] or null (then dhT / 0)
+    const float* dhT;
+    __nv_bfloat16* dq;
+    __nv_bfloat16* dk;
+    __nv_bfloat16* dv;
+    float* di;            // [BH*L] or null
+    float* dh0;           // [BH, Dk, Dv] or null
+    float* hT_ws;         // final state (for the dg term) or null
+    int* status;
+    int tiles_per_seg;
+    int nseg;
+};
+
+__device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity) {
+    const bool ok = mbar_wait(bar, parity);
+    return __syncthreads_and(ok) != 0;
+}
+
+__device__ __forceinline__ void store16_bf16_global(__nv_bfloat16* dst, const float* v) {
+    uint32_t w[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        __nv_bfloat162 p = __floats2bfloat162_rn(v[2 * u], v[2 * u + 1]);
+        w[u] = *reinterpret_cast<uint32_t*>(&p);
+    }
+    reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+constexpr uint32_t pow2cols(uint32_t n) { return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512; }
+
+// ============================================================================ dq
+template <int DKB, int DV, int GATE>
+struct QCfg {
+    static constexpr uint32_t KB = TR * DKB * 2;
+    static constexpr uint32_t GB = GATE == 1 ? TR * DKB * 4 : 0;
+    static constexpr uint32_t VB = TR * DV * 2;
+    static constexpr uint32_t OB = TR * DV * 2;
+    static constexpr uint32_t STAGE = KB + GB + VB + OB;
+    static constexpr uint32_t SB = DKB * DV * 2;
+    static constexpr uint32_t AB = TR * TR * 2;
+    static constexpr uint32_t SMALL = 256 + 4096 + 8 * DKB + 1024;
+    static constexpr int NS = (2 * STAGE + SB + AB + SMALL + 1024 <= 227 * 1024) ? 2 : 1;
+    static constexpr uint32_t SMEM = NS * STAGE + SB + AB + SMALL + 1024;
+    static constexpr uint32_t COL_R = DV;
+    static constexpr uint32_t NCOL = pow2cols(DV + (DKB > 64 ? DKB : 64));
+    static constexpr int HC = DV / 2;    // state columns per warpgroup
+    static constexpr int QC = DKB / 2;   // dq columns per warpgroup
+    static_assert(SMEM <= 227 * 1024, "shared memory");
+    static_assert(STAGE % 1024 == 0, "stage alignment");
+};
+
+template <int DKB, int DV, int GATE>
+__global__ void __launch_bounds__(NT_B, 1)
+    k_tc_bwd_dq(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tg,
+                const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo, BwdArgs A, Dims P) {
+    using C = QCfg<DKB, DV, GATE>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sS = sm + C::NS * C::STAGE;
+    uint8_t* sA = sS + C::SB;
+    uint8_t* small = sA + C::AB;
+    uint64_t* bar_full = reinterpret_cast<uint64_t*>(small);  // [2]
+    uint64_t* bar_mma1 = bar_full + 2;
+    uint64_t* bar_mma2 = bar_full + 3;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 64);
+    float* tot = reinterpret_cast<float*>(small + 256);
+    float* gam = tot + 1024;            // [DKB]
+    float* rowE = gam + DKB;            // [64]
+    float* rowEi = rowE + TR;
+    float* igs = rowEi + TR;
+    float* ghs = igs + TR;
+
+    const int bh = blockIdx.x, kb = blockIdx.y, z = blockIdx.z;
+    const int d0 = kb * DKB;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2, qd = warp & 3;
+    const int ntiles_all = cdiv(P.L, TR);
+    const int tile0 = z * A.tiles_per_seg;
+    const int ntiles = min(ntiles_all, tile0 + A.tiles_per_seg) - tile0;
+    const long rowbase = (long)bh * P.L;
+    const bool srow_ok = (DKB != 64) || (lane < 16);
+    const int srow = DKB == 64 ? 16 * qd + (lane & 15) : 32 * qd + lane;
+
+    if (tid == 0) {
+        mbar_init(&bar_full[0], 1);
+        mbar_init(&bar_full[1], 1);
+        mbar_init(bar_mma1, 1);
+        mbar_init(bar_mma2, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, C::NCOL);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tlane = tbase + ((uint32_t)(32 * qd) << 16);
+
+    // ---- initial state into TMEM (fp32) and shared memory (bf16)
+    {
+        const float* src = nullptr;
+        if (z == 0) src = A.h0 ? A.h0 + ((long)bh * P.Dk + d0 + srow) * P.Dv : nullptr;
+        else src = A.sinit + (((long)bh * A.nseg + z) * P.Dk + d0 + srow) * P.Dv;
+        for (int c = wg * C::HC; c < (wg + 1) * C::HC; c += 16) {
+            float f[16];
+            uint32_t r[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                f[j] = (src && srow_ok) ? src[c + j] : 0.f;
+                r[j] = __float_as_uint(f[j]);
+            }
+            tmem_st16(tlane + c, r);
+            if (srow_ok) {
+                store8_bf16(sS, sw128_off(srow, c, DKB * 128), f);
+                store8_bf16(sS, sw128_off(srow, c + 8, DKB * 128), f + 8);
+            }
+        }
+        tmem_wait_st();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    auto issue_loads = [&](int i, int s) {
+        uint8_t* st = sm + s * C::STAGE;
+        const int t0 = (tile0 + i) * TR;
+        mbar_arrive_expect_tx(&bar_full[s], C::STAGE);
+        for (int cb = 0; cb < DKB / 64; ++cb) tma_load_3d(st + cb * BLK, &tk, d0 + cb * 64, t0, bh, &bar_full[s]);
+        if (GATE == 1) tma_load_3d(st + C::KB, &tg, d0, t0, bh, &bar_full[s]);
+        for (int vb = 0; vb < DV / 64; ++vb) {
+            tma_load_3d(st + C::KB + C::GB + vb * BLK, &tv, vb * 64, t0, bh, &bar_full[s]);
+            tma_load_3d(st + C::KB + C::GB + C::VB + vb * BLK, &tdo, vb * 64, t0, bh, &bar_full[s]);
+        }
+    };
+    if (tid == 0)
+        for (int i = 0; i < C::NS && i < ntiles; ++i) issue_loads(i, i);
+
+    int err = 0, n_mma = 0;
+    for (int i = 0; i < ntiles; ++i) {
+        const int s = i % C::NS;
+        uint8_t* st = sm + s * C::STAGE;
+        uint8_t* sk = st;
+        float* sg = reinterpret_cast<float*>(st + C::KB);
+        uint8_t* sv = st + C::KB + C::GB;
+        uint8_t* so = sv + C::VB;
+        const int t0 = (tile0 + i) * TR;
+        if (tid < TR) {
+            const int t = t0 + tid;
+            igs[tid] = (A.ig && t < P.L) ? A.ig[rowbase + t] : 1.f;
+            if (GATE == 2) ghs[tid] = (t < P.L) ? A.gh[rowbase + t] : 0.f;
+        }
+        if (!block_wait(&bar_full[s], (i / C::NS) & 1)) { err = 1; break; }
+
+        // ---- transform: k~ = i k e^-b in place; e^b kept (in place of g) for the dq epilogue
+        constexpr int NP = DKB / 2, RG = NT_B / NP, RPG = TR / RG;
+        const int cp = tid % NP, rg = tid / NP, d = 2 * cp;
+        if (GATE == 1) {
+            float ax = 0.f, ay = 0.f;
+            for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
+                const float2 gv = *reinterpret_cast<const float2*>(sg + r * DKB + d);
+                ax += gv.x;
+                ay += gv.y;
+            }
+            tot[rg * DKB + d] = ax;
+            tot[rg * DKB + d + 1] = ay;
+        } else if (GATE == 2 && warp == 0) {
+            const float g0 = ghs[2 * lane], g1 = ghs[2 * lane + 1];
+            float v = g0 + g1;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float n = __shfl_up_sync(0xffffffffu, v, off);
+                if (lane >= off) v += n;
+            }
+            const float b1 = v, b0 = v - g1;
+            rowE[2 * lane] = __expf(b0);
+            rowE[2 * lane + 1] = __expf(b1);
+            rowEi[2 * lane] = __expf(-b0);
+            rowEi[2 * lane + 1] = __expf(-b1);
+            const float G = __shfl_sync(0xffffffffu, b1, 31);
+            if (lane == 0) gam[0] = __expf(G);
+        }
+        __syncthreads();
+        {
+            float bx = 0.f, by = 0.f;
+            if (GATE == 1) {
+                float Gx = 0.f, Gy = 0.f;
+                for (int r2 = 0; r2 < RG; ++r2) {
+                    const float tx = tot[r2 * DKB + d], ty = tot[r2 * DKB + d + 1];
+                    if (r2 < rg) { bx += tx; by += ty; }
+                    Gx += tx;
+                    Gy += ty;
+                }
+                if (rg == 0) { gam[d] = __expf(Gx); gam[d + 1] = __expf(Gy); }
+            }
+            for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
+                float ekx = 1.f, eky = 1.f;
+                if (GATE == 1) {
+                    float2* gp = reinterpret_cast<float2*>(sg + r * DKB + d);
+                    const float2 gv = *gp;
+                    bx += gv.x;
+                    by += gv.y;
+                    ekx = __expf(-bx);
+                    eky = __expf(-by);
+                    *gp = make_float2(__expf(bx), __expf(by));
+                } else if (GATE == 2) {
+                    ekx = eky = rowEi[r];
+                }
+                const float iv = igs[r];
+                __nv_bfloat162* pk = reinterpret_cast<__nv_bfloat162*>(sk + sw128_off(r, d, BLK));
+                const float2 kf = __bfloat1622float2(*pk);
+                *pk = __floats2bfloat162_rn(kf.x * iv * ekx, kf.y * iv * eky);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ---- MMA group 1: dA = dO V^T, D = dO S^T, S += k~^T V
+        if (tid == 0) {
+            const uint32_t ka = smem_u32(sk), va = smem_u32(sv), oa = smem_u32(so), sa = smem_u32(sS);
+            const uint32_t idA = idesc_bf16(64, 64, 0, 0), idQ = idesc_bf16(64, DKB, 0, 0);
+            const uint32_t idS = idesc_bf16(DKB, DV, 1, 1);
+#pragma unroll
+            for (int kk = 0; kk < DV / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+                mma_bf16(tbase + C::COL_R, sw128_desc(oa + koff, 16, 1024), sw128_desc(va + koff, 16, 1024), idA,
+                         kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < DV / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+                const uint32_t soff = (kk >> 2) * (DKB * 128) + (kk & 3) * 32;
+                mma_bf16(tbase + (16u << 16) + C::COL_R, sw128_desc(oa + koff, 16, 1024),
+                         sw128_desc(sa + soff, 16, 1024), idQ, kk > 0);
+            }
+#pragma unroll
+            for (int ks = 0; ks < TR / 16; ++ks)
+                mma_bf16(tbase, sw128_desc(ka + ks * 2048, BLK, 1024), sw128_desc(va + ks * 2048, BLK, 1024), idS, 1);
+            mma_commit(bar_mma1);
+        }
+        ++n_mma;
+        if (!block_wait(bar_mma1, i & 1)) { err = 1; break; }
+        tc_fence_after();
+
+        // ---- masked dA -> shared; state pass S = e^Gamma (S + dS') in TMEM, bf16 copy
+        {
+            uint32_t r[32];
+            tmem_ld32(tlane + C::COL_R + 32 * wg, r);
+            tmem_wait_ld();
+            if (lane < 16) {
+                const int t = 16 * qd + lane;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    float f[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int sidx = 32 * wg + 8 * u + j;
+                        f[j] = (sidx <= t) ? __uint_as_float(r[8 * u + j]) : 0.f;
+                    }
+                    store8_bf16(sA, sw128_off(t, 32 * wg + 8 * u, BLK), f);
+                }
+            }
+        }
+        {
+            const float eg = GATE == 0 ? 1.f : gam[GATE == 1 ? srow : 0];
+            for (int c = wg * C::HC; c < (wg + 1) * C::HC; c += 16) {
+                uint32_t r[16];
+                float f[16];
+                tmem_ld16(tlane + c, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    f[j] = eg * __uint_as_float(r[j]);
+                    r[j] = __float_as_uint(f[j]);
+                }
+                tmem_st16(tlane + c, r);
+                if (srow_ok) {
+                    store8_bf16(sS, sw128_off(srow, c, DKB * 128), f);
+                    store8_bf16(sS, sw128_off(srow, c + 8, DKB * 128), f + 8);
+                }
+            }
+            tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ---- MMA group 2: D += mask(dA) k~
+        if (tid == 0) {
+            const uint32_t aa = smem_u32(sA), ka = smem_u32(sk);
+            const uint32_t idQ = idesc_bf16(64, DKB, 0, 1);
+#pragma unroll
+            for (int ks = 0; ks < TR / 16; ++ks)
+                mma_bf16(tbase + (16u << 16) + C::COL_R, sw128_desc(aa + ks * 32, 16, 1024),
+                         sw128_desc(ka + ks * 2048, BLK, 1024), idQ, 1);
+            mma_commit(bar_mma2);
+        }
+        if (!block_wait(bar_mma2, i & 1)) { err = 1; break; }
+        tc_fence_after();
+
+        // ---- dq = scale e^b D
+        {
+            const int t = 16 * qd + (lane & 15);
+            const bool row_ok = lane >= 16 && t0 + t < P.L;
+            for (int c = wg * C::QC; c < (wg + 1) * C::QC; c += 16) {
+                uint32_t r[16];
+                tmem_ld16(tlane + C::COL_R + c, r);
+                tmem_wait_ld();
+                if (row_ok) {
+                    float f[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float eb = GATE == 1 ? sg[t * DKB + c + j] : (GATE == 2 ? rowE[t] : 1.f);
+                        f[j] = P.scale * eb * __uint_as_float(r[j]);
+                    }
+                    store16_bf16_global(A.dq + (rowbase + t0 + t) * P.Dk + d0 + c, f);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0 && i + C::NS < ntiles) issue_loads(i + C::NS, s);
+    }
+
+    if (err) {
+        if (tid == 0) {
+            atomicExch(A.status, kDevStatusTimeout);
+            if (n_mma) {
+                mbar_wait(bar_mma1, (n_mma - 1) & 1, 1u << 20);
+                mbar_wait(bar_mma2, (n_mma - 1) & 1, 1u << 20);
+            }
+        }
+    } else if (A.hT_ws && z == A.nseg - 1) {
+        // final state (for the dg term of an upstream final-state gradient)
+        for (int c = wg * C::HC; c < (wg + 1) * C::HC; c += 16) {
+            uint32_t r[16];
+            tmem_ld16(tlane + c, r);
+            tmem_wait_ld();
+            if (srow_ok) {
+                float* dst = A.hT_ws + ((long)bh * P.Dk + d0 + srow) * P.Dv + c;
+#pragma unroll
+                for (int j = 0; j < 16; j += 4)
+                    *reinterpret_cast<float4*>(dst + j) = make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                                                      __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, C::NCOL);
+}
+
+// ============================================================================ dk, dv
+template <int DK, int DV, int GATE>
+struct KVCfg {
+    static constexpr uint32_t QB = TR * DK * 2;
+    static constexpr uint32_t KB = TR * DK * 2;
+    static constexpr uint32_t GB = GATE == 1 ? TR * DK * 4 : 0;
+    static constexpr uint32_t VB = TR * DV * 2;
+    static constexpr uint32_t OB = TR * DV * 2;
+    static constexpr uint32_t STAGE = QB + KB + GB + VB + OB;
+    static constexpr uint32_t GTB = DK * DV * 2;
+    static constexpr uint32_t AB = TR * TR * 2;
+    static constexpr uint32_t SMALL = 256 + 4096 + 8 * DK + 1024 + 512;
+    static constexpr int NS = (2 * STAGE + GTB + 2 * AB + SMALL + 1024 <= 227 * 1024) ? 2 : 1;
+    static constexpr uint32_t SMEM = NS * STAGE + GTB + 2 * AB + SMALL + 1024;
+    static constexpr uint32_t COL_R = DV;
+    static constexpr uint32_t WR = DK > DV ? (DK > 64 ? DK : 64) : (DV > 64 ? DV : 64);
+    static constexpr uint32_t NCOL = pow2cols(DV + WR);
+    static constexpr int HC = DV / 2;
+    static constexpr int KC = DK / 2;
+    static_assert(SMEM <= 227 * 1024, "shared memory");
+    static_assert(DV + WR <= 512, "tensor memory");
+    static_assert(STAGE % 1024 == 0, "stage alignment");
+};
+
+template <int DK, int DV, int GATE>
+__global__ void __launch_bounds__(NT_B, 1)
+    k_tc_bwd_dkdv(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                  const __grid_constant__ CUtensorMap tg, const __grid_constant__ CUtensorMap tv,
+                  const __grid_constant__ CUtensorMap tdo, BwdArgs A, Dims P) {
+    using C = KVCfg<DK, DV, GATE>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sG = sm + C::NS * C::STAGE;
+    uint8_t* sAm = sG + C::GTB;
+    uint8_t* sdA = sAm + C::AB;
+    uint8_t* small = sdA + C::AB;
+    uint64_t* bar_full = reinterpret_cast<uint64_t*>(small);
+    uint64_t* bar_mma1 = bar_full + 2;
+    uint64_t* bar_mma2 = bar_full + 3;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 64);
+    float* tot = reinterpret_cast<float*>(small + 256);
+    float* gam = tot + 1024;      // [DK]
+    float* rowE = gam + DK;       // [64]
+    float* rowEi = rowE + TR;
+    float* igs = rowEi + TR;
+    float* ghs = igs + TR;
+    float* sdi = ghs + TR;        // [2][64]
+
+    const int bh = blockIdx.x, z = blockIdx.y;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2, qd = warp & 3;
+    const int ntiles_all = cdiv(P.L, TR);
+    const int tile0 = z * A.tiles_per_seg;
+    const int ntiles = min(ntiles_all, tile0 + A.tiles_per_seg) - tile0;
+    const long rowbase = (long)bh * P.L;
+    const bool srow_ok = (DK != 64) || (lane < 16);
+    const int srow = DK == 64 ? 16 * qd + (lane & 15) : 32 * qd + lane;
+    auto tile_at = [&](int j) { return tile0 + ntiles - 1 - j; };
+
+    if (tid == 0) {
+        mbar_init(&bar_full[0], 1);
+        mbar_init(&bar_full[1], 1);
+        mbar_init(bar_mma1, 1);
+        mbar_init(bar_mma2, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, C::NCOL);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tlane = tbase + ((uint32_t)(32 * qd) << 16);
+
+    // ---- state gradient at the end of the segment into TMEM
+    {
+        const float* src = nullptr;
+        if (z == A.nseg - 1) src = A.dhT ? A.dhT + ((long)bh * DK + srow) * P.Dv : nullptr;
+        else src = A.gend + (((long)bh * A.nseg + z) * DK + srow) * P.Dv;
+        for (int c = wg * C::HC; c < (wg + 1) * C::HC; c += 16) {
+            uint32_t r[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) r[j] = __float_as_uint((src && srow_ok) ? src[c + j] : 0.f);
+            tmem_st16(tlane + c, r);
+        }
+        tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    auto issue_loads = [&](int i, int s) {
+        uint8_t* st = sm + s * C::STAGE;
+        const int t0 = tile_at(i) * TR;
+        mbar_arrive_expect_tx(&bar_full[s], C::STAGE);
+        for (int cb = 0; cb < DK / 64; ++cb) {
+            tma_load_3d(st + cb * BLK, &tq, cb * 64, t0, bh, &bar_full[s]);
+            tma_load_3d(st + C::QB + cb * BLK, &tk, cb * 64, t0, bh, &bar_full[s]);
+        }
+        if (GATE == 1) tma_load_3d(st + C::QB + C::KB, &tg, 0, t0, bh, &bar_full[s]);
+        for (int vb = 0; vb < DV / 64; ++vb) {
+            tma_load_3d(st + C::QB + C::KB + C::GB + vb * BLK, &tv, vb * 64, t0, bh, &bar_full[s]);
+            tma_load_3d(st + C::QB + C::KB + C::GB + C::VB + vb * BLK, &tdo, vb * 64, t0, bh, &bar_full[s]);
+        }
+    };
+    if (tid == 0)
+        for (int i = 0; i < C::NS && i < ntiles; ++i) issue_loads(i, i);
+
+    int err = 0, n_mma = 0;
+    for (int i = 0; i < ntiles; ++i) {
+        const int s = i % C::NS;
+        uint8_t* st = sm + s * C::STAGE;
+        uint8_t* sq = st;
+        uint8_t* sk = st + C::QB;
+        float* sg = reinterpret_cast<float*>(st + C::QB + C::KB);
+        uint8_t* sv = st + C::QB + C::KB + C::GB;
+        uint8_t* so = sv + C::VB;
+        const int t0 = tile_at(i) * TR;
+        if (tid < TR) {
+            const int t = t0 + tid;
+            igs[tid] = (A.ig && t < P.L) ? A.ig[rowbase + t] : 1.f;
+            if (GATE == 2) ghs[tid] = (t < P.L) ? A.gh[rowbase + t] : 0.f;
+        }
+        if (!block_wait(&bar_full[s], (i / C::NS) & 1)) { err = 1; break; }
+
+        // ---- transform: q~ = scale q e^b, k~ = i k e^-b (in place); e^-b kept in place of g
+        constexpr int NP = DK / 2, RG = NT_B / NP, RPG = TR / RG;
+        const int cp = tid % NP, rg = tid / NP, d = 2 * cp;
+        if (GATE == 1) {
+            float ax = 0.f, ay = 0.f;
+            for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
+                const float2 gv = *reinterpret_cast<const float2*>(sg + r * DK + d);
+                ax += gv.x;
+                ay += gv.y;
+            }
+            tot[rg * DK + d] = ax;
+            tot[rg * DK + d + 1] = ay;
+        } else if (GATE == 2 && warp == 0) {
+            const float g0 = ghs[2 * lane], g1 = ghs[2 * lane + 1];
+            float v = g0 + g1;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float n = __shfl_up_sync(0xffffffffu, v, off);
+                if (lane >= off) v += n;
+            }
+            const float b1 = v, b0 = v - g1;
+            rowE[2 * lane] = __expf(b0);
+            rowE[2 * lane + 1] = __expf(b1);
+            rowEi[2 * lane] = __expf(-b0);
+            rowEi[2 * lane + 1] = __expf(-b1);
+            const float G = __shfl_sync(0xffffffffu, b1, 31);
+            if (lane == 0) gam[0] = __expf(G);
+        }
+        __syncthreads();
+        {
+            float bx = 0.f, by = 0.f;
+            if (GATE == 1) {
+                float Gx = 0.f, Gy = 0.f;
+                for (int r2 = 0; r2 < RG; ++r2) {
+                    const float tx = tot[r2 * DK + d], ty = tot[r2 * DK + d + 1];
+                    if (r2 < rg) { bx += tx; by += ty; }
+                    Gx += tx;
+                    Gy += ty;
+                }
+                if (rg == 0) { gam[d] = __expf(Gx); gam[d + 1] = __expf(Gy); }
+            }
+            for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
+                float eqx = 1.f, eqy = 1.f, ekx = 1.f, eky = 1.f;
+                if (GATE == 1) {
+                    float2* gp = reinterpret_cast<float2*>(sg + r * DK + d);
+                    const float2 gv = *gp;
+                    bx += gv.x;
+                    by += gv.y;
+                    eqx = __expf(bx);
+                    eqy = __expf(by);
+                    ekx = __expf(-bx);
+                    eky = __expf(-by);
+                    *gp = make_float2(ekx, eky);
+                } else if (GATE == 2) {
+                    eqx = eqy = rowE[r];
+                    ekx = eky = rowEi[r];
+                }
+                const float iv = igs[r];
+                const uint32_t off = sw128_off(r, d, BLK);
+                __nv_bfloat162* pq = reinterpret_cast<__nv_bfloat162*>(sq + off);
+                const float2 qf = __bfloat1622float2(*pq);
+                *pq = __floats2bfloat162_rn(qf.x * P.scale * eqx, qf.y * P.scale * eqy);
+                __nv_bfloat162* pk = reinterpret_cast<__nv_bfloat162*>(sk + off);
+                const float2 kf = __bfloat1622float2(*pk);
+                *pk = __floats2bfloat162_rn(kf.x * iv * ekx, kf.y * iv * eky);
+            }
+        }
+        __syncthreads();
+        // ---- G~ = e^Gamma G in TMEM; bf16 copy
+        {
+            const float eg = GATE == 0 ? 1.f : gam[GATE == 1 ? srow : 0];
+            for (int c = wg * C::HC; c < (wg + 1) * C::HC; c += 16) {
+                uint32_t r[16];
+                float f[16];
+                tmem_ld16(tlane + c, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    f[j] = eg * __uint_as_float(r[j]);
+                    r[j] = __float_as_uint(f[j]);
+                }
+                tmem_st16(tlane + c, r);
+                if (srow_ok) {
+                    store8_bf16(sG, sw128_off(srow, c, DK * 128), f);
+                    store8_bf16(sG, sw128_off(srow, c + 8, DK * 128), f + 8);
+                }
+            }
+            tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ---- MMA group 1: A = (scale q~) k~^T, dA = dO V^T
+        if (tid == 0) {
+            const uint32_t qa = smem_u32(sq), ka = smem_u32(sk), va = smem_u32(sv), oa = smem_u32(so);
+            const uint32_t id64 = idesc_bf16(64, 64, 0, 0);
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+                mma_bf16(tbase + C::COL_R, sw128_desc(qa + koff, 16, 1024), sw128_desc(ka + koff, 16, 1024), id64,
+                         kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < DV / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+                mma_bf16(tbase + (16u << 16) + C::COL_R, sw128_desc(oa + koff, 16, 1024),
+                         sw128_desc(va + koff, 16, 1024), id64, kk > 0);
+            }
+            mma_commit(bar_mma1);
+        }
+        ++n_mma;
+        if (!block_wait(bar_mma1, i & 1)) { err = 1; break; }
+        tc_fence_after();
+        {
+            uint32_t r[32];
+            tmem_ld32(tlane + C::COL_R + 32 * wg, r);
+            tmem_wait_ld();
+            const int t = 16 * qd + (lane & 15);
+            uint8_t* dst = lane < 16 ? sAm : sdA;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float f[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int sidx = 32 * wg + 8 * u + j;
+                    f[j] = (sidx <= t) ? __uint_as_float(r[8 * u + j]) : 0.f;
+                }
+                store8_bf16(dst, sw128_off(t, 32 * wg + 8 * u, BLK), f);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ---- MMA group 2: dk', dv, G update
+        if (tid == 0) {
+            const uint32_t qa = smem_u32(sq), ka = smem_u32(sk), va = smem_u32(sv), oa = smem_u32(so);
+            const uint32_t ga = smem_u32(sG), ama = smem_u32(sAm), dama = smem_u32(sdA);
+            const uint32_t tdk = tbase + C::COL_R, tdv = tbase + (16u << 16) + C::COL_R;
+            const uint32_t idK1 = idesc_bf16(64, DK, 1, 1), idK2 = idesc_bf16(64, DK, 0, 0);
+            const uint32_t idV1 = idesc_bf16(64, DV, 1, 1), idV2 = idesc_bf16(64, DV, 0, 1);
+            const uint32_t idG = idesc_bf16(DK, DV, 1, 1);
+#pragma unroll
+            for (int ks = 0; ks < TR / 16; ++ks)  // mask(dA)^T (scale q~)
+                mma_bf16(tdk, sw128_desc(dama + ks * 2048, BLK, 1024), sw128_desc(qa + ks * 2048, BLK, 1024), idK1,
+                         ks > 0);
+#pragma unroll
+            for (int kk = 0; kk < DV / 16; ++kk) {  // V G~^T
+                const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+                const uint32_t goff = (kk >> 2) * (DK * 128) + (kk & 3) * 32;
+                mma_bf16(tdk, sw128_desc(va + koff, 16, 1024), sw128_desc(ga + goff, 16, 1024), idK2, 1);
+            }
+#pragma unroll
+            for (int ks = 0; ks < TR / 16; ++ks)  // mask(A)^T dO
+                mma_bf16(tdv, sw128_desc(ama + ks * 2048, BLK, 1024), sw128_desc(oa + ks * 2048, BLK, 1024), idV1,
+                         ks > 0);
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk) {  // k~ G~
+                const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+                mma_bf16(tdv, sw128_desc(ka + koff, 16, 1024), sw128_desc(ga + kk * 2048, DK * 128, 1024), idV2, 1);
+            }
+#pragma unroll
+            for (int ks = 0; ks < TR / 16; ++ks)  // G += (scale q~)^T dO
+                mma_bf16(tbase, sw128_desc(qa + ks * 2048, BLK, 1024), sw128_desc(oa + ks * 2048, BLK, 1024), idG, 1);
+            mma_commit(bar_mma2);
+        }
+        if (!block_wait(bar_mma2, i & 1)) { err = 1; break; }
+        tc_fence_after();
+
+        // ---- dk = i e^-b X,  di = sum_d k~ X / i,  dv
+        {
+            const int srw = 16 * qd + (lane & 15);
+            const bool row_ok = t0 + srw < P.L;
+            float dsum = 0.f;
+            for (int c = wg * C::KC; c < (wg + 1) * C::KC; c += 16) {
+                uint32_t r[16];
+                tmem_ld16(tlane + C::COL_R + c, r);
+                tmem_wait_ld();
+                if (lane < 16 && row_ok) {
+                    const float iv = igs[srw];
+                    float f[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float x = __uint_as_float(r[j]);
+                        const float em = GATE == 1 ? sg[srw * DK + c + j] : (GATE == 2 ? rowEi[srw] : 1.f);
+                        f[j] = iv * em * x;
+                        const __nv_bfloat16 kt =
+                            *reinterpret_cast<const __nv_bfloat16*>(sk + sw128_off(srw, c + j, BLK));
+                        dsum += __bfloat162float(kt) * x;
+                    }
+                    store16_bf16_global(A.dk + (rowbase + t0 + srw) * DK + c, f);
+                }
+            }
+            if (lane < 16) sdi[wg * TR + srw] = dsum;
+            for (int c = wg * C::HC; c < (wg + 1) * C::HC; c += 16) {
+                uint32_t r[16];
+                tmem_ld16(tlane + C::COL_R + c, r);
+                tmem_wait_ld();
+                if (lane >= 16 && row_ok) {
+                    float f[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) f[j] = __uint_as_float(r[j]);
+                    store16_bf16_global(A.dv + (rowbase + t0 + srw) * DV + c, f);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (A.di && tid < TR && t0 + tid < P.L) A.di[rowbase + t0 + tid] = (sdi[tid] + sdi[TR + tid]) / igs[tid];
+        if (tid == 0 && i + C::NS < ntiles) issue_loads(i + C::NS, s);
+    }
+
+    if (err) {
+        if (tid == 0) {
+            atomicExch(A.status, kDevStatusTimeout);
+            if (n_mma) {
+                mbar_wait(bar_mma1, (n_mma - 1) & 1, 1u << 20);
+                mbar_wait(bar_mma2, (n_mma - 1) & 1, 1u << 20);
+            }
+        }
+    } else if (A.dh0 && z == 0) {
+        for (int c = wg * C::HC; c < (wg + 1) * C::HC; c += 16) {
+            uint32_t r[16];
+            tmem_ld16(tlane + c, r);
+            tmem_wait_ld();
+            if (srow_ok) {
+                float* dst = A.dh0 + ((long)bh * DK + srow) * P.Dv + c;
+#pragma unroll
+                for (int j = 0; j < 16; j += 4)
+                    *reinterpret_cast<float4*>(dst + j) = make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                                                      __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, C::NCOL);
+}
+
+// ============================================================================ dg
+// Per-key gates: block (b*h, 64 key dims); 256 threads = 64 columns x 4 row groups of 16.
+// Walks 64-token tiles from the end: dB = q dq - k dk, reverse cumsum with a carry.
+__global__ void __launch_bounds__(256) k_tc_bwd_dg_key(const __nv_bfloat16* __restrict__ q,
+                                                       const __nv_bfloat16* __restrict__ dq,
+                                                       const __nv_bfloat16* __restrict__ k,
+                                                       const __nv_bfloat16* __restrict__ dk,
+                                                       const float* __restrict__ dhT, const float* __restrict__ hT,
+                                                       float* __restrict__ dg, Dims P) {
+    const long bh = blockIdx.x;
+    const int col = threadIdx.x & 63, rg = threadIdx.x >> 6;
+    const int d = blockIdx.y * 64 + col;
+    __shared__ float tots[4][64];
+    float carry = 0.f;
+    if (dhT) {
+        const float* a = dhT + (bh * P.Dk + d) * (long)P.Dv;
+        const float* h = hT + (bh * P.Dk + d) * (long)P.Dv;
+        for (int e = 0; e < P.Dv; ++e) carry += a[e] * h[e];
+    }
+    const int ntiles = cdiv(P.L, TR);
+    for (int ti = ntiles - 1; ti >= 0; --ti) {
+        float x[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int t = ti * TR + rg * 16 + j;
+            float v = 0.f;
+            if (t < P.L) {
+                const long idx = (bh * P.L + t) * P.Dk + d;
+                v = __bfloat162float(q[idx]) * __bfloat162float(dq[idx]) -
+                    __bfloat162float(k[idx]) * __bfloat162float(dk[idx]);
+            }
+            x[j] = v;
+        }
+        float s = 0.f;
+#pragma unroll
+        for (int j = 15; j >= 0; --j) {
+            s += x[j];
+            x[j] = s;
+        }
+        tots[rg][col] = s;
+        __syncthreads();
+        float later = carry;
+        for (int r2 = rg + 1; r2 < 4; ++r2) later += tots[r2][col];
+        float tile_total = 0.f;
+#pragma unroll
+        for (int r2 = 0; r2 < 4; ++r2) tile_total += tots[r2][col];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int t = ti * TR + rg * 16 + j;
+            if (t < P.L) dg[(bh * P.L + t) * P.Dk + d] = x[j] + later;
+        }
+        carry += tile_total;
+        __syncthreads();
+    }
+}
+
+// Per-head gates: block per b*h; dB summed over key dims per token, then the scalar
+// reverse cumsum. Warp w handles tokens 8w..8w+7 of each tile.
+__global__ void __launch_bounds__(256) k_tc_bwd_dg_head(const __nv_bfloat16* __restrict__ q,
+                                                        const __nv_bfloat16* __restrict__ dq,
+                                                        const __nv_bfloat16* __restrict__ k,
+                                                        const __nv_bfloat16* __restrict__ dk,
+                                                        const float* __restrict__ dhT, const float* __restrict__ hT,
+                                                        float* __restrict__ dg, Dims P) {
+    const long bh = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ float rows[TR];
+    __shared__ float red[8];
+    float part = 0.f;
+    if (dhT) {
+        const long n = (long)P.Dk * P.Dv;
+        for (long i = threadIdx.x; i < n; i += blockDim.x) part += dhT[bh * n + i] * hT[bh * n + i];
+    }
+    for (int off = 16; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    if (lane == 0) red[warp] = part;
+    __syncthreads();
+    float carry = 0.f;
+    for (int w = 0; w < 8; ++w) carry += red[w];
+    const int ntiles = cdiv(P.L, TR);
+    for (int ti = ntiles - 1; ti >= 0; --ti) {
+        for (int j = 0; j < 8; ++j) {
+            const int r = warp * 8 + j, t = ti * TR + r;
+            float sacc = 0.f;
+            if (t < P.L)
+                for (int dd = lane; dd < P.Dk; dd += 32) {
+                    const long idx = (bh * P.L + t) * P.Dk + dd;
+                    sacc += __bfloat162float(q[idx]) * __bfloat162float(dq[idx]) -
+                            __bfloat162float(k[idx]) * __bfloat162float(dk[idx]);
+                }
+            for (int off = 16; off >= 1; off >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, off);
+            if (lane == 0) rows[r] = sacc;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            // reverse inclusive scan over 64 rows, two per lane
+            const float a0 = rows[2 * lane], a1 = rows[2 * lane + 1];
+            float v = a0 + a1;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float n = __shfl_down_sync(0xffffffffu, v, off);
+                if (lane + off < 32) v += n;
+            }
+            const float s0 = v + carry, s1 = v - a0 + carry;
+            const int t0 = ti * TR + 2 * lane;
+            if (t0 < P.L) dg[bh * P.L + t0] = s0;
+            if (t0 + 1 < P.L) dg[bh * P.L + t0 + 1] = s1;
+            const float total = __shfl_sync(0xffffffffu, v, 0);
+            carry += total;
+        }
+        carry = __shfl_sync(0xffffffffu, carry, 0);
+        __syncthreads();
+        if (threadIdx.x == 0) red[0] = carry;
+        __syncthreads();
+        carry = red[0];
+        __syncthreads();
+    }
+}
+
+// ============================================================================ host side
+struct BwdPlan {
+    int nseg, tiles_per_seg, dkb;
+};
+
+static BwdPlan plan_bwd(const Dims& P) {
+    BwdPlan pl{};
+    pl.dkb = P.Dk > 128 ? 128 : P.Dk;
+    const int ntiles = cdiv(P.L, TR);
+    const long base = (long)P.B * P.H;
+    const int sms = num_sms();
+    int nseg = 1;
+    if (base * 4 < (long)sms * 3 && ntiles > 1) nseg = (int)((long)sms / base);
+    if (nseg < 1) nseg = 1;
+    const int tiles_per_chunk = P.C / TR;
+    const int nchunks = cdiv(P.L, P.C);
+    if (nseg > nchunks) nseg = nchunks;
+    const int chunks_per_seg = cdiv(nchunks, nseg);
+    pl.tiles_per_seg = chunks_per_seg * tiles_per_chunk;
+    pl.nseg = cdiv(ntiles, pl.tiles_per_seg);
+    if (pl.nseg < 1) pl.nseg = 1;
+    return pl;
+}
+
+bool bwd_supports(const Dims& P) {
+    return P.C % TR == 0 && (P.Dk == 64 || P.Dk == 128) && (P.Dv == 64 || P.Dv == 128 || P.Dv == 256);
+}
+
+struct BwdWs {
+    float *seg_state, *seg_gamma, *sinit, *gend, *hT;
+    size_t total;
+};
+
+static BwdWs bwd_layout(const Dims& P, char* base) {
+    const BwdPlan pl = plan_bwd(P);
+    const size_t BH = (size_t)P.B * P.H, st = 4 * BH * (size_t)P.Dk * P.Dv;
+    BwdWs w{};
+    size_t off = kStatusBytes;
+    w.hT = reinterpret_cast<float*>(base + off);
+    off = align_up(off + st, 256);
+    if (pl.nseg > 1) {
+        w.seg_state = reinterpret_cast<float*>(base + off);
+        off = align_up(off + st * pl.nseg, 256);
+        w.seg_gamma = reinterpret_cast<float*>(base + off);
+        off = align_up(off + 4 * BH * pl.nseg * P.Dk, 256);
+        w.sinit = reinterpret_cast<float*>(base + off);
+        off = align_up(off + st * pl.nseg, 256);
+        w.gend = reinterpret_cast<float*>(base + off);
+        off = align_up(off + st * pl.nseg, 256);
+    }
+    w.total = off;
+    return w;
+}
+
+size_t bwd_workspace_bytes(const Dims& P) { return bwd_layout(P, nullptr).total; }
+
+template <int DKB, int DV, int GATE>
+static cudaError_t launch_dq(const Dims& P, const BwdPlan& pl, const CUtensorMap& mk, const CUtensorMap& mg,
+                             const CUtensorMap& mv, const CUtensorMap& mo, const BwdArgs& a, cudaStream_t st) {
+    using C = QCfg<DKB, DV, GATE>;
+    auto kern = k_tc_bwd_dq<DKB, DV, GATE>;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    dim3 grid(P.B * P.H, P.Dk / DKB, pl.nseg);
+    GLA_LAUNCH("tc_bwd_dq", st, kern<<<grid, NT_B, C::SMEM, st>>>(mk, mg, mv, mo, a, P));
+    return cudaGetLastError();
+}
+
+template <int DK, int DV, int GATE>
+static cudaError_t launch_dkdv(const Dims& P, const BwdPlan& pl, const CUtensorMap& mq, const CUtensorMap& mk,
+                               const CUtensorMap& mg, const CUtensorMap& mv, const CUtensorMap& mo, const BwdArgs& a,
+                               cudaStream_t st) {
+    using C = KVCfg<DK, DV, GATE>;
+    auto kern = k_tc_bwd_dkdv<DK, DV, GATE>;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    dim3 grid(P.B * P.H, pl.nseg);
+    GLA_LAUNCH("tc_bwd_dkdv", st, kern<<<grid, NT_B, C::SMEM, st>>>(mq, mk, mg, mv, mo, a, P));
+    return cudaGetLastError();
+}
+
+template <int DK, int DV, int GATE>
+static cudaError_t run_bwd(const Dims& P, const void* q, const void* k, const void* v, const float* g,
+                           const float* ig, const float* h0, const void* dO, const float* dhT, void* dq, void* dk,
+                           void* dv, float* dg, float* di, float* dh0, void* ws, cudaStream_t st) {
+    const BwdPlan pl = plan_bwd(P);
+    const BwdWs w = bwd_layout(P, static_cast<char*>(ws));
+    const int BH = P.B * P.H;
+    constexpr int DKB = DK > 128 ? 128 : DK;
+    CUtensorMap mq, mk, mv, mo, mg, mgb;
+    if (!make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dk, P.L, BH, 64, true) ||
+        !make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dk, P.L, BH, 64, true) ||
+        !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dv, P.L, BH, 64, true) ||
+        !make_map(&mo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dv, P.L, BH, 64, true))
+        return cudaErrorInvalidValue;
+    if (GATE == 1) {
+        if (!make_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, P.Dk, P.L, BH, P.Dk, false) ||
+            !make_map(&mgb, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, P.Dk, P.L, BH, DKB, false))
+            return cudaErrorInvalidValue;
+    } else {
+        mg = mk;
+        mgb = mk;
+    }
+    int* status = static_cast<int*>(ws);
+    cudaError_t e;
+    if (pl.nseg > 1) {
+        e = state_pass(P, 1, k, v, g, ig, pl.nseg, pl.tiles_per_seg, w.seg_state, w.seg_gamma, status, st);
+        if (e != cudaSuccess) return e;
+        e = seg_scan(P, pl.nseg, w.seg_state, w.seg_gamma, h0, w.sinit, st);
+        if (e != cudaSuccess) return e;
+    }
+    BwdArgs a{};
+    a.gh = GATE == 2 ? g : nullptr;
+    a.ig = ig;
+    a.sinit = w.sinit;
+    a.h0 = h0;
+    a.gend = w.gend;
+    a.dhT = dhT;
+    a.dq = static_cast<__nv_bfloat16*>(dq);
+    a.dk = static_cast<__nv_bfloat16*>(dk);
+    a.dv = static_cast<__nv_bfloat16*>(dv);
+    a.di = di;
+    a.dh0 = dh0;
+    a.hT_ws = (dhT && GATE != 0) ? w.hT : nullptr;
+    a.status = status;
+    a.tiles_per_seg = pl.tiles_per_seg;
+    a.nseg = pl.nseg;
+    e = launch_dq<DKB, DV, GATE>(P, pl, mk, mgb, mv, mo, a, st);
+    if (e != cudaSuccess) return e;
+    if (pl.nseg > 1) {
+        e = state_pass(P, 2, q, dO, g, ig, pl.nseg, pl.tiles_per_seg, w.seg_state, w.seg_gamma, status, st);
+        if (e != cudaSuccess) return e;
+        e = seg_rscan(P, pl.nseg, w.seg_state, w.seg_gamma, dhT, w.gend, st);
+        if (e != cudaSuccess) return e;
+    }
+    e = launch_dkdv<DK, DV, GATE>(P, pl, mq, mk, mg, mv, mo, a, st);
+    if (e != cudaSuccess) return e;
+    if (GATE == 1) {
+        GLA_LAUNCH("tc_bwd_dg", st,
+                   k_tc_bwd_dg_key<<<dim3(BH, P.Dk / 64), 256, 0, st>>>(
+                       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dq),
+                       static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(dk), dhT, w.hT, dg, P));
+    } else if (GATE == 2) {
+        GLA_LAUNCH("tc_bwd_dg", st,
+                   k_tc_bwd_dg_head<<<BH, 256, 0, st>>>(
+                       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dq),
+                       static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(dk), dhT, w.hT, dg, P));
+    }
+    return cudaGetLastError();
+}
+
+template <int DK, int DV>
+static cudaError_t bwd_gate(const Dims& P, const void* q, const void* k, const void* v, const float* g,
+                            const float* ig, const float* h0, const void* dO, const float* dhT, void* dq, void* dk,
+                            void* dv, float* dg, float* di, float* dh0, void* ws, cudaStream_t st) {
+    switch (P.gate) {
+        case GLA_GATE_NONE: return run_bwd<DK, DV, 0>(P, q, k, v, g, ig, h0, dO, dhT, dq, dk, dv, dg, di, dh0, ws, st);
+        case GLA_GATE_PER_KEY:
+            return run_bwd<DK, DV, 1>(P, q, k, v, g, ig, h0, dO, dhT, dq, dk, dv, dg, di, dh0, ws, st);
+        default: return run_bwd<DK, DV, 2>(P, q, k, v, g, ig, h0, dO, dhT, dq, dk, dv, dg, di, dh0, ws, st);
+    }
+}
+
+cudaError_t bwd(const Dims& P, const void* q, const void* k, const void* v, const float* g, const float* ig,
+                const float* h0, const void* dO, const float* dhT, void* dq, void* dk, void* dv, float* dg, float* di,
+                float* dh0, void* ws, cudaStream_t st) {
+#define GLA_BWD_CASE(DK_, DV_)                                                                      \
+    if (P.Dk == DK_ && P.Dv == DV_)                                                                 \
+        return bwd_gate<DK_, DV_>(P, q, k, v, g, ig, h0, dO, dhT, dq, dk, dv, dg, di, dh0, ws, st);
+    GLA_BWD_CASE(64, 64)
+    GLA_BWD_CASE(64, 128)
+    GLA_BWD_CASE(64, 256)
+    GLA_BWD_CASE(128, 64)
+    GLA_BWD_CASE(128, 128)
+    GLA_BWD_CASE(128, 256)
+#undef GLA_BWD_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace tc
+}  // namespace gla

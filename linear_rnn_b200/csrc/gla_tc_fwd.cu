@@ -28,19 +28,18 @@
 
 #include "gla_common.cuh"
 #include "gla_plans.h"
-#include "sm100.cuh"
+#include "gla_tc_common.cuh"
 
 namespace gla {
 namespace tc {
 
 using namespace sm100;
 
-constexpr int TR = 64;        // tokens per tile
-constexpr uint32_t BLK = 8192;  // one 64-column bf16 block of a 64-row tile (64 x 128 B)
 
 template <int DK, int DVT, int GATE, int MODE>
 struct Cfg {
     // MODE 0: output pass (q, k, g, v). MODE 1: state-only pass (k, g, v).
+    // MODE 2: reverse state-gradient pass (q in the k slot, g, dO in the v slot).
     static constexpr uint32_t QB = MODE == 0 ? TR * DK * 2 : 0;
     static constexpr uint32_t KB = TR * DK * 2;
     static constexpr uint32_t GB = GATE == 1 ? TR * DK * 4 : 0;
@@ -76,17 +75,8 @@ struct FwdArgs {
     int* status;
     int tiles_per_seg;
     int nseg;
+    int seg_offset;       // segment index = blockIdx.z + seg_offset
 };
-
-__device__ __forceinline__ void store8_bf16(uint8_t* base, uint32_t off, const float* v) {
-    uint32_t w[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        __nv_bfloat162 p = __floats2bfloat162_rn(v[2 * u], v[2 * u + 1]);
-        w[u] = *reinterpret_cast<uint32_t*>(&p);
-    }
-    *reinterpret_cast<uint4*>(base + off) = make_uint4(w[0], w[1], w[2], w[3]);
-}
 
 // Thread roles: warps 0-15 (four warpgroups) transform tiles and run the epilogues; warp 16
 // issues the tcgen05 MMAs; warp 17 issues the TMA loads. They hand tiles to each other
@@ -132,13 +122,15 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     float* igs = rowEi + TR;                                 // [64] input gate
     float* ghs = igs + TR;                                   // [64] per-head gate
 
-    const int bh = blockIdx.x, vt = blockIdx.y, z = blockIdx.z;
+    const int bh = blockIdx.x, vt = blockIdx.y, z = blockIdx.z + A.seg_offset;
     const int e0 = vt * DVT;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = (warp >> 2) & 3, qd = warp & 3;
     const int ntiles_all = cdiv(P.L, TR);
     const int tile0 = z * A.tiles_per_seg;
     const int ntiles = min(ntiles_all, tile0 + A.tiles_per_seg) - tile0;
     const long rowbase = (long)bh * P.L;
+    // the j-th tile this CTA processes (MODE 2 walks its segment backwards)
+    auto tile_at = [&](int j) { return MODE == 2 ? tile0 + ntiles - 1 - j : tile0 + j; };
 
     if (tid == 0) {
         for (int j = 0; j < 15; ++j) mbar_init(&bars[j], 1);
@@ -190,7 +182,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 const int s = j % C::NS;
                 if (j >= C::NS && !mbar_wait_abort(&bar_empty[s], ((j / C::NS) - 1) & 1, abortp)) break;
                 uint8_t* st = sm + s * C::STAGE;
-                const int t0 = (tile0 + j) * TR;
+                const int t0 = tile_at(j) * TR;
                 mbar_arrive_expect_tx(&bar_full[s], C::STAGE);
                 if (MODE == 0)
                     for (int cb = 0; cb < DK / 64; ++cb)
@@ -272,7 +264,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
             const float* sg = reinterpret_cast<const float*>(st + C::QB + C::KB);
             float* gam = gamb + b * DK;
             float* gaml = gamlb + b * DK;
-            const int t0 = (tile0 + j) * TR;
+            const int t0 = tile_at(j) * TR;
             if (ctid < TR) {
                 const int t = t0 + ctid;
                 igs[ctid] = (A.ig && t < P.L) ? A.ig[rowbase + t] : 1.f;
@@ -356,7 +348,10 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 }
                 __nv_bfloat162* pk = reinterpret_cast<__nv_bfloat162*>(sk + off);
                 const float2 kf = __bfloat1622float2(*pk);
-                *pk = __floats2bfloat162_rn(kf.x * iv * ekx, kf.y * iv * eky);
+                if (MODE == 2)  // the k slot holds q: scale * q * e^b
+                    *pk = __floats2bfloat162_rn(kf.x * P.scale * eqx, kf.y * P.scale * eqy);
+                else
+                    *pk = __floats2bfloat162_rn(kf.x * iv * ekx, kf.y * iv * eky);
             }
             fence_proxy_async_smem();
             named_bar_sync(BAR_COMP, NCOMP);
@@ -373,7 +368,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 if (!named_bar_and(BAR_COMP, NCOMP, ok)) break;
             }
             tc_fence_after();
-            const int t0 = (tile0 + i) * TR;
+            const int t0 = tile_at(i) * TR;
             // ---- P = causal mask of A -> shared (double-buffered)
             if (MODE == 0) {
                 uint8_t* sP = sPb + b * (TR * TR * 2);
@@ -413,7 +408,10 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                         tmem_ld16(tb + ((uint32_t)(32 * qd) << 16) + C::COL_S + h * DVT + wg * C::HALF + c, r);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) Sreg[h][c + j] = egv * (Sreg[h][c + j] + __uint_as_float(r[j]));
+                        if (MODE == 2)  // G_before = e^Gamma G_after + scale q~^T dO
+                            for (int j = 0; j < 16; ++j) Sreg[h][c + j] = egv * Sreg[h][c + j] + __uint_as_float(r[j]);
+                        else
+                            for (int j = 0; j < 16; ++j) Sreg[h][c + j] = egv * (Sreg[h][c + j] + __uint_as_float(r[j]));
                     }
                     if (MODE == 0 && srow_ok) {
 #pragma unroll
@@ -531,34 +529,42 @@ __global__ void k_seg_scan(const float* __restrict__ seg_state, const float* __r
     }
 }
 
-// ------------------------------------------------------------------ host side
-static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+// Reverse segment scan for the backward: gend[z] = gradient w.r.t. the state at the end of
+// segment z; gend[nseg-1] = dhT (or 0), gend[z] = e^{Gamma_{z+1}} gend[z+1] + dG_{z+1},
+// where dG_z (seg_state[z]) is segment z's own state-gradient accumulated from zero at
+// its end and Gamma_z (seg_gamma[z]) its total log-decay.
+__global__ void k_seg_rscan(const float* __restrict__ seg_state, const float* __restrict__ seg_gamma,
+                            const float* __restrict__ dhT, float* __restrict__ gend, int BH, int Dk, int Dv, int nseg) {
+    const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long per = (long)Dk * Dv;
+    if (idx >= (long)BH * per) return;
+    const long bh = idx / per, de = idx % per;
+    const int d = (int)(de / Dv);
+    float G = dhT ? dhT[idx] : 0.f;
+    gend[((bh * nseg + nseg - 1) * per) + de] = G;
+    constexpr int BATCH = 16;
+    for (int z0 = nseg - 1; z0 >= 1; z0 -= BATCH) {
+        float dg[BATCH], gl[BATCH];
+#pragma unroll
+        for (int u = 0; u < BATCH; ++u) {
+            const int z = z0 - u;
+            if (z >= 1) {
+                dg[u] = seg_state[((bh * nseg + z) * per) + de];
+                gl[u] = seg_gamma[(bh * nseg + z) * Dk + d];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < BATCH; ++u) {
+            const int z = z0 - u;
+            if (z >= 1) {
+                G = __expf(gl[u]) * G + dg[u];
+                gend[((bh * nseg + z - 1) * per) + de] = G;
+            }
+        }
     }
-    return fn;
 }
 
-// 3D map over [BH][L][D] (D innermost) with a box of {box0, 64, 1}.
-static bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int D, int L, int BH,
-                     int box0, bool swz) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)L, (cuuint64_t)BH};
-    cuuint64_t strides[2] = {(cuuint64_t)D * esize, (cuuint64_t)D * esize * L};
-    cuuint32_t box[3] = {(cuuint32_t)box0, (cuuint32_t)TR, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
+// ------------------------------------------------------------------ host side
 template <int DK, int DVT, int GATE, int MODE>
 static cudaError_t launch_one(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                               const CUtensorMap& mg, const FwdArgs& a, const Dims& P, int nseg, cudaStream_t st) {
@@ -571,13 +577,14 @@ static cudaError_t launch_one(const CUtensorMap& mq, const CUtensorMap& mk, cons
         attr = true;
     }
     dim3 grid(P.B * P.H, P.Dv / DVT, nseg);
-    GLA_LAUNCH(MODE == 0 ? "tc_fwd" : "tc_fwd_state", st, kern<<<grid, NTHR_WS, C::SMEM, st>>>(mq, mk, mv, mg, a, P));
+    GLA_LAUNCH(MODE == 0 ? "tc_fwd" : MODE == 1 ? "tc_state" : "tc_gstate", st,
+               kern<<<grid, NTHR_WS, C::SMEM, st>>>(mq, mk, mv, mg, a, P));
     return cudaGetLastError();
 }
 
 int pick_dvt(const Dims& P) { return (P.Dk == 256 || P.Dv % 128 != 0) ? 64 : 128; }
 
-static int num_sms() {
+int num_sms() {
     static int n = 0;
     if (!n) {
         int dev = 0;
@@ -623,6 +630,39 @@ bool supports(const Dims& P) {
     return P.C % TR == 0 && (P.Dk == 64 || P.Dk == 128 || P.Dk == 256) && P.Dv % 64 == 0;
 }
 
+cudaError_t seg_scan(const Dims& P, int nseg, const float* seg_state, const float* seg_gamma, const float* h0,
+                     float* sinit, cudaStream_t st);
+
+// State-only pass over every segment but one: MODE 1 (forward states: a = k, b = v) runs
+// segments 0..nseg-2, MODE 2 (reverse state gradients: a = q, b = dO) segments 1..nseg-1.
+template <int DK, int DVT, int GATE>
+static cudaError_t state_run(const Dims& P, int mode, const void* a_src, const void* b_src, const float* g,
+                             const float* ig, int nseg, int tps, float* seg_state, float* seg_gamma, int* status,
+                             cudaStream_t st) {
+    CUtensorMap mk, mv, mg;
+    const int BH = P.B * P.H;
+    if (!make_map(&mk, a_src, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dk, P.L, BH, 64, true) ||
+        !make_map(&mv, b_src, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dv, P.L, BH, 64, true))
+        return cudaErrorInvalidValue;
+    if (GATE == 1) {
+        if (!make_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, P.Dk, P.L, BH, P.Dk, false))
+            return cudaErrorInvalidValue;
+    } else {
+        mg = mk;
+    }
+    FwdArgs a{};
+    a.gh = GATE == 2 ? g : nullptr;
+    a.ig = ig;
+    a.seg_state = seg_state;
+    a.seg_gamma = seg_gamma;
+    a.status = status;
+    a.tiles_per_seg = tps;
+    a.nseg = nseg;
+    a.seg_offset = mode == 1 ? 0 : 1;
+    if (mode == 1) return launch_one<DK, DVT, GATE, 1>(mk, mk, mv, mg, a, P, nseg - 1, st);
+    return launch_one<DK, DVT, GATE, 2>(mk, mk, mv, mg, a, P, nseg - 1, st);
+}
+
 template <int DK, int DVT, int GATE>
 static cudaError_t run(const Dims& P, const void* q, const void* k, const void* v, const float* g,
                        const float* ig, const float* h0, void* o, float* hT, void* ws, cudaStream_t st) {
@@ -648,26 +688,41 @@ static cudaError_t run(const Dims& P, const void* q, const void* k, const void* 
     a.status = static_cast<int*>(ws);
     a.tiles_per_seg = pl.tiles_per_seg;
     a.nseg = pl.nseg;
+    a.seg_offset = 0;
     if (pl.nseg > 1) {
         char* w = static_cast<char*>(ws);
         size_t off = kStatusBytes;
-        a.seg_state = reinterpret_cast<float*>(w + off);
+        float* seg_state = reinterpret_cast<float*>(w + off);
         off = align_up(off + 4 * (size_t)BH * pl.nseg * P.Dk * P.Dv, 256);
-        a.seg_gamma = reinterpret_cast<float*>(w + off);
+        float* seg_gamma = reinterpret_cast<float*>(w + off);
         off = align_up(off + 4 * (size_t)BH * pl.nseg * P.Dk, 256);
-        a.sinit = reinterpret_cast<float*>(w + off);
-        // local end states of every segment but the last
-        Dims Ps = P;
-        cudaError_t e = launch_one<DK, DVT, GATE, 1>(mq, mk, mv, mg, a, Ps, pl.nseg - 1, st);
+        float* sinit = reinterpret_cast<float*>(w + off);
+        a.sinit = sinit;
+        cudaError_t e = state_run<DK, DVT, GATE>(P, 1, k, v, g, ig, pl.nseg, pl.tiles_per_seg, seg_state, seg_gamma,
+                                                 a.status, st);
         if (e != cudaSuccess) return e;
-        const long n = (long)BH * P.Dk * P.Dv;
-        GLA_LAUNCH("tc_seg_scan", st,
-                   k_seg_scan<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
-                       a.seg_state, a.seg_gamma, h0, const_cast<float*>(a.sinit), BH, P.Dk, P.Dv, pl.nseg));
-        e = cudaGetLastError();
+        e = seg_scan(P, pl.nseg, seg_state, seg_gamma, h0, sinit, st);
         if (e != cudaSuccess) return e;
     }
     return launch_one<DK, DVT, GATE, 0>(mq, mk, mv, mg, a, P, pl.nseg, st);
+}
+
+cudaError_t seg_scan(const Dims& P, int nseg, const float* seg_state, const float* seg_gamma, const float* h0,
+                     float* sinit, cudaStream_t st) {
+    const long n = (long)P.B * P.H * P.Dk * P.Dv;
+    GLA_LAUNCH("tc_seg_scan", st,
+               k_seg_scan<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(seg_state, seg_gamma, h0, sinit, P.B * P.H,
+                                                                       P.Dk, P.Dv, nseg));
+    return cudaGetLastError();
+}
+
+cudaError_t seg_rscan(const Dims& P, int nseg, const float* seg_state, const float* seg_gamma, const float* dhT,
+                      float* gend, cudaStream_t st) {
+    const long n = (long)P.B * P.H * P.Dk * P.Dv;
+    GLA_LAUNCH("tc_seg_rscan", st,
+               k_seg_rscan<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(seg_state, seg_gamma, dhT, gend, P.B * P.H,
+                                                                        P.Dk, P.Dv, nseg));
+    return cudaGetLastError();
 }
 
 template <int DK, int DVT>
@@ -678,6 +733,31 @@ static cudaError_t run_gate(const Dims& P, const void* q, const void* k, const v
         case GLA_GATE_PER_KEY: return run<DK, DVT, 1>(P, q, k, v, g, ig, h0, o, hT, ws, st);
         default: return run<DK, DVT, 2>(P, q, k, v, g, ig, h0, o, hT, ws, st);
     }
+}
+
+template <int DK, int DVT>
+static cudaError_t state_gate(const Dims& P, int mode, const void* a_src, const void* b_src, const float* g,
+                              const float* ig, int nseg, int tps, float* ss, float* sg, int* status, cudaStream_t st) {
+    switch (P.gate) {
+        case GLA_GATE_NONE: return state_run<DK, DVT, 0>(P, mode, a_src, b_src, g, ig, nseg, tps, ss, sg, status, st);
+        case GLA_GATE_PER_KEY: return state_run<DK, DVT, 1>(P, mode, a_src, b_src, g, ig, nseg, tps, ss, sg, status, st);
+        default: return state_run<DK, DVT, 2>(P, mode, a_src, b_src, g, ig, nseg, tps, ss, sg, status, st);
+    }
+}
+
+cudaError_t state_pass(const Dims& P, int mode, const void* a_src, const void* b_src, const float* g,
+                       const float* ig, int nseg, int tiles_per_seg, float* seg_state, float* seg_gamma, int* status,
+                       cudaStream_t st) {
+    const int dvt = pick_dvt(P);
+    if (P.Dk == 64) {
+        if (dvt == 128) return state_gate<64, 128>(P, mode, a_src, b_src, g, ig, nseg, tiles_per_seg, seg_state, seg_gamma, status, st);
+        return state_gate<64, 64>(P, mode, a_src, b_src, g, ig, nseg, tiles_per_seg, seg_state, seg_gamma, status, st);
+    }
+    if (P.Dk == 128) {
+        if (dvt == 128) return state_gate<128, 128>(P, mode, a_src, b_src, g, ig, nseg, tiles_per_seg, seg_state, seg_gamma, status, st);
+        return state_gate<128, 64>(P, mode, a_src, b_src, g, ig, nseg, tiles_per_seg, seg_state, seg_gamma, status, st);
+    }
+    return state_gate<256, 64>(P, mode, a_src, b_src, g, ig, nseg, tiles_per_seg, seg_state, seg_gamma, status, st);
 }
 
 cudaError_t fwd(const Dims& P, const void* q, const void* k, const void* v, const float* g, const float* ig,
