@@ -199,6 +199,15 @@ def dist_setup():
     return world, rank, local
 
 
+def max_over_ranks(value: float, device) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def base_line(w, args, world):
     return {"metric": "GLA chunkwise fwd/bwd tokens/s", "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
@@ -298,10 +307,7 @@ def main():
     clocks = sampler.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
     tokens = w.B * w.L * args.steps * world
     value = tokens / (total_ms / 1e3)
 
@@ -334,10 +340,7 @@ def main():
         s1.record()
         torch.cuda.synchronize()
         e_ms = s0.elapsed_time(s1)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e_ms, dev)
         h2d_step = h2d * (2 if w.backward else 1) + (sum(xh[n].numel() * xh[n].element_size() for n in ("dO",))
                                                      if w.backward else 0)
         e2e = {"value": tokens / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d_step),

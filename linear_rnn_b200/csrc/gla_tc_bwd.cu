@@ -16,7 +16,13 @@
 //                state MMA accumulates onto it, a TMEM pass applies e^Gamma) and bf16 in
 //                shared memory as the B operand of dO S^T.
 //   tc_bwd_dkdv  reverse tile walk per (b*h, segment); G in TMEM, bf16 G~ in shared memory.
-//   tc_bwd_dg    reverse cumulative sum of q*dq - k*dk, fp32.
+// dg in fp32 without a separate pass: the dq kernel writes the in-segment exclusive prefix
+// of q*dq (into the dg buffer) and its segment total; the dk/dv kernel forms the in-segment
+// reverse sum of k*dk and finishes dg_t = (total - prefix_t) - revsum_t + carry, where the
+// carry (everything after the segment, incl. the final-state term) is
+// sum_e G_end[d][e] S_end[d][e]: adding a constant to the log-gate at the segment's first
+// token scales the state entering it, so that sum is exactly the gradient of the
+// shifted cumulative decay.
 // Segment boundary states come from the forward state pass + scan; segment boundary
 // state gradients from the reverse state pass (gla_tc_fwd.cu, mode 2) + reverse scan.
 #include "gla_plans.h"
@@ -42,6 +48,9 @@ struct BwdArgs {
     float* di;            // [BH*L] or null
     float* dh0;           // [BH, Dk, Dv] or null
     float* hT_ws;         // final state (for the dg term) or null
+    float* dg;            // dg output; the dq kernel first stores there the in-segment
+                          // exclusive prefix of q*dq, the dk/dv kernel finishes it
+    float* tq;            // [BH, nseg, Dk] in-segment totals of q*dq
     int* status;
     int tiles_per_seg;
     int nseg;
@@ -68,14 +77,16 @@ constexpr uint32_t pow2cols(uint32_t n) { return n <= 32 ? 32 : n <= 64 ? 64 : n
 // ============================================================================ dq
 template <int DKB, int DV, int GATE>
 struct QCfg {
+    static constexpr uint32_t QB = GATE != 0 ? TR * DKB * 2 : 0;  // raw q (for q*dq)
     static constexpr uint32_t KB = TR * DKB * 2;
-    static constexpr uint32_t GB = GATE == 1 ? TR * DKB * 4 : 0;
+    static constexpr uint32_t GB = GATE != 0 ? TR * DKB * 4 : 0;  // g (per key), then q*dq scratch
     static constexpr uint32_t VB = TR * DV * 2;
     static constexpr uint32_t OB = TR * DV * 2;
-    static constexpr uint32_t STAGE = KB + GB + VB + OB;
+    static constexpr uint32_t STAGE = QB + KB + GB + VB + OB;
+    static constexpr uint32_t TXB = STAGE - (GATE == 1 ? 0 : GB); // bytes the copy engine writes
     static constexpr uint32_t SB = DKB * DV * 2;
     static constexpr uint32_t AB = TR * TR * 2;
-    static constexpr uint32_t SMALL = 256 + 4096 + 8 * DKB + 1024;
+    static constexpr uint32_t SMALL = 256 + 4096 + 8 * DKB + 1024 + 512;
     static constexpr int NS = (2 * STAGE + SB + AB + SMALL + 1024 <= 227 * 1024) ? 2 : 1;
     static constexpr uint32_t SMEM = NS * STAGE + SB + AB + SMALL + 1024;
     static constexpr uint32_t COL_R = DV;
@@ -88,8 +99,9 @@ struct QCfg {
 
 template <int DKB, int DV, int GATE>
 __global__ void __launch_bounds__(NT_B, 1)
-    k_tc_bwd_dq(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tg,
-                const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo, BwdArgs A, Dims P) {
+    k_tc_bwd_dq(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                const __grid_constant__ CUtensorMap tg, const __grid_constant__ CUtensorMap tv,
+                const __grid_constant__ CUtensorMap tdo, BwdArgs A, Dims P) {
     using C = QCfg<DKB, DV, GATE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -106,6 +118,8 @@ __global__ void __launch_bounds__(NT_B, 1)
     float* rowEi = rowE + TR;
     float* igs = rowEi + TR;
     float* ghs = igs + TR;
+    float* carry = ghs + TR;            // [DKB] running in-segment sum of q*dq per key dim
+    float* rows = carry + DKB;          // [64] per-row sums (per-head gate)
 
     const int bh = blockIdx.x, kb = blockIdx.y, z = blockIdx.z;
     const int d0 = kb * DKB;
@@ -124,6 +138,7 @@ __global__ void __launch_bounds__(NT_B, 1)
         mbar_init(bar_mma2, 1);
         mbar_fence_init();
     }
+    if (tid < DKB) carry[tid] = 0.f;
     if (warp == 0) tmem_alloc(tmem_slot, C::NCOL);
     tc_fence_before();
     __syncthreads();
@@ -160,12 +175,15 @@ __global__ void __launch_bounds__(NT_B, 1)
     auto issue_loads = [&](int i, int s) {
         uint8_t* st = sm + s * C::STAGE;
         const int t0 = (tile0 + i) * TR;
-        mbar_arrive_expect_tx(&bar_full[s], C::STAGE);
-        for (int cb = 0; cb < DKB / 64; ++cb) tma_load_3d(st + cb * BLK, &tk, d0 + cb * 64, t0, bh, &bar_full[s]);
-        if (GATE == 1) tma_load_3d(st + C::KB, &tg, d0, t0, bh, &bar_full[s]);
+        mbar_arrive_expect_tx(&bar_full[s], C::TXB);
+        for (int cb = 0; cb < DKB / 64; ++cb) {
+            if (GATE != 0) tma_load_3d(st + cb * BLK, &tq, d0 + cb * 64, t0, bh, &bar_full[s]);
+            tma_load_3d(st + C::QB + cb * BLK, &tk, d0 + cb * 64, t0, bh, &bar_full[s]);
+        }
+        if (GATE == 1) tma_load_3d(st + C::QB + C::KB, &tg, d0, t0, bh, &bar_full[s]);
         for (int vb = 0; vb < DV / 64; ++vb) {
-            tma_load_3d(st + C::KB + C::GB + vb * BLK, &tv, vb * 64, t0, bh, &bar_full[s]);
-            tma_load_3d(st + C::KB + C::GB + C::VB + vb * BLK, &tdo, vb * 64, t0, bh, &bar_full[s]);
+            tma_load_3d(st + C::QB + C::KB + C::GB + vb * BLK, &tv, vb * 64, t0, bh, &bar_full[s]);
+            tma_load_3d(st + C::QB + C::KB + C::GB + C::VB + vb * BLK, &tdo, vb * 64, t0, bh, &bar_full[s]);
         }
     };
     if (tid == 0)
@@ -175,9 +193,10 @@ __global__ void __launch_bounds__(NT_B, 1)
     for (int i = 0; i < ntiles; ++i) {
         const int s = i % C::NS;
         uint8_t* st = sm + s * C::STAGE;
-        uint8_t* sk = st;
-        float* sg = reinterpret_cast<float*>(st + C::KB);
-        uint8_t* sv = st + C::KB + C::GB;
+        uint8_t* sqr = st;
+        uint8_t* sk = st + C::QB;
+        float* sg = reinterpret_cast<float*>(st + C::QB + C::KB);
+        uint8_t* sv = st + C::QB + C::KB + C::GB;
         uint8_t* so = sv + C::VB;
         const int t0 = (tile0 + i) * TR;
         if (tid < TR) {
@@ -352,6 +371,68 @@ __global__ void __launch_bounds__(NT_B, 1)
                         f[j] = P.scale * eb * __uint_as_float(r[j]);
                     }
                     store16_bf16_global(A.dq + (rowbase + t0 + t) * P.Dk + d0 + c, f);
+                    if (GATE != 0)
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            sg[t * DKB + c + j] =
+                                __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sqr + sw128_off(t, c + j, BLK))) *
+                                f[j];
+                } else if (GATE != 0 && lane >= 16) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) sg[t * DKB + c + j] = 0.f;
+                }
+            }
+        }
+        // ---- in-segment exclusive prefix of q*dq (fp32) into the dg buffer
+        if (GATE != 0) {
+            __syncthreads();
+            if (GATE == 1) {
+                float ax = 0.f, ay = 0.f;
+                for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
+                    ax += sg[r * DKB + d];
+                    ay += sg[r * DKB + d + 1];
+                }
+                tot[rg * DKB + d] = ax;
+                tot[rg * DKB + d + 1] = ay;
+                __syncthreads();
+                float px = carry[d], py = carry[d + 1], Tx = 0.f, Ty = 0.f;
+                for (int r2 = 0; r2 < RG; ++r2) {
+                    if (r2 < rg) { px += tot[r2 * DKB + d]; py += tot[r2 * DKB + d + 1]; }
+                    Tx += tot[r2 * DKB + d];
+                    Ty += tot[r2 * DKB + d + 1];
+                }
+                for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
+                    if (t0 + r < P.L)
+                        *reinterpret_cast<float2*>(A.dg + (rowbase + t0 + r) * P.Dk + d0 + d) = make_float2(px, py);
+                    px += sg[r * DKB + d];
+                    py += sg[r * DKB + d + 1];
+                }
+                __syncthreads();
+                if (rg == 0) { carry[d] += Tx; carry[d + 1] += Ty; }
+            } else {
+                for (int j = 0; j < 8; ++j) {
+                    const int r = warp * 8 + j;
+                    float acc = 0.f;
+                    for (int dd = lane; dd < DKB; dd += 32) acc += sg[r * DKB + dd];
+                    for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+                    if (lane == 0) rows[r] = acc;
+                }
+                __syncthreads();
+                if (warp == 0) {  // exclusive scan over 64 rows, two per lane
+                    const float a0 = rows[2 * lane], a1 = rows[2 * lane + 1];
+                    float v = a0 + a1;
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const float n = __shfl_up_sync(0xffffffffu, v, off);
+                        if (lane >= off) v += n;
+                    }
+                    const float base = carry[0];
+                    const float e0 = base + v - a0 - a1, e1 = base + v - a1;
+                    if (t0 + 2 * lane < P.L) A.dg[rowbase + t0 + 2 * lane] = e0;
+                    if (t0 + 2 * lane + 1 < P.L) A.dg[rowbase + t0 + 2 * lane + 1] = e1;
+                    const float total = __shfl_sync(0xffffffffu, v, 31);
+                    __syncwarp();
+                    if (lane == 0) carry[0] = base + total;
                 }
             }
         }
@@ -361,6 +442,11 @@ __global__ void __launch_bounds__(NT_B, 1)
         if (tid == 0 && i + C::NS < ntiles) issue_loads(i + C::NS, s);
     }
 
+    if (!err) {
+        __syncthreads();
+        if (GATE == 1 && tid < DKB) A.tq[((long)bh * A.nseg + z) * P.Dk + d0 + tid] = carry[tid];
+        if (GATE == 2 && tid == 0) A.tq[(long)bh * A.nseg + z] = carry[0];
+    }
     if (err) {
         if (tid == 0) {
             atomicExch(A.status, kDevStatusTimeout);
@@ -394,13 +480,14 @@ template <int DK, int DV, int GATE>
 struct KVCfg {
     static constexpr uint32_t QB = TR * DK * 2;
     static constexpr uint32_t KB = TR * DK * 2;
-    static constexpr uint32_t GB = GATE == 1 ? TR * DK * 4 : 0;
+    static constexpr uint32_t GB = GATE != 0 ? TR * DK * 4 : 0;  // g (per key), then k*dk scratch
     static constexpr uint32_t VB = TR * DV * 2;
     static constexpr uint32_t OB = TR * DV * 2;
     static constexpr uint32_t STAGE = QB + KB + GB + VB + OB;
+    static constexpr uint32_t TXB = STAGE - (GATE == 1 ? 0 : GB);
     static constexpr uint32_t GTB = DK * DV * 2;
     static constexpr uint32_t AB = TR * TR * 2;
-    static constexpr uint32_t SMALL = 256 + 4096 + 8 * DK + 1024 + 512;
+    static constexpr uint32_t SMALL = 256 + 4096 + 4 * DK + 1024 + 512 + 16 * DK + 256 + 64;
     static constexpr int NS = (2 * STAGE + GTB + 2 * AB + SMALL + 1024 <= 227 * 1024) ? 2 : 1;
     static constexpr uint32_t SMEM = NS * STAGE + GTB + 2 * AB + SMALL + 1024;
     static constexpr uint32_t COL_R = DV;
@@ -436,6 +523,11 @@ __global__ void __launch_bounds__(NT_B, 1)
     float* igs = rowEi + TR;
     float* ghs = igs + TR;
     float* sdi = ghs + TR;        // [2][64]
+    float* cz = sdi + 2 * TR;     // [DK] in-segment q*dq total + carry from later segments
+    float* rk = cz + DK;          // [DK] running reverse sum of k*dk
+    float* red = rk + DK;         // [2][DK]
+    float* rows = red + 2 * DK;   // [64]
+    float* czs = rows + TR;       // [1] per-head: sum over key dims of cz
 
     const int bh = blockIdx.x, z = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2, qd = warp & 3;
@@ -466,13 +558,38 @@ __global__ void __launch_bounds__(NT_B, 1)
         const float* src = nullptr;
         if (z == A.nseg - 1) src = A.dhT ? A.dhT + ((long)bh * DK + srow) * P.Dv : nullptr;
         else src = A.gend + (((long)bh * A.nseg + z) * DK + srow) * P.Dv;
+        // dg at the segment's end: sum_e G_end[d][e] * S_end[d][e] (shift invariance of the
+        // cumulative log-decay), with S_end the forward state after the segment
+        const float* send = nullptr;
+        if (GATE != 0 && src) {
+            if (z < A.nseg - 1) send = A.sinit + (((long)bh * A.nseg + z + 1) * DK + srow) * P.Dv;
+            else send = A.hT_ws ? A.hT_ws + ((long)bh * DK + srow) * P.Dv : nullptr;
+        }
+        float part = 0.f;
         for (int c = wg * C::HC; c < (wg + 1) * C::HC; c += 16) {
             uint32_t r[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) r[j] = __float_as_uint((src && srow_ok) ? src[c + j] : 0.f);
+            for (int j = 0; j < 16; ++j) {
+                const float gv = (src && srow_ok) ? src[c + j] : 0.f;
+                r[j] = __float_as_uint(gv);
+                if (send && srow_ok) part += gv * send[c + j];
+            }
             tmem_st16(tlane + c, r);
         }
         tmem_wait_st();
+        if (srow_ok) red[wg * DK + srow] = part;
+        if (tid < DK) rk[tid] = 0.f;
+        __syncthreads();
+        if (tid < DK) {
+            const float tqv = GATE == 1 ? A.tq[((long)bh * A.nseg + z) * DK + tid] : 0.f;
+            cz[tid] = red[tid] + red[DK + tid] + tqv;
+        }
+        __syncthreads();
+        if (GATE == 2 && tid == 0) {
+            float sacc = A.tq[(long)bh * A.nseg + z];
+            for (int dd = 0; dd < DK; ++dd) sacc += cz[dd];
+            czs[0] = sacc;
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -481,7 +598,7 @@ __global__ void __launch_bounds__(NT_B, 1)
     auto issue_loads = [&](int i, int s) {
         uint8_t* st = sm + s * C::STAGE;
         const int t0 = tile_at(i) * TR;
-        mbar_arrive_expect_tx(&bar_full[s], C::STAGE);
+        mbar_arrive_expect_tx(&bar_full[s], C::TXB);
         for (int cb = 0; cb < DK / 64; ++cb) {
             tma_load_3d(st + cb * BLK, &tq, cb * 64, t0, bh, &bar_full[s]);
             tma_load_3d(st + C::QB + cb * BLK, &tk, cb * 64, t0, bh, &bar_full[s]);
@@ -703,9 +820,14 @@ __global__ void __launch_bounds__(NT_B, 1)
                         f[j] = iv * em * x;
                         const __nv_bfloat16 kt =
                             *reinterpret_cast<const __nv_bfloat16*>(sk + sw128_off(srw, c + j, BLK));
-                        dsum += __bfloat162float(kt) * x;
+                        const float kx = __bfloat162float(kt) * x;   // k' dk' = k~ X
+                        dsum += kx;
+                        if (GATE != 0) sg[srw * DK + c + j] = kx;
                     }
                     store16_bf16_global(A.dk + (rowbase + t0 + srw) * DK + c, f);
+                } else if (GATE != 0 && lane < 16) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) sg[srw * DK + c + j] = 0.f;
                 }
             }
             if (lane < 16) sdi[wg * TR + srw] = dsum;
@@ -725,6 +847,61 @@ __global__ void __launch_bounds__(NT_B, 1)
         __syncthreads();
         tc_fence_after();
         if (A.di && tid < TR && t0 + tid < P.L) A.di[rowbase + t0 + tid] = (sdi[tid] + sdi[TR + tid]) / igs[tid];
+        // ---- dg = (in-segment q*dq total - exclusive prefix) - reverse sum of k*dk + carry
+        if (GATE == 1) {
+            float ax = 0.f, ay = 0.f;
+            for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
+                ax += sg[r * DK + d];
+                ay += sg[r * DK + d + 1];
+            }
+            tot[rg * DK + d] = ax;
+            tot[rg * DK + d + 1] = ay;
+            __syncthreads();
+            float sx = rk[d], sy = rk[d + 1], Tx = 0.f, Ty = 0.f;
+            for (int r2 = 0; r2 < RG; ++r2) {
+                if (r2 > rg) { sx += tot[r2 * DK + d]; sy += tot[r2 * DK + d + 1]; }
+                Tx += tot[r2 * DK + d];
+                Ty += tot[r2 * DK + d + 1];
+            }
+            const float cx = cz[d], cy = cz[d + 1];
+            for (int r = (rg + 1) * RPG - 1; r >= rg * RPG; --r) {
+                sx += sg[r * DK + d];
+                sy += sg[r * DK + d + 1];
+                if (t0 + r < P.L) {
+                    float2* gp = reinterpret_cast<float2*>(A.dg + (rowbase + t0 + r) * DK + d);
+                    const float2 pq = *gp;
+                    *gp = make_float2(cx - pq.x - sx, cy - pq.y - sy);
+                }
+            }
+            __syncthreads();
+            if (rg == 0) { rk[d] += Tx; rk[d + 1] += Ty; }
+        } else if (GATE == 2) {
+            for (int j = 0; j < 8; ++j) {
+                const int r = warp * 8 + j;
+                float acc = 0.f;
+                for (int dd = lane; dd < DK; dd += 32) acc += sg[r * DK + dd];
+                for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+                if (lane == 0) rows[r] = acc;
+            }
+            __syncthreads();
+            if (warp == 0) {  // reverse inclusive scan over 64 rows, two per lane
+                const float a0 = rows[2 * lane], a1 = rows[2 * lane + 1];
+                float v = a0 + a1;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float n = __shfl_down_sync(0xffffffffu, v, off);
+                    if (lane + off < 32) v += n;
+                }
+                const float base = rk[0], cc = czs[0];
+                const float s0 = base + v, s1 = base + v - a0;
+                const int ta = t0 + 2 * lane;
+                if (ta < P.L) A.dg[rowbase + ta] = cc - A.dg[rowbase + ta] - s0;
+                if (ta + 1 < P.L) A.dg[rowbase + ta + 1] = cc - A.dg[rowbase + ta + 1] - s1;
+                const float total = __shfl_sync(0xffffffffu, v, 0);
+                __syncwarp();
+                if (lane == 0) rk[0] = base + total;
+            }
+        }
         if (tid == 0 && i + C::NS < ntiles) issue_loads(i + C::NS, s);
     }
 
@@ -753,124 +930,6 @@ __global__ void __launch_bounds__(NT_B, 1)
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, C::NCOL);
-}
-
-// ============================================================================ dg
-// Per-key gates: block (b*h, 64 key dims); 256 threads = 64 columns x 4 row groups of 16.
-// Walks 64-token tiles from the end: dB = q dq - k dk, reverse cumsum with a carry.
-__global__ void __launch_bounds__(256) k_tc_bwd_dg_key(const __nv_bfloat16* __restrict__ q,
-                                                       const __nv_bfloat16* __restrict__ dq,
-                                                       const __nv_bfloat16* __restrict__ k,
-                                                       const __nv_bfloat16* __restrict__ dk,
-                                                       const float* __restrict__ dhT, const float* __restrict__ hT,
-                                                       float* __restrict__ dg, Dims P) {
-    const long bh = blockIdx.x;
-    const int col = threadIdx.x & 63, rg = threadIdx.x >> 6;
-    const int d = blockIdx.y * 64 + col;
-    __shared__ float tots[4][64];
-    float carry = 0.f;
-    if (dhT) {
-        const float* a = dhT + (bh * P.Dk + d) * (long)P.Dv;
-        const float* h = hT + (bh * P.Dk + d) * (long)P.Dv;
-        for (int e = 0; e < P.Dv; ++e) carry += a[e] * h[e];
-    }
-    const int ntiles = cdiv(P.L, TR);
-    for (int ti = ntiles - 1; ti >= 0; --ti) {
-        float x[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const int t = ti * TR + rg * 16 + j;
-            float v = 0.f;
-            if (t < P.L) {
-                const long idx = (bh * P.L + t) * P.Dk + d;
-                v = __bfloat162float(q[idx]) * __bfloat162float(dq[idx]) -
-                    __bfloat162float(k[idx]) * __bfloat162float(dk[idx]);
-            }
-            x[j] = v;
-        }
-        float s = 0.f;
-#pragma unroll
-        for (int j = 15; j >= 0; --j) {
-            s += x[j];
-            x[j] = s;
-        }
-        tots[rg][col] = s;
-        __syncthreads();
-        float later = carry;
-        for (int r2 = rg + 1; r2 < 4; ++r2) later += tots[r2][col];
-        float tile_total = 0.f;
-#pragma unroll
-        for (int r2 = 0; r2 < 4; ++r2) tile_total += tots[r2][col];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const int t = ti * TR + rg * 16 + j;
-            if (t < P.L) dg[(bh * P.L + t) * P.Dk + d] = x[j] + later;
-        }
-        carry += tile_total;
-        __syncthreads();
-    }
-}
-
-// Per-head gates: block per b*h; dB summed over key dims per token, then the scalar
-// reverse cumsum. Warp w handles tokens 8w..8w+7 of each tile.
-__global__ void __launch_bounds__(256) k_tc_bwd_dg_head(const __nv_bfloat16* __restrict__ q,
-                                                        const __nv_bfloat16* __restrict__ dq,
-                                                        const __nv_bfloat16* __restrict__ k,
-                                                        const __nv_bfloat16* __restrict__ dk,
-                                                        const float* __restrict__ dhT, const float* __restrict__ hT,
-                                                        float* __restrict__ dg, Dims P) {
-    const long bh = blockIdx.x;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    __shared__ float rows[TR];
-    __shared__ float red[8];
-    float part = 0.f;
-    if (dhT) {
-        const long n = (long)P.Dk * P.Dv;
-        for (long i = threadIdx.x; i < n; i += blockDim.x) part += dhT[bh * n + i] * hT[bh * n + i];
-    }
-    for (int off = 16; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-    if (lane == 0) red[warp] = part;
-    __syncthreads();
-    float carry = 0.f;
-    for (int w = 0; w < 8; ++w) carry += red[w];
-    const int ntiles = cdiv(P.L, TR);
-    for (int ti = ntiles - 1; ti >= 0; --ti) {
-        for (int j = 0; j < 8; ++j) {
-            const int r = warp * 8 + j, t = ti * TR + r;
-            float sacc = 0.f;
-            if (t < P.L)
-                for (int dd = lane; dd < P.Dk; dd += 32) {
-                    const long idx = (bh * P.L + t) * P.Dk + dd;
-                    sacc += __bfloat162float(q[idx]) * __bfloat162float(dq[idx]) -
-                            __bfloat162float(k[idx]) * __bfloat162float(dk[idx]);
-                }
-            for (int off = 16; off >= 1; off >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, off);
-            if (lane == 0) rows[r] = sacc;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            // reverse inclusive scan over 64 rows, two per lane
-            const float a0 = rows[2 * lane], a1 = rows[2 * lane + 1];
-            float v = a0 + a1;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float n = __shfl_down_sync(0xffffffffu, v, off);
-                if (lane + off < 32) v += n;
-            }
-            const float s0 = v + carry, s1 = v - a0 + carry;
-            const int t0 = ti * TR + 2 * lane;
-            if (t0 < P.L) dg[bh * P.L + t0] = s0;
-            if (t0 + 1 < P.L) dg[bh * P.L + t0 + 1] = s1;
-            const float total = __shfl_sync(0xffffffffu, v, 0);
-            carry += total;
-        }
-        carry = __shfl_sync(0xffffffffu, carry, 0);
-        __syncthreads();
-        if (threadIdx.x == 0) red[0] = carry;
-        __syncthreads();
-        carry = red[0];
-        __syncthreads();
-    }
 }
 
 // ============================================================================ host side
@@ -902,7 +961,7 @@ bool bwd_supports(const Dims& P) {
 }
 
 struct BwdWs {
-    float *seg_state, *seg_gamma, *sinit, *gend, *hT;
+    float *seg_state, *seg_gamma, *sinit, *gend, *hT, *tq;
     size_t total;
 };
 
@@ -913,6 +972,8 @@ static BwdWs bwd_layout(const Dims& P, char* base) {
     size_t off = kStatusBytes;
     w.hT = reinterpret_cast<float*>(base + off);
     off = align_up(off + st, 256);
+    w.tq = reinterpret_cast<float*>(base + off);
+    off = align_up(off + 4 * BH * (size_t)pl.nseg * P.Dk, 256);
     if (pl.nseg > 1) {
         w.seg_state = reinterpret_cast<float*>(base + off);
         off = align_up(off + st * pl.nseg, 256);
@@ -930,8 +991,9 @@ static BwdWs bwd_layout(const Dims& P, char* base) {
 size_t bwd_workspace_bytes(const Dims& P) { return bwd_layout(P, nullptr).total; }
 
 template <int DKB, int DV, int GATE>
-static cudaError_t launch_dq(const Dims& P, const BwdPlan& pl, const CUtensorMap& mk, const CUtensorMap& mg,
-                             const CUtensorMap& mv, const CUtensorMap& mo, const BwdArgs& a, cudaStream_t st) {
+static cudaError_t launch_dq(const Dims& P, const BwdPlan& pl, const CUtensorMap& mq, const CUtensorMap& mk,
+                             const CUtensorMap& mg, const CUtensorMap& mv, const CUtensorMap& mo, const BwdArgs& a,
+                             cudaStream_t st) {
     using C = QCfg<DKB, DV, GATE>;
     auto kern = k_tc_bwd_dq<DKB, DV, GATE>;
     static bool attr = false;
@@ -941,7 +1003,7 @@ static cudaError_t launch_dq(const Dims& P, const BwdPlan& pl, const CUtensorMap
         attr = true;
     }
     dim3 grid(P.B * P.H, P.Dk / DKB, pl.nseg);
-    GLA_LAUNCH("tc_bwd_dq", st, kern<<<grid, NT_B, C::SMEM, st>>>(mk, mg, mv, mo, a, P));
+    GLA_LAUNCH("tc_bwd_dq", st, kern<<<grid, NT_B, C::SMEM, st>>>(mq, mk, mg, mv, mo, a, P));
     return cudaGetLastError();
 }
 
@@ -1005,10 +1067,12 @@ static cudaError_t run_bwd(const Dims& P, const void* q, const void* k, const vo
     a.di = di;
     a.dh0 = dh0;
     a.hT_ws = (dhT && GATE != 0) ? w.hT : nullptr;
+    a.dg = dg;
+    a.tq = w.tq;
     a.status = status;
     a.tiles_per_seg = pl.tiles_per_seg;
     a.nseg = pl.nseg;
-    e = launch_dq<DKB, DV, GATE>(P, pl, mk, mgb, mv, mo, a, st);
+    e = launch_dq<DKB, DV, GATE>(P, pl, mq, mk, mgb, mv, mo, a, st);
     if (e != cudaSuccess) return e;
     if (pl.nseg > 1) {
         e = state_pass(P, 2, q, dO, g, ig, pl.nseg, pl.tiles_per_seg, w.seg_state, w.seg_gamma, status, st);
@@ -1018,17 +1082,6 @@ static cudaError_t run_bwd(const Dims& P, const void* q, const void* k, const vo
     }
     e = launch_dkdv<DK, DV, GATE>(P, pl, mq, mk, mg, mv, mo, a, st);
     if (e != cudaSuccess) return e;
-    if (GATE == 1) {
-        GLA_LAUNCH("tc_bwd_dg", st,
-                   k_tc_bwd_dg_key<<<dim3(BH, P.Dk / 64), 256, 0, st>>>(
-                       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dq),
-                       static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(dk), dhT, w.hT, dg, P));
-    } else if (GATE == 2) {
-        GLA_LAUNCH("tc_bwd_dg", st,
-                   k_tc_bwd_dg_head<<<BH, 256, 0, st>>>(
-                       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dq),
-                       static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(dk), dhT, w.hT, dg, P));
-    }
     return cudaGetLastError();
 }
 

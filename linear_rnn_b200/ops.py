@@ -71,6 +71,21 @@ def _to_dev(t: Optional[torch.Tensor], device: torch.device) -> Optional[torch.T
     return t.to(device, non_blocking=True)
 
 
+def _to_host(tensors):
+    """Copy device results into pinned host tensors (asynchronously on the current
+    stream), then wait for the stream once."""
+    out = []
+    for t in tensors:
+        if t is None:
+            out.append(None)
+            continue
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t, non_blocking=True)
+        out.append(h)
+    torch.cuda.current_stream().synchronize()
+    return out
+
+
 def _check(status: int, where: str):
     if status != _lib.GLA_OK:
         raise GlaError(status, where)
@@ -103,8 +118,7 @@ def gla_fwd(q, k, v, g=None, igate=None, h0=None, *, scale: Optional[float] = No
                           _ptr(o), _ptr(hT), _ptr(ws), ws.numel() * ws.element_size(), _stream_handle(device))
     _check(st, "gla_fwd")
     if host:
-        o = o.cpu()
-        hT = hT.cpu() if hT is not None else None
+        o, hT = _to_host([o, hT])
     return o, hT
 
 
@@ -134,7 +148,8 @@ def gla_bwd(q, k, v, g, igate, h0, dO, dhT=None, *, scale: Optional[float] = Non
     _check(st, "gla_bwd")
     out = {"dq": dq, "dk": dk, "dv": dv, "dg": dg, "di": di, "dh0": dh0}
     if host:
-        out = {n: (t.cpu() if t is not None else None) for n, t in out.items()}
+        names = list(out)
+        out = dict(zip(names, _to_host([out[n] for n in names])))
     return out
 
 
