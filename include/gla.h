@@ -123,6 +123,10 @@ GLA_API const char* gla_status_string(gla_status s);
  * device-side wait gave up; GLA_ERR_CUDA if the synchronisation itself failed. */
 GLA_API gla_status gla_check_device_status(void* ws, void* stream);
 
+/* Text of the CUDA error behind the calling thread's last GLA_ERR_CUDA (where it happened,
+ * the CUDA error name and description); "no error" if there was none. Never NULL. */
+GLA_API const char* gla_last_error_detail(void);
+
 /* Library version as 10000*major + 100*minor + patch. */
 GLA_API int gla_version(void);
 

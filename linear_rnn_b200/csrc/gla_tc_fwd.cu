@@ -36,6 +36,22 @@ namespace tc {
 using namespace sm100;
 
 
+// Thread roles: warps [0, 4*NEWG) run the epilogues (P, state, output), warps
+// [4*NEWG, 4*(NEWG+NTWG)) transform tiles in place, warp W_MMA issues the tcgen05 MMAs
+// and warp W_TMA the TMA loads. They hand tiles to each other through mbarriers: the
+// transform runs up to two tiles ahead, the MMAs of tile i+1 overlap the epilogues of
+// tile i (two TMEM accumulator buffers). Epilogue warp w reads TMEM lane quadrant w % 4;
+// each epilogue warpgroup owns DVT/NEWG state columns.
+constexpr int NEWG = 2;
+constexpr int NTWG = 2;
+constexpr int NEP = NEWG * 128;
+constexpr int NTRF = NTWG * 128;
+constexpr int W_MMA = (NEP + NTRF) / 32;
+constexpr int W_TMA = W_MMA + 1;
+constexpr int NTHR_WS = NEP + NTRF + 64;
+constexpr int BAR_EP = 1;   // named barrier of the epilogue threads
+constexpr int BAR_TR = 2;   // named barrier of the transform threads
+
 template <int DK, int DVT, int GATE, int MODE>
 struct Cfg {
     // MODE 0: output pass (q, k, g, v). MODE 1: state-only pass (k, g, v).
@@ -47,7 +63,7 @@ struct Cfg {
     static constexpr uint32_t STAGE = QB + KB + GB + VB;
     static constexpr uint32_t PB = MODE == 0 ? 2 * TR * TR * 2 : 0;   // P, double-buffered
     static constexpr uint32_t SB = MODE == 0 ? DK * DVT * 2 : 0;      // bf16 state
-    static constexpr uint32_t SMALL = 256 + 4096 + 16 * DK + 1024;
+    static constexpr uint32_t SMALL = 256 + 2048 + 16 * DK + 1024;
     static constexpr int NS = (2 * STAGE + PB + SB + SMALL + 1024 <= 227 * 1024) ? 2 : 1;
     static constexpr uint32_t SMEM = NS * STAGE + PB + SB + SMALL + 1024;
     static constexpr int NH = DK == 256 ? 2 : 1;            // M=128 halves of the state
@@ -56,11 +72,13 @@ struct Cfg {
     static constexpr uint32_t BUF_USED = COL_S + NH * DVT;
     static constexpr uint32_t BUFCOLS = BUF_USED <= 32 ? 32 : BUF_USED <= 64 ? 64 : BUF_USED <= 128 ? 128 : 256;
     static constexpr uint32_t NCOL = 2 * BUFCOLS;            // two accumulator buffers
-    static constexpr int HALF = DVT / 4;                     // state columns per compute warpgroup
+    static constexpr int HALF = DVT / NEWG;                  // state columns per epilogue warpgroup
+    static constexpr int PCOLS = TR / NEWG;                  // P columns per epilogue warpgroup
     static_assert(STAGE % 1024 == 0, "stage alignment");
     static_assert(SMEM <= 227 * 1024, "shared memory");
-    static_assert(HALF % 16 == 0, "column chunks");
+    static_assert(HALF % 16 == 0 && PCOLS % 16 == 0, "column chunks");
     static_assert(BUF_USED <= 256 && NCOL <= 512, "tensor memory");
+    static_assert((DK / 2) <= NTRF && (TR * (DK / 2)) % NTRF == 0, "transform mapping");
 };
 
 struct FwdArgs {
@@ -78,19 +96,8 @@ struct FwdArgs {
     int seg_offset;       // segment index = blockIdx.z + seg_offset
 };
 
-// Thread roles: warps 0-15 (four warpgroups) transform tiles and run the epilogues; warp 16
-// issues the tcgen05 MMAs; warp 17 issues the TMA loads. They hand tiles to each other
-// through mbarriers, so the transform of tile i+1 runs while the tensor core works on
-// tile i, and the epilogues of tile i overlap the MMAs of tile i+1 (two TMEM buffers).
-// Each compute warpgroup owns a quarter of the state columns; warp w reads TMEM lane
-// quadrant w % 4.
-constexpr int NCOMP = 512;
-constexpr int NCWG = NCOMP / 128;
-constexpr int NTHR_WS = NCOMP + 64;
-constexpr int BAR_COMP = 1;   // named barrier of the 256 compute threads
-
 template <int DK, int DVT, int GATE, int MODE>
-__global__ void __launch_bounds__(NTHR_WS, 1)
+__global__ void __maxnreg__(112)
     k_tc_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
              const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg, FwdArgs A, Dims P) {
     using C = Cfg<DK, DVT, GATE, MODE>;
@@ -107,15 +114,17 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     uint64_t* bar_mma2 = bars + 8;     // [2] P V done
     uint64_t* bar_pready = bars + 10;  // [2] P written
     uint64_t* bar_tfree = bars + 12;   // [2] TMEM buffer read out
-    uint64_t* bar_sready = bars + 14;  // bf16 state of the last tile written
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 128);
-    volatile int* abortp = reinterpret_cast<volatile int*>(small + 132);
-    int* n_issued = reinterpret_cast<int*>(small + 136);
-    int* n_consumed = reinterpret_cast<int*>(small + 140);
-    int* n_mma1 = reinterpret_cast<int*>(small + 144);
-    int* n_mma2 = reinterpret_cast<int*>(small + 148);
-    float* tot = reinterpret_cast<float*>(small + 256);      // [1024] cumsum group totals
-    float* gamb = tot + 1024;                                // [2][DK] e^Gamma per buffer
+    uint64_t* bar_gfree = bars + 14;   // [2] e^Gamma buffer read by the state epilogue
+    uint64_t* bar_sready = bars + 16;  // bf16 state of the last tile written
+    constexpr int NBARS = 17;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 160);
+    volatile int* abortp = reinterpret_cast<volatile int*>(small + 164);
+    int* n_issued = reinterpret_cast<int*>(small + 168);
+    int* n_consumed = reinterpret_cast<int*>(small + 172);
+    int* n_mma1 = reinterpret_cast<int*>(small + 176);
+    int* n_mma2 = reinterpret_cast<int*>(small + 180);
+    float* tot = reinterpret_cast<float*>(small + 256);      // [512] cumsum group totals
+    float* gamb = tot + 512;                                 // [2][DK] e^Gamma per buffer
     float* gamlb = gamb + 2 * DK;                            // [2][DK] Gamma per buffer
     float* rowE = gamlb + 2 * DK;                            // [64] e^b   (per-head gate)
     float* rowEi = rowE + TR;                                // [64] e^-b
@@ -124,16 +133,18 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
 
     const int bh = blockIdx.x, vt = blockIdx.y, z = blockIdx.z + A.seg_offset;
     const int e0 = vt * DVT;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = (warp >> 2) & 3, qd = warp & 3;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wg = warp >> 2, qd = warp & 3;   // meaningful for the epilogue warps
     const int ntiles_all = cdiv(P.L, TR);
     const int tile0 = z * A.tiles_per_seg;
     const int ntiles = min(ntiles_all, tile0 + A.tiles_per_seg) - tile0;
     const long rowbase = (long)bh * P.L;
     // the j-th tile this CTA processes (MODE 2 walks its segment backwards)
     auto tile_at = [&](int j) { return MODE == 2 ? tile0 + ntiles - 1 - j : tile0 + j; };
+    const bool is_ep = tid < NEP;
 
     if (tid == 0) {
-        for (int j = 0; j < 15; ++j) mbar_init(&bars[j], 1);
+        for (int j = 0; j < NBARS; ++j) mbar_init(&bars[j], 1);
         *abortp = 0;
         *n_issued = 0;
         *n_consumed = 0;
@@ -143,11 +154,11 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     }
     if (warp == 0) tmem_alloc(tmem_slot, C::NCOL);
 
-    // ---- compute threads: state registers (rows d, HALF columns of the Dv tile)
+    // ---- epilogue threads: state registers (rows d, HALF columns of the Dv tile)
     const bool srow_ok = (DK != 64) || (lane < 16);
     float Sreg[C::NH][C::HALF];
     float glog[C::NH];
-    if (tid < NCOMP) {
+    if (is_ep) {
 #pragma unroll
         for (int h = 0; h < C::NH; ++h) {
             const int d = (DK == 64 ? 16 * qd + (lane & 15) : 32 * qd + lane) + 128 * h;
@@ -171,7 +182,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
 
-    if (warp == NCOMP / 32 + 1) {
+    if (warp == W_TMA) {
         // ================================================================ TMA producer
         if (lane == 0) {
             if (MODE == 0) tma_prefetch_desc(&tq);
@@ -195,44 +206,47 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 *n_issued = j + 1;
             }
         }
-    } else if (warp == NCOMP / 32) {
+    } else if (warp == W_MMA) {
         // ================================================================ MMA issuer
         if (lane == 0) {
+            const uint32_t idA = idesc_bf16(64, 64, 0, 0);
+            const uint32_t idO = idesc_bf16(64, DVT, 0, 1);
+            const uint32_t idS = idesc_bf16(C::MS, DVT, 1, 1);
+            const uint64_t dS0 = sw128_desc(smem_u32(sS), DK * 128, 1024);
             for (int i = 0; i < ntiles; ++i) {
                 const int s = i % C::NS, b = i & 1;
                 if (!mbar_wait_abort(&bar_trans[s], (i / C::NS) & 1, abortp)) break;
                 if (i >= 2 && !mbar_wait_abort(&bar_tfree[b], ((i >> 1) - 1) & 1, abortp)) break;
                 tc_fence_after();
                 uint8_t* st = sm + s * C::STAGE;
-                const uint32_t qa = smem_u32(st), ka = smem_u32(st + C::QB), va = smem_u32(st + C::QB + C::KB + C::GB);
+                // descriptors of the stage's tiles; K steps advance the 16-byte start field
+                const uint64_t dQ = sw128_desc(smem_u32(st), 16, 1024);
+                const uint64_t dKk = sw128_desc(smem_u32(st + C::QB), 16, 1024);       // k~, K-major
+                const uint64_t dKm = sw128_desc(smem_u32(st + C::QB), BLK, 1024);      // k~, MN-major
+                const uint64_t dV = sw128_desc(smem_u32(st + C::QB + C::KB + C::GB), BLK, 1024);
                 const uint32_t tb = tbase + b * C::BUFCOLS;
                 if (MODE == 0) {
-                    const uint32_t idA = idesc_bf16(64, 64, 0, 0);
 #pragma unroll
                     for (int kk = 0; kk < DK / 16; ++kk) {
-                        const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
-                        mma_bf16(tb, sw128_desc(qa + koff, 16, 1024), sw128_desc(ka + koff, 16, 1024), idA, kk > 0);
+                        const uint64_t ko = ((kk >> 2) * BLK + (kk & 3) * 32) >> 4;
+                        mma_bf16(tb, dQ + ko, dKk + ko, idA, kk > 0);
                     }
                 }
-                const uint32_t idS = idesc_bf16(C::MS, DVT, 1, 1);
 #pragma unroll
                 for (int h = 0; h < C::NH; ++h)
 #pragma unroll
                     for (int ks = 0; ks < TR / 16; ++ks)
-                        mma_bf16(tb + C::COL_S + h * DVT, sw128_desc(ka + h * 2 * BLK + ks * 2048, BLK, 1024),
-                                 sw128_desc(va + ks * 2048, BLK, 1024), idS, ks > 0);
+                        mma_bf16(tb + C::COL_S + h * DVT, dKm + ((h * 2 * BLK + ks * 2048) >> 4),
+                                 dV + ((ks * 2048) >> 4), idS, ks > 0);
                 if (MODE == 0) {
                     if (i >= 1) {
                         if (!mbar_wait_abort(bar_sready, (i - 1) & 1, abortp)) break;
                         tc_fence_after();
                     }
-                    const uint32_t sa = smem_u32(sS);
-                    const uint32_t idO = idesc_bf16(64, DVT, 0, 1);
 #pragma unroll
                     for (int kk = 0; kk < DK / 16; ++kk) {
-                        const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
-                        mma_bf16(tb + (16u << 16), sw128_desc(qa + koff, 16, 1024),
-                                 sw128_desc(sa + kk * 2048, DK * 128, 1024), idO, kk > 0);
+                        const uint64_t ko = ((kk >> 2) * BLK + (kk & 3) * 32) >> 4;
+                        mma_bf16(tb + (16u << 16), dQ + ko, dS0 + ((kk * 2048) >> 4), idO, kk > 0);
                     }
                 }
                 mma_commit(&bar_mma1[b]);
@@ -240,23 +254,23 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 if (MODE == 0) {
                     if (!mbar_wait_abort(&bar_pready[b], (i >> 1) & 1, abortp)) break;
                     tc_fence_after();
-                    const uint32_t pa = smem_u32(sPb + b * (TR * TR * 2));
-                    const uint32_t idO = idesc_bf16(64, DVT, 0, 1);
+                    const uint64_t dP = sw128_desc(smem_u32(sPb + b * (TR * TR * 2)), 16, 1024);
 #pragma unroll
                     for (int ks = 0; ks < TR / 16; ++ks)
-                        mma_bf16(tb + (16u << 16), sw128_desc(pa + ks * 32, 16, 1024),
-                                 sw128_desc(va + ks * 2048, BLK, 1024), idO, 1);
+                        mma_bf16(tb + (16u << 16), dP + ((ks * 32) >> 4), dV + ((ks * 2048) >> 4), idO, 1);
                     mma_commit(&bar_mma2[b]);
                     *n_mma2 = i + 1;
                 }
                 if (i + C::NS < ntiles) mma_commit(&bar_empty[s]);
             }
         }
-    } else {
-        // ================================================================ compute warpgroups
-        const int ctid = tid;  // 0..NCOMP-1
-        // Transform tile j in place: q~ = q e^b, k~ = i k e^-b; e^Gamma into buffer j&1.
-        auto transform = [&](int j) -> bool {
+    } else if (!is_ep) {
+        // ================================================================ transform warpgroups
+        const int ttid = tid - NEP;
+        const int twarp = ttid >> 5;
+        constexpr int NP = DK / 2, RG = NTRF / NP, RPG = TR / RG;
+        const int cp = ttid % NP, rg = ttid / NP, d = 2 * cp;
+        for (int j = 0; j < ntiles; ++j) {
             const int s = j % C::NS, b = j & 1;
             uint8_t* st = sm + s * C::STAGE;
             uint8_t* sq = st;
@@ -265,18 +279,18 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
             float* gam = gamb + b * DK;
             float* gaml = gamlb + b * DK;
             const int t0 = tile_at(j) * TR;
-            if (ctid < TR) {
-                const int t = t0 + ctid;
-                igs[ctid] = (A.ig && t < P.L) ? A.ig[rowbase + t] : 1.f;
-                if (GATE == 2) ghs[ctid] = (t < P.L) ? A.gh[rowbase + t] : 0.f;
+            if (ttid < TR) {
+                const int t = t0 + ttid;
+                igs[ttid] = (A.ig && t < P.L) ? A.ig[rowbase + t] : 1.f;
+                if (GATE == 2) ghs[ttid] = (t < P.L) ? A.gh[rowbase + t] : 0.f;
             }
-            const bool ok = mbar_wait_abort(&bar_full[s], (j / C::NS) & 1, abortp);
-            if (!named_bar_and(BAR_COMP, NCOMP, ok)) return false;
-            if (ctid == 0) *n_consumed = j + 1;
-            constexpr int NP = DK / 2, RG = NCOMP / NP, RPG = TR / RG;
-            const int cp = ctid % NP, rg = ctid / NP, d = 2 * cp;
+            bool ok = mbar_wait_abort(&bar_full[s], (j / C::NS) & 1, abortp);
+            if (ok && j >= 2) ok = mbar_wait_abort(&bar_gfree[b], ((j >> 1) - 1) & 1, abortp);
+            if (!named_bar_and(BAR_TR, NTRF, ok)) break;
+            if (ttid == 0) *n_consumed = j + 1;
             if (GATE == 1) {
                 float ax = 0.f, ay = 0.f;
+#pragma unroll 4
                 for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
                     const float2 gv = *reinterpret_cast<const float2*>(sg + r * DK + d);
                     ax += gv.x;
@@ -285,7 +299,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 tot[rg * DK + d] = ax;
                 tot[rg * DK + d + 1] = ay;
             } else if (GATE == 2) {
-                if (warp == 0) {  // warp scan over 64 rows, two rows per lane
+                if (twarp == 0) {  // warp scan over 64 rows, two rows per lane
                     const float g0 = ghs[2 * lane], g1 = ghs[2 * lane + 1];
                     float v = g0 + g1;
 #pragma unroll
@@ -305,10 +319,11 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     }
                 }
             }
-            named_bar_sync(BAR_COMP, NCOMP);
+            named_bar_sync(BAR_TR, NTRF);
             float bx = 0.f, by = 0.f;
             if (GATE == 1) {
                 float Gx = 0.f, Gy = 0.f;
+#pragma unroll
                 for (int r2 = 0; r2 < RG; ++r2) {
                     const float tx = tot[r2 * DK + d], ty = tot[r2 * DK + d + 1];
                     if (r2 < rg) {
@@ -325,6 +340,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     gaml[d + 1] = Gy;
                 }
             }
+#pragma unroll 4
             for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
                 float eqx = 1.f, eqy = 1.f, ekx = 1.f, eky = 1.f;
                 if (GATE == 1) {
@@ -354,45 +370,49 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     *pk = __floats2bfloat162_rn(kf.x * iv * ekx, kf.y * iv * eky);
             }
             fence_proxy_async_smem();
-            named_bar_sync(BAR_COMP, NCOMP);
-            if (ctid == 0) mbar_arrive(&bar_trans[s]);
-            return true;
-        };
-
-        bool alive = ntiles > 0 ? transform(0) : true;
-        for (int i = 0; alive && i < ntiles; ++i) {
+            named_bar_sync(BAR_TR, NTRF);
+            if (ttid == 0) mbar_arrive(&bar_trans[s]);
+        }
+    } else {
+        // ================================================================ epilogue warpgroups
+        const int etid = tid;
+        for (int i = 0; i < ntiles; ++i) {
             const int b = i & 1;
             const uint32_t tb = tbase + b * C::BUFCOLS;
             {
                 const bool ok = mbar_wait_abort(&bar_mma1[b], (i >> 1) & 1, abortp);
-                if (!named_bar_and(BAR_COMP, NCOMP, ok)) break;
+                if (!named_bar_and(BAR_EP, NEP, ok)) break;
             }
             tc_fence_after();
             const int t0 = tile_at(i) * TR;
             // ---- P = causal mask of A -> shared (double-buffered)
             if (MODE == 0) {
                 uint8_t* sP = sPb + b * (TR * TR * 2);
-                uint32_t r[16];
-                tmem_ld16(tb + ((uint32_t)(32 * qd) << 16) + 16 * wg, r);
-                tmem_wait_ld();
-                if (lane < 16) {
-                    const int t = 16 * qd + lane;
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        float f[8];
+                for (int c = 0; c < C::PCOLS; c += 16) {
+                    uint32_t r[16];
+                    const int c0 = wg * C::PCOLS + c;
+                    tmem_ld16(tb + ((uint32_t)(32 * qd) << 16) + c0, r);
+                    tmem_wait_ld();
+                    if (lane < 16) {
+                        const int t = 16 * qd + lane;
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const int sidx = 16 * wg + 8 * u + j;
-                            f[j] = (sidx <= t) ? __uint_as_float(r[8 * u + j]) : 0.f;
+                        for (int u = 0; u < 2; ++u) {
+                            float f[8];
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const int sidx = c0 + 8 * u + j;
+                                f[j] = (sidx <= t) ? __uint_as_float(r[8 * u + j]) : 0.f;
+                            }
+                            store8_bf16(sP, sw128_off(t, c0 + 8 * u, BLK), f);
                         }
-                        store8_bf16(sP, sw128_off(t, 16 * wg + 8 * u, BLK), f);
                     }
                 }
                 fence_proxy_async_smem();
-                named_bar_sync(BAR_COMP, NCOMP);
-                if (ctid == 0) mbar_arrive(&bar_pready[b]);
+                named_bar_sync(BAR_EP, NEP);
+                if (etid == 0) mbar_arrive(&bar_pready[b]);
             }
-            // ---- state: S = e^Gamma (S + dS'); bf16 copy for the next tile's inter product
+            // ---- state: S = e^Gamma (S + dS') (MODE 2: S = e^Gamma S + dS'); bf16 copy
             {
                 const float* gam = gamb + b * DK;
                 const float* gaml = gamlb + b * DK;
@@ -407,11 +427,13 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                         uint32_t r[16];
                         tmem_ld16(tb + ((uint32_t)(32 * qd) << 16) + C::COL_S + h * DVT + wg * C::HALF + c, r);
                         tmem_wait_ld();
+                        if (MODE == 2)
 #pragma unroll
-                        if (MODE == 2)  // G_before = e^Gamma G_after + scale q~^T dO
                             for (int j = 0; j < 16; ++j) Sreg[h][c + j] = egv * Sreg[h][c + j] + __uint_as_float(r[j]);
                         else
-                            for (int j = 0; j < 16; ++j) Sreg[h][c + j] = egv * (Sreg[h][c + j] + __uint_as_float(r[j]));
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                Sreg[h][c + j] = egv * (Sreg[h][c + j] + __uint_as_float(r[j]));
                     }
                     if (MODE == 0 && srow_ok) {
 #pragma unroll
@@ -419,18 +441,17 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                             store8_bf16(sS, sw128_off(d, wg * C::HALF + j, DK * 128), &Sreg[h][j]);
                     }
                 }
-                if (MODE == 0) {
-                    fence_proxy_async_smem();
-                    named_bar_sync(BAR_COMP, NCOMP);
-                    if (ctid == 0) mbar_arrive(bar_sready);
+                if (MODE == 0) fence_proxy_async_smem();
+                named_bar_sync(BAR_EP, NEP);
+                if (etid == 0) {
+                    if (MODE == 0) mbar_arrive(bar_sready);
+                    mbar_arrive(&bar_gfree[b]);
                 }
             }
-            // ---- next tile's transform overlaps this tile's P V product
-            if (C::NS == 2 && i + 1 < ntiles && !transform(i + 1)) break;
             // ---- output tile
             if (MODE == 0) {
                 const bool ok = mbar_wait_abort(&bar_mma2[b], (i >> 1) & 1, abortp);
-                if (!named_bar_and(BAR_COMP, NCOMP, ok)) break;
+                if (!named_bar_and(BAR_EP, NEP, ok)) break;
                 tc_fence_after();
                 const int t = 16 * qd + (lane & 15);
                 const bool row_ok = (lane >= 16) && (t0 + t < P.L);
@@ -457,9 +478,8 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 }
             }
             tc_fence_before();
-            named_bar_sync(BAR_COMP, NCOMP);
-            if (ctid == 0) mbar_arrive(&bar_tfree[b]);
-            if (C::NS == 1 && i + 1 < ntiles && !transform(i + 1)) break;
+            named_bar_sync(BAR_EP, NEP);
+            if (etid == 0) mbar_arrive(&bar_tfree[b]);
         }
     }
 
@@ -473,7 +493,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
             if (*n_mma1) mbar_wait(&bar_mma1[(*n_mma1 - 1) & 1], ((*n_mma1 - 1) >> 1) & 1, 1u << 20);
             if (*n_mma2) mbar_wait(&bar_mma2[(*n_mma2 - 1) & 1], ((*n_mma2 - 1) >> 1) & 1, 1u << 20);
         }
-    } else if (tid < NCOMP && srow_ok) {
+    } else if (is_ep && srow_ok) {
         // final state of the segment
 #pragma unroll
         for (int h = 0; h < C::NH; ++h) {
