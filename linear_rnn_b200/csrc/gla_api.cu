@@ -1,5 +1,6 @@
 // C ABI of the library: argument validation, plan choice, workspace accounting and
 // error mapping. Every numerical step runs in the plans' CUDA kernels.
+#include <stdio.h>
 #include <string.h>
 
 #include <mutex>
@@ -90,7 +91,17 @@ gla_status resolve(const gla_problem* p, const Dims& P, bool bwd, int* plan) {
     return GLA_OK;
 }
 
-gla_status map_cuda(cudaError_t e) { return e == cudaSuccess ? GLA_OK : GLA_ERR_CUDA; }
+thread_local char g_last_detail[256] = "no error";
+
+void set_detail(const char* where, cudaError_t e) {
+    snprintf(g_last_detail, sizeof(g_last_detail), "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+gla_status map_cuda(cudaError_t e, const char* where = "launch") {
+    if (e == cudaSuccess) return GLA_OK;
+    set_detail(where, e);
+    return GLA_ERR_CUDA;
+}
 
 size_t ws_bytes(const Dims& P, int plan, bool bwd) {
     if (plan == GLA_PLAN_TC) return bwd ? tc::bwd_workspace_bytes(P) : tc::fwd_workspace_bytes(P);
@@ -128,7 +139,7 @@ gla_status gla_fwd(const gla_problem* p, const void* q, const void* k, const voi
     if (ws_bytes_given < ws_bytes(P, plan, false)) return GLA_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, st);
-    if (e != cudaSuccess) return GLA_ERR_CUDA;
+    if (e != cudaSuccess) return map_cuda(e, "status word reset");
     if ((size_t)P.B * P.H == 0) return GLA_OK;
     if (plan == GLA_PLAN_TC && P.L > 0)
         e = tc::fwd(P, q, k, v, g, igate, h0, o, hT, ws, st);
@@ -158,7 +169,7 @@ gla_status gla_bwd(const gla_problem* p, const void* q, const void* k, const voi
     if (ws_bytes_given < ws_bytes(P, plan, true)) return GLA_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, st);
-    if (e != cudaSuccess) return GLA_ERR_CUDA;
+    if (e != cudaSuccess) return map_cuda(e, "status word reset");
     if ((size_t)P.B * P.H == 0) return GLA_OK;
     if (plan == GLA_PLAN_TC && P.L > 0)
         e = tc::bwd(P, q, k, v, g, igate, h0, dO, dhT, dq, dk, dv, dg, di, dh0, ws, st);
@@ -190,6 +201,8 @@ gla_status gla_check_device_status(void* ws, void* stream) {
 }
 
 int gla_version(void) { return 100; }
+
+const char* gla_last_error_detail(void) { return g_last_detail; }
 
 unsigned long long gla_launch_count(void) {
     std::lock_guard<std::mutex> lk(g_prof_mu);

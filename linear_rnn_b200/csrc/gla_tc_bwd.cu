@@ -371,12 +371,18 @@ __global__ void __launch_bounds__(NT_B, 1)
                         f[j] = P.scale * eb * __uint_as_float(r[j]);
                     }
                     store16_bf16_global(A.dq + (rowbase + t0 + t) * P.Dk + d0 + c, f);
+                    // q*dq for dg, formed as bf16(scale q e^b) * D with the same rounding the dk/dv
+                    // kernel applies to q~, so the pairwise cancellation inside dg's reverse sum
+                    // survives the bf16 operands
                     if (GATE != 0)
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            sg[t * DKB + c + j] =
-                                __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sqr + sw128_off(t, c + j, BLK))) *
-                                f[j];
+                        for (int j = 0; j < 16; ++j) {
+                            const float qr =
+                                __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sqr + sw128_off(t, c + j, BLK)));
+                            const float eb = GATE == 1 ? sg[t * DKB + c + j] : rowE[t];
+                            const float qs = __bfloat162float(__float2bfloat16_rn(qr * P.scale * eb));
+                            sg[t * DKB + c + j] = qs * __uint_as_float(r[j]);
+                        }
                 } else if (GATE != 0 && lane >= 16) {
 #pragma unroll
                     for (int j = 0; j < 16; ++j) sg[t * DKB + c + j] = 0.f;
@@ -946,6 +952,10 @@ static BwdPlan plan_bwd(const Dims& P) {
     int nseg = 1;
     if (base * 4 < (long)sms * 3 && ntiles > 1) nseg = (int)((long)sms / base);
     if (nseg < 1) nseg = 1;
+    // dg's reverse sum restarts from an exact fp32 carry at every segment boundary; keeping
+    // segments to about ten tiles bounds how far bf16 operand rounding can accumulate
+    const int acc_seg = cdiv(ntiles, 10);
+    if (nseg < acc_seg) nseg = acc_seg;
     const int tiles_per_chunk = P.C / TR;
     const int nchunks = cdiv(P.L, P.C);
     if (nseg > nchunks) nseg = nchunks;
