@@ -43,7 +43,7 @@ using namespace sm100;
 // tile i (two TMEM accumulator buffers). Epilogue warp w reads TMEM lane quadrant w % 4;
 // each epilogue warpgroup owns DVT/NEWG state columns.
 constexpr int NEWG = 2;
-constexpr int NTWG = 2;
+constexpr int NTWG = 1;
 constexpr int NEP = NEWG * 128;
 constexpr int NTRF = NTWG * 128;
 constexpr int W_MMA = (NEP + NTRF) / 32;
@@ -97,7 +97,7 @@ struct FwdArgs {
 };
 
 template <int DK, int DVT, int GATE, int MODE>
-__global__ void __maxnreg__(112)
+__global__ void __launch_bounds__(NTHR_WS, 1)
     k_tc_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
              const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg, FwdArgs A, Dims P) {
     using C = Cfg<DK, DVT, GATE, MODE>;
