@@ -130,6 +130,26 @@ GLA_API const char* gla_last_error_detail(void);
 /* Library version as 10000*major + 100*minor + patch. */
 GLA_API int gla_version(void);
 
+/* Forward pass that allocates nothing, for callers that cannot allocate device memory
+ * themselves (for example a host whose device memory is all owned by another allocator
+ * under a fixed budget, or code that must not call cudaMalloc because it synchronises the
+ * device). The pages describe no such call; it is an addition of this library.
+ * Same arguments and results as gla_fwd, without the workspace: the scratch memory of the
+ * CUDA-core forward (GLA_PLAN_SIMT, any supported shape, fp32 or bf16 I/O) comes from one
+ * array of 16 MiB compiled into the library, which every GPU that loads the library holds
+ * until the process exits. The caller still provides inputs and outputs.
+ *  - Problems whose scratch exceeds 16 MiB (gla_workspace_bytes of the same problem with
+ *    plan GLA_PLAN_SIMT and for_backward = 0) return GLA_ERR_WORKSPACE before any launch.
+ *  - The first call on a device looks up that device's address of the array
+ *    (cudaGetSymbolAddress with the device current); make that first call before any
+ *    stream capture.
+ *  - All calls share the array and it keeps the last call's contents; calls whose work
+ *    overlaps on the GPU (other streams, other host threads) race on it.
+ *  - No cudaMalloc, cudaFree or allocating library routine is called. */
+GLA_API gla_status gla_fwd_static_scratch(const gla_problem* p, const void* q, const void* k, const void* v,
+                                          const float* g, const float* igate, const float* h0,
+                                          void* o, float* hT, void* stream);
+
 /* Measurement support (not needed for computing).
  * gla_launch_count: number of kernels this process has launched through the library.
  * gla_profiler_enable(1): from now on every kernel launch is bracketed by two CUDA events

@@ -19,7 +19,7 @@ GLA_PLAN_AUTO, GLA_PLAN_SIMT, GLA_PLAN_TC = 0, 1, 2
 # Every symbol include/gla.h declares (checked by tests/test_abi_symbols.py).
 EXPORTED = ("gla_workspace_bytes", "gla_fwd", "gla_bwd", "gla_status_string",
             "gla_check_device_status", "gla_version", "gla_launch_count", "gla_profiler_enable",
-            "gla_profiler_read", "gla_last_error_detail")
+            "gla_profiler_read", "gla_fwd_static_scratch", "gla_last_error_detail")
 
 
 class GlaProblem(ctypes.Structure):
@@ -63,6 +63,8 @@ def _load():
     lib.gla_version.restype = ctypes.c_int
     lib.gla_last_error_detail.argtypes = []
     lib.gla_last_error_detail.restype = ctypes.c_char_p
+    lib.gla_fwd_static_scratch.argtypes = [pp, vp, vp, vp, fp, fp, fp, vp, fp, vp]
+    lib.gla_fwd_static_scratch.restype = ctypes.c_int
     lib.gla_launch_count.argtypes = []
     lib.gla_launch_count.restype = ctypes.c_ulonglong
     lib.gla_profiler_enable.argtypes = [ctypes.c_int]
