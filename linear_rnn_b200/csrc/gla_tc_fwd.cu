@@ -63,7 +63,7 @@ struct Cfg {
     static constexpr uint32_t STAGE = QB + KB + GB + VB;
     static constexpr uint32_t PB = MODE == 0 ? 2 * TR * TR * 2 : 0;   // P, double-buffered
     static constexpr uint32_t SB = MODE == 0 ? DK * DVT * 2 : 0;      // bf16 state
-    static constexpr uint32_t SMALL = 256 + 2048 + 16 * DK + 1024;
+    static constexpr uint32_t SMALL = 256 + 4096 + 16 * DK + 1024;
     static constexpr int NS = (2 * STAGE + PB + SB + SMALL + 1024 <= 227 * 1024) ? 2 : 1;
     static constexpr uint32_t SMEM = NS * STAGE + PB + SB + SMALL + 1024;
     static constexpr int NH = DK == 256 ? 2 : 1;            // M=128 halves of the state
@@ -78,7 +78,8 @@ struct Cfg {
     static_assert(SMEM <= 227 * 1024, "shared memory");
     static_assert(HALF % 16 == 0 && PCOLS % 16 == 0, "column chunks");
     static_assert(BUF_USED <= 256 && NCOL <= 512, "tensor memory");
-    static_assert((DK / 2) <= NTRF && (TR * (DK / 2)) % NTRF == 0, "transform mapping");
+    static_assert((DK / 8) <= NTRF && NTRF % (DK / 8) == 0 && TR % (NTRF / (DK / 8)) == 0, "transform mapping");
+    static_assert((NTRF / (DK / 8)) * DK <= 1024, "cumsum group totals");
 };
 
 struct FwdArgs {
@@ -123,8 +124,8 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     int* n_consumed = reinterpret_cast<int*>(small + 172);
     int* n_mma1 = reinterpret_cast<int*>(small + 176);
     int* n_mma2 = reinterpret_cast<int*>(small + 180);
-    float* tot = reinterpret_cast<float*>(small + 256);      // [512] cumsum group totals
-    float* gamb = tot + 512;                                 // [2][DK] e^Gamma per buffer
+    float* tot = reinterpret_cast<float*>(small + 256);      // [1024] cumsum group totals
+    float* gamb = tot + 1024;                                // [2][DK] e^Gamma per buffer
     float* gamlb = gamb + 2 * DK;                            // [2][DK] Gamma per buffer
     float* rowE = gamlb + 2 * DK;                            // [64] e^b   (per-head gate)
     float* rowEi = rowE + TR;                                // [64] e^-b
@@ -266,10 +267,11 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
         }
     } else if (!is_ep) {
         // ================================================================ transform warpgroups
+        // Thread = (8 consecutive key dims = one 16-byte swizzle chunk, group of RPG rows).
         const int ttid = tid - NEP;
         const int twarp = ttid >> 5;
-        constexpr int NP = DK / 2, RG = NTRF / NP, RPG = TR / RG;
-        const int cp = ttid % NP, rg = ttid / NP, d = 2 * cp;
+        constexpr int NO = DK / 8, RG = NTRF / NO, RPG = TR / RG;
+        const int oc = ttid % NO, rg = ttid / NO, d0 = 8 * oc;
         for (int j = 0; j < ntiles; ++j) {
             const int s = j % C::NS, b = j & 1;
             uint8_t* st = sm + s * C::STAGE;
@@ -288,16 +290,19 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
             if (ok && j >= 2) ok = mbar_wait_abort(&bar_gfree[b], ((j >> 1) - 1) & 1, abortp);
             if (!named_bar_and(BAR_TR, NTRF, ok)) break;
             if (ttid == 0) *n_consumed = j + 1;
+            float bb[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) bb[u] = 0.f;
             if (GATE == 1) {
-                float ax = 0.f, ay = 0.f;
 #pragma unroll 4
                 for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
-                    const float2 gv = *reinterpret_cast<const float2*>(sg + r * DK + d);
-                    ax += gv.x;
-                    ay += gv.y;
+                    const float4 g0 = *reinterpret_cast<const float4*>(sg + r * DK + d0);
+                    const float4 g1 = *reinterpret_cast<const float4*>(sg + r * DK + d0 + 4);
+                    bb[0] += g0.x; bb[1] += g0.y; bb[2] += g0.z; bb[3] += g0.w;
+                    bb[4] += g1.x; bb[5] += g1.y; bb[6] += g1.z; bb[7] += g1.w;
                 }
-                tot[rg * DK + d] = ax;
-                tot[rg * DK + d + 1] = ay;
+                *reinterpret_cast<float4*>(tot + rg * DK + d0) = make_float4(bb[0], bb[1], bb[2], bb[3]);
+                *reinterpret_cast<float4*>(tot + rg * DK + d0 + 4) = make_float4(bb[4], bb[5], bb[6], bb[7]);
             } else if (GATE == 2) {
                 if (twarp == 0) {  // warp scan over 64 rows, two rows per lane
                     const float g0 = ghs[2 * lane], g1 = ghs[2 * lane + 1];
@@ -320,54 +325,84 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 }
             }
             named_bar_sync(BAR_TR, NTRF);
-            float bx = 0.f, by = 0.f;
             if (GATE == 1) {
-                float Gx = 0.f, Gy = 0.f;
+                float G8[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    bb[u] = 0.f;
+                    G8[u] = 0.f;
+                }
 #pragma unroll
                 for (int r2 = 0; r2 < RG; ++r2) {
-                    const float tx = tot[r2 * DK + d], ty = tot[r2 * DK + d + 1];
-                    if (r2 < rg) {
-                        bx += tx;
-                        by += ty;
+                    const float4 t0v = *reinterpret_cast<const float4*>(tot + r2 * DK + d0);
+                    const float4 t1v = *reinterpret_cast<const float4*>(tot + r2 * DK + d0 + 4);
+                    const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        if (r2 < rg) bb[u] += tv[u];
+                        G8[u] += tv[u];
                     }
-                    Gx += tx;
-                    Gy += ty;
                 }
                 if (rg == 0) {
-                    gam[d] = __expf(Gx);
-                    gam[d + 1] = __expf(Gy);
-                    gaml[d] = Gx;
-                    gaml[d + 1] = Gy;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        gam[d0 + u] = __expf(G8[u]);
+                        gaml[d0 + u] = G8[u];
+                    }
                 }
             }
-#pragma unroll 4
+#pragma unroll 2
             for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
-                float eqx = 1.f, eqy = 1.f, ekx = 1.f, eky = 1.f;
+                float eq[8], ek[8];
                 if (GATE == 1) {
-                    const float2 gv = *reinterpret_cast<const float2*>(sg + r * DK + d);
-                    bx += gv.x;
-                    by += gv.y;
-                    eqx = __expf(bx);
-                    eqy = __expf(by);
-                    ekx = __expf(-bx);
-                    eky = __expf(-by);
-                } else if (GATE == 2) {
-                    eqx = eqy = rowE[r];
-                    ekx = eky = rowEi[r];
+                    const float4 g0 = *reinterpret_cast<const float4*>(sg + r * DK + d0);
+                    const float4 g1 = *reinterpret_cast<const float4*>(sg + r * DK + d0 + 4);
+                    const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        bb[u] += gv[u];
+                        eq[u] = __expf(bb[u]);
+                        ek[u] = __expf(-bb[u]);
+                    }
+                } else {
+                    const float e1 = GATE == 2 ? rowE[r] : 1.f, e2 = GATE == 2 ? rowEi[r] : 1.f;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        eq[u] = e1;
+                        ek[u] = e2;
+                    }
                 }
-                const float iv = igs[r];
-                const uint32_t off = sw128_off(r, d, BLK);
+                const uint32_t off = (uint32_t)(d0 >> 6) * BLK + (uint32_t)r * 128 +
+                                     ((((uint32_t)((d0 & 63) >> 3)) ^ (uint32_t)(r & 7)) << 4);
                 if (MODE == 0) {
-                    __nv_bfloat162* pq = reinterpret_cast<__nv_bfloat162*>(sq + off);
-                    const float2 qf = __bfloat1622float2(*pq);
-                    *pq = __floats2bfloat162_rn(qf.x * eqx, qf.y * eqy);
+                    uint4* pq = reinterpret_cast<uint4*>(sq + off);
+                    uint4 w = *pq;
+                    uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wp[u]));
+                        __nv_bfloat162 h = __floats2bfloat162_rn(f.x * eq[2 * u], f.y * eq[2 * u + 1]);
+                        wp[u] = *reinterpret_cast<uint32_t*>(&h);
+                    }
+                    *pq = w;
                 }
-                __nv_bfloat162* pk = reinterpret_cast<__nv_bfloat162*>(sk + off);
-                const float2 kf = __bfloat1622float2(*pk);
-                if (MODE == 2)  // the k slot holds q: scale * q * e^b
-                    *pk = __floats2bfloat162_rn(kf.x * P.scale * eqx, kf.y * P.scale * eqy);
-                else
-                    *pk = __floats2bfloat162_rn(kf.x * iv * ekx, kf.y * iv * eky);
+                {
+                    uint4* pk = reinterpret_cast<uint4*>(sk + off);
+                    uint4 w = *pk;
+                    uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+                    const float iv = igs[r];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wp[u]));
+                        __nv_bfloat162 h;
+                        if (MODE == 2)  // the k slot holds q: scale * q * e^b
+                            h = __floats2bfloat162_rn(f.x * P.scale * eq[2 * u], f.y * P.scale * eq[2 * u + 1]);
+                        else
+                            h = __floats2bfloat162_rn(f.x * iv * ek[2 * u], f.y * iv * ek[2 * u + 1]);
+                        wp[u] = *reinterpret_cast<uint32_t*>(&h);
+                    }
+                    *pk = w;
+                }
             }
             fence_proxy_async_smem();
             named_bar_sync(BAR_TR, NTRF);
