@@ -74,6 +74,126 @@ __device__ __forceinline__ void store16_bf16_global(__nv_bfloat16* dst, const fl
 
 constexpr uint32_t pow2cols(uint32_t n) { return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512; }
 
+// In-place transform of one 64-token tile over 8-key-dim (16-byte swizzle chunk) groups,
+// 256 threads: b = column cumsum of the log-gate, then
+//   k~ = i * k * e^-b  (k tile),   DO_Q: q~ = scale * q * e^b  (q tile),
+//   per-key gates: the g tile is overwritten with e^b (G_SLOT_EB) or e^-b,
+//   gam[d] = e^Gamma.  Per-head gates use the row factors rowE / rowEi instead.
+// Both backward kernels use this one routine so they form bit-identical q~ and k~.
+template <int D, int GATE, bool DO_Q, bool G_SLOT_EB>
+__device__ __forceinline__ void bwd_transform(uint8_t* sq, uint8_t* sk, float* sg, float* tot, float* gam,
+                                              float* rowE, float* rowEi, const float* ghs, const float* igs,
+                                              float scale, int tid) {
+    constexpr int NO = D / 8, RG = NT_B / NO, RPG = TR / RG;
+    static_assert(RG * D <= 2048, "cumsum group totals");
+    const int oc = tid % NO, rg = tid / NO, d0 = 8 * oc;
+    const int warp = tid >> 5, lane = tid & 31;
+    float bb[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) bb[u] = 0.f;
+    if (GATE == 1) {
+#pragma unroll 4
+        for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
+            const float4 g0 = *reinterpret_cast<const float4*>(sg + r * D + d0);
+            const float4 g1 = *reinterpret_cast<const float4*>(sg + r * D + d0 + 4);
+            bb[0] += g0.x; bb[1] += g0.y; bb[2] += g0.z; bb[3] += g0.w;
+            bb[4] += g1.x; bb[5] += g1.y; bb[6] += g1.z; bb[7] += g1.w;
+        }
+        *reinterpret_cast<float4*>(tot + rg * D + d0) = make_float4(bb[0], bb[1], bb[2], bb[3]);
+        *reinterpret_cast<float4*>(tot + rg * D + d0 + 4) = make_float4(bb[4], bb[5], bb[6], bb[7]);
+    } else if (GATE == 2 && warp == 0) {
+        const float g0 = ghs[2 * lane], g1 = ghs[2 * lane + 1];
+        float v = g0 + g1;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float n = __shfl_up_sync(0xffffffffu, v, off);
+            if (lane >= off) v += n;
+        }
+        const float b1 = v, b0 = v - g1;
+        rowE[2 * lane] = __expf(b0);
+        rowE[2 * lane + 1] = __expf(b1);
+        rowEi[2 * lane] = __expf(-b0);
+        rowEi[2 * lane + 1] = __expf(-b1);
+        const float G = __shfl_sync(0xffffffffu, b1, 31);
+        if (lane == 0) gam[0] = __expf(G);
+    }
+    __syncthreads();
+    if (GATE == 1) {
+        float G8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            bb[u] = 0.f;
+            G8[u] = 0.f;
+        }
+#pragma unroll
+        for (int r2 = 0; r2 < RG; ++r2) {
+            const float4 t0v = *reinterpret_cast<const float4*>(tot + r2 * D + d0);
+            const float4 t1v = *reinterpret_cast<const float4*>(tot + r2 * D + d0 + 4);
+            const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (r2 < rg) bb[u] += tv[u];
+                G8[u] += tv[u];
+            }
+        }
+        if (rg == 0)
+#pragma unroll
+            for (int u = 0; u < 8; ++u) gam[d0 + u] = __expf(G8[u]);
+    }
+#pragma unroll 2
+    for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
+        float eq[8], ek[8];
+        if (GATE == 1) {
+            float4* gp = reinterpret_cast<float4*>(sg + r * D + d0);
+            const float4 g0 = gp[0], g1 = gp[1];
+            const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                bb[u] += gv[u];
+                eq[u] = __expf(bb[u]);
+                ek[u] = __expf(-bb[u]);
+            }
+            const float* keep = G_SLOT_EB ? eq : ek;
+            gp[0] = make_float4(keep[0], keep[1], keep[2], keep[3]);
+            gp[1] = make_float4(keep[4], keep[5], keep[6], keep[7]);
+        } else {
+            const float e1 = GATE == 2 ? rowE[r] : 1.f, e2 = GATE == 2 ? rowEi[r] : 1.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                eq[u] = e1;
+                ek[u] = e2;
+            }
+        }
+        const uint32_t off = (uint32_t)(d0 >> 6) * BLK + (uint32_t)r * 128 +
+                             ((((uint32_t)((d0 & 63) >> 3)) ^ (uint32_t)(r & 7)) << 4);
+        if (DO_Q) {
+            uint4* pq = reinterpret_cast<uint4*>(sq + off);
+            uint4 w = *pq;
+            uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wp[u]));
+                __nv_bfloat162 h = __floats2bfloat162_rn(f.x * scale * eq[2 * u], f.y * scale * eq[2 * u + 1]);
+                wp[u] = *reinterpret_cast<uint32_t*>(&h);
+            }
+            *pq = w;
+        }
+        {
+            uint4* pk = reinterpret_cast<uint4*>(sk + off);
+            uint4 w = *pk;
+            uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+            const float iv = igs[r];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wp[u]));
+                __nv_bfloat162 h = __floats2bfloat162_rn(f.x * iv * ek[2 * u], f.y * iv * ek[2 * u + 1]);
+                wp[u] = *reinterpret_cast<uint32_t*>(&h);
+            }
+            *pk = w;
+        }
+    }
+}
+
 // ============================================================================ dq
 template <int DKB, int DV, int GATE>
 struct QCfg {
@@ -86,7 +206,7 @@ struct QCfg {
     static constexpr uint32_t TXB = STAGE - (GATE == 1 ? 0 : GB); // bytes the copy engine writes
     static constexpr uint32_t SB = DKB * DV * 2;
     static constexpr uint32_t AB = TR * TR * 2;
-    static constexpr uint32_t SMALL = 256 + 4096 + 8 * DKB + 1024 + 512;
+    static constexpr uint32_t SMALL = 256 + 8192 + 8 * DKB + 1024 + 512;
     static constexpr int NS = (2 * STAGE + SB + AB + SMALL + 1024 <= 227 * 1024) ? 2 : 1;
     static constexpr uint32_t SMEM = NS * STAGE + SB + AB + SMALL + 1024;
     static constexpr uint32_t COL_R = DV;
@@ -113,7 +233,7 @@ __global__ void __launch_bounds__(NT_B, 1)
     uint64_t* bar_mma2 = bar_full + 3;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 64);
     float* tot = reinterpret_cast<float*>(small + 256);
-    float* gam = tot + 1024;            // [DKB]
+    float* gam = tot + 2048;            // [DKB]
     float* rowE = gam + DKB;            // [64]
     float* rowEi = rowE + TR;
     float* igs = rowEi + TR;
@@ -207,65 +327,10 @@ __global__ void __launch_bounds__(NT_B, 1)
         if (!block_wait(&bar_full[s], (i / C::NS) & 1)) { err = 1; break; }
 
         // ---- transform: k~ = i k e^-b in place; e^b kept (in place of g) for the dq epilogue
+        bwd_transform<DKB, GATE, false, true>(sqr, sk, sg, tot, gam, rowE, rowEi, ghs, igs, P.scale, tid);
+        // pair mapping of the later q*dq prefix phase
         constexpr int NP = DKB / 2, RG = NT_B / NP, RPG = TR / RG;
         const int cp = tid % NP, rg = tid / NP, d = 2 * cp;
-        if (GATE == 1) {
-            float ax = 0.f, ay = 0.f;
-            for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
-                const float2 gv = *reinterpret_cast<const float2*>(sg + r * DKB + d);
-                ax += gv.x;
-                ay += gv.y;
-            }
-            tot[rg * DKB + d] = ax;
-            tot[rg * DKB + d + 1] = ay;
-        } else if (GATE == 2 && warp == 0) {
-            const float g0 = ghs[2 * lane], g1 = ghs[2 * lane + 1];
-            float v = g0 + g1;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float n = __shfl_up_sync(0xffffffffu, v, off);
-                if (lane >= off) v += n;
-            }
-            const float b1 = v, b0 = v - g1;
-            rowE[2 * lane] = __expf(b0);
-            rowE[2 * lane + 1] = __expf(b1);
-            rowEi[2 * lane] = __expf(-b0);
-            rowEi[2 * lane + 1] = __expf(-b1);
-            const float G = __shfl_sync(0xffffffffu, b1, 31);
-            if (lane == 0) gam[0] = __expf(G);
-        }
-        __syncthreads();
-        {
-            float bx = 0.f, by = 0.f;
-            if (GATE == 1) {
-                float Gx = 0.f, Gy = 0.f;
-                for (int r2 = 0; r2 < RG; ++r2) {
-                    const float tx = tot[r2 * DKB + d], ty = tot[r2 * DKB + d + 1];
-                    if (r2 < rg) { bx += tx; by += ty; }
-                    Gx += tx;
-                    Gy += ty;
-                }
-                if (rg == 0) { gam[d] = __expf(Gx); gam[d + 1] = __expf(Gy); }
-            }
-            for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
-                float ekx = 1.f, eky = 1.f;
-                if (GATE == 1) {
-                    float2* gp = reinterpret_cast<float2*>(sg + r * DKB + d);
-                    const float2 gv = *gp;
-                    bx += gv.x;
-                    by += gv.y;
-                    ekx = __expf(-bx);
-                    eky = __expf(-by);
-                    *gp = make_float2(__expf(bx), __expf(by));
-                } else if (GATE == 2) {
-                    ekx = eky = rowEi[r];
-                }
-                const float iv = igs[r];
-                __nv_bfloat162* pk = reinterpret_cast<__nv_bfloat162*>(sk + sw128_off(r, d, BLK));
-                const float2 kf = __bfloat1622float2(*pk);
-                *pk = __floats2bfloat162_rn(kf.x * iv * ekx, kf.y * iv * eky);
-            }
-        }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -493,7 +558,7 @@ struct KVCfg {
     static constexpr uint32_t TXB = STAGE - (GATE == 1 ? 0 : GB);
     static constexpr uint32_t GTB = DK * DV * 2;
     static constexpr uint32_t AB = TR * TR * 2;
-    static constexpr uint32_t SMALL = 256 + 4096 + 4 * DK + 1024 + 512 + 16 * DK + 256 + 64;
+    static constexpr uint32_t SMALL = 256 + 8192 + 4 * DK + 1024 + 512 + 16 * DK + 256 + 64;
     static constexpr int NS = (2 * STAGE + GTB + 2 * AB + SMALL + 1024 <= 227 * 1024) ? 2 : 1;
     static constexpr uint32_t SMEM = NS * STAGE + GTB + 2 * AB + SMALL + 1024;
     static constexpr uint32_t COL_R = DV;
@@ -523,7 +588,7 @@ __global__ void __launch_bounds__(NT_B, 1)
     uint64_t* bar_mma2 = bar_full + 3;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 64);
     float* tot = reinterpret_cast<float*>(small + 256);
-    float* gam = tot + 1024;      // [DK]
+    float* gam = tot + 2048;      // [DK]
     float* rowE = gam + DK;       // [64]
     float* rowEi = rowE + TR;
     float* igs = rowEi + TR;
@@ -636,72 +701,10 @@ __global__ void __launch_bounds__(NT_B, 1)
         if (!block_wait(&bar_full[s], (i / C::NS) & 1)) { err = 1; break; }
 
         // ---- transform: q~ = scale q e^b, k~ = i k e^-b (in place); e^-b kept in place of g
+        bwd_transform<DK, GATE, true, false>(sq, sk, sg, tot, gam, rowE, rowEi, ghs, igs, P.scale, tid);
+        // pair mapping of the later dg phase
         constexpr int NP = DK / 2, RG = NT_B / NP, RPG = TR / RG;
         const int cp = tid % NP, rg = tid / NP, d = 2 * cp;
-        if (GATE == 1) {
-            float ax = 0.f, ay = 0.f;
-            for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
-                const float2 gv = *reinterpret_cast<const float2*>(sg + r * DK + d);
-                ax += gv.x;
-                ay += gv.y;
-            }
-            tot[rg * DK + d] = ax;
-            tot[rg * DK + d + 1] = ay;
-        } else if (GATE == 2 && warp == 0) {
-            const float g0 = ghs[2 * lane], g1 = ghs[2 * lane + 1];
-            float v = g0 + g1;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float n = __shfl_up_sync(0xffffffffu, v, off);
-                if (lane >= off) v += n;
-            }
-            const float b1 = v, b0 = v - g1;
-            rowE[2 * lane] = __expf(b0);
-            rowE[2 * lane + 1] = __expf(b1);
-            rowEi[2 * lane] = __expf(-b0);
-            rowEi[2 * lane + 1] = __expf(-b1);
-            const float G = __shfl_sync(0xffffffffu, b1, 31);
-            if (lane == 0) gam[0] = __expf(G);
-        }
-        __syncthreads();
-        {
-            float bx = 0.f, by = 0.f;
-            if (GATE == 1) {
-                float Gx = 0.f, Gy = 0.f;
-                for (int r2 = 0; r2 < RG; ++r2) {
-                    const float tx = tot[r2 * DK + d], ty = tot[r2 * DK + d + 1];
-                    if (r2 < rg) { bx += tx; by += ty; }
-                    Gx += tx;
-                    Gy += ty;
-                }
-                if (rg == 0) { gam[d] = __expf(Gx); gam[d + 1] = __expf(Gy); }
-            }
-            for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
-                float eqx = 1.f, eqy = 1.f, ekx = 1.f, eky = 1.f;
-                if (GATE == 1) {
-                    float2* gp = reinterpret_cast<float2*>(sg + r * DK + d);
-                    const float2 gv = *gp;
-                    bx += gv.x;
-                    by += gv.y;
-                    eqx = __expf(bx);
-                    eqy = __expf(by);
-                    ekx = __expf(-bx);
-                    eky = __expf(-by);
-                    *gp = make_float2(ekx, eky);
-                } else if (GATE == 2) {
-                    eqx = eqy = rowE[r];
-                    ekx = eky = rowEi[r];
-                }
-                const float iv = igs[r];
-                const uint32_t off = sw128_off(r, d, BLK);
-                __nv_bfloat162* pq = reinterpret_cast<__nv_bfloat162*>(sq + off);
-                const float2 qf = __bfloat1622float2(*pq);
-                *pq = __floats2bfloat162_rn(qf.x * P.scale * eqx, qf.y * P.scale * eqy);
-                __nv_bfloat162* pk = reinterpret_cast<__nv_bfloat162*>(sk + off);
-                const float2 kf = __bfloat1622float2(*pk);
-                *pk = __floats2bfloat162_rn(kf.x * iv * ekx, kf.y * iv * eky);
-            }
-        }
         __syncthreads();
         // ---- G~ = e^Gamma G in TMEM; bf16 copy
         {

@@ -76,7 +76,7 @@ struct Cfg {
     static constexpr int PCOLS = TR / NEWG;                  // P columns per epilogue warpgroup
     static_assert(STAGE % 1024 == 0, "stage alignment");
     static_assert(SMEM <= 227 * 1024, "shared memory");
-    static_assert(HALF % 16 == 0 && PCOLS % 16 == 0, "column chunks");
+    static_assert(HALF % 32 == 0 && PCOLS % 32 == 0, "column chunks");
     static_assert(BUF_USED <= 256 && NCOL <= 512, "tensor memory");
     static_assert((DK / 8) <= NTRF && NTRF % (DK / 8) == 0 && TR % (NTRF / (DK / 8)) == 0, "transform mapping");
     static_assert((NTRF / (DK / 8)) * DK <= 1024, "cumsum group totals");
@@ -424,15 +424,15 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
             if (MODE == 0) {
                 uint8_t* sP = sPb + b * (TR * TR * 2);
 #pragma unroll
-                for (int c = 0; c < C::PCOLS; c += 16) {
-                    uint32_t r[16];
+                for (int c = 0; c < C::PCOLS; c += 32) {
+                    uint32_t r[32];
                     const int c0 = wg * C::PCOLS + c;
-                    tmem_ld16(tb + ((uint32_t)(32 * qd) << 16) + c0, r);
+                    tmem_ld32(tb + ((uint32_t)(32 * qd) << 16) + c0, r);
                     tmem_wait_ld();
                     if (lane < 16) {
                         const int t = 16 * qd + lane;
 #pragma unroll
-                        for (int u = 0; u < 2; ++u) {
+                        for (int u = 0; u < 4; ++u) {
                             float f[8];
 #pragma unroll
                             for (int j = 0; j < 8; ++j) {
@@ -458,16 +458,16 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     const float egv = GATE == 0 ? 1.f : gam[gi];
                     if (GATE != 0) glog[h] += gaml[gi];
 #pragma unroll
-                    for (int c = 0; c < C::HALF; c += 16) {
-                        uint32_t r[16];
-                        tmem_ld16(tb + ((uint32_t)(32 * qd) << 16) + C::COL_S + h * DVT + wg * C::HALF + c, r);
+                    for (int c = 0; c < C::HALF; c += 32) {
+                        uint32_t r[32];
+                        tmem_ld32(tb + ((uint32_t)(32 * qd) << 16) + C::COL_S + h * DVT + wg * C::HALF + c, r);
                         tmem_wait_ld();
                         if (MODE == 2)
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) Sreg[h][c + j] = egv * Sreg[h][c + j] + __uint_as_float(r[j]);
+                            for (int j = 0; j < 32; ++j) Sreg[h][c + j] = egv * Sreg[h][c + j] + __uint_as_float(r[j]);
                         else
 #pragma unroll
-                            for (int j = 0; j < 16; ++j)
+                            for (int j = 0; j < 32; ++j)
                                 Sreg[h][c + j] = egv * (Sreg[h][c + j] + __uint_as_float(r[j]));
                     }
                     if (MODE == 0 && srow_ok) {
@@ -492,13 +492,13 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 const bool row_ok = (lane >= 16) && (t0 + t < P.L);
                 __nv_bfloat16* orow = A.o + (rowbase + t0 + t) * P.Dv + e0 + wg * C::HALF;
 #pragma unroll
-                for (int c = 0; c < C::HALF; c += 16) {
-                    uint32_t r[16];
-                    tmem_ld16(tb + ((uint32_t)(32 * qd) << 16) + wg * C::HALF + c, r);
+                for (int c = 0; c < C::HALF; c += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tb + ((uint32_t)(32 * qd) << 16) + wg * C::HALF + c, r);
                     tmem_wait_ld();
                     if (row_ok) {
 #pragma unroll
-                        for (int u = 0; u < 2; ++u) {
+                        for (int u = 0; u < 4; ++u) {
                             uint32_t w[4];
 #pragma unroll
                             for (int p2 = 0; p2 < 4; ++p2) {
@@ -553,34 +553,22 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
 }
 
 // Segment scan: sinit[z] = e^{Gamma_{z-1}} sinit[z-1] + dS_{z-1}, sinit[0] = h0 (or 0).
-// One thread per (bh, d, e) element; loads a batch of segment values before the chain.
-__global__ void k_seg_scan(const float* __restrict__ seg_state, const float* __restrict__ seg_gamma,
-                           const float* __restrict__ h0, float* __restrict__ sinit, int BH, int Dk, int Dv, int nseg) {
+// One thread per (bh, d, e) state element, walking the segments in order.
+__global__ void __launch_bounds__(256) k_seg_scan(const float* __restrict__ seg_state,
+                                                  const float* __restrict__ seg_gamma, const float* __restrict__ h0,
+                                                  float* __restrict__ sinit, int BH, int Dk, int Dv, int nseg) {
+    const int per = Dk * Dv;
     const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long per = (long)Dk * Dv;
     if (idx >= (long)BH * per) return;
-    const long bh = idx / per, de = idx % per;
-    const int d = (int)(de / Dv);
+    const int bh = (int)(idx / per), de = (int)(idx - (long)bh * per), d = de / Dv;
+    const float* src = seg_state + (size_t)bh * nseg * per + de;
+    const float* gam = seg_gamma + (size_t)bh * nseg * Dk + d;
+    float* dst = sinit + (size_t)bh * nseg * per + de;
     float S = h0 ? h0[idx] : 0.f;
-    constexpr int BATCH = 16;
-    for (int z0 = 0; z0 < nseg - 1; z0 += BATCH) {
-        float ds[BATCH], gl[BATCH];
-#pragma unroll
-        for (int u = 0; u < BATCH; ++u) {
-            const int z = z0 + u;
-            if (z < nseg - 1) {
-                ds[u] = seg_state[((bh * nseg + z) * per) + de];
-                gl[u] = seg_gamma[(bh * nseg + z) * Dk + d];
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < BATCH; ++u) {
-            const int z = z0 + u;
-            if (z < nseg - 1) {
-                S = __expf(gl[u]) * S + ds[u];
-                sinit[((bh * nseg + z + 1) * per) + de] = S;
-            }
-        }
+#pragma unroll 4
+    for (int z = 0; z < nseg - 1; ++z) {
+        S = __expf(gam[(size_t)z * Dk]) * S + src[(size_t)z * per];
+        dst[(size_t)(z + 1) * per] = S;
     }
 }
 
@@ -588,34 +576,22 @@ __global__ void k_seg_scan(const float* __restrict__ seg_state, const float* __r
 // segment z; gend[nseg-1] = dhT (or 0), gend[z] = e^{Gamma_{z+1}} gend[z+1] + dG_{z+1},
 // where dG_z (seg_state[z]) is segment z's own state-gradient accumulated from zero at
 // its end and Gamma_z (seg_gamma[z]) its total log-decay.
-__global__ void k_seg_rscan(const float* __restrict__ seg_state, const float* __restrict__ seg_gamma,
-                            const float* __restrict__ dhT, float* __restrict__ gend, int BH, int Dk, int Dv, int nseg) {
+__global__ void __launch_bounds__(256) k_seg_rscan(const float* __restrict__ seg_state,
+                                                   const float* __restrict__ seg_gamma, const float* __restrict__ dhT,
+                                                   float* __restrict__ gend, int BH, int Dk, int Dv, int nseg) {
+    const int per = Dk * Dv;
     const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long per = (long)Dk * Dv;
     if (idx >= (long)BH * per) return;
-    const long bh = idx / per, de = idx % per;
-    const int d = (int)(de / Dv);
+    const int bh = (int)(idx / per), de = (int)(idx - (long)bh * per), d = de / Dv;
+    const float* src = seg_state + (size_t)bh * nseg * per + de;
+    const float* gam = seg_gamma + (size_t)bh * nseg * Dk + d;
+    float* dst = gend + (size_t)bh * nseg * per + de;
     float G = dhT ? dhT[idx] : 0.f;
-    gend[((bh * nseg + nseg - 1) * per) + de] = G;
-    constexpr int BATCH = 16;
-    for (int z0 = nseg - 1; z0 >= 1; z0 -= BATCH) {
-        float dg[BATCH], gl[BATCH];
-#pragma unroll
-        for (int u = 0; u < BATCH; ++u) {
-            const int z = z0 - u;
-            if (z >= 1) {
-                dg[u] = seg_state[((bh * nseg + z) * per) + de];
-                gl[u] = seg_gamma[(bh * nseg + z) * Dk + d];
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < BATCH; ++u) {
-            const int z = z0 - u;
-            if (z >= 1) {
-                G = __expf(gl[u]) * G + dg[u];
-                gend[((bh * nseg + z - 1) * per) + de] = G;
-            }
-        }
+    dst[(size_t)(nseg - 1) * per] = G;
+#pragma unroll 4
+    for (int z = nseg - 1; z >= 1; --z) {
+        G = __expf(gam[(size_t)z * Dk]) * G + src[(size_t)z * per];
+        dst[(size_t)(z - 1) * per] = G;
     }
 }
 

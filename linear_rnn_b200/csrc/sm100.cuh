@@ -35,22 +35,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return done != 0;
 }
+// try_wait with a suspend-time hint: a thread whose phase has not completed is suspended
+// (it issues nothing) until the phase completes or about `hint_ns` nanoseconds pass, so
+// waiting warps leave the issue slots to the warps doing work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred P1;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2, %3;\n\t"
+        "selp.b32 %0, 1, 0, P1;\n\t}\n"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return done != 0;
+}
+constexpr uint32_t kWaitHintNs = 10000;         // per poll
+constexpr uint32_t kWaitPolls = 1u << 20;       // bound: about ten seconds at most
+
 // Bounded wait: returns false after `limit` polls without completion (the caller then
-// records a timeout and winds down). try_wait itself suspends for a hardware-defined
-// interval per poll, so the limit bounds the wait to well under a second.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = (1u << 24)) {
+// records a timeout and winds down).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = kWaitPolls) {
     for (uint32_t i = 0; i < limit; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, kWaitHintNs)) return true;
     return false;
 }
 
 // Bounded wait that also gives up when another role has raised the CTA's abort flag;
 // raising the flag itself when the poll limit is reached.
 __device__ __forceinline__ bool mbar_wait_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                                uint32_t limit = (1u << 24)) {
+                                                uint32_t limit = kWaitPolls) {
     for (uint32_t i = 0; i < limit; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 31u) == 31u && *abort_flag) return false;
+        if (mbar_try_wait_sleep(bar, parity, kWaitHintNs)) return true;
+        if ((i & 7u) == 7u && *abort_flag) return false;
     }
     *abort_flag = 1;
     return false;
