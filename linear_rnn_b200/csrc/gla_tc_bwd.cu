@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(NT_B, 1)
                 const __grid_constant__ CUtensorMap tdo, BwdArgs A, Dims P) {
     using C = QCfg<DKB, DV, GATE>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sm = smem_align1024(smem_raw);
     uint8_t* sS = sm + C::NS * C::STAGE;
     uint8_t* sA = sS + C::SB;
     uint8_t* small = sA + C::AB;
@@ -578,7 +578,7 @@ __global__ void __launch_bounds__(NT_B, 1)
                   const __grid_constant__ CUtensorMap tdo, BwdArgs A, Dims P) {
     using C = KVCfg<DK, DV, GATE>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sm = smem_align1024(smem_raw);
     uint8_t* sG = sm + C::NS * C::STAGE;
     uint8_t* sAm = sG + C::GTB;
     uint8_t* sdA = sAm + C::AB;

@@ -1,18 +1,18 @@
 // Tensor-core (tcgen05 / TMEM / TMA) forward of chunkwise gated linear attention, bf16 I/O.
 //
 // One CTA owns a (batch*head, Dv tile, sequence segment) and walks its segment in tiles
-// of 64 tokens, keeping the Dk x DVT state on chip: fp32 in registers (each thread owns
-// key-dim rows of it, the layout a tcgen05.ld of an M=128 accumulator delivers) and a
-// bf16 copy in shared memory as the B operand of the inter-chunk product. Per tile
-// (the chunk ("trunk") step of the talk summary "Hardware-Efficient Training of Linear
-// Attention Models", section 11:58, with the gates of the GLA abstract):
+// of 64 tokens, keeping the Dk x DVT state on chip: fp32 in tensor memory, where the
+// state product accumulates onto it, and a bf16 copy in shared memory as the B operand
+// of the inter-chunk product. Per tile (the chunk ("trunk") step of the talk summary
+// "Hardware-Efficient Training of Linear Attention Models", section 11:58, with the gates
+// of the GLA abstract):
 //   b      = in-tile inclusive cumsum of the log-gate (fp32), Gamma = b at the last row
 //   q~     = q * e^b,   k~ = i * k * e^-b            (bf16, in place in the TMA tile)
 //   A      = q~ k~^T                (tcgen05, M=64 N=64 K=Dk, TMEM lanes 0-15 of each quadrant)
 //   O      = q~ S_prev              (tcgen05, M=64 N=DVT K=Dk, TMEM lanes 16-31)
-//   dS'    = k~^T V                 (tcgen05, M=128 (or 64) N=DVT K=64)
+//   S     += k~^T V                 (tcgen05, M=128 (or 64) N=DVT K=64, onto the TMEM state)
+//   S      = diag(e^Gamma) S        (TMEM load, scale, store; bf16 copy for the next tile)
 //   P      = causal mask of A (bf16 in shared memory);  O += P V   (tcgen05)
-//   S      = diag(e^Gamma) (S_prev + dS')      (registers; bf16 copy for the next tile)
 //   o      = scale * O
 // q~ k~^T equals sum_d q_td k_sd e^(b_td - b_sd): the single in-tile reference point keeps
 // every exponent inside the tile's span. The state update uses k~ (not k e^(Gamma-b))
@@ -36,14 +36,14 @@ namespace tc {
 using namespace sm100;
 
 
-// Thread roles: warps [0, 4*NEWG) run the epilogues (P, state, output), warps
+// Thread roles: warps [0, 4*NEWG) run the epilogues (state, P, output), warps
 // [4*NEWG, 4*(NEWG+NTWG)) transform tiles in place, warp W_MMA issues the tcgen05 MMAs
 // and warp W_TMA the TMA loads. They hand tiles to each other through mbarriers: the
 // transform runs up to two tiles ahead, the MMAs of tile i+1 overlap the epilogues of
-// tile i (two TMEM accumulator buffers). Epilogue warp w reads TMEM lane quadrant w % 4;
+// tile i (two TMEM buffers for A and O). Epilogue warp w reads TMEM lane quadrant w % 4;
 // each epilogue warpgroup owns DVT/NEWG state columns.
 constexpr int NEWG = 2;
-constexpr int NTWG = 1;
+constexpr int NTWG = 2;
 constexpr int NEP = NEWG * 128;
 constexpr int NTRF = NTWG * 128;
 constexpr int W_MMA = (NEP + NTRF) / 32;
@@ -51,6 +51,8 @@ constexpr int W_TMA = W_MMA + 1;
 constexpr int NTHR_WS = NEP + NTRF + 64;
 constexpr int BAR_EP = 1;   // named barrier of the epilogue threads
 constexpr int BAR_TR = 2;   // named barrier of the transform threads
+
+constexpr uint32_t pow2_cols(uint32_t n) { return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512; }
 
 template <int DK, int DVT, int GATE, int MODE>
 struct Cfg {
@@ -63,23 +65,28 @@ struct Cfg {
     static constexpr uint32_t STAGE = QB + KB + GB + VB;
     static constexpr uint32_t PB = MODE == 0 ? 2 * TR * TR * 2 : 0;   // P, double-buffered
     static constexpr uint32_t SB = MODE == 0 ? DK * DVT * 2 : 0;      // bf16 state
-    static constexpr uint32_t SMALL = 256 + 4096 + 16 * DK + 1024;
-    static constexpr int NS = (2 * STAGE + PB + SB + SMALL + 1024 <= 227 * 1024) ? 2 : 1;
+    static constexpr uint32_t SMALL = 256 + 16 * DK + 1024;
+    static constexpr uint32_t FIXED = PB + SB + SMALL + 1024;
+    // as many ring stages (up to 4) as shared memory holds: the loads of a tile are in
+    // flight while the tiles before it are transformed and multiplied
+    static constexpr int NS = (4 * STAGE + FIXED <= 227 * 1024) ? 4 : (3 * STAGE + FIXED <= 227 * 1024) ? 3
+                              : (2 * STAGE + FIXED <= 227 * 1024) ? 2 : 1;
     static constexpr uint32_t SMEM = NS * STAGE + PB + SB + SMALL + 1024;
     static constexpr int NH = DK == 256 ? 2 : 1;            // M=128 halves of the state
     static constexpr int MS = DK == 64 ? 64 : 128;           // M of the state MMA
-    static constexpr uint32_t COL_S = (MODE == 0) ? (DVT > 64 ? DVT : 64) : 0;
-    static constexpr uint32_t BUF_USED = COL_S + NH * DVT;
-    static constexpr uint32_t BUFCOLS = BUF_USED <= 32 ? 32 : BUF_USED <= 64 ? 64 : BUF_USED <= 128 ? 128 : 256;
-    static constexpr uint32_t NCOL = 2 * BUFCOLS;            // two accumulator buffers
+    // TMEM columns: the fp32 state [0, COLS_S), then two buffers of COLA columns holding
+    // A (lanes 0-15 of each quadrant) and O (lanes 16-31) of a tile
+    static constexpr uint32_t COLS_S = NH * DVT;
+    static constexpr uint32_t COLA = MODE == 0 ? (DVT > 64 ? DVT : 64) : 0;
+    static constexpr uint32_t NCOL = pow2_cols(COLS_S + 2 * COLA);
     static constexpr int HALF = DVT / NEWG;                  // state columns per epilogue warpgroup
     static constexpr int PCOLS = TR / NEWG;                  // P columns per epilogue warpgroup
+    static constexpr int CH = 32;                            // TMEM columns per tcgen05.ld / st
     static_assert(STAGE % 1024 == 0, "stage alignment");
     static_assert(SMEM <= 227 * 1024, "shared memory");
-    static_assert(HALF % 32 == 0 && PCOLS % 32 == 0, "column chunks");
-    static_assert(BUF_USED <= 256 && NCOL <= 512, "tensor memory");
-    static_assert((DK / 8) <= NTRF && NTRF % (DK / 8) == 0 && TR % (NTRF / (DK / 8)) == 0, "transform mapping");
-    static_assert((NTRF / (DK / 8)) * DK <= 1024, "cumsum group totals");
+    static_assert(HALF % CH == 0 && PCOLS % CH == 0, "column chunks");
+    static_assert(COLS_S + 2 * COLA <= 512, "tensor memory");
+    static_assert(DK <= NTRF, "one transform thread per key dim in the cumsum");
 };
 
 struct FwdArgs {
@@ -103,29 +110,28 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
              const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg, FwdArgs A, Dims P) {
     using C = Cfg<DK, DVT, GATE, MODE>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sm = smem_align1024(smem_raw);
     uint8_t* sPb = sm + C::NS * C::STAGE;
     uint8_t* sS = sPb + C::PB;
     uint8_t* small = sS + C::SB;
     uint64_t* bars = reinterpret_cast<uint64_t*>(small);
-    uint64_t* bar_full = bars + 0;     // [2] TMA landed
-    uint64_t* bar_empty = bars + 2;    // [2] stage's MMAs done
-    uint64_t* bar_trans = bars + 4;    // [2] stage transformed
-    uint64_t* bar_mma1 = bars + 6;     // [2] A, dS', O_inter of the buffer done
-    uint64_t* bar_mma2 = bars + 8;     // [2] P V done
-    uint64_t* bar_pready = bars + 10;  // [2] P written
-    uint64_t* bar_tfree = bars + 12;   // [2] TMEM buffer read out
-    uint64_t* bar_gfree = bars + 14;   // [2] e^Gamma buffer read by the state epilogue
-    uint64_t* bar_sready = bars + 16;  // bf16 state of the last tile written
-    constexpr int NBARS = 17;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 160);
-    volatile int* abortp = reinterpret_cast<volatile int*>(small + 164);
-    int* n_issued = reinterpret_cast<int*>(small + 168);
-    int* n_consumed = reinterpret_cast<int*>(small + 172);
-    int* n_mma1 = reinterpret_cast<int*>(small + 176);
-    int* n_mma2 = reinterpret_cast<int*>(small + 180);
-    float* tot = reinterpret_cast<float*>(small + 256);      // [1024] cumsum group totals
-    float* gamb = tot + 1024;                                // [2][DK] e^Gamma per buffer
+    uint64_t* bar_full = bars + 0;     // [NS] TMA landed
+    uint64_t* bar_empty = bars + 4;    // [NS] stage's MMAs done
+    uint64_t* bar_trans = bars + 8;    // [NS] stage transformed
+    uint64_t* bar_mma1 = bars + 12;    // [2] A, O_inter and the state product of the tile done
+    uint64_t* bar_mma2 = bars + 14;    // [2] P V done
+    uint64_t* bar_pready = bars + 16;  // [2] P written
+    uint64_t* bar_tfree = bars + 18;   // [2] A/O buffer read out
+    uint64_t* bar_gfree = bars + 20;   // [2] e^Gamma buffer read by the state epilogue
+    uint64_t* bar_sready = bars + 22;  // state of the last tile decayed (and its bf16 copy written)
+    constexpr int NBARS = 23;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 192);
+    volatile int* abortp = reinterpret_cast<volatile int*>(small + 196);
+    int* n_issued = reinterpret_cast<int*>(small + 200);
+    int* n_consumed = reinterpret_cast<int*>(small + 204);
+    int* n_mma1 = reinterpret_cast<int*>(small + 208);
+    int* n_mma2 = reinterpret_cast<int*>(small + 212);
+    float* gamb = reinterpret_cast<float*>(small + 256);     // [2][DK] e^Gamma per buffer
     float* gamlb = gamb + 2 * DK;                            // [2][DK] Gamma per buffer
     float* rowE = gamlb + 2 * DK;                            // [64] e^b   (per-head gate)
     float* rowEi = rowE + TR;                                // [64] e^-b
@@ -143,6 +149,9 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     // the j-th tile this CTA processes (MODE 2 walks its segment backwards)
     auto tile_at = [&](int j) { return MODE == 2 ? tile0 + ntiles - 1 - j : tile0 + j; };
     const bool is_ep = tid < NEP;
+    // epilogue threads: key-dim row of the state this lane holds (M=64 state: lanes 0-15)
+    const bool srow_ok = (DK != 64) || (lane < 16);
+    auto srow = [&](int h) { return (DK == 64 ? 16 * qd + (lane & 15) : 32 * qd + lane) + 128 * h; };
 
     if (tid == 0) {
         for (int j = 0; j < NBARS; ++j) mbar_init(&bars[j], 1);
@@ -154,15 +163,17 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
         mbar_fence_init();
     }
     if (warp == 0) tmem_alloc(tmem_slot, C::NCOL);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
 
-    // ---- epilogue threads: state registers (rows d, HALF columns of the Dv tile)
-    const bool srow_ok = (DK != 64) || (lane < 16);
-    float Sreg[C::NH][C::HALF];
+    // ---- initial state -> TMEM (fp32) and its bf16 copy -> shared memory
     float glog[C::NH];
     if (is_ep) {
 #pragma unroll
         for (int h = 0; h < C::NH; ++h) {
-            const int d = (DK == 64 ? 16 * qd + (lane & 15) : 32 * qd + lane) + 128 * h;
+            const int d = srow(h);
             glog[h] = 0.f;
             const float* src = nullptr;
             if (MODE == 0) {
@@ -170,18 +181,27 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 else src = A.sinit + (((long)bh * A.nseg + z) * DK + d) * P.Dv;
             }
 #pragma unroll
-            for (int j = 0; j < C::HALF; ++j) Sreg[h][j] = (src && srow_ok) ? src[e0 + wg * C::HALF + j] : 0.f;
-            if (MODE == 0 && srow_ok)
+            for (int c = 0; c < C::HALF; c += C::CH) {
+                const int col = wg * C::HALF + c;
+                float f[C::CH];
 #pragma unroll
-                for (int j = 0; j < C::HALF; j += 8)
-                    store8_bf16(sS, sw128_off(d, wg * C::HALF + j, DK * 128), &Sreg[h][j]);
+                for (int j = 0; j < C::CH; j += 4) {
+                    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (src && srow_ok) x = *reinterpret_cast<const float4*>(src + e0 + col + j);
+                    f[j] = x.x; f[j + 1] = x.y; f[j + 2] = x.z; f[j + 3] = x.w;
+                }
+                tmem_stn<C::CH>(tbase + ((uint32_t)(32 * qd) << 16) + h * DVT + col, reinterpret_cast<uint32_t*>(f));
+                if (MODE == 0 && srow_ok)
+#pragma unroll
+                    for (int j = 0; j < C::CH; j += 8) store8_bf16(sS, sw128_off(d, col + j, DK * 128), &f[j]);
+            }
         }
+        tmem_wait_st();
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tbase = *tmem_slot;
 
     if (warp == W_TMA) {
         // ================================================================ TMA producer
@@ -217,7 +237,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
             for (int i = 0; i < ntiles; ++i) {
                 const int s = i % C::NS, b = i & 1;
                 if (!mbar_wait_abort(&bar_trans[s], (i / C::NS) & 1, abortp)) break;
-                if (i >= 2 && !mbar_wait_abort(&bar_tfree[b], ((i >> 1) - 1) & 1, abortp)) break;
+                if (MODE == 0 && i >= 2 && !mbar_wait_abort(&bar_tfree[b], ((i >> 1) - 1) & 1, abortp)) break;
                 tc_fence_after();
                 uint8_t* st = sm + s * C::STAGE;
                 // descriptors of the stage's tiles; K steps advance the 16-byte start field
@@ -225,31 +245,32 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 const uint64_t dKk = sw128_desc(smem_u32(st + C::QB), 16, 1024);       // k~, K-major
                 const uint64_t dKm = sw128_desc(smem_u32(st + C::QB), BLK, 1024);      // k~, MN-major
                 const uint64_t dV = sw128_desc(smem_u32(st + C::QB + C::KB + C::GB), BLK, 1024);
-                const uint32_t tb = tbase + b * C::BUFCOLS;
+                const uint32_t tAO = tbase + C::COLS_S + b * C::COLA;
                 if (MODE == 0) {
 #pragma unroll
                     for (int kk = 0; kk < DK / 16; ++kk) {
                         const uint64_t ko = ((kk >> 2) * BLK + (kk & 3) * 32) >> 4;
-                        mma_bf16(tb, dQ + ko, dKk + ko, idA, kk > 0);
+                        mma_bf16(tAO, dQ + ko, dKk + ko, idA, kk > 0);
+                    }
+                }
+                // the state of the previous tile must be decayed (and copied) first
+                if (i >= 1) {
+                    if (!mbar_wait_abort(bar_sready, (i - 1) & 1, abortp)) break;
+                    tc_fence_after();
+                }
+                if (MODE == 0) {
+#pragma unroll
+                    for (int kk = 0; kk < DK / 16; ++kk) {
+                        const uint64_t ko = ((kk >> 2) * BLK + (kk & 3) * 32) >> 4;
+                        mma_bf16(tAO + (16u << 16), dQ + ko, dS0 + ((kk * 2048) >> 4), idO, kk > 0);
                     }
                 }
 #pragma unroll
                 for (int h = 0; h < C::NH; ++h)
 #pragma unroll
                     for (int ks = 0; ks < TR / 16; ++ks)
-                        mma_bf16(tb + C::COL_S + h * DVT, dKm + ((h * 2 * BLK + ks * 2048) >> 4),
-                                 dV + ((ks * 2048) >> 4), idS, ks > 0);
-                if (MODE == 0) {
-                    if (i >= 1) {
-                        if (!mbar_wait_abort(bar_sready, (i - 1) & 1, abortp)) break;
-                        tc_fence_after();
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk) {
-                        const uint64_t ko = ((kk >> 2) * BLK + (kk & 3) * 32) >> 4;
-                        mma_bf16(tb + (16u << 16), dQ + ko, dS0 + ((kk * 2048) >> 4), idO, kk > 0);
-                    }
-                }
+                        mma_bf16(tbase + h * DVT, dKm + ((h * 2 * BLK + ks * 2048) >> 4), dV + ((ks * 2048) >> 4),
+                                 idS, 1);
                 mma_commit(&bar_mma1[b]);
                 *n_mma1 = i + 1;
                 if (MODE == 0) {
@@ -258,7 +279,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     const uint64_t dP = sw128_desc(smem_u32(sPb + b * (TR * TR * 2)), 16, 1024);
 #pragma unroll
                     for (int ks = 0; ks < TR / 16; ++ks)
-                        mma_bf16(tb + (16u << 16), dP + ((ks * 32) >> 4), dV + ((ks * 2048) >> 4), idO, 1);
+                        mma_bf16(tAO + (16u << 16), dP + ((ks * 32) >> 4), dV + ((ks * 2048) >> 4), idO, 1);
                     mma_commit(&bar_mma2[b]);
                     *n_mma2 = i + 1;
                 }
@@ -267,17 +288,19 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
         }
     } else if (!is_ep) {
         // ================================================================ transform warpgroups
-        // Thread = (8 consecutive key dims = one 16-byte swizzle chunk, group of RPG rows).
+        // Step A: b = inclusive column cumsum of the log-gate, written over g in place (one
+        // thread per key dim). Step B: every 16-byte chunk (8 key dims of one row) of the
+        // q and k tiles is scaled in place by its exponentials and rounded to bf16.
         const int ttid = tid - NEP;
-        const int twarp = ttid >> 5;
-        constexpr int NO = DK / 8, RG = NTRF / NO, RPG = TR / RG;
-        const int oc = ttid % NO, rg = ttid / NO, d0 = 8 * oc;
+        constexpr int NO = DK / 8;
+        constexpr int NQK = (MODE == 0 ? 2 : 1) * TR * NO;   // chunks of k (then q)
+        static_assert(NQK % NTRF == 0 && (TR * NO) % NTRF == 0, "chunk mapping");
         for (int j = 0; j < ntiles; ++j) {
             const int s = j % C::NS, b = j & 1;
             uint8_t* st = sm + s * C::STAGE;
             uint8_t* sq = st;
             uint8_t* sk = st + C::QB;
-            const float* sg = reinterpret_cast<const float*>(st + C::QB + C::KB);
+            float* sg = reinterpret_cast<float*>(st + C::QB + C::KB);
             float* gam = gamb + b * DK;
             float* gaml = gamlb + b * DK;
             const int t0 = tile_at(j) * TR;
@@ -290,21 +313,29 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
             if (ok && j >= 2) ok = mbar_wait_abort(&bar_gfree[b], ((j >> 1) - 1) & 1, abortp);
             if (!named_bar_and(BAR_TR, NTRF, ok)) break;
             if (ttid == 0) *n_consumed = j + 1;
-            float bb[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) bb[u] = 0.f;
+            // ---- step A
             if (GATE == 1) {
-#pragma unroll 4
-                for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
-                    const float4 g0 = *reinterpret_cast<const float4*>(sg + r * DK + d0);
-                    const float4 g1 = *reinterpret_cast<const float4*>(sg + r * DK + d0 + 4);
-                    bb[0] += g0.x; bb[1] += g0.y; bb[2] += g0.z; bb[3] += g0.w;
-                    bb[4] += g1.x; bb[5] += g1.y; bb[6] += g1.z; bb[7] += g1.w;
+                if (ttid < DK) {
+                    float* col = sg + ttid;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int r0 = 0; r0 < TR; r0 += 16) {
+                        float x[16];
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) x[u] = col[(r0 + u) * DK];
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) {
+                            acc += x[u];
+                            x[u] = acc;
+                        }
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) col[(r0 + u) * DK] = x[u];
+                    }
+                    gam[ttid] = __expf(acc);
+                    gaml[ttid] = acc;
                 }
-                *reinterpret_cast<float4*>(tot + rg * DK + d0) = make_float4(bb[0], bb[1], bb[2], bb[3]);
-                *reinterpret_cast<float4*>(tot + rg * DK + d0 + 4) = make_float4(bb[4], bb[5], bb[6], bb[7]);
             } else if (GATE == 2) {
-                if (twarp == 0) {  // warp scan over 64 rows, two rows per lane
+                if (ttid < 32) {  // warp scan over 64 rows, two rows per lane
                     const float g0 = ghs[2 * lane], g1 = ghs[2 * lane + 1];
                     float v = g0 + g1;
 #pragma unroll
@@ -313,11 +344,13 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                         if (lane >= off) v += n;
                     }
                     const float b1 = v, b0 = v - g1;
-                    rowE[2 * lane] = __expf(b0);
-                    rowE[2 * lane + 1] = __expf(b1);
+                    const float G = __shfl_sync(0xffffffffu, b1, 31);
+                    // MODE 2 scales q by e^(b - Gamma): the state epilogue applies e^Gamma after the add
+                    const float bq0 = MODE == 2 ? b0 - G : b0, bq1 = MODE == 2 ? b1 - G : b1;
+                    rowE[2 * lane] = __expf(bq0);
+                    rowE[2 * lane + 1] = __expf(bq1);
                     rowEi[2 * lane] = __expf(-b0);
                     rowEi[2 * lane + 1] = __expf(-b1);
-                    const float G = __shfl_sync(0xffffffffu, b1, 31);
                     if (lane == 0) {
                         gam[0] = __expf(G);
                         gaml[0] = G;
@@ -325,84 +358,46 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 }
             }
             named_bar_sync(BAR_TR, NTRF);
-            if (GATE == 1) {
-                float G8[8];
+            // ---- step B
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    bb[u] = 0.f;
-                    G8[u] = 0.f;
-                }
-#pragma unroll
-                for (int r2 = 0; r2 < RG; ++r2) {
-                    const float4 t0v = *reinterpret_cast<const float4*>(tot + r2 * DK + d0);
-                    const float4 t1v = *reinterpret_cast<const float4*>(tot + r2 * DK + d0 + 4);
-                    const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        if (r2 < rg) bb[u] += tv[u];
-                        G8[u] += tv[u];
-                    }
-                }
-                if (rg == 0) {
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        gam[d0 + u] = __expf(G8[u]);
-                        gaml[d0 + u] = G8[u];
-                    }
-                }
-            }
-#pragma unroll 2
-            for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
-                float eq[8], ek[8];
+            for (int it = 0; it < NQK / NTRF; ++it) {
+                const int c = ttid + it * NTRF;
+                const bool is_q = MODE == 0 && it * NTRF >= TR * NO;   // uniform per iteration
+                const int rem = c % (TR * NO);
+                const int r = rem / NO, d0 = 8 * (rem % NO);
+                // MODE 0/1: k slot -> i k e^-b, q slot -> q e^b; MODE 2: k slot holds q -> scale q e^(b-Gamma)
+                const bool up = is_q || MODE == 2;
+                float e[8];
                 if (GATE == 1) {
-                    const float4 g0 = *reinterpret_cast<const float4*>(sg + r * DK + d0);
-                    const float4 g1 = *reinterpret_cast<const float4*>(sg + r * DK + d0 + 4);
-                    const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        bb[u] += gv[u];
-                        eq[u] = __expf(bb[u]);
-                        ek[u] = __expf(-bb[u]);
+                    const float4 b0 = *reinterpret_cast<const float4*>(sg + r * DK + d0);
+                    const float4 b1 = *reinterpret_cast<const float4*>(sg + r * DK + d0 + 4);
+                    float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                    if (MODE == 2) {
+                        const float4 G0 = *reinterpret_cast<const float4*>(gaml + d0);
+                        const float4 G1 = *reinterpret_cast<const float4*>(gaml + d0 + 4);
+                        bv[0] -= G0.x; bv[1] -= G0.y; bv[2] -= G0.z; bv[3] -= G0.w;
+                        bv[4] -= G1.x; bv[5] -= G1.y; bv[6] -= G1.z; bv[7] -= G1.w;
                     }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) e[u] = __expf(up ? bv[u] : -bv[u]);
                 } else {
-                    const float e1 = GATE == 2 ? rowE[r] : 1.f, e2 = GATE == 2 ? rowEi[r] : 1.f;
+                    const float f = GATE == 2 ? (up ? rowE[r] : rowEi[r]) : 1.f;
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        eq[u] = e1;
-                        ek[u] = e2;
-                    }
+                    for (int u = 0; u < 8; ++u) e[u] = f;
                 }
+                const float m = MODE == 2 ? P.scale : (is_q ? 1.f : igs[r]);
                 const uint32_t off = (uint32_t)(d0 >> 6) * BLK + (uint32_t)r * 128 +
                                      ((((uint32_t)((d0 & 63) >> 3)) ^ (uint32_t)(r & 7)) << 4);
-                if (MODE == 0) {
-                    uint4* pq = reinterpret_cast<uint4*>(sq + off);
-                    uint4 w = *pq;
-                    uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+                uint4* p = reinterpret_cast<uint4*>((is_q ? sq : sk) + off);
+                uint4 w = *p;
+                uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wp[u]));
-                        __nv_bfloat162 h = __floats2bfloat162_rn(f.x * eq[2 * u], f.y * eq[2 * u + 1]);
-                        wp[u] = *reinterpret_cast<uint32_t*>(&h);
-                    }
-                    *pq = w;
+                for (int u = 0; u < 4; ++u) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wp[u]));
+                    __nv_bfloat162 h = __floats2bfloat162_rn(f.x * m * e[2 * u], f.y * m * e[2 * u + 1]);
+                    wp[u] = *reinterpret_cast<uint32_t*>(&h);
                 }
-                {
-                    uint4* pk = reinterpret_cast<uint4*>(sk + off);
-                    uint4 w = *pk;
-                    uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
-                    const float iv = igs[r];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wp[u]));
-                        __nv_bfloat162 h;
-                        if (MODE == 2)  // the k slot holds q: scale * q * e^b
-                            h = __floats2bfloat162_rn(f.x * P.scale * eq[2 * u], f.y * P.scale * eq[2 * u + 1]);
-                        else
-                            h = __floats2bfloat162_rn(f.x * iv * ek[2 * u], f.y * iv * ek[2 * u + 1]);
-                        wp[u] = *reinterpret_cast<uint32_t*>(&h);
-                    }
-                    *pk = w;
-                }
+                *p = w;
             }
             fence_proxy_async_smem();
             named_bar_sync(BAR_TR, NTRF);
@@ -411,28 +406,65 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     } else {
         // ================================================================ epilogue warpgroups
         const int etid = tid;
+        const uint32_t lq = (uint32_t)(32 * qd) << 16;   // this warp's TMEM lane quadrant
         for (int i = 0; i < ntiles; ++i) {
             const int b = i & 1;
-            const uint32_t tb = tbase + b * C::BUFCOLS;
+            const uint32_t tAO = tbase + C::COLS_S + b * C::COLA;
             {
                 const bool ok = mbar_wait_abort(&bar_mma1[b], (i >> 1) & 1, abortp);
                 if (!named_bar_and(BAR_EP, NEP, ok)) break;
             }
             tc_fence_after();
             const int t0 = tile_at(i) * TR;
+            // ---- state: S = e^Gamma (S_prev + dS'), where the MMA has added dS' onto S_prev
+            //      in TMEM; the decayed state goes back to TMEM and, as bf16, to shared memory
+            {
+                const float* gam = gamb + b * DK;
+                const float* gaml = gamlb + b * DK;
+#pragma unroll
+                for (int h = 0; h < C::NH; ++h) {
+                    const int d = srow(h);
+                    const int gi = GATE == 1 ? d : 0;
+                    const float egv = GATE == 0 ? 1.f : gam[gi];
+                    if (GATE != 0) glog[h] += gaml[gi];
+#pragma unroll
+                    for (int c = 0; c < C::HALF; c += C::CH) {
+                        const int col = wg * C::HALF + c;
+                        float f[C::CH];
+                        uint32_t* r = reinterpret_cast<uint32_t*>(f);
+                        tmem_ldn<C::CH>(tbase + lq + h * DVT + col, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < C::CH; ++j) f[j] *= egv;
+                        tmem_stn<C::CH>(tbase + lq + h * DVT + col, r);
+                        if (MODE == 0 && srow_ok)
+#pragma unroll
+                            for (int j = 0; j < C::CH; j += 8) store8_bf16(sS, sw128_off(d, col + j, DK * 128), &f[j]);
+                    }
+                }
+                tmem_wait_st();
+                if (MODE == 0) fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar_sync(BAR_EP, NEP);
+                if (etid == 0) {
+                    mbar_arrive(bar_sready);
+                    mbar_arrive(&bar_gfree[b]);
+                }
+            }
+            if (MODE != 0) continue;
             // ---- P = causal mask of A -> shared (double-buffered)
-            if (MODE == 0) {
+            {
                 uint8_t* sP = sPb + b * (TR * TR * 2);
 #pragma unroll
-                for (int c = 0; c < C::PCOLS; c += 32) {
-                    uint32_t r[32];
+                for (int c = 0; c < C::PCOLS; c += C::CH) {
+                    uint32_t r[C::CH];
                     const int c0 = wg * C::PCOLS + c;
-                    tmem_ld32(tb + ((uint32_t)(32 * qd) << 16) + c0, r);
+                    tmem_ldn<C::CH>(tAO + lq + c0, r);
                     tmem_wait_ld();
                     if (lane < 16) {
                         const int t = 16 * qd + lane;
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
+                        for (int u = 0; u < C::CH / 8; ++u) {
                             float f[8];
 #pragma unroll
                             for (int j = 0; j < 8; ++j) {
@@ -447,44 +479,8 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 named_bar_sync(BAR_EP, NEP);
                 if (etid == 0) mbar_arrive(&bar_pready[b]);
             }
-            // ---- state: S = e^Gamma (S + dS') (MODE 2: S = e^Gamma S + dS'); bf16 copy
-            {
-                const float* gam = gamb + b * DK;
-                const float* gaml = gamlb + b * DK;
-#pragma unroll
-                for (int h = 0; h < C::NH; ++h) {
-                    const int d = (DK == 64 ? 16 * qd + (lane & 15) : 32 * qd + lane) + 128 * h;
-                    const int gi = GATE == 1 ? d : 0;
-                    const float egv = GATE == 0 ? 1.f : gam[gi];
-                    if (GATE != 0) glog[h] += gaml[gi];
-#pragma unroll
-                    for (int c = 0; c < C::HALF; c += 32) {
-                        uint32_t r[32];
-                        tmem_ld32(tb + ((uint32_t)(32 * qd) << 16) + C::COL_S + h * DVT + wg * C::HALF + c, r);
-                        tmem_wait_ld();
-                        if (MODE == 2)
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) Sreg[h][c + j] = egv * Sreg[h][c + j] + __uint_as_float(r[j]);
-                        else
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                Sreg[h][c + j] = egv * (Sreg[h][c + j] + __uint_as_float(r[j]));
-                    }
-                    if (MODE == 0 && srow_ok) {
-#pragma unroll
-                        for (int j = 0; j < C::HALF; j += 8)
-                            store8_bf16(sS, sw128_off(d, wg * C::HALF + j, DK * 128), &Sreg[h][j]);
-                    }
-                }
-                if (MODE == 0) fence_proxy_async_smem();
-                named_bar_sync(BAR_EP, NEP);
-                if (etid == 0) {
-                    if (MODE == 0) mbar_arrive(bar_sready);
-                    mbar_arrive(&bar_gfree[b]);
-                }
-            }
             // ---- output tile
-            if (MODE == 0) {
+            {
                 const bool ok = mbar_wait_abort(&bar_mma2[b], (i >> 1) & 1, abortp);
                 if (!named_bar_and(BAR_EP, NEP, ok)) break;
                 tc_fence_after();
@@ -492,13 +488,13 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 const bool row_ok = (lane >= 16) && (t0 + t < P.L);
                 __nv_bfloat16* orow = A.o + (rowbase + t0 + t) * P.Dv + e0 + wg * C::HALF;
 #pragma unroll
-                for (int c = 0; c < C::HALF; c += 32) {
-                    uint32_t r[32];
-                    tmem_ld32(tb + ((uint32_t)(32 * qd) << 16) + wg * C::HALF + c, r);
+                for (int c = 0; c < C::HALF; c += C::CH) {
+                    uint32_t r[C::CH];
+                    tmem_ldn<C::CH>(tAO + lq + wg * C::HALF + c, r);
                     tmem_wait_ld();
                     if (row_ok) {
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
+                        for (int u = 0; u < C::CH / 8; ++u) {
                             uint32_t w[4];
 #pragma unroll
                             for (int p2 = 0; p2 < 4; ++p2) {
@@ -518,7 +514,9 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
         }
     }
 
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
     if (*abortp) {
         if (tid == 0) {
             atomicExch(A.status, kDevStatusTimeout);
@@ -528,23 +526,31 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
             if (*n_mma1) mbar_wait(&bar_mma1[(*n_mma1 - 1) & 1], ((*n_mma1 - 1) >> 1) & 1, 1u << 20);
             if (*n_mma2) mbar_wait(&bar_mma2[(*n_mma2 - 1) & 1], ((*n_mma2 - 1) >> 1) & 1, 1u << 20);
         }
-    } else if (is_ep && srow_ok) {
-        // final state of the segment
+    } else if (is_ep) {
+        // final state of the segment, read back from TMEM
 #pragma unroll
+        const uint32_t lq = (uint32_t)(32 * qd) << 16;
         for (int h = 0; h < C::NH; ++h) {
-            const int d = (DK == 64 ? 16 * qd + lane : 32 * qd + lane) + 128 * h;
+            const int d = srow(h);
             float* dst = nullptr;
             if (MODE == 0) {
                 if (z == A.nseg - 1 && A.hT) dst = A.hT + ((long)bh * DK + d) * P.Dv;
             } else {
                 dst = A.seg_state + (((long)bh * A.nseg + z) * DK + d) * P.Dv;
-                if (vt == 0 && wg == 0) A.seg_gamma[((long)bh * A.nseg + z) * DK + d] = glog[h];
+                if (vt == 0 && wg == 0 && srow_ok) A.seg_gamma[((long)bh * A.nseg + z) * DK + d] = glog[h];
             }
-            if (dst)
+            if (!dst) continue;
 #pragma unroll
-                for (int j = 0; j < C::HALF; j += 4)
-                    *reinterpret_cast<float4*>(dst + e0 + wg * C::HALF + j) =
-                        make_float4(Sreg[h][j], Sreg[h][j + 1], Sreg[h][j + 2], Sreg[h][j + 3]);
+            for (int c = 0; c < C::HALF; c += C::CH) {
+                const int col = wg * C::HALF + c;
+                float f[C::CH];
+                tmem_ldn<C::CH>(tbase + lq + h * DVT + col, reinterpret_cast<uint32_t*>(f));
+                tmem_wait_ld();
+                if (srow_ok)
+#pragma unroll
+                    for (int j = 0; j < C::CH; j += 4)
+                        *reinterpret_cast<float4*>(dst + e0 + col + j) = make_float4(f[j], f[j + 1], f[j + 2], f[j + 3]);
+            }
         }
     }
     tc_fence_before();
