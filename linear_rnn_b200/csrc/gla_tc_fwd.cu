@@ -49,8 +49,17 @@ constexpr int NTRF = NTWG * 128;
 constexpr int W_MMA = (NEP + NTRF) / 32;
 constexpr int W_TMA = W_MMA + 1;
 constexpr int NTHR_WS = NEP + NTRF + 64;
-constexpr int BAR_EP = 1;   // named barrier of the epilogue threads
+constexpr int BAR_S = 1;    // named barrier of the state-epilogue threads
 constexpr int BAR_TR = 2;   // named barrier of the transform threads
+constexpr int BAR_PO = 3;   // named barrier of the P/output-epilogue threads (output pass)
+constexpr float kLog2e = 1.4426950408889634f;
+
+// 2^x on the special-function unit (inputs here are log-gate sums times log2(e))
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 constexpr uint32_t pow2_cols(uint32_t n) { return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512; }
 
@@ -63,29 +72,34 @@ struct Cfg {
     static constexpr uint32_t GB = GATE == 1 ? TR * DK * 4 : 0;
     static constexpr uint32_t VB = TR * DVT * 2;
     static constexpr uint32_t STAGE = QB + KB + GB + VB;
-    static constexpr uint32_t PB = MODE == 0 ? 2 * TR * TR * 2 : 0;   // P, double-buffered
+    static constexpr uint32_t PB = MODE == 0 ? TR * TR * 2 : 0;       // P
     static constexpr uint32_t SB = MODE == 0 ? DK * DVT * 2 : 0;      // bf16 state
-    static constexpr uint32_t SMALL = 256 + 16 * DK + 1024;
-    static constexpr uint32_t FIXED = PB + SB + SMALL + 1024;
+    static constexpr uint32_t OB = MODE == 0 ? TR * DVT * 2 : 0;      // output tile staged for the TMA store
+    static constexpr uint32_t SMALL = 256 + 4 * NTRF + 16 * DK + 1024;
+    static constexpr uint32_t FIXED = PB + SB + OB + SMALL + 1024;
     // as many ring stages (up to 4) as shared memory holds: the loads of a tile are in
     // flight while the tiles before it are transformed and multiplied
     static constexpr int NS = (4 * STAGE + FIXED <= 227 * 1024) ? 4 : (3 * STAGE + FIXED <= 227 * 1024) ? 3
                               : (2 * STAGE + FIXED <= 227 * 1024) ? 2 : 1;
-    static constexpr uint32_t SMEM = NS * STAGE + PB + SB + SMALL + 1024;
+    static constexpr uint32_t SMEM = NS * STAGE + FIXED;
     static constexpr int NH = DK == 256 ? 2 : 1;            // M=128 halves of the state
     static constexpr int MS = DK == 64 ? 64 : 128;           // M of the state MMA
-    // TMEM columns: the fp32 state [0, COLS_S), then two buffers of COLA columns holding
+    // TMEM columns: the fp32 state [0, COLS_S), then NAB buffers of COLA columns holding
     // A (lanes 0-15 of each quadrant) and O (lanes 16-31) of a tile
+    static constexpr int NAB = 3;
     static constexpr uint32_t COLS_S = NH * DVT;
     static constexpr uint32_t COLA = MODE == 0 ? (DVT > 64 ? DVT : 64) : 0;
-    static constexpr uint32_t NCOL = pow2_cols(COLS_S + 2 * COLA);
-    static constexpr int HALF = DVT / NEWG;                  // state columns per epilogue warpgroup
-    static constexpr int PCOLS = TR / NEWG;                  // P columns per epilogue warpgroup
+    static constexpr uint32_t NCOL = pow2_cols(COLS_S + NAB * COLA);
+    // Epilogue split. Output pass: warpgroup 0 runs the state pass over all DVT columns
+    // (the recurrence's critical path), warpgroup 1 the P and output passes. State-only
+    // passes: both warpgroups run the state pass, DVT/2 columns each.
+    static constexpr int SCOLS = MODE == 0 ? DVT : DVT / 2;  // state columns per state-pass thread
+    static constexpr int NSW = MODE == 0 ? 128 : 256;        // state-pass threads
     static constexpr int CH = 32;                            // TMEM columns per tcgen05.ld / st
     static_assert(STAGE % 1024 == 0, "stage alignment");
     static_assert(SMEM <= 227 * 1024, "shared memory");
-    static_assert(HALF % CH == 0 && PCOLS % CH == 0, "column chunks");
-    static_assert(COLS_S + 2 * COLA <= 512, "tensor memory");
+    static_assert(SCOLS % CH == 0 && DVT % CH == 0 && TR % CH == 0, "column chunks");
+    static_assert(COLS_S + NAB * COLA <= 512, "tensor memory");
     static_assert(DK <= NTRF, "one transform thread per key dim in the cumsum");
 };
 
@@ -107,31 +121,35 @@ struct FwdArgs {
 template <int DK, int DVT, int GATE, int MODE>
 __global__ void __launch_bounds__(NTHR_WS, 1)
     k_tc_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-             const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg, FwdArgs A, Dims P) {
+             const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg,
+             const __grid_constant__ CUtensorMap to, FwdArgs A, Dims P) {
     using C = Cfg<DK, DVT, GATE, MODE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = smem_align1024(smem_raw);
     uint8_t* sPb = sm + C::NS * C::STAGE;
     uint8_t* sS = sPb + C::PB;
-    uint8_t* small = sS + C::SB;
+    uint8_t* sO = sS + C::SB;
+    uint8_t* small = sO + C::OB;
     uint64_t* bars = reinterpret_cast<uint64_t*>(small);
     uint64_t* bar_full = bars + 0;     // [NS] TMA landed
     uint64_t* bar_empty = bars + 4;    // [NS] stage's MMAs done
     uint64_t* bar_trans = bars + 8;    // [NS] stage transformed
-    uint64_t* bar_mma1 = bars + 12;    // [2] A, O_inter and the state product of the tile done
-    uint64_t* bar_mma2 = bars + 14;    // [2] P V done
-    uint64_t* bar_pready = bars + 16;  // [2] P written
-    uint64_t* bar_tfree = bars + 18;   // [2] A/O buffer read out
-    uint64_t* bar_gfree = bars + 20;   // [2] e^Gamma buffer read by the state epilogue
-    uint64_t* bar_sready = bars + 22;  // state of the last tile decayed (and its bf16 copy written)
-    constexpr int NBARS = 23;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 192);
-    volatile int* abortp = reinterpret_cast<volatile int*>(small + 196);
-    int* n_issued = reinterpret_cast<int*>(small + 200);
-    int* n_consumed = reinterpret_cast<int*>(small + 204);
-    int* n_mma1 = reinterpret_cast<int*>(small + 208);
-    int* n_mma2 = reinterpret_cast<int*>(small + 212);
-    float* gamb = reinterpret_cast<float*>(small + 256);     // [2][DK] e^Gamma per buffer
+    uint64_t* bar_mma1 = bars + 12;    // [2] O_inter and the state product of the tile done
+    uint64_t* bar_mma2 = bars + 14;    // [NAB] P V done
+    uint64_t* bar_pready = bars + 17;  // [2] P written
+    uint64_t* bar_tfree = bars + 19;   // [NAB] A/O buffer read out
+    uint64_t* bar_gfree = bars + 22;   // [2] e^Gamma buffer read by the state epilogue
+    uint64_t* bar_sready = bars + 24;  // state of the last tile decayed (and its bf16 copy written)
+    uint64_t* bar_aready = bars + 25;  // [NAB] A of the tile done
+    constexpr int NBARS = 28;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 224);
+    volatile int* abortp = reinterpret_cast<volatile int*>(small + 228);
+    int* n_issued = reinterpret_cast<int*>(small + 232);
+    int* n_consumed = reinterpret_cast<int*>(small + 236);
+    int* n_mma1 = reinterpret_cast<int*>(small + 240);
+    int* n_mma2 = reinterpret_cast<int*>(small + 244);
+    float* tot = reinterpret_cast<float*>(small + 256);      // [NTRF] cumsum segment totals
+    float* gamb = tot + NTRF;                                // [2][DK] e^Gamma per buffer
     float* gamlb = gamb + 2 * DK;                            // [2][DK] Gamma per buffer
     float* rowE = gamlb + 2 * DK;                            // [64] e^b   (per-head gate)
     float* rowEi = rowE + TR;                                // [64] e^-b
@@ -169,8 +187,10 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     const uint32_t tbase = *tmem_slot;
 
     // ---- initial state -> TMEM (fp32) and its bf16 copy -> shared memory
+    const bool s_worker = is_ep && (MODE != 0 || wg == 0);
+    const int scol0 = MODE == 0 ? 0 : wg * C::SCOLS;   // first state column of this state-pass thread
     float glog[C::NH];
-    if (is_ep) {
+    if (s_worker) {
 #pragma unroll
         for (int h = 0; h < C::NH; ++h) {
             const int d = srow(h);
@@ -181,8 +201,8 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 else src = A.sinit + (((long)bh * A.nseg + z) * DK + d) * P.Dv;
             }
 #pragma unroll
-            for (int c = 0; c < C::HALF; c += C::CH) {
-                const int col = wg * C::HALF + c;
+            for (int c = 0; c < C::SCOLS; c += C::CH) {
+                const int col = scol0 + c;
                 float f[C::CH];
 #pragma unroll
                 for (int j = 0; j < C::CH; j += 4) {
@@ -229,15 +249,47 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
         }
     } else if (warp == W_MMA) {
         // ================================================================ MMA issuer
-        if (lane == 0) {
+        // Per tile i: P V of tile i-1 (once its P is written; this releases its ring stage),
+        // A(i) = q~ k~^T (commit: the P epilogue may start), then, once the state of tile
+        // i-1 is decayed, O(i) = q~ S_prev and S += k~^T V (commit: the state epilogue may
+        // start).
+        {
+            const bool leader = elect_one();
+            // every lane waits; the vote keeps the warp's decision uniform
+            auto warp_wait = [&](uint64_t* bar, uint32_t parity, volatile int* ab) -> bool {
+                return __all_sync(0xffffffffu, mbar_wait_abort(bar, parity, ab));
+            };
             const uint32_t idA = idesc_bf16(64, 64, 0, 0);
             const uint32_t idO = idesc_bf16(64, DVT, 0, 1);
             const uint32_t idS = idesc_bf16(C::MS, DVT, 1, 1);
             const uint64_t dS0 = sw128_desc(smem_u32(sS), DK * 128, 1024);
-            for (int i = 0; i < ntiles; ++i) {
-                const int s = i % C::NS, b = i & 1;
-                if (!mbar_wait_abort(&bar_trans[s], (i / C::NS) & 1, abortp)) break;
-                if (MODE == 0 && i >= 2 && !mbar_wait_abort(&bar_tfree[b], ((i >> 1) - 1) & 1, abortp)) break;
+            const uint64_t dP = sw128_desc(smem_u32(sPb), 16, 1024);
+            auto issue_pv = [&](int j) -> bool {
+                const int sj = j % C::NS, aj = j % C::NAB;
+                if (!warp_wait(&bar_pready[j & 1], (j >> 1) & 1, abortp)) return false;
+                tc_fence_after();
+                const uint64_t dVj = sw128_desc(smem_u32(sm + sj * C::STAGE + C::QB + C::KB + C::GB), BLK, 1024);
+                const uint32_t tOj = tbase + C::COLS_S + aj * C::COLA + (16u << 16);
+                if (leader) {
+#pragma unroll
+                    for (int ks = 0; ks < TR / 16; ++ks)
+                        mma_bf16(tOj, dP + ((ks * 32) >> 4), dVj + ((ks * 2048) >> 4), idO, 1);
+                    mma_commit(&bar_mma2[aj]);
+                    *n_mma2 = j + 1;
+                    if (j + C::NS < ntiles) mma_commit(&bar_empty[sj]);
+                }
+                __syncwarp();
+                return true;
+            };
+            bool alive = true;
+            for (int i = 0; i < ntiles && alive; ++i) {
+                const int s = i % C::NS, b = i & 1, ab = i % C::NAB;
+                // P V of the previous tile first: it releases that tile's ring stage
+                if (MODE == 0 && i >= 1 && !issue_pv(i - 1)) break;
+                if (!warp_wait(&bar_trans[s], (i / C::NS) & 1, abortp)) break;
+                if (MODE == 0 && i >= C::NAB &&
+                    !warp_wait(&bar_tfree[ab], ((i / C::NAB) - 1) & 1, abortp))
+                    break;
                 tc_fence_after();
                 uint8_t* st = sm + s * C::STAGE;
                 // descriptors of the stage's tiles; K steps advance the 16-byte start field
@@ -245,56 +297,58 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 const uint64_t dKk = sw128_desc(smem_u32(st + C::QB), 16, 1024);       // k~, K-major
                 const uint64_t dKm = sw128_desc(smem_u32(st + C::QB), BLK, 1024);      // k~, MN-major
                 const uint64_t dV = sw128_desc(smem_u32(st + C::QB + C::KB + C::GB), BLK, 1024);
-                const uint32_t tAO = tbase + C::COLS_S + b * C::COLA;
-                if (MODE == 0) {
+                const uint32_t tAO = tbase + C::COLS_S + ab * C::COLA;
+                if (MODE == 0 && leader) {
 #pragma unroll
                     for (int kk = 0; kk < DK / 16; ++kk) {
                         const uint64_t ko = ((kk >> 2) * BLK + (kk & 3) * 32) >> 4;
                         mma_bf16(tAO, dQ + ko, dKk + ko, idA, kk > 0);
                     }
+                    mma_commit(&bar_aready[ab]);
                 }
+                __syncwarp();
                 // the state of the previous tile must be decayed (and copied) first
                 if (i >= 1) {
-                    if (!mbar_wait_abort(bar_sready, (i - 1) & 1, abortp)) break;
+                    if (!warp_wait(bar_sready, (i - 1) & 1, abortp)) break;
                     tc_fence_after();
                 }
-                if (MODE == 0) {
+                if (leader) {
+                    if (MODE == 0) {
 #pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk) {
-                        const uint64_t ko = ((kk >> 2) * BLK + (kk & 3) * 32) >> 4;
-                        mma_bf16(tAO + (16u << 16), dQ + ko, dS0 + ((kk * 2048) >> 4), idO, kk > 0);
+                        for (int kk = 0; kk < DK / 16; ++kk) {
+                            const uint64_t ko = ((kk >> 2) * BLK + (kk & 3) * 32) >> 4;
+                            mma_bf16(tAO + (16u << 16), dQ + ko, dS0 + ((kk * 2048) >> 4), idO, kk > 0);
+                        }
                     }
+#pragma unroll
+                    for (int h = 0; h < C::NH; ++h)
+#pragma unroll
+                        for (int ks = 0; ks < TR / 16; ++ks)
+                            mma_bf16(tbase + h * DVT, dKm + ((h * 2 * BLK + ks * 2048) >> 4),
+                                     dV + ((ks * 2048) >> 4), idS, 1);
+                    mma_commit(&bar_mma1[b]);
+                    *n_mma1 = i + 1;
+                    if (MODE != 0 && i + C::NS < ntiles) mma_commit(&bar_empty[s]);
                 }
-#pragma unroll
-                for (int h = 0; h < C::NH; ++h)
-#pragma unroll
-                    for (int ks = 0; ks < TR / 16; ++ks)
-                        mma_bf16(tbase + h * DVT, dKm + ((h * 2 * BLK + ks * 2048) >> 4), dV + ((ks * 2048) >> 4),
-                                 idS, 1);
-                mma_commit(&bar_mma1[b]);
-                *n_mma1 = i + 1;
-                if (MODE == 0) {
-                    if (!mbar_wait_abort(&bar_pready[b], (i >> 1) & 1, abortp)) break;
-                    tc_fence_after();
-                    const uint64_t dP = sw128_desc(smem_u32(sPb + b * (TR * TR * 2)), 16, 1024);
-#pragma unroll
-                    for (int ks = 0; ks < TR / 16; ++ks)
-                        mma_bf16(tAO + (16u << 16), dP + ((ks * 32) >> 4), dV + ((ks * 2048) >> 4), idO, 1);
-                    mma_commit(&bar_mma2[b]);
-                    *n_mma2 = i + 1;
-                }
-                if (i + C::NS < ntiles) mma_commit(&bar_empty[s]);
+                __syncwarp();
+                if (MODE == 0 && i == ntiles - 1) alive = issue_pv(i);
             }
         }
     } else if (!is_ep) {
         // ================================================================ transform warpgroups
-        // Step A: b = inclusive column cumsum of the log-gate, written over g in place (one
-        // thread per key dim). Step B: every 16-byte chunk (8 key dims of one row) of the
-        // q and k tiles is scaled in place by its exponentials and rounded to bf16.
+        // Step A: b = inclusive column cumsum of the log-gate, in row segments (thread = key
+        // dim x segment) joined through the segment totals, written over g in place in
+        // base-2 units (b * log2 e; MODE 2 writes (b - Gamma) * log2 e). Step B: every 16-byte
+        // chunk (8 key dims of one row) of the k tile, and of the q tile in the output pass,
+        // is scaled in place by its exponentials and rounded to bf16 (q also by the output
+        // scale, so that A, P and O carry it).
         const int ttid = tid - NEP;
         constexpr int NO = DK / 8;
-        constexpr int NQK = (MODE == 0 ? 2 : 1) * TR * NO;   // chunks of k (then q)
-        static_assert(NQK % NTRF == 0 && (TR * NO) % NTRF == 0, "chunk mapping");
+        constexpr int SEG = NTRF / DK, RS = TR / SEG;        // step A: segments, rows per segment
+        constexpr int NPOS = TR * NO;                        // step B: (row, chunk) positions
+        constexpr int NB = 2;                                // positions per batch of loads
+        static_assert(NPOS % (NB * NTRF) == 0 && TR % SEG == 0, "transform mapping");
+        const int dA = ttid % DK, sA = ttid / DK;
         for (int j = 0; j < ntiles; ++j) {
             const int s = j % C::NS, b = j & 1;
             uint8_t* st = sm + s * C::STAGE;
@@ -315,24 +369,34 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
             if (ttid == 0) *n_consumed = j + 1;
             // ---- step A
             if (GATE == 1) {
-                if (ttid < DK) {
-                    float* col = sg + ttid;
-                    float acc = 0.f;
+                float* col = sg + sA * RS * DK + dA;
+                float x[RS];
 #pragma unroll
-                    for (int r0 = 0; r0 < TR; r0 += 16) {
-                        float x[16];
+                for (int u = 0; u < RS; ++u) x[u] = col[u * DK];
+                float acc = 0.f;
 #pragma unroll
-                        for (int u = 0; u < 16; ++u) x[u] = col[(r0 + u) * DK];
+                for (int u = 0; u < RS; ++u) {
+                    acc += x[u];
+                    x[u] = acc;
+                }
+                float off = 0.f, G = acc;
+                if constexpr (SEG > 1) {
+                    tot[ttid] = acc;
+                    named_bar_sync(BAR_TR, NTRF);
+                    G = 0.f;
 #pragma unroll
-                        for (int u = 0; u < 16; ++u) {
-                            acc += x[u];
-                            x[u] = acc;
-                        }
-#pragma unroll
-                        for (int u = 0; u < 16; ++u) col[(r0 + u) * DK] = x[u];
+                    for (int s2 = 0; s2 < SEG; ++s2) {
+                        const float t = tot[s2 * DK + dA];
+                        if (s2 < sA) off += t;
+                        G += t;
                     }
-                    gam[ttid] = __expf(acc);
-                    gaml[ttid] = acc;
+                }
+                const float sub = MODE == 2 ? G - off : -off;
+#pragma unroll
+                for (int u = 0; u < RS; ++u) col[u * DK] = (x[u] - sub) * kLog2e;
+                if (sA == 0) {
+                    gam[dA] = __expf(G);
+                    gaml[dA] = G;
                 }
             } else if (GATE == 2) {
                 if (ttid < 32) {  // warp scan over 64 rows, two rows per lane
@@ -358,107 +422,140 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 }
             }
             named_bar_sync(BAR_TR, NTRF);
-            // ---- step B
+            // ---- step B: MODE 0/1 k -> i k e^-b, MODE 0 q -> q e^b, MODE 2 (q in the k slot) -> scale q e^(b-Gamma)
 #pragma unroll
-            for (int it = 0; it < NQK / NTRF; ++it) {
-                const int c = ttid + it * NTRF;
-                const bool is_q = MODE == 0 && it * NTRF >= TR * NO;   // uniform per iteration
-                const int rem = c % (TR * NO);
-                const int r = rem / NO, d0 = 8 * (rem % NO);
-                // MODE 0/1: k slot -> i k e^-b, q slot -> q e^b; MODE 2: k slot holds q -> scale q e^(b-Gamma)
-                const bool up = is_q || MODE == 2;
-                float e[8];
-                if (GATE == 1) {
-                    const float4 b0 = *reinterpret_cast<const float4*>(sg + r * DK + d0);
-                    const float4 b1 = *reinterpret_cast<const float4*>(sg + r * DK + d0 + 4);
-                    float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-                    if (MODE == 2) {
-                        const float4 G0 = *reinterpret_cast<const float4*>(gaml + d0);
-                        const float4 G1 = *reinterpret_cast<const float4*>(gaml + d0 + 4);
-                        bv[0] -= G0.x; bv[1] -= G0.y; bv[2] -= G0.z; bv[3] -= G0.w;
-                        bv[4] -= G1.x; bv[5] -= G1.y; bv[6] -= G1.z; bv[7] -= G1.w;
+            for (int it0 = 0; it0 < NPOS / NTRF; it0 += NB) {
+                float bv[NB][8];
+                uint4 wq[NB], wk[NB];
+                uint32_t offs[NB];
+                int rows[NB];
+#pragma unroll
+                for (int k = 0; k < NB; ++k) {
+                    const int c = ttid + (it0 + k) * NTRF;
+                    const int r = c / NO, d0 = 8 * (c % NO);
+                    rows[k] = r;
+                    if (GATE == 1) {
+                        const float4 b0 = *reinterpret_cast<const float4*>(sg + r * DK + d0);
+                        const float4 b1 = *reinterpret_cast<const float4*>(sg + r * DK + d0 + 4);
+                        bv[k][0] = b0.x; bv[k][1] = b0.y; bv[k][2] = b0.z; bv[k][3] = b0.w;
+                        bv[k][4] = b1.x; bv[k][5] = b1.y; bv[k][6] = b1.z; bv[k][7] = b1.w;
                     }
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) e[u] = __expf(up ? bv[u] : -bv[u]);
-                } else {
-                    const float f = GATE == 2 ? (up ? rowE[r] : rowEi[r]) : 1.f;
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) e[u] = f;
+                    offs[k] = (uint32_t)(d0 >> 6) * BLK + (uint32_t)r * 128 +
+                              ((((uint32_t)((d0 & 63) >> 3)) ^ (uint32_t)(r & 7)) << 4);
+                    if (MODE == 0) wq[k] = *reinterpret_cast<const uint4*>(sq + offs[k]);
+                    wk[k] = *reinterpret_cast<const uint4*>(sk + offs[k]);
                 }
-                const float m = MODE == 2 ? P.scale : (is_q ? 1.f : igs[r]);
-                const uint32_t off = (uint32_t)(d0 >> 6) * BLK + (uint32_t)r * 128 +
-                                     ((((uint32_t)((d0 & 63) >> 3)) ^ (uint32_t)(r & 7)) << 4);
-                uint4* p = reinterpret_cast<uint4*>((is_q ? sq : sk) + off);
-                uint4 w = *p;
-                uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wp[u]));
-                    __nv_bfloat162 h = __floats2bfloat162_rn(f.x * m * e[2 * u], f.y * m * e[2 * u + 1]);
-                    wp[u] = *reinterpret_cast<uint32_t*>(&h);
+                for (int k = 0; k < NB; ++k) {
+                    const int r = rows[k];
+                    const float mk = MODE == 2 ? P.scale : igs[r];
+                    float eu[8], ed[8];   // e^(+b) for q (MODE 0 and 2), e^(-b) for k (MODE 0 and 1)
+                    if (GATE == 1) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            eu[u] = MODE != 1 ? ex2_approx(bv[k][u]) : 1.f;
+                            ed[u] = MODE != 2 ? ex2_approx(-bv[k][u]) : 1.f;
+                        }
+                    } else {
+                        const float fu = GATE == 2 ? rowE[r] : 1.f, fd = GATE == 2 ? rowEi[r] : 1.f;
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            eu[u] = fu;
+                            ed[u] = fd;
+                        }
+                    }
+                    uint32_t* pk = reinterpret_cast<uint32_t*>(&wk[k]);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&pk[u]));
+                        const float e0 = MODE == 2 ? eu[2 * u] : ed[2 * u];
+                        const float e1 = MODE == 2 ? eu[2 * u + 1] : ed[2 * u + 1];
+                        __nv_bfloat162 h = __floats2bfloat162_rn(f.x * mk * e0, f.y * mk * e1);
+                        pk[u] = *reinterpret_cast<uint32_t*>(&h);
+                    }
+                    *reinterpret_cast<uint4*>(sk + offs[k]) = wk[k];
+                    if (MODE == 0) {
+                        uint32_t* pq = reinterpret_cast<uint32_t*>(&wq[k]);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&pq[u]));
+                            __nv_bfloat162 h =
+                                __floats2bfloat162_rn(f.x * P.scale * eu[2 * u], f.y * P.scale * eu[2 * u + 1]);
+                            pq[u] = *reinterpret_cast<uint32_t*>(&h);
+                        }
+                        *reinterpret_cast<uint4*>(sq + offs[k]) = wq[k];
+                    }
                 }
-                *p = w;
             }
             fence_proxy_async_smem();
             named_bar_sync(BAR_TR, NTRF);
             if (ttid == 0) mbar_arrive(&bar_trans[s]);
         }
-    } else {
-        // ================================================================ epilogue warpgroups
-        const int etid = tid;
+    } else if (s_worker) {
+        // ================================================================ state epilogue
+        // S = e^Gamma (S_prev + dS'), where the MMA has added dS' onto S_prev in TMEM; the
+        // decayed state goes back to TMEM and, as bf16, to shared memory (next tile's q~ S)
         const uint32_t lq = (uint32_t)(32 * qd) << 16;   // this warp's TMEM lane quadrant
         for (int i = 0; i < ntiles; ++i) {
             const int b = i & 1;
-            const uint32_t tAO = tbase + C::COLS_S + b * C::COLA;
             {
                 const bool ok = mbar_wait_abort(&bar_mma1[b], (i >> 1) & 1, abortp);
-                if (!named_bar_and(BAR_EP, NEP, ok)) break;
+                if (!named_bar_and(BAR_S, C::NSW, ok)) break;
+            }
+            tc_fence_after();
+            const float* gam = gamb + b * DK;
+            const float* gaml = gamlb + b * DK;
+#pragma unroll
+            for (int h = 0; h < C::NH; ++h) {
+                const int d = srow(h);
+                const int gi = GATE == 1 ? d : 0;
+                const float egv = GATE == 0 ? 1.f : gam[gi];
+                if (GATE != 0) glog[h] += gaml[gi];
+#pragma unroll
+                for (int c = 0; c < C::SCOLS; c += C::CH) {
+                    const int col = scol0 + c;
+                    float f[C::CH];
+                    uint32_t* r = reinterpret_cast<uint32_t*>(f);
+                    tmem_ldn<C::CH>(tbase + lq + h * DVT + col, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < C::CH; ++j) f[j] *= egv;
+                    tmem_stn<C::CH>(tbase + lq + h * DVT + col, r);
+                    if (MODE == 0 && srow_ok)
+#pragma unroll
+                        for (int j = 0; j < C::CH; j += 8) store8_bf16(sS, sw128_off(d, col + j, DK * 128), &f[j]);
+                }
+            }
+            tmem_wait_st();
+            if (MODE == 0) fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(BAR_S, C::NSW);
+            if (tid == 0) {
+                mbar_arrive(bar_sready);
+                mbar_arrive(&bar_gfree[b]);
+            }
+        }
+    } else if (MODE == 0 && is_ep) {
+        // ================================================================ P and output epilogue
+        const uint32_t lq = (uint32_t)(32 * qd) << 16;
+        const int ptid = tid - 128;
+        for (int i = 0; i < ntiles; ++i) {
+            const int b = i & 1;
+            const int ab = i % C::NAB;
+            const uint32_t tAO = tbase + C::COLS_S + ab * C::COLA;
+            {
+                const bool ok = mbar_wait_abort(&bar_aready[ab], (i / C::NAB) & 1, abortp);
+                if (!named_bar_and(BAR_PO, 128, ok)) break;
             }
             tc_fence_after();
             const int t0 = tile_at(i) * TR;
-            // ---- state: S = e^Gamma (S_prev + dS'), where the MMA has added dS' onto S_prev
-            //      in TMEM; the decayed state goes back to TMEM and, as bf16, to shared memory
+            // ---- P = causal mask of A -> shared (single buffer: P V of the previous tile is
+            //      complete, its output pass waited for it)
             {
-                const float* gam = gamb + b * DK;
-                const float* gaml = gamlb + b * DK;
+                uint8_t* sP = sPb;
 #pragma unroll
-                for (int h = 0; h < C::NH; ++h) {
-                    const int d = srow(h);
-                    const int gi = GATE == 1 ? d : 0;
-                    const float egv = GATE == 0 ? 1.f : gam[gi];
-                    if (GATE != 0) glog[h] += gaml[gi];
-#pragma unroll
-                    for (int c = 0; c < C::HALF; c += C::CH) {
-                        const int col = wg * C::HALF + c;
-                        float f[C::CH];
-                        uint32_t* r = reinterpret_cast<uint32_t*>(f);
-                        tmem_ldn<C::CH>(tbase + lq + h * DVT + col, r);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < C::CH; ++j) f[j] *= egv;
-                        tmem_stn<C::CH>(tbase + lq + h * DVT + col, r);
-                        if (MODE == 0 && srow_ok)
-#pragma unroll
-                            for (int j = 0; j < C::CH; j += 8) store8_bf16(sS, sw128_off(d, col + j, DK * 128), &f[j]);
-                    }
-                }
-                tmem_wait_st();
-                if (MODE == 0) fence_proxy_async_smem();
-                tc_fence_before();
-                named_bar_sync(BAR_EP, NEP);
-                if (etid == 0) {
-                    mbar_arrive(bar_sready);
-                    mbar_arrive(&bar_gfree[b]);
-                }
-            }
-            if (MODE != 0) continue;
-            // ---- P = causal mask of A -> shared (double-buffered)
-            {
-                uint8_t* sP = sPb + b * (TR * TR * 2);
-#pragma unroll
-                for (int c = 0; c < C::PCOLS; c += C::CH) {
+                for (int c0 = 0; c0 < TR; c0 += C::CH) {
                     uint32_t r[C::CH];
-                    const int c0 = wg * C::PCOLS + c;
                     tmem_ldn<C::CH>(tAO + lq + c0, r);
                     tmem_wait_ld();
                     if (lane < 16) {
@@ -476,41 +573,35 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     }
                 }
                 fence_proxy_async_smem();
-                named_bar_sync(BAR_EP, NEP);
-                if (etid == 0) mbar_arrive(&bar_pready[b]);
+                named_bar_sync(BAR_PO, 128);
+                if (ptid == 0) mbar_arrive(&bar_pready[b]);
             }
-            // ---- output tile
+            // ---- output tile: TMEM -> bf16 tile in shared memory -> TMA store
             {
-                const bool ok = mbar_wait_abort(&bar_mma2[b], (i >> 1) & 1, abortp);
-                if (!named_bar_and(BAR_EP, NEP, ok)) break;
+                bool ok = mbar_wait_abort(&bar_mma2[ab], (i / C::NAB) & 1, abortp);
+                if (ptid == 0) bulk_wait_read<0>();   // the previous tile's store has read the staging tile
+                if (!named_bar_and(BAR_PO, 128, ok)) break;
                 tc_fence_after();
                 const int t = 16 * qd + (lane & 15);
-                const bool row_ok = (lane >= 16) && (t0 + t < P.L);
-                __nv_bfloat16* orow = A.o + (rowbase + t0 + t) * P.Dv + e0 + wg * C::HALF;
 #pragma unroll
-                for (int c = 0; c < C::HALF; c += C::CH) {
+                for (int c = 0; c < DVT; c += C::CH) {
                     uint32_t r[C::CH];
-                    tmem_ldn<C::CH>(tAO + lq + wg * C::HALF + c, r);
+                    tmem_ldn<C::CH>(tAO + lq + c, r);
                     tmem_wait_ld();
-                    if (row_ok) {
+                    if (lane >= 16)
 #pragma unroll
-                        for (int u = 0; u < C::CH / 8; ++u) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int p2 = 0; p2 < 4; ++p2) {
-                                __nv_bfloat162 b2 =
-                                    __floats2bfloat162_rn(P.scale * __uint_as_float(r[8 * u + 2 * p2]),
-                                                          P.scale * __uint_as_float(r[8 * u + 2 * p2 + 1]));
-                                w[p2] = *reinterpret_cast<uint32_t*>(&b2);
-                            }
-                            *reinterpret_cast<uint4*>(orow + c + 8 * u) = make_uint4(w[0], w[1], w[2], w[3]);
-                        }
-                    }
+                        for (int u = 0; u < C::CH / 8; ++u)
+                            store8_bf16(sO, sw128_off(t, c + 8 * u, BLK), reinterpret_cast<const float*>(&r[8 * u]));
                 }
+                fence_proxy_async_smem();
             }
             tc_fence_before();
-            named_bar_sync(BAR_EP, NEP);
-            if (etid == 0) mbar_arrive(&bar_tfree[b]);
+            named_bar_sync(BAR_PO, 128);
+            if (ptid == 0) {
+                for (int vb = 0; vb < DVT / 64; ++vb) tma_store_3d(&to, sO + vb * BLK, e0 + 64 * vb, t0, bh);
+                bulk_commit();
+            }
+            if (ptid == 0) mbar_arrive(&bar_tfree[ab]);
         }
     }
 
@@ -524,9 +615,9 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
             for (int j = *n_consumed; j < *n_issued; ++j)
                 mbar_wait(&bar_full[j % C::NS], (j / C::NS) & 1, 1u << 20);
             if (*n_mma1) mbar_wait(&bar_mma1[(*n_mma1 - 1) & 1], ((*n_mma1 - 1) >> 1) & 1, 1u << 20);
-            if (*n_mma2) mbar_wait(&bar_mma2[(*n_mma2 - 1) & 1], ((*n_mma2 - 1) >> 1) & 1, 1u << 20);
+            if (*n_mma2) mbar_wait(&bar_mma2[(*n_mma2 - 1) % C::NAB], ((*n_mma2 - 1) / C::NAB) & 1, 1u << 20);
         }
-    } else if (is_ep) {
+    } else if (s_worker) {
         // final state of the segment, read back from TMEM
 #pragma unroll
         const uint32_t lq = (uint32_t)(32 * qd) << 16;
@@ -537,12 +628,12 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 if (z == A.nseg - 1 && A.hT) dst = A.hT + ((long)bh * DK + d) * P.Dv;
             } else {
                 dst = A.seg_state + (((long)bh * A.nseg + z) * DK + d) * P.Dv;
-                if (vt == 0 && wg == 0 && srow_ok) A.seg_gamma[((long)bh * A.nseg + z) * DK + d] = glog[h];
+                if (vt == 0 && scol0 == 0 && srow_ok) A.seg_gamma[((long)bh * A.nseg + z) * DK + d] = glog[h];
             }
             if (!dst) continue;
 #pragma unroll
-            for (int c = 0; c < C::HALF; c += C::CH) {
-                const int col = wg * C::HALF + c;
+            for (int c = 0; c < C::SCOLS; c += C::CH) {
+                const int col = scol0 + c;
                 float f[C::CH];
                 tmem_ldn<C::CH>(tbase + lq + h * DVT + col, reinterpret_cast<uint32_t*>(f));
                 tmem_wait_ld();
@@ -553,6 +644,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
             }
         }
     }
+    if (MODE == 0 && tid == 128) bulk_wait<0>();   // the last output stores have completed
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, C::NCOL);
@@ -604,7 +696,8 @@ __global__ void __launch_bounds__(256) k_seg_rscan(const float* __restrict__ seg
 // ------------------------------------------------------------------ host side
 template <int DK, int DVT, int GATE, int MODE>
 static cudaError_t launch_one(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                              const CUtensorMap& mg, const FwdArgs& a, const Dims& P, int nseg, cudaStream_t st) {
+                              const CUtensorMap& mg, const CUtensorMap& mo, const FwdArgs& a, const Dims& P, int nseg,
+                              cudaStream_t st) {
     using C = Cfg<DK, DVT, GATE, MODE>;
     auto kern = k_tc_fwd<DK, DVT, GATE, MODE>;
     static bool attr = false;
@@ -615,7 +708,7 @@ static cudaError_t launch_one(const CUtensorMap& mq, const CUtensorMap& mk, cons
     }
     dim3 grid(P.B * P.H, P.Dv / DVT, nseg);
     GLA_LAUNCH(MODE == 0 ? "tc_fwd" : MODE == 1 ? "tc_state" : "tc_gstate", st,
-               kern<<<grid, NTHR_WS, C::SMEM, st>>>(mq, mk, mv, mg, a, P));
+               kern<<<grid, NTHR_WS, C::SMEM, st>>>(mq, mk, mv, mg, mo, a, P));
     return cudaGetLastError();
 }
 
@@ -696,19 +789,20 @@ static cudaError_t state_run(const Dims& P, int mode, const void* a_src, const v
     a.tiles_per_seg = tps;
     a.nseg = nseg;
     a.seg_offset = mode == 1 ? 0 : 1;
-    if (mode == 1) return launch_one<DK, DVT, GATE, 1>(mk, mk, mv, mg, a, P, nseg - 1, st);
-    return launch_one<DK, DVT, GATE, 2>(mk, mk, mv, mg, a, P, nseg - 1, st);
+    if (mode == 1) return launch_one<DK, DVT, GATE, 1>(mk, mk, mv, mg, mk, a, P, nseg - 1, st);
+    return launch_one<DK, DVT, GATE, 2>(mk, mk, mv, mg, mk, a, P, nseg - 1, st);
 }
 
 template <int DK, int DVT, int GATE>
 static cudaError_t run(const Dims& P, const void* q, const void* k, const void* v, const float* g,
                        const float* ig, const float* h0, void* o, float* hT, void* ws, cudaStream_t st) {
     const FwdPlan pl = plan_fwd(P);
-    CUtensorMap mq, mk, mv, mg;
+    CUtensorMap mq, mk, mv, mg, mo;
     const int BH = P.B * P.H;
     if (!make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dk, P.L, BH, 64, true) ||
         !make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dk, P.L, BH, 64, true) ||
-        !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dv, P.L, BH, 64, true))
+        !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dv, P.L, BH, 64, true) ||
+        !make_map(&mo, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dv, P.L, BH, 64, true))
         return cudaErrorInvalidValue;
     if (GATE == 1) {
         if (!make_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, P.Dk, P.L, BH, P.Dk, false))
@@ -741,7 +835,7 @@ static cudaError_t run(const Dims& P, const void* q, const void* k, const void* 
         e = seg_scan(P, pl.nseg, seg_state, seg_gamma, h0, sinit, st);
         if (e != cudaSuccess) return e;
     }
-    return launch_one<DK, DVT, GATE, 0>(mq, mk, mv, mg, a, P, pl.nseg, st);
+    return launch_one<DK, DVT, GATE, 0>(mq, mk, mv, mg, mo, a, P, pl.nseg, st);
 }
 
 cudaError_t seg_scan(const Dims& P, int nseg, const float* seg_state, const float* seg_gamma, const float* h0,
