@@ -72,16 +72,28 @@ def compulsory_bytes(w, backward):
     return float(fwd + bwd)
 
 
-def kernel_bytes(name, w):
+def _mean(xs):
+    return sum(xs) / len(xs) if xs else 0.0
+
+
+def kernel_bytes(name, w, fseg=1, bseg=1):
     """Algorithmic bytes of one launch of each kernel: its own inputs read once and its
-    outputs written once (workspace tensors it exchanges with other kernels included)."""
+    outputs written once, workspace tensors it exchanges with other kernels included.
+    fseg / bseg: sequence segments of the forward / backward plan (gla_plan_info)."""
     th = w.B * w.H * w.L
+    BH = w.B * w.H
     e = io_bytes(w)
     ge = 4 * th * gate_elems(w)
+    ig = 4 * th if w.input_gate else 0
     N = math.ceil(w.L / w.chunk)
-    states = 4.0 * w.B * w.H * N * w.Dk * w.Dv
+    s1 = 4.0 * BH * w.Dk * w.Dv                  # one fp32 state per head
+    h0 = s1 if w.h0_std > 0 else 0
+    states = s1 * N
     q = k = th * w.Dk * e
     v = o = th * w.Dv * e
+    dgb = 4 * th * gate_elems(w)                 # fp32 dg (or its in-segment prefix)
+    frac_f = (fseg - 1) / fseg                    # share of the sequence the state passes cover
+    frac_b = (bseg - 1) / bseg
     table = {
         "simt_cumsum": 2 * ge,
         "simt_state": k + v + ge + states,
@@ -91,7 +103,17 @@ def kernel_bytes(name, w):
         "simt_dk": q + k + v + o + ge + states + k + 2 * 4 * th * w.Dk,
         "simt_dv": q + k + o + ge + states + v,
         "simt_dg_key": 2 * 4 * th * w.Dk,
-        "tc_fwd": q + k + v + ge + o + 4 * w.B * w.H * w.Dk * w.Dv * (2 if w.h0_std > 0 else 1),
+        # forward: state pass over segments 0..nseg-2, scan, output pass (reads the segment initial states)
+        "tc_fwd": q + k + v + ge + ig + o + s1 + h0 + s1 * (fseg - 1),
+        "tc_seg_scan": _mean([2 * s1 * (fseg - 1) + h0] * (fseg > 1) + [2 * s1 * (bseg - 1) + h0] * (bseg > 1)),
+        # the backward's own forward-state pass / reverse state-gradient pass and scans
+        # the forward and the backward plan may both launch a state pass: bytes per launch averaged
+        "tc_state": _mean([frac_f * (k + v + ge + ig) + s1 * (fseg - 1)] * (fseg > 1) +
+                          [frac_b * (k + v + ge + ig) + s1 * (bseg - 1)] * (bseg > 1)),
+        "tc_gstate": frac_b * (q + o + ge) + s1 * (bseg - 1),
+        "tc_seg_rscan": 2 * s1 * (bseg - 1) + s1,
+        "tc_bwd_dq": q + k + v + o + ge + ig + s1 * bseg + h0 + q + dgb + s1 + 4 * BH * bseg * w.Dk,
+        "tc_bwd_dkdv": q + k + v + o + ge + ig + 2 * s1 * bseg + dgb + 4 * BH * bseg * w.Dk + s1 + k + v + dgb + ig + h0,
     }
     return float(table.get(name, 0.0))
 
@@ -252,10 +274,14 @@ def main():
     ap.add_argument("--plan", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch B (smaller cases for profiling; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     w = I.WORKLOADS[args.workload]
+    if args.batch is not None:
+        w = w.replace(B=args.batch)
     world, rank, local = dist_setup()
     if args.impl == "reference":
         run_reference(args, w, world, rank)
@@ -270,6 +296,9 @@ def main():
     xd = {k: (None if v is None else v.to(dev)) for k, v in x.items()}
     kw = dict(scale=w.scale, chunk=w.chunk, plan=args.plan)
     prob = ops.make_problem(xd["q"], xd["v"], xd["g"], **kw)
+    _, fseg, _ = _lib.plan_info(prob, False)
+    bplan, bseg, _ = _lib.plan_info(prob, True)
+    bseg = bseg if (w.backward and bplan == _lib.GLA_PLAN_TC) else 1
     ws = torch.empty(max(ops.gla_workspace_bytes(prob, False), ops.gla_workspace_bytes(prob, True) if w.backward
                          else 0), dtype=torch.uint8, device=dev)
 
@@ -361,7 +390,7 @@ def main():
     if dom:
         name, (cnt, ms) = dom
         avg_s = ms / cnt / 1e3
-        kb = kernel_bytes(name, w)
+        kb = kernel_bytes(name, w, fseg, bseg)
         ach = kb / avg_s / 1e9
         share = ms / sum(v[1] for v in kprof.values())
         roofline = {"bound": "hbm", "kernel": name, "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",

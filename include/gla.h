@@ -130,6 +130,15 @@ GLA_API const char* gla_last_error_detail(void);
 /* Library version as 10000*major + 100*minor + patch. */
 GLA_API int gla_version(void);
 
+/* How gla_fwd (for_backward = 0) or gla_bwd (1) would run `p`, for measurement and
+ * capacity planning: *plan_out = the resolved GLA_PLAN_SIMT or GLA_PLAN_TC; *nseg_out =
+ * sequence segments processed in parallel (1 = one pass over the whole sequence);
+ * *tiles_out = 64-token tiles per segment (the chunk count for the SIMT plan). Any output
+ * pointer may be NULL. Returns the same status that gla_fwd / gla_bwd would return for an
+ * invalid or unsupported problem, else GLA_OK. Launches nothing. */
+GLA_API gla_status gla_plan_info(const gla_problem* p, int for_backward, int* plan_out, int* nseg_out,
+                                 int* tiles_out);
+
 /* Forward pass that allocates nothing, for callers that cannot allocate device memory
  * themselves (for example a host whose device memory is all owned by another allocator
  * under a fixed budget, or code that must not call cudaMalloc because it synchronises the

@@ -19,7 +19,7 @@ GLA_PLAN_AUTO, GLA_PLAN_SIMT, GLA_PLAN_TC = 0, 1, 2
 # Every symbol include/gla.h declares (checked by tests/test_abi_symbols.py).
 EXPORTED = ("gla_workspace_bytes", "gla_fwd", "gla_bwd", "gla_status_string",
             "gla_check_device_status", "gla_version", "gla_launch_count", "gla_profiler_enable",
-            "gla_profiler_read", "gla_fwd_static_scratch", "gla_last_error_detail")
+            "gla_profiler_read", "gla_fwd_static_scratch", "gla_last_error_detail", "gla_plan_info")
 
 
 class GlaProblem(ctypes.Structure):
@@ -65,6 +65,9 @@ def _load():
     lib.gla_last_error_detail.restype = ctypes.c_char_p
     lib.gla_fwd_static_scratch.argtypes = [pp, vp, vp, vp, fp, fp, fp, vp, fp, vp]
     lib.gla_fwd_static_scratch.restype = ctypes.c_int
+    ip = ctypes.POINTER(ctypes.c_int)
+    lib.gla_plan_info.argtypes = [pp, ctypes.c_int, ip, ip, ip]
+    lib.gla_plan_info.restype = ctypes.c_int
     lib.gla_launch_count.argtypes = []
     lib.gla_launch_count.restype = ctypes.c_ulonglong
     lib.gla_profiler_enable.argtypes = [ctypes.c_int]
@@ -101,3 +104,13 @@ def profiler_read(max_kernels: int = 64):
 
 def launch_count() -> int:
     return int(lib.gla_launch_count())
+
+
+def plan_info(problem: GlaProblem, for_backward: bool):
+    """(plan, nseg, tiles_per_seg) that gla_fwd / gla_bwd would use; GlaError if invalid."""
+    plan, nseg, tiles = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    st = lib.gla_plan_info(ctypes.byref(problem), int(for_backward), ctypes.byref(plan), ctypes.byref(nseg),
+                           ctypes.byref(tiles))
+    if st != GLA_OK:
+        raise GlaError(st, "gla_plan_info")
+    return plan.value, nseg.value, tiles.value

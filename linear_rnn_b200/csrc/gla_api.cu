@@ -202,6 +202,29 @@ gla_status gla_check_device_status(void* ws, void* stream) {
 
 int gla_version(void) { return 100; }
 
+gla_status gla_plan_info(const gla_problem* p, int for_backward, int* plan_out, int* nseg_out, int* tiles_out) {
+    Dims P;
+    int plan;
+    gla_status s = check_problem(p, &P, &plan);
+    if (s != GLA_OK) return s;
+    s = resolve(p, P, for_backward != 0, &plan);
+    if (s != GLA_OK) return s;
+    int nseg = 1, tiles = P.N;
+    if (plan == GLA_PLAN_TC) {
+        if (for_backward) {
+            tc::bwd_plan_info(P, &nseg, &tiles);
+        } else {
+            const tc::FwdPlan pl = tc::plan_fwd(P);
+            nseg = pl.nseg;
+            tiles = pl.tiles_per_seg;
+        }
+    }
+    if (plan_out) *plan_out = plan;
+    if (nseg_out) *nseg_out = nseg;
+    if (tiles_out) *tiles_out = tiles;
+    return GLA_OK;
+}
+
 const char* gla_last_error_detail(void) { return g_last_detail; }
 
 unsigned long long gla_launch_count(void) {

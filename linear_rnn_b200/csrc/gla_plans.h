@@ -39,6 +39,7 @@ int num_sms();
 // Backward (gla_tc_bwd.cu)
 bool bwd_supports(const Dims& P);
 size_t bwd_workspace_bytes(const Dims& P);
+void bwd_plan_info(const Dims& P, int* nseg, int* tiles_per_seg);
 cudaError_t bwd(const Dims& P, const void* q, const void* k, const void* v, const float* g, const float* ig,
                 const float* h0, const void* dO, const float* dhT, void* dq, void* dk, void* dv, float* dg, float* di,
                 float* dh0, void* ws, cudaStream_t st);

@@ -1003,6 +1003,12 @@ static BwdWs bwd_layout(const Dims& P, char* base) {
 
 size_t bwd_workspace_bytes(const Dims& P) { return bwd_layout(P, nullptr).total; }
 
+void bwd_plan_info(const Dims& P, int* nseg, int* tiles_per_seg) {
+    const BwdPlan pl = plan_bwd(P);
+    *nseg = pl.nseg;
+    *tiles_per_seg = pl.tiles_per_seg;
+}
+
 template <int DKB, int DV, int GATE>
 static cudaError_t launch_dq(const Dims& P, const BwdPlan& pl, const CUtensorMap& mq, const CUtensorMap& mk,
                              const CUtensorMap& mg, const CUtensorMap& mv, const CUtensorMap& mo, const BwdArgs& a,
