@@ -18,6 +18,7 @@ ranks. `--impl reference` times the float64 CPU oracle on a bounded sample inste
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -116,6 +117,31 @@ def kernel_bytes(name, w, fseg=1, bseg=1):
         "tc_bwd_dkdv": q + k + v + o + ge + ig + 2 * s1 * bseg + dgb + 4 * BH * bseg * w.Dk + s1 + k + v + dgb + ig + h0,
     }
     return float(table.get(name, 0.0))
+
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one ncu capture
+# (summaries under profiles/), with the SHA-256 prefix of the kernel's source file at capture
+# time: a kernel whose source has changed since reports traffic null. `scale`: the capture
+# ran a smaller case of the same workload; traffic grows with the heads processed.
+MEASURED_TRAFFIC = {
+    ("tc_bwd_dkdv", "c3"): {"bytes": 247e6, "scale": 4, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
+                            "sha": "884daa7fc0af09b6", "profile": "profiles/tc_bwd_dkdv_c3_b1.md"},
+    ("tc_fwd", "c2"): {"bytes": 188.7e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_fwd.cu",
+                       "sha": "4a086ac9bf5840d7", "profile": "profiles/tc_fwd_c2.md"},
+}
+
+
+def measured_traffic(kernel, workload):
+    m = MEASURED_TRAFFIC.get((kernel, workload))
+    if not m:
+        return None
+    try:
+        with open(os.path.join(ROOT, m["src"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest()[:16] != m["sha"]:
+                return None
+    except OSError:
+        return None
+    return m["bytes"] * m["scale"]
 
 
 def load_peaks():
@@ -394,7 +420,9 @@ def main():
         ach = kb / avg_s / 1e9
         share = ms / sum(v[1] for v in kprof.values())
         roofline = {"bound": "hbm", "kernel": name, "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": ach / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
+                    "frac": ach / peaks["hbm_gbs"], "traffic": measured_traffic(name, w.name if args.batch is None
+                                                                                 else None),
+                    "peak_source": peak_src,
                     "algorithmic_bytes_per_launch": kb, "avg_launch_us": avg_s * 1e6, "share_of_step": share}
     line = base_line(w, args, world)
     line.update({"value": value, "ms_per_step": total_ms / args.steps, "e2e": e2e, "gpu_launches": int(launches),
