@@ -335,19 +335,22 @@ def main():
                         **kw)
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
+    # warm-up right before the timed steps (same pattern, flush included), so that the timed
+    # region starts with warm clocks and the host already ahead of the device
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        step()
+    torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     n0 = _lib.launch_count()
     _lib.profiler_enable(True)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    flush.fill_(0xA5)   # lead-in (outside the events): the host queues step 0 while this runs
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
         ev[i][0].record()
