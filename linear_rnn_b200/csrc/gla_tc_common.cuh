@@ -11,6 +11,30 @@ namespace tc {
 constexpr int TR = 64;          // tokens per tile
 constexpr uint32_t BLK = 8192;  // one 64-column bf16 block of a 64-row tile (64 x 128 B)
 
+// Packed pairs of fp32 in one 64-bit register, multiplied lane-wise by the sm_100 packed
+// fp32 instruction (IEEE round-to-nearest per lane, like two separate multiplies).
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// bf16 pair (element 0 in the low half) -> fp32 pair
+__device__ __forceinline__ uint64_t bf2_to_f2(uint32_t w) {
+    return f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+// fp32 pair -> bf16 pair, round to nearest even
+__device__ __forceinline__ uint32_t f2_to_bf2(uint64_t x) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
 __device__ __forceinline__ void store8_bf16(uint8_t* base, uint32_t off, const float* v) {
     uint32_t w[4];
 #pragma unroll
