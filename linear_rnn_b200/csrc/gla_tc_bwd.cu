@@ -94,8 +94,8 @@ __device__ __forceinline__ void bwd_transform(uint8_t* sq, uint8_t* sk, float* s
     if (GATE == 1) {
 #pragma unroll 4
         for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
-            const float4 g0 = *reinterpret_cast<const float4*>(sg + r * D + d0);
-            const float4 g1 = *reinterpret_cast<const float4*>(sg + r * D + d0 + 4);
+            const float4 g0 = *reinterpret_cast<const float4*>(sg + gsw(r, d0));
+            const float4 g1 = *reinterpret_cast<const float4*>(sg + gsw(r, d0 + 4));
             bb[0] += g0.x; bb[1] += g0.y; bb[2] += g0.z; bb[3] += g0.w;
             bb[4] += g1.x; bb[5] += g1.y; bb[6] += g1.z; bb[7] += g1.w;
         }
@@ -144,8 +144,9 @@ __device__ __forceinline__ void bwd_transform(uint8_t* sq, uint8_t* sk, float* s
     for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
         float eq[8], ek[8];
         if (GATE == 1) {
-            float4* gp = reinterpret_cast<float4*>(sg + r * D + d0);
-            const float4 g0 = gp[0], g1 = gp[1];
+            float4* gp0 = reinterpret_cast<float4*>(sg + gsw(r, d0));
+            float4* gp1 = reinterpret_cast<float4*>(sg + gsw(r, d0 + 4));
+            const float4 g0 = *gp0, g1 = *gp1;
             const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
@@ -154,8 +155,8 @@ __device__ __forceinline__ void bwd_transform(uint8_t* sq, uint8_t* sk, float* s
                 ek[u] = __expf(-bb[u]);
             }
             const float* keep = G_SLOT_EB ? eq : ek;
-            gp[0] = make_float4(keep[0], keep[1], keep[2], keep[3]);
-            gp[1] = make_float4(keep[4], keep[5], keep[6], keep[7]);
+            *gp0 = make_float4(keep[0], keep[1], keep[2], keep[3]);
+            *gp1 = make_float4(keep[4], keep[5], keep[6], keep[7]);
         } else {
             const float e1 = GATE == 2 ? rowE[r] : 1.f, e2 = GATE == 2 ? rowEi[r] : 1.f;
 #pragma unroll
@@ -221,7 +222,8 @@ template <int DKB, int DV, int GATE>
 __global__ void __launch_bounds__(NT_B, 1)
     k_tc_bwd_dq(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tg, const __grid_constant__ CUtensorMap tv,
-                const __grid_constant__ CUtensorMap tdo, BwdArgs A, Dims P) {
+                const __grid_constant__ CUtensorMap tdo, const __grid_constant__ CUtensorMap tout, BwdArgs A,
+                Dims P) {
     using C = QCfg<DKB, DV, GATE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = smem_align1024(smem_raw);
@@ -300,7 +302,9 @@ __global__ void __launch_bounds__(NT_B, 1)
             if (GATE != 0) tma_load_3d(st + cb * BLK, &tq, d0 + cb * 64, t0, bh, &bar_full[s]);
             tma_load_3d(st + C::QB + cb * BLK, &tk, d0 + cb * 64, t0, bh, &bar_full[s]);
         }
-        if (GATE == 1) tma_load_3d(st + C::QB + C::KB, &tg, d0, t0, bh, &bar_full[s]);
+        if (GATE == 1)
+            for (int gb = 0; gb < DKB / 32; ++gb)
+                tma_load_3d(st + C::QB + C::KB + gb * BLK, &tg, d0 + 32 * gb, t0, bh, &bar_full[s]);
         for (int vb = 0; vb < DV / 64; ++vb) {
             tma_load_3d(st + C::QB + C::KB + C::GB + vb * BLK, &tv, vb * 64, t0, bh, &bar_full[s]);
             tma_load_3d(st + C::QB + C::KB + C::GB + C::VB + vb * BLK, &tdo, vb * 64, t0, bh, &bar_full[s]);
@@ -420,96 +424,120 @@ __global__ void __launch_bounds__(NT_B, 1)
         if (!block_wait(bar_mma2, i & 1)) { err = 1; break; }
         tc_fence_after();
 
-        // ---- dq = scale e^b D
+        // ---- dq = scale e^b D -> bf16 tile staged in the k slot (k~ is no longer read) -> TMA
+        //      store; q*dq into the g slot for dg. Row t of D sits in TMEM lane 16 + (t % 16) of
+        //      quadrant t / 16; the g slot holds e^b in the swizzled fp32 layout (gsw).
         {
             const int t = 16 * qd + (lane & 15);
-            const bool row_ok = lane >= 16 && t0 + t < P.L;
+            const bool row_ok = t0 + t < P.L;
+            uint8_t* sdq = sk;
             for (int c = wg * C::QC; c < (wg + 1) * C::QC; c += 16) {
                 uint32_t r[16];
                 tmem_ld16(tlane + C::COL_R + c, r);
                 tmem_wait_ld();
-                if (row_ok) {
+                if (lane >= 16) {
+                    float eb[16];
+                    if (GATE == 1) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const float4 e4 = *reinterpret_cast<const float4*>(sg + gsw(t, c + 4 * q4));
+                            eb[4 * q4] = e4.x; eb[4 * q4 + 1] = e4.y; eb[4 * q4 + 2] = e4.z; eb[4 * q4 + 3] = e4.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) eb[j] = GATE == 2 ? rowE[t] : 1.f;
+                    }
                     float f[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float eb = GATE == 1 ? sg[t * DKB + c + j] : (GATE == 2 ? rowE[t] : 1.f);
-                        f[j] = P.scale * eb * __uint_as_float(r[j]);
-                    }
-                    store16_bf16_global(A.dq + (rowbase + t0 + t) * P.Dk + d0 + c, f);
-                    // q*dq for dg, formed as bf16(scale q e^b) * D with the same rounding the dk/dv
-                    // kernel applies to q~, so the pairwise cancellation inside dg's reverse sum
-                    // survives the bf16 operands
-                    if (GATE != 0)
+                    for (int j = 0; j < 16; ++j) f[j] = P.scale * eb[j] * __uint_as_float(r[j]);
+                    store8_bf16(sdq, sw128_off(t, c, BLK), f);
+                    store8_bf16(sdq, sw128_off(t, c + 8, BLK), f + 8);
+                    if (GATE != 0) {
+                        // q*dq, formed as bf16(scale q e^b) * D with the rounding the dk/dv kernel
+                        // applies to q~, so the pairwise cancellation inside dg's reverse sum survives
+                        uint4 qw[2];
+                        qw[0] = *reinterpret_cast<const uint4*>(sqr + sw128_off(t, c, BLK));
+                        qw[1] = *reinterpret_cast<const uint4*>(sqr + sw128_off(t, c + 8, BLK));
+                        const uint32_t* qp = reinterpret_cast<const uint32_t*>(qw);
+                        float x[16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const float qr =
-                                __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sqr + sw128_off(t, c + j, BLK)));
-                            const float eb = GATE == 1 ? sg[t * DKB + c + j] : rowE[t];
-                            const float qs = __bfloat162float(__float2bfloat16_rn(qr * P.scale * eb));
-                            sg[t * DKB + c + j] = qs * __uint_as_float(r[j]);
+                        for (int u = 0; u < 8; ++u) {
+                            const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qp[u]));
+                            const float qs0 = __bfloat162float(__float2bfloat16_rn(qf.x * P.scale * eb[2 * u]));
+                            const float qs1 = __bfloat162float(__float2bfloat16_rn(qf.y * P.scale * eb[2 * u + 1]));
+                            x[2 * u] = row_ok ? qs0 * __uint_as_float(r[2 * u]) : 0.f;
+                            x[2 * u + 1] = row_ok ? qs1 * __uint_as_float(r[2 * u + 1]) : 0.f;
                         }
-                } else if (GATE != 0 && lane >= 16) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) sg[t * DKB + c + j] = 0.f;
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            *reinterpret_cast<float4*>(sg + gsw(t, c + 4 * q4)) =
+                                make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
+                    }
                 }
             }
         }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            for (int cb = 0; cb < DKB / 64; ++cb) tma_store_3d(&tout, sk + cb * BLK, d0 + 64 * cb, t0, bh);
+            bulk_commit();
+        }
         // ---- in-segment exclusive prefix of q*dq (fp32) into the dg buffer
-        if (GATE != 0) {
+        if (GATE == 1) {
+            // thread = (key dim dc, group of RPR rows): local sums, exchange, then the prefix walk
+            constexpr int NGR = NT_B / DKB, RPR = TR / NGR;
+            const int dc = tid % DKB, gr = tid / DKB;
+            float loc = 0.f;
+#pragma unroll 8
+            for (int rr = 0; rr < RPR; ++rr) loc += sg[gsw(gr * RPR + rr, dc)];
+            tot[gr * DKB + dc] = loc;
             __syncthreads();
-            if (GATE == 1) {
-                float ax = 0.f, ay = 0.f;
-                for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
-                    ax += sg[r * DKB + d];
-                    ay += sg[r * DKB + d + 1];
-                }
-                tot[rg * DKB + d] = ax;
-                tot[rg * DKB + d + 1] = ay;
-                __syncthreads();
-                float px = carry[d], py = carry[d + 1], Tx = 0.f, Ty = 0.f;
-                for (int r2 = 0; r2 < RG; ++r2) {
-                    if (r2 < rg) { px += tot[r2 * DKB + d]; py += tot[r2 * DKB + d + 1]; }
-                    Tx += tot[r2 * DKB + d];
-                    Ty += tot[r2 * DKB + d + 1];
-                }
-                for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
-                    if (t0 + r < P.L)
-                        *reinterpret_cast<float2*>(A.dg + (rowbase + t0 + r) * P.Dk + d0 + d) = make_float2(px, py);
-                    px += sg[r * DKB + d];
-                    py += sg[r * DKB + d + 1];
-                }
-                __syncthreads();
-                if (rg == 0) { carry[d] += Tx; carry[d + 1] += Ty; }
-            } else {
-                for (int j = 0; j < 8; ++j) {
-                    const int r = warp * 8 + j;
-                    float acc = 0.f;
-                    for (int dd = lane; dd < DKB; dd += 32) acc += sg[r * DKB + dd];
-                    for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-                    if (lane == 0) rows[r] = acc;
-                }
-                __syncthreads();
-                if (warp == 0) {  // exclusive scan over 64 rows, two per lane
-                    const float a0 = rows[2 * lane], a1 = rows[2 * lane + 1];
-                    float v = a0 + a1;
+            float px = carry[dc], T = 0.f;
 #pragma unroll
-                    for (int off = 1; off < 32; off <<= 1) {
-                        const float n = __shfl_up_sync(0xffffffffu, v, off);
-                        if (lane >= off) v += n;
-                    }
-                    const float base = carry[0];
-                    const float e0 = base + v - a0 - a1, e1 = base + v - a1;
-                    if (t0 + 2 * lane < P.L) A.dg[rowbase + t0 + 2 * lane] = e0;
-                    if (t0 + 2 * lane + 1 < P.L) A.dg[rowbase + t0 + 2 * lane + 1] = e1;
-                    const float total = __shfl_sync(0xffffffffu, v, 31);
-                    __syncwarp();
-                    if (lane == 0) carry[0] = base + total;
+            for (int g2 = 0; g2 < NGR; ++g2) {
+                const float v = tot[g2 * DKB + dc];
+                if (g2 < gr) px += v;
+                T += v;
+            }
+            float* dgp = A.dg + (rowbase + t0 + gr * RPR) * P.Dk + d0 + dc;
+#pragma unroll 8
+            for (int rr = 0; rr < RPR; ++rr) {
+                if (t0 + gr * RPR + rr < P.L) dgp[(long)rr * P.Dk] = px;
+                px += sg[gsw(gr * RPR + rr, dc)];
+            }
+            __syncthreads();
+            if (gr == 0) carry[dc] += T;
+        } else if (GATE == 2) {
+            __syncthreads();
+            for (int j = 0; j < 8; ++j) {
+                const int r = warp * 8 + j;
+                float acc = 0.f;
+                for (int dd = lane; dd < DKB; dd += 32) acc += sg[gsw(r, dd)];
+                for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+                if (lane == 0) rows[r] = acc;
+            }
+            __syncthreads();
+            if (warp == 0) {  // exclusive scan over 64 rows, two per lane
+                const float a0 = rows[2 * lane], a1 = rows[2 * lane + 1];
+                float v = a0 + a1;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float n = __shfl_up_sync(0xffffffffu, v, off);
+                    if (lane >= off) v += n;
                 }
+                const float base = carry[0];
+                const float e0 = base + v - a0 - a1, e1 = base + v - a1;
+                if (t0 + 2 * lane < P.L) A.dg[rowbase + t0 + 2 * lane] = e0;
+                if (t0 + 2 * lane + 1 < P.L) A.dg[rowbase + t0 + 2 * lane + 1] = e1;
+                const float total = __shfl_sync(0xffffffffu, v, 31);
+                __syncwarp();
+                if (lane == 0) carry[0] = base + total;
             }
         }
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        if (tid == 0) bulk_wait_read<0>();   // the dq store has read the k slot before it is reloaded
         if (tid == 0 && i + C::NS < ntiles) issue_loads(i + C::NS, s);
     }
 
@@ -541,6 +569,7 @@ __global__ void __launch_bounds__(NT_B, 1)
             }
         }
     }
+    if (tid == 0) bulk_wait<0>();   // the last output stores have completed
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, C::NCOL);
@@ -575,7 +604,8 @@ template <int DK, int DV, int GATE>
 __global__ void __launch_bounds__(NT_B, 1)
     k_tc_bwd_dkdv(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tg, const __grid_constant__ CUtensorMap tv,
-                  const __grid_constant__ CUtensorMap tdo, BwdArgs A, Dims P) {
+                  const __grid_constant__ CUtensorMap tdo, const __grid_constant__ CUtensorMap tout,
+                  const __grid_constant__ CUtensorMap tout2, BwdArgs A, Dims P) {
     using C = KVCfg<DK, DV, GATE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = smem_align1024(smem_raw);
@@ -674,7 +704,9 @@ __global__ void __launch_bounds__(NT_B, 1)
             tma_load_3d(st + cb * BLK, &tq, cb * 64, t0, bh, &bar_full[s]);
             tma_load_3d(st + C::QB + cb * BLK, &tk, cb * 64, t0, bh, &bar_full[s]);
         }
-        if (GATE == 1) tma_load_3d(st + C::QB + C::KB, &tg, 0, t0, bh, &bar_full[s]);
+        if (GATE == 1)
+            for (int gb = 0; gb < DK / 32; ++gb)
+                tma_load_3d(st + C::QB + C::KB + gb * BLK, &tg, 32 * gb, t0, bh, &bar_full[s]);
         for (int vb = 0; vb < DV / 64; ++vb) {
             tma_load_3d(st + C::QB + C::KB + C::GB + vb * BLK, &tv, vb * 64, t0, bh, &bar_full[s]);
             tma_load_3d(st + C::QB + C::KB + C::GB + C::VB + vb * BLK, &tdo, vb * 64, t0, bh, &bar_full[s]);
@@ -810,7 +842,9 @@ __global__ void __launch_bounds__(NT_B, 1)
         if (!block_wait(bar_mma2, i & 1)) { err = 1; break; }
         tc_fence_after();
 
-        // ---- dk = i e^-b X,  di = sum_d k~ X / i,  dv
+        // ---- dk = i e^-b X (bf16, staged in the q slot), k*dk = k~ X (into the g slot for dg),
+        //      di = sum_d k~ X / i, and dv (bf16, staged in the v slot); q~ and V are no longer
+        //      read. Row s of X / dv sits in TMEM lane (s % 16) / 16 + (s % 16) of quadrant s / 16.
         {
             const int srw = 16 * qd + (lane & 15);
             const bool row_ok = t0 + srw < P.L;
@@ -819,24 +853,41 @@ __global__ void __launch_bounds__(NT_B, 1)
                 uint32_t r[16];
                 tmem_ld16(tlane + C::COL_R + c, r);
                 tmem_wait_ld();
-                if (lane < 16 && row_ok) {
+                if (lane < 16) {
                     const float iv = igs[srw];
-                    float f[16];
+                    float em[16];
+                    if (GATE == 1) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float x = __uint_as_float(r[j]);
-                        const float em = GATE == 1 ? sg[srw * DK + c + j] : (GATE == 2 ? rowEi[srw] : 1.f);
-                        f[j] = iv * em * x;
-                        const __nv_bfloat16 kt =
-                            *reinterpret_cast<const __nv_bfloat16*>(sk + sw128_off(srw, c + j, BLK));
-                        const float kx = __bfloat162float(kt) * x;   // k' dk' = k~ X
-                        dsum += kx;
-                        if (GATE != 0) sg[srw * DK + c + j] = kx;
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const float4 e4 = *reinterpret_cast<const float4*>(sg + gsw(srw, c + 4 * q4));
+                            em[4 * q4] = e4.x; em[4 * q4 + 1] = e4.y; em[4 * q4 + 2] = e4.z; em[4 * q4 + 3] = e4.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) em[j] = GATE == 2 ? rowEi[srw] : 1.f;
                     }
-                    store16_bf16_global(A.dk + (rowbase + t0 + srw) * DK + c, f);
-                } else if (GATE != 0 && lane < 16) {
+                    uint4 kw[2];
+                    kw[0] = *reinterpret_cast<const uint4*>(sk + sw128_off(srw, c, BLK));
+                    kw[1] = *reinterpret_cast<const uint4*>(sk + sw128_off(srw, c + 8, BLK));
+                    const uint32_t* kp = reinterpret_cast<const uint32_t*>(kw);
+                    float f[16], kx[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) sg[srw * DK + c + j] = 0.f;
+                    for (int u = 0; u < 8; ++u) {
+                        const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kp[u]));
+                        const float x0 = __uint_as_float(r[2 * u]), x1 = __uint_as_float(r[2 * u + 1]);
+                        f[2 * u] = iv * em[2 * u] * x0;
+                        f[2 * u + 1] = iv * em[2 * u + 1] * x1;
+                        kx[2 * u] = row_ok ? kf.x * x0 : 0.f;         // k' dk' = k~ X
+                        kx[2 * u + 1] = row_ok ? kf.y * x1 : 0.f;
+                        dsum += kx[2 * u] + kx[2 * u + 1];
+                    }
+                    store8_bf16(sq, sw128_off(srw, c, BLK), f);
+                    store8_bf16(sq, sw128_off(srw, c + 8, BLK), f + 8);
+                    if (GATE != 0)
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            *reinterpret_cast<float4*>(sg + gsw(srw, c + 4 * q4)) =
+                                make_float4(kx[4 * q4], kx[4 * q4 + 1], kx[4 * q4 + 2], kx[4 * q4 + 3]);
                 }
             }
             if (lane < 16) sdi[wg * TR + srw] = dsum;
@@ -844,51 +895,57 @@ __global__ void __launch_bounds__(NT_B, 1)
                 uint32_t r[16];
                 tmem_ld16(tlane + C::COL_R + c, r);
                 tmem_wait_ld();
-                if (lane >= 16 && row_ok) {
-                    float f[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) f[j] = __uint_as_float(r[j]);
-                    store16_bf16_global(A.dv + (rowbase + t0 + srw) * DV + c, f);
+                if (lane >= 16) {
+                    store8_bf16(sv, sw128_off(srw, c, BLK), reinterpret_cast<const float*>(r));
+                    store8_bf16(sv, sw128_off(srw, c + 8, BLK), reinterpret_cast<const float*>(r + 8));
                 }
             }
         }
+        fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        if (tid == 0) {
+            for (int cb = 0; cb < DK / 64; ++cb) tma_store_3d(&tout, sq + cb * BLK, 64 * cb, t0, bh);
+            for (int vb = 0; vb < DV / 64; ++vb) tma_store_3d(&tout2, sv + vb * BLK, 64 * vb, t0, bh);
+            bulk_commit();
+        }
         if (A.di && tid < TR && t0 + tid < P.L) A.di[rowbase + t0 + tid] = (sdi[tid] + sdi[TR + tid]) / igs[tid];
         // ---- dg = (in-segment q*dq total - exclusive prefix) - reverse sum of k*dk + carry
         if (GATE == 1) {
-            float ax = 0.f, ay = 0.f;
-            for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
-                ax += sg[r * DK + d];
-                ay += sg[r * DK + d + 1];
-            }
-            tot[rg * DK + d] = ax;
-            tot[rg * DK + d + 1] = ay;
+            // thread = (key dim dc, group of RPR rows): prefetch the dq kernel's prefixes, local
+            // sums, exchange, then the reverse walk
+            constexpr int NGR = NT_B / DK, RPR = TR / NGR;
+            const int dc = tid % DK, gr = tid / DK;
+            float* dgp = A.dg + (rowbase + t0 + gr * RPR) * DK + dc;
+            float pre[RPR];
+#pragma unroll
+            for (int rr = 0; rr < RPR; ++rr) pre[rr] = (t0 + gr * RPR + rr < P.L) ? dgp[(long)rr * DK] : 0.f;
+            float loc = 0.f;
+#pragma unroll 8
+            for (int rr = 0; rr < RPR; ++rr) loc += sg[gsw(gr * RPR + rr, dc)];
+            tot[gr * DK + dc] = loc;
             __syncthreads();
-            float sx = rk[d], sy = rk[d + 1], Tx = 0.f, Ty = 0.f;
-            for (int r2 = 0; r2 < RG; ++r2) {
-                if (r2 > rg) { sx += tot[r2 * DK + d]; sy += tot[r2 * DK + d + 1]; }
-                Tx += tot[r2 * DK + d];
-                Ty += tot[r2 * DK + d + 1];
+            float sx = rk[dc], T = 0.f;
+#pragma unroll
+            for (int g2 = 0; g2 < NGR; ++g2) {
+                const float v = tot[g2 * DK + dc];
+                if (g2 > gr) sx += v;
+                T += v;
             }
-            const float cx = cz[d], cy = cz[d + 1];
-            for (int r = (rg + 1) * RPG - 1; r >= rg * RPG; --r) {
-                sx += sg[r * DK + d];
-                sy += sg[r * DK + d + 1];
-                if (t0 + r < P.L) {
-                    float2* gp = reinterpret_cast<float2*>(A.dg + (rowbase + t0 + r) * DK + d);
-                    const float2 pq = *gp;
-                    *gp = make_float2(cx - pq.x - sx, cy - pq.y - sy);
-                }
+            const float cx = cz[dc];
+#pragma unroll
+            for (int rr = RPR - 1; rr >= 0; --rr) {
+                sx += sg[gsw(gr * RPR + rr, dc)];
+                if (t0 + gr * RPR + rr < P.L) dgp[(long)rr * DK] = cx - pre[rr] - sx;
             }
             __syncthreads();
-            if (rg == 0) { rk[d] += Tx; rk[d + 1] += Ty; }
+            if (gr == 0) rk[dc] += T;
         } else if (GATE == 2) {
             for (int j = 0; j < 8; ++j) {
                 const int r = warp * 8 + j;
                 float acc = 0.f;
-                for (int dd = lane; dd < DK; dd += 32) acc += sg[r * DK + dd];
+                for (int dd = lane; dd < DK; dd += 32) acc += sg[gsw(r, dd)];
                 for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
                 if (lane == 0) rows[r] = acc;
             }
@@ -911,6 +968,8 @@ __global__ void __launch_bounds__(NT_B, 1)
                 if (lane == 0) rk[0] = base + total;
             }
         }
+        __syncthreads();
+        if (tid == 0) bulk_wait_read<0>();   // the dk / dv stores have read the q and v slots
         if (tid == 0 && i + C::NS < ntiles) issue_loads(i + C::NS, s);
     }
 
@@ -936,6 +995,7 @@ __global__ void __launch_bounds__(NT_B, 1)
             }
         }
     }
+    if (tid == 0) bulk_wait<0>();   // the last output stores have completed
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, C::NCOL);
@@ -1011,8 +1071,8 @@ void bwd_plan_info(const Dims& P, int* nseg, int* tiles_per_seg) {
 
 template <int DKB, int DV, int GATE>
 static cudaError_t launch_dq(const Dims& P, const BwdPlan& pl, const CUtensorMap& mq, const CUtensorMap& mk,
-                             const CUtensorMap& mg, const CUtensorMap& mv, const CUtensorMap& mo, const BwdArgs& a,
-                             cudaStream_t st) {
+                             const CUtensorMap& mg, const CUtensorMap& mv, const CUtensorMap& mo,
+                             const CUtensorMap& mdq, const BwdArgs& a, cudaStream_t st) {
     using C = QCfg<DKB, DV, GATE>;
     auto kern = k_tc_bwd_dq<DKB, DV, GATE>;
     static bool attr = false;
@@ -1022,14 +1082,14 @@ static cudaError_t launch_dq(const Dims& P, const BwdPlan& pl, const CUtensorMap
         attr = true;
     }
     dim3 grid(P.B * P.H, P.Dk / DKB, pl.nseg);
-    GLA_LAUNCH("tc_bwd_dq", st, kern<<<grid, NT_B, C::SMEM, st>>>(mq, mk, mg, mv, mo, a, P));
+    GLA_LAUNCH("tc_bwd_dq", st, kern<<<grid, NT_B, C::SMEM, st>>>(mq, mk, mg, mv, mo, mdq, a, P));
     return cudaGetLastError();
 }
 
 template <int DK, int DV, int GATE>
 static cudaError_t launch_dkdv(const Dims& P, const BwdPlan& pl, const CUtensorMap& mq, const CUtensorMap& mk,
-                               const CUtensorMap& mg, const CUtensorMap& mv, const CUtensorMap& mo, const BwdArgs& a,
-                               cudaStream_t st) {
+                               const CUtensorMap& mg, const CUtensorMap& mv, const CUtensorMap& mo,
+                               const CUtensorMap& mdk, const CUtensorMap& mdv, const BwdArgs& a, cudaStream_t st) {
     using C = KVCfg<DK, DV, GATE>;
     auto kern = k_tc_bwd_dkdv<DK, DV, GATE>;
     static bool attr = false;
@@ -1039,7 +1099,7 @@ static cudaError_t launch_dkdv(const Dims& P, const BwdPlan& pl, const CUtensorM
         attr = true;
     }
     dim3 grid(P.B * P.H, pl.nseg);
-    GLA_LAUNCH("tc_bwd_dkdv", st, kern<<<grid, NT_B, C::SMEM, st>>>(mq, mk, mg, mv, mo, a, P));
+    GLA_LAUNCH("tc_bwd_dkdv", st, kern<<<grid, NT_B, C::SMEM, st>>>(mq, mk, mg, mv, mo, mdk, mdv, a, P));
     return cudaGetLastError();
 }
 
@@ -1051,19 +1111,21 @@ static cudaError_t run_bwd(const Dims& P, const void* q, const void* k, const vo
     const BwdWs w = bwd_layout(P, static_cast<char*>(ws));
     const int BH = P.B * P.H;
     constexpr int DKB = DK > 128 ? 128 : DK;
-    CUtensorMap mq, mk, mv, mo, mg, mgb;
-    if (!make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dk, P.L, BH, 64, true) ||
+    CUtensorMap mq, mk, mv, mo, mg, mdq, mdk, mdv;
+    if (!make_map(&mdq, dq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dk, P.L, BH, 64, true) ||
+        !make_map(&mdk, dk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dk, P.L, BH, 64, true) ||
+        !make_map(&mdv, dv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dv, P.L, BH, 64, true) ||
+        !make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dk, P.L, BH, 64, true) ||
         !make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dk, P.L, BH, 64, true) ||
         !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dv, P.L, BH, 64, true) ||
         !make_map(&mo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dv, P.L, BH, 64, true))
         return cudaErrorInvalidValue;
     if (GATE == 1) {
-        if (!make_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, P.Dk, P.L, BH, P.Dk, false) ||
-            !make_map(&mgb, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, P.Dk, P.L, BH, DKB, false))
+        // 32-column fp32 boxes with the 128-byte swizzle (see gsw)
+        if (!make_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, P.Dk, P.L, BH, 32, true))
             return cudaErrorInvalidValue;
     } else {
         mg = mk;
-        mgb = mk;
     }
     int* status = static_cast<int*>(ws);
     cudaError_t e;
@@ -1091,7 +1153,7 @@ static cudaError_t run_bwd(const Dims& P, const void* q, const void* k, const vo
     a.status = status;
     a.tiles_per_seg = pl.tiles_per_seg;
     a.nseg = pl.nseg;
-    e = launch_dq<DKB, DV, GATE>(P, pl, mq, mk, mgb, mv, mo, a, st);
+    e = launch_dq<DKB, DV, GATE>(P, pl, mq, mk, mg, mv, mo, mdq, a, st);
     if (e != cudaSuccess) return e;
     if (pl.nseg > 1) {
         e = state_pass(P, 2, q, dO, g, ig, pl.nseg, pl.tiles_per_seg, w.seg_state, w.seg_gamma, status, st);
@@ -1099,7 +1161,7 @@ static cudaError_t run_bwd(const Dims& P, const void* q, const void* k, const vo
         e = seg_rscan(P, pl.nseg, w.seg_state, w.seg_gamma, dhT, w.gend, st);
         if (e != cudaSuccess) return e;
     }
-    e = launch_dkdv<DK, DV, GATE>(P, pl, mq, mk, mg, mv, mo, a, st);
+    e = launch_dkdv<DK, DV, GATE>(P, pl, mq, mk, mg, mv, mo, mdk, mdv, a, st);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

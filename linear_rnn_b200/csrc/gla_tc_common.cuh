@@ -11,6 +11,14 @@ namespace tc {
 constexpr int TR = 64;          // tokens per tile
 constexpr uint32_t BLK = 8192;  // one 64-column bf16 block of a 64-row tile (64 x 128 B)
 
+// Float index of element (r, d) of a 64-row fp32 tile loaded by TMA in 32-column boxes with
+// the 128-byte swizzle: boxes of 64 rows x 128 B, 16-byte chunks XOR-ed with the row. Eight
+// consecutive rows reading the same column range then hit eight different bank groups, and a
+// row read column-wise stays conflict-free.
+__device__ __forceinline__ int gsw(int r, int d) {
+    return ((d >> 5) << 11) + (r << 5) + ((((d >> 2) & 7) ^ (r & 7)) << 2) + (d & 3);
+}
+
 // Packed pairs of fp32 in one 64-bit register, multiplied lane-wise by the sm_100 packed
 // fp32 instruction (IEEE round-to-nearest per lane, like two separate multiplies).
 __device__ __forceinline__ uint64_t f2(float lo, float hi) {
