@@ -74,33 +74,49 @@ __device__ __forceinline__ void store16_bf16_global(__nv_bfloat16* dst, const fl
 
 constexpr uint32_t pow2cols(uint32_t n) { return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512; }
 
-// In-place transform of one 64-token tile over 8-key-dim (16-byte swizzle chunk) groups,
-// 256 threads: b = column cumsum of the log-gate, then
-//   k~ = i * k * e^-b  (k tile),   DO_Q: q~ = scale * q * e^b  (q tile),
-//   per-key gates: the g tile is overwritten with e^b (G_SLOT_EB) or e^-b,
-//   gam[d] = e^Gamma.  Per-head gates use the row factors rowE / rowEi instead.
-// Both backward kernels use this one routine so they form bit-identical q~ and k~.
+// In-place transform of one 64-token tile by all NT_B threads:
+//   step A (per-key gates): b = column cumsum of the log-gate in row segments (thread = key
+//     dim x segment) joined through the segment totals, written over g; gam[d] = e^Gamma;
+//   step B: every 16-byte chunk (8 key dims of one row): k~ = i * k * e^-b (k tile),
+//     DO_Q: q~ = scale * q * e^b (q tile), and the g slot keeps e^b (G_SLOT_EB) or e^-b.
+// Per-head gates use the row factors rowE / rowEi (warp 0 scans the 64 gates) instead.
+// Both backward kernels use this one routine so they form bit-identical q~ and k~. The g tile
+// is in the swizzled fp32 layout (gsw).
 template <int D, int GATE, bool DO_Q, bool G_SLOT_EB>
 __device__ __forceinline__ void bwd_transform(uint8_t* sq, uint8_t* sk, float* sg, float* tot, float* gam,
                                               float* rowE, float* rowEi, const float* ghs, const float* igs,
                                               float scale, int tid) {
-    constexpr int NO = D / 8, RG = NT_B / NO, RPG = TR / RG;
-    static_assert(RG * D <= 2048, "cumsum group totals");
-    const int oc = tid % NO, rg = tid / NO, d0 = 8 * oc;
+    constexpr int SEG = NT_B / D, RS = TR / SEG;   // step A
+    constexpr int NO = D / 8, NPOS = TR * NO;       // step B
+    constexpr int NB = 2;
+    static_assert(NT_B % D == 0 && NPOS % (NB * NT_B) == 0, "transform mapping");
     const int warp = tid >> 5, lane = tid & 31;
-    float bb[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) bb[u] = 0.f;
     if (GATE == 1) {
-#pragma unroll 4
-        for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
-            const float4 g0 = *reinterpret_cast<const float4*>(sg + gsw(r, d0));
-            const float4 g1 = *reinterpret_cast<const float4*>(sg + gsw(r, d0 + 4));
-            bb[0] += g0.x; bb[1] += g0.y; bb[2] += g0.z; bb[3] += g0.w;
-            bb[4] += g1.x; bb[5] += g1.y; bb[6] += g1.z; bb[7] += g1.w;
+        const int dA = tid % D, sA = tid / D;
+        float x[RS];
+#pragma unroll
+        for (int u = 0; u < RS; ++u) x[u] = sg[gsw(sA * RS + u, dA)];
+        float acc = 0.f;
+#pragma unroll
+        for (int u = 0; u < RS; ++u) {
+            acc += x[u];
+            x[u] = acc;
         }
-        *reinterpret_cast<float4*>(tot + rg * D + d0) = make_float4(bb[0], bb[1], bb[2], bb[3]);
-        *reinterpret_cast<float4*>(tot + rg * D + d0 + 4) = make_float4(bb[4], bb[5], bb[6], bb[7]);
+        float off = 0.f, G = acc;
+        if constexpr (SEG > 1) {
+            tot[tid] = acc;
+            __syncthreads();
+            G = 0.f;
+#pragma unroll
+            for (int s2 = 0; s2 < SEG; ++s2) {
+                const float t = tot[s2 * D + dA];
+                if (s2 < sA) off += t;
+                G += t;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < RS; ++u) sg[gsw(sA * RS + u, dA)] = x[u] + off;
+        if (sA == 0) gam[dA] = __expf(G);
     } else if (GATE == 2 && warp == 0) {
         const float g0 = ghs[2 * lane], g1 = ghs[2 * lane + 1];
         float v = g0 + g1;
@@ -118,79 +134,69 @@ __device__ __forceinline__ void bwd_transform(uint8_t* sq, uint8_t* sk, float* s
         if (lane == 0) gam[0] = __expf(G);
     }
     __syncthreads();
-    if (GATE == 1) {
-        float G8[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            bb[u] = 0.f;
-            G8[u] = 0.f;
+    for (int it0 = 0; it0 < NPOS / NT_B; it0 += NB) {
+        float bv[NB][8];
+        uint4 wq[NB], wk[NB];
+        uint32_t offs[NB];
+        int rows[NB], d0s[NB];
+#pragma unroll
+        for (int k = 0; k < NB; ++k) {
+            const int c = tid + (it0 + k) * NT_B;
+            const int r = c / NO, d0 = 8 * (c % NO);
+            rows[k] = r;
+            d0s[k] = d0;
+            if (GATE == 1) {
+                const float4 b0 = *reinterpret_cast<const float4*>(sg + gsw(r, d0));
+                const float4 b1 = *reinterpret_cast<const float4*>(sg + gsw(r, d0 + 4));
+                bv[k][0] = b0.x; bv[k][1] = b0.y; bv[k][2] = b0.z; bv[k][3] = b0.w;
+                bv[k][4] = b1.x; bv[k][5] = b1.y; bv[k][6] = b1.z; bv[k][7] = b1.w;
+            }
+            offs[k] = (uint32_t)(d0 >> 6) * BLK + (uint32_t)r * 128 +
+                      ((((uint32_t)((d0 & 63) >> 3)) ^ (uint32_t)(r & 7)) << 4);
+            if (DO_Q) wq[k] = *reinterpret_cast<const uint4*>(sq + offs[k]);
+            wk[k] = *reinterpret_cast<const uint4*>(sk + offs[k]);
         }
 #pragma unroll
-        for (int r2 = 0; r2 < RG; ++r2) {
-            const float4 t0v = *reinterpret_cast<const float4*>(tot + r2 * D + d0);
-            const float4 t1v = *reinterpret_cast<const float4*>(tot + r2 * D + d0 + 4);
-            const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
+        for (int k = 0; k < NB; ++k) {
+            const int r = rows[k], d0 = d0s[k];
+            float eq[8], ek[8];
+            if (GATE == 1) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                if (r2 < rg) bb[u] += tv[u];
-                G8[u] += tv[u];
+                for (int u = 0; u < 8; ++u) {
+                    eq[u] = __expf(bv[k][u]);
+                    ek[u] = rcp_newton(eq[u]);
+                }
+                const float* keep = G_SLOT_EB ? eq : ek;
+                *reinterpret_cast<float4*>(sg + gsw(r, d0)) = make_float4(keep[0], keep[1], keep[2], keep[3]);
+                *reinterpret_cast<float4*>(sg + gsw(r, d0 + 4)) = make_float4(keep[4], keep[5], keep[6], keep[7]);
+            } else {
+                const float e1 = GATE == 2 ? rowE[r] : 1.f, e2 = GATE == 2 ? rowEi[r] : 1.f;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    eq[u] = e1;
+                    ek[u] = e2;
+                }
             }
-        }
-        if (rg == 0)
-#pragma unroll
-            for (int u = 0; u < 8; ++u) gam[d0 + u] = __expf(G8[u]);
-    }
-#pragma unroll 2
-    for (int r = rg * RPG; r < (rg + 1) * RPG; ++r) {
-        float eq[8], ek[8];
-        if (GATE == 1) {
-            float4* gp0 = reinterpret_cast<float4*>(sg + gsw(r, d0));
-            float4* gp1 = reinterpret_cast<float4*>(sg + gsw(r, d0 + 4));
-            const float4 g0 = *gp0, g1 = *gp1;
-            const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                bb[u] += gv[u];
-                eq[u] = __expf(bb[u]);
-                ek[u] = __expf(-bb[u]);
-            }
-            const float* keep = G_SLOT_EB ? eq : ek;
-            *gp0 = make_float4(keep[0], keep[1], keep[2], keep[3]);
-            *gp1 = make_float4(keep[4], keep[5], keep[6], keep[7]);
-        } else {
-            const float e1 = GATE == 2 ? rowE[r] : 1.f, e2 = GATE == 2 ? rowEi[r] : 1.f;
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                eq[u] = e1;
-                ek[u] = e2;
-            }
-        }
-        const uint32_t off = (uint32_t)(d0 >> 6) * BLK + (uint32_t)r * 128 +
-                             ((((uint32_t)((d0 & 63) >> 3)) ^ (uint32_t)(r & 7)) << 4);
-        if (DO_Q) {
-            uint4* pq = reinterpret_cast<uint4*>(sq + off);
-            uint4 w = *pq;
-            uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wp[u]));
-                __nv_bfloat162 h = __floats2bfloat162_rn(f.x * scale * eq[2 * u], f.y * scale * eq[2 * u + 1]);
-                wp[u] = *reinterpret_cast<uint32_t*>(&h);
-            }
-            *pq = w;
-        }
-        {
-            uint4* pk = reinterpret_cast<uint4*>(sk + off);
-            uint4 w = *pk;
-            uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
             const float iv = igs[r];
+            uint32_t* pk = reinterpret_cast<uint32_t*>(&wk[k]);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&wp[u]));
+                const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&pk[u]));
                 __nv_bfloat162 h = __floats2bfloat162_rn(f.x * iv * ek[2 * u], f.y * iv * ek[2 * u + 1]);
-                wp[u] = *reinterpret_cast<uint32_t*>(&h);
+                pk[u] = *reinterpret_cast<uint32_t*>(&h);
             }
-            *pk = w;
+            *reinterpret_cast<uint4*>(sk + offs[k]) = wk[k];
+            if (DO_Q) {
+                uint32_t* pq = reinterpret_cast<uint32_t*>(&wq[k]);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&pq[u]));
+                    __nv_bfloat162 h = __floats2bfloat162_rn(f.x * scale * eq[2 * u], f.y * scale * eq[2 * u + 1]);
+                    pq[u] = *reinterpret_cast<uint32_t*>(&h);
+                }
+                *reinterpret_cast<uint4*>(sq + offs[k]) = wq[k];
+            }
         }
     }
 }

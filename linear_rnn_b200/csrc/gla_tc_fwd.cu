@@ -61,18 +61,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
-// 1/x on the FMA pipe (keeps the special-function unit free for the exponentials): a bit-level
-// seed -- the integer constant minus the bits of x, which for any normal x lands within 5.1 %
-// of 1/x; the constant was chosen by a search minimising that worst case over one binade --
-// then two Newton steps y <- y (2 - x y), each squaring the relative error (5.1e-2 -> 2.6e-3
-// -> 6.6e-6), far below the bf16 rounding its result goes into.
-__device__ __forceinline__ float rcp_newton(float x) {
-    float y = __int_as_float(0x7EF311C2 - __float_as_int(x));
-    float e = fmaf(-x, y, 1.f);
-    y = fmaf(y, e, y);
-    e = fmaf(-x, y, 1.f);
-    return fmaf(y, e, y);
-}
 
 constexpr uint32_t pow2_cols(uint32_t n) { return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512; }
 
