@@ -56,7 +56,8 @@ typedef enum {
     GLA_ERR_UNSUPPORTED = 2,  /* valid request this build cannot run (shape, plan) */
     GLA_ERR_WORKSPACE = 3,    /* ws_bytes smaller than gla_workspace_bytes() */
     GLA_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
-    GLA_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up (see below) */
+    GLA_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up (see below) */
+    GLA_ERR_RANGE = 6         /* log-gate decay too strong for the tensor-core plan (see below) */
 } gla_status;
 
 typedef enum { GLA_F32 = 0, GLA_BF16 = 1 } gla_dtype;
@@ -119,8 +120,11 @@ GLA_API gla_status gla_bwd(const gla_problem* p, const void* q, const void* k, c
 GLA_API const char* gla_status_string(gla_status s);
 
 /* Synchronises `stream`, then reads the device status word kept at the start of the
- * workspace of the last call that used `ws`: GLA_OK, or GLA_ERR_TIMEOUT when a bounded
- * device-side wait gave up; GLA_ERR_CUDA if the synchronisation itself failed. */
+ * workspace of the last call that used `ws`: GLA_OK; GLA_ERR_TIMEOUT when a bounded
+ * device-side wait gave up; GLA_ERR_RANGE when the tensor-core plan met a 64-token tile whose
+ * total log-decay in some key dim is below -60 (its in-tile factors e^-b would leave the fp32
+ * range, so that call's results are not valid; GLA_PLAN_SIMT evaluates such gates in log-space
+ * sub-tiles); GLA_ERR_CUDA if the synchronisation itself failed. */
 GLA_API gla_status gla_check_device_status(void* ws, void* stream);
 
 /* Text of the CUDA error behind the calling thread's last GLA_ERR_CUDA (where it happened,

@@ -11,7 +11,7 @@ import os
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgla_b200.so")
 
-GLA_OK, GLA_ERR_INVALID_ARG, GLA_ERR_UNSUPPORTED, GLA_ERR_WORKSPACE, GLA_ERR_CUDA, GLA_ERR_TIMEOUT = range(6)
+GLA_OK, GLA_ERR_INVALID_ARG, GLA_ERR_UNSUPPORTED, GLA_ERR_WORKSPACE, GLA_ERR_CUDA, GLA_ERR_TIMEOUT, GLA_ERR_RANGE = range(7)
 GLA_F32, GLA_BF16 = 0, 1
 GLA_GATE_NONE, GLA_GATE_PER_KEY, GLA_GATE_PER_HEAD = 0, 1, 2
 GLA_PLAN_AUTO, GLA_PLAN_SIMT, GLA_PLAN_TC = 0, 1, 2

@@ -187,6 +187,7 @@ const char* gla_status_string(gla_status status) {
         case GLA_ERR_WORKSPACE: return "workspace too small";
         case GLA_ERR_CUDA: return "CUDA runtime error";
         case GLA_ERR_TIMEOUT: return "bounded device-side wait timed out";
+        case GLA_ERR_RANGE: return "log-gate decay within a 64-token tile beyond the tensor-core plan's range";
     }
     return "unknown status";
 }
@@ -197,6 +198,8 @@ gla_status gla_check_device_status(void* ws, void* stream) {
     cudaStream_t st = (cudaStream_t)stream;
     if (cudaMemcpyAsync(&word, ws, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return GLA_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return GLA_ERR_CUDA;
+    if (word & kDevStatusTimeout) return GLA_ERR_TIMEOUT;
+    if (word & kDevStatusRange) return GLA_ERR_RANGE;
     return word == kDevStatusOk ? GLA_OK : GLA_ERR_TIMEOUT;
 }
 

@@ -27,7 +27,11 @@ __host__ __device__ __forceinline__ size_t align_up(size_t x, size_t a) { return
 // Device status word at the start of every workspace (first 256 bytes).
 constexpr size_t kStatusBytes = 256;
 constexpr int kDevStatusOk = 0;
-constexpr int kDevStatusTimeout = 1;
+constexpr int kDevStatusTimeout = 1;   // bits of the device status word
+constexpr int kDevStatusRange = 2;
+// Most negative in-tile total log-decay the tensor-core plans evaluate: their q e^b and
+// k e^-b factors span e^{|Gamma|} within a 64-token tile and must stay inside fp32.
+constexpr float kMinTileLogDecay = -60.f;
 
 // Launch accounting (gla_api.cu): every kernel launch of the library goes through
 // GLA_LAUNCH, which counts it and, while the profiler is enabled, brackets it with CUDA

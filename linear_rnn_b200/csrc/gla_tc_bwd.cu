@@ -85,7 +85,7 @@ constexpr uint32_t pow2cols(uint32_t n) { return n <= 32 ? 32 : n <= 64 ? 64 : n
 template <int D, int GATE, bool DO_Q, bool G_SLOT_EB>
 __device__ __forceinline__ void bwd_transform(uint8_t* sq, uint8_t* sk, float* sg, float* tot, float* gam,
                                               float* rowE, float* rowEi, const float* ghs, const float* igs,
-                                              float scale, int tid) {
+                                              float scale, int tid, int* status) {
     constexpr int SEG = NT_B / D, RS = TR / SEG;   // step A
     constexpr int NO = D / 8, NPOS = TR * NO;       // step B
     constexpr int NB = 2;
@@ -116,7 +116,10 @@ __device__ __forceinline__ void bwd_transform(uint8_t* sq, uint8_t* sk, float* s
         }
 #pragma unroll
         for (int u = 0; u < RS; ++u) sg[gsw(sA * RS + u, dA)] = x[u] + off;
-        if (sA == 0) gam[dA] = __expf(G);
+        if (sA == 0) {
+            gam[dA] = __expf(G);
+            if (G < kMinTileLogDecay) atomicOr(status, kDevStatusRange);
+        }
     } else if (GATE == 2 && warp == 0) {
         const float g0 = ghs[2 * lane], g1 = ghs[2 * lane + 1];
         float v = g0 + g1;
@@ -131,7 +134,10 @@ __device__ __forceinline__ void bwd_transform(uint8_t* sq, uint8_t* sk, float* s
         rowEi[2 * lane] = __expf(-b0);
         rowEi[2 * lane + 1] = __expf(-b1);
         const float G = __shfl_sync(0xffffffffu, b1, 31);
-        if (lane == 0) gam[0] = __expf(G);
+        if (lane == 0) {
+            gam[0] = __expf(G);
+            if (G < kMinTileLogDecay) atomicOr(status, kDevStatusRange);
+        }
     }
     __syncthreads();
 #pragma unroll
@@ -337,7 +343,7 @@ __global__ void __launch_bounds__(NT_B, 1)
         if (!block_wait(&bar_full[s], (i / C::NS) & 1)) { err = 1; break; }
 
         // ---- transform: k~ = i k e^-b in place; e^b kept (in place of g) for the dq epilogue
-        bwd_transform<DKB, GATE, false, true>(sqr, sk, sg, tot, gam, rowE, rowEi, ghs, igs, P.scale, tid);
+        bwd_transform<DKB, GATE, false, true>(sqr, sk, sg, tot, gam, rowE, rowEi, ghs, igs, P.scale, tid, A.status);
         // pair mapping of the later q*dq prefix phase
         constexpr int NP = DKB / 2, RG = NT_B / NP, RPG = TR / RG;
         const int cp = tid % NP, rg = tid / NP, d = 2 * cp;
@@ -554,7 +560,7 @@ __global__ void __launch_bounds__(NT_B, 1)
     }
     if (err) {
         if (tid == 0) {
-            atomicExch(A.status, kDevStatusTimeout);
+            atomicOr(A.status, kDevStatusTimeout);
             if (n_mma) {
                 mbar_wait(bar_mma1, (n_mma - 1) & 1, 1u << 20);
                 mbar_wait(bar_mma2, (n_mma - 1) & 1, 1u << 20);
@@ -739,7 +745,7 @@ __global__ void __launch_bounds__(NT_B, 1)
         if (!block_wait(&bar_full[s], (i / C::NS) & 1)) { err = 1; break; }
 
         // ---- transform: q~ = scale q e^b, k~ = i k e^-b (in place); e^-b kept in place of g
-        bwd_transform<DK, GATE, true, false>(sq, sk, sg, tot, gam, rowE, rowEi, ghs, igs, P.scale, tid);
+        bwd_transform<DK, GATE, true, false>(sq, sk, sg, tot, gam, rowE, rowEi, ghs, igs, P.scale, tid, A.status);
         // pair mapping of the later dg phase
         constexpr int NP = DK / 2, RG = NT_B / NP, RPG = TR / RG;
         const int cp = tid % NP, rg = tid / NP, d = 2 * cp;
@@ -981,7 +987,7 @@ __global__ void __launch_bounds__(NT_B, 1)
 
     if (err) {
         if (tid == 0) {
-            atomicExch(A.status, kDevStatusTimeout);
+            atomicOr(A.status, kDevStatusTimeout);
             if (n_mma) {
                 mbar_wait(bar_mma1, (n_mma - 1) & 1, 1u << 20);
                 mbar_wait(bar_mma2, (n_mma - 1) & 1, 1u << 20);

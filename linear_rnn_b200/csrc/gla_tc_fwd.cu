@@ -398,6 +398,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 if (sA == 0) {
                     gam[dA] = __expf(G);
                     gaml[dA] = G;
+                    if (G < kMinTileLogDecay) atomicOr(A.status, kDevStatusRange);
                 }
             } else if (GATE == 2) {
                 if (ttid < 32) {  // warp scan over 64 rows, two rows per lane
@@ -419,6 +420,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     if (lane == 0) {
                         gam[0] = __expf(G);
                         gaml[0] = G;
+                        if (G < kMinTileLogDecay) atomicOr(A.status, kDevStatusRange);
                     }
                 }
             }
@@ -611,7 +613,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     tc_fence_after();
     if (*abortp) {
         if (tid == 0) {
-            atomicExch(A.status, kDevStatusTimeout);
+            atomicOr(A.status, kDevStatusTimeout);
             // let every issued copy and product land before shared memory and TMEM go away
             for (int j = *n_consumed; j < *n_issued; ++j)
                 mbar_wait(&bar_full[j % C::NS], (j / C::NS) & 1, 1u << 20);

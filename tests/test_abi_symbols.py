@@ -70,8 +70,9 @@ def test_workspace_sizes():
 
 
 def test_status_strings():
-    for s in range(6):
+    for s in range(7):
         assert len(_lib.status_string(s)) >= 2
+    assert "range" in _lib.status_string(_lib.GLA_ERR_RANGE)
     assert "unknown" in _lib.status_string(99)
 
 

@@ -197,6 +197,33 @@ def test_outputs_fully_written_over_nan_poison():
     assert not torch.isnan(o).any() and not torch.isnan(hT).any()
 
 
+def test_strong_gates_flagged_on_tensor_cores_and_exact_on_simt():
+    """A tile whose total log-decay is below the tensor-core plans' bound (-60) raises the range
+    status (the call's results are not trusted); the CUDA-core plan, whose per-tile-pair
+    reference rows keep every factor within e^64 here, still matches the oracle."""
+    from linear_rnn_b200 import _lib
+    w = I.small(I.WORKLOADS["c3"])
+    x = I.make_inputs(w, seed=5)
+    x["g"] = torch.full_like(x["g"], -1.0)           # -64 per 64-token tile
+    xd = to_cuda(x)
+    prob = ops().make_problem(xd["q"], xd["v"], xd["g"], scale=w.scale, chunk=w.chunk, plan="tc")
+    ws = torch.empty(max(ops().gla_workspace_bytes(prob, False), ops().gla_workspace_bytes(prob, True)),
+                     dtype=torch.uint8, device="cuda")
+    ops().gla_fwd(xd["q"], xd["k"], xd["v"], xd["g"], None, None, scale=w.scale, chunk=w.chunk, plan="tc",
+                  workspace=ws)
+    assert ops().gla_check_device_status(ws) == _lib.GLA_ERR_RANGE
+    ops().gla_bwd(xd["q"], xd["k"], xd["v"], xd["g"], None, None, xd["dO"], None, scale=w.scale, chunk=w.chunk,
+                  plan="tc", workspace=ws)
+    assert ops().gla_check_device_status(ws) == _lib.GLA_ERR_RANGE
+    # ordinary gates leave the status clean
+    xd2 = to_cuda(I.make_inputs(w, seed=5))
+    ops().gla_fwd(xd2["q"], xd2["k"], xd2["v"], xd2["g"], None, None, scale=w.scale, chunk=w.chunk, plan="tc",
+                  workspace=ws)
+    assert ops().gla_check_device_status(ws) == _lib.GLA_OK
+    check_fwd(x, w, plan="simt")
+    check_bwd(x, w, plan="simt")
+
+
 def test_host_tensors_round_trip():
     """The end-to-end call with host tensors (copies in, compute, copies out)."""
     w = I.small(I.WORKLOADS["c2"])
