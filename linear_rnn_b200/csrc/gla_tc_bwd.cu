@@ -216,7 +216,8 @@ struct QCfg {
     static constexpr uint32_t VB = TR * DV * 2;
     static constexpr uint32_t OB = TR * DV * 2;
     static constexpr uint32_t STAGE = QB + KB + GB + VB + OB;
-    static constexpr uint32_t TXB = STAGE - (GATE == 1 ? 0 : GB); // bytes the copy engine writes
+    static constexpr uint32_t TXA = QB + KB + (GATE == 1 ? GB : 0);  // bytes of the q, k, g loads
+    static constexpr uint32_t TXV = VB + OB;                         // bytes of the v, dO loads
     static constexpr uint32_t SB = DKB * DV * 2;
     static constexpr uint32_t AB = TR * TR * 2;
     static constexpr uint32_t SMALL = 256 + 8192 + 8 * DKB + 1024 + 512;
@@ -245,6 +246,8 @@ __global__ void __launch_bounds__(NT_B, 1)
     uint64_t* bar_full = reinterpret_cast<uint64_t*>(small);  // [2]
     uint64_t* bar_mma1 = bar_full + 2;
     uint64_t* bar_mma2 = bar_full + 3;
+    uint64_t* bar_drain = bar_full + 4;   // error path: completion of every product issued
+    uint64_t* bar_fullv = bar_full + 5;   // [2] v and dO landed (bar_full: q, k, g)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 64);
     float* tot = reinterpret_cast<float*>(small + 256);
     float* gam = tot + 2048;            // [DKB]
@@ -270,6 +273,9 @@ __global__ void __launch_bounds__(NT_B, 1)
         mbar_init(&bar_full[1], 1);
         mbar_init(bar_mma1, 1);
         mbar_init(bar_mma2, 1);
+        mbar_init(bar_drain, 1);
+        mbar_init(&bar_fullv[0], 1);
+        mbar_init(&bar_fullv[1], 1);
         mbar_fence_init();
     }
     if (tid < DKB) carry[tid] = 0.f;
@@ -306,10 +312,12 @@ __global__ void __launch_bounds__(NT_B, 1)
     __syncthreads();
     tc_fence_after();
 
-    auto issue_loads = [&](int i, int s) {
+    // q, k, g of a tile are read until its epilogue ends; v and dO only by the first product
+    // group, so the next tile's v and dO are loaded as soon as that group completes
+    auto issue_qkg = [&](int i, int s) {
         uint8_t* st = sm + s * C::STAGE;
         const int t0 = (tile0 + i) * TR;
-        mbar_arrive_expect_tx(&bar_full[s], C::TXB);
+        mbar_arrive_expect_tx(&bar_full[s], C::TXA);
         for (int cb = 0; cb < DKB / 64; ++cb) {
             if (GATE != 0) tma_load_3d(st + cb * BLK, &tq, d0 + cb * 64, t0, bh, &bar_full[s]);
             tma_load_3d(st + C::QB + cb * BLK, &tk, d0 + cb * 64, t0, bh, &bar_full[s]);
@@ -317,13 +325,21 @@ __global__ void __launch_bounds__(NT_B, 1)
         if (GATE == 1)
             for (int gb = 0; gb < DKB / 32; ++gb)
                 tma_load_3d(st + C::QB + C::KB + gb * BLK, &tg, d0 + 32 * gb, t0, bh, &bar_full[s]);
+    };
+    auto issue_vo = [&](int i, int s) {
+        uint8_t* st = sm + s * C::STAGE;
+        const int t0 = (tile0 + i) * TR;
+        mbar_arrive_expect_tx(&bar_fullv[s], C::TXV);
         for (int vb = 0; vb < DV / 64; ++vb) {
-            tma_load_3d(st + C::QB + C::KB + C::GB + vb * BLK, &tv, vb * 64, t0, bh, &bar_full[s]);
-            tma_load_3d(st + C::QB + C::KB + C::GB + C::VB + vb * BLK, &tdo, vb * 64, t0, bh, &bar_full[s]);
+            tma_load_3d(st + C::QB + C::KB + C::GB + vb * BLK, &tv, vb * 64, t0, bh, &bar_fullv[s]);
+            tma_load_3d(st + C::QB + C::KB + C::GB + C::VB + vb * BLK, &tdo, vb * 64, t0, bh, &bar_fullv[s]);
         }
     };
     if (tid == 0)
-        for (int i = 0; i < C::NS && i < ntiles; ++i) issue_loads(i, i);
+        for (int i = 0; i < C::NS && i < ntiles; ++i) {
+            issue_qkg(i, i);
+            issue_vo(i, i);
+        }
 
     int err = 0, n_mma = 0;
     for (int i = 0; i < ntiles; ++i) {
@@ -344,40 +360,41 @@ __global__ void __launch_bounds__(NT_B, 1)
 
         // ---- transform: k~ = i k e^-b in place; e^b kept (in place of g) for the dq epilogue
         bwd_transform<DKB, GATE, false, true>(sqr, sk, sg, tot, gam, rowE, rowEi, ghs, igs, P.scale, tid, A.status);
-        // pair mapping of the later q*dq prefix phase
-        constexpr int NP = DKB / 2, RG = NT_B / NP, RPG = TR / RG;
-        const int cp = tid % NP, rg = tid / NP, d = 2 * cp;
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        if (!block_wait(&bar_fullv[s], (i / C::NS) & 1)) { err = 1; break; }
 
         // ---- MMA group 1: dA = dO V^T, D = dO S^T, S += k~^T V
-        if (tid == 0) {
+        if (warp == 0) {
+            const bool leader = elect_one();
             const uint32_t ka = smem_u32(sk), va = smem_u32(sv), oa = smem_u32(so), sa = smem_u32(sS);
             const uint32_t idA = idesc_bf16(64, 64, 0, 0), idQ = idesc_bf16(64, DKB, 0, 0);
             const uint32_t idS = idesc_bf16(DKB, DV, 1, 1);
 #pragma unroll
             for (int kk = 0; kk < DV / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
-                mma_bf16(tbase + C::COL_R, sw128_desc(oa + koff, 16, 1024), sw128_desc(va + koff, 16, 1024), idA,
+                if (leader) mma_bf16(tbase + C::COL_R, sw128_desc(oa + koff, 16, 1024), sw128_desc(va + koff, 16, 1024), idA,
                          kk > 0);
             }
 #pragma unroll
             for (int kk = 0; kk < DV / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
                 const uint32_t soff = (kk >> 2) * (DKB * 128) + (kk & 3) * 32;
-                mma_bf16(tbase + (16u << 16) + C::COL_R, sw128_desc(oa + koff, 16, 1024),
+                if (leader) mma_bf16(tbase + (16u << 16) + C::COL_R, sw128_desc(oa + koff, 16, 1024),
                          sw128_desc(sa + soff, 16, 1024), idQ, kk > 0);
             }
 #pragma unroll
             for (int ks = 0; ks < TR / 16; ++ks)
-                mma_bf16(tbase, sw128_desc(ka + ks * 2048, BLK, 1024), sw128_desc(va + ks * 2048, BLK, 1024), idS, 1);
-            mma_commit(bar_mma1);
+                if (leader) mma_bf16(tbase, sw128_desc(ka + ks * 2048, BLK, 1024), sw128_desc(va + ks * 2048, BLK, 1024), idS, 1);
+            if (leader) mma_commit(bar_mma1);
+            __syncwarp();
         }
         ++n_mma;
         if (!block_wait(bar_mma1, i & 1)) { err = 1; break; }
         tc_fence_after();
+        if (tid == 0 && i + C::NS < ntiles) issue_vo(i + C::NS, s);
 
         // ---- masked dA -> shared; state pass S = e^Gamma (S + dS') in TMEM, bf16 copy
         {
@@ -424,14 +441,16 @@ __global__ void __launch_bounds__(NT_B, 1)
         tc_fence_after();
 
         // ---- MMA group 2: D += mask(dA) k~
-        if (tid == 0) {
+        if (warp == 0) {
+            const bool leader = elect_one();
             const uint32_t aa = smem_u32(sA), ka = smem_u32(sk);
             const uint32_t idQ = idesc_bf16(64, DKB, 0, 1);
 #pragma unroll
             for (int ks = 0; ks < TR / 16; ++ks)
-                mma_bf16(tbase + (16u << 16) + C::COL_R, sw128_desc(aa + ks * 32, 16, 1024),
+                if (leader) mma_bf16(tbase + (16u << 16) + C::COL_R, sw128_desc(aa + ks * 32, 16, 1024),
                          sw128_desc(ka + ks * 2048, BLK, 1024), idQ, 1);
-            mma_commit(bar_mma2);
+            if (leader) mma_commit(bar_mma2);
+            __syncwarp();
         }
         if (!block_wait(bar_mma2, i & 1)) { err = 1; break; }
         tc_fence_after();
@@ -550,7 +569,7 @@ __global__ void __launch_bounds__(NT_B, 1)
         __syncthreads();
         tc_fence_after();
         if (tid == 0) bulk_wait_read<0>();   // the dq store has read the k slot before it is reloaded
-        if (tid == 0 && i + C::NS < ntiles) issue_loads(i + C::NS, s);
+        if (tid == 0 && i + C::NS < ntiles) issue_qkg(i + C::NS, s);
     }
 
     if (!err) {
@@ -559,12 +578,15 @@ __global__ void __launch_bounds__(NT_B, 1)
         if (GATE == 2 && tid == 0) A.tq[(long)bh * A.nseg + z] = carry[0];
     }
     if (err) {
-        if (tid == 0) {
-            atomicOr(A.status, kDevStatusTimeout);
-            if (n_mma) {
-                mbar_wait(bar_mma1, (n_mma - 1) & 1, 1u << 20);
-                mbar_wait(bar_mma2, (n_mma - 1) & 1, 1u << 20);
+        if (warp == 0) {
+            // every product the issuing lane issued completes before TMEM and shared memory go away
+            const bool leader = elect_one();
+            if (leader) {
+                atomicOr(A.status, kDevStatusTimeout);
+                mma_commit(bar_drain);
+                mbar_wait(bar_drain, 0, 1u << 20);
             }
+            __syncwarp();
         }
     } else if (A.hT_ws && z == A.nseg - 1) {
         // final state (for the dg term of an upstream final-state gradient)
@@ -592,7 +614,7 @@ template <int DK, int DV, int GATE>
 struct KVCfg {
     static constexpr uint32_t QB = TR * DK * 2;
     static constexpr uint32_t KB = TR * DK * 2;
-    static constexpr uint32_t GB = GATE != 0 ? TR * DK * 4 : 0;  // g (per key), then k*dk scratch
+    static constexpr uint32_t GB = TR * DK * 4;  // g (per key: loaded; e^-b after the transform), k*dk scratch
     static constexpr uint32_t VB = TR * DV * 2;
     static constexpr uint32_t OB = TR * DV * 2;
     static constexpr uint32_t STAGE = QB + KB + GB + VB + OB;
@@ -602,8 +624,12 @@ struct KVCfg {
     static constexpr uint32_t SMALL = 256 + 8192 + 4 * DK + 1024 + 512 + 16 * DK + 256 + 64;
     static constexpr int NS = (2 * STAGE + GTB + 2 * AB + SMALL + 1024 <= 227 * 1024) ? 2 : 1;
     static constexpr uint32_t SMEM = NS * STAGE + GTB + 2 * AB + SMALL + 1024;
+    // TMEM: G [0, DV); from COL_R the dv accumulator (lanes 16-31, DV columns) and, in lanes
+    // 0-15, the dk' accumulator (DK columns) followed by A and dA (64 columns each)
     static constexpr uint32_t COL_R = DV;
-    static constexpr uint32_t WR = DK > DV ? (DK > 64 ? DK : 64) : (DV > 64 ? DV : 64);
+    static constexpr uint32_t COL_A = COL_R + DK;
+    static constexpr uint32_t COL_DA = COL_A + 64;
+    static constexpr uint32_t WR = DV > DK + 128 ? DV : DK + 128;
     static constexpr uint32_t NCOL = pow2cols(DV + WR);
     static constexpr int HC = DV / 2;
     static constexpr int KC = DK / 2;
@@ -628,6 +654,7 @@ __global__ void __launch_bounds__(NT_B, 1)
     uint64_t* bar_full = reinterpret_cast<uint64_t*>(small);
     uint64_t* bar_mma1 = bar_full + 2;
     uint64_t* bar_mma2 = bar_full + 3;
+    uint64_t* bar_drain = bar_full + 4;   // error path: completion of every product issued
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 64);
     float* tot = reinterpret_cast<float*>(small + 256);
     float* gam = tot + 2048;      // [DK]
@@ -657,6 +684,7 @@ __global__ void __launch_bounds__(NT_B, 1)
         mbar_init(&bar_full[1], 1);
         mbar_init(bar_mma1, 1);
         mbar_init(bar_mma2, 1);
+        mbar_init(bar_drain, 1);
         mbar_fence_init();
     }
     if (warp == 0) tmem_alloc(tmem_slot, C::NCOL);
@@ -746,11 +774,32 @@ __global__ void __launch_bounds__(NT_B, 1)
 
         // ---- transform: q~ = scale q e^b, k~ = i k e^-b (in place); e^-b kept in place of g
         bwd_transform<DK, GATE, true, false>(sq, sk, sg, tot, gam, rowE, rowEi, ghs, igs, P.scale, tid, A.status);
-        // pair mapping of the later dg phase
-        constexpr int NP = DK / 2, RG = NT_B / NP, RPG = TR / RG;
-        const int cp = tid % NP, rg = tid / NP, d = 2 * cp;
+        fence_proxy_async_smem();
         __syncthreads();
-        // ---- G~ = e^Gamma G in TMEM; bf16 copy
+        // ---- MMA group 1 (needs only this tile): A = (scale q~) k~^T, dA = dO V^T, both M=64 in
+        //      TMEM lanes 0-15 next to the dk' accumulator
+        if (warp == 0) {
+            const bool leader = elect_one();
+            tc_fence_after();
+            const uint32_t qa = smem_u32(sq), ka = smem_u32(sk), va = smem_u32(sv), oa = smem_u32(so);
+            const uint32_t id64 = idesc_bf16(64, 64, 0, 0);
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+                if (leader) mma_bf16(tbase + C::COL_A, sw128_desc(qa + koff, 16, 1024), sw128_desc(ka + koff, 16, 1024), id64,
+                         kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < DV / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+                if (leader) mma_bf16(tbase + C::COL_DA, sw128_desc(oa + koff, 16, 1024), sw128_desc(va + koff, 16, 1024), id64,
+                         kk > 0);
+            }
+            if (leader) mma_commit(bar_mma1);
+            __syncwarp();
+        }
+        ++n_mma;
+        // ---- G~ = e^Gamma G in TMEM; bf16 copy (runs while group 1 is in flight)
         {
             const float eg = GATE == 0 ? 1.f : gam[GATE == 1 ? srow : 0];
             for (int c = wg * C::HC; c < (wg + 1) * C::HC; c += 16) {
@@ -775,43 +824,53 @@ __global__ void __launch_bounds__(NT_B, 1)
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-
-        // ---- MMA group 1: A = (scale q~) k~^T, dA = dO V^T
-        if (tid == 0) {
+        // ---- MMA group 2a (needs G~, not P): dk' = V G~^T, dv = k~ G~, G += (scale q~)^T dO
+        const uint32_t tdk = tbase + C::COL_R, tdv = tbase + (16u << 16) + C::COL_R;
+        if (warp == 0) {
+            const bool leader = elect_one();
             const uint32_t qa = smem_u32(sq), ka = smem_u32(sk), va = smem_u32(sv), oa = smem_u32(so);
-            const uint32_t id64 = idesc_bf16(64, 64, 0, 0);
+            const uint32_t ga = smem_u32(sG);
+            const uint32_t idK2 = idesc_bf16(64, DK, 0, 0), idV2 = idesc_bf16(64, DV, 0, 1);
+            const uint32_t idG = idesc_bf16(DK, DV, 1, 1);
 #pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk) {
+            for (int kk = 0; kk < DV / 16; ++kk) {  // V G~^T
                 const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
-                mma_bf16(tbase + C::COL_R, sw128_desc(qa + koff, 16, 1024), sw128_desc(ka + koff, 16, 1024), id64,
+                const uint32_t goff = (kk >> 2) * (DK * 128) + (kk & 3) * 32;
+                if (leader) mma_bf16(tdk, sw128_desc(va + koff, 16, 1024), sw128_desc(ga + goff, 16, 1024), idK2, kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk) {  // k~ G~
+                const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+                if (leader) mma_bf16(tdv, sw128_desc(ka + koff, 16, 1024), sw128_desc(ga + kk * 2048, DK * 128, 1024), idV2,
                          kk > 0);
             }
 #pragma unroll
-            for (int kk = 0; kk < DV / 16; ++kk) {
-                const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
-                mma_bf16(tbase + (16u << 16) + C::COL_R, sw128_desc(oa + koff, 16, 1024),
-                         sw128_desc(va + koff, 16, 1024), id64, kk > 0);
-            }
-            mma_commit(bar_mma1);
+            for (int ks = 0; ks < TR / 16; ++ks)  // G += (scale q~)^T dO
+                if (leader) mma_bf16(tbase, sw128_desc(qa + ks * 2048, BLK, 1024), sw128_desc(oa + ks * 2048, BLK, 1024), idG, 1);
+            __syncwarp();
         }
-        ++n_mma;
         if (!block_wait(bar_mma1, i & 1)) { err = 1; break; }
         tc_fence_after();
+        // ---- P pass: masked A and masked dA -> bf16 in shared memory (rows in lanes 0-15)
         {
-            uint32_t r[32];
-            tmem_ld32(tlane + C::COL_R + 32 * wg, r);
+            uint32_t ra[32], rd[32];
+            tmem_ld32(tlane + C::COL_A + 32 * wg, ra);
+            tmem_ld32(tlane + C::COL_DA + 32 * wg, rd);
             tmem_wait_ld();
-            const int t = 16 * qd + (lane & 15);
-            uint8_t* dst = lane < 16 ? sAm : sdA;
+            if (lane < 16) {
+                const int t = 16 * qd + lane;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                float f[8];
+                for (int u = 0; u < 4; ++u) {
+                    float fa[8], fd[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int sidx = 32 * wg + 8 * u + j;
-                    f[j] = (sidx <= t) ? __uint_as_float(r[8 * u + j]) : 0.f;
+                    for (int j = 0; j < 8; ++j) {
+                        const int sidx = 32 * wg + 8 * u + j;
+                        fa[j] = (sidx <= t) ? __uint_as_float(ra[8 * u + j]) : 0.f;
+                        fd[j] = (sidx <= t) ? __uint_as_float(rd[8 * u + j]) : 0.f;
+                    }
+                    store8_bf16(sAm, sw128_off(t, 32 * wg + 8 * u, BLK), fa);
+                    store8_bf16(sdA, sw128_off(t, 32 * wg + 8 * u, BLK), fd);
                 }
-                store8_bf16(dst, sw128_off(t, 32 * wg + 8 * u, BLK), f);
             }
         }
         fence_proxy_async_smem();
@@ -819,38 +878,29 @@ __global__ void __launch_bounds__(NT_B, 1)
         __syncthreads();
         tc_fence_after();
 
-        // ---- MMA group 2: dk', dv, G update
-        if (tid == 0) {
-            const uint32_t qa = smem_u32(sq), ka = smem_u32(sk), va = smem_u32(sv), oa = smem_u32(so);
-            const uint32_t ga = smem_u32(sG), ama = smem_u32(sAm), dama = smem_u32(sdA);
-            const uint32_t tdk = tbase + C::COL_R, tdv = tbase + (16u << 16) + C::COL_R;
-            const uint32_t idK1 = idesc_bf16(64, DK, 1, 1), idK2 = idesc_bf16(64, DK, 0, 0);
-            const uint32_t idV1 = idesc_bf16(64, DV, 1, 1), idV2 = idesc_bf16(64, DV, 0, 1);
-            const uint32_t idG = idesc_bf16(DK, DV, 1, 1);
+        // ---- MMA group 2b: dk' += mask(dA)^T (scale q~), dv += mask(A)^T dO
+        if (warp == 0) {
+            const bool leader = elect_one();
+            const uint32_t qa = smem_u32(sq), oa = smem_u32(so);
+            const uint32_t ama = smem_u32(sAm), dama = smem_u32(sdA);
+            const uint32_t idK1 = idesc_bf16(64, DK, 1, 1), idV1 = idesc_bf16(64, DV, 1, 1);
 #pragma unroll
-            for (int ks = 0; ks < TR / 16; ++ks)  // mask(dA)^T (scale q~)
-                mma_bf16(tdk, sw128_desc(dama + ks * 2048, BLK, 1024), sw128_desc(qa + ks * 2048, BLK, 1024), idK1,
-                         ks > 0);
+            for (int ks = 0; ks < TR / 16; ++ks)
+                if (leader) mma_bf16(tdk, sw128_desc(dama + ks * 2048, BLK, 1024), sw128_desc(qa + ks * 2048, BLK, 1024), idK1, 1);
 #pragma unroll
-            for (int kk = 0; kk < DV / 16; ++kk) {  // V G~^T
-                const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
-                const uint32_t goff = (kk >> 2) * (DK * 128) + (kk & 3) * 32;
-                mma_bf16(tdk, sw128_desc(va + koff, 16, 1024), sw128_desc(ga + goff, 16, 1024), idK2, 1);
-            }
-#pragma unroll
-            for (int ks = 0; ks < TR / 16; ++ks)  // mask(A)^T dO
-                mma_bf16(tdv, sw128_desc(ama + ks * 2048, BLK, 1024), sw128_desc(oa + ks * 2048, BLK, 1024), idV1,
-                         ks > 0);
-#pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk) {  // k~ G~
-                const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
-                mma_bf16(tdv, sw128_desc(ka + koff, 16, 1024), sw128_desc(ga + kk * 2048, DK * 128, 1024), idV2, 1);
-            }
-#pragma unroll
-            for (int ks = 0; ks < TR / 16; ++ks)  // G += (scale q~)^T dO
-                mma_bf16(tbase, sw128_desc(qa + ks * 2048, BLK, 1024), sw128_desc(oa + ks * 2048, BLK, 1024), idG, 1);
-            mma_commit(bar_mma2);
+            for (int ks = 0; ks < TR / 16; ++ks)
+                if (leader) mma_bf16(tdv, sw128_desc(ama + ks * 2048, BLK, 1024), sw128_desc(oa + ks * 2048, BLK, 1024), idV1, 1);
+            if (leader) mma_commit(bar_mma2);
+            __syncwarp();
         }
+        // the dq kernel's exclusive prefixes of this tile's rows, in flight during the epilogue
+        constexpr int NGR = NT_B / DK, RPR = TR / NGR;
+        const int dc = tid % DK, gr = tid / DK;
+        float* dgp = A.dg + (rowbase + t0 + gr * RPR) * DK + dc;
+        float pre[GATE == 1 ? RPR : 1];
+        if (GATE == 1)
+#pragma unroll
+            for (int rr = 0; rr < RPR; ++rr) pre[rr] = (t0 + gr * RPR + rr < P.L) ? dgp[(long)rr * DK] : 0.f;
         if (!block_wait(bar_mma2, i & 1)) { err = 1; break; }
         tc_fence_after();
 
@@ -925,14 +975,8 @@ __global__ void __launch_bounds__(NT_B, 1)
         if (A.di && tid < TR && t0 + tid < P.L) A.di[rowbase + t0 + tid] = (sdi[tid] + sdi[TR + tid]) / igs[tid];
         // ---- dg = (in-segment q*dq total - exclusive prefix) - reverse sum of k*dk + carry
         if (GATE == 1) {
-            // thread = (key dim dc, group of RPR rows): prefetch the dq kernel's prefixes, local
+            // thread = (key dim dc, group of RPR rows; the prefixes were fetched above): local
             // sums, exchange, then the reverse walk
-            constexpr int NGR = NT_B / DK, RPR = TR / NGR;
-            const int dc = tid % DK, gr = tid / DK;
-            float* dgp = A.dg + (rowbase + t0 + gr * RPR) * DK + dc;
-            float pre[RPR];
-#pragma unroll
-            for (int rr = 0; rr < RPR; ++rr) pre[rr] = (t0 + gr * RPR + rr < P.L) ? dgp[(long)rr * DK] : 0.f;
             float loc = 0.f;
 #pragma unroll 8
             for (int rr = 0; rr < RPR; ++rr) loc += sg[gsw(gr * RPR + rr, dc)];
@@ -986,12 +1030,15 @@ __global__ void __launch_bounds__(NT_B, 1)
     }
 
     if (err) {
-        if (tid == 0) {
-            atomicOr(A.status, kDevStatusTimeout);
-            if (n_mma) {
-                mbar_wait(bar_mma1, (n_mma - 1) & 1, 1u << 20);
-                mbar_wait(bar_mma2, (n_mma - 1) & 1, 1u << 20);
+        if (warp == 0) {
+            // every product the issuing lane issued completes before TMEM and shared memory go away
+            const bool leader = elect_one();
+            if (leader) {
+                atomicOr(A.status, kDevStatusTimeout);
+                mma_commit(bar_drain);
+                mbar_wait(bar_drain, 0, 1u << 20);
             }
+            __syncwarp();
         }
     } else if (A.dh0 && z == 0) {
         for (int c = wg * C::HC; c < (wg + 1) * C::HC; c += 16) {
