@@ -328,11 +328,16 @@ def main():
     ws = torch.empty(max(ops.gla_workspace_bytes(prob, False), ops.gla_workspace_bytes(prob, True) if w.backward
                          else 0), dtype=torch.uint8, device=dev)
 
+    # training pair: the forward leaves the states the backward's segments start from
+    nsaved = ops.gla_saved_states_bytes(prob) if w.backward else 0
+    saved = torch.empty(max(nsaved // 4, 1), dtype=torch.float32, device=dev) if nsaved else None
+
     def step():
-        ops.gla_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["igate"], xd["h0"], workspace=ws, **kw)
+        ops.gla_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["igate"], xd["h0"], workspace=ws, saved_states=saved,
+                    **kw)
         if w.backward:
             ops.gla_bwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["igate"], xd["h0"], xd["dO"], None, workspace=ws,
-                        **kw)
+                        saved_states=saved, **kw)
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     sampler = ClockSampler(local)
@@ -379,10 +384,12 @@ def main():
 
         def e2e_step():
             nonlocal d2h
-            o, hT = ops.gla_fwd(xh["q"], xh["k"], xh["v"], xh["g"], xh["igate"], xh["h0"], **kw)
+            o, hT = ops.gla_fwd(xh["q"], xh["k"], xh["v"], xh["g"], xh["igate"], xh["h0"], saved_states=saved,
+                                **kw)
             nb = o.numel() * o.element_size() + hT.numel() * hT.element_size()
             if w.backward:
-                r = ops.gla_bwd(xh["q"], xh["k"], xh["v"], xh["g"], xh["igate"], xh["h0"], xh["dO"], None, **kw)
+                r = ops.gla_bwd(xh["q"], xh["k"], xh["v"], xh["g"], xh["igate"], xh["h0"], xh["dO"], None,
+                                saved_states=saved, **kw)
                 nb += sum(t.numel() * t.element_size() for t in r.values() if t is not None)
             d2h = nb
 

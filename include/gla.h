@@ -116,6 +116,29 @@ GLA_API gla_status gla_bwd(const gla_problem* p, const void* q, const void* k, c
                    void* dq, void* dk, void* dv, float* dg, float* di, float* dh0,
                    void* ws, size_t ws_bytes, void* stream);
 
+/* Saved states: the training pair forward -> backward without recomputation.
+ * gla_saved_states_bytes: bytes of the f32 buffer in which gla_fwd_save leaves, for
+ *   gla_bwd_saved, the states at the segment boundaries of the backward's tensor-core plan
+ *   (layout [B*H][nseg][Dk][Dv], entry 0 unused); 0 when that backward needs none (CUDA-core
+ *   plan, one segment) or the problem is invalid.
+ * gla_fwd_save: gla_fwd that also writes those states into `saved` (NULL, or a buffer of
+ *   gla_saved_states_bytes(p) bytes owned by the caller; ignored when that is 0). They come
+ *   from the tensor-core forward: GLA_ERR_UNSUPPORTED if the forward's plan is the CUDA-core
+ *   one while the backward needs saved states.
+ * gla_bwd_saved: gla_bwd that takes them instead of recomputing (skips one pass over k, v, g
+ *   and a scan). `saved` must come from gla_fwd_save with the same problem and the same q, k,
+ *   v, g, igate, h0; NULL means recompute (the same as gla_bwd).
+ * Other arguments, results and errors as for gla_fwd / gla_bwd. */
+GLA_API size_t gla_saved_states_bytes(const gla_problem* p);
+GLA_API gla_status gla_fwd_save(const gla_problem* p, const void* q, const void* k, const void* v,
+                                const float* g, const float* igate, const float* h0,
+                                void* o, float* hT, float* saved, void* ws, size_t ws_bytes, void* stream);
+GLA_API gla_status gla_bwd_saved(const gla_problem* p, const void* q, const void* k, const void* v,
+                                 const float* g, const float* igate, const float* h0,
+                                 const void* dO, const float* dhT, const float* saved,
+                                 void* dq, void* dk, void* dv, float* dg, float* di, float* dh0,
+                                 void* ws, size_t ws_bytes, void* stream);
+
 /* Static description of a status code (never NULL). */
 GLA_API const char* gla_status_string(gla_status s);
 

@@ -19,7 +19,8 @@ GLA_PLAN_AUTO, GLA_PLAN_SIMT, GLA_PLAN_TC = 0, 1, 2
 # Every symbol include/gla.h declares (checked by tests/test_abi_symbols.py).
 EXPORTED = ("gla_workspace_bytes", "gla_fwd", "gla_bwd", "gla_status_string",
             "gla_check_device_status", "gla_version", "gla_launch_count", "gla_profiler_enable",
-            "gla_profiler_read", "gla_fwd_static_scratch", "gla_last_error_detail", "gla_plan_info")
+            "gla_profiler_read", "gla_fwd_static_scratch", "gla_last_error_detail", "gla_plan_info",
+            "gla_saved_states_bytes", "gla_fwd_save", "gla_bwd_saved")
 
 
 class GlaProblem(ctypes.Structure):
@@ -55,6 +56,12 @@ def _load():
     lib.gla_fwd.restype = ctypes.c_int
     lib.gla_bwd.argtypes = [pp, vp, vp, vp, fp, fp, fp, vp, fp, vp, vp, vp, fp, fp, fp, vp, sz, vp]
     lib.gla_bwd.restype = ctypes.c_int
+    lib.gla_saved_states_bytes.argtypes = [pp]
+    lib.gla_saved_states_bytes.restype = sz
+    lib.gla_fwd_save.argtypes = [pp, vp, vp, vp, fp, fp, fp, vp, fp, fp, vp, sz, vp]
+    lib.gla_fwd_save.restype = ctypes.c_int
+    lib.gla_bwd_saved.argtypes = [pp, vp, vp, vp, fp, fp, fp, vp, fp, fp, vp, vp, vp, fp, fp, fp, vp, sz, vp]
+    lib.gla_bwd_saved.restype = ctypes.c_int
     lib.gla_status_string.argtypes = [ctypes.c_int]
     lib.gla_status_string.restype = ctypes.c_char_p
     lib.gla_check_device_status.argtypes = [vp, vp]

@@ -120,9 +120,25 @@ size_t gla_workspace_bytes(const gla_problem* p, int for_backward) {
     return ws_bytes(P, plan, for_backward != 0);
 }
 
+size_t gla_saved_states_bytes(const gla_problem* p) {
+    Dims P;
+    int plan;
+    if (check_problem(p, &P, &plan) != GLA_OK) return 0;
+    if (resolve(p, P, true, &plan) != GLA_OK || plan != GLA_PLAN_TC) return 0;
+    int nseg = 1, tps = 0;
+    tc::bwd_plan_info(P, &nseg, &tps);
+    return nseg > 1 ? 4 * (size_t)P.B * P.H * nseg * P.Dk * P.Dv : 0;
+}
+
 gla_status gla_fwd(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
                    const float* igate, const float* h0, void* o, float* hT, void* ws, size_t ws_bytes_given,
                    void* stream) {
+    return gla_fwd_save(p, q, k, v, g, igate, h0, o, hT, nullptr, ws, ws_bytes_given, stream);
+}
+
+gla_status gla_fwd_save(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
+                        const float* igate, const float* h0, void* o, float* hT, float* saved, void* ws,
+                        size_t ws_bytes_given, void* stream) {
     Dims P;
     int plan;
     gla_status s = check_problem(p, &P, &plan);
@@ -133,16 +149,20 @@ gla_status gla_fwd(const gla_problem* p, const void* q, const void* k, const voi
     if (!empty && (!q || !k || !v || !o)) return GLA_ERR_INVALID_ARG;
     if ((p->gate == GLA_GATE_NONE) != (g == nullptr) && !empty) return GLA_ERR_INVALID_ARG;
     if (!ws) return GLA_ERR_INVALID_ARG;
-    const void* ptrs[] = {q, k, v, g, igate, h0, o, hT, ws};
+    const void* ptrs[] = {q, k, v, g, igate, h0, o, hT, saved, ws};
     for (const void* x : ptrs)
         if (!aligned16(x)) return GLA_ERR_INVALID_ARG;
     if (ws_bytes_given < ws_bytes(P, plan, false)) return GLA_ERR_WORKSPACE;
+    // saved states are only needed (and written) when the backward runs on tensor cores in
+    // more than one segment; they are written by the tensor-core forward
+    if (saved && gla_saved_states_bytes(p) == 0) saved = nullptr;
+    if (saved && plan != GLA_PLAN_TC) return GLA_ERR_UNSUPPORTED;
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, st);
     if (e != cudaSuccess) return map_cuda(e, "status word reset");
     if ((size_t)P.B * P.H == 0) return GLA_OK;
     if (plan == GLA_PLAN_TC && P.L > 0)
-        e = tc::fwd(P, q, k, v, g, igate, h0, o, hT, ws, st);
+        e = tc::fwd(P, q, k, v, g, igate, h0, o, hT, saved, ws, st);
     else
         e = simt::fwd(P, p->io, q, k, v, g, igate, h0, o, hT, ws, st);
     return map_cuda(e);
@@ -151,6 +171,14 @@ gla_status gla_fwd(const gla_problem* p, const void* q, const void* k, const voi
 gla_status gla_bwd(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
                    const float* igate, const float* h0, const void* dO, const float* dhT, void* dq, void* dk,
                    void* dv, float* dg, float* di, float* dh0, void* ws, size_t ws_bytes_given, void* stream) {
+    return gla_bwd_saved(p, q, k, v, g, igate, h0, dO, dhT, nullptr, dq, dk, dv, dg, di, dh0, ws, ws_bytes_given,
+                         stream);
+}
+
+gla_status gla_bwd_saved(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
+                         const float* igate, const float* h0, const void* dO, const float* dhT, const float* saved,
+                         void* dq, void* dk, void* dv, float* dg, float* di, float* dh0, void* ws,
+                         size_t ws_bytes_given, void* stream) {
     Dims P;
     int plan;
     gla_status s = check_problem(p, &P, &plan);
@@ -163,7 +191,7 @@ gla_status gla_bwd(const gla_problem* p, const void* q, const void* k, const voi
     if (!empty && (p->gate == GLA_GATE_NONE) != (dg == nullptr)) return GLA_ERR_INVALID_ARG;
     if (di && !igate) return GLA_ERR_INVALID_ARG;
     if (!ws) return GLA_ERR_INVALID_ARG;
-    const void* ptrs[] = {q, k, v, g, igate, h0, dO, dhT, dq, dk, dv, dg, di, dh0, ws};
+    const void* ptrs[] = {q, k, v, g, igate, h0, dO, dhT, saved, dq, dk, dv, dg, di, dh0, ws};
     for (const void* x : ptrs)
         if (!aligned16(x)) return GLA_ERR_INVALID_ARG;
     if (ws_bytes_given < ws_bytes(P, plan, true)) return GLA_ERR_WORKSPACE;
@@ -172,7 +200,8 @@ gla_status gla_bwd(const gla_problem* p, const void* q, const void* k, const voi
     if (e != cudaSuccess) return map_cuda(e, "status word reset");
     if ((size_t)P.B * P.H == 0) return GLA_OK;
     if (plan == GLA_PLAN_TC && P.L > 0)
-        e = tc::bwd(P, q, k, v, g, igate, h0, dO, dhT, dq, dk, dv, dg, di, dh0, ws, st);
+        e = tc::bwd(P, q, k, v, g, igate, h0, dO, dhT, dq, dk, dv, dg, di, dh0,
+                    gla_saved_states_bytes(p) ? saved : nullptr, ws, st);
     else
         e = simt::bwd(P, p->io, q, k, v, g, igate, h0, dO, dhT, dq, dk, dv, dg, di, dh0, ws, st);
     return map_cuda(e);

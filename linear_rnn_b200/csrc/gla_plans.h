@@ -23,8 +23,10 @@ struct FwdPlan {
 FwdPlan plan_fwd(const Dims& P);
 bool supports(const Dims& P);
 size_t fwd_workspace_bytes(const Dims& P);
+// saved (nullable): [BH, nseg_b, Dk, Dv] states entering the backward plan's segments
+// z = 1 .. nseg_b-1 (bwd_plan_info), written on the way
 cudaError_t fwd(const Dims& P, const void* q, const void* k, const void* v, const float* g, const float* ig,
-                const float* h0, void* o, float* hT, void* ws, cudaStream_t st);
+                const float* h0, void* o, float* hT, float* saved, void* ws, cudaStream_t st);
 // Segment state passes and scans shared by the forward and the backward.
 //   mode 1: forward local end states of segments 0..nseg-2 (a = k, b = v)
 //   mode 2: reverse local state gradients of segments 1..nseg-1 (a = q, b = dO)
@@ -40,8 +42,9 @@ int num_sms();
 bool bwd_supports(const Dims& P);
 size_t bwd_workspace_bytes(const Dims& P);
 void bwd_plan_info(const Dims& P, int* nseg, int* tiles_per_seg);
+// saved (nullable): the states a forward wrote for this problem; skips the forward state pass
 cudaError_t bwd(const Dims& P, const void* q, const void* k, const void* v, const float* g, const float* ig,
                 const float* h0, const void* dO, const float* dhT, void* dq, void* dk, void* dv, float* dg, float* di,
-                float* dh0, void* ws, cudaStream_t st);
+                float* dh0, const float* saved, void* ws, cudaStream_t st);
 }  // namespace tc
 }  // namespace gla

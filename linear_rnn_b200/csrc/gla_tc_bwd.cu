@@ -1165,7 +1165,8 @@ static cudaError_t launch_dkdv(const Dims& P, const BwdPlan& pl, const CUtensorM
 template <int DK, int DV, int GATE>
 static cudaError_t run_bwd(const Dims& P, const void* q, const void* k, const void* v, const float* g,
                            const float* ig, const float* h0, const void* dO, const float* dhT, void* dq, void* dk,
-                           void* dv, float* dg, float* di, float* dh0, void* ws, cudaStream_t st) {
+                           void* dv, float* dg, float* di, float* dh0, const float* saved, void* ws,
+                           cudaStream_t st) {
     const BwdPlan pl = plan_bwd(P);
     const BwdWs w = bwd_layout(P, static_cast<char*>(ws));
     const int BH = P.B * P.H;
@@ -1188,7 +1189,9 @@ static cudaError_t run_bwd(const Dims& P, const void* q, const void* k, const vo
     }
     int* status = static_cast<int*>(ws);
     cudaError_t e;
-    if (pl.nseg > 1) {
+    // segment initial states: from the forward that saved them, else a state pass + scan
+    const float* sinit = saved ? saved : w.sinit;
+    if (pl.nseg > 1 && !saved) {
         e = state_pass(P, 1, k, v, g, ig, pl.nseg, pl.tiles_per_seg, w.seg_state, w.seg_gamma, status, st);
         if (e != cudaSuccess) return e;
         e = seg_scan(P, pl.nseg, w.seg_state, w.seg_gamma, h0, w.sinit, st);
@@ -1197,7 +1200,7 @@ static cudaError_t run_bwd(const Dims& P, const void* q, const void* k, const vo
     BwdArgs a{};
     a.gh = GATE == 2 ? g : nullptr;
     a.ig = ig;
-    a.sinit = w.sinit;
+    a.sinit = sinit;
     a.h0 = h0;
     a.gend = w.gend;
     a.dhT = dhT;
@@ -1228,21 +1231,22 @@ static cudaError_t run_bwd(const Dims& P, const void* q, const void* k, const vo
 template <int DK, int DV>
 static cudaError_t bwd_gate(const Dims& P, const void* q, const void* k, const void* v, const float* g,
                             const float* ig, const float* h0, const void* dO, const float* dhT, void* dq, void* dk,
-                            void* dv, float* dg, float* di, float* dh0, void* ws, cudaStream_t st) {
+                            void* dv, float* dg, float* di, float* dh0, const float* saved, void* ws,
+                            cudaStream_t st) {
     switch (P.gate) {
-        case GLA_GATE_NONE: return run_bwd<DK, DV, 0>(P, q, k, v, g, ig, h0, dO, dhT, dq, dk, dv, dg, di, dh0, ws, st);
+        case GLA_GATE_NONE: return run_bwd<DK, DV, 0>(P, q, k, v, g, ig, h0, dO, dhT, dq, dk, dv, dg, di, dh0, saved, ws, st);
         case GLA_GATE_PER_KEY:
-            return run_bwd<DK, DV, 1>(P, q, k, v, g, ig, h0, dO, dhT, dq, dk, dv, dg, di, dh0, ws, st);
-        default: return run_bwd<DK, DV, 2>(P, q, k, v, g, ig, h0, dO, dhT, dq, dk, dv, dg, di, dh0, ws, st);
+            return run_bwd<DK, DV, 1>(P, q, k, v, g, ig, h0, dO, dhT, dq, dk, dv, dg, di, dh0, saved, ws, st);
+        default: return run_bwd<DK, DV, 2>(P, q, k, v, g, ig, h0, dO, dhT, dq, dk, dv, dg, di, dh0, saved, ws, st);
     }
 }
 
 cudaError_t bwd(const Dims& P, const void* q, const void* k, const void* v, const float* g, const float* ig,
                 const float* h0, const void* dO, const float* dhT, void* dq, void* dk, void* dv, float* dg, float* di,
-                float* dh0, void* ws, cudaStream_t st) {
+                float* dh0, const float* saved, void* ws, cudaStream_t st) {
 #define GLA_BWD_CASE(DK_, DV_)                                                                      \
     if (P.Dk == DK_ && P.Dv == DV_)                                                                 \
-        return bwd_gate<DK_, DV_>(P, q, k, v, g, ig, h0, dO, dhT, dq, dk, dv, dg, di, dh0, ws, st);
+        return bwd_gate<DK_, DV_>(P, q, k, v, g, ig, h0, dO, dhT, dq, dk, dv, dg, di, dh0, saved, ws, st);
     GLA_BWD_CASE(64, 64)
     GLA_BWD_CASE(64, 128)
     GLA_BWD_CASE(64, 256)

@@ -117,6 +117,10 @@ struct FwdArgs {
     int tiles_per_seg;
     int nseg;
     int seg_offset;       // segment index = blockIdx.z + seg_offset
+    float* saved;         // output pass: [BH, save_nseg, Dk, Dv] states entering the backward's
+                          // segments (entry z after save_tps * z tiles), or null
+    int save_tps;
+    int save_nseg;
 };
 
 template <int DK, int DVT, int GATE, int MODE>
@@ -505,6 +509,12 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
             tc_fence_after();
             const float* gam = gamb + b * DK;
             const float* gaml = gamlb + b * DK;
+            // the state after this tile enters backward segment save_z when a boundary follows it
+            int save_z = 0;
+            if (MODE == 0 && A.saved) {
+                const int nxt = tile_at(i) + 1;
+                if (nxt % A.save_tps == 0 && nxt / A.save_tps < A.save_nseg) save_z = nxt / A.save_tps;
+            }
 #pragma unroll
             for (int h = 0; h < C::NH; ++h) {
                 const int d = srow(h);
@@ -527,6 +537,12 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     if (MODE == 0 && srow_ok)
 #pragma unroll
                         for (int j = 0; j < C::CH; j += 8) store8_bf16(sS, sw128_off(d, col + j, DK * 128), &f[j]);
+                    if (MODE == 0 && save_z > 0 && srow_ok) {
+                        float* dst = A.saved + (((long)bh * A.save_nseg + save_z) * DK + d) * P.Dv + e0 + col;
+#pragma unroll
+                        for (int j = 0; j < C::CH; j += 4)
+                            *reinterpret_cast<float4*>(dst + j) = make_float4(f[j], f[j + 1], f[j + 2], f[j + 3]);
+                    }
                 }
             }
             tmem_wait_st();
@@ -798,7 +814,8 @@ static cudaError_t state_run(const Dims& P, int mode, const void* a_src, const v
 
 template <int DK, int DVT, int GATE>
 static cudaError_t run(const Dims& P, const void* q, const void* k, const void* v, const float* g,
-                       const float* ig, const float* h0, void* o, float* hT, void* ws, cudaStream_t st) {
+                       const float* ig, const float* h0, void* o, float* hT, float* saved, void* ws,
+                       cudaStream_t st) {
     const FwdPlan pl = plan_fwd(P);
     CUtensorMap mq, mk, mv, mg, mo;
     const int BH = P.B * P.H;
@@ -823,6 +840,10 @@ static cudaError_t run(const Dims& P, const void* q, const void* k, const void* 
     a.tiles_per_seg = pl.tiles_per_seg;
     a.nseg = pl.nseg;
     a.seg_offset = 0;
+    if (saved) {
+        a.saved = saved;
+        bwd_plan_info(P, &a.save_nseg, &a.save_tps);
+    }
     if (pl.nseg > 1) {
         char* w = static_cast<char*>(ws);
         size_t off = kStatusBytes;
@@ -861,11 +882,12 @@ cudaError_t seg_rscan(const Dims& P, int nseg, const float* seg_state, const flo
 
 template <int DK, int DVT>
 static cudaError_t run_gate(const Dims& P, const void* q, const void* k, const void* v, const float* g,
-                            const float* ig, const float* h0, void* o, float* hT, void* ws, cudaStream_t st) {
+                            const float* ig, const float* h0, void* o, float* hT, float* saved, void* ws,
+                            cudaStream_t st) {
     switch (P.gate) {
-        case GLA_GATE_NONE: return run<DK, DVT, 0>(P, q, k, v, g, ig, h0, o, hT, ws, st);
-        case GLA_GATE_PER_KEY: return run<DK, DVT, 1>(P, q, k, v, g, ig, h0, o, hT, ws, st);
-        default: return run<DK, DVT, 2>(P, q, k, v, g, ig, h0, o, hT, ws, st);
+        case GLA_GATE_NONE: return run<DK, DVT, 0>(P, q, k, v, g, ig, h0, o, hT, saved, ws, st);
+        case GLA_GATE_PER_KEY: return run<DK, DVT, 1>(P, q, k, v, g, ig, h0, o, hT, saved, ws, st);
+        default: return run<DK, DVT, 2>(P, q, k, v, g, ig, h0, o, hT, saved, ws, st);
     }
 }
 
@@ -895,17 +917,17 @@ cudaError_t state_pass(const Dims& P, int mode, const void* a_src, const void* b
 }
 
 cudaError_t fwd(const Dims& P, const void* q, const void* k, const void* v, const float* g, const float* ig,
-                const float* h0, void* o, float* hT, void* ws, cudaStream_t st) {
+                const float* h0, void* o, float* hT, float* saved, void* ws, cudaStream_t st) {
     const int dvt = pick_dvt(P);
     if (P.Dk == 64) {
-        if (dvt == 128) return run_gate<64, 128>(P, q, k, v, g, ig, h0, o, hT, ws, st);
-        return run_gate<64, 64>(P, q, k, v, g, ig, h0, o, hT, ws, st);
+        if (dvt == 128) return run_gate<64, 128>(P, q, k, v, g, ig, h0, o, hT, saved, ws, st);
+        return run_gate<64, 64>(P, q, k, v, g, ig, h0, o, hT, saved, ws, st);
     }
     if (P.Dk == 128) {
-        if (dvt == 128) return run_gate<128, 128>(P, q, k, v, g, ig, h0, o, hT, ws, st);
-        return run_gate<128, 64>(P, q, k, v, g, ig, h0, o, hT, ws, st);
+        if (dvt == 128) return run_gate<128, 128>(P, q, k, v, g, ig, h0, o, hT, saved, ws, st);
+        return run_gate<128, 64>(P, q, k, v, g, ig, h0, o, hT, saved, ws, st);
     }
-    return run_gate<256, 64>(P, q, k, v, g, ig, h0, o, hT, ws, st);
+    return run_gate<256, 64>(P, q, k, v, g, ig, h0, o, hT, saved, ws, st);
 }
 
 }  // namespace tc

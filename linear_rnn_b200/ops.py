@@ -99,10 +99,17 @@ def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
+def gla_saved_states_bytes(problem: GlaProblem) -> int:
+    return int(_lib.lib.gla_saved_states_bytes(ctypes.byref(problem)))
+
+
 def gla_fwd(q, k, v, g=None, igate=None, h0=None, *, scale: Optional[float] = None, chunk: int = 64,
             plan: str = "auto", output_final_state: bool = True,
-            workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """Forward pass. Returns (o, hT); hT is None when output_final_state is False."""
+            workspace: Optional[torch.Tensor] = None,
+            saved_states: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Forward pass. Returns (o, hT); hT is None when output_final_state is False.
+    saved_states: optional device buffer (at least gla_saved_states_bytes) that receives the
+    states gla_bwd(..., saved_states=) then uses instead of recomputing them."""
     host = q.device.type != "cuda"
     device = torch.device("cuda", torch.cuda.current_device()) if host else q.device
     q, k, v, g, igate, h0 = (_to_dev(t, device) for t in (q, k, v, g, igate, h0))
@@ -114,19 +121,32 @@ def gla_fwd(q, k, v, g=None, igate=None, h0=None, *, scale: Optional[float] = No
     if nbytes == 0:
         raise GlaError(_lib.GLA_ERR_UNSUPPORTED, "gla_workspace_bytes")
     ws = _workspace(nbytes, device, workspace)
-    st = _lib.lib.gla_fwd(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(igate), _ptr(h0),
-                          _ptr(o), _ptr(hT), _ptr(ws), ws.numel() * ws.element_size(), _stream_handle(device))
+    _check_saved(saved_states, prob)
+    st = _lib.lib.gla_fwd_save(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(igate), _ptr(h0),
+                               _ptr(o), _ptr(hT), _ptr(saved_states), _ptr(ws), ws.numel() * ws.element_size(),
+                               _stream_handle(device))
     _check(st, "gla_fwd")
     if host:
         o, hT = _to_host([o, hT])
     return o, hT
 
 
+def _check_saved(saved, prob):
+    if saved is None:
+        return
+    if saved.device.type != "cuda" or saved.dtype != torch.float32 or not saved.is_contiguous():
+        raise ValueError("saved_states must be a contiguous float32 CUDA tensor")
+    if saved.numel() * 4 < gla_saved_states_bytes(prob):
+        raise GlaError(_lib.GLA_ERR_WORKSPACE, "saved_states")
+
+
 def gla_bwd(q, k, v, g, igate, h0, dO, dhT=None, *, scale: Optional[float] = None, chunk: int = 64,
             plan: str = "auto", output_dh0: bool = True,
-            workspace: Optional[torch.Tensor] = None) -> Dict[str, Optional[torch.Tensor]]:
+            workspace: Optional[torch.Tensor] = None,
+            saved_states: Optional[torch.Tensor] = None) -> Dict[str, Optional[torch.Tensor]]:
     """Backward pass. Returns dict dq, dk, dv, dg (None if ungated), di (None without an
-    input gate), dh0 (None when output_dh0 is False)."""
+    input gate), dh0 (None when output_dh0 is False). saved_states: the buffer a gla_fwd on
+    the same inputs filled, or None to recompute."""
     host = q.device.type != "cuda"
     device = torch.device("cuda", torch.cuda.current_device()) if host else q.device
     q, k, v, g, igate, h0, dO, dhT = (_to_dev(t, device) for t in (q, k, v, g, igate, h0, dO, dhT))
@@ -142,9 +162,11 @@ def gla_bwd(q, k, v, g, igate, h0, dO, dhT=None, *, scale: Optional[float] = Non
     if nbytes == 0:
         raise GlaError(_lib.GLA_ERR_UNSUPPORTED, "gla_workspace_bytes")
     ws = _workspace(nbytes, device, workspace)
-    st = _lib.lib.gla_bwd(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(igate), _ptr(h0),
-                          _ptr(dO), _ptr(dhT), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(di), _ptr(dh0),
-                          _ptr(ws), ws.numel() * ws.element_size(), _stream_handle(device))
+    _check_saved(saved_states, prob)
+    st = _lib.lib.gla_bwd_saved(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(igate), _ptr(h0),
+                                _ptr(dO), _ptr(dhT), _ptr(saved_states), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
+                                _ptr(di), _ptr(dh0), _ptr(ws), ws.numel() * ws.element_size(),
+                                _stream_handle(device))
     _check(st, "gla_bwd")
     out = {"dq": dq, "dk": dk, "dv": dv, "dg": dg, "di": di, "dh0": dh0}
     if host:

@@ -69,6 +69,18 @@ def test_workspace_sizes():
     assert ws_bytes(chunk=256)[0] < ws_bytes(chunk=64)[0]
 
 
+def test_saved_state_sizes_follow_the_backward_plan():
+    saved = lambda **kw: _lib.lib.gla_saved_states_bytes(ctypes.byref(prob(**kw)))
+    # tensor-core backward in several segments: one f32 state per (head, segment)
+    p = prob(B=4, H=16, L=4096, Dk=128, Dv=256, plan=_lib.GLA_PLAN_AUTO)
+    _, nseg, _ = _lib.plan_info(p, True)
+    assert nseg > 1
+    assert saved(B=4, H=16, L=4096, Dk=128, Dv=256, plan=_lib.GLA_PLAN_AUTO) == 4 * 64 * nseg * 128 * 256
+    assert saved(plan=_lib.GLA_PLAN_SIMT) == 0            # CUDA-core backward recomputes
+    assert saved(io=_lib.GLA_F32, plan=_lib.GLA_PLAN_AUTO) == 0
+    assert saved(Dk=96) == 0                                # invalid problem
+
+
 def test_status_strings():
     for s in range(7):
         assert len(_lib.status_string(s)) >= 2

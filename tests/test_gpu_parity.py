@@ -224,6 +224,35 @@ def test_strong_gates_flagged_on_tensor_cores_and_exact_on_simt():
     check_bwd(x, w, plan="simt")
 
 
+@pytest.mark.parametrize("name,L", [("c3", None), ("c3", 1000), ("c2", 700)])
+def test_backward_from_saved_states(name, L):
+    """The training pair: the forward writes the states at the backward's segment starts and
+    the backward uses them instead of its own state pass; same oracle bound, and close to the
+    recomputing backward."""
+    w = I.WORKLOADS[name].replace(backward=True)
+    if L is not None:
+        w = w.replace(L=L)
+    heads = [3, 40] if L is None else None
+    x = I.make_inputs(w, seed=2)
+    xd = to_cuda(x)
+    prob = ops().make_problem(xd["q"], xd["v"], xd["g"], scale=w.scale, chunk=w.chunk, plan="auto")
+    nb = ops().gla_saved_states_bytes(prob)
+    assert nb > 0
+    saved = torch.full((nb // 4,), float("nan"), dtype=torch.float32, device="cuda")
+    ops().gla_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["igate"], xd["h0"], scale=w.scale, chunk=w.chunk,
+                  saved_states=saved)
+    r = ops().gla_bwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["igate"], xd["h0"], xd["dO"], None, scale=w.scale,
+                      chunk=w.chunk, saved_states=saved)
+    r0 = ops().gla_bwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["igate"], xd["h0"], xd["dO"], None, scale=w.scale,
+                       chunk=w.chunk)
+    xs = x if heads is None else {k: flat_heads(v, heads) for k, v in x.items()}
+    ref = oracle.gla_bwd(xs["q"], xs["k"], xs["v"], xs["g"], xs["igate"], xs["h0"], xs["dO"], None, w.scale)
+    for n in ("dq", "dk", "dv", "dg"):
+        got = f64(r[n]) if heads is None else flat_heads(f64(r[n]), heads)
+        assert err(got, ref[n]) <= TOL[w.dtype], (n, err(got, ref[n]))
+        assert err(f64(r[n]), f64(r0[n])) <= TOL[w.dtype], n
+
+
 def test_host_tensors_round_trip():
     """The end-to-end call with host tensors (copies in, compute, copies out)."""
     w = I.small(I.WORKLOADS["c2"])
