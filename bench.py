@@ -349,27 +349,35 @@ def main():
         flush.fill_(i & 0xFF)
         step()
     torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    n0 = _lib.launch_count()
-    _lib.profiler_enable(True)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    flush.fill_(0xA5)   # lead-in (outside the events): the host queues step 0 while this runs
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        ev[i][0].record()
-        step()
-        ev[i][1].record()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    _lib.profiler_enable(False)
-    launches = _lib.launch_count() - n0
-    kprof = _lib.profiler_read()
+    def timed_steps(per_kernel):
+        """K steps bracketed by barrier + synchronize; per-step CUDA events on the stream.
+        per_kernel: the library also brackets every launch with CUDA events (for the
+        per-kernel durations); this costs a few microseconds per launch, so `value` comes
+        from the pass without it and the roofline from the pass with it."""
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        n0 = _lib.launch_count()
+        _lib.profiler_enable(per_kernel)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        flush.fill_(0xA5)   # lead-in (outside the events): the host queues step 0 while this runs
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record()
+            step()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        _lib.profiler_enable(False)
+        n = _lib.launch_count() - n0
+        kp = _lib.profiler_read() if per_kernel else {}
+        return sum(a.elapsed_time(b) for a, b in ev), n, kp
+
+    total_ms, launches, _ = timed_steps(False)
+    prof_ms, _, kprof = timed_steps(True)
     clocks = sampler.stop()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = sum(step_ms)
     total_ms = max_over_ranks(total_ms, dev)
     tokens = w.B * w.L * args.steps * world
     value = tokens / (total_ms / 1e3)
@@ -440,6 +448,10 @@ def main():
                  "step_roofline": {"tflops": fl / t_step / 1e12, "gbs_compulsory": by / t_step / 1e9,
                                    "roofline_us": roof_t * 1e6, "frac": roof_t / t_step, "peak_source": peak_src},
                  "kernels": {n: {"launches": c, "avg_us": 1e3 * m / c} for n, (c, m) in sorted(kprof.items())},
+                 "kernel_timing": {"source": "a second pass of the same K steps with CUDA events around "
+                                             "every library launch (kernels, roofline); value and "
+                                             "ms_per_step come from the pass without them",
+                                   "ms_per_step_instrumented": prof_ms / args.steps},
                  "plan": args.plan})
     if world == 1 and not args.no_cpu_baseline:
         heads = oracle_heads(w)
