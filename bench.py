@@ -125,9 +125,9 @@ def kernel_bytes(name, w, fseg=1, bseg=1):
 # ran a smaller case of the same workload; traffic grows with the heads processed.
 MEASURED_TRAFFIC = {
     ("tc_bwd_dkdv", "c3"): {"bytes": 247e6, "scale": 4, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
-                            "sha": "884daa7fc0af09b6", "profile": "profiles/tc_bwd_dkdv_c3_b1.md"},
-    ("tc_fwd", "c2"): {"bytes": 188.7e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_fwd.cu",
-                       "sha": "4a086ac9bf5840d7", "profile": "profiles/tc_fwd_c2.md"},
+                            "sha": "fd3bdfbb36602fe1", "profile": "profiles/tc_bwd_dkdv_c3_b1.md"},
+    ("tc_fwd", "c2"): {"bytes": 187.2e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_fwd.cu",
+                       "sha": "7dc7063744a81ded", "profile": "profiles/tc_fwd_c2.md"},
 }
 
 
