@@ -56,6 +56,76 @@ __device__ __forceinline__ uint32_t f2_to_bf2(uint64_t x) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Coalesced staging of a row-major fp32 block (NR rows x CW columns, row stride ld floats) in
+// shared memory, for consumers that each want one whole row (a state row goes to one TMEM lane).
+// Loading rows thread by thread straight from global memory touches 32 rows per warp access and
+// thrashes L1; here a warp reads whole rows with 16-byte loads, several rows in flight, and
+// 16-byte chunk j of row r lands at chunk j ^ (r & 7) of that row, so that eight consecutive rows
+// read at one column hit eight different bank groups (staged_row16).  With b given (same shape
+// and stride as a), dot[r] = sum_c a[r][c] b[r][c] for every row.  All NT threads take part.
+template <int NR, int CW, int NT>
+__device__ __forceinline__ void stage_rows(float* stg, const float* __restrict__ a, const float* __restrict__ b,
+                                           long ld, float* dot, int tid) {
+    constexpr int CPR = CW / 4;                // 16-byte chunks per row
+    constexpr int LPR = CPR < 32 ? CPR : 32;   // lanes sharing a row
+    constexpr int RPI = 32 / LPR;              // rows per warp access
+    constexpr int CPL = CPR / LPR;             // chunks per lane and row
+    constexpr int W = NT / 32;
+    constexpr int U = 4;                       // row groups in flight per warp
+    static_assert(CPR >= 8 && CPR % LPR == 0 && NR % RPI == 0 && NT % 32 == 0, "staged block shape");
+    const int warp = tid >> 5, lane = tid & 31;
+    const int rsub = lane / LPR, csub = lane % LPR;
+    for (int r0 = warp * RPI; r0 < NR; r0 += U * W * RPI) {
+        float4 xa[U][CPL], xb[U][CPL];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int r = r0 + u * W * RPI + rsub;
+            if (r < NR) {
+                const float4* pa = reinterpret_cast<const float4*>(a + r * ld) + csub;
+                const float4* pb = b ? reinterpret_cast<const float4*>(b + r * ld) + csub : nullptr;
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) {
+                    xa[u][j] = __ldg(pa + j * LPR);
+                    if (b) xb[u][j] = __ldg(pb + j * LPR);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int r = r0 + u * W * RPI + rsub;  // r < NR is uniform over the lanes of a row
+            if (r < NR) {
+                float part = 0.f;
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) {
+                    const int ch = (csub + j * LPR) ^ (r & 7);
+                    *reinterpret_cast<float4*>(stg + r * CW + 4 * ch) = xa[u][j];
+                    if (b)
+                        part += xa[u][j].x * xb[u][j].x + xa[u][j].y * xb[u][j].y + xa[u][j].z * xb[u][j].z +
+                                xa[u][j].w * xb[u][j].w;
+                }
+                if (b) {
+#pragma unroll
+                    for (int off = LPR / 2; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+                    if (csub == 0) dot[r] = part;
+                }
+            }
+        }
+    }
+}
+
+// Columns [c, c + 16) of row r of a block staged by stage_rows (c a multiple of 16).
+template <int CW>
+__device__ __forceinline__ void staged_row16(const float* stg, int r, int c, float* f) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const float4 x = *reinterpret_cast<const float4*>(stg + r * CW + 4 * (((c >> 2) + u) ^ (r & 7)));
+        f[4 * u] = x.x;
+        f[4 * u + 1] = x.y;
+        f[4 * u + 2] = x.z;
+        f[4 * u + 3] = x.w;
+    }
+}
+
 __device__ __forceinline__ void store8_bf16(uint8_t* base, uint32_t off, const float* v) {
     uint32_t w[4];
 #pragma unroll

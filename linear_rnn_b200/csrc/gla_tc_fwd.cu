@@ -195,25 +195,34 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     const bool s_worker = is_ep && (MODE != 0 || wg == 0);
     const int scol0 = MODE == 0 ? 0 : wg * C::SCOLS;   // first state column of this state-pass thread
     float glog[C::NH];
+    // the output pass starts from h0 or the segment's initial state: all threads stage this
+    // CTA's [DK, DVT] block through the ring stages (free until the first loads), coalesced
+    static_assert(MODE != 0 || DK * DVT * 4 <= C::NS * C::STAGE, "state staging");
+    const float* src = nullptr;
+    if (MODE == 0) {
+        if (z == 0) src = A.h0 ? A.h0 + (long)bh * DK * P.Dv + e0 : nullptr;
+        else src = A.sinit + ((long)bh * A.nseg + z) * DK * P.Dv + e0;
+    }
+    const float* stg = reinterpret_cast<const float*>(sm);
+    if (src) {
+        stage_rows<DK, DVT, NTHR_WS>(reinterpret_cast<float*>(sm), src, nullptr, P.Dv, nullptr, tid);
+        __syncthreads();
+    }
     if (s_worker) {
 #pragma unroll
         for (int h = 0; h < C::NH; ++h) {
             const int d = srow(h);
             glog[h] = 0.f;
-            const float* src = nullptr;
-            if (MODE == 0) {
-                if (z == 0) src = A.h0 ? A.h0 + ((long)bh * DK + d) * P.Dv : nullptr;
-                else src = A.sinit + (((long)bh * A.nseg + z) * DK + d) * P.Dv;
-            }
 #pragma unroll
             for (int c = 0; c < C::SCOLS; c += C::CH) {
                 const int col = scol0 + c;
                 float f[C::CH];
 #pragma unroll
-                for (int j = 0; j < C::CH; j += 4) {
-                    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (src && srow_ok) x = *reinterpret_cast<const float4*>(src + e0 + col + j);
-                    f[j] = x.x; f[j + 1] = x.y; f[j + 2] = x.z; f[j + 3] = x.w;
+                for (int j = 0; j < C::CH; j += 16) {
+                    if (src && srow_ok) staged_row16<DVT>(stg, d, col + j, f + j);
+                    else
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) f[j + u] = 0.f;
                 }
                 tmem_stn<C::CH>(tbase + ((uint32_t)(32 * qd) << 16) + h * DVT + col, reinterpret_cast<uint32_t*>(f));
                 if (MODE == 0 && srow_ok)
