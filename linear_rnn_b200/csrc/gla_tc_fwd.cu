@@ -76,7 +76,7 @@ struct Cfg {
     static constexpr uint32_t PB = MODE == 0 ? TR * TR * 2 : 0;       // P
     static constexpr uint32_t SB = MODE == 0 ? DK * DVT * 2 : 0;      // bf16 state
     static constexpr uint32_t OB = MODE == 0 ? TR * DVT * 2 : 0;      // output tile staged for the TMA store
-    static constexpr uint32_t SMALL = 256 + 4 * NTRF + 16 * DK + 1024;
+    static constexpr uint32_t SMALL = 256 + 8 * NTRF + 16 * DK + 1024;
     static constexpr uint32_t FIXED = PB + SB + OB + SMALL + 1024;
     // as many ring stages (up to 4) as shared memory holds: the loads of a tile are in
     // flight while the tiles before it are transformed and multiplied
@@ -153,8 +153,8 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     int* n_consumed = reinterpret_cast<int*>(small + 236);
     int* n_mma1 = reinterpret_cast<int*>(small + 240);
     int* n_mma2 = reinterpret_cast<int*>(small + 244);
-    float* tot = reinterpret_cast<float*>(small + 256);      // [NTRF] cumsum segment totals
-    float* gamb = tot + NTRF;                                // [2][DK] e^Gamma per buffer
+    float* tot = reinterpret_cast<float*>(small + 256);      // [2 NTRF] cumsum segment totals
+    float* gamb = tot + 2 * NTRF;                            // [2][DK] e^Gamma per buffer
     float* gamlb = gamb + 2 * DK;                            // [2][DK] Gamma per buffer
     float* rowE = gamlb + 2 * DK;                            // [64] e^b   (per-head gate)
     float* rowEi = rowE + TR;                                // [64] e^-b
@@ -363,6 +363,99 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
         constexpr int NB = 2;                                // positions per batch of loads
         static_assert(NPOS % (NB * NTRF) == 0 && TR % SEG == 0, "transform mapping");
         const int dA = ttid % DK, sA = ttid / DK;
+        constexpr bool kFused = GATE == 1 && DK <= 128;
+        if constexpr (kFused) {
+            // Per-key gates, one pass per tile: thread = key-dim pair x run of RSF rows. The
+            // column cumsum of its rows stays in registers (b never goes through shared
+            // memory), the run totals are exchanged once, and each row's q, k pairs are scaled
+            // right away (MODE 1: k only; MODE 2, q in the k slot: scale q e^(b - Gamma)).
+            constexpr int NP = DK / 2, SEGF = NTRF / NP, RSF = TR / SEGF;
+            static_assert(NTRF % NP == 0 && TR % SEGF == 0 && 2 * NTRF >= SEGF * DK, "fused transform mapping");
+            const int p = ttid % NP, sgi = ttid / NP, d0 = 2 * p;
+            float2* tot2 = reinterpret_cast<float2*>(tot);   // [SEGF][NP] run totals
+            const uint64_t sc2 = f2(P.scale, P.scale);
+            for (int j = 0; j < ntiles; ++j) {
+                const int s = j % C::NS, b = j & 1;
+                uint8_t* st = sm + s * C::STAGE;
+                uint8_t* sq = st;
+                uint8_t* sk = st + C::QB;
+                const float* sgt = reinterpret_cast<const float*>(st + C::QB + C::KB);
+                const int t0 = tile_at(j) * TR;
+                if (ttid < TR) {
+                    const int t = t0 + ttid;
+                    igs[ttid] = (A.ig && t < P.L) ? A.ig[rowbase + t] : 1.f;
+                }
+                bool ok = mbar_wait_abort(&bar_full[s], (j / C::NS) & 1, abortp);
+                if (ok && j >= 2) ok = mbar_wait_abort(&bar_gfree[b], ((j >> 1) - 1) & 1, abortp);
+                float2 cs[RSF];
+                float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int u = 0; u < RSF; ++u) {
+                    const float2 x = *reinterpret_cast<const float2*>(sgt + (sgi * RSF + u) * DK + d0);
+                    acc.x += x.x;
+                    acc.y += x.y;
+                    cs[u] = acc;
+                }
+                tot2[sgi * NP + p] = acc;
+                if (!named_bar_and(BAR_TR, NTRF, ok)) break;
+                if (ttid == 0) *n_consumed = j + 1;
+                float2 off = make_float2(0.f, 0.f), G = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int s2 = 0; s2 < SEGF; ++s2) {
+                    const float2 t = tot2[s2 * NP + p];
+                    if (s2 < sgi) {
+                        off.x += t.x;
+                        off.y += t.y;
+                    }
+                    G.x += t.x;
+                    G.y += t.y;
+                }
+                // b of row u = cs[u] + c (MODE 2: b - Gamma)
+                const float cx = MODE == 2 ? off.x - G.x : off.x, cy = MODE == 2 ? off.y - G.y : off.y;
+                if (sgi == 0) {
+                    float* gam = gamb + b * DK;
+                    float* gaml = gamlb + b * DK;
+                    gam[d0] = __expf(G.x);
+                    gam[d0 + 1] = __expf(G.y);
+                    gaml[d0] = G.x;
+                    gaml[d0 + 1] = G.y;
+                    if (G.x < kMinTileLogDecay || G.y < kMinTileLogDecay) atomicOr(A.status, kDevStatusRange);
+                }
+#pragma unroll
+                for (int u = 0; u < RSF; ++u) {
+                    const int r = sgi * RSF + u;
+                    // byte offset of (r, d0) in a 128-byte-swizzled bf16 tile
+                    const uint32_t ob = (uint32_t)(d0 >> 6) * BLK + (uint32_t)r * 128 +
+                                        ((((uint32_t)((d0 & 63) >> 3)) ^ (uint32_t)(r & 7)) << 4) + (uint32_t)(d0 & 7) * 2;
+                    const float bx = (cs[u].x + cx) * kLog2e, by = (cs[u].y + cy) * kLog2e;
+                    uint32_t* pk = reinterpret_cast<uint32_t*>(sk + ob);
+                    if (MODE == 2) {
+                        *pk = f2_to_bf2(f2_mul(bf2_to_f2(*pk), f2_mul(sc2, f2(ex2_approx(bx), ex2_approx(by)))));
+                    } else {
+                        const float m = igs[r];
+                        float ex = 1.f, ey = 1.f, dx, dy;
+                        if (MODE == 0) {
+                            // e^-b = 1 / e^b on the FMA pipe (one exponential per element)
+                            ex = ex2_approx(bx);
+                            ey = ex2_approx(by);
+                            dx = rcp_newton(ex);
+                            dy = rcp_newton(ey);
+                        } else {
+                            dx = ex2_approx(-bx);
+                            dy = ex2_approx(-by);
+                        }
+                        *pk = f2_to_bf2(f2_mul(bf2_to_f2(*pk), f2_mul(f2(m, m), f2(dx, dy))));
+                        if (MODE == 0) {
+                            uint32_t* pq = reinterpret_cast<uint32_t*>(sq + ob);
+                            *pq = f2_to_bf2(f2_mul(bf2_to_f2(*pq), f2_mul(sc2, f2(ex, ey))));
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(BAR_TR, NTRF);
+                if (ttid == 0) mbar_arrive(&bar_trans[s]);
+            }
+        } else
         for (int j = 0; j < ntiles; ++j) {
             const int s = j % C::NS, b = j & 1;
             uint8_t* st = sm + s * C::STAGE;
@@ -647,8 +740,8 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
         }
     } else if (s_worker) {
         // final state of the segment, read back from TMEM
-#pragma unroll
         const uint32_t lq = (uint32_t)(32 * qd) << 16;
+#pragma unroll
         for (int h = 0; h < C::NH; ++h) {
             const int d = srow(h);
             float* dst = nullptr;
