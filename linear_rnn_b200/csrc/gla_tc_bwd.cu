@@ -336,6 +336,21 @@ __global__ void __launch_bounds__(NT_B, 1)
         if (GATE == 1)
             for (int gb = 0; gb < DKB / 32; ++gb)
                 tma_load_3d(st + C::QB + C::KB + gb * BLK, &tg, d0 + 32 * gb, t0, bh, &bar_full[s]);
+        // the tile that takes this stage next is brought into L2 now, so that its loads do
+        // not wait on DRAM
+        if (i + C::NS < ntiles) {
+            const int tp = (tile0 + i + C::NS) * TR;
+            for (int cb = 0; cb < DKB / 64; ++cb) {
+                if (GATE != 0) tma_prefetch_l2_3d(&tq, d0 + cb * 64, tp, bh);
+                tma_prefetch_l2_3d(&tk, d0 + cb * 64, tp, bh);
+            }
+            if (GATE == 1)
+                for (int gb = 0; gb < DKB / 32; ++gb) tma_prefetch_l2_3d(&tg, d0 + 32 * gb, tp, bh);
+            for (int vb = 0; vb < DV / 64; ++vb) {
+                tma_prefetch_l2_3d(&tv, vb * 64, tp, bh);
+                tma_prefetch_l2_3d(&tdo, vb * 64, tp, bh);
+            }
+        }
     };
     auto issue_vo = [&](int i, int s) {
         uint8_t* st = sm + s * C::STAGE;
@@ -762,6 +777,20 @@ __global__ void __launch_bounds__(NT_B, 1)
         for (int vb = 0; vb < DV / 64; ++vb) {
             tma_load_3d(st + C::QB + C::KB + C::GB + vb * BLK, &tv, vb * 64, t0, bh, &bar_full[s]);
             tma_load_3d(st + C::QB + C::KB + C::GB + C::VB + vb * BLK, &tdo, vb * 64, t0, bh, &bar_full[s]);
+        }
+        // the tile that takes this stage next is brought into L2 now
+        if (i + C::NS < ntiles) {
+            const int tp = tile_at(i + C::NS) * TR;
+            for (int cb = 0; cb < DK / 64; ++cb) {
+                tma_prefetch_l2_3d(&tq, cb * 64, tp, bh);
+                tma_prefetch_l2_3d(&tk, cb * 64, tp, bh);
+            }
+            if (GATE == 1)
+                for (int gb = 0; gb < DK / 32; ++gb) tma_prefetch_l2_3d(&tg, 32 * gb, tp, bh);
+            for (int vb = 0; vb < DV / 64; ++vb) {
+                tma_prefetch_l2_3d(&tv, vb * 64, tp, bh);
+                tma_prefetch_l2_3d(&tdo, vb * 64, tp, bh);
+            }
         }
     };
     if (tid == 0)

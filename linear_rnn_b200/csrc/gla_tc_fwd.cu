@@ -259,6 +259,18 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 for (int vb = 0; vb < DVT / 64; ++vb)
                     tma_load_3d(st + C::QB + C::KB + C::GB + vb * BLK, &tv, e0 + vb * 64, t0, bh, &bar_full[s]);
                 *n_issued = j + 1;
+                // with a shallow ring (output pass, two stages) the tile that takes this stage
+                // next is brought into L2 now, so that its load (issued once the stage is
+                // released) does not wait on DRAM; deeper rings and the streaming state-only
+                // passes keep enough loads in flight without it
+                if (MODE == 0 && C::NS <= 2 && j + C::NS < ntiles) {
+                    const int tp = tile_at(j + C::NS) * TR;
+                    if (MODE == 0)
+                        for (int cb = 0; cb < DK / 64; ++cb) tma_prefetch_l2_3d(&tq, cb * 64, tp, bh);
+                    for (int cb = 0; cb < DK / 64; ++cb) tma_prefetch_l2_3d(&tk, cb * 64, tp, bh);
+                    if (GATE == 1) tma_prefetch_l2_3d(&tg, 0, tp, bh);
+                    for (int vb = 0; vb < DVT / 64; ++vb) tma_prefetch_l2_3d(&tv, e0 + vb * 64, tp, bh);
+                }
             }
         }
     } else if (warp == W_MMA) {

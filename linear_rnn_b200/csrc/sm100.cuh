@@ -132,6 +132,14 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
+// Prefetch of one tensor-map tile into L2 (no shared memory, no completion to wait for): the
+// TMA load of the same tile issued later then reads it from L2 instead of DRAM.
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
 
 // Tiled TMA store of a shared-memory tile (same box and swizzle as the tensor map) to
 // global memory, tracked as a bulk group of the issuing thread. Rows outside the tensor
