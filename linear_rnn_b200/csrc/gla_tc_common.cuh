@@ -32,12 +32,25 @@ __device__ __forceinline__ float rcp_newton(float x) {
     return fmaf(y, e, y);
 }
 
+// 1/x on the special-function unit (PTX rcp.approx, about 1 ulp, subnormals flushed): where the
+// FMA pipe is the busier unit, this is cheaper than rcp_newton.
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Packed pairs of fp32 in one 64-bit register, multiplied lane-wise by the sm_100 packed
 // fp32 instruction (IEEE round-to-nearest per lane, like two separate multiplies).
 __device__ __forceinline__ uint64_t f2(float lo, float hi) {
     uint64_t r;
     asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
     return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
 }
 __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     uint64_t d;

@@ -447,11 +447,11 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                         const float m = igs[r];
                         float ex = 1.f, ey = 1.f, dx, dy;
                         if (MODE == 0) {
-                            // e^-b = 1 / e^b on the FMA pipe (one exponential per element)
+                            // e^-b = 1 / e^b (one exponential and one reciprocal per element)
                             ex = ex2_approx(bx);
                             ey = ex2_approx(by);
-                            dx = rcp_newton(ex);
-                            dy = rcp_newton(ey);
+                            dx = rcp_approx(ex);
+                            dy = rcp_approx(ey);
                         } else {
                             dx = ex2_approx(-bx);
                             dy = ex2_approx(-by);
@@ -574,9 +574,9 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     if (GATE == 1) {
 #pragma unroll
                         for (int u = 0; u < 8; ++u) {
-                            // output pass: e^-b = 1 / e^b on the FMA pipe (one exponential per element)
+                            // output pass: e^-b = 1 / e^b (one exponential per element)
                             eu[u] = MODE != 1 ? ex2_approx(bv[k][u]) : 1.f;
-                            ed[u] = MODE == 0 ? rcp_newton(eu[u]) : MODE == 1 ? ex2_approx(-bv[k][u]) : 1.f;
+                            ed[u] = MODE == 0 ? rcp_approx(eu[u]) : MODE == 1 ? ex2_approx(-bv[k][u]) : 1.f;
                         }
                     } else {
                         const float fu = GATE == 2 ? rowE[r] : 1.f, fd = GATE == 2 ? rowEi[r] : 1.f;
