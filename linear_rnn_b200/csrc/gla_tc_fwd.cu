@@ -66,7 +66,9 @@ constexpr uint32_t pow2_cols(uint32_t n) { return n <= 32 ? 32 : n <= 64 ? 64 : 
 
 template <int DK, int DVT, int GATE, int MODE>
 struct Cfg {
-    // MODE 0: output pass (q, k, g, v). MODE 1: state-only pass (k, g, v).
+    // MODE 0: output pass (q, k, g, v). MODE 1: state-only pass (k, g, v), walked from the
+    // segment's end with every k scaled by its whole decay to that end, e^(D + Gamma - b) <= 1
+    // (D: decay of the tiles after this one), so that the state only accumulates.
     // MODE 2: reverse state-gradient pass (q in the k slot, g, dO in the v slot).
     static constexpr uint32_t QB = MODE == 0 ? TR * DK * 2 : 0;
     static constexpr uint32_t KB = TR * DK * 2;
@@ -169,8 +171,8 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     const int tile0 = z * A.tiles_per_seg;
     const int ntiles = min(ntiles_all, tile0 + A.tiles_per_seg) - tile0;
     const long rowbase = (long)bh * P.L;
-    // the j-th tile this CTA processes (MODE 2 walks its segment backwards)
-    auto tile_at = [&](int j) { return MODE == 2 ? tile0 + ntiles - 1 - j : tile0 + j; };
+    // the j-th tile this CTA processes (the state-only passes walk their segment backwards)
+    auto tile_at = [&](int j) { return MODE != 0 ? tile0 + ntiles - 1 - j : tile0 + j; };
     const bool is_ep = tid < NEP;
     // epilogue threads: key-dim row of the state this lane holds (M=64 state: lanes 0-15)
     const bool srow_ok = (DK != 64) || (lane < 16);
@@ -334,7 +336,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 }
                 __syncwarp();
                 // the state of the previous tile must be decayed (and copied) first
-                if (i >= 1) {
+                if (MODE != 1 && i >= 1) {
                     if (!warp_wait(bar_sready, (i - 1) & 1, abortp)) break;
                     tc_fence_after();
                 }
@@ -375,6 +377,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
         constexpr int NB = 2;                                // positions per batch of loads
         static_assert(NPOS % (NB * NTRF) == 0 && TR % SEG == 0, "transform mapping");
         const int dA = ttid % DK, sA = ttid / DK;
+        float dlat1 = 0.f;   // MODE 1: log-decay of the tiles after this one (key dim dA, or per head)
         constexpr bool kFused = GATE == 1 && DK <= 128;
         if constexpr (kFused) {
             // Per-key gates, one pass per tile: thread = key-dim pair x run of RSF rows. The
@@ -386,6 +389,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
             const int p = ttid % NP, sgi = ttid / NP, d0 = 2 * p;
             float2* tot2 = reinterpret_cast<float2*>(tot);   // [SEGF][NP] run totals
             const uint64_t sc2 = f2(P.scale, P.scale);
+            float2 dlat = make_float2(0.f, 0.f);   // MODE 1: log-decay of the tiles after this one
             for (int j = 0; j < ntiles; ++j) {
                 const int s = j % C::NS, b = j & 1;
                 uint8_t* st = sm + s * C::STAGE;
@@ -422,8 +426,14 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     G.x += t.x;
                     G.y += t.y;
                 }
-                // b of row u = cs[u] + c (MODE 2: b - Gamma)
-                const float cx = MODE == 2 ? off.x - G.x : off.x, cy = MODE == 2 ? off.y - G.y : off.y;
+                // exponent of row u = cs[u] + c: b (output pass), b - Gamma (MODE 2), and in
+                // MODE 1 b - Gamma - D, whose negation scales k
+                const float cx = MODE == 0 ? off.x : MODE == 2 ? off.x - G.x : off.x - G.x - dlat.x;
+                const float cy = MODE == 0 ? off.y : MODE == 2 ? off.y - G.y : off.y - G.y - dlat.y;
+                if (MODE == 1) {
+                    dlat.x += G.x;
+                    dlat.y += G.y;
+                }
                 if (sgi == 0) {
                     float* gam = gamb + b * DK;
                     float* gaml = gamlb + b * DK;
@@ -510,7 +520,8 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                         G += t;
                     }
                 }
-                const float sub = MODE == 2 ? G - off : -off;
+                const float sub = MODE == 0 ? -off : MODE == 2 ? G - off : G - off + dlat1;
+                if (MODE == 1) dlat1 += G;
 #pragma unroll
                 for (int u = 0; u < RS; ++u) col[u * DK] = (x[u] - sub) * kLog2e;
                 if (sA == 0) {
@@ -533,8 +544,10 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     const float bq0 = MODE == 2 ? b0 - G : b0, bq1 = MODE == 2 ? b1 - G : b1;
                     rowE[2 * lane] = __expf(bq0);
                     rowE[2 * lane + 1] = __expf(bq1);
-                    rowEi[2 * lane] = __expf(-b0);
-                    rowEi[2 * lane + 1] = __expf(-b1);
+                    // MODE 1: e^(D + Gamma - b), the decay from the token to the segment's end
+                    rowEi[2 * lane] = __expf(MODE == 1 ? dlat1 + G - b0 : -b0);
+                    rowEi[2 * lane + 1] = __expf(MODE == 1 ? dlat1 + G - b1 : -b1);
+                    if (MODE == 1) dlat1 += G;
                     if (lane == 0) {
                         gam[0] = __expf(G);
                         gaml[0] = G;
@@ -635,8 +648,9 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 const int gi = GATE == 1 ? d : 0;
                 const float egv = GATE == 0 ? 1.f : gam[gi];
                 if (GATE != 0) glog[h] += gaml[gi];
+                // MODE 1 scaled its k by the whole decay to the segment's end: nothing to decay
 #pragma unroll
-                for (int c = 0; c < C::SCOLS; c += C::CH) {
+                for (int c = 0; c < (MODE == 1 ? 0 : C::SCOLS); c += C::CH) {
                     const int col = scol0 + c;
                     float f[C::CH];
                     uint32_t* r = reinterpret_cast<uint32_t*>(f);
