@@ -798,45 +798,71 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
 }
 
 // Segment scan: sinit[z] = e^{Gamma_{z-1}} sinit[z-1] + dS_{z-1}, sinit[0] = h0 (or 0).
-// One thread per (bh, d, e) state element, walking the segments in order.
+// One thread per four consecutive state elements of one (bh, d) row; the loads of SEGU
+// segments are issued before their dependent chain, so that the walk is bandwidth-bound.
+constexpr int SEGU = 8;
 __global__ void __launch_bounds__(256) k_seg_scan(const float* __restrict__ seg_state,
                                                   const float* __restrict__ seg_gamma, const float* __restrict__ h0,
                                                   float* __restrict__ sinit, int BH, int Dk, int Dv, int nseg) {
-    const int per = Dk * Dv;
+    const int per4 = Dk * Dv / 4;
     const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= (long)BH * per) return;
-    const int bh = (int)(idx / per), de = (int)(idx - (long)bh * per), d = de / Dv;
-    const float* src = seg_state + (size_t)bh * nseg * per + de;
+    if (idx >= (long)BH * per4) return;
+    const int bh = (int)(idx / per4), de4 = (int)(idx - (long)bh * per4), d = 4 * de4 / Dv;
+    const float4* src = reinterpret_cast<const float4*>(seg_state) + (size_t)bh * nseg * per4 + de4;
     const float* gam = seg_gamma + (size_t)bh * nseg * Dk + d;
-    float* dst = sinit + (size_t)bh * nseg * per + de;
-    float S = h0 ? h0[idx] : 0.f;
-#pragma unroll 4
-    for (int z = 0; z < nseg - 1; ++z) {
-        S = __expf(gam[(size_t)z * Dk]) * S + src[(size_t)z * per];
-        dst[(size_t)(z + 1) * per] = S;
+    float4* dst = reinterpret_cast<float4*>(sinit) + (size_t)bh * nseg * per4 + de4;
+    float4 S = h0 ? __ldg(reinterpret_cast<const float4*>(h0) + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int z0 = 0; z0 < nseg - 1; z0 += SEGU) {
+        float4 x[SEGU];
+        float e[SEGU];
+#pragma unroll
+        for (int u = 0; u < SEGU; ++u)
+            if (z0 + u < nseg - 1) {
+                x[u] = __ldg(src + (size_t)(z0 + u) * per4);
+                e[u] = __expf(__ldg(gam + (size_t)(z0 + u) * Dk));
+            }
+#pragma unroll
+        for (int u = 0; u < SEGU; ++u)
+            if (z0 + u < nseg - 1) {
+                S = make_float4(fmaf(e[u], S.x, x[u].x), fmaf(e[u], S.y, x[u].y), fmaf(e[u], S.z, x[u].z),
+                                fmaf(e[u], S.w, x[u].w));
+                dst[(size_t)(z0 + u + 1) * per4] = S;
+            }
     }
 }
 
 // Reverse segment scan for the backward: gend[z] = gradient w.r.t. the state at the end of
 // segment z; gend[nseg-1] = dhT (or 0), gend[z] = e^{Gamma_{z+1}} gend[z+1] + dG_{z+1},
 // where dG_z (seg_state[z]) is segment z's own state-gradient accumulated from zero at
-// its end and Gamma_z (seg_gamma[z]) its total log-decay.
+// its end and Gamma_z (seg_gamma[z]) its total log-decay. Same layout as k_seg_scan.
 __global__ void __launch_bounds__(256) k_seg_rscan(const float* __restrict__ seg_state,
                                                    const float* __restrict__ seg_gamma, const float* __restrict__ dhT,
                                                    float* __restrict__ gend, int BH, int Dk, int Dv, int nseg) {
-    const int per = Dk * Dv;
+    const int per4 = Dk * Dv / 4;
     const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= (long)BH * per) return;
-    const int bh = (int)(idx / per), de = (int)(idx - (long)bh * per), d = de / Dv;
-    const float* src = seg_state + (size_t)bh * nseg * per + de;
+    if (idx >= (long)BH * per4) return;
+    const int bh = (int)(idx / per4), de4 = (int)(idx - (long)bh * per4), d = 4 * de4 / Dv;
+    const float4* src = reinterpret_cast<const float4*>(seg_state) + (size_t)bh * nseg * per4 + de4;
     const float* gam = seg_gamma + (size_t)bh * nseg * Dk + d;
-    float* dst = gend + (size_t)bh * nseg * per + de;
-    float G = dhT ? dhT[idx] : 0.f;
-    dst[(size_t)(nseg - 1) * per] = G;
-#pragma unroll 4
-    for (int z = nseg - 1; z >= 1; --z) {
-        G = __expf(gam[(size_t)z * Dk]) * G + src[(size_t)z * per];
-        dst[(size_t)(z - 1) * per] = G;
+    float4* dst = reinterpret_cast<float4*>(gend) + (size_t)bh * nseg * per4 + de4;
+    float4 G = dhT ? __ldg(reinterpret_cast<const float4*>(dhT) + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+    dst[(size_t)(nseg - 1) * per4] = G;
+    for (int z0 = nseg - 1; z0 >= 1; z0 -= SEGU) {
+        float4 x[SEGU];
+        float e[SEGU];
+#pragma unroll
+        for (int u = 0; u < SEGU; ++u)
+            if (z0 - u >= 1) {
+                x[u] = __ldg(src + (size_t)(z0 - u) * per4);
+                e[u] = __expf(__ldg(gam + (size_t)(z0 - u) * Dk));
+            }
+#pragma unroll
+        for (int u = 0; u < SEGU; ++u)
+            if (z0 - u >= 1) {
+                G = make_float4(fmaf(e[u], G.x, x[u].x), fmaf(e[u], G.y, x[u].y), fmaf(e[u], G.z, x[u].z),
+                                fmaf(e[u], G.w, x[u].w));
+                dst[(size_t)(z0 - u - 1) * per4] = G;
+            }
     }
 }
 
@@ -992,7 +1018,7 @@ static cudaError_t run(const Dims& P, const void* q, const void* k, const void* 
 
 cudaError_t seg_scan(const Dims& P, int nseg, const float* seg_state, const float* seg_gamma, const float* h0,
                      float* sinit, cudaStream_t st) {
-    const long n = (long)P.B * P.H * P.Dk * P.Dv;
+    const long n = (long)P.B * P.H * P.Dk * P.Dv / 4;
     GLA_LAUNCH("tc_seg_scan", st,
                k_seg_scan<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(seg_state, seg_gamma, h0, sinit, P.B * P.H,
                                                                        P.Dk, P.Dv, nseg));
@@ -1001,7 +1027,7 @@ cudaError_t seg_scan(const Dims& P, int nseg, const float* seg_state, const floa
 
 cudaError_t seg_rscan(const Dims& P, int nseg, const float* seg_state, const float* seg_gamma, const float* dhT,
                       float* gend, cudaStream_t st) {
-    const long n = (long)P.B * P.H * P.Dk * P.Dv;
+    const long n = (long)P.B * P.H * P.Dk * P.Dv / 4;
     GLA_LAUNCH("tc_seg_rscan", st,
                k_seg_rscan<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(seg_state, seg_gamma, dhT, gend, P.B * P.H,
                                                                         P.Dk, P.Dv, nseg));
