@@ -69,7 +69,8 @@ struct Cfg {
     // MODE 0: output pass (q, k, g, v). MODE 1: state-only pass (k, g, v), walked from the
     // segment's end with every k scaled by its whole decay to that end, e^(D + Gamma - b) <= 1
     // (D: decay of the tiles after this one), so that the state only accumulates.
-    // MODE 2: reverse state-gradient pass (q in the k slot, g, dO in the v slot).
+    // MODE 2: state-gradient pass (q in the k slot, g, dO in the v slot), walked from the
+    // segment's start with every q scaled by its whole decay from that start, e^(D + b) <= 1.
     static constexpr uint32_t QB = MODE == 0 ? TR * DK * 2 : 0;
     static constexpr uint32_t KB = TR * DK * 2;
     static constexpr uint32_t GB = GATE == 1 ? TR * DK * 4 : 0;
@@ -171,8 +172,8 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     const int tile0 = z * A.tiles_per_seg;
     const int ntiles = min(ntiles_all, tile0 + A.tiles_per_seg) - tile0;
     const long rowbase = (long)bh * P.L;
-    // the j-th tile this CTA processes (the state-only passes walk their segment backwards)
-    auto tile_at = [&](int j) { return MODE != 0 ? tile0 + ntiles - 1 - j : tile0 + j; };
+    // the j-th tile this CTA processes (the forward state-only pass walks its segment backwards)
+    auto tile_at = [&](int j) { return MODE == 1 ? tile0 + ntiles - 1 - j : tile0 + j; };
     const bool is_ep = tid < NEP;
     // epilogue threads: key-dim row of the state this lane holds (M=64 state: lanes 0-15)
     const bool srow_ok = (DK != 64) || (lane < 16);
@@ -336,7 +337,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 }
                 __syncwarp();
                 // the state of the previous tile must be decayed (and copied) first
-                if (MODE != 1 && i >= 1) {
+                if (MODE == 0 && i >= 1) {
                     if (!warp_wait(bar_sready, (i - 1) & 1, abortp)) break;
                     tc_fence_after();
                 }
@@ -366,7 +367,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
         // ================================================================ transform warpgroups
         // Step A: b = inclusive column cumsum of the log-gate, in row segments (thread = key
         // dim x segment) joined through the segment totals, written over g in place in
-        // base-2 units (b * log2 e; MODE 2 writes (b - Gamma) * log2 e). Step B: every 16-byte
+        // base-2 units (b * log2 e; MODE 1 writes (b - Gamma - D), MODE 2 (b + D) * log2 e). Step B: every 16-byte
         // chunk (8 key dims of one row) of the k tile, and of the q tile in the output pass,
         // is scaled in place by its exponentials and rounded to bf16 (q also by the output
         // scale, so that A, P and O carry it).
@@ -377,19 +378,19 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
         constexpr int NB = 2;                                // positions per batch of loads
         static_assert(NPOS % (NB * NTRF) == 0 && TR % SEG == 0, "transform mapping");
         const int dA = ttid % DK, sA = ttid / DK;
-        float dlat1 = 0.f;   // MODE 1: log-decay of the tiles after this one (key dim dA, or per head)
+        float dlat1 = 0.f;   // MODE 1/2: log-decay of the tiles walked so far (key dim dA, or per head)
         constexpr bool kFused = GATE == 1 && DK <= 128;
         if constexpr (kFused) {
             // Per-key gates, one pass per tile: thread = key-dim pair x run of RSF rows. The
             // column cumsum of its rows stays in registers (b never goes through shared
             // memory), the run totals are exchanged once, and each row's q, k pairs are scaled
-            // right away (MODE 1: k only; MODE 2, q in the k slot: scale q e^(b - Gamma)).
+            // right away (MODE 1: k only; MODE 2, q in the k slot: scale q e^(D + b)).
             constexpr int NP = DK / 2, SEGF = NTRF / NP, RSF = TR / SEGF;
             static_assert(NTRF % NP == 0 && TR % SEGF == 0 && 2 * NTRF >= SEGF * DK, "fused transform mapping");
             const int p = ttid % NP, sgi = ttid / NP, d0 = 2 * p;
             float2* tot2 = reinterpret_cast<float2*>(tot);   // [SEGF][NP] run totals
             const uint64_t sc2 = f2(P.scale, P.scale);
-            float2 dlat = make_float2(0.f, 0.f);   // MODE 1: log-decay of the tiles after this one
+            float2 dlat = make_float2(0.f, 0.f);   // MODE 1/2: log-decay of the tiles walked so far
             for (int j = 0; j < ntiles; ++j) {
                 const int s = j % C::NS, b = j & 1;
                 uint8_t* st = sm + s * C::STAGE;
@@ -426,11 +427,12 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     G.x += t.x;
                     G.y += t.y;
                 }
-                // exponent of row u = cs[u] + c: b (output pass), b - Gamma (MODE 2), and in
-                // MODE 1 b - Gamma - D, whose negation scales k
-                const float cx = MODE == 0 ? off.x : MODE == 2 ? off.x - G.x : off.x - G.x - dlat.x;
-                const float cy = MODE == 0 ? off.y : MODE == 2 ? off.y - G.y : off.y - G.y - dlat.y;
-                if (MODE == 1) {
+                // exponent of row u = cs[u] + c: b (output pass), D + b (MODE 2, D the decay of
+                // the tiles before this one), and in MODE 1 b - Gamma - D (D the decay of the tiles
+                // after it), whose negation scales k
+                const float cx = MODE == 0 ? off.x : MODE == 2 ? off.x + dlat.x : off.x - G.x - dlat.x;
+                const float cy = MODE == 0 ? off.y : MODE == 2 ? off.y + dlat.y : off.y - G.y - dlat.y;
+                if (MODE != 0) {
                     dlat.x += G.x;
                     dlat.y += G.y;
                 }
@@ -520,8 +522,8 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                         G += t;
                     }
                 }
-                const float sub = MODE == 0 ? -off : MODE == 2 ? G - off : G - off + dlat1;
-                if (MODE == 1) dlat1 += G;
+                const float sub = MODE == 0 ? -off : MODE == 2 ? -off - dlat1 : G - off + dlat1;
+                if (MODE != 0) dlat1 += G;
 #pragma unroll
                 for (int u = 0; u < RS; ++u) col[u * DK] = (x[u] - sub) * kLog2e;
                 if (sA == 0) {
@@ -540,14 +542,14 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     }
                     const float b1 = v, b0 = v - g1;
                     const float G = __shfl_sync(0xffffffffu, b1, 31);
-                    // MODE 2 scales q by e^(b - Gamma): the state epilogue applies e^Gamma after the add
-                    const float bq0 = MODE == 2 ? b0 - G : b0, bq1 = MODE == 2 ? b1 - G : b1;
+                    // MODE 2 scales q by its decay from the segment's start, e^(D + b)
+                    const float bq0 = MODE == 2 ? b0 + dlat1 : b0, bq1 = MODE == 2 ? b1 + dlat1 : b1;
                     rowE[2 * lane] = __expf(bq0);
                     rowE[2 * lane + 1] = __expf(bq1);
                     // MODE 1: e^(D + Gamma - b), the decay from the token to the segment's end
                     rowEi[2 * lane] = __expf(MODE == 1 ? dlat1 + G - b0 : -b0);
                     rowEi[2 * lane + 1] = __expf(MODE == 1 ? dlat1 + G - b1 : -b1);
-                    if (MODE == 1) dlat1 += G;
+                    if (MODE != 0) dlat1 += G;
                     if (lane == 0) {
                         gam[0] = __expf(G);
                         gaml[0] = G;
@@ -556,7 +558,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 }
             }
             named_bar_sync(BAR_TR, NTRF);
-            // ---- step B: MODE 0/1 k -> i k e^-b, MODE 0 q -> q e^b, MODE 2 (q in the k slot) -> scale q e^(b-Gamma)
+            // ---- step B: MODE 0/1 k -> i k e^-b, MODE 0 q -> q e^b, MODE 2 (q in the k slot) -> scale q e^(D+b)
 #pragma unroll
             for (int it0 = 0; it0 < NPOS / NTRF; it0 += NB) {
                 float bv[NB][8];
@@ -648,9 +650,10 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 const int gi = GATE == 1 ? d : 0;
                 const float egv = GATE == 0 ? 1.f : gam[gi];
                 if (GATE != 0) glog[h] += gaml[gi];
-                // MODE 1 scaled its k by the whole decay to the segment's end: nothing to decay
+                // the state-only passes scaled k (q) by whole decays to the segment's end (from its
+                // start): nothing to decay
 #pragma unroll
-                for (int c = 0; c < (MODE == 1 ? 0 : C::SCOLS); c += C::CH) {
+                for (int c = 0; c < (MODE != 0 ? 0 : C::SCOLS); c += C::CH) {
                     const int col = scol0 + c;
                     float f[C::CH];
                     uint32_t* r = reinterpret_cast<uint32_t*>(f);
@@ -937,7 +940,7 @@ cudaError_t seg_scan(const Dims& P, int nseg, const float* seg_state, const floa
                      float* sinit, cudaStream_t st);
 
 // State-only pass over every segment but one: MODE 1 (forward states: a = k, b = v) runs
-// segments 0..nseg-2, MODE 2 (reverse state gradients: a = q, b = dO) segments 1..nseg-1.
+// segments 0..nseg-2, MODE 2 (state gradients: a = q, b = dO) segments 1..nseg-1.
 template <int DK, int DVT, int GATE>
 static cudaError_t state_run(const Dims& P, int mode, const void* a_src, const void* b_src, const float* g,
                              const float* ig, int nseg, int tps, float* seg_state, float* seg_gamma, int* status,
