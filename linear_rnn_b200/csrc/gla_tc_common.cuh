@@ -126,6 +126,35 @@ __device__ __forceinline__ void stage_rows(float* stg, const float* __restrict__
     }
 }
 
+// The reverse of stage_rows: rows written into shared memory one per thread (staged_put16)
+// go out to global memory with coalesced 16-byte stores, whole rows per warp.
+template <int NR, int CW, int NT>
+__device__ __forceinline__ void unstage_rows(const float* stg, float* __restrict__ dst, long ld, int tid) {
+    constexpr int CPR = CW / 4;
+    constexpr int LPR = CPR < 32 ? CPR : 32;
+    constexpr int RPI = 32 / LPR;
+    constexpr int CPL = CPR / LPR;
+    constexpr int W = NT / 32;
+    static_assert(CPR >= 8 && CPR % LPR == 0 && NR % RPI == 0 && NT % 32 == 0, "staged block shape");
+    const int warp = tid >> 5, lane = tid & 31;
+    const int rsub = lane / LPR, csub = lane % LPR;
+    for (int r = warp * RPI + rsub; r < NR; r += W * RPI) {
+        float4* pd = reinterpret_cast<float4*>(dst + r * ld) + csub;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j)
+            pd[j * LPR] = *reinterpret_cast<const float4*>(stg + r * CW + 4 * ((csub + j * LPR) ^ (r & 7)));
+    }
+}
+
+// Columns [c, c + 16) of row r into a block laid out as stage_rows does (c a multiple of 16).
+template <int CW>
+__device__ __forceinline__ void staged_put16(float* stg, int r, int c, const float* f) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        *reinterpret_cast<float4*>(stg + r * CW + 4 * (((c >> 2) + u) ^ (r & 7))) =
+            make_float4(f[4 * u], f[4 * u + 1], f[4 * u + 2], f[4 * u + 3]);
+}
+
 // Columns [c, c + 16) of row r of a block staged by stage_rows (c a multiple of 16).
 template <int CW>
 __device__ __forceinline__ void staged_row16(const float* stg, int r, int c, float* f) {

@@ -767,31 +767,40 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
             if (*n_mma1) mbar_wait(&bar_mma1[(*n_mma1 - 1) & 1], ((*n_mma1 - 1) >> 1) & 1, 1u << 20);
             if (*n_mma2) mbar_wait(&bar_mma2[(*n_mma2 - 1) % C::NAB], ((*n_mma2 - 1) / C::NAB) & 1, 1u << 20);
         }
-    } else if (s_worker) {
-        // final state of the segment, read back from TMEM
-        const uint32_t lq = (uint32_t)(32 * qd) << 16;
+    } else {
+        // final state of the segment: TMEM -> rows in shared memory (the ring stages are idle
+        // now) -> coalesced rows in global memory
+        float* dst = nullptr;   // row 0, column e0 of this CTA's block
+        if (MODE == 0) {
+            if (z == A.nseg - 1 && A.hT) dst = A.hT + (long)bh * DK * P.Dv + e0;
+        } else {
+            dst = A.seg_state + ((long)bh * A.nseg + z) * DK * P.Dv + e0;
+        }
+        static_assert(DK * DVT * 4 <= C::NS * C::STAGE, "state staging");
+        float* stg = reinterpret_cast<float*>(sm);
+        if (s_worker) {
+            const uint32_t lq = (uint32_t)(32 * qd) << 16;
 #pragma unroll
-        for (int h = 0; h < C::NH; ++h) {
-            const int d = srow(h);
-            float* dst = nullptr;
-            if (MODE == 0) {
-                if (z == A.nseg - 1 && A.hT) dst = A.hT + ((long)bh * DK + d) * P.Dv;
-            } else {
-                dst = A.seg_state + (((long)bh * A.nseg + z) * DK + d) * P.Dv;
-                if (vt == 0 && scol0 == 0 && srow_ok) A.seg_gamma[((long)bh * A.nseg + z) * DK + d] = glog[h];
+            for (int h = 0; h < C::NH; ++h) {
+                const int d = srow(h);
+                if (MODE != 0 && vt == 0 && scol0 == 0 && srow_ok)
+                    A.seg_gamma[((long)bh * A.nseg + z) * DK + d] = glog[h];
+                if (!dst) continue;
+#pragma unroll
+                for (int c = 0; c < C::SCOLS; c += C::CH) {
+                    const int col = scol0 + c;
+                    float f[C::CH];
+                    tmem_ldn<C::CH>(tbase + lq + h * DVT + col, reinterpret_cast<uint32_t*>(f));
+                    tmem_wait_ld();
+                    if (srow_ok)
+#pragma unroll
+                        for (int j = 0; j < C::CH; j += 16) staged_put16<DVT>(stg, d, col + j, f + j);
+                }
             }
-            if (!dst) continue;
-#pragma unroll
-            for (int c = 0; c < C::SCOLS; c += C::CH) {
-                const int col = scol0 + c;
-                float f[C::CH];
-                tmem_ldn<C::CH>(tbase + lq + h * DVT + col, reinterpret_cast<uint32_t*>(f));
-                tmem_wait_ld();
-                if (srow_ok)
-#pragma unroll
-                    for (int j = 0; j < C::CH; j += 4)
-                        *reinterpret_cast<float4*>(dst + e0 + col + j) = make_float4(f[j], f[j + 1], f[j + 2], f[j + 3]);
-            }
+        }
+        if (dst) {   // uniform over the block
+            __syncthreads();
+            unstage_rows<DK, DVT, NTHR_WS>(stg, dst, P.Dv, tid);
         }
     }
     if (MODE == 0 && tid == 128) bulk_wait<0>();   // the last output stores have completed
