@@ -223,10 +223,15 @@ struct QCfg {
     static constexpr uint32_t SMALL = 256 + 8192 + 8 * DKB + 1024 + 512;
     static constexpr int NS = (2 * STAGE + SB + AB + SMALL + 1024 <= 227 * 1024) ? 2 : 1;
     static constexpr uint32_t SMEM = NS * STAGE + SB + AB + SMALL + 1024;
+    // TMEM: S [0, DV). From COL_R the M=64 accumulators of D = dO S^T + mask(dA) k~ (rows in
+    // lanes 16-31) and dA (lanes 0-15); with SPLIT, D's two column halves sit in lanes 0-15 and
+    // 16-31 of the same columns, so that every lane of the epilogue holds a row, and dA follows.
+    static constexpr bool SPLIT = DKB == 128;
     static constexpr uint32_t COL_R = DV;
-    static constexpr uint32_t NCOL = pow2cols(DV + (DKB > 64 ? DKB : 64));
+    static constexpr uint32_t COL_A = SPLIT ? COL_R + DKB / 2 : COL_R;
+    static constexpr uint32_t NCOL = pow2cols(DV + (SPLIT ? DKB / 2 + 64 : (DKB > 64 ? DKB : 64)));
     static constexpr int HC = DV / 2;    // state columns per warpgroup
-    static constexpr int QC = DKB / 2;   // dq columns per warpgroup
+    static constexpr int QC = SPLIT ? DKB / 4 : DKB / 2;   // D columns (TMEM) per warpgroup
     static_assert(SMEM <= 227 * 1024, "shared memory");
     static_assert(STAGE % 1024 == 0, "stage alignment");
 };
@@ -396,20 +401,28 @@ __global__ void __launch_bounds__(NT_B, 1)
         if (warp == 0) {
             const bool leader = elect_one();
             const uint32_t ka = smem_u32(sk), va = smem_u32(sv), oa = smem_u32(so), sa = smem_u32(sS);
-            const uint32_t idA = idesc_bf16(64, 64, 0, 0), idQ = idesc_bf16(64, DKB, 0, 0);
+            const uint32_t idA = idesc_bf16(64, 64, 0, 0), idQ = idesc_bf16(64, C::SPLIT ? DKB / 2 : DKB, 0, 0);
             const uint32_t idS = idesc_bf16(DKB, DV, 1, 1);
 #pragma unroll
             for (int kk = 0; kk < DV / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
-                if (leader) mma_bf16(tbase + C::COL_R, sw128_desc(oa + koff, 16, 1024), sw128_desc(va + koff, 16, 1024), idA,
+                if (leader) mma_bf16(tbase + C::COL_A, sw128_desc(oa + koff, 16, 1024), sw128_desc(va + koff, 16, 1024), idA,
                          kk > 0);
             }
 #pragma unroll
             for (int kk = 0; kk < DV / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
                 const uint32_t soff = (kk >> 2) * (DKB * 128) + (kk & 3) * 32;
-                if (leader) mma_bf16(tbase + (16u << 16) + C::COL_R, sw128_desc(oa + koff, 16, 1024),
-                         sw128_desc(sa + soff, 16, 1024), idQ, kk > 0);
+                if (C::SPLIT) {
+                    // key dims [0, 64) into lanes 0-15, [64, 128) (state rows 64 on) into lanes 16-31
+                    if (leader) mma_bf16(tbase + C::COL_R, sw128_desc(oa + koff, 16, 1024), sw128_desc(sa + soff, 16, 1024),
+                             idQ, kk > 0);
+                    if (leader) mma_bf16(tbase + (16u << 16) + C::COL_R, sw128_desc(oa + koff, 16, 1024),
+                             sw128_desc(sa + soff + (DKB / 2) * 128, 16, 1024), idQ, kk > 0);
+                } else {
+                    if (leader) mma_bf16(tbase + (16u << 16) + C::COL_R, sw128_desc(oa + koff, 16, 1024),
+                             sw128_desc(sa + soff, 16, 1024), idQ, kk > 0);
+                }
             }
 #pragma unroll
             for (int ks = 0; ks < TR / 16; ++ks)
@@ -425,7 +438,7 @@ __global__ void __launch_bounds__(NT_B, 1)
         // ---- masked dA -> shared; state pass S = e^Gamma (S + dS') in TMEM, bf16 copy
         {
             uint32_t r[32];
-            tmem_ld32(tlane + C::COL_R + 32 * wg, r);
+            tmem_ld32(tlane + C::COL_A + 32 * wg, r);
             tmem_wait_ld();
             if (lane < 16) {
                 const int t = 16 * qd + lane;
@@ -470,11 +483,19 @@ __global__ void __launch_bounds__(NT_B, 1)
         if (warp == 0) {
             const bool leader = elect_one();
             const uint32_t aa = smem_u32(sA), ka = smem_u32(sk);
-            const uint32_t idQ = idesc_bf16(64, DKB, 0, 1);
+            const uint32_t idQ = idesc_bf16(64, C::SPLIT ? DKB / 2 : DKB, 0, 1);
 #pragma unroll
-            for (int ks = 0; ks < TR / 16; ++ks)
-                if (leader) mma_bf16(tbase + (16u << 16) + C::COL_R, sw128_desc(aa + ks * 32, 16, 1024),
-                         sw128_desc(ka + ks * 2048, BLK, 1024), idQ, 1);
+            for (int ks = 0; ks < TR / 16; ++ks) {
+                if (C::SPLIT) {   // key-dim blocks 0 and 1 of k~ into the two lane halves
+                    if (leader) mma_bf16(tbase + C::COL_R, sw128_desc(aa + ks * 32, 16, 1024),
+                             sw128_desc(ka + ks * 2048, BLK, 1024), idQ, 1);
+                    if (leader) mma_bf16(tbase + (16u << 16) + C::COL_R, sw128_desc(aa + ks * 32, 16, 1024),
+                             sw128_desc(ka + BLK + ks * 2048, BLK, 1024), idQ, 1);
+                } else {
+                    if (leader) mma_bf16(tbase + (16u << 16) + C::COL_R, sw128_desc(aa + ks * 32, 16, 1024),
+                             sw128_desc(ka + ks * 2048, BLK, 1024), idQ, 1);
+                }
+            }
             if (leader) mma_commit(bar_mma2);
             __syncwarp();
         }
@@ -482,17 +503,19 @@ __global__ void __launch_bounds__(NT_B, 1)
         tc_fence_after();
 
         // ---- dq = scale e^b D -> bf16 tile staged in the k slot (k~ is no longer read) -> TMA
-        //      store; q*dq into the g slot for dg. Row t of D sits in TMEM lane 16 + (t % 16) of
-        //      quadrant t / 16; the g slot holds e^b in the swizzled fp32 layout (gsw).
+        //      store; q*dq into the g slot for dg. Row t of D sits in lane (t % 16) of quadrant
+        //      t / 16, lanes 16-31 (SPLIT: lanes 0-15 hold key dims [0, DKB/2), 16-31 the rest);
+        //      the g slot holds e^b in the swizzled fp32 layout (gsw).
         {
             const int t = 16 * qd + (lane & 15);
             const bool row_ok = t0 + t < P.L;
             uint8_t* sdq = sk;
-            for (int c = wg * C::QC; c < (wg + 1) * C::QC; c += 16) {
+            for (int ct = wg * C::QC; ct < (wg + 1) * C::QC; ct += 16) {
                 uint32_t r[16];
-                tmem_ld16(tlane + C::COL_R + c, r);
+                tmem_ld16(tlane + C::COL_R + ct, r);
                 tmem_wait_ld();
-                if (lane >= 16) {
+                const int c = C::SPLIT ? (lane >> 4) * (DKB / 2) + ct : ct;   // key dim of r[0]
+                if (C::SPLIT || lane >= 16) {
                     float eb[16];
                     if (GATE == 1) {
 #pragma unroll
