@@ -679,11 +679,19 @@ struct KVCfg {
     static constexpr uint32_t COL_A = COL_R + DK;
     static constexpr uint32_t COL_DA = COL_A + 64;
     static constexpr uint32_t WR = DV > DK + 128 ? DV : DK + 128;
-    static constexpr uint32_t NCOL = pow2cols(DV + WR);
+    // SPLIT layout (whole 64-column blocks on both halves): from COL_K the dk' accumulator with
+    // key dims [0, DK/2) in lanes 0-15 and [DK/2, DK) in lanes 16-31, from COL_V dv likewise over
+    // the value dims, from COL_AD dA (lanes 0-15) and A (lanes 16-31), so that every epilogue
+    // lane holds a row.
+    static constexpr bool SPLIT = DK == 128 && DV >= 128;
+    static constexpr uint32_t COL_K = DV;
+    static constexpr uint32_t COL_V = COL_K + DK / 2;
+    static constexpr uint32_t COL_AD = COL_V + DV / 2;
+    static constexpr uint32_t NCOL = SPLIT ? pow2cols(COL_AD + 64) : pow2cols(DV + WR);
     static constexpr int HC = DV / 2;
     static constexpr int KC = DK / 2;
     static_assert(SMEM <= 227 * 1024, "shared memory");
-    static_assert(DV + WR <= 512, "tensor memory");
+    static_assert((SPLIT ? COL_AD + 64 : DV + WR) <= 512, "tensor memory");
     static_assert(STAGE % 1024 == 0, "stage alignment");
 };
 
@@ -847,17 +855,17 @@ __global__ void __launch_bounds__(NT_B, 1)
             tc_fence_after();
             const uint32_t qa = smem_u32(sq), ka = smem_u32(sk), va = smem_u32(sv), oa = smem_u32(so);
             const uint32_t id64 = idesc_bf16(64, 64, 0, 0);
+            const uint32_t tA = C::SPLIT ? tbase + (16u << 16) + C::COL_AD : tbase + C::COL_A;
+            const uint32_t tdA = C::SPLIT ? tbase + C::COL_AD : tbase + C::COL_DA;
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
-                if (leader) mma_bf16(tbase + C::COL_A, sw128_desc(qa + koff, 16, 1024), sw128_desc(ka + koff, 16, 1024), id64,
-                         kk > 0);
+                if (leader) mma_bf16(tA, sw128_desc(qa + koff, 16, 1024), sw128_desc(ka + koff, 16, 1024), id64, kk > 0);
             }
 #pragma unroll
             for (int kk = 0; kk < DV / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
-                if (leader) mma_bf16(tbase + C::COL_DA, sw128_desc(oa + koff, 16, 1024), sw128_desc(va + koff, 16, 1024), id64,
-                         kk > 0);
+                if (leader) mma_bf16(tdA, sw128_desc(oa + koff, 16, 1024), sw128_desc(va + koff, 16, 1024), id64, kk > 0);
             }
             if (leader) mma_commit(bar_mma1);
             __syncwarp();
@@ -889,24 +897,39 @@ __global__ void __launch_bounds__(NT_B, 1)
         __syncthreads();
         tc_fence_after();
         // ---- MMA group 2a (needs G~, not P): dk' = V G~^T, dv = k~ G~, G += (scale q~)^T dO
-        const uint32_t tdk = tbase + C::COL_R, tdv = tbase + (16u << 16) + C::COL_R;
+        const uint32_t tdk = C::SPLIT ? tbase + C::COL_K : tbase + C::COL_R;
+        const uint32_t tdv = C::SPLIT ? tbase + C::COL_V : tbase + (16u << 16) + C::COL_R;
         if (warp == 0) {
             const bool leader = elect_one();
             const uint32_t qa = smem_u32(sq), ka = smem_u32(sk), va = smem_u32(sv), oa = smem_u32(so);
             const uint32_t ga = smem_u32(sG);
-            const uint32_t idK2 = idesc_bf16(64, DK, 0, 0), idV2 = idesc_bf16(64, DV, 0, 1);
+            const uint32_t idK2 = idesc_bf16(64, C::SPLIT ? DK / 2 : DK, 0, 0);
+            const uint32_t idV2 = idesc_bf16(64, C::SPLIT ? DV / 2 : DV, 0, 1);
             const uint32_t idG = idesc_bf16(DK, DV, 1, 1);
 #pragma unroll
             for (int kk = 0; kk < DV / 16; ++kk) {  // V G~^T
                 const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
                 const uint32_t goff = (kk >> 2) * (DK * 128) + (kk & 3) * 32;
-                if (leader) mma_bf16(tdk, sw128_desc(va + koff, 16, 1024), sw128_desc(ga + goff, 16, 1024), idK2, kk > 0);
+                if (C::SPLIT) {   // key dims (rows of G~) [0, DK/2) and [DK/2, DK) into the two lane halves
+                    if (leader) mma_bf16(tdk, sw128_desc(va + koff, 16, 1024), sw128_desc(ga + goff, 16, 1024), idK2, kk > 0);
+                    if (leader) mma_bf16(tdk + (16u << 16), sw128_desc(va + koff, 16, 1024),
+                             sw128_desc(ga + goff + (DK / 2) * 128, 16, 1024), idK2, kk > 0);
+                } else {
+                    if (leader) mma_bf16(tdk, sw128_desc(va + koff, 16, 1024), sw128_desc(ga + goff, 16, 1024), idK2, kk > 0);
+                }
             }
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk) {  // k~ G~
                 const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
-                if (leader) mma_bf16(tdv, sw128_desc(ka + koff, 16, 1024), sw128_desc(ga + kk * 2048, DK * 128, 1024), idV2,
-                         kk > 0);
+                if (C::SPLIT) {   // value-dim blocks [0, DV/2) and [DV/2, DV) into the two lane halves
+                    if (leader) mma_bf16(tdv, sw128_desc(ka + koff, 16, 1024), sw128_desc(ga + kk * 2048, DK * 128, 1024),
+                             idV2, kk > 0);
+                    if (leader) mma_bf16(tdv + (16u << 16), sw128_desc(ka + koff, 16, 1024),
+                             sw128_desc(ga + (DV / 128) * (DK * 128) + kk * 2048, DK * 128, 1024), idV2, kk > 0);
+                } else {
+                    if (leader) mma_bf16(tdv, sw128_desc(ka + koff, 16, 1024), sw128_desc(ga + kk * 2048, DK * 128, 1024), idV2,
+                             kk > 0);
+                }
             }
 #pragma unroll
             for (int ks = 0; ks < TR / 16; ++ks)  // G += (scale q~)^T dO
@@ -915,8 +938,25 @@ __global__ void __launch_bounds__(NT_B, 1)
         }
         if (!block_wait(bar_mma1, i & 1)) { err = 1; break; }
         tc_fence_after();
-        // ---- P pass: masked A and masked dA -> bf16 in shared memory (rows in lanes 0-15)
-        {
+        // ---- P pass: masked A and masked dA -> bf16 in shared memory (rows in lanes 0-15;
+        //      SPLIT: one read, dA rows in lanes 0-15 and A rows in lanes 16-31)
+        if (C::SPLIT) {
+            uint32_t r[32];
+            tmem_ld32(tlane + C::COL_AD + 32 * wg, r);
+            tmem_wait_ld();
+            const int t = 16 * qd + (lane & 15);
+            uint8_t* dst = lane < 16 ? sdA : sAm;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float f[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int sidx = 32 * wg + 8 * u + j;
+                    f[j] = (sidx <= t) ? __uint_as_float(r[8 * u + j]) : 0.f;
+                }
+                store8_bf16(dst, sw128_off(t, 32 * wg + 8 * u, BLK), f);
+            }
+        } else {
             uint32_t ra[32], rd[32];
             tmem_ld32(tlane + C::COL_A + 32 * wg, ra);
             tmem_ld32(tlane + C::COL_DA + 32 * wg, rd);
@@ -947,13 +987,22 @@ __global__ void __launch_bounds__(NT_B, 1)
             const bool leader = elect_one();
             const uint32_t qa = smem_u32(sq), oa = smem_u32(so);
             const uint32_t ama = smem_u32(sAm), dama = smem_u32(sdA);
-            const uint32_t idK1 = idesc_bf16(64, DK, 1, 1), idV1 = idesc_bf16(64, DV, 1, 1);
+            const uint32_t idK1 = idesc_bf16(64, C::SPLIT ? DK / 2 : DK, 1, 1);
+            const uint32_t idV1 = idesc_bf16(64, C::SPLIT ? DV / 2 : DV, 1, 1);
 #pragma unroll
-            for (int ks = 0; ks < TR / 16; ++ks)
+            for (int ks = 0; ks < TR / 16; ++ks) {
                 if (leader) mma_bf16(tdk, sw128_desc(dama + ks * 2048, BLK, 1024), sw128_desc(qa + ks * 2048, BLK, 1024), idK1, 1);
+                if (C::SPLIT && leader)   // key-dim block 1 of q~ into lanes 16-31
+                    mma_bf16(tdk + (16u << 16), sw128_desc(dama + ks * 2048, BLK, 1024),
+                             sw128_desc(qa + BLK + ks * 2048, BLK, 1024), idK1, 1);
+            }
 #pragma unroll
-            for (int ks = 0; ks < TR / 16; ++ks)
+            for (int ks = 0; ks < TR / 16; ++ks) {
                 if (leader) mma_bf16(tdv, sw128_desc(ama + ks * 2048, BLK, 1024), sw128_desc(oa + ks * 2048, BLK, 1024), idV1, 1);
+                if (C::SPLIT && leader)   // value-dim blocks [DV/2, DV) of dO into lanes 16-31
+                    mma_bf16(tdv + (16u << 16), sw128_desc(ama + ks * 2048, BLK, 1024),
+                             sw128_desc(oa + (DV / 128) * BLK + ks * 2048, BLK, 1024), idV1, 1);
+            }
             if (leader) mma_commit(bar_mma2);
             __syncwarp();
         }
@@ -970,16 +1019,19 @@ __global__ void __launch_bounds__(NT_B, 1)
 
         // ---- dk = i e^-b X (bf16, staged in the q slot), k*dk = k~ X (into the g slot for dg),
         //      di = sum_d k~ X / i, and dv (bf16, staged in the v slot); q~ and V are no longer
-        //      read. Row s of X / dv sits in TMEM lane (s % 16) / 16 + (s % 16) of quadrant s / 16.
+        //      read. Row s of X / dv sits in TMEM lane (s % 16) / 16 + (s % 16) of quadrant s / 16
+        //      (SPLIT: both accumulators in both lane halves, by column half).
         {
             const int srw = 16 * qd + (lane & 15);
             const bool row_ok = t0 + srw < P.L;
             float dsum = 0.f;
-            for (int c = wg * C::KC; c < (wg + 1) * C::KC; c += 16) {
+            constexpr int KCW = C::SPLIT ? DK / 4 : C::KC, VCW = C::SPLIT ? DV / 4 : C::HC;   // TMEM columns per warpgroup
+            for (int ct = wg * KCW; ct < (wg + 1) * KCW; ct += 16) {
                 uint32_t r[16];
-                tmem_ld16(tlane + C::COL_R + c, r);
+                tmem_ld16(tlane + (C::SPLIT ? C::COL_K : C::COL_R) + ct, r);
                 tmem_wait_ld();
-                if (lane < 16) {
+                const int c = C::SPLIT ? (lane >> 4) * (DK / 2) + ct : ct;   // key dim of r[0]
+                if (C::SPLIT || lane < 16) {
                     const float iv = igs[srw];
                     float em[16];
                     if (GATE == 1) {
@@ -1016,12 +1068,14 @@ __global__ void __launch_bounds__(NT_B, 1)
                                 make_float4(kx[4 * q4], kx[4 * q4 + 1], kx[4 * q4 + 2], kx[4 * q4 + 3]);
                 }
             }
+            if (C::SPLIT) dsum += __shfl_xor_sync(0xffffffffu, dsum, 16);
             if (lane < 16) sdi[wg * TR + srw] = dsum;
-            for (int c = wg * C::HC; c < (wg + 1) * C::HC; c += 16) {
+            for (int ct = wg * VCW; ct < (wg + 1) * VCW; ct += 16) {
                 uint32_t r[16];
-                tmem_ld16(tlane + C::COL_R + c, r);
+                tmem_ld16(tlane + (C::SPLIT ? C::COL_V : C::COL_R) + ct, r);
                 tmem_wait_ld();
-                if (lane >= 16) {
+                const int c = C::SPLIT ? (lane >> 4) * (DV / 2) + ct : ct;   // value dim of r[0]
+                if (C::SPLIT || lane >= 16) {
                     store8_bf16(sv, sw128_off(srw, c, BLK), reinterpret_cast<const float*>(r));
                     store8_bf16(sv, sw128_off(srw, c + 8, BLK), reinterpret_cast<const float*>(r + 8));
                 }
