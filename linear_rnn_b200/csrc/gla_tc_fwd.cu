@@ -53,6 +53,10 @@ constexpr int BAR_S = 1;    // named barrier of the state-epilogue threads
 constexpr int BAR_TR = 2;   // named barrier of the transform threads
 constexpr int BAR_PO = 3;   // named barrier of the P/output-epilogue threads (output pass)
 constexpr float kLog2e = 1.4426950408889634f;
+// Tiles at the start of each segment that the state-only pass loads with the evict_last L2
+// policy (k, g, v: 64 KB a tile at Dk = Dv = 128, so ~9 tiles over ~140 CTAs keep about
+// 80 MB of the 126 MB L2)
+constexpr int kL2KeepTiles = 9;
 
 // 2^x on the special-function unit (inputs here are log-gate sums times log2(e))
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -256,11 +260,23 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 if (MODE == 0)
                     for (int cb = 0; cb < DK / 64; ++cb)
                         tma_load_3d(st + cb * BLK, &tq, cb * 64, t0, bh, &bar_full[s]);
-                for (int cb = 0; cb < DK / 64; ++cb)
-                    tma_load_3d(st + C::QB + cb * BLK, &tk, cb * 64, t0, bh, &bar_full[s]);
-                if (GATE == 1) tma_load_3d(st + C::QB + C::KB, &tg, 0, t0, bh, &bar_full[s]);
-                for (int vb = 0; vb < DVT / 64; ++vb)
-                    tma_load_3d(st + C::QB + C::KB + C::GB + vb * BLK, &tv, e0 + vb * 64, t0, bh, &bar_full[s]);
+                if (MODE == 1) {
+                    // the state-only pass walks its segment backwards, so the last tiles it
+                    // loads are the first ones the output pass loads next: those stay in L2
+                    const uint64_t pol = j >= ntiles - kL2KeepTiles ? l2_policy_evict_last() : l2_policy_evict_first();
+                    for (int cb = 0; cb < DK / 64; ++cb)
+                        tma_load_3d_hint(st + C::QB + cb * BLK, &tk, cb * 64, t0, bh, &bar_full[s], pol);
+                    if (GATE == 1) tma_load_3d_hint(st + C::QB + C::KB, &tg, 0, t0, bh, &bar_full[s], pol);
+                    for (int vb = 0; vb < DVT / 64; ++vb)
+                        tma_load_3d_hint(st + C::QB + C::KB + C::GB + vb * BLK, &tv, e0 + vb * 64, t0, bh, &bar_full[s],
+                                         pol);
+                } else {
+                    for (int cb = 0; cb < DK / 64; ++cb)
+                        tma_load_3d(st + C::QB + cb * BLK, &tk, cb * 64, t0, bh, &bar_full[s]);
+                    if (GATE == 1) tma_load_3d(st + C::QB + C::KB, &tg, 0, t0, bh, &bar_full[s]);
+                    for (int vb = 0; vb < DVT / 64; ++vb)
+                        tma_load_3d(st + C::QB + C::KB + C::GB + vb * BLK, &tv, e0 + vb * 64, t0, bh, &bar_full[s]);
+                }
                 *n_issued = j + 1;
                 // with a shallow ring (output pass, two stages) the tile that takes this stage
                 // next is brought into L2 now, so that its load (issued once the stage is
