@@ -16,6 +16,12 @@
 //                state MMA accumulates onto it, a TMEM pass applies e^Gamma) and bf16 in
 //                shared memory as the B operand of dO S^T.
 //   tc_bwd_dkdv  reverse tile walk per (b*h, segment); G in TMEM, bf16 G~ in shared memory.
+//                Dk = 256 (G does not fit one SM's TMEM next to the accumulators): a cluster
+//                of two CTAs per (b*h, segment), CTA kb holding G's key rows [128 kb, 128 kb
+//                + 128). Everything but dv (and the per-row sums behind di and a per-head dg)
+//                is complete in each CTA, because key dims only meet in those contractions;
+//                each CTA owns half of dv's value dims, receives the other CTA's partial sum
+//                of them into its shared memory (distributed shared memory, fp32) and adds it.
 // dg in fp32 without a separate pass: the dq kernel writes the in-segment exclusive prefix
 // of q*dq (into the dg buffer) and its segment total; the dk/dv kernel forms the in-segment
 // reverse sum of k*dk and finishes dg_t = (total - prefix_t) - revsum_t + carry, where the
@@ -50,7 +56,10 @@ struct BwdArgs {
     float* hT_ws;         // final state (for the dg term) or null
     float* dg;            // dg output; the dq kernel first stores there the in-segment
                           // exclusive prefix of q*dq, the dk/dv kernel finishes it
-    float* tq;            // [BH, nseg, Dk] in-segment totals of q*dq
+    float* tq;            // [BH, nseg, Dk] in-segment totals of q*dq (per-head gates: the
+                          // total of key block kb at key index 128 kb)
+    float* pre;           // per-head gates: [key blocks][BH*L] in-segment exclusive prefixes of
+                          // q*dq, one row per key block (the dg buffer when there is one block)
     int* status;
     int tiles_per_seg;
     int nseg;
@@ -58,6 +67,11 @@ struct BwdArgs {
 
 __device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity) {
     const bool ok = mbar_wait(bar, parity);
+    return __syncthreads_and(ok) != 0;
+}
+// The same for a barrier that the other CTA of the cluster arrives on.
+__device__ __forceinline__ bool block_wait_cluster(uint64_t* bar, uint32_t parity) {
+    const bool ok = mbar_wait_cluster(bar, parity);
     return __syncthreads_and(ok) != 0;
 }
 
@@ -607,8 +621,9 @@ __global__ void __launch_bounds__(NT_B, 1)
                 }
                 const float base = carry[0];
                 const float e0 = base + v - a0 - a1, e1 = base + v - a1;
-                if (t0 + 2 * lane < P.L) A.dg[rowbase + t0 + 2 * lane] = e0;
-                if (t0 + 2 * lane + 1 < P.L) A.dg[rowbase + t0 + 2 * lane + 1] = e1;
+                float* pre = A.pre + (long)kb * P.B * P.H * P.L + rowbase + t0;
+                if (t0 + 2 * lane < P.L) pre[2 * lane] = e0;
+                if (t0 + 2 * lane + 1 < P.L) pre[2 * lane + 1] = e1;
                 const float total = __shfl_sync(0xffffffffu, v, 31);
                 __syncwarp();
                 if (lane == 0) carry[0] = base + total;
@@ -624,7 +639,7 @@ __global__ void __launch_bounds__(NT_B, 1)
     if (!err) {
         __syncthreads();
         if (GATE == 1 && tid < DKB) A.tq[((long)bh * A.nseg + z) * P.Dk + d0 + tid] = carry[tid];
-        if (GATE == 2 && tid == 0) A.tq[(long)bh * A.nseg + z] = carry[0];
+        if (GATE == 2 && tid == 0) A.tq[((long)bh * A.nseg + z) * P.Dk + d0] = carry[0];
     }
     if (err) {
         if (warp == 0) {
@@ -690,12 +705,16 @@ struct KVCfg {
     static constexpr uint32_t NCOL = SPLIT ? pow2cols(COL_AD + 64) : pow2cols(DV + WR);
     static constexpr int HC = DV / 2;
     static constexpr int KC = DK / 2;
+    // key split: the G~ slot receives the other CTA's fp32 dv partial (half the value dims)
+    // and, from XROWS on, its 64 per-row sums of k' dk'
+    static constexpr uint32_t XROWS = (DV / 2) * TR * 4;
     static_assert(SMEM <= 227 * 1024, "shared memory");
     static_assert((SPLIT ? COL_AD + 64 : DV + WR) <= 512, "tensor memory");
     static_assert(STAGE % 1024 == 0, "stage alignment");
 };
 
-template <int DK, int DV, int GATE>
+// KS = key blocks of DK key dims (1, or 2 as a two-CTA cluster along x with DV >= 128).
+template <int DK, int DV, int GATE, int KS>
 __global__ void __launch_bounds__(NT_B, 1)
     k_tc_bwd_dkdv(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tg, const __grid_constant__ CUtensorMap tv,
@@ -712,7 +731,10 @@ __global__ void __launch_bounds__(NT_B, 1)
     uint64_t* bar_mma1 = bar_full + 2;
     uint64_t* bar_mma2 = bar_full + 3;
     uint64_t* bar_drain = bar_full + 4;   // error path: completion of every product issued
+    uint64_t* bar_free = bar_full + 5;    // KS = 2: the other CTA's G~ slot may take its dv partial
+    uint64_t* bar_recv = bar_full + 6;    // KS = 2: the other CTA's dv partial is in this G~ slot
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 64);
+    float* czs_peer = reinterpret_cast<float*>(small + 128);   // KS = 2: key block 1's part of czs
     float* tot = reinterpret_cast<float*>(small + 256);
     float* gam = tot + 2048;      // [DK]
     float* rowE = gam + DK;       // [64]
@@ -726,7 +748,12 @@ __global__ void __launch_bounds__(NT_B, 1)
     float* rows = red + 2 * DK;   // [64]
     float* czs = rows + TR;       // [1] per-head: sum over key dims of cz
 
-    const int bh = blockIdx.x, z = blockIdx.y;
+    static_assert(KS == 1 || (KS == 2 && C::SPLIT), "key split needs the split TMEM layout");
+    constexpr uint32_t kXRows = C::XROWS;
+    static_assert(KS == 1 || kXRows + 4 * TR <= C::GTB, "key-split exchange area");
+    const int bh = KS == 1 ? blockIdx.x : blockIdx.x >> 1, z = blockIdx.y;
+    const int kb = KS == 1 ? 0 : blockIdx.x & 1;   // = the CTA's rank in its cluster
+    const int d0 = kb * DK;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2, qd = warp & 3;
     const int ntiles_all = cdiv(P.L, TR);
     const int tile0 = z * A.tiles_per_seg;
@@ -742,26 +769,31 @@ __global__ void __launch_bounds__(NT_B, 1)
         mbar_init(bar_mma1, 1);
         mbar_init(bar_mma2, 1);
         mbar_init(bar_drain, 1);
+        if (KS == 2) {
+            mbar_init(bar_free, 1);
+            mbar_init(bar_recv, NT_B / 2);   // one arrival per sending thread of the other CTA
+        }
         mbar_fence_init();
     }
     if (warp == 0) tmem_alloc(tmem_slot, C::NCOL);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (KS == 2) cluster_sync();   // both CTAs' barriers are initialised before either touches the other
     const uint32_t tbase = *tmem_slot;
     const uint32_t tlane = tbase + ((uint32_t)(32 * qd) << 16);
 
     // ---- state gradient at the end of the segment into TMEM
     {
         const float* src = nullptr;
-        if (z == A.nseg - 1) src = A.dhT ? A.dhT + (long)bh * DK * P.Dv : nullptr;
-        else src = A.gend + ((long)bh * A.nseg + z) * DK * P.Dv;
+        if (z == A.nseg - 1) src = A.dhT ? A.dhT + ((long)bh * P.Dk + d0) * P.Dv : nullptr;
+        else src = A.gend + (((long)bh * A.nseg + z) * P.Dk + d0) * P.Dv;
         // dg at the segment's end: sum_e G_end[d][e] * S_end[d][e] (shift invariance of the
         // cumulative log-decay), with S_end the forward state after the segment
         const float* send = nullptr;
         if (GATE != 0 && src) {
-            if (z < A.nseg - 1) send = A.sinit + ((long)bh * A.nseg + z + 1) * DK * P.Dv;
-            else send = A.hT_ws ? A.hT_ws + (long)bh * DK * P.Dv : nullptr;
+            if (z < A.nseg - 1) send = A.sinit + (((long)bh * A.nseg + z + 1) * P.Dk + d0) * P.Dv;
+            else send = A.hT_ws ? A.hT_ws + ((long)bh * P.Dk + d0) * P.Dv : nullptr;
         }
         // staged through the ring stages, which are free until the first tile's loads
         static_assert(DK * DV * 4 <= C::NS * C::STAGE, "state staging");
@@ -780,14 +812,19 @@ __global__ void __launch_bounds__(NT_B, 1)
         }
         tmem_wait_st();
         if (tid < DK) {
-            const float tqv = GATE == 1 ? A.tq[((long)bh * A.nseg + z) * DK + tid] : 0.f;
+            const float tqv = GATE == 1 ? A.tq[((long)bh * A.nseg + z) * P.Dk + d0 + tid] : 0.f;
             cz[tid] = red[tid] + tqv;
         }
         __syncthreads();
         if (GATE == 2 && tid == 0) {
-            float sacc = A.tq[(long)bh * A.nseg + z];
+            float sacc = A.tq[((long)bh * A.nseg + z) * P.Dk + d0];
             for (int dd = 0; dd < DK; ++dd) sacc += cz[dd];
             czs[0] = sacc;
+            if (KS == 2 && kb == 1) st_cluster_f32(mapa_shared(czs_peer, 0), sacc);
+        }
+        if (KS == 2) {
+            cluster_sync();   // key block 1's part of czs has reached key block 0
+            if (GATE == 2 && kb == 0 && tid == 0) czs[0] += czs_peer[0];
         }
     }
     tc_fence_before();
@@ -799,12 +836,12 @@ __global__ void __launch_bounds__(NT_B, 1)
         const int t0 = tile_at(i) * TR;
         mbar_arrive_expect_tx(&bar_full[s], C::TXB);
         for (int cb = 0; cb < DK / 64; ++cb) {
-            tma_load_3d(st + cb * BLK, &tq, cb * 64, t0, bh, &bar_full[s]);
-            tma_load_3d(st + C::QB + cb * BLK, &tk, cb * 64, t0, bh, &bar_full[s]);
+            tma_load_3d(st + cb * BLK, &tq, d0 + cb * 64, t0, bh, &bar_full[s]);
+            tma_load_3d(st + C::QB + cb * BLK, &tk, d0 + cb * 64, t0, bh, &bar_full[s]);
         }
         if (GATE == 1)
             for (int gb = 0; gb < DK / 32; ++gb)
-                tma_load_3d(st + C::QB + C::KB + gb * BLK, &tg, 32 * gb, t0, bh, &bar_full[s]);
+                tma_load_3d(st + C::QB + C::KB + gb * BLK, &tg, d0 + 32 * gb, t0, bh, &bar_full[s]);
         for (int vb = 0; vb < DV / 64; ++vb) {
             tma_load_3d(st + C::QB + C::KB + C::GB + vb * BLK, &tv, vb * 64, t0, bh, &bar_full[s]);
             tma_load_3d(st + C::QB + C::KB + C::GB + C::VB + vb * BLK, &tdo, vb * 64, t0, bh, &bar_full[s]);
@@ -813,11 +850,11 @@ __global__ void __launch_bounds__(NT_B, 1)
         if (i + C::NS < ntiles) {
             const int tp = tile_at(i + C::NS) * TR;
             for (int cb = 0; cb < DK / 64; ++cb) {
-                tma_prefetch_l2_3d(&tq, cb * 64, tp, bh);
-                tma_prefetch_l2_3d(&tk, cb * 64, tp, bh);
+                tma_prefetch_l2_3d(&tq, d0 + cb * 64, tp, bh);
+                tma_prefetch_l2_3d(&tk, d0 + cb * 64, tp, bh);
             }
             if (GATE == 1)
-                for (int gb = 0; gb < DK / 32; ++gb) tma_prefetch_l2_3d(&tg, 32 * gb, tp, bh);
+                for (int gb = 0; gb < DK / 32; ++gb) tma_prefetch_l2_3d(&tg, d0 + 32 * gb, tp, bh);
             for (int vb = 0; vb < DV / 64; ++vb) {
                 tma_prefetch_l2_3d(&tv, vb * 64, tp, bh);
                 tma_prefetch_l2_3d(&tdo, vb * 64, tp, bh);
@@ -1009,13 +1046,15 @@ __global__ void __launch_bounds__(NT_B, 1)
         // the dq kernel's exclusive prefixes of this tile's rows, in flight during the epilogue
         constexpr int NGR = NT_B / DK, RPR = TR / NGR;
         const int dc = tid % DK, gr = tid / DK;
-        float* dgp = A.dg + (rowbase + t0 + gr * RPR) * DK + dc;
+        float* dgp = A.dg + (rowbase + t0 + gr * RPR) * P.Dk + d0 + dc;
         float pre[GATE == 1 ? RPR : 1];
         if (GATE == 1)
 #pragma unroll
-            for (int rr = 0; rr < RPR; ++rr) pre[rr] = (t0 + gr * RPR + rr < P.L) ? dgp[(long)rr * DK] : 0.f;
+            for (int rr = 0; rr < RPR; ++rr) pre[rr] = (t0 + gr * RPR + rr < P.L) ? dgp[(long)rr * P.Dk] : 0.f;
         if (!block_wait(bar_mma2, i & 1)) { err = 1; break; }
         tc_fence_after();
+        // every product that reads G~ is done: the other CTA may write its dv partial there
+        if (KS == 2 && tid == 0) mbar_arrive_remote(mapa_shared(bar_free, kb ^ 1));
 
         // ---- dk = i e^-b X (bf16, staged in the q slot), k*dk = k~ X (into the g slot for dg),
         //      di = sum_d k~ X / i, and dv (bf16, staged in the v slot); q~ and V are no longer
@@ -1070,14 +1109,60 @@ __global__ void __launch_bounds__(NT_B, 1)
             }
             if (C::SPLIT) dsum += __shfl_xor_sync(0xffffffffu, dsum, 16);
             if (lane < 16) sdi[wg * TR + srw] = dsum;
-            for (int ct = wg * VCW; ct < (wg + 1) * VCW; ct += 16) {
-                uint32_t r[16];
-                tmem_ld16(tlane + (C::SPLIT ? C::COL_V : C::COL_R) + ct, r);
-                tmem_wait_ld();
-                const int c = C::SPLIT ? (lane >> 4) * (DV / 2) + ct : ct;   // value dim of r[0]
-                if (C::SPLIT || lane >= 16) {
-                    store8_bf16(sv, sw128_off(srw, c, BLK), reinterpret_cast<const float*>(r));
-                    store8_bf16(sv, sw128_off(srw, c + 8, BLK), reinterpret_cast<const float*>(r + 8));
+            if (KS == 1) {
+                for (int ct = wg * VCW; ct < (wg + 1) * VCW; ct += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tlane + (C::SPLIT ? C::COL_V : C::COL_R) + ct, r);
+                    tmem_wait_ld();
+                    const int c = C::SPLIT ? (lane >> 4) * (DV / 2) + ct : ct;   // value dim of r[0]
+                    if (C::SPLIT || lane >= 16) {
+                        store8_bf16(sv, sw128_off(srw, c, BLK), reinterpret_cast<const float*>(r));
+                        store8_bf16(sv, sw128_off(srw, c + 8, BLK), reinterpret_cast<const float*>(r + 8));
+                    }
+                }
+            } else {
+                // dv over this key block is a partial sum. This CTA owns value dims [kb DV/2,
+                // (kb + 1) DV/2), the TMEM lane half kb; the lanes of the other half send theirs
+                // to the other CTA as fp32, 16-byte chunk j of row s at byte (64 j + s) * 16 of
+                // its G~ slot, followed (key block 1 only) by the rows' sums of k' dk'.
+                __syncthreads();   // sdi is complete
+                if (!block_wait_cluster(bar_free, i & 1)) { err = 1; break; }
+                const bool own = (lane >> 4) == kb;
+                const uint32_t peer_g = mapa_shared(sG, kb ^ 1);
+                for (int ct = wg * VCW; ct < (wg + 1) * VCW; ct += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tlane + C::COL_V + ct, r);
+                    tmem_wait_ld();
+                    if (!own)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            st_cluster_v4(peer_g + (uint32_t)((((ct >> 2) + u) * TR + srw) * 16),
+                                          __uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
+                                          __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
+                }
+                if (!own) {
+                    if (kb == 1 && wg == 0) st_cluster_f32(peer_g + kXRows + 4 * srw, sdi[srw] + sdi[TR + srw]);
+                    mbar_arrive_remote(mapa_shared(bar_recv, kb ^ 1));
+                }
+                if (!block_wait_cluster(bar_recv, i & 1)) { err = 1; break; }
+                const float* rx = reinterpret_cast<const float*>(sG);
+                for (int ct = wg * VCW; ct < (wg + 1) * VCW; ct += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tlane + C::COL_V + ct, r);
+                    tmem_wait_ld();
+                    if (own) {
+                        float f[16];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const float4 x = *reinterpret_cast<const float4*>(rx + (((ct >> 2) + u) * TR + srw) * 4);
+                            f[4 * u] = __uint_as_float(r[4 * u]) + x.x;
+                            f[4 * u + 1] = __uint_as_float(r[4 * u + 1]) + x.y;
+                            f[4 * u + 2] = __uint_as_float(r[4 * u + 2]) + x.z;
+                            f[4 * u + 3] = __uint_as_float(r[4 * u + 3]) + x.w;
+                        }
+                        store8_bf16(sv, sw128_off(srw, ct, BLK), f);
+                        store8_bf16(sv, sw128_off(srw, ct + 8, BLK), f + 8);
+                    }
                 }
             }
         }
@@ -1086,11 +1171,14 @@ __global__ void __launch_bounds__(NT_B, 1)
         __syncthreads();
         tc_fence_after();
         if (tid == 0) {
-            for (int cb = 0; cb < DK / 64; ++cb) tma_store_3d(&tout, sq + cb * BLK, 64 * cb, t0, bh);
-            for (int vb = 0; vb < DV / 64; ++vb) tma_store_3d(&tout2, sv + vb * BLK, 64 * vb, t0, bh);
+            for (int cb = 0; cb < DK / 64; ++cb) tma_store_3d(&tout, sq + cb * BLK, d0 + 64 * cb, t0, bh);
+            for (int vb = 0; vb < DV / 64 / KS; ++vb)
+                tma_store_3d(&tout2, sv + vb * BLK, kb * (DV / KS) + 64 * vb, t0, bh);
             bulk_commit();
         }
-        if (A.di && tid < TR && t0 + tid < P.L) A.di[rowbase + t0 + tid] = (sdi[tid] + sdi[TR + tid]) / igs[tid];
+        const float* prow = reinterpret_cast<const float*>(sG + kXRows);   // KS = 2, key block 0
+        if (A.di && kb == 0 && tid < TR && t0 + tid < P.L)
+            A.di[rowbase + t0 + tid] = (sdi[tid] + sdi[TR + tid] + (KS == 2 ? prow[tid] : 0.f)) / igs[tid];
         // ---- dg = (in-segment q*dq total - exclusive prefix) - reverse sum of k*dk + carry
         if (GATE == 1) {
             // thread = (key dim dc, group of RPR rows; the prefixes were fetched above): local
@@ -1111,17 +1199,18 @@ __global__ void __launch_bounds__(NT_B, 1)
 #pragma unroll
             for (int rr = RPR - 1; rr >= 0; --rr) {
                 sx += sg[gsw(gr * RPR + rr, dc)];
-                if (t0 + gr * RPR + rr < P.L) dgp[(long)rr * DK] = cx - pre[rr] - sx;
+                if (t0 + gr * RPR + rr < P.L) dgp[(long)rr * P.Dk] = cx - pre[rr] - sx;
             }
             __syncthreads();
             if (gr == 0) rk[dc] += T;
-        } else if (GATE == 2) {
+        } else if (GATE == 2 && kb == 0) {
+            // (key block 0 forms the per-head dg of both blocks)
             for (int j = 0; j < 8; ++j) {
                 const int r = warp * 8 + j;
                 float acc = 0.f;
                 for (int dd = lane; dd < DK; dd += 32) acc += sg[gsw(r, dd)];
                 for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-                if (lane == 0) rows[r] = acc;
+                if (lane == 0) rows[r] = acc + (KS == 2 ? prow[r] : 0.f);
             }
             __syncthreads();
             if (warp == 0) {  // reverse inclusive scan over 64 rows, two per lane
@@ -1135,8 +1224,11 @@ __global__ void __launch_bounds__(NT_B, 1)
                 const float base = rk[0], cc = czs[0];
                 const float s0 = base + v, s1 = base + v - a0;
                 const int ta = t0 + 2 * lane;
-                if (ta < P.L) A.dg[rowbase + ta] = cc - A.dg[rowbase + ta] - s0;
-                if (ta + 1 < P.L) A.dg[rowbase + ta + 1] = cc - A.dg[rowbase + ta + 1] - s1;
+                // the dq kernel's exclusive prefixes of q*dq, one row per key block
+                const long bhl = (long)P.B * P.H * P.L;
+                auto prefix = [&](int t) { return A.pre[rowbase + t] + (KS == 2 ? A.pre[bhl + rowbase + t] : 0.f); };
+                if (ta < P.L) A.dg[rowbase + ta] = cc - prefix(ta) - s0;
+                if (ta + 1 < P.L) A.dg[rowbase + ta + 1] = cc - prefix(ta + 1) - s1;
                 const float total = __shfl_sync(0xffffffffu, v, 0);
                 __syncwarp();
                 if (lane == 0) rk[0] = base + total;
@@ -1164,7 +1256,7 @@ __global__ void __launch_bounds__(NT_B, 1)
             tmem_ld16(tlane + c, r);
             tmem_wait_ld();
             if (srow_ok) {
-                float* dst = A.dh0 + ((long)bh * DK + srow) * P.Dv + c;
+                float* dst = A.dh0 + ((long)bh * P.Dk + d0 + srow) * P.Dv + c;
 #pragma unroll
                 for (int j = 0; j < 16; j += 4)
                     *reinterpret_cast<float4*>(dst + j) = make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
@@ -1176,6 +1268,8 @@ __global__ void __launch_bounds__(NT_B, 1)
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, C::NCOL);
+    // neither CTA of a pair leaves while the other may still write into its shared memory
+    if (KS == 2) cluster_sync();
 }
 
 // ============================================================================ host side
@@ -1206,12 +1300,16 @@ static BwdPlan plan_bwd(const Dims& P) {
     return pl;
 }
 
+// Dk = 256 splits the key dims over a CTA pair whose dv exchange needs the split TMEM layout
+// (Dv >= 128).
 bool bwd_supports(const Dims& P) {
-    return P.C % TR == 0 && (P.Dk == 64 || P.Dk == 128) && (P.Dv == 64 || P.Dv == 128 || P.Dv == 256);
+    if (P.C % TR != 0) return false;
+    if (P.Dk == 64 || P.Dk == 128) return P.Dv == 64 || P.Dv == 128 || P.Dv == 256;
+    return P.Dk == 256 && (P.Dv == 128 || P.Dv == 256);
 }
 
 struct BwdWs {
-    float *seg_state, *seg_gamma, *sinit, *gend, *hT, *tq;
+    float *seg_state, *seg_gamma, *sinit, *gend, *hT, *tq, *pre;
     size_t total;
 };
 
@@ -1224,6 +1322,10 @@ static BwdWs bwd_layout(const Dims& P, char* base) {
     off = align_up(off + st, 256);
     w.tq = reinterpret_cast<float*>(base + off);
     off = align_up(off + 4 * BH * (size_t)pl.nseg * P.Dk, 256);
+    if (P.gate == GLA_GATE_PER_HEAD && P.Dk > 128) {   // per-key-block prefixes of q*dq
+        w.pre = reinterpret_cast<float*>(base + off);
+        off = align_up(off + 4 * BH * (size_t)(P.Dk / 128) * P.L, 256);
+    }
     if (pl.nseg > 1) {
         w.seg_state = reinterpret_cast<float*>(base + off);
         off = align_up(off + st * pl.nseg, 256);
@@ -1263,20 +1365,39 @@ static cudaError_t launch_dq(const Dims& P, const BwdPlan& pl, const CUtensorMap
     return cudaGetLastError();
 }
 
-template <int DK, int DV, int GATE>
+template <int DK, int DV, int GATE, int KS>
 static cudaError_t launch_dkdv(const Dims& P, const BwdPlan& pl, const CUtensorMap& mq, const CUtensorMap& mk,
                                const CUtensorMap& mg, const CUtensorMap& mv, const CUtensorMap& mo,
                                const CUtensorMap& mdk, const CUtensorMap& mdv, const BwdArgs& a, cudaStream_t st) {
     using C = KVCfg<DK, DV, GATE>;
-    auto kern = k_tc_bwd_dkdv<DK, DV, GATE>;
+    auto kern = k_tc_bwd_dkdv<DK, DV, GATE, KS>;
     static bool attr = false;
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    dim3 grid(P.B * P.H, pl.nseg);
-    GLA_LAUNCH("tc_bwd_dkdv", st, kern<<<grid, NT_B, C::SMEM, st>>>(mq, mk, mg, mv, mo, mdk, mdv, a, P));
+    if (KS == 1) {
+        dim3 grid(P.B * P.H, pl.nseg);
+        GLA_LAUNCH("tc_bwd_dkdv", st, kern<<<grid, NT_B, C::SMEM, st>>>(mq, mk, mg, mv, mo, mdk, mdv, a, P));
+        return cudaGetLastError();
+    }
+    // the two key blocks of a (b*h, segment) run as one cluster of two CTAs
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(KS * P.B * P.H, pl.nseg);
+    cfg.blockDim = dim3(NT_B);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = KS;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaSuccess;
+    GLA_LAUNCH("tc_bwd_dkdv", st, e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mg, mv, mo, mdk, mdv, a, P));
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -1289,6 +1410,7 @@ static cudaError_t run_bwd(const Dims& P, const void* q, const void* k, const vo
     const BwdWs w = bwd_layout(P, static_cast<char*>(ws));
     const int BH = P.B * P.H;
     constexpr int DKB = DK > 128 ? 128 : DK;
+    constexpr int KS = DK / DKB;
     CUtensorMap mq, mk, mv, mo, mg, mdq, mdk, mdv;
     if (!make_map(&mdq, dq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dk, P.L, BH, 64, true) ||
         !make_map(&mdk, dk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P.Dk, P.L, BH, 64, true) ||
@@ -1330,6 +1452,7 @@ static cudaError_t run_bwd(const Dims& P, const void* q, const void* k, const vo
     a.hT_ws = (dhT && GATE != 0) ? w.hT : nullptr;
     a.dg = dg;
     a.tq = w.tq;
+    a.pre = (GATE == 2 && KS == 2) ? w.pre : dg;
     a.status = status;
     a.tiles_per_seg = pl.tiles_per_seg;
     a.nseg = pl.nseg;
@@ -1341,7 +1464,7 @@ static cudaError_t run_bwd(const Dims& P, const void* q, const void* k, const vo
         e = seg_rscan(P, pl.nseg, w.seg_state, w.seg_gamma, dhT, w.gend, st);
         if (e != cudaSuccess) return e;
     }
-    e = launch_dkdv<DK, DV, GATE>(P, pl, mq, mk, mg, mv, mo, mdk, mdv, a, st);
+    e = launch_dkdv<DKB, DV, GATE, KS>(P, pl, mq, mk, mg, mv, mo, mdk, mdv, a, st);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1371,6 +1494,8 @@ cudaError_t bwd(const Dims& P, const void* q, const void* k, const void* v, cons
     GLA_BWD_CASE(128, 64)
     GLA_BWD_CASE(128, 128)
     GLA_BWD_CASE(128, 256)
+    GLA_BWD_CASE(256, 128)
+    GLA_BWD_CASE(256, 256)
 #undef GLA_BWD_CASE
     return cudaErrorInvalidValue;
 }
