@@ -81,6 +81,25 @@ def test_saved_state_sizes_follow_the_backward_plan():
     assert saved(Dk=96) == 0                                # invalid problem
 
 
+def test_backward_segments_whole_chunks_and_bounded():
+    """Backward segments are whole chunks of about ten tiles at most (dg's accuracy bound)
+    unless one chunk is longer, and cover the sequence. Without a GPU the library assumes 148
+    SMs."""
+    auto = _lib.GLA_PLAN_AUTO
+    for B, H, L, Dk, Dv, C in [(4, 16, 4096, 128, 256, 64), (2, 8, 8192, 256, 256, 64), (1, 2, 333, 256, 128, 64),
+                               (1, 8, 65536, 128, 128, 256), (1, 1, 5000, 64, 64, 1024), (3, 5, 1, 64, 64, 64)]:
+        plan, nseg, tps = _lib.plan_info(prob(B=B, H=H, L=L, Dk=Dk, Dv=Dv, chunk=C, plan=auto), True)
+        ntiles = -(-L // 64)
+        assert plan == _lib.GLA_PLAN_TC
+        assert tps % (C // 64) == 0 and tps < 10 + C // 64   # ten tiles, rounded up to whole chunks
+        assert nseg == -(-ntiles // tps)
+    # c3: 7 segments of 10 tiles per head; c5: 13 of 10 per (head, key block)
+    assert _lib.plan_info(prob(B=4, H=16, L=4096, Dk=128, Dv=256, plan=auto), True) == (_lib.GLA_PLAN_TC, 7, 10)
+    assert _lib.plan_info(prob(B=2, H=8, L=8192, Dk=256, Dv=256, plan=auto), True) == (_lib.GLA_PLAN_TC, 13, 10)
+    # Dk = 256 runs on tensor cores with Dv >= 128 (the key-split CTA pair), else on CUDA cores
+    assert _lib.plan_info(prob(Dk=256, Dv=64, plan=auto), True)[0] == _lib.GLA_PLAN_SIMT
+
+
 def test_status_strings():
     for s in range(7):
         assert len(_lib.status_string(s)) >= 2

@@ -224,7 +224,7 @@ def test_strong_gates_flagged_on_tensor_cores_and_exact_on_simt():
     check_bwd(x, w, plan="simt")
 
 
-@pytest.mark.parametrize("name,L", [("c3", None), ("c3", 1000), ("c2", 700), ("c5", 2000)])
+@pytest.mark.parametrize("name,L", [("c3", None), ("c3", 1000), ("c2", 1500), ("c5", 2000)])
 def test_backward_from_saved_states(name, L):
     """The training pair: the forward writes the states at the backward's segment starts and
     the backward uses them instead of its own state pass; same oracle bound, and close to the
