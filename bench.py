@@ -124,8 +124,10 @@ def kernel_bytes(name, w, fseg=1, bseg=1):
 # time: a kernel whose source has changed since reports traffic null. `scale`: the capture
 # ran a smaller case of the same workload; traffic grows with the heads processed.
 MEASURED_TRAFFIC = {
-    ("tc_bwd_dkdv", "c3"): {"bytes": 246.6e6, "scale": 4, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
-                            "sha": "c42757ed5fd7e8db", "profile": "profiles/tc_bwd_dkdv_c3_b1.md"},
+    ("tc_bwd_dkdv", "c3"): {"bytes": 247.5e6, "scale": 4, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
+                            "sha": "34a4faebc4d36744", "profile": "profiles/tc_bwd_dkdv_c3_b1.md"},
+    ("tc_bwd_dkdv", "c5"): {"bytes": 243.6e6, "scale": 2, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
+                            "sha": "34a4faebc4d36744", "profile": "profiles/tc_bwd_dkdv_c5_b1.md"},
     ("tc_fwd", "c2"): {"bytes": 187.2e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_fwd.cu",
                        "sha": "f6c391e27d69d84e", "profile": "profiles/tc_fwd_c2.md"},
 }
