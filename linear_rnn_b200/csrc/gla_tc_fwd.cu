@@ -115,7 +115,10 @@ struct FwdArgs {
     const float* gh;      // per-head log-gate [BH*L] (GATE == 2)
     const float* ig;      // input gate [BH*L] or null
     const float* h0;      // [BH, Dk, Dv] or null
-    const float* sinit;   // [BH, nseg, Dk, Dv] initial states of segments z > 0 (output pass)
+    const float* sinit;   // [BH, sinit_nseg, Dk, Dv] initial states of the state pass's segments
+                          // (output pass: segment z starts from entry z * sinit_step)
+    int sinit_nseg;
+    int sinit_step;
     __nv_bfloat16* o;     // [BH, L, Dv]
     float* hT;            // [BH, Dk, Dv] or null
     float* seg_state;     // state-only pass: [BH, nseg, Dk, Dv] local end states
@@ -208,7 +211,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     const float* src = nullptr;
     if (MODE == 0) {
         if (z == 0) src = A.h0 ? A.h0 + (long)bh * DK * P.Dv + e0 : nullptr;
-        else src = A.sinit + ((long)bh * A.nseg + z) * DK * P.Dv + e0;
+        else src = A.sinit + ((long)bh * A.sinit_nseg + (long)z * A.sinit_step) * DK * P.Dv + e0;
     }
     const float* stg = reinterpret_cast<const float*>(sm);
     if (src) {
@@ -946,14 +949,36 @@ FwdPlan plan_fwd(const Dims& P) {
     return pl;
 }
 
+// Dv tile of the state-only passes: 128 columns wherever the ring keeps several stages (for
+// Dk = 256 with per-key gates a 128-column stage holds 112 KB and the ring a single stage).
+static int pick_state_dvt(const Dims& P) {
+    if (P.Dv % 128 != 0) return 64;
+    return (P.Dk == 256 && P.gate == GLA_GATE_PER_KEY) ? 64 : 128;
+}
+
+// The forward's state pass covers segments 0..nseg-2 of the output pass. It runs in R
+// sub-segments per output segment (R divides the segment's tiles), as many as keep its CTAs
+// within one wave; the scan then yields the initial state of every sub-segment and the
+// output pass reads every R-th.
+static int state_subsegments(const Dims& P, const FwdPlan& pl) {
+    if (pl.nseg <= 1) return 1;
+    const long per = (long)P.B * P.H * (P.Dv / pick_state_dvt(P)) * (pl.nseg - 1);
+    const long sms = num_sms();
+    int R = 1;
+    for (int r = 2; r <= pl.tiles_per_seg; ++r)
+        if (pl.tiles_per_seg % r == 0 && per * r <= sms) R = r;
+    return R;
+}
+
 size_t fwd_workspace_bytes(const Dims& P) {
     const FwdPlan pl = plan_fwd(P);
     if (pl.nseg <= 1) return kStatusBytes;
     const size_t BH = (size_t)P.B * P.H;
+    const size_t nsub = (size_t)(pl.nseg - 1) * state_subsegments(P, pl) + 1;
     size_t off = kStatusBytes;
-    off = align_up(off + 4 * BH * pl.nseg * P.Dk * P.Dv, 256);   // local end states
-    off = align_up(off + 4 * BH * pl.nseg * P.Dk, 256);          // log-decay totals
-    off = align_up(off + 4 * BH * pl.nseg * P.Dk * P.Dv, 256);   // initial states
+    off = align_up(off + 4 * BH * nsub * P.Dk * P.Dv, 256);   // local end states
+    off = align_up(off + 4 * BH * nsub * P.Dk, 256);          // log-decay totals
+    off = align_up(off + 4 * BH * nsub * P.Dk * P.Dv, 256);   // initial states
     return off;
 }
 
@@ -1022,23 +1047,28 @@ static cudaError_t run(const Dims& P, const void* q, const void* k, const void* 
     a.tiles_per_seg = pl.tiles_per_seg;
     a.nseg = pl.nseg;
     a.seg_offset = 0;
+    a.sinit_nseg = pl.nseg;
+    a.sinit_step = 1;
     if (saved) {
         a.saved = saved;
         bwd_plan_info(P, &a.save_nseg, &a.save_tps);
     }
     if (pl.nseg > 1) {
+        const int R = state_subsegments(P, pl);
+        const int nsub = (pl.nseg - 1) * R + 1;
         char* w = static_cast<char*>(ws);
         size_t off = kStatusBytes;
         float* seg_state = reinterpret_cast<float*>(w + off);
-        off = align_up(off + 4 * (size_t)BH * pl.nseg * P.Dk * P.Dv, 256);
+        off = align_up(off + 4 * (size_t)BH * nsub * P.Dk * P.Dv, 256);
         float* seg_gamma = reinterpret_cast<float*>(w + off);
-        off = align_up(off + 4 * (size_t)BH * pl.nseg * P.Dk, 256);
+        off = align_up(off + 4 * (size_t)BH * nsub * P.Dk, 256);
         float* sinit = reinterpret_cast<float*>(w + off);
         a.sinit = sinit;
-        cudaError_t e = state_run<DK, DVT, GATE>(P, 1, k, v, g, ig, pl.nseg, pl.tiles_per_seg, seg_state, seg_gamma,
-                                                 a.status, st);
+        a.sinit_nseg = nsub;
+        a.sinit_step = R;
+        cudaError_t e = state_pass(P, 1, k, v, g, ig, nsub, pl.tiles_per_seg / R, seg_state, seg_gamma, a.status, st);
         if (e != cudaSuccess) return e;
-        e = seg_scan(P, pl.nseg, seg_state, seg_gamma, h0, sinit, st);
+        e = seg_scan(P, nsub, seg_state, seg_gamma, h0, sinit, st);
         if (e != cudaSuccess) return e;
     }
     return launch_one<DK, DVT, GATE, 0>(mq, mk, mv, mg, mo, a, P, pl.nseg, st);
@@ -1078,7 +1108,10 @@ static cudaError_t state_gate(const Dims& P, int mode, const void* a_src, const 
                               const float* ig, int nseg, int tps, float* ss, float* sg, int* status, cudaStream_t st) {
     switch (P.gate) {
         case GLA_GATE_NONE: return state_run<DK, DVT, 0>(P, mode, a_src, b_src, g, ig, nseg, tps, ss, sg, status, st);
-        case GLA_GATE_PER_KEY: return state_run<DK, DVT, 1>(P, mode, a_src, b_src, g, ig, nseg, tps, ss, sg, status, st);
+        case GLA_GATE_PER_KEY:
+            // (pick_state_dvt keeps per-key gates with Dk = 256 on 64-column tiles)
+            if constexpr (DK == 256 && DVT == 128) return cudaErrorInvalidValue;
+            else return state_run<DK, DVT, 1>(P, mode, a_src, b_src, g, ig, nseg, tps, ss, sg, status, st);
         default: return state_run<DK, DVT, 2>(P, mode, a_src, b_src, g, ig, nseg, tps, ss, sg, status, st);
     }
 }
@@ -1086,7 +1119,7 @@ static cudaError_t state_gate(const Dims& P, int mode, const void* a_src, const 
 cudaError_t state_pass(const Dims& P, int mode, const void* a_src, const void* b_src, const float* g,
                        const float* ig, int nseg, int tiles_per_seg, float* seg_state, float* seg_gamma, int* status,
                        cudaStream_t st) {
-    const int dvt = pick_dvt(P);
+    const int dvt = pick_state_dvt(P);
     if (P.Dk == 64) {
         if (dvt == 128) return state_gate<64, 128>(P, mode, a_src, b_src, g, ig, nseg, tiles_per_seg, seg_state, seg_gamma, status, st);
         return state_gate<64, 64>(P, mode, a_src, b_src, g, ig, nseg, tiles_per_seg, seg_state, seg_gamma, status, st);
@@ -1095,6 +1128,7 @@ cudaError_t state_pass(const Dims& P, int mode, const void* a_src, const void* b
         if (dvt == 128) return state_gate<128, 128>(P, mode, a_src, b_src, g, ig, nseg, tiles_per_seg, seg_state, seg_gamma, status, st);
         return state_gate<128, 64>(P, mode, a_src, b_src, g, ig, nseg, tiles_per_seg, seg_state, seg_gamma, status, st);
     }
+    if (dvt == 128) return state_gate<256, 128>(P, mode, a_src, b_src, g, ig, nseg, tiles_per_seg, seg_state, seg_gamma, status, st);
     return state_gate<256, 64>(P, mode, a_src, b_src, g, ig, nseg, tiles_per_seg, seg_state, seg_gamma, status, st);
 }
 

@@ -168,3 +168,19 @@ def test_tc_bwd_dk256_deterministic_and_matches_simt():
     for n in ("dq", "dk", "dv", "dg", "di"):
         assert torch.equal(a[n], b[n]), n
         assert err(f64(a[n]), f64(c[n])) < 1e-2, n
+
+
+# ---------------------------------------------- forward state pass in finer sub-segments
+# With few (head, Dv tile) pairs the forward's state pass runs R sub-segments per output
+# segment (here R = 4 or 16) and the output pass starts from every R-th scanned state.
+
+@pytest.mark.parametrize("Dk,Dv,chunk,gate,ig", [(256, 256, 256, I.GATE_PER_HEAD, True),
+                                                 (256, 256, 256, I.GATE_PER_KEY, False),
+                                                 (128, 128, 1024, I.GATE_PER_KEY, True),
+                                                 (256, 128, 256, I.GATE_NONE, False)])
+def test_tc_fwd_state_subsegments(Dk, Dv, chunk, gate, ig):
+    w = base(B=1, H=1, L=2000 if chunk == 256 else 5000, Dk=Dk, Dv=Dv, chunk=chunk, gate=gate, input_gate=ig,
+             h0_std=0.3, gate_mean=3.0 if gate == I.GATE_PER_HEAD else 0.0,
+             gate_div=1.0 if gate == I.GATE_PER_HEAD else 16.0)
+    eo, eh = run_tc_fwd(w, 24)
+    assert eo <= TOL and eh <= TOL, (eo, eh)
