@@ -355,20 +355,19 @@ __global__ void __launch_bounds__(NT_B, 1)
         if (GATE == 1)
             for (int gb = 0; gb < DKB / 32; ++gb)
                 tma_load_3d(st + C::QB + C::KB + gb * BLK, &tg, d0 + 32 * gb, t0, bh, &bar_full[s]);
-        // the tile that takes this stage next is brought into L2 now, so that its loads do
-        // not wait on DRAM
-        if (i + C::NS < ntiles) {
-            const int tp = (tile0 + i + C::NS) * TR;
-            for (int cb = 0; cb < DKB / 64; ++cb) {
-                if (GATE != 0) tma_prefetch_l2_3d(&tq, d0 + cb * 64, tp, bh);
-                tma_prefetch_l2_3d(&tk, d0 + cb * 64, tp, bh);
-            }
-            if (GATE == 1)
-                for (int gb = 0; gb < DKB / 32; ++gb) tma_prefetch_l2_3d(&tg, d0 + 32 * gb, tp, bh);
-            for (int vb = 0; vb < DV / 64; ++vb) {
-                tma_prefetch_l2_3d(&tv, vb * 64, tp, bh);
-                tma_prefetch_l2_3d(&tdo, vb * 64, tp, bh);
-            }
+    };
+    // tile i into L2, ahead of its loads (issued by another warp than the loads and products)
+    auto issue_prefetch = [&](int i) {
+        const int tp = (tile0 + i) * TR;
+        for (int cb = 0; cb < DKB / 64; ++cb) {
+            if (GATE != 0) tma_prefetch_l2_3d(&tq, d0 + cb * 64, tp, bh);
+            tma_prefetch_l2_3d(&tk, d0 + cb * 64, tp, bh);
+        }
+        if (GATE == 1)
+            for (int gb = 0; gb < DKB / 32; ++gb) tma_prefetch_l2_3d(&tg, d0 + 32 * gb, tp, bh);
+        for (int vb = 0; vb < DV / 64; ++vb) {
+            tma_prefetch_l2_3d(&tv, vb * 64, tp, bh);
+            tma_prefetch_l2_3d(&tdo, vb * 64, tp, bh);
         }
     };
     auto issue_vo = [&](int i, int s) {
@@ -385,6 +384,16 @@ __global__ void __launch_bounds__(NT_B, 1)
             issue_qkg(i, i);
             issue_vo(i, i);
         }
+    if (tid == 32)
+        for (int i = C::NS; i < 2 * C::NS && i < ntiles; ++i) issue_prefetch(i);
+    // input and per-head gates of the next tile, loaded a tile ahead into registers
+    float nig = 1.f, ngh = 0.f;
+    auto fetch_gates = [&](int i) {
+        const int t = (tile0 + i) * TR + tid;
+        if (A.ig) nig = t < P.L ? A.ig[rowbase + t] : 1.f;
+        if (GATE == 2) ngh = t < P.L ? A.gh[rowbase + t] : 0.f;
+    };
+    if (tid < TR) fetch_gates(0);
 
     int err = 0, n_mma = 0;
     for (int i = 0; i < ntiles; ++i) {
@@ -397,9 +406,9 @@ __global__ void __launch_bounds__(NT_B, 1)
         uint8_t* so = sv + C::VB;
         const int t0 = (tile0 + i) * TR;
         if (tid < TR) {
-            const int t = t0 + tid;
-            igs[tid] = (A.ig && t < P.L) ? A.ig[rowbase + t] : 1.f;
-            if (GATE == 2) ghs[tid] = (t < P.L) ? A.gh[rowbase + t] : 0.f;
+            igs[tid] = nig;
+            if (GATE == 2) ghs[tid] = ngh;
+            if (i + 1 < ntiles) fetch_gates(i + 1);
         }
         if (!block_wait(&bar_full[s], (i / C::NS) & 1)) { err = 1; break; }
 
@@ -443,6 +452,8 @@ __global__ void __launch_bounds__(NT_B, 1)
                 if (leader) mma_bf16(tbase, sw128_desc(ka + ks * 2048, BLK, 1024), sw128_desc(va + ks * 2048, BLK, 1024), idS, 1);
             if (leader) mma_commit(bar_mma1);
             __syncwarp();
+        } else if (tid == 32 && i + 2 * C::NS < ntiles) {
+            issue_prefetch(i + 2 * C::NS);   // while warp 0 issues the products
         }
         ++n_mma;
         if (!block_wait(bar_mma1, i & 1)) { err = 1; break; }
@@ -524,6 +535,7 @@ __global__ void __launch_bounds__(NT_B, 1)
             const int t = 16 * qd + (lane & 15);
             const bool row_ok = t0 + t < P.L;
             uint8_t* sdq = sk;
+            float rsum = 0.f;   // per-head gates: this lane's part of the row's sum of q*dq
             for (int ct = wg * C::QC; ct < (wg + 1) * C::QC; ct += 16) {
                 uint32_t r[16];
                 tmem_ld16(tlane + C::COL_R + ct, r);
@@ -561,13 +573,19 @@ __global__ void __launch_bounds__(NT_B, 1)
                             const float qs1 = __bfloat162float(__float2bfloat16_rn(qf.y * P.scale * eb[2 * u + 1]));
                             x[2 * u] = row_ok ? qs0 * __uint_as_float(r[2 * u]) : 0.f;
                             x[2 * u + 1] = row_ok ? qs1 * __uint_as_float(r[2 * u + 1]) : 0.f;
+                            rsum += x[2 * u] + x[2 * u + 1];
                         }
+                        if (GATE == 1)
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4)
-                            *reinterpret_cast<float4*>(sg + gsw(t, c + 4 * q4)) =
-                                make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
+                            for (int q4 = 0; q4 < 4; ++q4)
+                                *reinterpret_cast<float4*>(sg + gsw(t, c + 4 * q4)) =
+                                    make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
                     }
                 }
+            }
+            if (GATE == 2) {   // the row's sum over this warpgroup's key dims (tot is free here)
+                if (C::SPLIT) rsum += __shfl_xor_sync(0xffffffffu, rsum, 16);
+                if (C::SPLIT ? lane < 16 : lane >= 16) tot[wg * TR + t] = rsum;
             }
         }
         fence_proxy_async_smem();
@@ -603,13 +621,7 @@ __global__ void __launch_bounds__(NT_B, 1)
             if (gr == 0) carry[dc] += T;
         } else if (GATE == 2) {
             __syncthreads();
-            for (int j = 0; j < 8; ++j) {
-                const int r = warp * 8 + j;
-                float acc = 0.f;
-                for (int dd = lane; dd < DKB; dd += 32) acc += sg[gsw(r, dd)];
-                for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-                if (lane == 0) rows[r] = acc;
-            }
+            if (tid < TR) rows[tid] = tot[tid] + tot[TR + tid];
             __syncthreads();
             if (warp == 0) {  // exclusive scan over 64 rows, two per lane
                 const float a0 = rows[2 * lane], a1 = rows[2 * lane + 1];
@@ -846,23 +858,33 @@ __global__ void __launch_bounds__(NT_B, 1)
             tma_load_3d(st + C::QB + C::KB + C::GB + vb * BLK, &tv, vb * 64, t0, bh, &bar_full[s]);
             tma_load_3d(st + C::QB + C::KB + C::GB + C::VB + vb * BLK, &tdo, vb * 64, t0, bh, &bar_full[s]);
         }
-        // the tile that takes this stage next is brought into L2 now
-        if (i + C::NS < ntiles) {
-            const int tp = tile_at(i + C::NS) * TR;
-            for (int cb = 0; cb < DK / 64; ++cb) {
-                tma_prefetch_l2_3d(&tq, d0 + cb * 64, tp, bh);
-                tma_prefetch_l2_3d(&tk, d0 + cb * 64, tp, bh);
-            }
-            if (GATE == 1)
-                for (int gb = 0; gb < DK / 32; ++gb) tma_prefetch_l2_3d(&tg, d0 + 32 * gb, tp, bh);
-            for (int vb = 0; vb < DV / 64; ++vb) {
-                tma_prefetch_l2_3d(&tv, vb * 64, tp, bh);
-                tma_prefetch_l2_3d(&tdo, vb * 64, tp, bh);
-            }
+    };
+    // the i-th tile of the walk into L2, ahead of its loads
+    auto issue_prefetch = [&](int i) {
+        const int tp = tile_at(i) * TR;
+        for (int cb = 0; cb < DK / 64; ++cb) {
+            tma_prefetch_l2_3d(&tq, d0 + cb * 64, tp, bh);
+            tma_prefetch_l2_3d(&tk, d0 + cb * 64, tp, bh);
+        }
+        if (GATE == 1)
+            for (int gb = 0; gb < DK / 32; ++gb) tma_prefetch_l2_3d(&tg, d0 + 32 * gb, tp, bh);
+        for (int vb = 0; vb < DV / 64; ++vb) {
+            tma_prefetch_l2_3d(&tv, vb * 64, tp, bh);
+            tma_prefetch_l2_3d(&tdo, vb * 64, tp, bh);
         }
     };
-    if (tid == 0)
+    if (tid == 0) {
         for (int i = 0; i < C::NS && i < ntiles; ++i) issue_loads(i, i);
+        for (int i = C::NS; i < 2 * C::NS && i < ntiles; ++i) issue_prefetch(i);
+    }
+    // input and per-head gates of the next tile, loaded a tile ahead into registers
+    float nig = 1.f, ngh = 0.f;
+    auto fetch_gates = [&](int i) {
+        const int t = tile_at(i) * TR + tid;
+        if (A.ig) nig = t < P.L ? A.ig[rowbase + t] : 1.f;
+        if (GATE == 2) ngh = t < P.L ? A.gh[rowbase + t] : 0.f;
+    };
+    if (tid < TR) fetch_gates(0);
 
     int err = 0, n_mma = 0;
     for (int i = 0; i < ntiles; ++i) {
@@ -875,9 +897,9 @@ __global__ void __launch_bounds__(NT_B, 1)
         uint8_t* so = sv + C::VB;
         const int t0 = tile_at(i) * TR;
         if (tid < TR) {
-            const int t = t0 + tid;
-            igs[tid] = (A.ig && t < P.L) ? A.ig[rowbase + t] : 1.f;
-            if (GATE == 2) ghs[tid] = (t < P.L) ? A.gh[rowbase + t] : 0.f;
+            igs[tid] = nig;
+            if (GATE == 2) ghs[tid] = ngh;
+            if (i + 1 < ntiles) fetch_gates(i + 1);
         }
         if (!block_wait(&bar_full[s], (i / C::NS) & 1)) { err = 1; break; }
 
@@ -1047,10 +1069,18 @@ __global__ void __launch_bounds__(NT_B, 1)
         constexpr int NGR = NT_B / DK, RPR = TR / NGR;
         const int dc = tid % DK, gr = tid / DK;
         float* dgp = A.dg + (rowbase + t0 + gr * RPR) * P.Dk + d0 + dc;
-        float pre[GATE == 1 ? RPR : 1];
+        float pre[GATE == 1 ? RPR : 2];
         if (GATE == 1)
 #pragma unroll
             for (int rr = 0; rr < RPR; ++rr) pre[rr] = (t0 + gr * RPR + rr < P.L) ? dgp[(long)rr * P.Dk] : 0.f;
+        if (GATE == 2 && kb == 0 && warp == 0) {   // rows 2 lane, 2 lane + 1: both key blocks' prefixes
+            const long bhl = (long)P.B * P.H * P.L;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int ta = t0 + 2 * lane + u;
+                pre[u] = ta < P.L ? A.pre[rowbase + ta] + (KS == 2 ? A.pre[bhl + rowbase + ta] : 0.f) : 0.f;
+            }
+        }
         if (!block_wait(bar_mma2, i & 1)) { err = 1; break; }
         tc_fence_after();
         // every product that reads G~ is done: the other CTA may write its dv partial there
@@ -1100,7 +1130,7 @@ __global__ void __launch_bounds__(NT_B, 1)
                     }
                     store8_bf16(sq, sw128_off(srw, c, BLK), f);
                     store8_bf16(sq, sw128_off(srw, c + 8, BLK), f + 8);
-                    if (GATE != 0)
+                    if (GATE == 1)
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4)
                             *reinterpret_cast<float4*>(sg + gsw(srw, c + 4 * q4)) =
@@ -1129,16 +1159,26 @@ __global__ void __launch_bounds__(NT_B, 1)
                 if (!block_wait_cluster(bar_free, i & 1)) { err = 1; break; }
                 const bool own = (lane >> 4) == kb;
                 const uint32_t peer_g = mapa_shared(sG, kb ^ 1);
-                for (int ct = wg * VCW; ct < (wg + 1) * VCW; ct += 16) {
+                // one pass over the dv accumulator: the sending lanes store theirs to the other
+                // CTA, the owning lanes keep theirs in registers until the other part arrives
+                constexpr int NIT = VCW / 16;
+                float keep[NIT][16];
+#pragma unroll
+                for (int it = 0; it < NIT; ++it) {
+                    const int ct = wg * VCW + 16 * it;
                     uint32_t r[16];
                     tmem_ld16(tlane + C::COL_V + ct, r);
                     tmem_wait_ld();
-                    if (!own)
+                    if (!own) {
 #pragma unroll
                         for (int u = 0; u < 4; ++u)
                             st_cluster_v4(peer_g + (uint32_t)((((ct >> 2) + u) * TR + srw) * 16),
                                           __uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
                                           __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) keep[it][j] = __uint_as_float(r[j]);
+                    }
                 }
                 if (!own) {
                     if (kb == 1 && wg == 0) st_cluster_f32(peer_g + kXRows + 4 * srw, sdi[srw] + sdi[TR + srw]);
@@ -1146,19 +1186,18 @@ __global__ void __launch_bounds__(NT_B, 1)
                 }
                 if (!block_wait_cluster(bar_recv, i & 1)) { err = 1; break; }
                 const float* rx = reinterpret_cast<const float*>(sG);
-                for (int ct = wg * VCW; ct < (wg + 1) * VCW; ct += 16) {
-                    uint32_t r[16];
-                    tmem_ld16(tlane + C::COL_V + ct, r);
-                    tmem_wait_ld();
-                    if (own) {
+                if (own) {
+#pragma unroll
+                    for (int it = 0; it < NIT; ++it) {
+                        const int ct = wg * VCW + 16 * it;
                         float f[16];
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
                             const float4 x = *reinterpret_cast<const float4*>(rx + (((ct >> 2) + u) * TR + srw) * 4);
-                            f[4 * u] = __uint_as_float(r[4 * u]) + x.x;
-                            f[4 * u + 1] = __uint_as_float(r[4 * u + 1]) + x.y;
-                            f[4 * u + 2] = __uint_as_float(r[4 * u + 2]) + x.z;
-                            f[4 * u + 3] = __uint_as_float(r[4 * u + 3]) + x.w;
+                            f[4 * u] = keep[it][4 * u] + x.x;
+                            f[4 * u + 1] = keep[it][4 * u + 1] + x.y;
+                            f[4 * u + 2] = keep[it][4 * u + 2] + x.z;
+                            f[4 * u + 3] = keep[it][4 * u + 3] + x.w;
                         }
                         store8_bf16(sv, sw128_off(srw, ct, BLK), f);
                         store8_bf16(sv, sw128_off(srw, ct + 8, BLK), f + 8);
@@ -1204,14 +1243,9 @@ __global__ void __launch_bounds__(NT_B, 1)
             __syncthreads();
             if (gr == 0) rk[dc] += T;
         } else if (GATE == 2 && kb == 0) {
-            // (key block 0 forms the per-head dg of both blocks)
-            for (int j = 0; j < 8; ++j) {
-                const int r = warp * 8 + j;
-                float acc = 0.f;
-                for (int dd = lane; dd < DK; dd += 32) acc += sg[gsw(r, dd)];
-                for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-                if (lane == 0) rows[r] = acc + (KS == 2 ? prow[r] : 0.f);
-            }
+            // key block 0 forms the per-head dg of both blocks; a row's sum of k' dk' over the
+            // key dims is the epilogue's per-row sum (sdi, and prow from key block 1)
+            if (tid < TR) rows[tid] = sdi[tid] + sdi[TR + tid] + (KS == 2 ? prow[tid] : 0.f);
             __syncthreads();
             if (warp == 0) {  // reverse inclusive scan over 64 rows, two per lane
                 const float a0 = rows[2 * lane], a1 = rows[2 * lane + 1];
@@ -1224,11 +1258,9 @@ __global__ void __launch_bounds__(NT_B, 1)
                 const float base = rk[0], cc = czs[0];
                 const float s0 = base + v, s1 = base + v - a0;
                 const int ta = t0 + 2 * lane;
-                // the dq kernel's exclusive prefixes of q*dq, one row per key block
-                const long bhl = (long)P.B * P.H * P.L;
-                auto prefix = [&](int t) { return A.pre[rowbase + t] + (KS == 2 ? A.pre[bhl + rowbase + t] : 0.f); };
-                if (ta < P.L) A.dg[rowbase + ta] = cc - prefix(ta) - s0;
-                if (ta + 1 < P.L) A.dg[rowbase + ta + 1] = cc - prefix(ta + 1) - s1;
+                // pre: the dq kernel's exclusive prefixes of q*dq (both key blocks), fetched above
+                if (ta < P.L) A.dg[rowbase + ta] = cc - pre[0] - s0;
+                if (ta + 1 < P.L) A.dg[rowbase + ta + 1] = cc - pre[1] - s1;
                 const float total = __shfl_sync(0xffffffffu, v, 0);
                 __syncwarp();
                 if (lane == 0) rk[0] = base + total;
@@ -1236,7 +1268,12 @@ __global__ void __launch_bounds__(NT_B, 1)
         }
         __syncthreads();
         if (tid == 0) bulk_wait_read<0>();   // the dk / dv stores have read the q and v slots
-        if (tid == 0 && i + C::NS < ntiles) issue_loads(i + C::NS, s);
+        // the next tile's loads, then the tile after it into L2 (issued from the same thread
+        // after the loads: an earlier prefetch, or one from another warp, measured slower)
+        if (tid == 0 && i + C::NS < ntiles) {
+            issue_loads(i + C::NS, s);
+            if (i + 2 * C::NS < ntiles) issue_prefetch(i + 2 * C::NS);
+        }
     }
 
     if (err) {

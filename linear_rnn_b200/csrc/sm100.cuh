@@ -44,28 +44,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return done != 0;
 }
-// try_wait with a suspend-time hint: a thread whose phase has not completed is suspended
-// (it issues nothing) until the phase completes or about `hint_ns` nanoseconds pass, so
-// waiting warps leave the issue slots to the warps doing work.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred P1;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2, %3;\n\t"
-        "selp.b32 %0, 1, 0, P1;\n\t}\n"
-        : "=r"(done)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-        : "memory");
-    return done != 0;
-}
-constexpr uint32_t kWaitHintNs = 10000;         // per poll
-constexpr uint32_t kWaitPolls = 1u << 20;       // bound: about ten seconds at most
+// Bound on the polls of one wait. A try_wait whose phase has not completed suspends the
+// thread for at most a system-dependent time limit and then returns false, so a wait that
+// never completes gives up after this many polls. (A 10-microsecond suspend-time hint on each
+// poll measured 1-2 % slower end to end.)
+constexpr uint32_t kWaitPolls = 1u << 20;
 
 // Bounded wait: returns false after `limit` polls without completion (the caller then
 // records a timeout and winds down).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = kWaitPolls) {
     for (uint32_t i = 0; i < limit; ++i)
-        if (mbar_try_wait_sleep(bar, parity, kWaitHintNs)) return true;
+        if (mbar_try_wait(bar, parity)) return true;
     return false;
 }
 
@@ -74,7 +63,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
 __device__ __forceinline__ bool mbar_wait_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                                 uint32_t limit = kWaitPolls) {
     for (uint32_t i = 0; i < limit; ++i) {
-        if (mbar_try_wait_sleep(bar, parity, kWaitHintNs)) return true;
+        if (mbar_try_wait(bar, parity)) return true;
         if ((i & 7u) == 7u && *abort_flag) return false;
     }
     *abort_flag = 1;
@@ -111,10 +100,10 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred P1;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 P1, [%1], %2, %3;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 P1, [%1], %2;\n\t"
             "selp.b32 %0, 1, 0, P1;\n\t}\n"
             : "=r"(done)
-            : "r"(smem_u32(bar)), "r"(parity), "r"(kWaitHintNs)
+            : "r"(smem_u32(bar)), "r"(parity)
             : "memory");
         if (done) return true;
     }
