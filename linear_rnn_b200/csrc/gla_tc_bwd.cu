@@ -42,6 +42,8 @@ using namespace sm100;
 constexpr int NT_B = 256;  // 8 warps: two warpgroups; thread 0 also issues TMA and MMA
 
 struct BwdArgs {
+    const __nv_bfloat16 *q, *k, *v, *dO;   // inputs (L2 prefetches of whole tile rows)
+    const float* g;       // per-key log-gate [BH*L*Dk] (L2 prefetch) or null
     const float* gh;      // per-head log-gate [BH*L]
     const float* ig;      // input gate [BH*L] or null
     const float* sinit;   // initial state per (bh, segment) [BH, nseg, Dk, Dv] or null (then h0 / 0)
@@ -69,10 +71,36 @@ __device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity) {
     const bool ok = mbar_wait(bar, parity);
     return __syncthreads_and(ok) != 0;
 }
+__device__ __forceinline__ float4 f4_add(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
+__device__ __forceinline__ float4 f4_zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+// four consecutive key dims d..d+3 (d a multiple of 4) of row r of a swizzled fp32 tile (gsw)
+__device__ __forceinline__ float4 gsw_ld4(const float* sg, int r, int d) {
+    return *reinterpret_cast<const float4*>(sg + gsw(r, d));
+}
+
 // The same for a barrier that the other CTA of the cluster arrives on.
 __device__ __forceinline__ bool block_wait_cluster(uint64_t* bar, uint32_t parity) {
     const bool ok = mbar_wait_cluster(bar, parity);
     return __syncthreads_and(ok) != 0;
+}
+
+// Tile rows [t, t + 64) (clipped at L) of the inputs of CTA (bh, key block kb of nkb) into L2,
+// one contiguous bulk prefetch per tensor (a tile's rows are contiguous in the BHLD layout);
+// the first key block fetches q, k, g, the last v and dO.
+__device__ __forceinline__ void prefetch_tile_rows(const BwdArgs& A, const Dims& P, long rowbase, int t, int kb,
+                                                   int nkb, bool with_q) {
+    if (t >= P.L) return;
+    const long r0 = rowbase + t;
+    const uint32_t rows = (uint32_t)min(TR, P.L - t);
+    if (kb == 0) {
+        if (with_q) prefetch_l2_bulk(A.q + r0 * P.Dk, rows * P.Dk * 2);
+        prefetch_l2_bulk(A.k + r0 * P.Dk, rows * P.Dk * 2);
+        if (A.g) prefetch_l2_bulk(A.g + r0 * P.Dk, rows * P.Dk * 4);
+    }
+    if (kb == nkb - 1) {
+        prefetch_l2_bulk(A.v + r0 * P.Dv, rows * P.Dv * 2);
+        prefetch_l2_bulk(A.dO + r0 * P.Dv, rows * P.Dv * 2);
+    }
 }
 
 __device__ __forceinline__ void store16_bf16_global(__nv_bfloat16* dst, const float* v) {
@@ -358,17 +386,7 @@ __global__ void __launch_bounds__(NT_B, 1)
     };
     // tile i into L2, ahead of its loads (issued by another warp than the loads and products)
     auto issue_prefetch = [&](int i) {
-        const int tp = (tile0 + i) * TR;
-        for (int cb = 0; cb < DKB / 64; ++cb) {
-            if (GATE != 0) tma_prefetch_l2_3d(&tq, d0 + cb * 64, tp, bh);
-            tma_prefetch_l2_3d(&tk, d0 + cb * 64, tp, bh);
-        }
-        if (GATE == 1)
-            for (int gb = 0; gb < DKB / 32; ++gb) tma_prefetch_l2_3d(&tg, d0 + 32 * gb, tp, bh);
-        for (int vb = 0; vb < DV / 64; ++vb) {
-            tma_prefetch_l2_3d(&tv, vb * 64, tp, bh);
-            tma_prefetch_l2_3d(&tdo, vb * 64, tp, bh);
-        }
+        prefetch_tile_rows(A, P, rowbase, (tile0 + i) * TR, kb, P.Dk / DKB, GATE != 0);
     };
     auto issue_vo = [&](int i, int s) {
         uint8_t* st = sm + s * C::STAGE;
@@ -481,21 +499,23 @@ __global__ void __launch_bounds__(NT_B, 1)
         }
         {
             const float eg = GATE == 0 ? 1.f : gam[GATE == 1 ? srow : 0];
-            for (int c = wg * C::HC; c < (wg + 1) * C::HC; c += 16) {
-                uint32_t r[16];
-                float f[16];
-                tmem_ld16(tlane + c, r);
+            const uint64_t eg2 = f2(eg, eg);
+            for (int c = wg * C::HC; c < (wg + 1) * C::HC; c += 32) {
+                uint32_t r[32];
+                float f[32];
+                tmem_ld32(tlane + c, r);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    f[j] = eg * __uint_as_float(r[j]);
+                for (int j = 0; j < 32; j += 2) {
+                    const uint64_t x = f2_mul(f2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])), eg2);
+                    asm("mov.b64 {%0, %1}, %2;" : "=f"(f[j]), "=f"(f[j + 1]) : "l"(x));
                     r[j] = __float_as_uint(f[j]);
+                    r[j + 1] = __float_as_uint(f[j + 1]);
                 }
-                tmem_st16(tlane + c, r);
-                if (srow_ok) {
-                    store8_bf16(sS, sw128_off(srow, c, DKB * 128), f);
-                    store8_bf16(sS, sw128_off(srow, c + 8, DKB * 128), f + 8);
-                }
+                tmem_st32(tlane + c, r);
+                if (srow_ok)
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8) store8_bf16(sS, sw128_off(srow, c + j, DKB * 128), f + j);
             }
             tmem_wait_st();
         }
@@ -596,29 +616,32 @@ __global__ void __launch_bounds__(NT_B, 1)
         }
         // ---- in-segment exclusive prefix of q*dq (fp32) into the dg buffer
         if (GATE == 1) {
-            // thread = (key dim dc, group of RPR rows): local sums, exchange, then the prefix walk
-            constexpr int NGR = NT_B / DKB, RPR = TR / NGR;
-            const int dc = tid % DKB, gr = tid / DKB;
-            float loc = 0.f;
-#pragma unroll 8
-            for (int rr = 0; rr < RPR; ++rr) loc += sg[gsw(gr * RPR + rr, dc)];
-            tot[gr * DKB + dc] = loc;
+            // thread = (key dims dc..dc+3, group of RPR rows): local sums, exchange, then the
+            // prefix walk with 16-byte stores
+            constexpr int NC4 = DKB / 4, NGR = NT_B / NC4, RPR = TR / NGR;
+            const int c4 = tid % NC4, gr = tid / NC4, dc = 4 * c4;
+            float4* tot4 = reinterpret_cast<float4*>(tot);
+            float4* carry4 = reinterpret_cast<float4*>(carry);
+            float4 loc = f4_zero();
+#pragma unroll
+            for (int rr = 0; rr < RPR; ++rr) loc = f4_add(loc, gsw_ld4(sg, gr * RPR + rr, dc));
+            tot4[gr * NC4 + c4] = loc;
             __syncthreads();
-            float px = carry[dc], T = 0.f;
+            float4 px = carry4[c4], T = f4_zero();
 #pragma unroll
             for (int g2 = 0; g2 < NGR; ++g2) {
-                const float v = tot[g2 * DKB + dc];
-                if (g2 < gr) px += v;
-                T += v;
+                const float4 v = tot4[g2 * NC4 + c4];
+                if (g2 < gr) px = f4_add(px, v);
+                T = f4_add(T, v);
             }
-            float* dgp = A.dg + (rowbase + t0 + gr * RPR) * P.Dk + d0 + dc;
-#pragma unroll 8
+            float4* dgp = reinterpret_cast<float4*>(A.dg + (rowbase + t0 + gr * RPR) * P.Dk + d0 + dc);
+#pragma unroll
             for (int rr = 0; rr < RPR; ++rr) {
-                if (t0 + gr * RPR + rr < P.L) dgp[(long)rr * P.Dk] = px;
-                px += sg[gsw(gr * RPR + rr, dc)];
+                if (t0 + gr * RPR + rr < P.L) dgp[(long)rr * (P.Dk / 4)] = px;
+                px = f4_add(px, gsw_ld4(sg, gr * RPR + rr, dc));
             }
             __syncthreads();
-            if (gr == 0) carry[dc] += T;
+            if (gr == 0) carry4[c4] = f4_add(carry4[c4], T);
         } else if (GATE == 2) {
             __syncthreads();
             if (tid < TR) rows[tid] = tot[tid] + tot[TR + tid];
@@ -860,19 +883,7 @@ __global__ void __launch_bounds__(NT_B, 1)
         }
     };
     // the i-th tile of the walk into L2, ahead of its loads
-    auto issue_prefetch = [&](int i) {
-        const int tp = tile_at(i) * TR;
-        for (int cb = 0; cb < DK / 64; ++cb) {
-            tma_prefetch_l2_3d(&tq, d0 + cb * 64, tp, bh);
-            tma_prefetch_l2_3d(&tk, d0 + cb * 64, tp, bh);
-        }
-        if (GATE == 1)
-            for (int gb = 0; gb < DK / 32; ++gb) tma_prefetch_l2_3d(&tg, d0 + 32 * gb, tp, bh);
-        for (int vb = 0; vb < DV / 64; ++vb) {
-            tma_prefetch_l2_3d(&tv, vb * 64, tp, bh);
-            tma_prefetch_l2_3d(&tdo, vb * 64, tp, bh);
-        }
-    };
+    auto issue_prefetch = [&](int i) { prefetch_tile_rows(A, P, rowbase, tile_at(i) * TR, kb, KS, true); };
     if (tid == 0) {
         for (int i = 0; i < C::NS && i < ntiles; ++i) issue_loads(i, i);
         for (int i = C::NS; i < 2 * C::NS && i < ntiles; ++i) issue_prefetch(i);
@@ -933,21 +944,23 @@ __global__ void __launch_bounds__(NT_B, 1)
         // ---- G~ = e^Gamma G in TMEM; bf16 copy (runs while group 1 is in flight)
         {
             const float eg = GATE == 0 ? 1.f : gam[GATE == 1 ? srow : 0];
-            for (int c = wg * C::HC; c < (wg + 1) * C::HC; c += 16) {
-                uint32_t r[16];
-                float f[16];
-                tmem_ld16(tlane + c, r);
+            const uint64_t eg2 = f2(eg, eg);
+            for (int c = wg * C::HC; c < (wg + 1) * C::HC; c += 32) {
+                uint32_t r[32];
+                float f[32];
+                tmem_ld32(tlane + c, r);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    f[j] = eg * __uint_as_float(r[j]);
+                for (int j = 0; j < 32; j += 2) {
+                    const uint64_t x = f2_mul(f2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])), eg2);
+                    asm("mov.b64 {%0, %1}, %2;" : "=f"(f[j]), "=f"(f[j + 1]) : "l"(x));
                     r[j] = __float_as_uint(f[j]);
+                    r[j + 1] = __float_as_uint(f[j + 1]);
                 }
-                tmem_st16(tlane + c, r);
-                if (srow_ok) {
-                    store8_bf16(sG, sw128_off(srow, c, DK * 128), f);
-                    store8_bf16(sG, sw128_off(srow, c + 8, DK * 128), f + 8);
-                }
+                tmem_st32(tlane + c, r);
+                if (srow_ok)
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8) store8_bf16(sG, sw128_off(srow, c + j, DK * 128), f + j);
             }
             tmem_wait_st();
         }
@@ -1065,20 +1078,22 @@ __global__ void __launch_bounds__(NT_B, 1)
             if (leader) mma_commit(bar_mma2);
             __syncwarp();
         }
-        // the dq kernel's exclusive prefixes of this tile's rows, in flight during the epilogue
-        constexpr int NGR = NT_B / DK, RPR = TR / NGR;
-        const int dc = tid % DK, gr = tid / DK;
-        float* dgp = A.dg + (rowbase + t0 + gr * RPR) * P.Dk + d0 + dc;
-        float pre[GATE == 1 ? RPR : 2];
+        // the dq kernel's exclusive prefixes of this tile's rows, in flight during the epilogue;
+        // per-key gates: thread = (key dims dc..dc+3, group of RPR rows)
+        constexpr int NC4 = DK / 4, NGR = NT_B / NC4, RPR = TR / NGR;
+        const int c4 = tid % NC4, gr = tid / NC4, dc = 4 * c4;
+        float4* dgp = reinterpret_cast<float4*>(A.dg + (rowbase + t0 + gr * RPR) * P.Dk + d0 + dc);
+        float4 pre[GATE == 1 ? RPR : 1];
+        float pre2[2];
         if (GATE == 1)
 #pragma unroll
-            for (int rr = 0; rr < RPR; ++rr) pre[rr] = (t0 + gr * RPR + rr < P.L) ? dgp[(long)rr * P.Dk] : 0.f;
+            for (int rr = 0; rr < RPR; ++rr) pre[rr] = (t0 + gr * RPR + rr < P.L) ? dgp[(long)rr * (P.Dk / 4)] : f4_zero();
         if (GATE == 2 && kb == 0 && warp == 0) {   // rows 2 lane, 2 lane + 1: both key blocks' prefixes
             const long bhl = (long)P.B * P.H * P.L;
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const int ta = t0 + 2 * lane + u;
-                pre[u] = ta < P.L ? A.pre[rowbase + ta] + (KS == 2 ? A.pre[bhl + rowbase + ta] : 0.f) : 0.f;
+                pre2[u] = ta < P.L ? A.pre[rowbase + ta] + (KS == 2 ? A.pre[bhl + rowbase + ta] : 0.f) : 0.f;
             }
         }
         if (!block_wait(bar_mma2, i & 1)) { err = 1; break; }
@@ -1220,28 +1235,32 @@ __global__ void __launch_bounds__(NT_B, 1)
             A.di[rowbase + t0 + tid] = (sdi[tid] + sdi[TR + tid] + (KS == 2 ? prow[tid] : 0.f)) / igs[tid];
         // ---- dg = (in-segment q*dq total - exclusive prefix) - reverse sum of k*dk + carry
         if (GATE == 1) {
-            // thread = (key dim dc, group of RPR rows; the prefixes were fetched above): local
-            // sums, exchange, then the reverse walk
-            float loc = 0.f;
-#pragma unroll 8
-            for (int rr = 0; rr < RPR; ++rr) loc += sg[gsw(gr * RPR + rr, dc)];
-            tot[gr * DK + dc] = loc;
+            // thread = (key dims dc..dc+3, group of RPR rows; the prefixes were fetched above):
+            // local sums, exchange, then the reverse walk with 16-byte stores
+            float4* tot4 = reinterpret_cast<float4*>(tot);
+            float4* rk4 = reinterpret_cast<float4*>(rk);
+            float4 loc = f4_zero();
+#pragma unroll
+            for (int rr = 0; rr < RPR; ++rr) loc = f4_add(loc, gsw_ld4(sg, gr * RPR + rr, dc));
+            tot4[gr * NC4 + c4] = loc;
             __syncthreads();
-            float sx = rk[dc], T = 0.f;
+            float4 sx = rk4[c4], T = f4_zero();
 #pragma unroll
             for (int g2 = 0; g2 < NGR; ++g2) {
-                const float v = tot[g2 * DK + dc];
-                if (g2 > gr) sx += v;
-                T += v;
+                const float4 v = tot4[g2 * NC4 + c4];
+                if (g2 > gr) sx = f4_add(sx, v);
+                T = f4_add(T, v);
             }
-            const float cx = cz[dc];
+            const float4 cx = reinterpret_cast<const float4*>(cz)[c4];
 #pragma unroll
             for (int rr = RPR - 1; rr >= 0; --rr) {
-                sx += sg[gsw(gr * RPR + rr, dc)];
-                if (t0 + gr * RPR + rr < P.L) dgp[(long)rr * P.Dk] = cx - pre[rr] - sx;
+                sx = f4_add(sx, gsw_ld4(sg, gr * RPR + rr, dc));
+                if (t0 + gr * RPR + rr < P.L)
+                    dgp[(long)rr * (P.Dk / 4)] = make_float4(cx.x - pre[rr].x - sx.x, cx.y - pre[rr].y - sx.y,
+                                                             cx.z - pre[rr].z - sx.z, cx.w - pre[rr].w - sx.w);
             }
             __syncthreads();
-            if (gr == 0) rk[dc] += T;
+            if (gr == 0) rk4[c4] = f4_add(rk4[c4], T);
         } else if (GATE == 2 && kb == 0) {
             // key block 0 forms the per-head dg of both blocks; a row's sum of k' dk' over the
             // key dims is the epilogue's per-row sum (sdi, and prow from key block 1)
@@ -1259,8 +1278,8 @@ __global__ void __launch_bounds__(NT_B, 1)
                 const float s0 = base + v, s1 = base + v - a0;
                 const int ta = t0 + 2 * lane;
                 // pre: the dq kernel's exclusive prefixes of q*dq (both key blocks), fetched above
-                if (ta < P.L) A.dg[rowbase + ta] = cc - pre[0] - s0;
-                if (ta + 1 < P.L) A.dg[rowbase + ta + 1] = cc - pre[1] - s1;
+                if (ta < P.L) A.dg[rowbase + ta] = cc - pre2[0] - s0;
+                if (ta + 1 < P.L) A.dg[rowbase + ta + 1] = cc - pre2[1] - s1;
                 const float total = __shfl_sync(0xffffffffu, v, 0);
                 __syncwarp();
                 if (lane == 0) rk[0] = base + total;
@@ -1475,6 +1494,11 @@ static cudaError_t run_bwd(const Dims& P, const void* q, const void* k, const vo
         if (e != cudaSuccess) return e;
     }
     BwdArgs a{};
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.k = static_cast<const __nv_bfloat16*>(k);
+    a.v = static_cast<const __nv_bfloat16*>(v);
+    a.dO = static_cast<const __nv_bfloat16*>(dO);
+    a.g = GATE == 1 ? g : nullptr;
     a.gh = GATE == 2 ? g : nullptr;
     a.ig = ig;
     a.sinit = sinit;
