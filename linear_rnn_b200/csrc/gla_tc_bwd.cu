@@ -622,9 +622,13 @@ __global__ void __launch_bounds__(NT_B, 1)
             const int c4 = tid % NC4, gr = tid / NC4, dc = 4 * c4;
             float4* tot4 = reinterpret_cast<float4*>(tot);
             float4* carry4 = reinterpret_cast<float4*>(carry);
+            float4 x[RPR];   // the thread's rows of q*dq, read once
             float4 loc = f4_zero();
 #pragma unroll
-            for (int rr = 0; rr < RPR; ++rr) loc = f4_add(loc, gsw_ld4(sg, gr * RPR + rr, dc));
+            for (int rr = 0; rr < RPR; ++rr) {
+                x[rr] = gsw_ld4(sg, gr * RPR + rr, dc);
+                loc = f4_add(loc, x[rr]);
+            }
             tot4[gr * NC4 + c4] = loc;
             __syncthreads();
             float4 px = carry4[c4], T = f4_zero();
@@ -638,7 +642,7 @@ __global__ void __launch_bounds__(NT_B, 1)
 #pragma unroll
             for (int rr = 0; rr < RPR; ++rr) {
                 if (t0 + gr * RPR + rr < P.L) dgp[(long)rr * (P.Dk / 4)] = px;
-                px = f4_add(px, gsw_ld4(sg, gr * RPR + rr, dc));
+                px = f4_add(px, x[rr]);
             }
             __syncthreads();
             if (gr == 0) carry4[c4] = f4_add(carry4[c4], T);
@@ -912,6 +916,15 @@ __global__ void __launch_bounds__(NT_B, 1)
             if (GATE == 2) ghs[tid] = ngh;
             if (i + 1 < ntiles) fetch_gates(i + 1);
         }
+        // per-key gates: the dq kernel's exclusive prefixes of q*dq for this tile, fetched now so
+        // that the loads have the whole tile to land; thread = (key dims dc..dc+3, RPR rows)
+        constexpr int NC4 = DK / 4, NGR = NT_B / NC4, RPR = TR / NGR;
+        const int c4 = tid % NC4, gr = tid / NC4, dc = 4 * c4;
+        float4* dgp = reinterpret_cast<float4*>(A.dg + (rowbase + t0 + gr * RPR) * P.Dk + d0 + dc);
+        float4 pre[GATE == 1 ? RPR : 1];
+        if (GATE == 1)
+#pragma unroll
+            for (int rr = 0; rr < RPR; ++rr) pre[rr] = (t0 + gr * RPR + rr < P.L) ? dgp[(long)rr * (P.Dk / 4)] : f4_zero();
         if (!block_wait(&bar_full[s], (i / C::NS) & 1)) { err = 1; break; }
 
         // ---- transform: q~ = scale q e^b, k~ = i k e^-b (in place); e^-b kept in place of g
@@ -1078,16 +1091,9 @@ __global__ void __launch_bounds__(NT_B, 1)
             if (leader) mma_commit(bar_mma2);
             __syncwarp();
         }
-        // the dq kernel's exclusive prefixes of this tile's rows, in flight during the epilogue;
-        // per-key gates: thread = (key dims dc..dc+3, group of RPR rows)
-        constexpr int NC4 = DK / 4, NGR = NT_B / NC4, RPR = TR / NGR;
-        const int c4 = tid % NC4, gr = tid / NC4, dc = 4 * c4;
-        float4* dgp = reinterpret_cast<float4*>(A.dg + (rowbase + t0 + gr * RPR) * P.Dk + d0 + dc);
-        float4 pre[GATE == 1 ? RPR : 1];
+        // per-head gates: the dq kernel's exclusive prefixes of this tile's rows, in flight during
+        // the epilogue (per-key gates fetched theirs at the top of the tile)
         float pre2[2];
-        if (GATE == 1)
-#pragma unroll
-            for (int rr = 0; rr < RPR; ++rr) pre[rr] = (t0 + gr * RPR + rr < P.L) ? dgp[(long)rr * (P.Dk / 4)] : f4_zero();
         if (GATE == 2 && kb == 0 && warp == 0) {   // rows 2 lane, 2 lane + 1: both key blocks' prefixes
             const long bhl = (long)P.B * P.H * P.L;
 #pragma unroll
@@ -1239,9 +1245,13 @@ __global__ void __launch_bounds__(NT_B, 1)
             // local sums, exchange, then the reverse walk with 16-byte stores
             float4* tot4 = reinterpret_cast<float4*>(tot);
             float4* rk4 = reinterpret_cast<float4*>(rk);
+            float4 x[RPR];   // the thread's rows of k*dk, read once
             float4 loc = f4_zero();
 #pragma unroll
-            for (int rr = 0; rr < RPR; ++rr) loc = f4_add(loc, gsw_ld4(sg, gr * RPR + rr, dc));
+            for (int rr = 0; rr < RPR; ++rr) {
+                x[rr] = gsw_ld4(sg, gr * RPR + rr, dc);
+                loc = f4_add(loc, x[rr]);
+            }
             tot4[gr * NC4 + c4] = loc;
             __syncthreads();
             float4 sx = rk4[c4], T = f4_zero();
@@ -1254,7 +1264,7 @@ __global__ void __launch_bounds__(NT_B, 1)
             const float4 cx = reinterpret_cast<const float4*>(cz)[c4];
 #pragma unroll
             for (int rr = RPR - 1; rr >= 0; --rr) {
-                sx = f4_add(sx, gsw_ld4(sg, gr * RPR + rr, dc));
+                sx = f4_add(sx, x[rr]);
                 if (t0 + gr * RPR + rr < P.L)
                     dgp[(long)rr * (P.Dk / 4)] = make_float4(cx.x - pre[rr].x - sx.x, cx.y - pre[rr].y - sx.y,
                                                              cx.z - pre[rr].z - sx.z, cx.w - pre[rr].w - sx.w);
