@@ -124,10 +124,75 @@ constexpr uint32_t pow2cols(uint32_t n) { return n <= 32 ? 32 : n <= 64 ? 64 : n
 // Per-head gates use the row factors rowE / rowEi (warp 0 scans the 64 gates) instead.
 // Both backward kernels use this one routine so they form bit-identical q~ and k~. The g tile
 // is in the swizzled fp32 layout (gsw).
+//
+// Per-key gates (GATE 1) run it in one pass instead: thread = key-dim pair x run of RSF rows;
+// the column cumsum of its rows stays in registers, the run totals are exchanged once, and each
+// row's k (and q) pair is scaled right away, with the products formed in the same order as
+// above ((k i) e^-b, (q scale) e^b) so that both kernels, and the dq kernel's q*dq, see the same
+// bf16 values.
+template <int D, bool DO_Q, bool G_SLOT_EB>
+__device__ __forceinline__ void bwd_transform_key(uint8_t* sq, uint8_t* sk, float* sg, float* tot, float* gam,
+                                                  const float* igs, float scale, int tid, int* status) {
+    constexpr int NP = D / 2, SEGF = NT_B / NP, RSF = TR / SEGF;
+    static_assert(NT_B % NP == 0 && TR % SEGF == 0 && SEGF * NP * 2 <= 2048, "fused transform mapping");
+    const int p = tid % NP, sgi = tid / NP, d0 = 2 * p;
+    float2* tot2 = reinterpret_cast<float2*>(tot);   // [SEGF][NP] run totals
+    float2 cs[RSF];
+    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < RSF; ++u) {
+        const float2 x = *reinterpret_cast<const float2*>(sg + gsw(sgi * RSF + u, d0));
+        acc.x += x.x;
+        acc.y += x.y;
+        cs[u] = acc;
+    }
+    tot2[sgi * NP + p] = acc;
+    __syncthreads();
+    float2 off = make_float2(0.f, 0.f), G = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int s2 = 0; s2 < SEGF; ++s2) {
+        const float2 t = tot2[s2 * NP + p];
+        if (s2 < sgi) {
+            off.x += t.x;
+            off.y += t.y;
+        }
+        G.x += t.x;
+        G.y += t.y;
+    }
+    if (sgi == 0) {
+        gam[d0] = __expf(G.x);
+        gam[d0 + 1] = __expf(G.y);
+        if (G.x < kMinTileLogDecay || G.y < kMinTileLogDecay) atomicOr(status, kDevStatusRange);
+    }
+#pragma unroll
+    for (int u = 0; u < RSF; ++u) {
+        const int r = sgi * RSF + u;
+        const float ex = __expf(cs[u].x + off.x), ey = __expf(cs[u].y + off.y);
+        const float dx = rcp_newton(ex), dy = rcp_newton(ey);
+        *reinterpret_cast<float2*>(sg + gsw(r, d0)) = G_SLOT_EB ? make_float2(ex, ey) : make_float2(dx, dy);
+        // byte offset of (r, d0) in a 128-byte-swizzled bf16 tile
+        const uint32_t ob = (uint32_t)(d0 >> 6) * BLK + (uint32_t)r * 128 +
+                            ((((uint32_t)((d0 & 63) >> 3)) ^ (uint32_t)(r & 7)) << 4) + (uint32_t)(d0 & 7) * 2;
+        const float iv = igs[r];
+        __nv_bfloat162* pk = reinterpret_cast<__nv_bfloat162*>(sk + ob);
+        const float2 kf = __bfloat1622float2(*pk);
+        *pk = __floats2bfloat162_rn(kf.x * iv * dx, kf.y * iv * dy);
+        if (DO_Q) {
+            __nv_bfloat162* pq = reinterpret_cast<__nv_bfloat162*>(sq + ob);
+            const float2 qf = __bfloat1622float2(*pq);
+            *pq = __floats2bfloat162_rn(qf.x * scale * ex, qf.y * scale * ey);
+        }
+    }
+}
+
 template <int D, int GATE, bool DO_Q, bool G_SLOT_EB>
 __device__ __forceinline__ void bwd_transform(uint8_t* sq, uint8_t* sk, float* sg, float* tot, float* gam,
                                               float* rowE, float* rowEi, const float* ghs, const float* igs,
                                               float scale, int tid, int* status) {
+    if constexpr (GATE == 1 && D <= 128) {
+        bwd_transform_key<D, DO_Q, G_SLOT_EB>(sq, sk, sg, tot, gam, igs, scale, tid, status);
+        return;
+    }
     constexpr int SEG = NT_B / D, RS = TR / SEG;   // step A
     constexpr int NO = D / 8, NPOS = TR * NO;       // step B
     constexpr int NB = 2;
