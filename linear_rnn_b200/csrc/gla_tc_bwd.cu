@@ -1181,6 +1181,27 @@ __global__ void __launch_bounds__(NT_B, 1)
             const bool row_ok = t0 + srw < P.L;
             float dsum = 0.f;
             constexpr int KCW = C::SPLIT ? DK / 4 : C::KC, VCW = C::SPLIT ? DV / 4 : C::HC;   // TMEM columns per warpgroup
+            // key split: dv over this key block is a partial sum. This CTA owns value dims
+            // [kb DV/2, (kb + 1) DV/2), the TMEM lane half kb; the lanes of the other half send
+            // theirs to the other CTA first (so that the transfer overlaps the dk epilogue), as
+            // fp32, 16-byte chunk j of row s at byte (64 j + s) * 16 of its G~ slot, followed
+            // (key block 1 only) by the rows' sums of k' dk'.
+            const bool own = (lane >> 4) == kb;
+            const uint32_t peer_g = KS == 2 ? mapa_shared(sG, kb ^ 1) : 0u;
+            if (KS == 2) {
+                if (!block_wait_cluster(bar_free, i & 1)) { err = 1; break; }
+                for (int ct = wg * VCW; ct < (wg + 1) * VCW; ct += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tlane + C::COL_V + ct, r);
+                    tmem_wait_ld();
+                    if (!own)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            st_cluster_v4(peer_g + (uint32_t)((((ct >> 2) + u) * TR + srw) * 16),
+                                          __uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
+                                          __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
+                }
+            }
             for (int ct = wg * KCW; ct < (wg + 1) * KCW; ct += 16) {
                 uint32_t r[16];
                 tmem_ld16(tlane + (C::SPLIT ? C::COL_K : C::COL_R) + ct, r);
@@ -1237,53 +1258,27 @@ __global__ void __launch_bounds__(NT_B, 1)
                     }
                 }
             } else {
-                // dv over this key block is a partial sum. This CTA owns value dims [kb DV/2,
-                // (kb + 1) DV/2), the TMEM lane half kb; the lanes of the other half send theirs
-                // to the other CTA as fp32, 16-byte chunk j of row s at byte (64 j + s) * 16 of
-                // its G~ slot, followed (key block 1 only) by the rows' sums of k' dk'.
                 __syncthreads();   // sdi is complete
-                if (!block_wait_cluster(bar_free, i & 1)) { err = 1; break; }
-                const bool own = (lane >> 4) == kb;
-                const uint32_t peer_g = mapa_shared(sG, kb ^ 1);
-                // one pass over the dv accumulator: the sending lanes store theirs to the other
-                // CTA, the owning lanes keep theirs in registers until the other part arrives
-                constexpr int NIT = VCW / 16;
-                float keep[NIT][16];
-#pragma unroll
-                for (int it = 0; it < NIT; ++it) {
-                    const int ct = wg * VCW + 16 * it;
-                    uint32_t r[16];
-                    tmem_ld16(tlane + C::COL_V + ct, r);
-                    tmem_wait_ld();
-                    if (!own) {
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            st_cluster_v4(peer_g + (uint32_t)((((ct >> 2) + u) * TR + srw) * 16),
-                                          __uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
-                                          __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) keep[it][j] = __uint_as_float(r[j]);
-                    }
-                }
                 if (!own) {
                     if (kb == 1 && wg == 0) st_cluster_f32(peer_g + kXRows + 4 * srw, sdi[srw] + sdi[TR + srw]);
                     mbar_arrive_remote(mapa_shared(bar_recv, kb ^ 1));
                 }
                 if (!block_wait_cluster(bar_recv, i & 1)) { err = 1; break; }
+                // the owning lanes add the other CTA's part to theirs
                 const float* rx = reinterpret_cast<const float*>(sG);
-                if (own) {
-#pragma unroll
-                    for (int it = 0; it < NIT; ++it) {
-                        const int ct = wg * VCW + 16 * it;
+                for (int ct = wg * VCW; ct < (wg + 1) * VCW; ct += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tlane + C::COL_V + ct, r);
+                    tmem_wait_ld();
+                    if (own) {
                         float f[16];
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
                             const float4 x = *reinterpret_cast<const float4*>(rx + (((ct >> 2) + u) * TR + srw) * 4);
-                            f[4 * u] = keep[it][4 * u] + x.x;
-                            f[4 * u + 1] = keep[it][4 * u + 1] + x.y;
-                            f[4 * u + 2] = keep[it][4 * u + 2] + x.z;
-                            f[4 * u + 3] = keep[it][4 * u + 3] + x.w;
+                            f[4 * u] = __uint_as_float(r[4 * u]) + x.x;
+                            f[4 * u + 1] = __uint_as_float(r[4 * u + 1]) + x.y;
+                            f[4 * u + 2] = __uint_as_float(r[4 * u + 2]) + x.z;
+                            f[4 * u + 3] = __uint_as_float(r[4 * u + 3]) + x.w;
                         }
                         store8_bf16(sv, sw128_off(srw, ct, BLK), f);
                         store8_bf16(sv, sw128_off(srw, ct + 8, BLK), f + 8);
