@@ -938,12 +938,12 @@ FwdPlan plan_fwd(const Dims& P) {
     int nseg = 1;
     if (base * 4 < (long)sms * 3 && ntiles > 1) nseg = (int)((long)sms / base);
     if (nseg < 1) nseg = 1;
-    // segments are whole chunks (the chunk is a multiple of the 64-token tile)
-    const int tiles_per_chunk = P.C / TR;
-    const int nchunks = cdiv(P.L, P.C);
-    if (nseg > nchunks) nseg = nchunks;
-    int chunks_per_seg = cdiv(nchunks, nseg);
-    pl.tiles_per_seg = chunks_per_seg * tiles_per_chunk;
+    // Segments are whole 64-token tiles, as equal as the tile count allows: the tensor-core
+    // plan carries the state through every tile, so the chunk size does not constrain them
+    // (chunk-aligned segments left c4, 1024 tiles in 18 segments, with 17 of 60 tiles and one
+    // of 4).
+    if (nseg > ntiles) nseg = ntiles;
+    pl.tiles_per_seg = cdiv(ntiles, nseg);
     pl.nseg = cdiv(ntiles, pl.tiles_per_seg);
     if (pl.nseg < 1) pl.nseg = 1;
     return pl;
