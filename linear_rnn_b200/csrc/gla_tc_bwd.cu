@@ -885,6 +885,9 @@ __global__ void __launch_bounds__(NT_B, 1)
     tc_fence_after();
     if (KS == 2) cluster_sync();   // both CTAs' barriers are initialised before either touches the other
     const uint32_t tbase = *tmem_slot;
+    // launched to overlap the reverse scan (or the dq kernel) before it: everything read from
+    // earlier kernels of the call is read after this
+    grid_dep_wait();
     const uint32_t tlane = tbase + ((uint32_t)(32 * qd) << 16);
 
     // ---- state gradient at the end of the segment into TMEM
@@ -1503,26 +1506,12 @@ static cudaError_t launch_dkdv(const Dims& P, const BwdPlan& pl, const CUtensorM
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    if (KS == 1) {
-        dim3 grid(P.B * P.H, pl.nseg);
-        GLA_LAUNCH("tc_bwd_dkdv", st, kern<<<grid, NT_B, C::SMEM, st>>>(mq, mk, mg, mv, mo, mdk, mdv, a, P));
-        return cudaGetLastError();
-    }
-    // the two key blocks of a (b*h, segment) run as one cluster of two CTAs
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(KS * P.B * P.H, pl.nseg);
-    cfg.blockDim = dim3(NT_B);
-    cfg.dynamicSmemBytes = C::SMEM;
-    cfg.stream = st;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = KS;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
+    // the two key blocks of a (b*h, segment) run as one cluster of two CTAs; the kernel may start
+    // before the kernel ahead of it (reverse scan or dq) ends, and waits for it in grid_dep_wait
     cudaError_t e = cudaSuccess;
-    GLA_LAUNCH("tc_bwd_dkdv", st, e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mg, mv, mo, mdk, mdv, a, P));
+    GLA_LAUNCH("tc_bwd_dkdv", st,
+               e = launch_ex(kern, dim3(KS * P.B * P.H, pl.nseg), dim3(NT_B), C::SMEM, st, true, KS, mq, mk, mg, mv, mo,
+                             mdk, mdv, a, P));
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -2,11 +2,43 @@
 #pragma once
 #include <cudaTypedefs.h>
 
+#include <utility>
+
 #include "gla_common.cuh"
 #include "sm100.cuh"
 
 namespace gla {
 namespace tc {
+
+// Launch with optional programmatic stream serialization (the kernel may start before the
+// previous kernel in the stream ends, and waits in grid_dep_wait for what it reads from it) and
+// an optional cluster of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                             int cluster_x, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[2];
+    unsigned n = 0;
+    if (pdl) {
+        at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    if (cluster_x > 1) {
+        at[n].id = cudaLaunchAttributeClusterDimension;
+        at[n].val.clusterDim.x = cluster_x;
+        at[n].val.clusterDim.y = 1;
+        at[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = at;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 constexpr int TR = 64;          // tokens per tile
 constexpr uint32_t BLK = 8192;  // one 64-column bf16 block of a 64-row tile (64 x 128 B)

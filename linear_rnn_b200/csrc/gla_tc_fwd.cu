@@ -186,6 +186,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     const bool srow_ok = (DK != 64) || (lane < 16);
     auto srow = [&](int h) { return (DK == 64 ? 16 * qd + (lane & 15) : 32 * qd + lane) + 128 * h; };
 
+    grid_dep_launch();   // a kernel launched after this one to overlap it may start now
     if (tid == 0) {
         for (int j = 0; j < NBARS; ++j) mbar_init(&bars[j], 1);
         *abortp = 0;
@@ -200,6 +201,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
+    grid_dep_wait();   // output pass after a segment scan: the initial states are written
 
     // ---- initial state -> TMEM (fp32) and its bf16 copy -> shared memory
     const bool s_worker = is_ep && (MODE != 0 || wg == 0);
@@ -835,6 +837,8 @@ constexpr int SEGU = 8;
 __global__ void __launch_bounds__(256) k_seg_scan(const float* __restrict__ seg_state,
                                                   const float* __restrict__ seg_gamma, const float* __restrict__ h0,
                                                   float* __restrict__ sinit, int BH, int Dk, int Dv, int nseg) {
+    grid_dep_launch();
+    grid_dep_wait();   // the state pass has written seg_state, seg_gamma
     const int per4 = Dk * Dv / 4;
     const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (long)BH * per4) return;
@@ -869,6 +873,8 @@ __global__ void __launch_bounds__(256) k_seg_scan(const float* __restrict__ seg_
 __global__ void __launch_bounds__(256) k_seg_rscan(const float* __restrict__ seg_state,
                                                    const float* __restrict__ seg_gamma, const float* __restrict__ dhT,
                                                    float* __restrict__ gend, int BH, int Dk, int Dv, int nseg) {
+    grid_dep_launch();
+    grid_dep_wait();   // the state-gradient pass has written seg_state, seg_gamma
     const int per4 = Dk * Dv / 4;
     const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (long)BH * per4) return;
@@ -898,10 +904,11 @@ __global__ void __launch_bounds__(256) k_seg_rscan(const float* __restrict__ seg
 }
 
 // ------------------------------------------------------------------ host side
+// pdl: the kernel follows the segment scan of the same call and may start before it ends
 template <int DK, int DVT, int GATE, int MODE>
 static cudaError_t launch_one(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                               const CUtensorMap& mg, const CUtensorMap& mo, const FwdArgs& a, const Dims& P, int nseg,
-                              cudaStream_t st) {
+                              cudaStream_t st, bool pdl = false) {
     using C = Cfg<DK, DVT, GATE, MODE>;
     auto kern = k_tc_fwd<DK, DVT, GATE, MODE>;
     static bool attr = false;
@@ -911,8 +918,10 @@ static cudaError_t launch_one(const CUtensorMap& mq, const CUtensorMap& mk, cons
         attr = true;
     }
     dim3 grid(P.B * P.H, P.Dv / DVT, nseg);
+    cudaError_t e = cudaSuccess;
     GLA_LAUNCH(MODE == 0 ? "tc_fwd" : MODE == 1 ? "tc_state" : "tc_gstate", st,
-               kern<<<grid, NTHR_WS, C::SMEM, st>>>(mq, mk, mv, mg, mo, a, P));
+               e = launch_ex(kern, grid, dim3(NTHR_WS), C::SMEM, st, pdl, 1, mq, mk, mv, mg, mo, a, P));
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -940,8 +949,7 @@ FwdPlan plan_fwd(const Dims& P) {
     if (nseg < 1) nseg = 1;
     // Segments are whole 64-token tiles, as equal as the tile count allows: the tensor-core
     // plan carries the state through every tile, so the chunk size does not constrain them
-    // (chunk-aligned segments left c4, 1024 tiles in 18 segments, with 17 of 60 tiles and one
-    // of 4).
+    // (segments of whole 256-token chunks cut 1024 tiles into 17 of 60 tiles and one of 4).
     if (nseg > ntiles) nseg = ntiles;
     pl.tiles_per_seg = cdiv(ntiles, nseg);
     pl.nseg = cdiv(ntiles, pl.tiles_per_seg);
@@ -1071,24 +1079,30 @@ static cudaError_t run(const Dims& P, const void* q, const void* k, const void* 
         e = seg_scan(P, nsub, seg_state, seg_gamma, h0, sinit, st);
         if (e != cudaSuccess) return e;
     }
-    return launch_one<DK, DVT, GATE, 0>(mq, mk, mv, mg, mo, a, P, pl.nseg, st);
+    return launch_one<DK, DVT, GATE, 0>(mq, mk, mv, mg, mo, a, P, pl.nseg, st, pl.nseg > 1);
 }
 
 cudaError_t seg_scan(const Dims& P, int nseg, const float* seg_state, const float* seg_gamma, const float* h0,
                      float* sinit, cudaStream_t st) {
     const long n = (long)P.B * P.H * P.Dk * P.Dv / 4;
+    // follows the state pass of the same call, and may start before it ends
+    cudaError_t e = cudaSuccess;
     GLA_LAUNCH("tc_seg_scan", st,
-               k_seg_scan<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(seg_state, seg_gamma, h0, sinit, P.B * P.H,
-                                                                       P.Dk, P.Dv, nseg));
+               e = launch_ex(k_seg_scan, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, true, 1, seg_state,
+                             seg_gamma, h0, sinit, P.B * P.H, P.Dk, P.Dv, nseg));
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 cudaError_t seg_rscan(const Dims& P, int nseg, const float* seg_state, const float* seg_gamma, const float* dhT,
                       float* gend, cudaStream_t st) {
     const long n = (long)P.B * P.H * P.Dk * P.Dv / 4;
+    // follows the state-gradient pass of the same call, and may start before it ends
+    cudaError_t e = cudaSuccess;
     GLA_LAUNCH("tc_seg_rscan", st,
-               k_seg_rscan<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(seg_state, seg_gamma, dhT, gend, P.B * P.H,
-                                                                        P.Dk, P.Dv, nseg));
+               e = launch_ex(k_seg_rscan, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, true, 1, seg_state,
+                             seg_gamma, dhT, gend, P.B * P.H, P.Dk, P.Dv, nseg));
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

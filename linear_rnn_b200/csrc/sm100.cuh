@@ -114,6 +114,14 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the kernel before
+// it in the stream is still running; it must wait here before reading anything that kernel
+// writes (returns at once when there is no such prerequisite). The running kernel lets its
+// dependent start early with grid_dep_launch (no effect when nothing depends on it that way).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // One lane of the (fully active) warp is elected; the others get false. Issuing
 // tcgen05 instructions from an elected lane while the whole warp runs the loop keeps the
 // operand descriptors warp-uniform.
