@@ -186,6 +186,16 @@ GLA_API gla_status gla_fwd_static_scratch(const gla_problem* p, const void* q, c
                                           const float* g, const float* igate, const float* h0,
                                           void* o, float* hT, void* stream);
 
+/* Diagnostics of the device-side failure path (not needed for computing): launches one small
+ * kernel on `stream` whose bounded mbarrier wait is never completed, so that it gives up after
+ * `polls` polls (1 .. 2^20; each poll suspends the thread for at most a system-dependent time)
+ * and sets the timeout bit of the device status word in `ws` (at least 256 bytes, 16-byte
+ * aligned, device memory owned by the caller), as a timed-out wait inside gla_fwd / gla_bwd
+ * does. gla_check_device_status(ws, stream) then returns GLA_ERR_TIMEOUT and the CUDA context
+ * stays usable. Nothing faults, traps or hangs. Errors: GLA_ERR_INVALID_ARG (before any
+ * launch), GLA_ERR_CUDA. */
+GLA_API gla_status gla_debug_wait_timeout(void* ws, unsigned polls, void* stream);
+
 /* Measurement support (not needed for computing).
  * gla_launch_count: number of kernels this process has launched through the library.
  * gla_profiler_enable(1): from now on every kernel launch is bracketed by two CUDA events

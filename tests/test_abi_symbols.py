@@ -148,6 +148,13 @@ def test_bwd_argument_validation_happens_before_launch():
     assert call(nbytes=4096) == _lib.GLA_ERR_WORKSPACE
 
 
+def test_debug_wait_timeout_validates_before_launch():
+    assert _lib.lib.gla_debug_wait_timeout(None, 100, None) == _lib.GLA_ERR_INVALID_ARG
+    assert _lib.lib.gla_debug_wait_timeout(ctypes.c_void_p(24), 100, None) == _lib.GLA_ERR_INVALID_ARG  # misaligned
+    assert _lib.lib.gla_debug_wait_timeout(ctypes.c_void_p(16), 0, None) == _lib.GLA_ERR_INVALID_ARG
+    assert _lib.lib.gla_debug_wait_timeout(ctypes.c_void_p(16), (1 << 20) + 1, None) == _lib.GLA_ERR_INVALID_ARG
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     import importlib
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
