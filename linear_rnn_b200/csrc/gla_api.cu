@@ -45,6 +45,10 @@ void prof_begin(const char* name, cudaStream_t st) {
     cudaEventRecord(r.start, st);
     g_prof_open.push_back(r);
 }
+bool prof_enabled() {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    return g_prof_on;
+}
 void prof_end(cudaStream_t st) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
     if (!g_prof_on || g_prof_open.empty()) return;

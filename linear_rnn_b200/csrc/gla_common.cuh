@@ -38,6 +38,9 @@ constexpr float kMinTileLogDecay = -60.f;
 // events recorded on the launching stream.
 void prof_begin(const char* name, cudaStream_t st);
 void prof_end(cudaStream_t st);
+// Whether launches are being timed (gla_profiler_enable): plans then keep every kernel on the
+// caller's stream, so that each launch's events time that kernel alone.
+bool prof_enabled();
 
 }  // namespace gla
 

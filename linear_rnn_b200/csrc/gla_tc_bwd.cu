@@ -31,6 +31,8 @@
 // shifted cumulative decay.
 // Segment boundary states come from the forward state pass + scan; segment boundary
 // state gradients from the reverse state pass (gla_tc_fwd.cu, mode 2) + reverse scan.
+#include <mutex>
+
 #include "gla_plans.h"
 #include "gla_tc_common.cuh"
 
@@ -1402,6 +1404,21 @@ __global__ void __launch_bounds__(NT_B, 1)
 }
 
 // ============================================================================ host side
+// A second stream per device, created on first use, on which the state-gradient pass and its
+// reverse scan run beside the dq kernel (they do not depend on it): their CTAs fill the SMs the
+// dq kernel's last partial wave leaves idle. nullptr if it cannot be created.
+static cudaStream_t aux_stream() {
+    constexpr int kMaxDev = 64;
+    static std::once_flag once[kMaxDev];
+    static cudaStream_t streams[kMaxDev];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+    std::call_once(once[dev], [dev] {
+        if (cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess) streams[dev] = nullptr;
+    });
+    return streams[dev];
+}
+
 struct BwdPlan {
     int nseg, tiles_per_seg, dkb;
 };
@@ -1497,7 +1514,8 @@ static cudaError_t launch_dq(const Dims& P, const BwdPlan& pl, const CUtensorMap
 template <int DK, int DV, int GATE, int KS>
 static cudaError_t launch_dkdv(const Dims& P, const BwdPlan& pl, const CUtensorMap& mq, const CUtensorMap& mk,
                                const CUtensorMap& mg, const CUtensorMap& mv, const CUtensorMap& mo,
-                               const CUtensorMap& mdk, const CUtensorMap& mdv, const BwdArgs& a, cudaStream_t st) {
+                               const CUtensorMap& mdk, const CUtensorMap& mdv, const BwdArgs& a, cudaStream_t st,
+                               bool pdl) {
     using C = KVCfg<DK, DV, GATE>;
     auto kern = k_tc_bwd_dkdv<DK, DV, GATE, KS>;
     static bool attr = false;
@@ -1506,11 +1524,12 @@ static cudaError_t launch_dkdv(const Dims& P, const BwdPlan& pl, const CUtensorM
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    // the two key blocks of a (b*h, segment) run as one cluster of two CTAs; the kernel may start
-    // before the kernel ahead of it (reverse scan or dq) ends, and waits for it in grid_dep_wait
+    // the two key blocks of a (b*h, segment) run as one cluster of two CTAs; with pdl the kernel
+    // may start before the kernel ahead of it in the stream (reverse scan or dq) ends, and waits
+    // for it in grid_dep_wait
     cudaError_t e = cudaSuccess;
     GLA_LAUNCH("tc_bwd_dkdv", st,
-               e = launch_ex(kern, dim3(KS * P.B * P.H, pl.nseg), dim3(NT_B), C::SMEM, st, true, KS, mq, mk, mg, mv, mo,
+               e = launch_ex(kern, dim3(KS * P.B * P.H, pl.nseg), dim3(NT_B), C::SMEM, st, pdl, KS, mq, mk, mg, mv, mo,
                              mdk, mdv, a, P));
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
@@ -1576,15 +1595,45 @@ static cudaError_t run_bwd(const Dims& P, const void* q, const void* k, const vo
     a.status = status;
     a.tiles_per_seg = pl.tiles_per_seg;
     a.nseg = pl.nseg;
-    e = launch_dq<DKB, DV, GATE>(P, pl, mq, mk, mg, mv, mo, mdq, a, st);
-    if (e != cudaSuccess) return e;
-    if (pl.nseg > 1) {
-        e = state_pass(P, 2, q, dO, g, ig, pl.nseg, pl.tiles_per_seg, w.seg_state, w.seg_gamma, status, st);
-        if (e != cudaSuccess) return e;
-        e = seg_rscan(P, pl.nseg, w.seg_state, w.seg_gamma, dhT, w.gend, st);
-        if (e != cudaSuccess) return e;
+    // the state-gradient pass and reverse scan (segment-end state gradients for the dk/dv kernel)
+    // depend on the inputs only: forked onto a second stream after everything the call has
+    // enqueued so far (the forward state pass and scan above use the same segment buffers), and
+    // joined before the dk/dv kernel
+    cudaStream_t st2 = (pl.nseg > 1 && !prof_enabled()) ? aux_stream() : nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+    if (st2 && (cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&ev_join, cudaEventDisableTiming) != cudaSuccess)) {
+        if (ev_fork) cudaEventDestroy(ev_fork);
+        ev_fork = nullptr;
+        st2 = nullptr;
     }
-    e = launch_dkdv<DKB, DV, GATE, KS>(P, pl, mq, mk, mg, mv, mo, mdk, mdv, a, st);
+    auto release = [&] {
+        if (ev_fork) cudaEventDestroy(ev_fork);
+        if (ev_join) cudaEventDestroy(ev_join);
+    };
+    cudaStream_t sg = st;
+    if (st2) {
+        if ((e = cudaEventRecord(ev_fork, st)) != cudaSuccess || (e = cudaStreamWaitEvent(st2, ev_fork, 0)) != cudaSuccess) {
+            release();
+            return e;
+        }
+        sg = st2;
+    }
+    e = launch_dq<DKB, DV, GATE>(P, pl, mq, mk, mg, mv, mo, mdq, a, st);
+    if (e == cudaSuccess && pl.nseg > 1) {
+        e = state_pass(P, 2, q, dO, g, ig, pl.nseg, pl.tiles_per_seg, w.seg_state, w.seg_gamma, status, sg);
+        if (e == cudaSuccess) e = seg_rscan(P, pl.nseg, w.seg_state, w.seg_gamma, dhT, w.gend, sg);
+    }
+    if (st2) {
+        // the join is enqueued even after a launch error, so that st never races ahead of st2
+        const cudaError_t e1 = cudaEventRecord(ev_join, st2);
+        const cudaError_t e2 = e1 == cudaSuccess ? cudaStreamWaitEvent(st, ev_join, 0) : e1;
+        if (e == cudaSuccess) e = e2;
+    }
+    release();
+    if (e != cudaSuccess) return e;
+    // after the join the kernel ahead of it in st is an event wait: launched without overlap
+    e = launch_dkdv<DKB, DV, GATE, KS>(P, pl, mq, mk, mg, mv, mo, mdk, mdv, a, st, st2 == nullptr);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
