@@ -32,6 +32,10 @@
  *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL means
  *    the legacy default stream). Argument errors are detected on the host before any
  *    launch; launch failures map to GLA_ERR_CUDA. No exception crosses the ABI.
+ *    The tensor-core backward runs its state-gradient pass on a second stream of its own
+ *    (one per device, created on first use), forked from `stream` by an event after all
+ *    work enqueued before the call and joined back by an event before its last kernel, so
+ *    the call still orders like a single launch sequence on `stream`.
  *  - Thread safety: concurrent calls are safe when they use distinct workspaces.
  */
 #ifndef GLA_B200_H
