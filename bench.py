@@ -124,14 +124,14 @@ def kernel_bytes(name, w, fseg=1, bseg=1):
 # time: a kernel whose source has changed since reports traffic null. `scale`: the capture
 # ran a smaller case of the same workload; traffic grows with the heads processed.
 MEASURED_TRAFFIC = {
-    ("tc_bwd_dkdv", "c3"): {"bytes": 248.7e6, "scale": 4, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
-                            "sha": "1db7704b815f809e", "profile": "profiles/tc_bwd_c3_b1.md"},
-    ("tc_bwd_dq", "c3"): {"bytes": 174.5e6, "scale": 4, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
-                          "sha": "1db7704b815f809e", "profile": "profiles/tc_bwd_c3_b1.md"},
-    ("tc_bwd_dkdv", "c5"): {"bytes": 243.1e6, "scale": 2, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
-                            "sha": "1db7704b815f809e", "profile": "profiles/tc_bwd_dkdv_c5_b1.md"},
+    ("tc_bwd_dkdv", "c3"): {"bytes": 246.9e6, "scale": 4, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
+                            "sha": "b602016964e3abce", "profile": "profiles/tc_bwd_c3_b1.md"},
+    ("tc_bwd_dq", "c3"): {"bytes": 174.0e6, "scale": 4, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
+                          "sha": "b602016964e3abce", "profile": "profiles/tc_bwd_c3_b1.md"},
+    ("tc_bwd_dkdv", "c5"): {"bytes": 247.0e6, "scale": 2, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
+                            "sha": "b602016964e3abce", "profile": "profiles/tc_bwd_dkdv_c5_b1.md"},
     ("tc_fwd", "c2"): {"bytes": 187.1e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_fwd.cu",
-                       "sha": "b88d1f96544c9517", "profile": "profiles/tc_fwd_c2.md"},
+                       "sha": "925397156e2eb2d0", "profile": "profiles/tc_fwd_c2.md"},
 }
 
 
