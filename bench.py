@@ -51,6 +51,8 @@ def flops(w, backward):
     """Algorithmic FLOPs: per token-head C*Dk + C*Dv + 4*Dk*Dv forward (causal-half intra
     products, inter q~S, state K^T V) and C*(3Dk+2Dv) + 8*Dk*Dv backward."""
     th = w.B * w.H * w.L
+    if w.name == "decode":   # one token from a given state: the state update and q S
+        return float(th * 4 * w.Dk * w.Dv)
     f = th * (w.chunk * w.Dk + w.chunk * w.Dv + 4 * w.Dk * w.Dv)
     if backward:
         f += th * (w.chunk * (3 * w.Dk + 2 * w.Dv) + 8 * w.Dk * w.Dv)
@@ -115,6 +117,8 @@ def kernel_bytes(name, w, fseg=1, bseg=1):
         "tc_seg_rscan": 2 * s1 * (bseg - 1) + s1,
         "tc_bwd_dq": q + k + v + o + ge + ig + s1 * bseg + h0 + q + dgb + s1 + 4 * BH * bseg * w.Dk,
         "tc_bwd_dkdv": q + k + v + o + ge + ig + 2 * s1 * bseg + dgb + 4 * BH * bseg * w.Dk + s1 + k + v + dgb + ig + h0,
+        # decode step: q, k, v, g, i read, o written, the state read and written once
+        "decode": compulsory_bytes(w, False),
     }
     return float(table.get(name, 0.0))
 
@@ -264,7 +268,7 @@ def base_line(w, args, world):
     return {"metric": "GLA chunkwise fwd/bwd tokens/s", "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded; workload recipe in DESIGN.md)",
-            "config": {"workload": f"{w.name}: {'GLA forward+backward' if w.backward else 'GLA forward'}, "
+            "config": {"workload": f"{w.name}: {'GLA decode step' if w.name == 'decode' else 'GLA forward+backward' if w.backward else 'GLA forward'}, "
                                    f"B={w.B} H={w.H} L={w.L} Dk={w.Dk} Dv={w.Dv} chunk={w.chunk} {w.dtype}",
                        "global_batch": w.B * world, "seq_len": w.L, "parallelism": f"replicas x{world}",
                        "l2": "256 MiB L2 flush between steps, outside the per-step events; inputs > L2"}}
@@ -299,7 +303,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="c3", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--workload", default="c3", choices=sorted(I.WORKLOADS) + ["decode"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--plan", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--no-e2e", action="store_true")
@@ -309,7 +313,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    w = I.WORKLOADS[args.workload]
+    w = I.DECODE if args.workload == "decode" else I.WORKLOADS[args.workload]
+    decode = w.name == "decode"
     if args.batch is not None:
         w = w.replace(B=args.batch)
     world, rank, local = dist_setup()
@@ -337,6 +342,9 @@ def main():
     saved = torch.empty(max(nsaved // 4, 1), dtype=torch.float32, device=dev) if nsaved else None
 
     def step():
+        if decode:   # one token per (b, h) from the state, updated in place (xd["h0"])
+            ops.gla_decode(xd["q"], xd["k"], xd["v"], xd["g"], xd["igate"], xd["h0"], scale=w.scale)
+            return
         ops.gla_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["igate"], xd["h0"], workspace=ws, saved_states=saved,
                     **kw)
         if w.backward:
@@ -396,6 +404,11 @@ def main():
 
         def e2e_step():
             nonlocal d2h
+            if decode:   # the state stays on the device; the token's inputs come from the host
+                o = ops.gla_decode(*(None if xh[n] is None else xh[n].to(dev, non_blocking=True)
+                                     for n in ("q", "k", "v", "g", "igate")), xd["h0"], scale=w.scale).cpu()
+                d2h = o.numel() * o.element_size()
+                return
             o, hT = ops.gla_fwd(xh["q"], xh["k"], xh["v"], xh["g"], xh["igate"], xh["h0"], saved_states=saved,
                                 **kw)
             nb = o.numel() * o.element_size() + hT.numel() * hT.element_size()
@@ -420,6 +433,9 @@ def main():
         e_ms = max_over_ranks(e_ms, dev)
         h2d_step = h2d * (2 if w.backward else 1) + (sum(xh[n].numel() * xh[n].element_size() for n in ("dO",))
                                                      if w.backward else 0)
+        if decode:
+            h2d_step = sum(xh[n].numel() * xh[n].element_size() for n in ("q", "k", "v", "g", "igate")
+                           if xh[n] is not None)
         e2e = {"value": tokens / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d_step),
                "d2h_bytes_per_step": int(d2h)}
 

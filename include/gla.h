@@ -143,6 +143,19 @@ GLA_API gla_status gla_bwd_saved(const gla_problem* p, const void* q, const void
                                  void* dq, void* dk, void* dv, float* dg, float* di, float* dh0,
                                  void* ws, size_t ws_bytes, void* stream);
 
+/* Recurrent single-token step from a given state (the inference use of the same state):
+ *     S <- diag(alpha) S + k'^T v,   o = scale * q S   (alpha = e^g, k' = i k, S updated first),
+ * per (b, h), with the state updated in place. p->L must be 1 (one token per (b, h));
+ * p->chunk and p->plan are ignored. q,k [B,H,1,Dk]; v,o [B,H,1,Dv] (I/O dtype); g as for
+ * gla_fwd with L = 1 ([B,H,1,Dk] or [B,H,1]) or NULL iff gate == GLA_GATE_NONE; igate [B,H,1]
+ * or NULL; state [B,H,Dk,Dv] f32, read and overwritten (must not alias the other buffers).
+ * The result equals gla_fwd over the one token with h0 = state: o, and hT into state. Needs
+ * no workspace; bound by HBM bandwidth (the state is read and written once).
+ * Errors: GLA_ERR_INVALID_ARG (null or misaligned pointer, L != 1, bad enum),
+ * GLA_ERR_UNSUPPORTED (head dims), GLA_ERR_CUDA. */
+GLA_API gla_status gla_decode(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
+                              const float* igate, float* state, void* o, void* stream);
+
 /* Static description of a status code (never NULL). */
 GLA_API const char* gla_status_string(gla_status s);
 

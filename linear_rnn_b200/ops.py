@@ -131,6 +131,24 @@ def gla_fwd(q, k, v, g=None, igate=None, h0=None, *, scale: Optional[float] = No
     return o, hT
 
 
+def gla_decode(q, k, v, g, igate, state, *, scale: Optional[float] = None) -> torch.Tensor:
+    """One recurrent step per (b, h) from `state` (fp32 [B,H,Dk,Dv] on the GPU, updated in
+    place): q, k [B,H,1,Dk], v [B,H,1,Dv], g [B,H,1,Dk] / [B,H,1] / None, igate [B,H,1] / None.
+    Returns o [B,H,1,Dv]."""
+    if state.device.type != "cuda" or state.dtype != torch.float32 or not state.is_contiguous():
+        raise ValueError("state must be a contiguous float32 CUDA tensor (it is updated in place)")
+    device = state.device
+    q, k, v, g, igate = (_to_dev(t, device) for t in (q, k, v, g, igate))
+    if q.shape[2] != 1:
+        raise ValueError("gla_decode takes one token per (b, h): q must be [B, H, 1, Dk]")
+    prob = make_problem(q, v, g, scale=scale, chunk=64, plan="auto")
+    o = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=device)
+    st = _lib.lib.gla_decode(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(igate), _ptr(state),
+                             _ptr(o), _stream_handle(device))
+    _check(st, "gla_decode")
+    return o
+
+
 def _check_saved(saved, prob):
     if saved is None:
         return

@@ -148,6 +148,25 @@ def test_bwd_argument_validation_happens_before_launch():
     assert call(nbytes=4096) == _lib.GLA_ERR_WORKSPACE
 
 
+def test_decode_validates_before_launch():
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+
+    def call(p, **kw):
+        a = dict(q=16, k=16, v=16, g=16, ig=None, state=16, o=16)
+        a.update(kw)
+        return _lib.lib.gla_decode(ctypes.byref(p), *(vp(a[n]) for n in ("q", "k", "v", "g", "ig", "state", "o")),
+                                   None)
+    one = prob(L=1)
+    assert call(prob(L=2)) == _lib.GLA_ERR_INVALID_ARG              # one token per (b, h)
+    assert call(one, state=None) == _lib.GLA_ERR_INVALID_ARG
+    assert call(one, g=None) == _lib.GLA_ERR_INVALID_ARG            # gate mode says per-key
+    assert call(prob(L=1, gate=_lib.GLA_GATE_NONE)) == _lib.GLA_ERR_INVALID_ARG   # g given, no gate
+    assert call(one, v=24) == _lib.GLA_ERR_INVALID_ARG              # misaligned
+    assert call(prob(L=1, Dk=96)) == _lib.GLA_ERR_UNSUPPORTED
+    assert call(prob(L=1, io=7)) == _lib.GLA_ERR_INVALID_ARG
+    assert _lib.lib.gla_decode(None, None, None, None, None, None, None, None, None) == _lib.GLA_ERR_INVALID_ARG
+
+
 def test_debug_wait_timeout_validates_before_launch():
     assert _lib.lib.gla_debug_wait_timeout(None, 100, None) == _lib.GLA_ERR_INVALID_ARG
     assert _lib.lib.gla_debug_wait_timeout(ctypes.c_void_p(24), 100, None) == _lib.GLA_ERR_INVALID_ARG  # misaligned
