@@ -77,8 +77,8 @@ def _round_io(x: torch.Tensor, dtype: str) -> torch.Tensor:
     raise ValueError(f"unknown io dtype {dtype!r}")
 
 
-# Single-token decode step from a given state at a serving batch: 64 sequences x 16 heads, the
-# c3 head dims, bf16 I/O, per-key log-gate logsigmoid(N(0,1))/16 (the forward workloads'
+# Single-token decode step from a given state at a serving batch: 64 sequences x 16 heads,
+# Dk=128 Dv=256, bf16 I/O, per-key log-gate logsigmoid(N(0,1))/16 (the forward workloads'
 # gates), state ~ N(0, 1) fp32 (1024 states of 128 x 256 = 128 MiB, more than L2).
 DECODE = Workload("decode", 64, 16, 1, 128, 256, 64, "bf16", GATE_PER_KEY, False, 128 ** -0.5,
                   h0_std=1.0, gate_div=16.0)
