@@ -83,13 +83,19 @@ struct Cfg {
     static constexpr uint32_t PB = MODE == 0 ? TR * TR * 2 : 0;       // P
     static constexpr uint32_t SB = MODE == 0 ? DK * DVT * 2 : 0;      // bf16 state
     static constexpr uint32_t OB = MODE == 0 ? TR * DVT * 2 : 0;      // output tile staged for the TMA store
-    static constexpr uint32_t SMALL = 256 + 8 * NTRF + 16 * DK + 1024;
+    // (+ a ring of NS + 1 row-factor vectors of the output pass)
+    static constexpr uint32_t SMALL = 256 + 8 * NTRF + 16 * DK + 1024 + 256 * 5;
+    // Output pass with per-head or no gates: q enters the products untransformed, the O
+    // accumulator holds q S_prev + P V, and the output pass scales row t by scale e^(b_t)
+    // (P = mask(q k~^T) already carries e^(-b_s)). Per-key gates transform q (scale q e^b).
+    static constexpr bool XQ = MODE == 0 && GATE == 1;
     static constexpr uint32_t FIXED = PB + SB + OB + SMALL + 1024;
     // as many ring stages (up to 4) as shared memory holds: the loads of a tile are in
     // flight while the tiles before it are transformed and multiplied
     static constexpr int NS = (4 * STAGE + FIXED <= 227 * 1024) ? 4 : (3 * STAGE + FIXED <= 227 * 1024) ? 3
                               : (2 * STAGE + FIXED <= 227 * 1024) ? 2 : 1;
     static constexpr uint32_t SMEM = NS * STAGE + FIXED;
+    static constexpr int NF = NS + 1;   // row-factor ring: a tile's factors live until its output pass
     static constexpr int NH = DK == 256 ? 2 : 1;            // M=128 halves of the state
     static constexpr int MS = DK == 64 ? 64 : 128;           // M of the state MMA
     // TMEM columns: the fp32 state [0, COLS_S), then NAB buffers of COLA columns holding
@@ -170,6 +176,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
     float* rowEi = rowE + TR;                                // [64] e^-b
     float* igs = rowEi + TR;                                 // [64] input gate
     float* ghs = igs + TR;                                   // [64] per-head gate
+    float* orf = ghs + TR;                                   // [NF][64] output row factors (!XQ)
 
     const int bh = blockIdx.x, vt = blockIdx.y, z = blockIdx.z + A.seg_offset;
     const int e0 = vt * DVT;
@@ -566,6 +573,10 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     // MODE 2 scales q by its decay from the segment's start, e^(D + b)
                     const float bq0 = MODE == 2 ? b0 + dlat1 : b0, bq1 = MODE == 2 ? b1 + dlat1 : b1;
                     rowE[2 * lane] = __expf(bq0);
+                    if (MODE == 0) {   // the output pass's row factors of this tile
+                        orf[(j % C::NF) * TR + 2 * lane] = P.scale * rowE[2 * lane];
+                        orf[(j % C::NF) * TR + 2 * lane + 1] = P.scale * __expf(bq1);
+                    }
                     rowE[2 * lane + 1] = __expf(bq1);
                     // MODE 1: e^(D + Gamma - b), the decay from the token to the segment's end
                     rowEi[2 * lane] = __expf(MODE == 1 ? dlat1 + G - b0 : -b0);
@@ -599,7 +610,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     }
                     offs[k] = (uint32_t)(d0 >> 6) * BLK + (uint32_t)r * 128 +
                               ((((uint32_t)((d0 & 63) >> 3)) ^ (uint32_t)(r & 7)) << 4);
-                    if (MODE == 0) wq[k] = *reinterpret_cast<const uint4*>(sq + offs[k]);
+                    if (C::XQ) wq[k] = *reinterpret_cast<const uint4*>(sq + offs[k]);
                     wk[k] = *reinterpret_cast<const uint4*>(sk + offs[k]);
                 }
 #pragma unroll
@@ -631,7 +642,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                         pk[u] = f2_to_bf2(f2_mul(bf2_to_f2(pk[u]), f2_mul(mk2, e2)));
                     }
                     *reinterpret_cast<uint4*>(sk + offs[k]) = wk[k];
-                    if (MODE == 0) {
+                    if (C::XQ) {
                         uint32_t* pq = reinterpret_cast<uint32_t*>(&wq[k]);
                         const uint64_t sc2 = f2(P.scale, P.scale);
 #pragma unroll
@@ -754,6 +765,8 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 if (!named_bar_and(BAR_PO, 128, ok)) break;
                 tc_fence_after();
                 const int t = 16 * qd + (lane & 15);
+                // per-head or no gates: row t of O is q S_prev + P V, scaled here by scale e^(b_t)
+                const float rf = C::XQ ? 1.f : GATE == 2 ? orf[(i % C::NF) * TR + t] : P.scale;
 #pragma unroll
                 for (int c = 0; c < DVT; c += C::CH) {
                     uint32_t r[C::CH];
@@ -761,8 +774,12 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     tmem_wait_ld();
                     if (lane >= 16)
 #pragma unroll
-                        for (int u = 0; u < C::CH / 8; ++u)
-                            store8_bf16(sO, sw128_off(t, c + 8 * u, BLK), reinterpret_cast<const float*>(&r[8 * u]));
+                        for (int u = 0; u < C::CH / 8; ++u) {
+                            float f[8];
+#pragma unroll
+                            for (int jj = 0; jj < 8; ++jj) f[jj] = C::XQ ? __uint_as_float(r[8 * u + jj]) : rf * __uint_as_float(r[8 * u + jj]);
+                            store8_bf16(sO, sw128_off(t, c + 8 * u, BLK), f);
+                        }
                 }
                 fence_proxy_async_smem();
             }
