@@ -184,3 +184,56 @@ def test_tc_fwd_state_subsegments(Dk, Dv, chunk, gate, ig):
              gate_div=1.0 if gate == I.GATE_PER_HEAD else 16.0)
     eo, eh = run_tc_fwd(w, 24)
     assert eo <= TOL and eh <= TOL, (eo, eh)
+
+
+# ------------------------------------------------- backward on the second stream
+# The state-gradient pass and its reverse scan run on a library-owned second stream beside the
+# dq kernel (one stream while the launch profiler is on); the results must not depend on that.
+
+def _bwd_inputs(seed):
+    w = I.WORKLOADS["c3"].replace(B=1, H=4, L=1500)
+    x = {k: (None if v is None else v.cuda()) for k, v in I.make_inputs(w, seed=seed).items()}
+    return w, x
+
+
+def test_tc_bwd_second_stream_bitwise_equal_to_one_stream():
+    from linear_rnn_b200 import _lib, ops
+    w, x = _bwd_inputs(41)
+    args = (x["q"], x["k"], x["v"], x["g"], x["igate"], x["h0"], x["dO"], None)
+    assert _lib.plan_info(ops.make_problem(x["q"], x["v"], x["g"], scale=w.scale, chunk=w.chunk, plan="tc"),
+                          True)[1] > 1   # segmented: the second stream is used
+    a = ops.gla_bwd(*args, scale=w.scale, chunk=w.chunk, plan="tc")
+    _lib.profiler_enable(True)
+    try:
+        b = ops.gla_bwd(*args, scale=w.scale, chunk=w.chunk, plan="tc")
+        torch.cuda.synchronize()
+    finally:
+        _lib.profiler_enable(False)
+        _lib.profiler_read()
+    for n in ("dq", "dk", "dv", "dg", "dh0"):
+        assert torch.equal(a[n], b[n]), n
+
+
+def test_tc_bwd_concurrent_calls_on_two_streams():
+    """Two backward calls on two streams (distinct workspaces) share the library's second
+    stream; each matches its own result computed alone."""
+    from linear_rnn_b200 import ops
+    w, x1 = _bwd_inputs(42)
+    _, x2 = _bwd_inputs(43)
+    args = lambda x: (x["q"], x["k"], x["v"], x["g"], x["igate"], x["h0"], x["dO"], None)
+    ref1 = ops.gla_bwd(*args(x1), scale=w.scale, chunk=w.chunk, plan="tc")
+    ref2 = ops.gla_bwd(*args(x2), scale=w.scale, chunk=w.chunk, plan="tc")
+    torch.cuda.synchronize()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    outs = []
+    for _ in range(3):
+        with torch.cuda.stream(s1):
+            r1 = ops.gla_bwd(*args(x1), scale=w.scale, chunk=w.chunk, plan="tc")
+        with torch.cuda.stream(s2):
+            r2 = ops.gla_bwd(*args(x2), scale=w.scale, chunk=w.chunk, plan="tc")
+        outs.append((r1, r2))
+    torch.cuda.synchronize()
+    for r1, r2 in outs:
+        for n in ("dq", "dk", "dv", "dg", "dh0"):
+            assert torch.equal(r1[n], ref1[n]), n
+            assert torch.equal(r2[n], ref2[n]), n
