@@ -156,6 +156,26 @@ GLA_API gla_status gla_bwd_saved(const gla_problem* p, const void* q, const void
 GLA_API gla_status gla_decode(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
                               const float* igate, float* state, void* o, void* stream);
 
+/* Sequence sharding (one exchange step per pass). A sequence cut into contiguous shards, one per
+ * rank, runs as: each rank calls gla_shard_state on its shard; the (state, gamma) pairs of all
+ * ranks are all-gathered (rank order); each rank calls gla_state_fold with count = its rank to
+ * get its shard's initial state, and gla_fwd on its shard from that state. The outputs are
+ * those of one gla_fwd over the whole sequence; the last rank's hT is the sequence's.
+ * gla_shard_state: the shard's end state from a zero initial state, state [B,H,Dk,Dv] f32, and
+ *   its total log-decay per key dim, gamma [B,H,Dk] f32 (per-head gates: the head's total in
+ *   every key slot). p describes the shard (L = its tokens; L = 0 gives zeros). Tensor-core
+ *   state pass: bf16 I/O, chunk a multiple of 64; otherwise GLA_ERR_UNSUPPORTED. ws: at least
+ *   256 bytes (device status word, as for gla_fwd). q is not read.
+ * gla_state_fold: out = S after S <- h0 (or 0), then for i = 0 .. count-1:
+ *   S <- diag(e^{gammas[i]}) S + states[i], with states [count][B,H,Dk,Dv] and gammas
+ *   [count][B,H,Dk] f32 as all-gathered; p gives B, H, Dk, Dv. out may not alias the inputs.
+ * Errors: GLA_ERR_INVALID_ARG, GLA_ERR_UNSUPPORTED, GLA_ERR_WORKSPACE, GLA_ERR_CUDA. */
+GLA_API gla_status gla_shard_state(const gla_problem* p, const void* k, const void* v, const float* g,
+                                   const float* igate, float* state, float* gamma, void* ws, size_t ws_bytes,
+                                   void* stream);
+GLA_API gla_status gla_state_fold(const gla_problem* p, int count, const float* states, const float* gammas,
+                                  const float* h0, float* out, void* stream);
+
 /* Static description of a status code (never NULL). */
 GLA_API const char* gla_status_string(gla_status s);
 

@@ -149,6 +149,59 @@ def gla_decode(q, k, v, g, igate, state, *, scale: Optional[float] = None) -> to
     return o
 
 
+def gla_shard_state(k, v, g=None, igate=None, *, chunk: int = 64) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(state, gamma) of one sequence shard: its end state from a zero initial state
+    [B,H,Dk,Dv] and its total log-decay per key dim [B,H,Dk], both fp32 on the GPU."""
+    device = k.device
+    prob = make_problem(k, v, g, scale=1.0, chunk=chunk, plan="tc")
+    B, H, _, Dk = k.shape
+    state = torch.empty(B, H, Dk, v.shape[-1], dtype=torch.float32, device=device)
+    gamma = torch.empty(B, H, Dk, dtype=torch.float32, device=device)
+    ws = torch.empty(256, dtype=torch.uint8, device=device)
+    st = _lib.lib.gla_shard_state(ctypes.byref(prob), _ptr(k), _ptr(v), _ptr(g), _ptr(igate), _ptr(state),
+                                  _ptr(gamma), _ptr(ws), 256, _stream_handle(device))
+    _check(st, "gla_shard_state")
+    return state, gamma
+
+
+def gla_state_fold(states: torch.Tensor, gammas: torch.Tensor, count: int,
+                   h0: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The state after the first `count` shards, given all shards' (state, gamma) stacked along
+    a leading shard axis ([n,B,H,Dk,Dv], [n,B,H,Dk]), starting from h0 (or 0)."""
+    if states.dim() != 5 or gammas.dim() != 4 or not (0 <= count <= states.shape[0]):
+        raise ValueError("states [n,B,H,Dk,Dv], gammas [n,B,H,Dk], 0 <= count <= n")
+    _, B, H, Dk, Dv = states.shape
+    prob = GlaProblem(B, H, 1, Dk, Dv, 64, 1.0, _lib.GLA_F32, _lib.GLA_GATE_PER_KEY, _PLANS["auto"])
+    out = torch.empty(B, H, Dk, Dv, dtype=torch.float32, device=states.device)
+    st = _lib.lib.gla_state_fold(ctypes.byref(prob), int(count), _ptr(states.contiguous()), _ptr(gammas.contiguous()),
+                                 _ptr(h0), _ptr(out), _stream_handle(states.device))
+    _check(st, "gla_state_fold")
+    return out
+
+
+def gla_fwd_sequence_sharded(q, k, v, g=None, igate=None, h0=None, *, scale: Optional[float] = None,
+                             chunk: int = 64, group=None, _shard_ops=None):
+    """Forward over a sequence cut into contiguous shards, one per rank of `group` (rank order =
+    sequence order): each rank passes its own shard of q, k, v, g, igate (and every rank the
+    same h0), and gets its shard's o and end state (the last rank's is the sequence's hT).
+    One all-gather of the shards' (end state from zero, total log-decay) is the only exchange.
+    _shard_ops replaces the three per-rank steps (shard_state, fold, forward) for tests of the
+    exchange on CPU ranks."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    shard_state, fold, fwd = _shard_ops or (
+        lambda: gla_shard_state(k, v, g, igate, chunk=chunk),
+        lambda states, gammas: gla_state_fold(states, gammas, rank, h0),
+        lambda s_in: gla_fwd(q, k, v, g, igate, s_in, scale=scale, chunk=chunk))
+    state, gamma = shard_state()
+    parts_s = [torch.empty_like(state) for _ in range(world)]
+    parts_g = [torch.empty_like(gamma) for _ in range(world)]
+    dist.all_gather(parts_s, state.contiguous(), group=group)
+    dist.all_gather(parts_g, gamma.contiguous(), group=group)
+    return fwd(fold(torch.stack(parts_s), torch.stack(parts_g)))
+
+
 def _check_saved(saved, prob):
     if saved is None:
         return

@@ -167,6 +167,34 @@ def test_decode_validates_before_launch():
     assert _lib.lib.gla_decode(None, None, None, None, None, None, None, None, None) == _lib.GLA_ERR_INVALID_ARG
 
 
+def test_shard_calls_validate_before_launch():
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+
+    def shard(p, **kw):
+        a = dict(k=16, v=16, g=16, ig=None, state=16, gamma=16, ws=16, nbytes=256)
+        a.update(kw)
+        return _lib.lib.gla_shard_state(ctypes.byref(p), *(vp(a[n]) for n in ("k", "v", "g", "ig", "state", "gamma",
+                                                                              "ws")), a["nbytes"], None)
+    bf = prob(io=_lib.GLA_BF16)
+    assert shard(prob(io=_lib.GLA_F32)) == _lib.GLA_ERR_UNSUPPORTED      # tensor-core state pass: bf16
+    assert shard(prob(chunk=96)) == _lib.GLA_ERR_UNSUPPORTED             # whole 64-token tiles
+    assert shard(bf, state=None) == _lib.GLA_ERR_INVALID_ARG
+    assert shard(bf, g=None) == _lib.GLA_ERR_INVALID_ARG                 # gate mode says per-key
+    assert shard(bf, k=24) == _lib.GLA_ERR_INVALID_ARG                   # misaligned
+    assert shard(bf, nbytes=100) == _lib.GLA_ERR_WORKSPACE
+
+    def fold(p, count, **kw):
+        a = dict(states=16, gammas=16, h0=None, out=16)
+        a.update(kw)
+        return _lib.lib.gla_state_fold(ctypes.byref(p), count, *(vp(a[n]) for n in ("states", "gammas", "h0", "out")),
+                                       None)
+    assert fold(bf, -1) == _lib.GLA_ERR_INVALID_ARG
+    assert fold(bf, 2, out=None) == _lib.GLA_ERR_INVALID_ARG
+    assert fold(bf, 2, states=None) == _lib.GLA_ERR_INVALID_ARG
+    assert fold(bf, 2, gammas=8) == _lib.GLA_ERR_INVALID_ARG             # misaligned
+    assert fold(prob(Dv=96), 1) == _lib.GLA_ERR_UNSUPPORTED
+
+
 def test_debug_wait_timeout_validates_before_launch():
     assert _lib.lib.gla_debug_wait_timeout(None, 100, None) == _lib.GLA_ERR_INVALID_ARG
     assert _lib.lib.gla_debug_wait_timeout(ctypes.c_void_p(24), 100, None) == _lib.GLA_ERR_INVALID_ARG  # misaligned

@@ -80,3 +80,61 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert r.returncode == 0, r.stderr[-3000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
     assert len(lines) == 1 and json.loads(lines[0])["impl"] == "reference"
+
+
+# ----------------------------------------------- sequence-sharded forward, exchange on CPU ranks
+def _shard_worker(rank, world, port, out):
+    """Each rank holds one contiguous shard; the per-rank steps are the float64 oracle (this
+    tests the exchange and the fold order, not the kernels)."""
+    import datetime
+
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=world,
+                                         timeout=datetime.timedelta(seconds=60))
+    import oracle
+    from linear_rnn_b200 import inputs as I
+    from linear_rnn_b200 import ops
+    w = I.WORKLOADS["c3"].replace(B=1, H=2, L=150, Dk=64, Dv=64, dtype="f32", input_gate=True, h0_std=0.5)
+    x = I.make_inputs(w, seed=7)
+    cuts = [0, 70, 150]
+    sl = lambda t: None if t is None else t[:, :, cuts[rank]:cuts[rank + 1]].contiguous()
+    xs = {n: sl(x[n]) for n in ("q", "k", "v", "g", "igate")}
+
+    def shard_state():
+        _, S = oracle.gla_fwd(xs["q"], xs["k"], xs["v"], xs["g"], xs["igate"], None, w.scale)
+        gam = xs["g"].double().sum(dim=2)
+        return torch.from_numpy(S), gam
+
+    def fold(states, gammas):
+        S = x["h0"].double().clone()
+        for p in range(rank):
+            S = torch.exp(gammas[p])[..., None] * S + states[p]
+        return S
+
+    def fwd(s_in):
+        return oracle.gla_fwd(xs["q"], xs["k"], xs["v"], xs["g"], xs["igate"], s_in.numpy(), w.scale)
+
+    o, hT = ops.gla_fwd_sequence_sharded(None, None, None, _shard_ops=(shard_state, fold, fwd))
+    ro, rS = oracle.gla_fwd(x["q"], x["k"], x["v"], x["g"], x["igate"], x["h0"], w.scale)
+    err_o = float(np.abs(o - ro[:, :, cuts[rank]:cuts[rank + 1]]).max() / np.abs(ro).max())
+    err_h = float(np.abs(hT - rS).max() / np.abs(rS).max()) if rank == world - 1 else 0.0
+    torch.distributed.barrier()
+    torch.distributed.destroy_process_group()
+    out.put((rank, err_o, err_h))
+
+
+def test_sequence_sharded_forward_exchange_on_two_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, err_o, err_h in res:
+        assert err_o < 1e-10 and err_h < 1e-10, (rank, err_o, err_h)
