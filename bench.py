@@ -135,7 +135,7 @@ MEASURED_TRAFFIC = {
     ("tc_bwd_dkdv", "c5"): {"bytes": 247.0e6, "scale": 2, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
                             "sha": "b602016964e3abce", "profile": "profiles/tc_bwd_dkdv_c5_b1.md"},
     ("tc_fwd", "c2"): {"bytes": 187.1e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_fwd.cu",
-                       "sha": "ed49a587f7ec0740", "profile": "profiles/tc_fwd_c2.md"},
+                       "sha": "c365d80ff3420b75", "profile": "profiles/tc_fwd_c2.md"},
     ("decode", "decode"): {"bytes": 215.2e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_decode.cu",
                            "sha": "1b7b1b10ae6dd931", "profile": "profiles/decode_1024heads.md"},
 }

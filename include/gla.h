@@ -176,6 +176,22 @@ GLA_API gla_status gla_shard_state(const gla_problem* p, const void* k, const vo
 GLA_API gla_status gla_state_fold(const gla_problem* p, int count, const float* states, const float* gammas,
                                   const float* h0, float* out, void* stream);
 
+/* Sequence-sharded backward (same single exchange step). A shard's state gradient obeys the
+ * reverse recurrence dS_{t-1} = diag(alpha_t) dS_t + scale q_t^T dO_t, so the gradient w.r.t.
+ * the state at a shard's end is a fold of the LATER shards in reverse order: each rank calls
+ * gla_shard_state and gla_shard_state_grad on its shard; the triples (state, state_grad, gamma)
+ * of all ranks are all-gathered; rank r folds states 0..r-1 from h0 (its initial state, as in
+ * the forward) and state_grads P-1 .. r+1 (reverse order, with their gammas) from dhT (the
+ * gradient at its end); then gla_bwd on its shard with those two gives its dq, dk, dv, dg, di,
+ * and on rank 0 the sequence's dh0.
+ * gla_shard_state_grad: the gradient w.r.t. the state before the shard's first token from the
+ *   shard's own outputs alone (a zero gradient at its end), state_grad [B,H,Dk,Dv] f32, and the
+ *   same total log-decay as gla_shard_state, gamma [B,H,Dk] f32. q [B,H,L,Dk] and dO
+ *   [B,H,L,Dv] bf16, g as for gla_fwd; the input gate does not enter it. p->scale is the output
+ *   scale. Same support, workspace and errors as gla_shard_state; L = 0 gives zeros. */
+GLA_API gla_status gla_shard_state_grad(const gla_problem* p, const void* q, const void* dO, const float* g,
+                                        float* state_grad, float* gamma, void* ws, size_t ws_bytes, void* stream);
+
 /* Static description of a status code (never NULL). */
 GLA_API const char* gla_status_string(gla_status s);
 

@@ -31,6 +31,7 @@ cudaError_t fwd(const Dims& P, const void* q, const void* k, const void* v, cons
 //   mode 1: forward local end states of segments 0..nseg-2 (a = k, b = v)
 //   mode 2: reverse local state gradients of segments 1..nseg-1 (a = q, b = dO)
 //   mode 3: forward local end states of all segments 0..nseg-1 (a = k, b = v)
+//   mode 4: reverse local state gradients of all segments 0..nseg-1 (a = q, b = dO)
 cudaError_t state_pass(const Dims& P, int mode, const void* a_src, const void* b_src, const float* g,
                        const float* ig, int nseg, int tiles_per_seg, float* seg_state, float* seg_gamma, int* status,
                        cudaStream_t st);

@@ -7,7 +7,10 @@
 // where S_loc(p') is shard p''s end state from a zero initial state and Gamma_p' its total
 // log-decay (the state-passing form of the Tiled Flash Linear Attention abstract, with the
 // shards as the tiles). gla_shard_state gives (S_loc, Gamma) of a shard, gla_state_fold the
-// fold; one all-gather of the (S_loc, Gamma) pairs between them is the only exchange.
+// fold; one all-gather of the (S_loc, Gamma) pairs between them is the only exchange. The
+// backward mirrors it: gla_shard_state_grad gives a shard's state gradient at its start from a
+// zero gradient at its end, G_loc, and the same fold run over the later shards in reverse
+// order, from the upstream dhT, gives the gradient flowing into the shard's end.
 #include "gla_common.cuh"
 #include "gla_plans.h"
 #include "gla_tc_common.cuh"
@@ -77,6 +80,43 @@ extern "C" gla_status gla_shard_state(const gla_problem* p, const void* k, const
     // walks it (the shards themselves are the sequence parallelism)
     const int ntiles = gla::cdiv(p->L, gla::tc::TR);
     const cudaError_t e = gla::tc::state_pass(P, 3, k, v, g, igate, 1, ntiles, state, gamma, static_cast<int*>(ws), st);
+    return e == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
+}
+
+extern "C" gla_status gla_shard_state_grad(const gla_problem* p, const void* q, const void* dO, const float* g,
+                                           float* state_grad, float* gamma, void* ws, size_t ws_bytes, void* stream) {
+    if (!p || p->B < 0 || p->H < 0 || p->L < 0) return GLA_ERR_INVALID_ARG;
+    if (p->gate != GLA_GATE_NONE && p->gate != GLA_GATE_PER_KEY && p->gate != GLA_GATE_PER_HEAD)
+        return GLA_ERR_INVALID_ARG;
+    if (p->io != GLA_BF16 || !gla::dims_ok(p) || p->chunk < 64 || p->chunk > 1024 || p->chunk % 64 != 0)
+        return GLA_ERR_UNSUPPORTED;
+    if ((long long)p->B * p->H > 65535LL) return GLA_ERR_UNSUPPORTED;
+    if (!state_grad || !gamma || !ws) return GLA_ERR_INVALID_ARG;
+    if (ws_bytes < gla::kStatusBytes) return GLA_ERR_WORKSPACE;
+    const bool empty = (size_t)p->B * p->H * p->L == 0;
+    if (!empty && (!q || !dO)) return GLA_ERR_INVALID_ARG;
+    if (!empty && (p->gate == GLA_GATE_NONE) != (g == nullptr)) return GLA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, dO, g, state_grad, gamma, ws};
+    for (const void* x : ptrs)
+        if (!gla::aligned16(x)) return GLA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemsetAsync(ws, 0, gla::kStatusBytes, st) != cudaSuccess) return GLA_ERR_CUDA;
+    const size_t BH = (size_t)p->B * p->H;
+    if (BH == 0) return GLA_OK;
+    if (p->L == 0) {
+        if (cudaMemsetAsync(state_grad, 0, 4 * BH * p->Dk * p->Dv, st) != cudaSuccess ||
+            cudaMemsetAsync(gamma, 0, 4 * BH * p->Dk, st) != cudaSuccess)
+            return GLA_ERR_CUDA;
+        return GLA_OK;
+    }
+    gla::Dims P;
+    P.B = p->B; P.H = p->H; P.L = p->L; P.Dk = p->Dk; P.Dv = p->Dv; P.C = p->chunk;
+    P.N = gla::cdiv(p->L, p->chunk);
+    P.gate = p->gate;
+    P.scale = p->scale;
+    const int ntiles = gla::cdiv(p->L, gla::tc::TR);
+    const cudaError_t e =
+        gla::tc::state_pass(P, 4, q, dO, g, nullptr, 1, ntiles, state_grad, gamma, static_cast<int*>(ws), st);
     return e == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
 }
 

@@ -1040,10 +1040,11 @@ static cudaError_t state_run(const Dims& P, int mode, const void* a_src, const v
     a.tiles_per_seg = tps;
     a.nseg = nseg;
     a.seg_offset = mode == 2 ? 1 : 0;
-    // mode 3: the forward state of every segment (a sequence shard as one segment)
+    // modes 3 and 4: the forward state / the state gradient of every segment (a sequence shard
+    // as one segment)
     if (mode == 1 || mode == 3)
         return launch_one<DK, DVT, GATE, 1>(mk, mk, mv, mg, mk, a, P, mode == 3 ? nseg : nseg - 1, st);
-    return launch_one<DK, DVT, GATE, 2>(mk, mk, mv, mg, mk, a, P, nseg - 1, st);
+    return launch_one<DK, DVT, GATE, 2>(mk, mk, mv, mg, mk, a, P, mode == 4 ? nseg : nseg - 1, st);
 }
 
 template <int DK, int DVT, int GATE>

@@ -164,6 +164,23 @@ def gla_shard_state(k, v, g=None, igate=None, *, chunk: int = 64) -> Tuple[torch
     return state, gamma
 
 
+def gla_shard_state_grad(q, dO, g=None, *, scale: Optional[float] = None,
+                         chunk: int = 64) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(state_grad, gamma) of one sequence shard: the gradient w.r.t. the state before its
+    first token from its own outputs alone [B,H,Dk,Dv], and its total log-decay per key dim
+    [B,H,Dk], both fp32 on the GPU."""
+    device = q.device
+    prob = make_problem(q, dO, g, scale=scale, chunk=chunk, plan="tc")
+    B, H, _, Dk = q.shape
+    dS = torch.empty(B, H, Dk, dO.shape[-1], dtype=torch.float32, device=device)
+    gamma = torch.empty(B, H, Dk, dtype=torch.float32, device=device)
+    ws = torch.empty(256, dtype=torch.uint8, device=device)
+    st = _lib.lib.gla_shard_state_grad(ctypes.byref(prob), _ptr(q), _ptr(dO), _ptr(g), _ptr(dS), _ptr(gamma),
+                                       _ptr(ws), 256, _stream_handle(device))
+    _check(st, "gla_shard_state_grad")
+    return dS, gamma
+
+
 def gla_state_fold(states: torch.Tensor, gammas: torch.Tensor, count: int,
                    h0: Optional[torch.Tensor] = None) -> torch.Tensor:
     """The state after the first `count` shards, given all shards' (state, gamma) stacked along
@@ -200,6 +217,40 @@ def gla_fwd_sequence_sharded(q, k, v, g=None, igate=None, h0=None, *, scale: Opt
     dist.all_gather(parts_s, state.contiguous(), group=group)
     dist.all_gather(parts_g, gamma.contiguous(), group=group)
     return fwd(fold(torch.stack(parts_s), torch.stack(parts_g)))
+
+
+def gla_bwd_sequence_sharded(q, k, v, g, igate, h0, dO, dhT=None, *, scale: Optional[float] = None,
+                             chunk: int = 64, group=None, _shard_ops=None) -> Dict[str, Optional[torch.Tensor]]:
+    """Backward over a sequence cut into contiguous shards, one per rank of `group` (rank order =
+    sequence order): each rank passes its own shard of q, k, v, g, igate, dO, and every rank the
+    same h0 and dhT (the gradient at the sequence's end). Returns gla_bwd's dict for the rank's
+    shard; rank 0's dh0 is the sequence's, the other ranks' dh0 is None. One all-gather of the
+    shards' (end state from zero, start-state gradient from zero, total log-decay) is the only
+    exchange: rank r's initial state folds shards 0..r-1 from h0, the gradient at its end folds
+    shards P-1..r+1 in reverse order from dhT. _shard_ops replaces the per-rank steps
+    (shard_state, shard_state_grad, fold, backward) for tests of the exchange on CPU ranks."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    shard_state, shard_grad, fold, bwd = _shard_ops or (
+        lambda: gla_shard_state(k, v, g, igate, chunk=chunk),
+        lambda: gla_shard_state_grad(q, dO, g, scale=scale, chunk=chunk),
+        gla_state_fold,
+        lambda s_in, d_end: gla_bwd(q, k, v, g, igate, s_in, dO, d_end, scale=scale, chunk=chunk,
+                                    output_dh0=rank == 0))
+    S, gamma = shard_state()
+    dS, _ = shard_grad()
+    n_s, n_g = S.numel(), gamma.numel()
+    pack = torch.cat([S.reshape(-1), dS.reshape(-1), gamma.reshape(-1)])
+    parts = [torch.empty_like(pack) for _ in range(world)]
+    dist.all_gather(parts, pack, group=group)
+    allp = torch.stack(parts)
+    states = allp[:, :n_s].reshape(world, *S.shape)
+    grads = allp[:, n_s:2 * n_s].reshape(world, *S.shape)
+    gammas = allp[:, 2 * n_s:2 * n_s + n_g].reshape(world, *gamma.shape)
+    s_in = fold(states, gammas, rank, h0)
+    d_end = fold(grads.flip(0).contiguous(), gammas.flip(0).contiguous(), world - 1 - rank, dhT)
+    return bwd(s_in, d_end)
 
 
 def _check_saved(saved, prob):

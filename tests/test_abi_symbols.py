@@ -183,6 +183,19 @@ def test_shard_calls_validate_before_launch():
     assert shard(bf, k=24) == _lib.GLA_ERR_INVALID_ARG                   # misaligned
     assert shard(bf, nbytes=100) == _lib.GLA_ERR_WORKSPACE
 
+    def grad(p, **kw):
+        a = dict(q=16, dO=16, g=16, dS=16, gamma=16, ws=16, nbytes=256)
+        a.update(kw)
+        return _lib.lib.gla_shard_state_grad(ctypes.byref(p), *(vp(a[n]) for n in ("q", "dO", "g", "dS", "gamma",
+                                                                                   "ws")), a["nbytes"], None)
+    assert grad(prob(io=_lib.GLA_F32)) == _lib.GLA_ERR_UNSUPPORTED
+    assert grad(prob(chunk=96)) == _lib.GLA_ERR_UNSUPPORTED
+    assert grad(bf, dS=None) == _lib.GLA_ERR_INVALID_ARG
+    assert grad(bf, dO=None) == _lib.GLA_ERR_INVALID_ARG
+    assert grad(bf, g=None) == _lib.GLA_ERR_INVALID_ARG                  # gate mode says per-key
+    assert grad(bf, q=24) == _lib.GLA_ERR_INVALID_ARG                    # misaligned
+    assert grad(bf, nbytes=100) == _lib.GLA_ERR_WORKSPACE
+
     def fold(p, count, **kw):
         a = dict(states=16, gammas=16, h0=None, out=16)
         a.update(kw)

@@ -138,3 +138,73 @@ def test_sequence_sharded_forward_exchange_on_two_ranks():
         assert p.exitcode == 0
     for rank, err_o, err_h in res:
         assert err_o < 1e-10 and err_h < 1e-10, (rank, err_o, err_h)
+
+
+# ---------------------------------------------- sequence-sharded backward, exchange on CPU ranks
+def _shard_bwd_worker(rank, world, port, out):
+    """Three ranks, one contiguous shard each; the per-rank steps are the float64 oracle (the
+    start-state gradient from zero of a shard is the oracle's dh0 of that shard alone), so
+    this tests the single packed all-gather and both fold orders, not the kernels."""
+    import datetime
+
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=world,
+                                         timeout=datetime.timedelta(seconds=60))
+    import oracle
+    from linear_rnn_b200 import inputs as I
+    from linear_rnn_b200 import ops
+    w = I.WORKLOADS["c3"].replace(B=1, H=2, L=150, Dk=64, Dv=64, dtype="f32", input_gate=True, h0_std=0.5)
+    x = I.make_inputs(w, seed=8)
+    dhT = I.make_dhT(w, seed=9)
+    cuts = [0, 40, 41, 150]
+    sl = lambda t: None if t is None else t[:, :, cuts[rank]:cuts[rank + 1]].contiguous()
+    xs = {n: sl(x[n]) for n in ("q", "k", "v", "g", "igate", "dO")}
+
+    def shard_state():
+        _, S = oracle.gla_fwd(xs["q"], xs["k"], xs["v"], xs["g"], xs["igate"], None, w.scale)
+        return torch.from_numpy(S), xs["g"].double().sum(dim=2)
+
+    def shard_grad():
+        r = oracle.gla_bwd(xs["q"], xs["k"], xs["v"], xs["g"], xs["igate"], None, xs["dO"], None, w.scale)
+        return torch.from_numpy(r["dh0"]), xs["g"].double().sum(dim=2)
+
+    def fold(states, gammas, count, init):
+        S = torch.zeros_like(states[0]) if init is None else init.double().clone()
+        for p in range(count):
+            S = torch.exp(gammas[p])[..., None] * S + states[p]
+        return S
+
+    def bwd(s_in, d_end):
+        return oracle.gla_bwd(xs["q"], xs["k"], xs["v"], xs["g"], xs["igate"], s_in.numpy(), xs["dO"],
+                              d_end.numpy(), w.scale)
+
+    r = ops.gla_bwd_sequence_sharded(None, None, None, None, None, x["h0"], None, dhT,
+                                     _shard_ops=(shard_state, shard_grad, fold, bwd))
+    ref = oracle.gla_bwd(x["q"], x["k"], x["v"], x["g"], x["igate"], x["h0"], x["dO"], dhT, w.scale)
+    errs = {}
+    for n in ("dq", "dk", "dv", "dg", "di"):
+        part = ref[n][:, :, cuts[rank]:cuts[rank + 1]]
+        errs[n] = float(np.abs(r[n] - part).max() / np.abs(ref[n]).max())
+    if rank == 0:
+        errs["dh0"] = float(np.abs(r["dh0"] - ref["dh0"]).max() / np.abs(ref["dh0"]).max())
+    torch.distributed.barrier()
+    torch.distributed.destroy_process_group()
+    out.put((rank, errs))
+
+
+def test_sequence_sharded_backward_exchange_on_three_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_bwd_worker, args=(r, 3, port, q)) for r in range(3)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, errs in res:
+        assert (rank != 0) or "dh0" in errs
+        assert all(e < 1e-10 for e in errs.values()), (rank, errs)
