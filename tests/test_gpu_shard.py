@@ -103,7 +103,9 @@ def test_sharded_backward_equals_the_whole_sequence(gate, ig, Dk, Dv):
         s = {n: shard(xd[n], p) for n in names}
         S, gam = ops.gla_shard_state(s["k"], s["v"], s["g"], s["igate"], chunk=64)
         dS, gam2 = ops.gla_shard_state_grad(s["q"], s["dO"], s["g"], scale=w.scale, chunk=64)
-        assert torch.equal(gam, gam2)
+        # the forward-state pass sums the log-gates from the shard's end, the gradient pass from
+        # its start: the same float32 sum in another order
+        assert torch.allclose(gam, gam2, rtol=1e-5, atol=1e-4)
         hs = {n: shard(x[n], p) for n in names}
         rl = oracle.gla_bwd(hs["q"], hs["k"], hs["v"], hs["g"], hs["igate"], None, hs["dO"], None, w.scale)
         assert err(f64(dS), rl["dh0"]) <= TOL
