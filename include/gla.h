@@ -192,6 +192,23 @@ GLA_API gla_status gla_state_fold(const gla_problem* p, int count, const float* 
 GLA_API gla_status gla_shard_state_grad(const gla_problem* p, const void* q, const void* dO, const float* g,
                                         float* state_grad, float* gamma, void* ws, size_t ws_bytes, void* stream);
 
+/* Chunkwise DeltaNet (delta-rule) forward, after the talk summary "Hardware-Efficient Training of
+ * Linear Attention Models", sections 22:36 and 31:16 (writing strength beta_t; one gradient step
+ * per token on the key-to-value regression loss; the WY representation for the chunk form):
+ *   S_t = (I - beta_t k_t^T k_t) S_{t-1} + beta_t k_t^T v_t,   o_t = scale q_t S_t.
+ * p: B, H, L >= 0; Dk 64 or 128; Dv a multiple of 64 up to 4096; chunk = 64; scale; io bf16 or
+ *   f32; gate must be GLA_GATE_NONE (no decay gates); plan is ignored.
+ * q, k [B,H,L,Dk] and v [B,H,L,Dv] in io dtype; beta [B,H,L] f32; h0 [B,H,Dk,Dv] f32 or NULL
+ *   (zero); o [B,H,L,Dv] io dtype (written); hT [B,H,Dk,Dv] f32 or NULL (final state, written).
+ *   Keys are used as given (unit-norm keys with beta in [0, 1] keep each transition's
+ *   eigenvalues in [1 - beta, 1]). All pointers 16-byte aligned, device memory, owned by the
+ *   caller; no workspace. L = 0 copies h0 (or zero) to hT.
+ * CUDA cores, fp32 arithmetic; asynchronous on `stream`.
+ * Errors: GLA_ERR_INVALID_ARG (null or misaligned pointer, bad enum, a gate mode),
+ *   GLA_ERR_UNSUPPORTED (head dims, chunk), GLA_ERR_CUDA. */
+GLA_API gla_status gla_deltanet_fwd(const gla_problem* p, const void* q, const void* k, const void* v,
+                                    const float* beta, const float* h0, void* o, float* hT, void* stream);
+
 /* Static description of a status code (never NULL). */
 GLA_API const char* gla_status_string(gla_status s);
 

@@ -138,3 +138,24 @@ def small(w: Workload, B: int = 1, H: int = 2, L: Optional[int] = None) -> Workl
 
 def default_scale(Dk: int) -> float:
     return 1.0 / math.sqrt(Dk)
+
+
+def make_deltanet_inputs(B: int, H: int, L: int, Dk: int, Dv: int, dtype: str = "bf16", seed: int = 0,
+                         h0_std: float = 0.0) -> Dict[str, Optional[torch.Tensor]]:
+    """Inputs of the delta-rule (DeltaNet) forward, drawn on the CPU: q, v ~ N(0,1); k ~ N(0,1)
+    with each row scaled to unit L2 norm before rounding to the io dtype; beta =
+    sigmoid(N(0,1)) in (0, 1), fp32 [B,H,L]; h0 ~ N(0, h0_std^2) fp32 or None. The unit-norm
+    keys and beta in (0, 1) keep every transition I - beta k^T k contractive."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(20_000 + seed)
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=gen, dtype=torch.float32)
+
+    q = _round_io(randn(B, H, L, Dk), dtype)
+    k = randn(B, H, L, Dk)
+    k = _round_io(k / k.norm(dim=-1, keepdim=True).clamp_min(1e-6), dtype)
+    v = _round_io(randn(B, H, L, Dv), dtype)
+    beta = torch.sigmoid(randn(B, H, L))
+    h0 = randn(B, H, Dk, Dv) * h0_std if h0_std > 0 else None
+    return {"q": q, "k": k, "v": v, "beta": beta, "h0": h0}

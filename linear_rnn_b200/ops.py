@@ -149,6 +149,29 @@ def gla_decode(q, k, v, g, igate, state, *, scale: Optional[float] = None) -> to
     return o
 
 
+def gla_deltanet_fwd(q, k, v, beta, h0=None, *, scale: Optional[float] = None,
+                 output_final_state: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunkwise DeltaNet forward: q, k [B,H,L,Dk], v [B,H,L,Dv] (bf16 or fp32), beta [B,H,L]
+    fp32, h0 [B,H,Dk,Dv] fp32 or None. Returns o [B,H,L,Dv] and the final state (fp32, or None
+    when output_final_state is False). Host tensors are copied to the current device and the
+    results back."""
+    host = q.device.type != "cuda"
+    device = torch.device("cuda", torch.cuda.current_device()) if host else q.device
+    q, k, v, beta, h0 = (_to_dev(t, device) for t in (q, k, v, beta, h0))
+    if beta is None or beta.dtype != torch.float32 or tuple(beta.shape) != tuple(q.shape[:3]):
+        raise ValueError("beta must be float32 [B, H, L]")
+    prob = make_problem(q, v, None, scale=scale, chunk=64, plan="auto")
+    o = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=device)
+    hT = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
+                     device=device) if output_final_state else None
+    st = _lib.lib.gla_deltanet_fwd(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(h0), _ptr(o),
+                                   _ptr(hT), _stream_handle(device))
+    _check(st, "gla_deltanet_fwd")
+    if host:
+        o, hT = _to_host([o, hT])
+    return o, hT
+
+
 def gla_shard_state(k, v, g=None, igate=None, *, chunk: int = 64) -> Tuple[torch.Tensor, torch.Tensor]:
     """(state, gamma) of one sequence shard: its end state from a zero initial state
     [B,H,Dk,Dv] and its total log-decay per key dim [B,H,Dk], both fp32 on the GPU."""

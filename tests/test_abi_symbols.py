@@ -208,6 +208,30 @@ def test_shard_calls_validate_before_launch():
     assert fold(prob(Dv=96), 1) == _lib.GLA_ERR_UNSUPPORTED
 
 
+def test_deltanet_validates_before_launch():
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+
+    def call(p, **kw):
+        a = dict(q=16, k=16, v=16, beta=16, h0=None, o=16, hT=None)
+        a.update(kw)
+        return _lib.lib.gla_deltanet_fwd(ctypes.byref(p), *(vp(a[n]) for n in ("q", "k", "v", "beta", "h0", "o",
+                                                                              "hT")), None)
+    dn = lambda **kw: prob(**dict(dict(gate=_lib.GLA_GATE_NONE, Dk=64, Dv=64), **kw))
+    assert call(dn(gate=_lib.GLA_GATE_PER_KEY)) == _lib.GLA_ERR_INVALID_ARG   # no decay gates
+    assert call(dn(io=7)) == _lib.GLA_ERR_INVALID_ARG
+    assert call(dn(Dk=256)) == _lib.GLA_ERR_UNSUPPORTED
+    assert call(dn(Dv=96)) == _lib.GLA_ERR_UNSUPPORTED                        # 64-column slices
+    assert call(dn(chunk=128)) == _lib.GLA_ERR_UNSUPPORTED
+    assert call(dn(), beta=None) == _lib.GLA_ERR_INVALID_ARG
+    assert call(dn(), o=None) == _lib.GLA_ERR_INVALID_ARG
+    assert call(dn(), k=24) == _lib.GLA_ERR_INVALID_ARG                       # misaligned
+    assert call(dn(), hT=8) == _lib.GLA_ERR_INVALID_ARG
+    assert call(dn(L=-1)) == _lib.GLA_ERR_INVALID_ARG
+    assert call(dn(B=0)) == _lib.GLA_OK                                      # nothing to do, no launch
+    assert _lib.lib.gla_deltanet_fwd(None, None, None, None, None, None, None, None, None) == \
+        _lib.GLA_ERR_INVALID_ARG
+
+
 def test_debug_wait_timeout_validates_before_launch():
     assert _lib.lib.gla_debug_wait_timeout(None, 100, None) == _lib.GLA_ERR_INVALID_ARG
     assert _lib.lib.gla_debug_wait_timeout(ctypes.c_void_p(24), 100, None) == _lib.GLA_ERR_INVALID_ARG  # misaligned

@@ -1,0 +1,88 @@
+"""Parity of the chunkwise DeltaNet forward (gla_deltanet_fwd) with the float64 delta-rule
+oracle (oracle/deltanet.py, pinned in test_oracle_deltanet.py), element by element, on seeded
+inputs: unit-norm keys, beta = sigmoid(N(0,1)). Cases span several 64-token chunks and a ragged
+tail, both key widths, several 64-column value slices, with and without h0, and the edge
+lengths L = 0, 1 and 64. Bound: the max-normalised error, 1e-4 for fp32 I/O and 1e-2 for bf16
+(the fp32 kernel against float64: rounding only; bf16 adds the output's rounding)."""
+import numpy as np
+import pytest
+import torch
+
+from linear_rnn_b200 import inputs as I
+from oracle import deltanet as DN
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 1e-2}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def f64(t):
+    return None if t is None else t.detach().to("cpu", torch.float64).numpy()
+
+
+def err(got, ref):
+    return float(np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-30))
+
+
+def check(B, H, L, Dk, Dv, dtype, h0_std, seed=0):
+    from linear_rnn_b200 import ops
+    x = I.make_deltanet_inputs(B, H, L, Dk, Dv, dtype, seed=seed, h0_std=h0_std)
+    xd = {n: (None if t is None else t.cuda()) for n, t in x.items()}
+    scale = Dk ** -0.5
+    o, hT = ops.gla_deltanet_fwd(xd["q"], xd["k"], xd["v"], xd["beta"], xd["h0"], scale=scale)
+    torch.cuda.synchronize()
+    ro, rS = DN.deltanet_fwd(x["q"], x["k"], x["v"], x["beta"], x["h0"], scale)
+    if L:
+        assert err(f64(o), ro) <= TOL[dtype]
+    assert err(f64(hT), rS) <= TOL[dtype]
+    return o, hT
+
+
+@pytest.mark.parametrize("B,H,L,Dk,Dv,dtype,h0_std", [
+    (1, 2, 150, 64, 64, "f32", 0.5),
+    (2, 1, 300, 128, 128, "bf16", 0.5),
+    (1, 3, 200, 128, 256, "bf16", 0.0),
+    (1, 2, 333, 128, 64, "f32", 1.0),
+    (2, 2, 64, 64, 192, "bf16", 0.5),
+])
+def test_parity(B, H, L, Dk, Dv, dtype, h0_std):
+    check(B, H, L, Dk, Dv, dtype, h0_std)
+
+
+@pytest.mark.parametrize("L", [1, 63, 65])
+def test_edge_lengths(L):
+    check(1, 2, L, 64, 64, "f32", 0.5, seed=3)
+
+
+def test_empty_sequence_returns_h0():
+    from linear_rnn_b200 import ops
+    q = torch.zeros(1, 2, 0, 64, dtype=torch.bfloat16, device="cuda")
+    v = torch.zeros(1, 2, 0, 128, dtype=torch.bfloat16, device="cuda")
+    beta = torch.zeros(1, 2, 0, device="cuda")
+    h0 = torch.randn(1, 2, 64, 128, device="cuda")
+    o, hT = ops.gla_deltanet_fwd(q, q, v, beta, h0)
+    assert o.shape == (1, 2, 0, 128) and torch.equal(hT, h0)
+    _, hz = ops.gla_deltanet_fwd(q, q, v, beta, None)
+    assert not torch.any(hz)
+
+
+def test_long_sequence():
+    # 32 chunks: the state hand-off between chunks over a long walk
+    check(2, 4, 2048, 128, 128, "bf16", 0.5, seed=5)
+
+
+def test_deterministic_and_host_round_trip():
+    from linear_rnn_b200 import ops
+    x = I.make_deltanet_inputs(1, 2, 257, 128, 128, "bf16", seed=9, h0_std=0.5)
+    xd = {n: t.cuda() for n, t in x.items()}
+    o1, h1 = ops.gla_deltanet_fwd(xd["q"], xd["k"], xd["v"], xd["beta"], xd["h0"])
+    o2, h2 = ops.gla_deltanet_fwd(xd["q"], xd["k"], xd["v"], xd["beta"], xd["h0"])
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+    oh, hh = ops.gla_deltanet_fwd(x["q"], x["k"], x["v"], x["beta"], x["h0"])
+    assert oh.device.type == "cpu" and torch.equal(oh, o1.cpu()) and torch.equal(hh, h1.cpu())

@@ -246,3 +246,15 @@ def test_planted_mistake_is_caught(i):
         except AssertionError:
             caught.append(pin.__name__)
     assert caught, f"mutant {i} passed every pin"
+
+
+def test_input_recipe():
+    """The generator's keys have unit norm up to bf16 rounding and beta lies in (0, 1)."""
+    import torch
+    from linear_rnn_b200 import inputs as I
+    x = I.make_deltanet_inputs(2, 3, 100, 64, 128, "bf16", seed=1, h0_std=0.5)
+    n = x["k"].float().norm(dim=-1)
+    assert torch.all((n - 1).abs() < 1e-2)
+    assert torch.all(x["beta"] > 0) and torch.all(x["beta"] < 1)
+    assert x["q"].dtype == torch.bfloat16 and x["beta"].dtype == torch.float32
+    assert x["h0"].shape == (2, 3, 64, 128)
