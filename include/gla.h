@@ -209,6 +209,23 @@ GLA_API gla_status gla_shard_state_grad(const gla_problem* p, const void* q, con
 GLA_API gla_status gla_deltanet_fwd(const gla_problem* p, const void* q, const void* k, const void* v,
                                     const float* beta, const float* h0, void* o, float* hT, void* stream);
 
+/* DeltaNet backward: gradients of sum(dO * o) + sum(dhT * hT) for gla_deltanet_fwd's inputs.
+ * The chunk form runs in reverse: dX = scale P^T dO + K dS', dR = T^T dX, dV = diag(beta) dR,
+ * dS <- dS' + scale Q^T dO - K^T diag(beta) dR (P = lower(Q K^T), T, X as in the forward, dS'
+ * the gradient at the chunk's end), then per chunk dQ, dK, dbeta from those products.
+ * Same p and inputs as gla_deltanet_fwd; dO [B,H,L,Dv] io dtype; dhT [B,H,Dk,Dv] f32 or NULL.
+ * Outputs (written): dq, dk [B,H,L,Dk] and dv [B,H,L,Dv] io dtype; dbeta [B,H,L] f32; dh0
+ * [B,H,Dk,Dv] f32 or NULL. ws: device workspace of gla_deltanet_bwd_workspace_bytes(p) bytes
+ * (the chunk start states, X, dR, the chunk end gradients and per-slice sums), caller-owned.
+ * Three launches on `stream` (the forward's state pass, the reverse walk, the per-chunk
+ * gradients). B*H at most 65535.
+ * Errors: as gla_deltanet_fwd, plus GLA_ERR_WORKSPACE. */
+GLA_API size_t gla_deltanet_bwd_workspace_bytes(const gla_problem* p);
+GLA_API gla_status gla_deltanet_bwd(const gla_problem* p, const void* q, const void* k, const void* v,
+                                    const float* beta, const float* h0, const void* dO, const float* dhT,
+                                    void* dq, void* dk, void* dv, float* dbeta, float* dh0, void* ws,
+                                    size_t ws_bytes, void* stream);
+
 /* Static description of a status code (never NULL). */
 GLA_API const char* gla_status_string(gla_status s);
 

@@ -21,7 +21,8 @@ EXPORTED = ("gla_workspace_bytes", "gla_fwd", "gla_bwd", "gla_status_string",
             "gla_check_device_status", "gla_version", "gla_launch_count", "gla_profiler_enable",
             "gla_profiler_read", "gla_fwd_static_scratch", "gla_last_error_detail", "gla_plan_info",
             "gla_saved_states_bytes", "gla_fwd_save", "gla_bwd_saved", "gla_debug_wait_timeout",
-            "gla_decode", "gla_shard_state", "gla_state_fold", "gla_shard_state_grad", "gla_deltanet_fwd")
+            "gla_decode", "gla_shard_state", "gla_state_fold", "gla_shard_state_grad", "gla_deltanet_fwd",
+            "gla_deltanet_bwd_workspace_bytes", "gla_deltanet_bwd")
 
 
 class GlaProblem(ctypes.Structure):
@@ -82,6 +83,10 @@ def _load():
     lib.gla_shard_state_grad.restype = ctypes.c_int
     lib.gla_deltanet_fwd.argtypes = [pp] + [ctypes.c_void_p] * 8
     lib.gla_deltanet_fwd.restype = ctypes.c_int
+    lib.gla_deltanet_bwd_workspace_bytes.argtypes = [pp]
+    lib.gla_deltanet_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.gla_deltanet_bwd.argtypes = [pp] + [ctypes.c_void_p] * 13 + [ctypes.c_size_t, ctypes.c_void_p]
+    lib.gla_deltanet_bwd.restype = ctypes.c_int
     lib.gla_state_fold.argtypes = [pp, ctypes.c_int] + [ctypes.c_void_p] * 5
     lib.gla_state_fold.restype = ctypes.c_int
     lib.gla_decode.argtypes = [pp] + [ctypes.c_void_p] * 8

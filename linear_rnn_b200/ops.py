@@ -172,6 +172,36 @@ def gla_deltanet_fwd(q, k, v, beta, h0=None, *, scale: Optional[float] = None,
     return o, hT
 
 
+def gla_deltanet_bwd(q, k, v, beta, h0, dO, dhT=None, *, scale: Optional[float] = None,
+                     output_dh0: bool = True) -> Dict[str, Optional[torch.Tensor]]:
+    """DeltaNet backward: dict dq, dk, dv (io dtype), dbeta (fp32 [B,H,L]) and dh0 (fp32, or
+    None when output_dh0 is False). Host tensors are copied to the current device and the
+    results back."""
+    host = q.device.type != "cuda"
+    device = torch.device("cuda", torch.cuda.current_device()) if host else q.device
+    q, k, v, beta, h0, dO, dhT = (_to_dev(t, device) for t in (q, k, v, beta, h0, dO, dhT))
+    if beta is None or beta.dtype != torch.float32 or tuple(beta.shape) != tuple(q.shape[:3]):
+        raise ValueError("beta must be float32 [B, H, L]")
+    prob = make_problem(q, v, None, scale=scale, chunk=64, plan="auto")
+    nbytes = _lib.lib.gla_deltanet_bwd_workspace_bytes(ctypes.byref(prob))
+    if nbytes == 0:
+        raise GlaError(_lib.GLA_ERR_UNSUPPORTED, "gla_deltanet_bwd_workspace_bytes")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dbeta = torch.empty_like(beta)
+    dh0 = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
+                      device=device) if output_dh0 else None
+    st = _lib.lib.gla_deltanet_bwd(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(h0), _ptr(dO),
+                                   _ptr(dhT), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dbeta), _ptr(dh0), _ptr(ws),
+                                   nbytes, _stream_handle(device))
+    _check(st, "gla_deltanet_bwd")
+    out = {"dq": dq, "dk": dk, "dv": dv, "dbeta": dbeta, "dh0": dh0}
+    if host:
+        names = list(out)
+        out = dict(zip(names, _to_host([out[n] for n in names])))
+    return out
+
+
 def gla_shard_state(k, v, g=None, igate=None, *, chunk: int = 64) -> Tuple[torch.Tensor, torch.Tensor]:
     """(state, gamma) of one sequence shard: its end state from a zero initial state
     [B,H,Dk,Dv] and its total log-decay per key dim [B,H,Dk], both fp32 on the GPU."""

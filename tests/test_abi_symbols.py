@@ -232,6 +232,35 @@ def test_deltanet_validates_before_launch():
         _lib.GLA_ERR_INVALID_ARG
 
 
+def test_deltanet_backward_validates_before_launch():
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    names = ("q", "k", "v", "beta", "h0", "dO", "dhT", "dq", "dk", "dv", "dbeta", "dh0", "ws")
+
+    def call(p, **kw):
+        a = dict(q=16, k=16, v=16, beta=16, h0=None, dO=16, dhT=None, dq=16, dk=16, dv=16, dbeta=16, dh0=None,
+                 ws=16, nbytes=1 << 40)
+        a.update(kw)
+        return _lib.lib.gla_deltanet_bwd(ctypes.byref(p), *(vp(a[n]) for n in names), a["nbytes"], None)
+    dn = lambda **kw: prob(**dict(dict(gate=_lib.GLA_GATE_NONE, Dk=64, Dv=64), **kw))
+    need = _lib.lib.gla_deltanet_bwd_workspace_bytes(ctypes.byref(dn()))
+    # chunk start states and end gradients (2 x B*H*5 chunks*Dk*Dv), X and dR (2 x B*H*L*Dv),
+    # per-slice sums (B*H*L), each region rounded up to 256 bytes
+    BH, L = 6, 300
+    parts = [BH * 5 * 64 * 64, BH * L * 64, BH * L * 64, BH * 5 * 64 * 64, BH * L]
+    assert need == sum((4 * n + 255) // 256 * 256 for n in parts)
+    assert _lib.lib.gla_deltanet_bwd_workspace_bytes(ctypes.byref(dn(Dk=256))) == 0
+    assert _lib.lib.gla_deltanet_bwd_workspace_bytes(ctypes.byref(dn(L=0))) == 256   # empty, still usable
+    assert call(dn(), nbytes=need - 1) == _lib.GLA_ERR_WORKSPACE
+    assert call(dn(), ws=None) == _lib.GLA_ERR_WORKSPACE
+    assert call(dn(gate=_lib.GLA_GATE_PER_HEAD)) == _lib.GLA_ERR_INVALID_ARG
+    assert call(dn(Dv=32)) == _lib.GLA_ERR_UNSUPPORTED
+    assert call(dn(B=300, H=300)) == _lib.GLA_ERR_UNSUPPORTED             # B*H above 65535
+    assert call(dn(), dO=None) == _lib.GLA_ERR_INVALID_ARG
+    assert call(dn(), dbeta=None) == _lib.GLA_ERR_INVALID_ARG
+    assert call(dn(), dq=8) == _lib.GLA_ERR_INVALID_ARG                   # misaligned
+    assert call(dn(H=0)) == _lib.GLA_OK
+
+
 def test_debug_wait_timeout_validates_before_launch():
     assert _lib.lib.gla_debug_wait_timeout(None, 100, None) == _lib.GLA_ERR_INVALID_ARG
     assert _lib.lib.gla_debug_wait_timeout(ctypes.c_void_p(24), 100, None) == _lib.GLA_ERR_INVALID_ARG  # misaligned

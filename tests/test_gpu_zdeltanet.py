@@ -1,6 +1,6 @@
-"""Parity of the chunkwise DeltaNet forward (gla_deltanet_fwd) with the float64 delta-rule
-oracle (oracle/deltanet.py, pinned in test_oracle_deltanet.py), element by element, on seeded
-inputs: unit-norm keys, beta = sigmoid(N(0,1)). Cases span several 64-token chunks and a ragged
+"""Parity of the chunkwise DeltaNet forward (gla_deltanet_fwd) and backward (gla_deltanet_bwd)
+with the float64 delta-rule oracle (oracle/deltanet.py: the recurrence and its back-propagation
+through time, pinned in test_oracle_deltanet.py), element by element, on seeded inputs: unit-norm keys, beta = sigmoid(N(0,1)). Cases span several 64-token chunks and a ragged
 tail, both key widths, several 64-column value slices, with and without h0, and the edge
 lengths L = 0, 1 and 64. Bound: the max-normalised error, 1e-4 for fp32 I/O and 1e-2 for bf16
 (the fp32 kernel against float64: rounding only; bf16 adds the output's rounding)."""
@@ -86,3 +86,42 @@ def test_deterministic_and_host_round_trip():
     assert torch.equal(o1, o2) and torch.equal(h1, h2)
     oh, hh = ops.gla_deltanet_fwd(x["q"], x["k"], x["v"], x["beta"], x["h0"])
     assert oh.device.type == "cpu" and torch.equal(oh, o1.cpu()) and torch.equal(hh, h1.cpu())
+
+
+def check_bwd(B, H, L, Dk, Dv, dtype, h0_std, with_dhT, seed=0):
+    from linear_rnn_b200 import ops
+    x = I.make_deltanet_inputs(B, H, L, Dk, Dv, dtype, seed=seed, h0_std=h0_std)
+    gen = torch.Generator().manual_seed(100 + seed)
+    dO = torch.randn(B, H, L, Dv, generator=gen).to(x["q"].dtype)
+    dhT = torch.randn(B, H, Dk, Dv, generator=gen) if with_dhT else None
+    xd = {n: (None if t is None else t.cuda()) for n, t in x.items()}
+    scale = Dk ** -0.5
+    r = ops.gla_deltanet_bwd(xd["q"], xd["k"], xd["v"], xd["beta"], xd["h0"], dO.cuda(),
+                             None if dhT is None else dhT.cuda(), scale=scale)
+    torch.cuda.synchronize()
+    ref = DN.deltanet_bwd(x["q"], x["k"], x["v"], x["beta"], x["h0"], dO, dhT, scale)
+    for name in ("dq", "dk", "dv", "dbeta", "dh0"):
+        if ref[name].size:
+            assert err(f64(r[name]), ref[name]) <= TOL[dtype], name
+    return r
+
+
+@pytest.mark.parametrize("B,H,L,Dk,Dv,dtype,h0_std,with_dhT", [
+    (1, 2, 150, 64, 64, "f32", 0.5, True),
+    (2, 1, 300, 128, 128, "bf16", 0.5, True),
+    (1, 3, 200, 128, 256, "bf16", 0.0, False),
+    (1, 2, 333, 128, 64, "f32", 1.0, False),
+    (2, 2, 64, 64, 192, "bf16", 0.5, True),
+])
+def test_backward_parity(B, H, L, Dk, Dv, dtype, h0_std, with_dhT):
+    check_bwd(B, H, L, Dk, Dv, dtype, h0_std, with_dhT)
+
+
+@pytest.mark.parametrize("L", [0, 1, 63, 65])
+def test_backward_edge_lengths(L):
+    r = check_bwd(1, 2, L, 64, 64, "f32", 0.5, True, seed=7)
+    assert r["dq"].shape == (1, 2, L, 64)
+
+
+def test_backward_long_sequence():
+    check_bwd(1, 4, 2048, 128, 128, "bf16", 0.5, True, seed=8)
