@@ -269,7 +269,7 @@ def max_over_ranks(value: float, device) -> float:
 def base_line(w, args, world):
     return {"metric": "GLA chunkwise fwd/bwd tokens/s", "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded; workload recipe in DESIGN.md)",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded; linear_rnn_b200/inputs.py)",
             "config": {"workload": f"{w.name}: {'GLA decode step' if w.name == 'decode' else 'GLA forward+backward' if w.backward else 'GLA forward'}, "
                                    f"B={w.B} H={w.H} L={w.L} Dk={w.Dk} Dv={w.Dv} chunk={w.chunk} {w.dtype}",
                        "global_batch": w.B * world, "seq_len": w.L, "parallelism": f"replicas x{world}",

@@ -124,4 +124,4 @@ def test_backward_edge_lengths(L):
 
 
 def test_backward_long_sequence():
-    check_bwd(1, 4, 2048, 128, 128, "bf16", 0.5, True, seed=8)
+    check_bwd(1, 2, 2048, 128, 128, "bf16", 0.5, True, seed=8)
