@@ -300,12 +300,189 @@ def run_reference(args, w, world, rank):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ DeltaNet workload
+DN_C = 64
+
+
+def deltanet_kernel_flops(name, B, H, L, Dk, Dv):
+    """Algorithmic FLOPs of one launch (per token-head, multiplied by B*H*L): causal C x C
+    products count their lower half, K K^T and Q K^T once per head (not per value slice), the
+    chunk's triangular inverse C^2/3 per token."""
+    C = DN_C
+    per = {
+        # K K^T, Q K^T; K S, Q S, K^T X; T R, lower(Q K^T) X; the inverse
+        "deltanet_fwd": 2 * C * Dk + 6 * Dk * Dv + 2 * C * Dv + C * C / 3,
+        # K K^T, P; K S, K dS', the dS update (2 products); P^T dO, T R, T^T dX; the inverse
+        "deltanet_bwd_walk": 2 * C * Dk + 8 * Dk * Dv + 3 * C * Dv + C * C / 3,
+        # dO X^T, dR X^T; dO S^T, X dS'^T, dR S^T; dP K, dP^T Q, G K, G^T (beta K)
+        "deltanet_bwd_grads": 2 * C * Dv + 6 * Dk * Dv + 4 * C * Dk,
+    }
+    return float(per.get(name, 0.0)) * B * H * L
+
+
+def deltanet_alu_peak_tflops(sm_mhz):
+    """FP32 FMA peak from the unit counts: 148 SMs x 128 FP32 lanes x 2 FLOPs x the SM clock."""
+    return 148 * 128 * 2 * (sm_mhz or 1965.0) * 1e6 / 1e12
+
+
+def deltanet_line(args, world, tokens, ms, extra):
+    cfg = I.DELTANET
+    line = {"metric": "DeltaNet chunkwise fwd+bwd tokens/s", "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; linear_rnn_b200/inputs.py)",
+            "config": {"workload": "deltanet: DeltaNet forward+backward, B={B} H={H} L={L} Dk={Dk} Dv={Dv} "
+                                   "chunk=64 {dtype} I/O".format(**cfg),
+                       "global_batch": cfg["B"] * world, "seq_len": cfg["L"], "parallelism": f"replicas x{world}",
+                       "l2": "256 MiB L2 flush between steps, outside the per-step events; inputs > L2"},
+            "value": tokens / (ms / 1e3), "ms_per_step": ms / args.steps}
+    line.update(extra)
+    return line
+
+
+def deltanet_oracle_sample(seed, heads):
+    """Times the float64 delta-rule oracle (forward, then back-propagation through time) on
+    `heads` whole heads. Returns (tokens_equivalent, seconds)."""
+    from oracle import deltanet as DN
+    cfg = I.DELTANET
+    x = I.make_deltanet_inputs(1, heads, cfg["L"], cfg["Dk"], cfg["Dv"], cfg["dtype"], seed=seed, h0_std=0.5)
+    dO = torch.randn(1, heads, cfg["L"], cfg["Dv"], generator=torch.Generator().manual_seed(seed))
+    sc = cfg["Dk"] ** -0.5
+    t0 = time.perf_counter()
+    DN.deltanet_fwd(x["q"], x["k"], x["v"], x["beta"], x["h0"], sc)
+    DN.deltanet_bwd(x["q"], x["k"], x["v"], x["beta"], x["h0"], dO, None, sc)
+    return cfg["L"] * heads / cfg["H"], time.perf_counter() - t0
+
+
+def run_deltanet(args, world, rank, local):
+    cfg = I.DELTANET
+    heads = 1   # the oracle keeps every state of a head (L x Dk x Dv float64): one head per sample
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        for _ in range(args.warmup):
+            deltanet_oracle_sample(0, heads)
+        tok = tot = 0.0
+        for i in range(args.steps):
+            t, dt = deltanet_oracle_sample(i, heads)
+            tok += t
+            tot += dt
+        val = tok / tot
+        base = deltanet_line(args, 1, tok, 1e3 * tot, {})
+        base.update({"impl": "reference", "value": val, "dtype": "f64", "gpu_launches": 0,
+                     "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": torch.get_num_threads(),
+                                      "kind": "oracle", "sample": f"{heads} of {cfg['B'] * cfg['H']} heads, "
+                                                                  f"full L={cfg['L']}, fwd+bwd per step"},
+                     "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
+        print(json.dumps(base), flush=True)
+        return
+
+    from linear_rnn_b200 import _lib, ops
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B, H, L, Dk, Dv = cfg["B"], cfg["H"], cfg["L"], cfg["Dk"], cfg["Dv"]
+    x = I.make_deltanet_inputs(B, H, L, Dk, Dv, cfg["dtype"], seed=rank, h0_std=0.5)
+    dO = torch.randn(B, H, L, Dv, generator=torch.Generator().manual_seed(1000 + rank)).to(x["q"].dtype)
+    xd = {n: t.to(dev) for n, t in x.items()}
+    dOd = dO.to(dev)
+    sc = Dk ** -0.5
+
+    def step():
+        ops.gla_deltanet_fwd(xd["q"], xd["k"], xd["v"], xd["beta"], xd["h0"], scale=sc)
+        ops.gla_deltanet_bwd(xd["q"], xd["k"], xd["v"], xd["beta"], xd["h0"], dOd, None, scale=sc)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        step()
+    torch.cuda.synchronize()
+
+    def timed(per_kernel):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        n0 = _lib.launch_count()
+        _lib.profiler_enable(per_kernel)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record()
+            step()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        _lib.profiler_enable(False)
+        return sum(a.elapsed_time(b) for a, b in ev), _lib.launch_count() - n0, (_lib.profiler_read() if per_kernel
+                                                                                 else {})
+
+    total_ms, launches, _ = timed(False)
+    _, _, kprof = timed(True)
+    clocks = sampler.stop()
+    total_ms = max_over_ranks(total_ms, dev)
+    tokens = B * L * args.steps * world
+
+    e2e = None
+    if not args.no_e2e:
+        xh = {n: t.pin_memory() for n, t in x.items()}
+        dOh = dO.pin_memory()
+        h2d = 2 * sum(t.numel() * t.element_size() for t in xh.values()) + dOh.numel() * dOh.element_size()
+        d2h = 0
+
+        def e2e_step():
+            nonlocal d2h
+            o, hT = ops.gla_deltanet_fwd(xh["q"], xh["k"], xh["v"], xh["beta"], xh["h0"], scale=sc)
+            r = ops.gla_deltanet_bwd(xh["q"], xh["k"], xh["v"], xh["beta"], xh["h0"], dOh, None, scale=sc)
+            d2h = sum(t.numel() * t.element_size() for t in [o, hT, *r.values()] if t is not None)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(args.steps):
+            e2e_step()
+        s1.record()
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(s0.elapsed_time(s1), dev)
+        e2e = {"value": tokens / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h)}
+
+    if rank != 0:
+        return
+    peak = deltanet_alu_peak_tflops(clocks.get("sm_max_mhz"))
+    roofline = None
+    if kprof:
+        name, (cnt, ms) = max(kprof.items(), key=lambda kv: kv[1][1])
+        avg_s = ms / cnt / 1e3
+        fl = deltanet_kernel_flops(name, B, H, L, Dk, Dv)
+        # the forward kernel runs twice per step: with its output, and as the backward's state pass
+        ach = fl / avg_s / 1e12
+        roofline = {"bound": "alu", "kernel": name, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                    "frac": ach / peak, "traffic": None,
+                    "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 FLOPs x max SM clock",
+                    "algorithmic_flops_per_launch": fl, "avg_launch_us": avg_s * 1e6,
+                    "share_of_step": ms / sum(v[1] for v in kprof.values())}
+    extra = {"e2e": e2e, "gpu_launches": int(launches), "roofline": roofline, "clocks": clocks,
+             "kernels": {n: {"launches": c, "avg_us": 1e3 * m / c} for n, (c, m) in sorted(kprof.items())}}
+    if world == 1 and not args.no_cpu_baseline:
+        tk, dt = deltanet_oracle_sample(0, heads)
+        extra["cpu_baseline"] = {"value": tk / dt, "unit": "tokens/s", "cores": torch.get_num_threads(),
+                                 "kind": "oracle", "sample": f"{heads} of {B * H} heads, full L={L}, fwd+bwd, "
+                                                             f"float64 numpy, {dt:.1f} s"}
+    print(json.dumps(deltanet_line(args, world, tokens, total_ms, extra)), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="c3", choices=sorted(I.WORKLOADS) + ["decode"])
+    ap.add_argument("--workload", default="c3", choices=sorted(I.WORKLOADS) + ["decode", "deltanet"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--plan", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--no-e2e", action="store_true")
@@ -315,6 +492,12 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.workload == "deltanet":
+        world, rank, local = dist_setup()
+        run_deltanet(args, world, rank, local)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     w = I.DECODE if args.workload == "decode" else I.WORKLOADS[args.workload]
     decode = w.name == "decode"
     if args.batch is not None:

@@ -159,3 +159,8 @@ def make_deltanet_inputs(B: int, H: int, L: int, Dk: int, Dv: int, dtype: str = 
     beta = torch.sigmoid(randn(B, H, L))
     h0 = randn(B, H, Dk, Dv) * h0_std if h0_std > 0 else None
     return {"q": q, "k": k, "v": v, "beta": beta, "h0": h0}
+
+
+# DeltaNet forward+backward: the pages give the method but no benchmark shape, so this takes
+# the gated workloads' batch and length with square heads (Dk = Dv = 128), bf16 I/O.
+DELTANET = dict(B=4, H=16, L=4096, Dk=128, Dv=128, dtype="bf16")

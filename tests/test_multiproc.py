@@ -71,6 +71,25 @@ def test_reference_arm_json_contract():
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["value"] > 0
 
 
+def test_deltanet_reference_arm_and_flop_model():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                        "deltanet", "--steps", "1", "--warmup", "3"], capture_output=True, text=True, timeout=600,
+                       cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"].startswith("DeltaNet") and d["value"] > 0
+    assert d["config"]["workload"].startswith("deltanet:") and d["e2e"]["d2h_bytes_per_step"] == 0
+    sys.path.insert(0, ROOT)
+    import bench
+    # per token-head at C = 64, Dk = Dv = 128: 2*64*128 + 6*128^2 + 2*64*128 + 64^2/3
+    per = 2 * 64 * 128 + 6 * 128 * 128 + 2 * 64 * 128 + 64 * 64 / 3
+    assert bench.deltanet_kernel_flops("deltanet_fwd", 1, 2, 10, 128, 128) == per * 20
+    assert bench.deltanet_kernel_flops("other", 1, 1, 1, 64, 64) == 0.0
+    assert abs(bench.deltanet_alu_peak_tflops(1965.0) - 74.45) < 0.01
+
+
 def test_reference_arm_under_torchrun_two_ranks():
     port = _free_port()
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
