@@ -312,6 +312,8 @@ def deltanet_kernel_flops(name, B, H, L, Dk, Dv):
     per = {
         # K K^T, Q K^T; K S, Q S, K^T X; T R, lower(Q K^T) X; the inverse
         "deltanet_fwd": 2 * C * Dk + 6 * Dk * Dv + 2 * C * Dv + C * C / 3,
+        # the backward's state pass (no output): K K^T; K S, K^T X; T R; the inverse
+        "deltanet_state": C * Dk + 4 * Dk * Dv + C * Dv + C * C / 3,
         # K K^T, P; K S, K dS', the dS update (2 products); P^T dO, T R, T^T dX; the inverse
         "deltanet_bwd_walk": 2 * C * Dk + 8 * Dk * Dv + 3 * C * Dv + C * C / 3,
         # dO X^T, dR X^T; dO S^T, X dS'^T, dR S^T; dP K, dP^T Q, G K, G^T (beta K)
@@ -460,7 +462,6 @@ def run_deltanet(args, world, rank, local):
         name, (cnt, ms) = max(kprof.items(), key=lambda kv: kv[1][1])
         avg_s = ms / cnt / 1e3
         fl = deltanet_kernel_flops(name, B, H, L, Dk, Dv)
-        # the forward kernel runs twice per step: with its output, and as the backward's state pass
         ach = fl / avg_s / 1e12
         roofline = {"bound": "alu", "kernel": name, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                     "frac": ach / peak, "traffic": None,

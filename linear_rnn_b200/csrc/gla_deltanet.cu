@@ -252,7 +252,8 @@ cudaError_t dn_launch(const gla_problem* p, const void* q, const void* k, const 
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(p->B * p->H, p->Dv / DN_VT);
-    GLA_LAUNCH("deltanet_fwd", st,
+    // without an output it is the backward's state pass: timed under its own name
+    GLA_LAUNCH(o ? "deltanet_fwd" : "deltanet_state", st,
                (kern<<<grid, DN_NT, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
                                                 static_cast<const T*>(v), beta, h0, static_cast<T*>(o), hT, saved,
                                                 p->L, p->Dv, p->scale)));
