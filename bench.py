@@ -80,9 +80,13 @@ def _mean(xs):
 
 
 def kernel_bytes(name, w, fseg=1, bseg=1):
-    """Algorithmic bytes of one launch of each kernel: its own inputs read once and its
-    outputs written once, workspace tensors it exchanges with other kernels included.
-    fseg / bseg: sequence segments of the forward / backward plan (gla_plan_info)."""
+    """Bytes of one launch of each kernel, split in two:
+    method: the path's own inputs the kernel reads and outputs it writes, each once (q, k, v,
+            dO, g, i, h0, dhT in; o, hT, dq, dk, dv, dg, di, dh0 out);
+    plan:   the plan's intermediates it reads or writes in the workspace (segment states and
+            log-decay totals, the dq kernel's in-segment prefixes of q*dq, saved states).
+    fseg / bseg: sequence segments of the forward / backward plan (gla_plan_info). Returns
+    (method, plan)."""
     th = w.B * w.H * w.L
     BH = w.B * w.H
     e = io_bytes(w)
@@ -95,49 +99,51 @@ def kernel_bytes(name, w, fseg=1, bseg=1):
     q = k = th * w.Dk * e
     v = o = th * w.Dv * e
     dgb = 4 * th * gate_elems(w)                 # fp32 dg (or its in-segment prefix)
-    frac_f = (fseg - 1) / fseg                    # share of the sequence the state passes cover
+    gam = 4.0 * BH * w.Dk                        # one segment's log-decay totals
+    frac_f = (fseg - 1) / fseg                   # share of the sequence the state passes cover
     frac_b = (bseg - 1) / bseg
+    di = ig
     table = {
-        "simt_cumsum": 2 * ge,
-        "simt_state": k + v + ge + states,
-        "simt_out": q + k + v + ge + states + o,
-        "simt_dstate": q + o + ge + states,
-        "simt_dq": q + k + v + o + ge + states + q + 4 * th * w.Dk,
-        "simt_dk": q + k + v + o + ge + states + k + 2 * 4 * th * w.Dk,
-        "simt_dv": q + k + o + ge + states + v,
-        "simt_dg_key": 2 * 4 * th * w.Dk,
-        # forward: state pass over segments 0..nseg-2, scan, output pass (reads the segment initial states)
-        "tc_fwd": q + k + v + ge + ig + o + s1 + h0 + s1 * (fseg - 1),
-        "tc_seg_scan": _mean([2 * s1 * (fseg - 1) + h0] * (fseg > 1) + [2 * s1 * (bseg - 1) + h0] * (bseg > 1)),
-        # the backward's own forward-state pass / reverse state-gradient pass and scans
-        # the forward and the backward plan may both launch a state pass: bytes per launch averaged
-        "tc_state": _mean([frac_f * (k + v + ge + ig) + s1 * (fseg - 1)] * (fseg > 1) +
-                          [frac_b * (k + v + ge + ig) + s1 * (bseg - 1)] * (bseg > 1)),
-        "tc_gstate": frac_b * (q + o + ge) + s1 * (bseg - 1),
-        "tc_seg_rscan": 2 * s1 * (bseg - 1) + s1,
-        "tc_bwd_dq": q + k + v + o + ge + ig + s1 * bseg + h0 + q + dgb + s1 + 4 * BH * bseg * w.Dk,
-        "tc_bwd_dkdv": q + k + v + o + ge + ig + 2 * s1 * bseg + dgb + 4 * BH * bseg * w.Dk + s1 + k + v + dgb + ig + h0,
+        "simt_cumsum": (ge, ge),
+        "simt_state": (k + v + ge + h0, states),
+        "simt_out": (q + k + v + ge + o, states),
+        "simt_dstate": (q + o + ge, states),
+        "simt_dq": (q + k + v + o + ge + q, states + 4 * th * w.Dk),
+        "simt_dk": (q + k + v + o + ge + k, states + 2 * 4 * th * w.Dk),
+        "simt_dv": (q + k + o + ge + v, states),
+        "simt_dg_key": (dgb, 4 * th * w.Dk),
+        # forward output pass: reads the segment initial states; the training pair also writes
+        # the states the backward's segments start from
+        "tc_fwd": (q + k + v + ge + ig + o + s1 + h0, s1 * (fseg - 1) + s1 * (bseg - 1)),
+        "tc_seg_scan": (_mean([h0] * (fseg > 1) + [h0] * (bseg > 1)),
+                        _mean([2 * s1 * (fseg - 1) + 2 * gam * (fseg - 1)] * (fseg > 1) +
+                              [2 * s1 * (bseg - 1) + 2 * gam * (bseg - 1)] * (bseg > 1))),
+        # the forward's (or the backward's own) state pass over segments 0..nseg-2; per launch
+        # averaged when both plans launch one
+        "tc_state": (_mean([frac_f * (k + v + ge + ig)] * (fseg > 1) + [frac_b * (k + v + ge + ig)] * (bseg > 1)),
+                     _mean([(s1 + gam) * (fseg - 1)] * (fseg > 1) + [(s1 + gam) * (bseg - 1)] * (bseg > 1))),
+        "tc_gstate": (frac_b * (q + o + ge), (s1 + gam) * (bseg - 1)),
+        "tc_seg_rscan": (0.0, 2 * (s1 + gam) * (bseg - 1)),
+        "tc_bwd_dq": (q + k + v + o + ge + ig + h0 + q,
+                      s1 * (bseg - 1) + dgb + 4 * BH * bseg * w.Dk),
+        "tc_bwd_dkdv": (q + k + v + o + ge + ig + k + v + dgb + di + h0,
+                        2 * s1 * bseg + dgb + 4 * BH * bseg * w.Dk),
         # decode step: q, k, v, g, i read, o written, the state read and written once
-        "decode": compulsory_bytes(w, False),
+        "decode": (compulsory_bytes(w, False), 0.0),
     }
-    return float(table.get(name, 0.0))
+    m, pl = table.get(name, (0.0, 0.0))
+    return float(m), float(pl)
 
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one ncu capture
-# (summaries under profiles/), with the SHA-256 prefix of the kernel's source file at capture
-# time: a kernel whose source has changed since reports traffic null. `scale`: the capture
-# ran a smaller case of the same workload; traffic grows with the heads processed.
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one ncu capture,
+# with the SHA-256 prefix of the kernel's source file at capture time: a kernel whose source has
+# changed since reports traffic null. `scale`: the capture ran a smaller case of the same
+# workload (`case`); traffic grows with the heads processed.
 MEASURED_TRAFFIC = {
-    ("tc_bwd_dkdv", "c3"): {"bytes": 246.9e6, "scale": 4, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
-                            "sha": "b602016964e3abce", "profile": "profiles/tc_bwd_c3_b1.md"},
-    ("tc_bwd_dq", "c3"): {"bytes": 174.0e6, "scale": 4, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
-                          "sha": "b602016964e3abce", "profile": "profiles/tc_bwd_c3_b1.md"},
-    ("tc_bwd_dkdv", "c5"): {"bytes": 247.0e6, "scale": 2, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
-                            "sha": "b602016964e3abce", "profile": "profiles/tc_bwd_dkdv_c5_b1.md"},
     ("tc_fwd", "c2"): {"bytes": 187.1e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_fwd.cu",
-                       "sha": "c365d80ff3420b75", "profile": "profiles/tc_fwd_c2.md"},
+                       "sha": "c365d80ff3420b75", "case": "c2"},
     ("decode", "decode"): {"bytes": 215.2e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_decode.cu",
-                           "sha": "1b7b1b10ae6dd931", "profile": "profiles/decode_1024heads.md"},
+                           "sha": "1b7b1b10ae6dd931", "case": "decode, 1024 heads"},
 }
 
 
@@ -277,6 +283,9 @@ def base_line(w, args, world):
 
 
 def run_reference(args, w, world, rank):
+    """The float64 oracle on the host cores, each step a bounded sample of whole heads of the
+    workload (full L); `value` = tokens per second of the sample, `ms_per_step` = the time
+    the oracle would take for the workload's whole batch at that rate."""
     if rank != 0:
         return
     heads = max(1, oracle_heads(w) // 2)
@@ -291,10 +300,12 @@ def run_reference(args, w, world, rank):
         tot += dt
     val = tok / tot
     line = base_line(w, args, 1)
-    line.update({"impl": "reference", "value": val, "ms_per_step": 1e3 * tot / args.steps, "dtype": "f64",
+    line.update({"impl": "reference", "value": val, "ms_per_step": 1e3 * w.B * w.L / val, "dtype": "f64",
                  "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": thr, "kind": "oracle",
                                   "sample": f"{heads} of {w.B * w.H} heads, full L={w.L}, "
-                                            f"{'fwd+bwd' if w.backward else 'fwd'} per step"},
+                                            f"{'fwd+bwd' if w.backward else 'fwd'} per step; ms_per_step is the "
+                                            f"whole batch at the sample's rate ({1e3 * tot / args.steps:.0f} ms per "
+                                            f"sample step)"},
                  "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
                  "gpu_launches": 0})
     print(json.dumps(line), flush=True)
@@ -331,7 +342,7 @@ def deltanet_line(args, world, tokens, ms, extra):
     cfg = I.DELTANET
     line = {"metric": "DeltaNet chunkwise fwd+bwd tokens/s", "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; linear_rnn_b200/inputs.py)",
+            "vs_baseline": None, "dtype": cfg["dtype"], "data": "synthetic (seeded; linear_rnn_b200/inputs.py)",
             "config": {"workload": "deltanet: DeltaNet forward+backward, B={B} H={H} L={L} Dk={Dk} Dv={Dv} "
                                    "chunk=64 {dtype} I/O".format(**cfg),
                        "global_batch": cfg["B"] * world, "seq_len": cfg["L"], "parallelism": f"replicas x{world}",
@@ -339,6 +350,18 @@ def deltanet_line(args, world, tokens, ms, extra):
             "value": tokens / (ms / 1e3), "ms_per_step": ms / args.steps}
     line.update(extra)
     return line
+
+
+def blas_threads():
+    """Threads of the BLAS library numpy's matrix products (the DeltaNet oracle) run on."""
+    try:
+        import threadpoolctl
+        n = [i.get("num_threads") for i in threadpoolctl.threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return torch.get_num_threads()
 
 
 def deltanet_oracle_sample(seed, heads):
@@ -371,7 +394,8 @@ def run_deltanet(args, world, rank, local):
         val = tok / tot
         base = deltanet_line(args, 1, tok, 1e3 * tot, {})
         base.update({"impl": "reference", "value": val, "dtype": "f64", "gpu_launches": 0,
-                     "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": torch.get_num_threads(),
+                     "ms_per_step": 1e3 * cfg["B"] * cfg["L"] / val,
+                     "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": blas_threads(),
                                       "kind": "oracle", "sample": f"{heads} of {cfg['B'] * cfg['H']} heads, "
                                                                   f"full L={cfg['L']}, fwd+bwd per step"},
                      "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
@@ -465,17 +489,152 @@ def run_deltanet(args, world, rank, local):
         ach = fl / avg_s / 1e12
         roofline = {"bound": "alu", "kernel": name, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                     "frac": ach / peak, "traffic": None,
-                    "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 FLOPs x max SM clock",
+                    "peak_source": "nominal, derived (not measured): 148 SMs x 128 FP32 lanes x 2 FLOPs x "
+                                   "the sampled max SM clock",
                     "algorithmic_flops_per_launch": fl, "avg_launch_us": avg_s * 1e6,
                     "share_of_step": ms / sum(v[1] for v in kprof.values())}
     extra = {"e2e": e2e, "gpu_launches": int(launches), "roofline": roofline, "clocks": clocks,
              "kernels": {n: {"launches": c, "avg_us": 1e3 * m / c} for n, (c, m) in sorted(kprof.items())}}
     if world == 1 and not args.no_cpu_baseline:
         tk, dt = deltanet_oracle_sample(0, heads)
-        extra["cpu_baseline"] = {"value": tk / dt, "unit": "tokens/s", "cores": torch.get_num_threads(),
+        extra["cpu_baseline"] = {"value": tk / dt, "unit": "tokens/s", "cores": blas_threads(),
                                  "kind": "oracle", "sample": f"{heads} of {B * H} heads, full L={L}, fwd+bwd, "
                                                              f"float64 numpy, {dt:.1f} s"}
     print(json.dumps(deltanet_line(args, world, tokens, total_ms, extra)), flush=True)
+
+
+def run_shard(args, world, rank, local, nshards=8):
+    """Sequence-sharded forward on one GPU: workload c4 (B=1 H=8 L=65536) cut into `nshards`
+    contiguous shards that run one after another (virtual ranks, nothing waits across them).
+    Per step: gla_shard_state on every shard, then per shard gla_state_fold (its initial state
+    from the earlier shards' pairs) and gla_fwd from that state. Timed against one gla_fwd over
+    the whole sequence, with the same method as the main line. The per-rank estimate on
+    `nshards` GPUs is one shard's state pass + fold + forward (the all-gather, ~0.5 MB per rank,
+    is not measured here: every call of this build has one GPU)."""
+    from linear_rnn_b200 import _lib, ops
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = I.WORKLOADS["c4"]
+    x = I.make_inputs(w, seed=rank)
+    xd = {k: (None if v is None else v.to(dev)) for k, v in x.items()}
+    Ls = w.L // nshards
+    sh = [{n: (None if xd[n] is None else xd[n][:, :, r * Ls:(r + 1) * Ls].contiguous())
+           for n in ("q", "k", "v", "g", "igate")} for r in range(nshards)]
+    kw = dict(scale=w.scale, chunk=w.chunk)
+
+    def whole():
+        ops.gla_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["igate"], xd["h0"], **kw)
+
+    def sharded():
+        pairs = [ops.gla_shard_state(t["k"], t["v"], t["g"], t["igate"], chunk=w.chunk) for t in sh]
+        states = torch.stack([p[0] for p in pairs])
+        gammas = torch.stack([p[1] for p in pairs])
+        for r, t in enumerate(sh):
+            s_in = ops.gla_state_fold(states, gammas, r, xd["h0"])
+            ops.gla_fwd(t["q"], t["k"], t["v"], t["g"], t["igate"], s_in, **kw)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    res = {}
+    for name, fn in (("whole", whole), ("sharded", sharded)):
+        for i in range(args.warmup):
+            flush.fill_(i & 0xFF)
+            fn()
+        torch.cuda.synchronize()
+        tot, per, n, _ = time_steps(fn, flush, args.steps, world)
+        _, _, _, kp = time_steps(fn, flush, args.steps, world, per_kernel=True)
+        res[name] = {"us_per_step": 1e3 * max_over_ranks(tot, dev) / args.steps, "launches_per_step": n / args.steps,
+                     "kernels_us_per_step": {k: 1e3 * m / args.steps for k, (c, m) in sorted(kp.items())}}
+    clocks = sampler.stop()
+    if rank != 0:
+        return
+    ks = res["sharded"]["kernels_us_per_step"]
+    per_rank = sum(ks.values()) / nshards
+    t_whole = res["whole"]["us_per_step"]
+    line = {"metric": "sequence-sharded GLA forward, one GPU with virtual shards", "unit": "us",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "higher_is_better": False,
+            "scaling": "strong", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic (seeded; linear_rnn_b200/inputs.py)",
+            "config": {"workload": f"c4 forward, B={w.B} H={w.H} L={w.L} Dk={w.Dk} Dv={w.Dv} chunk={w.chunk} bf16, "
+                                   f"cut into {nshards} shards of {Ls} tokens",
+                       "l2": "256 MiB L2 flush between steps, outside the per-step events; inputs > L2"},
+            "value": res["sharded"]["us_per_step"], "ms_per_step": res["sharded"]["us_per_step"] / 1e3,
+            "whole_sequence_us": t_whole, "sharded": res["sharded"], "whole": res["whole"],
+            "per_rank_estimate_us": per_rank,
+            "per_rank_estimate_note": f"kernel time of one shard's state pass + fold + forward (sum over the "
+                                      f"{nshards} shards / {nshards}); all-gather not included",
+            "overhead_vs_ideal": per_rank / (t_whole / nshards), "clocks": clocks,
+            "gpu_launches": int(res["sharded"]["launches_per_step"] * args.steps)}
+    print(json.dumps(line), flush=True)
+
+
+def time_steps(step, flush, steps, world, per_kernel=False, flush_l2=True):
+    """K steps bracketed by barrier + synchronize; per-step CUDA events on the stream, with the
+    256 MiB L2 flush before each step outside the events (flush_l2=False: warm L2). per_kernel:
+    the library also brackets every launch with CUDA events (per-kernel durations), which costs
+    a few microseconds per launch, so step times come from a pass without it.
+    Returns (total_ms, per-step ms list, library launches, per-kernel profile)."""
+    from linear_rnn_b200 import _lib
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    n0 = _lib.launch_count()
+    _lib.profiler_enable(per_kernel)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    flush.fill_(0xA5)   # lead-in (outside the events): the host queues step 0 while this runs
+    for i in range(steps):
+        if flush_l2:
+            flush.fill_(i & 0xFF)
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    _lib.profiler_enable(False)
+    n = _lib.launch_count() - n0
+    kp = _lib.profiler_read() if per_kernel else {}
+    per = [a.elapsed_time(b) for a, b in ev]
+    return sum(per), per, n, kp
+
+
+def forward_targets(args, world, dev, flush):
+    """The bf16 GLA forward at L >= 2048 on its own (workloads c2 and c4, forward only),
+    timed like the main line: warm-up, then K steps with the L2 flush between them, CUDA
+    events per step, max over ranks. Returns {workload: {...}} with each step's fraction of
+    its roofline max(FLOPs / bf16 peak, compulsory bytes / HBM peak)."""
+    from linear_rnn_b200 import ops
+    peaks, peak_src = load_peaks()
+    out = {}
+    for name in ("c2", "c4"):
+        w = I.WORKLOADS[name]
+        x = I.make_inputs(w, seed=0)
+        xd = {k: (None if v is None else v.to(dev)) for k, v in x.items()}
+        kw = dict(scale=w.scale, chunk=w.chunk, plan=args.plan)
+        prob = ops.make_problem(xd["q"], xd["v"], xd["g"], **kw)
+        ws = torch.empty(ops.gla_workspace_bytes(prob, False), dtype=torch.uint8, device=dev)
+
+        def step():
+            ops.gla_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["igate"], xd["h0"], workspace=ws, **kw)
+
+        for i in range(args.warmup):
+            flush.fill_(i & 0xFF)
+            step()
+        torch.cuda.synchronize()
+        tot, per, _, _ = time_steps(step, flush, args.steps, world)
+        tot = max_over_ranks(tot, dev)
+        t = tot / args.steps / 1e3
+        fl, by = flops(w, False), compulsory_bytes(w, False)
+        roof = max(fl / (peaks["bf16_tflops"] * 1e12), by / (peaks["hbm_gbs"] * 1e9))
+        out[name] = {"workload": f"GLA forward, B={w.B} H={w.H} L={w.L} Dk={w.Dk} Dv={w.Dv} chunk={w.chunk} bf16",
+                     "us_per_step": t * 1e6, "us_median": statistics.median(per) * 1e3,
+                     "tokens_per_s": w.B * w.L * world / t, "tflops": fl / t / 1e12,
+                     "gbs_compulsory": by / t / 1e9, "roofline_us": roof * 1e6, "frac": roof / t,
+                     "peak_source": peak_src}
+        del xd, ws
+    return out
 
 
 def main():
@@ -483,19 +642,27 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="c3", choices=sorted(I.WORKLOADS) + ["decode", "deltanet"])
+    ap.add_argument("--workload", default="c3", choices=sorted(I.WORKLOADS) + ["decode", "deltanet", "shard"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--plan", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fwd-target", action="store_true",
+                    help="skip the forward-only c2 / c4 measurements added to the c3 line")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch B (smaller cases for profiling; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.workload == "deltanet":
+    if args.workload in ("deltanet", "shard"):
         world, rank, local = dist_setup()
-        run_deltanet(args, world, rank, local)
+        if args.workload == "deltanet":
+            run_deltanet(args, world, rank, local)
+        elif args.impl != "reference":
+            run_shard(args, world, rank, local)
+        elif rank == 0:
+            print(json.dumps({"impl": "reference", "unavailable": "the sharded forward has no oracle arm of its own; "
+                              "its parity is tested against the oracle over the whole sequence"}), flush=True)
         if world > 1:
             torch.distributed.destroy_process_group()
         return
@@ -547,34 +714,13 @@ def main():
         flush.fill_(i & 0xFF)
         step()
     torch.cuda.synchronize()
-    def timed_steps(per_kernel):
-        """K steps bracketed by barrier + synchronize; per-step CUDA events on the stream.
-        per_kernel: the library also brackets every launch with CUDA events (for the
-        per-kernel durations); this costs a few microseconds per launch, so `value` comes
-        from the pass without it and the roofline from the pass with it."""
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
-        n0 = _lib.launch_count()
-        _lib.profiler_enable(per_kernel)
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize()
-        flush.fill_(0xA5)   # lead-in (outside the events): the host queues step 0 while this runs
-        for i in range(args.steps):
-            flush.fill_(i & 0xFF)
-            ev[i][0].record()
-            step()
-            ev[i][1].record()
-        torch.cuda.synchronize()
-        if world > 1:
-            torch.distributed.barrier()
-        _lib.profiler_enable(False)
-        n = _lib.launch_count() - n0
-        kp = _lib.profiler_read() if per_kernel else {}
-        return sum(a.elapsed_time(b) for a, b in ev), n, kp
 
-    total_ms, launches, _ = timed_steps(False)
-    prof_ms, _, kprof = timed_steps(True)
+    total_ms, per_ms, launches, _ = time_steps(step, flush, args.steps, world)
+    prof_ms, _, _, kprof = time_steps(step, flush, args.steps, world, per_kernel=True)
+    warm_ms, warm_per, _, _ = time_steps(step, flush, args.steps, world, flush_l2=False)
+    ftarget = None
+    if w.name == "c3" and args.batch is None and not args.no_fwd_target and args.plan != "simt":
+        ftarget = forward_targets(args, world, dev, flush)
     clocks = sampler.stop()
     total_ms = max_over_ranks(total_ms, dev)
     tokens = w.B * w.L * args.steps * world
@@ -640,25 +786,35 @@ def main():
     if dom:
         name, (cnt, ms) = dom
         avg_s = ms / cnt / 1e3
-        kb = kernel_bytes(name, w, fseg, bseg)
-        ach = kb / avg_s / 1e9
+        mb, pb = kernel_bytes(name, w, fseg, bseg)
+        ach = mb / avg_s / 1e9
         share = ms / sum(v[1] for v in kprof.values())
         roofline = {"bound": "hbm", "kernel": name, "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": ach / peaks["hbm_gbs"], "traffic": measured_traffic(name, w.name if args.batch is None
-                                                                                 else None),
+                    "frac": ach / peaks["hbm_gbs"],
+                    "traffic": measured_traffic(name, w.name if args.batch is None else None),
                     "peak_source": peak_src,
-                    "algorithmic_bytes_per_launch": kb, "avg_launch_us": avg_s * 1e6, "share_of_step": share}
+                    "algorithmic_bytes_per_launch": mb, "plan_bytes_per_launch": pb,
+                    "frac_with_plan_bytes": (mb + pb) / avg_s / 1e9 / peaks["hbm_gbs"],
+                    "bytes_note": "algorithmic = the path's inputs this kernel reads and outputs it writes, "
+                                  "once each; plan = workspace intermediates (segment states, prefixes)",
+                    "avg_launch_us": avg_s * 1e6, "share_of_step": share}
     line = base_line(w, args, world)
     line.update({"value": value, "ms_per_step": total_ms / args.steps, "e2e": e2e, "gpu_launches": int(launches),
                  "roofline": roofline, "clocks": clocks,
                  "step_roofline": {"tflops": fl / t_step / 1e12, "gbs_compulsory": by / t_step / 1e9,
                                    "roofline_us": roof_t * 1e6, "frac": roof_t / t_step, "peak_source": peak_src},
+                 "step_ms": {"median": statistics.median(per_ms), "min": min(per_ms), "max": max(per_ms),
+                             "warm_l2_median": statistics.median(warm_per),
+                             "note": "rank 0's per-step CUDA-event times; warm_l2 = a third pass without the "
+                                     "L2 flush"},
                  "kernels": {n: {"launches": c, "avg_us": 1e3 * m / c} for n, (c, m) in sorted(kprof.items())},
                  "kernel_timing": {"source": "a second pass of the same K steps with CUDA events around "
                                              "every library launch (kernels, roofline); value and "
                                              "ms_per_step come from the pass without them",
                                    "ms_per_step_instrumented": prof_ms / args.steps},
                  "plan": args.plan})
+    if ftarget is not None:
+        line["fwd_target"] = ftarget
     if world == 1 and not args.no_cpu_baseline:
         heads = oracle_heads(w)
         tk, dt, thr = oracle_sample(w, 0, heads)

@@ -23,9 +23,11 @@
  *  - q,k,v,o,dO,dq,dk,dv have the I/O dtype of the problem (GLA_F32 or GLA_BF16);
  *    g, i, h0, hT and all their gradients are always float32. Accumulation is fp32.
  *  - g is the log of the decay (g <= 0 for a decay in (0,1]); the library applies no
- *    activation to it. It must be finite; within any 64-token tile the decay of one key
- *    dim should span less than about 80 nats (exp stays inside fp32 range), otherwise
- *    results lose accuracy (no fault, no error code).
+ *    activation to it. It must be finite. The tensor-core plan factors each tile's in-tile
+ *    decays into exponentials that must stay inside the fp32 range; a tile whose decay in
+ *    some key dim is stronger than that plan evaluates sets the device status word, so that
+ *    gla_check_device_status returns GLA_ERR_RANGE (the results of that call are then not
+ *    valid; nothing faults). GLA_PLAN_SIMT evaluates any finite gate.
  *  - Every pointer is a DEVICE pointer owned by the caller, 16-byte aligned. The
  *    library allocates nothing; scratch memory is the caller's workspace `ws` of at
  *    least gla_workspace_bytes() bytes (16-byte aligned, contents need not be zeroed).
@@ -196,8 +198,9 @@ GLA_API gla_status gla_shard_state_grad(const gla_problem* p, const void* q, con
  * Linear Attention Models", sections 22:36 and 31:16 (writing strength beta_t; one gradient step
  * per token on the key-to-value regression loss; the WY representation for the chunk form):
  *   S_t = (I - beta_t k_t^T k_t) S_{t-1} + beta_t k_t^T v_t,   o_t = scale q_t S_t.
- * p: B, H, L >= 0; Dk 64 or 128; Dv a multiple of 64 up to 4096; chunk = 64; scale; io bf16 or
- *   f32; gate must be GLA_GATE_NONE (no decay gates); plan is ignored.
+ * p: B, H, L >= 0 with B*H at most 65535; Dk 64 or 128; Dv a multiple of 64 up to 4096;
+ *   chunk = 64; scale; io bf16 or f32; gate must be GLA_GATE_NONE (no decay gates); plan is
+ *   ignored. The backward accepts exactly the problems the forward accepts.
  * q, k [B,H,L,Dk] and v [B,H,L,Dv] in io dtype; beta [B,H,L] f32; h0 [B,H,Dk,Dv] f32 or NULL
  *   (zero); o [B,H,L,Dv] io dtype (written); hT [B,H,Dk,Dv] f32 or NULL (final state, written).
  *   Keys are used as given (unit-norm keys with beta in [0, 1] keep each transition's
@@ -205,7 +208,8 @@ GLA_API gla_status gla_shard_state_grad(const gla_problem* p, const void* q, con
  *   caller; no workspace. L = 0 copies h0 (or zero) to hT.
  * CUDA cores, fp32 arithmetic; asynchronous on `stream`.
  * Errors: GLA_ERR_INVALID_ARG (null or misaligned pointer, bad enum, a gate mode),
- *   GLA_ERR_UNSUPPORTED (head dims, chunk), GLA_ERR_CUDA. */
+ *   GLA_ERR_UNSUPPORTED (head dims, chunk, B*H), GLA_ERR_CUDA (gla_last_error_detail says
+ *   which call failed). */
 GLA_API gla_status gla_deltanet_fwd(const gla_problem* p, const void* q, const void* k, const void* v,
                                     const float* beta, const float* h0, void* o, float* hT, void* stream);
 
@@ -218,7 +222,7 @@ GLA_API gla_status gla_deltanet_fwd(const gla_problem* p, const void* q, const v
  * [B,H,Dk,Dv] f32 or NULL. ws: device workspace of gla_deltanet_bwd_workspace_bytes(p) bytes
  * (the chunk start states, X, dR, the chunk end gradients and per-slice sums), caller-owned.
  * Three launches on `stream` (the forward's state pass, the reverse walk, the per-chunk
- * gradients). B*H at most 65535.
+ * gradients).
  * Errors: as gla_deltanet_fwd, plus GLA_ERR_WORKSPACE. */
 GLA_API size_t gla_deltanet_bwd_workspace_bytes(const gla_problem* p);
 GLA_API gla_status gla_deltanet_bwd(const gla_problem* p, const void* q, const void* k, const void* v,
@@ -264,10 +268,14 @@ GLA_API gla_status gla_plan_info(const gla_problem* p, int for_backward, int* pl
  *  - Problems whose scratch exceeds 16 MiB (gla_workspace_bytes of the same problem with
  *    plan GLA_PLAN_SIMT and for_backward = 0) return GLA_ERR_WORKSPACE before any launch.
  *  - The first call on a device looks up that device's address of the array
- *    (cudaGetSymbolAddress with the device current); make that first call before any
+ *    (cudaGetSymbolAddress with the device current), and so does the first call after the
+ *    device's CUDA context was replaced (cudaDeviceReset); make those calls before any
  *    stream capture.
  *  - All calls share the array and it keeps the last call's contents; calls whose work
  *    overlaps on the GPU (other streams, other host threads) race on it.
+ *  - The CUDA-core forward has no device-side waits or range checks, so it reports every
+ *    failure through the return value (GLA_ERR_CUDA with gla_last_error_detail); there is no
+ *    device status word to read for this call.
  *  - No cudaMalloc, cudaFree or allocating library routine is called. */
 GLA_API gla_status gla_fwd_static_scratch(const gla_problem* p, const void* q, const void* k, const void* v,
                                           const float* g, const float* igate, const float* h0,

@@ -14,6 +14,7 @@ using namespace gla;
 
 // ------------------------------------------------------------ launch accounting
 namespace {
+thread_local char g_last_detail[256] = "no error";
 struct ProfRecord {
     std::string name;
     cudaEvent_t start, stop;
@@ -37,6 +38,11 @@ cudaEvent_t take_event() {
 }  // namespace
 
 namespace gla {
+gla_status record_cuda(cudaError_t e, const char* where) {
+    if (e == cudaSuccess) return GLA_OK;
+    snprintf(g_last_detail, sizeof(g_last_detail), "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+    return GLA_ERR_CUDA;
+}
 void prof_begin(const char* name, cudaStream_t st) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
     ++g_launches;
@@ -95,17 +101,7 @@ gla_status resolve(const gla_problem* p, const Dims& P, bool bwd, int* plan) {
     return GLA_OK;
 }
 
-thread_local char g_last_detail[256] = "no error";
-
-void set_detail(const char* where, cudaError_t e) {
-    snprintf(g_last_detail, sizeof(g_last_detail), "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
-}
-
-gla_status map_cuda(cudaError_t e, const char* where = "launch") {
-    if (e == cudaSuccess) return GLA_OK;
-    set_detail(where, e);
-    return GLA_ERR_CUDA;
-}
+gla_status map_cuda(cudaError_t e, const char* where = "launch") { return gla::record_cuda(e, where); }
 
 size_t ws_bytes(const Dims& P, int plan, bool bwd) {
     if (plan == GLA_PLAN_TC) return bwd ? tc::bwd_workspace_bytes(P) : tc::fwd_workspace_bytes(P);
@@ -229,8 +225,10 @@ gla_status gla_check_device_status(void* ws, void* stream) {
     if (!ws) return GLA_ERR_INVALID_ARG;
     int word = 0;
     cudaStream_t st = (cudaStream_t)stream;
-    if (cudaMemcpyAsync(&word, ws, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return GLA_ERR_CUDA;
-    if (cudaStreamSynchronize(st) != cudaSuccess) return GLA_ERR_CUDA;
+    cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof(int), cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return map_cuda(e, "status word read");
+    e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return map_cuda(e, "stream synchronisation");
     if (word & kDevStatusTimeout) return GLA_ERR_TIMEOUT;
     if (word & kDevStatusRange) return GLA_ERR_RANGE;
     return word == kDevStatusOk ? GLA_OK : GLA_ERR_TIMEOUT;

@@ -42,6 +42,11 @@ void prof_end(cudaStream_t st);
 // caller's stream, so that each launch's events time that kernel alone.
 bool prof_enabled();
 
+// Maps a CUDA error to the C ABI's status: GLA_OK for cudaSuccess, otherwise GLA_ERR_CUDA after
+// recording where it happened and the CUDA error's name and text for gla_last_error_detail
+// (gla_api.cu; one record per host thread).
+gla_status record_cuda(cudaError_t e, const char* where);
+
 }  // namespace gla
 
 #define GLA_LAUNCH(name, stream, ...)      \

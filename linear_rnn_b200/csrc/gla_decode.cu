@@ -136,5 +136,5 @@ extern "C" gla_status gla_decode(const gla_problem* p, const void* q, const void
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e = p->io == GLA_BF16 ? gla::launch_gate<__nv_bfloat16>(p, q, k, v, g, igate, state, o, st)
                                       : gla::launch_gate<float>(p, q, k, v, g, igate, state, o, st);
-    return e == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
+    return gla::record_cuda(e, "decode launch");
 }

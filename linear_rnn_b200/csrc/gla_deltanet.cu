@@ -754,18 +754,26 @@ bool dn_aligned16(const void* x) { return x == nullptr || (reinterpret_cast<uint
 
 static_assert(DnSmem<128>::BYTES <= 227 * 1024, "shared memory of the Dk = 128 plan");
 
+// Validation shared by the forward and the backward, so that a problem one accepts the other
+// accepts too. B*H is at most 65535: the backward's per-chunk gradient kernel puts the heads on
+// the grid's y extent.
+gla_status dn_check(const gla_problem* p) {
+    if (!p || p->B < 0 || p->H < 0 || p->L < 0) return GLA_ERR_INVALID_ARG;
+    if (p->io != GLA_F32 && p->io != GLA_BF16) return GLA_ERR_INVALID_ARG;
+    if (p->gate != GLA_GATE_NONE) return GLA_ERR_INVALID_ARG;
+    if ((p->Dk != 64 && p->Dk != 128) || p->Dv <= 0 || p->Dv % DN_VT != 0 || p->Dv > 4096 || p->chunk != DN_C)
+        return GLA_ERR_UNSUPPORTED;
+    if ((long long)p->B * p->H > 65535LL) return GLA_ERR_UNSUPPORTED;
+    return GLA_OK;
+}
+
 }  // namespace
 }  // namespace gla
 
 extern "C" gla_status gla_deltanet_fwd(const gla_problem* p, const void* q, const void* k, const void* v,
                                        const float* beta, const float* h0, void* o, float* hT, void* stream) {
-    if (!p || p->B < 0 || p->H < 0 || p->L < 0) return GLA_ERR_INVALID_ARG;
-    if (p->io != GLA_F32 && p->io != GLA_BF16) return GLA_ERR_INVALID_ARG;
-    if (p->gate != GLA_GATE_NONE) return GLA_ERR_INVALID_ARG;
-    if ((p->Dk != 64 && p->Dk != 128) || p->Dv <= 0 || p->Dv % gla::DN_VT != 0 || p->Dv > 4096 ||
-        p->chunk != gla::DN_C)
-        return GLA_ERR_UNSUPPORTED;
-    if ((long long)p->B * p->H > 2147483647LL) return GLA_ERR_UNSUPPORTED;
+    const gla_status c = gla::dn_check(p);
+    if (c != GLA_OK) return c;
     if ((size_t)p->B * p->H == 0) return GLA_OK;
     if (p->L > 0 && (!q || !k || !v || !beta || !o)) return GLA_ERR_INVALID_ARG;
     const void* ptrs[] = {q, k, v, beta, h0, o, hT};
@@ -775,22 +783,11 @@ extern "C" gla_status gla_deltanet_fwd(const gla_problem* p, const void* q, cons
     const cudaError_t e = p->io == GLA_BF16
                               ? gla::dn_launch_dk<__nv_bfloat16>(p, q, k, v, beta, h0, o, hT, nullptr, st)
                               : gla::dn_launch_dk<float>(p, q, k, v, beta, h0, o, hT, nullptr, st);
-    return e == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
-}
-
-static gla_status dn_check(const gla_problem* p) {
-    if (!p || p->B < 0 || p->H < 0 || p->L < 0) return GLA_ERR_INVALID_ARG;
-    if (p->io != GLA_F32 && p->io != GLA_BF16) return GLA_ERR_INVALID_ARG;
-    if (p->gate != GLA_GATE_NONE) return GLA_ERR_INVALID_ARG;
-    if ((p->Dk != 64 && p->Dk != 128) || p->Dv <= 0 || p->Dv % gla::DN_VT != 0 || p->Dv > 4096 ||
-        p->chunk != gla::DN_C)
-        return GLA_ERR_UNSUPPORTED;
-    if ((long long)p->B * p->H > 65535LL) return GLA_ERR_UNSUPPORTED;
-    return GLA_OK;
+    return gla::record_cuda(e, "DeltaNet forward launch");
 }
 
 extern "C" size_t gla_deltanet_bwd_workspace_bytes(const gla_problem* p) {
-    if (dn_check(p) != GLA_OK) return 0;
+    if (gla::dn_check(p) != GLA_OK) return 0;
     return gla::dn_bwd_ws(p, nullptr).bytes;
 }
 
@@ -798,7 +795,7 @@ extern "C" gla_status gla_deltanet_bwd(const gla_problem* p, const void* q, cons
                                        const float* beta, const float* h0, const void* dO, const float* dhT,
                                        void* dq, void* dk, void* dv, float* dbeta, float* dh0, void* ws,
                                        size_t ws_bytes, void* stream) {
-    const gla_status c = dn_check(p);
+    const gla_status c = gla::dn_check(p);
     if (c != GLA_OK) return c;
     if ((size_t)p->B * p->H == 0) return GLA_OK;
     if (p->L > 0 && (!q || !k || !v || !beta || !dO || !dq || !dk || !dv || !dbeta)) return GLA_ERR_INVALID_ARG;
@@ -815,5 +812,5 @@ extern "C" gla_status gla_deltanet_bwd(const gla_problem* p, const void* q, cons
     else
         e = p->Dk == 64 ? gla::dn_bwd_launch<float, 64>(p, q, k, v, beta, h0, dO, dhT, dq, dk, dv, dbeta, dh0, w, st)
                         : gla::dn_bwd_launch<float, 128>(p, q, k, v, beta, h0, dO, dhT, dq, dk, dv, dbeta, dh0, w, st);
-    return e == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
+    return gla::record_cuda(e, "DeltaNet backward launch");
 }

@@ -26,7 +26,8 @@ extern "C" gla_status gla_debug_wait_timeout(void* ws, unsigned polls, void* str
     if (!ws || (reinterpret_cast<uintptr_t>(ws) & 15u) != 0) return GLA_ERR_INVALID_ARG;
     if (polls == 0 || polls > gla::sm100::kWaitPolls) return GLA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
-    if (cudaMemsetAsync(ws, 0, gla::kStatusBytes, st) != cudaSuccess) return GLA_ERR_CUDA;
+    const cudaError_t e = cudaMemsetAsync(ws, 0, gla::kStatusBytes, st);
+    if (e != cudaSuccess) return gla::record_cuda(e, "status word reset");
     GLA_LAUNCH("debug_wait_timeout", st, gla::k_wait_timeout<<<1, 32, 0, st>>>(static_cast<int*>(ws), polls));
-    return cudaGetLastError() == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
+    return gla::record_cuda(cudaGetLastError(), "wait-timeout kernel launch");
 }

@@ -62,14 +62,14 @@ extern "C" gla_status gla_shard_state(const gla_problem* p, const void* k, const
     for (const void* x : ptrs)
         if (!gla::aligned16(x)) return GLA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
-    if (cudaMemsetAsync(ws, 0, gla::kStatusBytes, st) != cudaSuccess) return GLA_ERR_CUDA;
+    cudaError_t e = cudaMemsetAsync(ws, 0, gla::kStatusBytes, st);
+    if (e != cudaSuccess) return gla::record_cuda(e, "status word reset");
     const size_t BH = (size_t)p->B * p->H;
     if (BH == 0) return GLA_OK;
     if (p->L == 0) {   // an empty shard passes the state through: zero state, zero log-decay
-        if (cudaMemsetAsync(state, 0, 4 * BH * p->Dk * p->Dv, st) != cudaSuccess ||
-            cudaMemsetAsync(gamma, 0, 4 * BH * p->Dk, st) != cudaSuccess)
-            return GLA_ERR_CUDA;
-        return GLA_OK;
+        e = cudaMemsetAsync(state, 0, 4 * BH * p->Dk * p->Dv, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(gamma, 0, 4 * BH * p->Dk, st);
+        return gla::record_cuda(e, "empty shard");
     }
     gla::Dims P;
     P.B = p->B; P.H = p->H; P.L = p->L; P.Dk = p->Dk; P.Dv = p->Dv; P.C = p->chunk;
@@ -79,8 +79,8 @@ extern "C" gla_status gla_shard_state(const gla_problem* p, const void* k, const
     // the whole shard as the one segment of the state-only pass: one CTA per (head, Dv tile)
     // walks it (the shards themselves are the sequence parallelism)
     const int ntiles = gla::cdiv(p->L, gla::tc::TR);
-    const cudaError_t e = gla::tc::state_pass(P, 3, k, v, g, igate, 1, ntiles, state, gamma, static_cast<int*>(ws), st);
-    return e == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
+    e = gla::tc::state_pass(P, 3, k, v, g, igate, 1, ntiles, state, gamma, static_cast<int*>(ws), st);
+    return gla::record_cuda(e, "shard state pass");
 }
 
 extern "C" gla_status gla_shard_state_grad(const gla_problem* p, const void* q, const void* dO, const float* g,
@@ -100,14 +100,14 @@ extern "C" gla_status gla_shard_state_grad(const gla_problem* p, const void* q, 
     for (const void* x : ptrs)
         if (!gla::aligned16(x)) return GLA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
-    if (cudaMemsetAsync(ws, 0, gla::kStatusBytes, st) != cudaSuccess) return GLA_ERR_CUDA;
+    cudaError_t e = cudaMemsetAsync(ws, 0, gla::kStatusBytes, st);
+    if (e != cudaSuccess) return gla::record_cuda(e, "status word reset");
     const size_t BH = (size_t)p->B * p->H;
     if (BH == 0) return GLA_OK;
     if (p->L == 0) {
-        if (cudaMemsetAsync(state_grad, 0, 4 * BH * p->Dk * p->Dv, st) != cudaSuccess ||
-            cudaMemsetAsync(gamma, 0, 4 * BH * p->Dk, st) != cudaSuccess)
-            return GLA_ERR_CUDA;
-        return GLA_OK;
+        e = cudaMemsetAsync(state_grad, 0, 4 * BH * p->Dk * p->Dv, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(gamma, 0, 4 * BH * p->Dk, st);
+        return gla::record_cuda(e, "empty shard");
     }
     gla::Dims P;
     P.B = p->B; P.H = p->H; P.L = p->L; P.Dk = p->Dk; P.Dv = p->Dv; P.C = p->chunk;
@@ -115,9 +115,8 @@ extern "C" gla_status gla_shard_state_grad(const gla_problem* p, const void* q, 
     P.gate = p->gate;
     P.scale = p->scale;
     const int ntiles = gla::cdiv(p->L, gla::tc::TR);
-    const cudaError_t e =
-        gla::tc::state_pass(P, 4, q, dO, g, nullptr, 1, ntiles, state_grad, gamma, static_cast<int*>(ws), st);
-    return e == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
+    e = gla::tc::state_pass(P, 4, q, dO, g, nullptr, 1, ntiles, state_grad, gamma, static_cast<int*>(ws), st);
+    return gla::record_cuda(e, "shard state-gradient pass");
 }
 
 extern "C" gla_status gla_state_fold(const gla_problem* p, int count, const float* states, const float* gammas,
@@ -135,5 +134,5 @@ extern "C" gla_status gla_state_fold(const gla_problem* p, int count, const floa
     GLA_LAUNCH("state_fold", st,
                gla::k_state_fold<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(states, gammas, h0, out, count, (int)BH,
                                                                              p->Dk, p->Dv));
-    return cudaGetLastError() == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
+    return gla::record_cuda(cudaGetLastError(), "state fold launch");
 }

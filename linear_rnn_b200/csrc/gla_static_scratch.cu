@@ -14,6 +14,8 @@
 // keeps the last call's contents; two calls whose work overlaps on the GPU (different
 // streams, or different host threads) race on it. Problems whose scratch need exceeds the
 // array are rejected with GLA_ERR_WORKSPACE before any launch.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "gla_common.cuh"
@@ -27,22 +29,51 @@ static __device__ __align__(256) unsigned char g_static_scratch[GLA_STATIC_SCRAT
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
+// Per device: the array's device address and the id of the CUDA context it was looked up in.
+// A device reset (cudaDeviceReset) ends that context and the next one loads the array anew, so
+// the address is looked up again whenever the current context's id differs.
 void* g_scratch_ptr[kMaxDevices] = {nullptr};
+unsigned long long g_scratch_ctx[kMaxDevices] = {0};
 
-// Device address of the array on the current device. In host code the array's name is
-// only a host-side stand-in, so the address must come from cudaGetSymbolAddress, once per
-// device, with that device current.
+// Id of the calling thread's current CUDA context (unique for the process's lifetime), or 0
+// when there is none or the driver cannot say.
+unsigned long long current_context_id() {
+    static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Device address of the array on the current device. In host code the array's name is only a
+// host-side stand-in, so the address comes from cudaGetSymbolAddress, with the device current:
+// once per device and CUDA context, then from the cache.
 cudaError_t scratch_on_current_device(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_scratch_ptr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (!g_scratch_ptr[dev] || ctx == 0 || ctx != g_scratch_ctx[dev]) {
         void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_static_scratch);
+        e = cudaGetSymbolAddress(&p, g_static_scratch);   // also makes the device's context current
         if (e != cudaSuccess) return e;
         g_scratch_ptr[dev] = p;
+        g_scratch_ctx[dev] = current_context_id();
     }
     *out = g_scratch_ptr[dev];
     return cudaSuccess;
@@ -79,13 +110,15 @@ gla_status gla_fwd_static_scratch(const gla_problem* p, const void* q, const voi
         if (!aligned16(x)) return GLA_ERR_INVALID_ARG;
     if (simt::workspace_bytes(P, false) > GLA_STATIC_SCRATCH_BYTES) return GLA_ERR_WORKSPACE;
     void* ws = nullptr;
-    if (scratch_on_current_device(&ws) != cudaSuccess) return GLA_ERR_CUDA;
+    cudaError_t e = scratch_on_current_device(&ws);
+    if (e != cudaSuccess) return record_cuda(e, "static scratch address lookup");
     cudaStream_t st = (cudaStream_t)stream;
     // the status word must start at zero; everything else is written before it is read
-    if (cudaMemsetAsync(ws, 0, kStatusBytes, st) != cudaSuccess) return GLA_ERR_CUDA;
+    e = cudaMemsetAsync(ws, 0, kStatusBytes, st);
+    if (e != cudaSuccess) return record_cuda(e, "status word reset");
     if ((size_t)P.B * P.H == 0) return GLA_OK;
-    const cudaError_t e = simt::fwd(P, p->io, q, k, v, g, igate, h0, o, hT, ws, st);
-    return e == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
+    e = simt::fwd(P, p->io, q, k, v, g, igate, h0, o, hT, ws, st);
+    return record_cuda(e, "launch");
 }
 
 }  // extern "C"

@@ -170,7 +170,7 @@ __device__ __forceinline__ void bwd_transform_key(uint8_t* sq, uint8_t* sk, floa
     for (int u = 0; u < RSF; ++u) {
         const int r = sgi * RSF + u;
         const float ex = __expf(cs[u].x + off.x), ey = __expf(cs[u].y + off.y);
-        const float dx = rcp_newton(ex), dy = rcp_newton(ey);
+        const float dx = rcp_approx(ex), dy = rcp_approx(ey);
         *reinterpret_cast<float2*>(sg + gsw(r, d0)) = G_SLOT_EB ? make_float2(ex, ey) : make_float2(dx, dy);
         // byte offset of (r, d0) in a 128-byte-swizzled bf16 tile
         const uint32_t ob = (uint32_t)(d0 >> 6) * BLK + (uint32_t)r * 128 +
@@ -280,7 +280,7 @@ __device__ __forceinline__ void bwd_transform(uint8_t* sq, uint8_t* sk, float* s
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     eq[u] = __expf(bv[k][u]);
-                    ek[u] = rcp_newton(eq[u]);
+                    ek[u] = rcp_approx(eq[u]);
                 }
                 const float* keep = G_SLOT_EB ? eq : ek;
                 *reinterpret_cast<float4*>(sg + gsw(r, d0)) = make_float4(keep[0], keep[1], keep[2], keep[3]);

@@ -51,21 +51,9 @@ __device__ __forceinline__ int gsw(int r, int d) {
     return ((d >> 5) << 11) + (r << 5) + ((((d >> 2) & 7) ^ (r & 7)) << 2) + (d & 3);
 }
 
-// 1/x on the FMA pipe (keeps the special-function unit free for the exponentials): a bit-level
-// seed -- the integer constant minus the bits of x, which for any normal x lands within 5.1 %
-// of 1/x; the constant was chosen by a search minimising that worst case over one binade --
-// then two Newton steps y <- y (2 - x y), each squaring the relative error (5.1e-2 -> 2.6e-3
-// -> 6.6e-6), far below the bf16 rounding its result goes into.
-__device__ __forceinline__ float rcp_newton(float x) {
-    float y = __int_as_float(0x7EF311C2 - __float_as_int(x));
-    float e = fmaf(-x, y, 1.f);
-    y = fmaf(y, e, y);
-    e = fmaf(-x, y, 1.f);
-    return fmaf(y, e, y);
-}
-
-// 1/x on the special-function unit (PTX rcp.approx, about 1 ulp, subnormals flushed): where the
-// FMA pipe is the busier unit, this is cheaper than rcp_newton.
+// 1/x on the special-function unit (PTX rcp.approx.ftz: at most 1 ulp of error over the whole
+// input range per the PTX ISA, subnormal results flushed to zero). Its results e^-b go into bf16
+// operands (relative rounding 2^-9) or fp32 epilogue factors.
 __device__ __forceinline__ float rcp_approx(float x) {
     float y;
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
