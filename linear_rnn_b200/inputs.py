@@ -164,3 +164,31 @@ def make_deltanet_inputs(B: int, H: int, L: int, Dk: int, Dv: int, dtype: str = 
 # DeltaNet forward+backward: the pages give the method but no benchmark shape, so this takes
 # the gated workloads' batch and length with square heads (Dk = Dv = 128), bf16 I/O.
 DELTANET = dict(B=4, H=16, L=4096, Dk=128, Dv=128, dtype="bf16")
+
+
+# mLSTM cell with an exponential input gate, normaliser and stabiliser: the shapes of the
+# scalar-gate workload c5 (B=2 H=8 L=8192 Dk=Dv=256, bf16, log forget gate logsigmoid(N(3,1))
+# per head, scale Dk^-1/2), with the log input gate i~ ~ N(0, 1) (the gate is e^{i~}).
+MLSTM = Workload("mlstm", 2, 8, 8192, 256, 256, 64, "bf16", GATE_PER_HEAD, True, 256 ** -0.5,
+                 gate_mean=3.0, gate_div=1.0)
+
+
+def make_mlstm_inputs(w: Workload, seed: int = 0, itil_shift: float = 0.0) -> Dict[str, Optional[torch.Tensor]]:
+    """Inputs of the mLSTM cell, drawn on the CPU from one generator in the order q, k, v,
+    forget-gate pre-activation, log input gate, dh: q, k, v, dh ~ N(0,1) in the io dtype;
+    g = logsigmoid(N(gate_mean, 1)) / gate_div fp32 [B,H,L] (log forget gate); itil ~ N(0,1) +
+    itil_shift fp32 [B,H,L] (log of the exponential input gate)."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(30_000 + seed)
+    B, H, L, Dk, Dv = w.B, w.H, w.L, w.Dk, w.Dv
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=gen, dtype=torch.float32)
+
+    q = _round_io(randn(B, H, L, Dk), w.dtype)
+    k = _round_io(randn(B, H, L, Dk), w.dtype)
+    v = _round_io(randn(B, H, L, Dv), w.dtype)
+    g = torch.nn.functional.logsigmoid(randn(B, H, L) + w.gate_mean) / w.gate_div
+    itil = randn(B, H, L) + itil_shift
+    dh = _round_io(randn(B, H, L, Dv), w.dtype) if w.backward else None
+    return {"q": q, "k": k, "v": v, "g": g, "itil": itil, "dh": dh}

@@ -237,3 +237,18 @@ def test_tc_bwd_concurrent_calls_on_two_streams():
         for n in ("dq", "dk", "dv", "dg", "dh0"):
             assert torch.equal(r1[n], ref1[n]), n
             assert torch.equal(r2[n], ref2[n]), n
+
+
+@pytest.mark.parametrize("Dk,Dv", [(128, 256), (128, 128), (64, 256)])
+@pytest.mark.parametrize("gate,ig", [(I.GATE_PER_KEY, True), (I.GATE_PER_HEAD, True), (I.GATE_NONE, False)])
+def test_tc_bwd_single_stage_ring(Dk, Dv, gate, ig):
+    """Backward shapes whose kernels hold one tile at a time and issue the next tile's loads as
+    each slot's last reader finishes: 16 heads cut into segments of several tiles each, a
+    ragged last tile, initial state and final-state gradient; two heads against the oracle."""
+    from test_gpu_parity import check_bwd, with_dhT
+    w = I.WORKLOADS["c3"].replace(B=2, H=8, L=1765, Dk=Dk, Dv=Dv, dtype="bf16", gate=gate, input_gate=ig,
+                                  h0_std=0.3, backward=True,
+                                  gate_mean=3.0 if gate == I.GATE_PER_HEAD else 0.0,
+                                  gate_div=1.0 if gate == I.GATE_PER_HEAD else 16.0)
+    x = with_dhT(I.make_inputs(w, seed=16), w)
+    check_bwd(x, w, plan="tc", heads=[3, 12])
