@@ -570,6 +570,124 @@ def run_shard(args, world, rank, local, nshards=8):
     print(json.dumps(line), flush=True)
 
 
+def mlstm_oracle_sample(seed, heads):
+    """Times the float64 mLSTM oracle (stabilised recurrence, then its gradients) on `heads`
+    whole heads of the mLSTM workload. Returns (tokens_equivalent, seconds)."""
+    from oracle import mlstm as ML
+    w = I.MLSTM.replace(B=1, H=heads)
+    x = I.make_mlstm_inputs(w, seed=seed)
+    t0 = time.perf_counter()
+    ML.mlstm_fwd(x["q"], x["k"], x["v"], x["g"], x["itil"], w.scale)
+    ML.mlstm_bwd(x["q"], x["k"], x["v"], x["g"], x["itil"], x["dh"], w.scale)
+    return w.L * heads / I.MLSTM.H, time.perf_counter() - t0
+
+
+def run_mlstm(args, world, rank, local):
+    """mLSTM cell forward+backward on its workload (B=2 H=8 L=8192 Dk=Dv=256, bf16): one step is
+    gla_mlstm_fwd then gla_mlstm_bwd through the C ABI on HBM-resident inputs."""
+    w = I.MLSTM
+    th = w.B * w.H * w.L
+    e = 2
+    # compulsory bytes: q, k, v, g, i~ read and h written (forward); q, k, v, g, i~, dh read and
+    # dq, dk, dv, dg, d i~ written (backward)
+    fwd_b = th * ((2 * w.Dk + w.Dv) * e + 8 + w.Dv * e)
+    bwd_b = th * ((2 * w.Dk + 2 * w.Dv) * e + 8 + (2 * w.Dk + w.Dv) * e + 8)
+    base = {"metric": "mLSTM cell fwd+bwd tokens/s", "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic (seeded; linear_rnn_b200/inputs.py)",
+            "config": {"workload": f"mlstm: exponential input gate, normaliser, stabiliser; B={w.B} H={w.H} L={w.L} "
+                                   f"Dk={w.Dk} Dv={w.Dv} chunk={w.chunk} bf16",
+                       "global_batch": w.B * world, "seq_len": w.L, "parallelism": f"replicas x{world}",
+                       "l2": "256 MiB L2 flush between steps, outside the per-step events; inputs > L2"}}
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        for _ in range(args.warmup):
+            mlstm_oracle_sample(0, 1)
+        tok = tot = 0.0
+        for i in range(args.steps):
+            t, dt = mlstm_oracle_sample(i, 1)
+            tok += t
+            tot += dt
+        val = tok / tot
+        base.update({"impl": "reference", "value": val, "ms_per_step": 1e3 * w.B * w.L / val, "dtype": "f64",
+                     "gpu_launches": 0,
+                     "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                      "sample": f"1 of {w.B * w.H} heads, full L={w.L}, fwd+bwd per step"},
+                     "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
+        print(json.dumps(base), flush=True)
+        return
+    from linear_rnn_b200 import ops
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    x = I.make_mlstm_inputs(w, seed=rank)
+    xd = {k: v.to(dev) for k, v in x.items()}
+    kw = dict(scale=w.scale, chunk=w.chunk)
+    prob = ops.make_problem(xd["q"], xd["v"], xd["g"], scale=w.scale, chunk=w.chunk, plan="auto")
+    import ctypes
+    from linear_rnn_b200 import _lib
+    ws = torch.empty(max(_lib.lib.gla_mlstm_workspace_bytes(ctypes.byref(prob), 0),
+                         _lib.lib.gla_mlstm_workspace_bytes(ctypes.byref(prob), 1)), dtype=torch.uint8, device=dev)
+
+    def step():
+        ops.gla_mlstm_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["itil"], workspace=ws, **kw)
+        ops.gla_mlstm_bwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["itil"], xd["dh"], workspace=ws, **kw)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        step()
+    torch.cuda.synchronize()
+    tot, per, launches, _ = time_steps(step, flush, args.steps, world)
+    _, _, _, kp = time_steps(step, flush, args.steps, world, per_kernel=True)
+    clocks = sampler.stop()
+    tot = max_over_ranks(tot, dev)
+    e2e = None
+    if not args.no_e2e:
+        xh = {k: v.pin_memory() for k, v in x.items()}
+        h2d = 2 * sum(t.numel() * t.element_size() for n, t in xh.items() if n != "dh") + \
+            xh["dh"].numel() * xh["dh"].element_size()
+        d2h = 0
+
+        def e2e_step():
+            nonlocal d2h
+            h = ops.gla_mlstm_fwd(xh["q"], xh["k"], xh["v"], xh["g"], xh["itil"], **kw)
+            r = ops.gla_mlstm_bwd(xh["q"], xh["k"], xh["v"], xh["g"], xh["itil"], xh["dh"], **kw)
+            d2h = sum(t.numel() * t.element_size() for t in [h, *r.values()])
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(args.steps):
+            e2e_step()
+        s1.record()
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(s0.elapsed_time(s1), dev)
+        e2e = {"value": w.B * w.L * args.steps * world / (e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    t = tot / args.steps / 1e3
+    by = fwd_b + bwd_b
+    base.update({"value": w.B * w.L * world / t, "ms_per_step": tot / args.steps, "e2e": e2e,
+                 "gpu_launches": int(launches), "clocks": clocks,
+                 "step_roofline": {"gbs_compulsory": by / t / 1e9, "roofline_us": by / (peaks["hbm_gbs"] * 1e9) * 1e6,
+                                   "frac": by / (peaks["hbm_gbs"] * 1e9) / t, "peak_source": peak_src,
+                                   "bound": "hbm (compulsory bytes of the cell's inputs and outputs)"},
+                 "kernels": {n: {"launches": c, "avg_us": 1e3 * m / c} for n, (c, m) in sorted(kp.items())}})
+    if world == 1 and not args.no_cpu_baseline:
+        tk, dt = mlstm_oracle_sample(0, 1)
+        base["cpu_baseline"] = {"value": tk / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"1 of {w.B * w.H} heads, full L={w.L}, fwd+bwd, float64, {dt:.1f} s"}
+    print(json.dumps(base), flush=True)
+
+
 def time_steps(step, flush, steps, world, per_kernel=False, flush_l2=True):
     """K steps bracketed by barrier + synchronize; per-step CUDA events on the stream, with the
     256 MiB L2 flush before each step outside the events (flush_l2=False: warm L2). per_kernel:
@@ -642,7 +760,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="c3", choices=sorted(I.WORKLOADS) + ["decode", "deltanet", "shard"])
+    ap.add_argument("--workload", default="c3",
+                    choices=sorted(I.WORKLOADS) + ["decode", "deltanet", "shard", "mlstm"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--plan", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--no-e2e", action="store_true")
@@ -654,10 +773,12 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.workload in ("deltanet", "shard"):
+    if args.workload in ("deltanet", "shard", "mlstm"):
         world, rank, local = dist_setup()
         if args.workload == "deltanet":
             run_deltanet(args, world, rank, local)
+        elif args.workload == "mlstm":
+            run_mlstm(args, world, rank, local)
         elif args.impl != "reference":
             run_shard(args, world, rank, local)
         elif rank == 0:

@@ -23,11 +23,13 @@
  *  - q,k,v,o,dO,dq,dk,dv have the I/O dtype of the problem (GLA_F32 or GLA_BF16);
  *    g, i, h0, hT and all their gradients are always float32. Accumulation is fp32.
  *  - g is the log of the decay (g <= 0 for a decay in (0,1]); the library applies no
- *    activation to it. It must be finite. The tensor-core plan factors each tile's in-tile
- *    decays into exponentials that must stay inside the fp32 range; a tile whose decay in
- *    some key dim is stronger than that plan evaluates sets the device status word, so that
- *    gla_check_device_status returns GLA_ERR_RANGE (the results of that call are then not
- *    valid; nothing faults). GLA_PLAN_SIMT evaluates any finite gate.
+ *    activation to it. It must be finite. The tensor-core forward and backward factor each
+ *    64-token tile's in-tile decays into exponentials about one reference row, which must stay
+ *    inside the fp32 range: a tile whose total log-decay in some key dim is below -70 sets the
+ *    device status word, so that gla_check_device_status returns GLA_ERR_RANGE (the results of
+ *    that call are then not valid; nothing faults). GLA_PLAN_SIMT evaluates any finite gate
+ *    (log-space sub-tiles), and the state-only passes (gla_shard_state, gla_shard_state_grad)
+ *    any gate on the tensor cores.
  *  - Every pointer is a DEVICE pointer owned by the caller, 16-byte aligned. The
  *    library allocates nothing; scratch memory is the caller's workspace `ws` of at
  *    least gla_workspace_bytes() bytes (16-byte aligned, contents need not be zeroed).
@@ -166,12 +168,15 @@ GLA_API gla_status gla_decode(const gla_problem* p, const void* q, const void* k
  * gla_shard_state: the shard's end state from a zero initial state, state [B,H,Dk,Dv] f32, and
  *   its total log-decay per key dim, gamma [B,H,Dk] f32 (per-head gates: the head's total in
  *   every key slot). p describes the shard (L = its tokens; L = 0 gives zeros). Tensor-core
- *   state pass: bf16 I/O, chunk a multiple of 64; otherwise GLA_ERR_UNSUPPORTED. ws: at least
- *   256 bytes (device status word, as for gla_fwd). q is not read.
+ *   state pass: bf16 I/O, chunk a multiple of 64; otherwise GLA_ERR_UNSUPPORTED. The pass runs
+ *   in as many segments of the shard as fill the GPU, whose (state, log-decay) pairs one small
+ *   kernel then folds. ws: at least gla_shard_workspace_bytes(p) bytes (the device status word,
+ *   as for gla_fwd, then the segments' pairs), caller-owned device memory. q is not read.
  * gla_state_fold: out = S after S <- h0 (or 0), then for i = 0 .. count-1:
  *   S <- diag(e^{gammas[i]}) S + states[i], with states [count][B,H,Dk,Dv] and gammas
  *   [count][B,H,Dk] f32 as all-gathered; p gives B, H, Dk, Dv. out may not alias the inputs.
  * Errors: GLA_ERR_INVALID_ARG, GLA_ERR_UNSUPPORTED, GLA_ERR_WORKSPACE, GLA_ERR_CUDA. */
+GLA_API size_t gla_shard_workspace_bytes(const gla_problem* p);   /* 0 when p is invalid */
 GLA_API gla_status gla_shard_state(const gla_problem* p, const void* k, const void* v, const float* g,
                                    const float* igate, float* state, float* gamma, void* ws, size_t ws_bytes,
                                    void* stream);
@@ -230,13 +235,38 @@ GLA_API gla_status gla_deltanet_bwd(const gla_problem* p, const void* q, const v
                                     void* dq, void* dk, void* dv, float* dbeta, float* dh0, void* ws,
                                     size_t ws_bytes, void* stream);
 
+/* mLSTM cell: matrix memory with an exponential input gate, a normaliser state and a
+ * max-stabiliser (named by the Tiled Flash Linear Attention abstract as the xLSTM cell its kernels
+ * speed up; the cell is the published xLSTM one). Per (batch, head), with g_t the log forget gate
+ * (<= 0) and i~_t the log of the exponential input gate (any finite real), from zero states:
+ *     C_t = e^{g_t} C_{t-1} + e^{i~_t} k_t^T v_t,   n_t = e^{g_t} n_{t-1} + e^{i~_t} k_t,
+ *     h_t = (scale q_t) C_t / max(|(scale q_t) . n_t|, 1).
+ * The stabilised recurrence (running max m_t of the log weights, states kept times e^{-m_t}, bound
+ * e^{-m_t}) gives the same h_t; here the two sums are gated linear attention passes (values v and a
+ * tile of ones) with the input gate e^{i~ - c}, c the head's largest i~, so no gate exceeds 1.
+ * p: as for gla_fwd with gate = GLA_GATE_PER_HEAD (g [B,H,L] f32 is the log forget gate); plan as
+ *   for gla_fwd (bf16 I/O runs the tensor-core kernels). itil [B,H,L] f32: i~.
+ * gla_mlstm_fwd: h [B,H,L,Dv] (I/O dtype, written).
+ * gla_mlstm_bwd: gradients of sum(dh * h): dq, dk [B,H,L,Dk], dv [B,H,L,Dv] (I/O dtype), dg and
+ *   ditil [B,H,L] f32 (all written). dh [B,H,L,Dv] I/O dtype.
+ * ws: caller-owned device workspace of gla_mlstm_workspace_bytes(p, for_backward) bytes (0 when p
+ *   is invalid or unsupported); gla_check_device_status(ws, stream) reports both passes.
+ * Asynchronous on `stream`: the gated linear attention launches of both passes plus a few small
+ * kernels. Errors: as gla_fwd / gla_bwd; GLA_ERR_INVALID_ARG also for another gate mode. */
+GLA_API size_t gla_mlstm_workspace_bytes(const gla_problem* p, int for_backward);
+GLA_API gla_status gla_mlstm_fwd(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
+                                 const float* itil, void* h, void* ws, size_t ws_bytes, void* stream);
+GLA_API gla_status gla_mlstm_bwd(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
+                                 const float* itil, const void* dh, void* dq, void* dk, void* dv, float* dg,
+                                 float* ditil, void* ws, size_t ws_bytes, void* stream);
+
 /* Static description of a status code (never NULL). */
 GLA_API const char* gla_status_string(gla_status s);
 
 /* Synchronises `stream`, then reads the device status word kept at the start of the
  * workspace of the last call that used `ws`: GLA_OK; GLA_ERR_TIMEOUT when a bounded
  * device-side wait gave up; GLA_ERR_RANGE when the tensor-core plan met a 64-token tile whose
- * total log-decay in some key dim is below -60 (its in-tile factors e^-b would leave the fp32
+ * total log-decay in some key dim is below -70 (its in-tile factors e^-b would leave the fp32
  * range, so that call's results are not valid; GLA_PLAN_SIMT evaluates such gates in log-space
  * sub-tiles); GLA_ERR_CUDA if the synchronisation itself failed. */
 GLA_API gla_status gla_check_device_status(void* ws, void* stream);

@@ -22,7 +22,8 @@ EXPORTED = ("gla_workspace_bytes", "gla_fwd", "gla_bwd", "gla_status_string",
             "gla_profiler_read", "gla_fwd_static_scratch", "gla_last_error_detail", "gla_plan_info",
             "gla_saved_states_bytes", "gla_fwd_save", "gla_bwd_saved", "gla_debug_wait_timeout",
             "gla_decode", "gla_shard_state", "gla_state_fold", "gla_shard_state_grad", "gla_deltanet_fwd",
-            "gla_deltanet_bwd_workspace_bytes", "gla_deltanet_bwd")
+            "gla_deltanet_bwd_workspace_bytes", "gla_deltanet_bwd", "gla_mlstm_workspace_bytes", "gla_mlstm_fwd",
+            "gla_mlstm_bwd", "gla_shard_workspace_bytes")
 
 
 class GlaProblem(ctypes.Structure):
@@ -77,6 +78,8 @@ def _load():
     ip = ctypes.POINTER(ctypes.c_int)
     lib.gla_plan_info.argtypes = [pp, ctypes.c_int, ip, ip, ip]
     lib.gla_plan_info.restype = ctypes.c_int
+    lib.gla_shard_workspace_bytes.argtypes = [pp]
+    lib.gla_shard_workspace_bytes.restype = ctypes.c_size_t
     lib.gla_shard_state.argtypes = [pp] + [ctypes.c_void_p] * 7 + [ctypes.c_size_t, ctypes.c_void_p]
     lib.gla_shard_state.restype = ctypes.c_int
     lib.gla_shard_state_grad.argtypes = [pp] + [ctypes.c_void_p] * 6 + [ctypes.c_size_t, ctypes.c_void_p]
@@ -87,6 +90,12 @@ def _load():
     lib.gla_deltanet_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.gla_deltanet_bwd.argtypes = [pp] + [ctypes.c_void_p] * 13 + [ctypes.c_size_t, ctypes.c_void_p]
     lib.gla_deltanet_bwd.restype = ctypes.c_int
+    lib.gla_mlstm_workspace_bytes.argtypes = [pp, ctypes.c_int]
+    lib.gla_mlstm_workspace_bytes.restype = ctypes.c_size_t
+    lib.gla_mlstm_fwd.argtypes = [pp] + [ctypes.c_void_p] * 7 + [ctypes.c_size_t, ctypes.c_void_p]
+    lib.gla_mlstm_fwd.restype = ctypes.c_int
+    lib.gla_mlstm_bwd.argtypes = [pp] + [ctypes.c_void_p] * 12 + [ctypes.c_size_t, ctypes.c_void_p]
+    lib.gla_mlstm_bwd.restype = ctypes.c_int
     lib.gla_state_fold.argtypes = [pp, ctypes.c_int] + [ctypes.c_void_p] * 5
     lib.gla_state_fold.restype = ctypes.c_int
     lib.gla_decode.argtypes = [pp] + [ctypes.c_void_p] * 8

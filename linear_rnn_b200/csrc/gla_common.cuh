@@ -29,9 +29,12 @@ constexpr size_t kStatusBytes = 256;
 constexpr int kDevStatusOk = 0;
 constexpr int kDevStatusTimeout = 1;   // bits of the device status word
 constexpr int kDevStatusRange = 2;
-// Most negative in-tile total log-decay the tensor-core plans evaluate: their q e^b and
-// k e^-b factors span e^{|Gamma|} within a 64-token tile and must stay inside fp32.
-constexpr float kMinTileLogDecay = -60.f;
+// Most negative in-tile total log-decay the tensor-core plans evaluate. They factor the in-tile
+// decay e^(b_t - b_s) as e^(b_t) e^(-b_s) with one reference row per 64-token tile, so their
+// operands and accumulators carry factors up to e^|Gamma| (k e^-b, sums of up to 64 such terms
+// times O(Dk) products) and down to e^-|Gamma| (q e^b): at |Gamma| = 70 the largest stays about
+// 1e4 below the fp32 / bf16 maximum and the smallest above the smallest normal.
+constexpr float kMinTileLogDecay = -70.f;
 
 // Launch accounting (gla_api.cu): every kernel launch of the library goes through
 // GLA_LAUNCH, which counts it and, while the profiler is enabled, brackets it with CUDA

@@ -36,13 +36,102 @@ __global__ void __launch_bounds__(256) k_state_fold(const float* __restrict__ st
     reinterpret_cast<float4*>(out)[idx] = S;
 }
 
+// A shard's state (or state gradient) from the pairs of its segments, laid out [BH][nseg][Dk][Dv]
+// and [BH][nseg][Dk] by the state pass: S <- diag(e^{Gamma_z}) S + S_z over z = 0 .. nseg-1 from
+// zero (reverse = 1: z = nseg-1 .. 0, the gradient at the shard's start from zero at its end);
+// gamma_out = sum_z Gamma_z. One thread per four consecutive elements of one (bh, key dim) row.
+__global__ void __launch_bounds__(256) k_seg_reduce(const float* __restrict__ seg_state,
+                                                    const float* __restrict__ seg_gamma, float* __restrict__ out,
+                                                    float* __restrict__ gamma_out, int BH, int Dk, int Dv, int nseg,
+                                                    int reverse) {
+    const int per4 = Dk * Dv / 4;
+    const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (long)BH * per4) return;
+    const int bh = (int)(idx / per4), de4 = (int)(idx - (long)bh * per4), d = 4 * de4 / Dv;
+    const float4* src = reinterpret_cast<const float4*>(seg_state) + (size_t)bh * nseg * per4 + de4;
+    const float* gam = seg_gamma + (size_t)bh * nseg * Dk + d;
+    float4 S = make_float4(0.f, 0.f, 0.f, 0.f);
+    float gsum = 0.f;
+    for (int j = 0; j < nseg; ++j) {
+        const int z = reverse ? nseg - 1 - j : j;
+        const float gz = __ldg(gam + (size_t)z * Dk);
+        const float e = __expf(gz);
+        const float4 x = __ldg(src + (size_t)z * per4);
+        S = make_float4(fmaf(e, S.x, x.x), fmaf(e, S.y, x.y), fmaf(e, S.z, x.z), fmaf(e, S.w, x.w));
+        gsum += gz;
+    }
+    reinterpret_cast<float4*>(out)[idx] = S;
+    if (4 * de4 % Dv == 0) gamma_out[(size_t)bh * Dk + d] = gsum;
+}
+
 bool aligned16(const void* x) { return x == nullptr || (reinterpret_cast<uintptr_t>(x) & 15u) == 0; }
 bool dims_ok(const gla_problem* p) {
     return (p->Dk == 64 || p->Dk == 128 || p->Dk == 256) && (p->Dv == 64 || p->Dv == 128 || p->Dv == 256);
 }
 
+// Segments of a shard's state pass: as many as keep its CTAs (one per head, Dv tile and
+// segment) within one wave of the GPU, in whole 64-token tiles.
+struct ShardPlan {
+    int nseg, tps;
+    size_t ws;   // workspace bytes: the status word, then the segments' states and log-decays
+};
+ShardPlan shard_plan(const gla_problem* p) {
+    ShardPlan pl{1, 0, kStatusBytes};
+    const int ntiles = cdiv(p->L, tc::TR);
+    pl.tps = ntiles;
+    // the state-only pass's Dv tile (the rule of the tensor-core forward's state passes)
+    const int sdvt = p->Dv % 128 != 0 ? 64 : p->Dk == 256 ? (p->gate == GLA_GATE_PER_KEY ? 64 : 128)
+                                                           : (p->Dv == 256 ? 256 : 128);
+    const long base = (long)p->B * p->H * (p->Dv / sdvt);
+    if (ntiles <= 1 || base <= 0) return pl;
+    int nseg = (int)(tc::num_sms() / base);
+    if (nseg > ntiles) nseg = ntiles;
+    if (nseg <= 1) return pl;
+    pl.tps = cdiv(ntiles, nseg);
+    pl.nseg = cdiv(ntiles, pl.tps);
+    if (pl.nseg <= 1) {
+        pl.nseg = 1;
+        pl.tps = ntiles;
+        return pl;
+    }
+    const size_t BH = (size_t)p->B * p->H;
+    pl.ws = align_up(kStatusBytes + 4 * BH * pl.nseg * p->Dk * p->Dv, 256) + 4 * BH * pl.nseg * p->Dk;
+    return pl;
+}
+
+// The state-only pass over the shard (mode 3: end states from zero, mode 4: start-state
+// gradients from zero), in segments reduced by k_seg_reduce when the plan has several.
+cudaError_t shard_pass(const gla_problem* p, int mode, const void* a, const void* b, const float* g,
+                       const float* ig, float* out, float* gamma, void* ws, cudaStream_t st) {
+    Dims P;
+    P.B = p->B; P.H = p->H; P.L = p->L; P.Dk = p->Dk; P.Dv = p->Dv; P.C = p->chunk;
+    P.N = cdiv(p->L, p->chunk);
+    P.gate = p->gate;
+    P.scale = p->scale;
+    const ShardPlan pl = shard_plan(p);
+    int* status = static_cast<int*>(ws);
+    if (pl.nseg <= 1) return tc::state_pass(P, mode, a, b, g, ig, 1, pl.tps, out, gamma, status, st);
+    const size_t BH = (size_t)p->B * p->H;
+    float* ss = reinterpret_cast<float*>(static_cast<char*>(ws) + kStatusBytes);
+    float* sg = reinterpret_cast<float*>(static_cast<char*>(ws) +
+                                         align_up(kStatusBytes + 4 * BH * pl.nseg * p->Dk * p->Dv, 256));
+    cudaError_t e = tc::state_pass(P, mode, a, b, g, ig, pl.nseg, pl.tps, ss, sg, status, st);
+    if (e != cudaSuccess) return e;
+    const long n = (long)BH * p->Dk * p->Dv / 4;
+    GLA_LAUNCH("seg_reduce", st,
+               k_seg_reduce<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(ss, sg, out, gamma, (int)BH, p->Dk, p->Dv,
+                                                                          pl.nseg, mode == 4 ? 1 : 0));
+    return cudaGetLastError();
+}
+
 }  // namespace
 }  // namespace gla
+
+extern "C" size_t gla_shard_workspace_bytes(const gla_problem* p) {
+    if (!p || p->B < 0 || p->H < 0 || p->L < 0 || !gla::dims_ok(p)) return 0;
+    if (p->chunk < 64 || p->chunk > 1024 || p->chunk % 64 != 0) return 0;
+    return gla::shard_plan(p).ws;
+}
 
 extern "C" gla_status gla_shard_state(const gla_problem* p, const void* k, const void* v, const float* g,
                                       const float* igate, float* state, float* gamma, void* ws, size_t ws_bytes,
@@ -54,13 +143,13 @@ extern "C" gla_status gla_shard_state(const gla_problem* p, const void* k, const
         return GLA_ERR_UNSUPPORTED;   // the tensor-core state pass: bf16 I/O, whole 64-token tiles
     if ((long long)p->B * p->H > 65535LL) return GLA_ERR_UNSUPPORTED;
     if (!state || !gamma || !ws) return GLA_ERR_INVALID_ARG;
-    if (ws_bytes < gla::kStatusBytes) return GLA_ERR_WORKSPACE;
     const bool empty = (size_t)p->B * p->H * p->L == 0;
     if (!empty && (!k || !v)) return GLA_ERR_INVALID_ARG;
     if (!empty && (p->gate == GLA_GATE_NONE) != (g == nullptr)) return GLA_ERR_INVALID_ARG;
     const void* ptrs[] = {k, v, g, igate, state, gamma, ws};
     for (const void* x : ptrs)
         if (!gla::aligned16(x)) return GLA_ERR_INVALID_ARG;
+    if (ws_bytes < gla::shard_plan(p).ws) return GLA_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e = cudaMemsetAsync(ws, 0, gla::kStatusBytes, st);
     if (e != cudaSuccess) return gla::record_cuda(e, "status word reset");
@@ -71,15 +160,7 @@ extern "C" gla_status gla_shard_state(const gla_problem* p, const void* k, const
         if (e == cudaSuccess) e = cudaMemsetAsync(gamma, 0, 4 * BH * p->Dk, st);
         return gla::record_cuda(e, "empty shard");
     }
-    gla::Dims P;
-    P.B = p->B; P.H = p->H; P.L = p->L; P.Dk = p->Dk; P.Dv = p->Dv; P.C = p->chunk;
-    P.N = gla::cdiv(p->L, p->chunk);
-    P.gate = p->gate;
-    P.scale = p->scale;
-    // the whole shard as the one segment of the state-only pass: one CTA per (head, Dv tile)
-    // walks it (the shards themselves are the sequence parallelism)
-    const int ntiles = gla::cdiv(p->L, gla::tc::TR);
-    e = gla::tc::state_pass(P, 3, k, v, g, igate, 1, ntiles, state, gamma, static_cast<int*>(ws), st);
+    e = gla::shard_pass(p, 3, k, v, g, igate, state, gamma, ws, st);
     return gla::record_cuda(e, "shard state pass");
 }
 
@@ -92,13 +173,13 @@ extern "C" gla_status gla_shard_state_grad(const gla_problem* p, const void* q, 
         return GLA_ERR_UNSUPPORTED;
     if ((long long)p->B * p->H > 65535LL) return GLA_ERR_UNSUPPORTED;
     if (!state_grad || !gamma || !ws) return GLA_ERR_INVALID_ARG;
-    if (ws_bytes < gla::kStatusBytes) return GLA_ERR_WORKSPACE;
     const bool empty = (size_t)p->B * p->H * p->L == 0;
     if (!empty && (!q || !dO)) return GLA_ERR_INVALID_ARG;
     if (!empty && (p->gate == GLA_GATE_NONE) != (g == nullptr)) return GLA_ERR_INVALID_ARG;
     const void* ptrs[] = {q, dO, g, state_grad, gamma, ws};
     for (const void* x : ptrs)
         if (!gla::aligned16(x)) return GLA_ERR_INVALID_ARG;
+    if (ws_bytes < gla::shard_plan(p).ws) return GLA_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e = cudaMemsetAsync(ws, 0, gla::kStatusBytes, st);
     if (e != cudaSuccess) return gla::record_cuda(e, "status word reset");
@@ -109,13 +190,7 @@ extern "C" gla_status gla_shard_state_grad(const gla_problem* p, const void* q, 
         if (e == cudaSuccess) e = cudaMemsetAsync(gamma, 0, 4 * BH * p->Dk, st);
         return gla::record_cuda(e, "empty shard");
     }
-    gla::Dims P;
-    P.B = p->B; P.H = p->H; P.L = p->L; P.Dk = p->Dk; P.Dv = p->Dv; P.C = p->chunk;
-    P.N = gla::cdiv(p->L, p->chunk);
-    P.gate = p->gate;
-    P.scale = p->scale;
-    const int ntiles = gla::cdiv(p->L, gla::tc::TR);
-    e = gla::tc::state_pass(P, 4, q, dO, g, nullptr, 1, ntiles, state_grad, gamma, static_cast<int*>(ws), st);
+    e = gla::shard_pass(p, 4, q, dO, g, nullptr, state_grad, gamma, ws, st);
     return gla::record_cuda(e, "shard state-gradient pass");
 }
 

@@ -1439,6 +1439,11 @@ static BwdPlan plan_bwd(const Dims& P) {
     const int tiles_per_chunk = P.C / TR;
     const int nchunks = cdiv(P.L, P.C);
     if (nseg > nchunks) nseg = nchunks;
+    if (nchunks == 0) {   // L = 0: one empty segment
+        pl.nseg = 1;
+        pl.tiles_per_seg = 0;
+        return pl;
+    }
     const int chunks_per_seg = cdiv(nchunks, nseg);
     pl.tiles_per_seg = chunks_per_seg * tiles_per_chunk;
     pl.nseg = cdiv(ntiles, pl.tiles_per_seg);

@@ -471,7 +471,8 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     gam[d0 + 1] = __expf(G.y);
                     gaml[d0] = G.x;
                     gaml[d0 + 1] = G.y;
-                    if (G.x < kMinTileLogDecay || G.y < kMinTileLogDecay) atomicOr(A.status, kDevStatusRange);
+                    // (the state-only passes scale by whole decays <= 1: any gate strength)
+                    if (MODE == 0 && (G.x < kMinTileLogDecay || G.y < kMinTileLogDecay)) atomicOr(A.status, kDevStatusRange);
                 }
 #pragma unroll
                 for (int u = 0; u < RSF; ++u) {
@@ -557,7 +558,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                 if (sA == 0) {
                     gam[dA] = __expf(G);
                     gaml[dA] = G;
-                    if (G < kMinTileLogDecay) atomicOr(A.status, kDevStatusRange);
+                    if (MODE == 0 && G < kMinTileLogDecay) atomicOr(A.status, kDevStatusRange);
                 }
             } else if (GATE == 2) {
                 if (ttid < 32) {  // warp scan over 64 rows, two rows per lane
@@ -585,7 +586,7 @@ __global__ void __launch_bounds__(NTHR_WS, 1)
                     if (lane == 0) {
                         gam[0] = __expf(G);
                         gaml[0] = G;
-                        if (G < kMinTileLogDecay) atomicOr(A.status, kDevStatusRange);
+                        if (MODE == 0 && G < kMinTileLogDecay) atomicOr(A.status, kDevStatusRange);
                     }
                 }
             }
@@ -968,17 +969,26 @@ FwdPlan plan_fwd(const Dims& P) {
     // plan carries the state through every tile, so the chunk size does not constrain them
     // (segments of whole 256-token chunks cut 1024 tiles into 17 of 60 tiles and one of 4).
     if (nseg > ntiles) nseg = ntiles;
+    if (ntiles == 0) {   // L = 0: one empty segment
+        pl.nseg = 1;
+        pl.tiles_per_seg = 0;
+        return pl;
+    }
     pl.tiles_per_seg = cdiv(ntiles, nseg);
     pl.nseg = cdiv(ntiles, pl.tiles_per_seg);
     if (pl.nseg < 1) pl.nseg = 1;
     return pl;
 }
 
-// Dv tile of the state-only passes: 128 columns wherever the ring keeps several stages (for
-// Dk = 256 with per-key gates a 128-column stage holds 112 KB and the ring a single stage).
+// Dv tile of the state-only passes: the widest whose ring keeps several stages, so that the k
+// (q) and gate tiles a CTA loads serve as many state columns as possible. Dv = 256 in one tile
+// for Dk <= 128 (256 TMEM columns; the final state, up to 128 KB, is staged through the ring);
+// Dk = 256 takes 128 columns, or 64 with per-key gates (a 128-column stage already holds 112 KB
+// and the ring a single stage).
 static int pick_state_dvt(const Dims& P) {
     if (P.Dv % 128 != 0) return 64;
-    return (P.Dk == 256 && P.gate == GLA_GATE_PER_KEY) ? 64 : 128;
+    if (P.Dk == 256) return P.gate == GLA_GATE_PER_KEY ? 64 : 128;
+    return P.Dv == 256 ? 256 : 128;
 }
 
 // The forward's state pass covers segments 0..nseg-2 of the output pass. It runs in R
@@ -1155,10 +1165,12 @@ cudaError_t state_pass(const Dims& P, int mode, const void* a_src, const void* b
                        cudaStream_t st) {
     const int dvt = pick_state_dvt(P);
     if (P.Dk == 64) {
+        if (dvt == 256) return state_gate<64, 256>(P, mode, a_src, b_src, g, ig, nseg, tiles_per_seg, seg_state, seg_gamma, status, st);
         if (dvt == 128) return state_gate<64, 128>(P, mode, a_src, b_src, g, ig, nseg, tiles_per_seg, seg_state, seg_gamma, status, st);
         return state_gate<64, 64>(P, mode, a_src, b_src, g, ig, nseg, tiles_per_seg, seg_state, seg_gamma, status, st);
     }
     if (P.Dk == 128) {
+        if (dvt == 256) return state_gate<128, 256>(P, mode, a_src, b_src, g, ig, nseg, tiles_per_seg, seg_state, seg_gamma, status, st);
         if (dvt == 128) return state_gate<128, 128>(P, mode, a_src, b_src, g, ig, nseg, tiles_per_seg, seg_state, seg_gamma, status, st);
         return state_gate<128, 64>(P, mode, a_src, b_src, g, ig, nseg, tiles_per_seg, seg_state, seg_gamma, status, st);
     }

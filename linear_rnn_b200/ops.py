@@ -131,6 +131,58 @@ def gla_fwd(q, k, v, g=None, igate=None, h0=None, *, scale: Optional[float] = No
     return o, hT
 
 
+def _mlstm_problem(q, v, g, itil, scale, chunk, plan):
+    if g is None or g.dim() != 3 or g.dtype != torch.float32:
+        raise ValueError("g (log forget gate) must be float32 [B, H, L]")
+    if itil is None or itil.dtype != torch.float32 or tuple(itil.shape) != tuple(g.shape):
+        raise ValueError("itil (log input gate) must be float32 [B, H, L] like g")
+    return make_problem(q, v, g, scale=scale, chunk=chunk, plan=plan)
+
+
+def gla_mlstm_fwd(q, k, v, g, itil, *, scale: Optional[float] = None, chunk: int = 64, plan: str = "auto",
+                  workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """mLSTM cell (exponential input gate, normaliser, stabiliser): q, k [B,H,L,Dk], v [B,H,L,Dv],
+    g = log forget gate and itil = log input gate, both fp32 [B,H,L]. Returns h [B,H,L,Dv]."""
+    host = q.device.type != "cuda"
+    device = torch.device("cuda", torch.cuda.current_device()) if host else q.device
+    q, k, v, g, itil = (_to_dev(t, device) for t in (q, k, v, g, itil))
+    prob = _mlstm_problem(q, v, g, itil, scale, chunk, plan)
+    nbytes = int(_lib.lib.gla_mlstm_workspace_bytes(ctypes.byref(prob), 0))
+    if nbytes == 0:
+        raise GlaError(_lib.GLA_ERR_UNSUPPORTED, "gla_mlstm_workspace_bytes")
+    ws = _workspace(nbytes, device, workspace)
+    h = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=device)
+    st = _lib.lib.gla_mlstm_fwd(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(itil), _ptr(h),
+                                _ptr(ws), ws.numel() * ws.element_size(), _stream_handle(device))
+    _check(st, "gla_mlstm_fwd")
+    if host:
+        (h,) = _to_host([h])
+    return h
+
+
+def gla_mlstm_bwd(q, k, v, g, itil, dh, *, scale: Optional[float] = None, chunk: int = 64, plan: str = "auto",
+                  workspace: Optional[torch.Tensor] = None) -> Dict[str, torch.Tensor]:
+    """Gradients of sum(dh * h) of gla_mlstm_fwd: dict dq, dk, dv (io dtype), dg, ditil (fp32)."""
+    host = q.device.type != "cuda"
+    device = torch.device("cuda", torch.cuda.current_device()) if host else q.device
+    q, k, v, g, itil, dh = (_to_dev(t, device) for t in (q, k, v, g, itil, dh))
+    prob = _mlstm_problem(q, v, g, itil, scale, chunk, plan)
+    nbytes = int(_lib.lib.gla_mlstm_workspace_bytes(ctypes.byref(prob), 1))
+    if nbytes == 0:
+        raise GlaError(_lib.GLA_ERR_UNSUPPORTED, "gla_mlstm_workspace_bytes")
+    ws = _workspace(nbytes, device, workspace)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dg, ditil = torch.empty_like(g), torch.empty_like(itil)
+    st = _lib.lib.gla_mlstm_bwd(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(itil), _ptr(dh),
+                                _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(ditil), _ptr(ws),
+                                ws.numel() * ws.element_size(), _stream_handle(device))
+    _check(st, "gla_mlstm_bwd")
+    out = {"dq": dq, "dk": dk, "dv": dv, "dg": dg, "ditil": ditil}
+    if host:
+        out = dict(zip(out, _to_host(list(out.values()))))
+    return out
+
+
 def gla_decode(q, k, v, g, igate, state, *, scale: Optional[float] = None) -> torch.Tensor:
     """One recurrent step per (b, h) from `state` (fp32 [B,H,Dk,Dv] on the GPU, updated in
     place): q, k [B,H,1,Dk], v [B,H,1,Dv], g [B,H,1,Dk] / [B,H,1] / None, igate [B,H,1] / None.
@@ -210,9 +262,10 @@ def gla_shard_state(k, v, g=None, igate=None, *, chunk: int = 64) -> Tuple[torch
     B, H, _, Dk = k.shape
     state = torch.empty(B, H, Dk, v.shape[-1], dtype=torch.float32, device=device)
     gamma = torch.empty(B, H, Dk, dtype=torch.float32, device=device)
-    ws = torch.empty(256, dtype=torch.uint8, device=device)
+    nb = max(int(_lib.lib.gla_shard_workspace_bytes(ctypes.byref(prob))), 256)
+    ws = torch.empty(nb, dtype=torch.uint8, device=device)
     st = _lib.lib.gla_shard_state(ctypes.byref(prob), _ptr(k), _ptr(v), _ptr(g), _ptr(igate), _ptr(state),
-                                  _ptr(gamma), _ptr(ws), 256, _stream_handle(device))
+                                  _ptr(gamma), _ptr(ws), nb, _stream_handle(device))
     _check(st, "gla_shard_state")
     return state, gamma
 
@@ -227,9 +280,10 @@ def gla_shard_state_grad(q, dO, g=None, *, scale: Optional[float] = None,
     B, H, _, Dk = q.shape
     dS = torch.empty(B, H, Dk, dO.shape[-1], dtype=torch.float32, device=device)
     gamma = torch.empty(B, H, Dk, dtype=torch.float32, device=device)
-    ws = torch.empty(256, dtype=torch.uint8, device=device)
+    nb = max(int(_lib.lib.gla_shard_workspace_bytes(ctypes.byref(prob))), 256)
+    ws = torch.empty(nb, dtype=torch.uint8, device=device)
     st = _lib.lib.gla_shard_state_grad(ctypes.byref(prob), _ptr(q), _ptr(dO), _ptr(g), _ptr(dS), _ptr(gamma),
-                                       _ptr(ws), 256, _stream_handle(device))
+                                       _ptr(ws), nb, _stream_handle(device))
     _check(st, "gla_shard_state_grad")
     return dS, gamma
 

@@ -1,0 +1,138 @@
+"""GPU parity of the mLSTM cell (gla_mlstm_fwd / gla_mlstm_bwd) against the float64 oracle
+(oracle/mlstm.py: the stabilised token recurrence and its gradients), on the same seeded
+inputs. Metric per output tensor: max|x - x_ref| / max|x_ref|; bound 1e-2 for bf16 I/O
+(tensor-core plan), 1e-4 for fp32 I/O (CUDA-core plan)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_rnn_b200 import inputs as I
+from oracle import mlstm as ML
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 1e-2}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def f64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def err(got, ref):
+    """max|got - ref| / max|ref|; where the reference is identically zero (dg of a single token),
+    the absolute error instead."""
+    scale = np.abs(ref).max() if ref.size else 0.0
+    return float(np.abs(got - ref).max() / scale) if scale > 0 else float(np.abs(got).max(initial=0.0))
+
+
+def heads_of(t, heads):
+    if heads is None:
+        return t
+    B, H = t.shape[0], t.shape[1]
+    return t.reshape((B * H,) + tuple(t.shape[2:]))[heads][None]
+
+
+def run(w, seed=0, itil_shift=0.0, backward=True, heads=None, plan="auto"):
+    from linear_rnn_b200 import ops
+    x = I.make_mlstm_inputs(w, seed=seed, itil_shift=itil_shift)
+    xd = {k: v.cuda() for k, v in x.items() if v is not None}
+    h = ops.gla_mlstm_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["itil"], scale=w.scale, chunk=w.chunk, plan=plan)
+    xs = {k: heads_of(v, heads) for k, v in x.items() if v is not None}
+    rh, _ = ML.mlstm_fwd(xs["q"], xs["k"], xs["v"], xs["g"], xs["itil"], w.scale)
+    errs = {"h": err(heads_of(f64(h), heads), rh)}
+    if backward:
+        r = ops.gla_mlstm_bwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["itil"], xd["dh"], scale=w.scale, chunk=w.chunk,
+                              plan=plan)
+        ref = ML.mlstm_bwd(xs["q"], xs["k"], xs["v"], xs["g"], xs["itil"], xs["dh"], w.scale)
+        for n in ("dq", "dk", "dv", "dg", "ditil"):
+            errs[n] = err(heads_of(f64(r[n]), heads), ref[n])
+    tol = TOL[w.dtype]
+    bad = {n: e for n, e in errs.items() if not e <= tol}
+    assert not bad, (bad, errs)
+    return errs
+
+
+def small(**kw):
+    return I.MLSTM.replace(B=1, H=2, L=300, **kw)
+
+
+@pytest.mark.parametrize("Dk,Dv", [(64, 64), (128, 128), (128, 256), (256, 256), (64, 256)])
+def test_head_dims_bf16(Dk, Dv):
+    run(small(Dk=Dk, Dv=Dv, scale=Dk ** -0.5), seed=1)
+
+
+@pytest.mark.parametrize("L", [1, 63, 64, 65, 200])
+def test_ragged_lengths(L):
+    run(I.MLSTM.replace(B=2, H=1, L=L, Dk=128, Dv=128, scale=128 ** -0.5), seed=2)
+
+
+def test_fp32_cuda_core_plan():
+    run(small(Dk=64, Dv=128, dtype="f32", scale=64 ** -0.5), seed=3)
+
+
+@pytest.mark.parametrize("shift", [60.0, -20.0])
+def test_input_gates_far_from_zero(shift):
+    """exp(i~) far outside [e^-20, e^60]: the per-head shift keeps the gates in range and h equals
+    the stabilised recurrence."""
+    run(small(Dk=128, Dv=128, scale=128 ** -0.5), seed=4, itil_shift=shift)
+
+
+def test_normaliser_bound_active():
+    """A small scale puts |den| below 1 for many tokens (the bound 1 is the divisor there)."""
+    w = small(Dk=128, Dv=128, scale=0.002)
+    x = I.make_mlstm_inputs(w, seed=5)
+    den, _ = oracle.gla_fwd(x["q"], x["k"], np.ones(tuple(x["v"].shape[:-1]) + (1,)), x["g"], np.exp(f64(x["itil"])),
+                            None, w.scale)
+    frac = float((np.abs(den) < 1).mean())
+    assert 0.2 < frac < 1.0, frac
+    run(w, seed=5)
+
+
+def test_full_size_workload():
+    """The mLSTM workload (B=2 H=8 L=8192 Dk=Dv=256, bf16) on the GPU; two heads against the
+    oracle."""
+    run(I.MLSTM, seed=0, heads=[1, 14])
+
+
+def test_empty_and_deterministic():
+    from linear_rnn_b200 import ops
+    w = small(Dk=128, Dv=128, scale=128 ** -0.5)
+    x = {k: v.cuda() for k, v in I.make_mlstm_inputs(w, seed=6).items()}
+    a = ops.gla_mlstm_bwd(x["q"], x["k"], x["v"], x["g"], x["itil"], x["dh"], scale=w.scale)
+    b = ops.gla_mlstm_bwd(x["q"], x["k"], x["v"], x["g"], x["itil"], x["dh"], scale=w.scale)
+    for n in a:
+        assert torch.equal(a[n], b[n]), n
+    e = {k: v[:, :, :0].contiguous() for k, v in x.items()}
+    h = ops.gla_mlstm_fwd(e["q"], e["k"], e["v"], e["g"], e["itil"], scale=w.scale)
+    assert h.shape == (1, 2, 0, 128)
+
+
+def test_tensor_core_passes_run():
+    """GLA_PLAN_TC runs the two passes on the tensor cores in bf16 (faster; less accurate where
+    |den| sits just above the bound): finite results with a clean status, and h close to the
+    oracle on this input."""
+    from linear_rnn_b200 import ops
+    w = small(Dk=128, Dv=128, scale=128 ** -0.5)
+    x = I.make_mlstm_inputs(w, seed=7)
+    xd = {k: v.cuda() for k, v in x.items()}
+    h = ops.gla_mlstm_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["itil"], scale=w.scale, plan="tc")
+    r = ops.gla_mlstm_bwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["itil"], xd["dh"], scale=w.scale, plan="tc")
+    assert torch.isfinite(h.float()).all() and all(torch.isfinite(t.float()).all() for t in r.values())
+    rh, _ = ML.mlstm_fwd(x["q"], x["k"], x["v"], x["g"], x["itil"], w.scale)
+    assert err(f64(h), rh) <= 0.1
+
+
+def test_rejects_per_key_gates():
+    import ctypes
+    from linear_rnn_b200 import _lib, ops
+    q = torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16, device="cuda")
+    g = torch.zeros(1, 1, 64, 64, device="cuda")
+    p = ops.make_problem(q, q, g, scale=1.0, chunk=64, plan="auto")
+    assert _lib.lib.gla_mlstm_workspace_bytes(ctypes.byref(p), 0) == 0
