@@ -79,14 +79,15 @@ def _mean(xs):
     return sum(xs) / len(xs) if xs else 0.0
 
 
-def kernel_bytes(name, w, fseg=1, bseg=1):
+def kernel_bytes(name, w, fseg=1, bseg=1, bwd_state=False):
     """Bytes of one launch of each kernel, split in two:
     method: the path's own inputs the kernel reads and outputs it writes, each once (q, k, v,
             dO, g, i, h0, dhT in; o, hT, dq, dk, dv, dg, di, dh0 out);
     plan:   the plan's intermediates it reads or writes in the workspace (segment states and
             log-decay totals, the dq kernel's in-segment prefixes of q*dq, saved states).
-    fseg / bseg: sequence segments of the forward / backward plan (gla_plan_info). Returns
-    (method, plan)."""
+    fseg / bseg: sequence segments of the forward / backward plan (gla_plan_info). bwd_state:
+    the backward runs its own state pass and scan (gla_bwd without saved states); the training
+    pair's backward starts from the states its forward saved. Returns (method, plan)."""
     th = w.B * w.H * w.L
     BH = w.B * w.H
     e = io_bytes(w)
@@ -102,6 +103,7 @@ def kernel_bytes(name, w, fseg=1, bseg=1):
     gam = 4.0 * BH * w.Dk                        # one segment's log-decay totals
     frac_f = (fseg - 1) / fseg                   # share of the sequence the state passes cover
     frac_b = (bseg - 1) / bseg
+    bs = bseg > 1 and bwd_state                  # a backward state pass and scan are launched
     di = ig
     table = {
         "simt_cumsum": (ge, ge),
@@ -115,13 +117,13 @@ def kernel_bytes(name, w, fseg=1, bseg=1):
         # forward output pass: reads the segment initial states; the training pair also writes
         # the states the backward's segments start from
         "tc_fwd": (q + k + v + ge + ig + o + s1 + h0, s1 * (fseg - 1) + s1 * (bseg - 1)),
-        "tc_seg_scan": (_mean([h0] * (fseg > 1) + [h0] * (bseg > 1)),
+        "tc_seg_scan": (_mean([h0] * (fseg > 1) + [h0] * bs),
                         _mean([2 * s1 * (fseg - 1) + 2 * gam * (fseg - 1)] * (fseg > 1) +
-                              [2 * s1 * (bseg - 1) + 2 * gam * (bseg - 1)] * (bseg > 1))),
+                              [2 * s1 * (bseg - 1) + 2 * gam * (bseg - 1)] * bs)),
         # the forward's (or the backward's own) state pass over segments 0..nseg-2; per launch
         # averaged when both plans launch one
-        "tc_state": (_mean([frac_f * (k + v + ge + ig)] * (fseg > 1) + [frac_b * (k + v + ge + ig)] * (bseg > 1)),
-                     _mean([(s1 + gam) * (fseg - 1)] * (fseg > 1) + [(s1 + gam) * (bseg - 1)] * (bseg > 1))),
+        "tc_state": (_mean([frac_f * (k + v + ge + ig)] * (fseg > 1) + [frac_b * (k + v + ge + ig)] * bs),
+                     _mean([(s1 + gam) * (fseg - 1)] * (fseg > 1) + [(s1 + gam) * (bseg - 1)] * bs)),
         "tc_gstate": (frac_b * (q + o + ge), (s1 + gam) * (bseg - 1)),
         "tc_seg_rscan": (0.0, 2 * (s1 + gam) * (bseg - 1)),
         "tc_bwd_dq": (q + k + v + o + ge + ig + h0 + q,
@@ -140,8 +142,22 @@ def kernel_bytes(name, w, fseg=1, bseg=1):
 # changed since reports traffic null. `scale`: the capture ran a smaller case of the same
 # workload (`case`); traffic grows with the heads processed.
 MEASURED_TRAFFIC = {
-    ("tc_fwd", "c2"): {"bytes": 187.1e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_fwd.cu",
-                       "sha": "c365d80ff3420b75", "case": "c2"},
+    ("tc_fwd", "c2"): {"bytes": 187.0e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_fwd.cu",
+                       "sha": "889e2c92d7bbe04b", "case": "c2"},
+    ("tc_fwd", "c4"): {"bytes": 805.2e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_fwd.cu",
+                       "sha": "889e2c92d7bbe04b", "case": "c4"},
+    ("tc_fwd", "c3"): {"bytes": 566.8e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_fwd.cu",
+                       "sha": "889e2c92d7bbe04b", "case": "c3 training pair"},
+    ("tc_fwd", "c5"): {"bytes": 295.9e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_fwd.cu",
+                       "sha": "889e2c92d7bbe04b", "case": "c5 training pair"},
+    ("tc_bwd_dkdv", "c3"): {"bytes": 1086.7e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
+                            "sha": "fab635eb697cc988", "case": "c3"},
+    ("tc_bwd_dkdv", "c5"): {"bytes": 484.1e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
+                            "sha": "fab635eb697cc988", "case": "c5"},
+    ("tc_bwd_dq", "c3"): {"bytes": 782.2e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
+                          "sha": "fab635eb697cc988", "case": "c3"},
+    ("tc_bwd_dq", "c5"): {"bytes": 392.6e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
+                          "sha": "fab635eb697cc988", "case": "c5"},
     ("decode", "decode"): {"bytes": 215.2e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_decode.cu",
                            "sha": "1b7b1b10ae6dd931", "case": "decode, 1024 heads"},
 }
