@@ -158,8 +158,8 @@ MEASURED_TRAFFIC = {
                           "sha": "fab635eb697cc988", "case": "c3"},
     ("tc_bwd_dq", "c5"): {"bytes": 392.6e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
                           "sha": "fab635eb697cc988", "case": "c5"},
-    ("decode", "decode"): {"bytes": 215.2e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_decode.cu",
-                           "sha": "1b7b1b10ae6dd931", "case": "decode, 1024 heads"},
+    ("decode", "decode"): {"bytes": 214.9e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_decode.cu",
+                           "sha": "45347f72608393eb", "case": "decode, 1024 heads"},
 }
 
 
@@ -600,8 +600,11 @@ def mlstm_oracle_sample(seed, heads):
 
 def run_mlstm(args, world, rank, local):
     """mLSTM cell forward+backward on its workload (B=2 H=8 L=8192 Dk=Dv=256, bf16): one step is
-    gla_mlstm_fwd then gla_mlstm_bwd through the C ABI on HBM-resident inputs."""
+    gla_mlstm_fwd then gla_mlstm_bwd through the C ABI on HBM-resident inputs. The plan is the
+    tensor-core one (numerator on the tensor cores in bf16, normaliser recurrence in fp32) unless
+    --plan names another."""
     w = I.MLSTM
+    mplan = "tc" if args.plan == "auto" else args.plan
     th = w.B * w.H * w.L
     e = 2
     # compulsory bytes: q, k, v, g, i~ read and h written (forward); q, k, v, g, i~, dh read and
@@ -614,6 +617,7 @@ def run_mlstm(args, world, rank, local):
             "config": {"workload": f"mlstm: exponential input gate, normaliser, stabiliser; B={w.B} H={w.H} L={w.L} "
                                    f"Dk={w.Dk} Dv={w.Dv} chunk={w.chunk} bf16",
                        "global_batch": w.B * world, "seq_len": w.L, "parallelism": f"replicas x{world}",
+                       "plan": mplan,
                        "l2": "256 MiB L2 flush between steps, outside the per-step events; inputs > L2"}}
     if args.impl == "reference":
         if rank != 0:
@@ -638,8 +642,8 @@ def run_mlstm(args, world, rank, local):
     dev = torch.device("cuda", local)
     x = I.make_mlstm_inputs(w, seed=rank)
     xd = {k: v.to(dev) for k, v in x.items()}
-    kw = dict(scale=w.scale, chunk=w.chunk)
-    prob = ops.make_problem(xd["q"], xd["v"], xd["g"], scale=w.scale, chunk=w.chunk, plan="auto")
+    kw = dict(scale=w.scale, chunk=w.chunk, plan=mplan)
+    prob = ops.make_problem(xd["q"], xd["v"], xd["g"], scale=w.scale, chunk=w.chunk, plan=mplan)
     import ctypes
     from linear_rnn_b200 import _lib
     ws = torch.empty(max(_lib.lib.gla_mlstm_workspace_bytes(ctypes.byref(prob), 0),

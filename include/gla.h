@@ -242,10 +242,16 @@ GLA_API gla_status gla_deltanet_bwd(const gla_problem* p, const void* q, const v
  *     C_t = e^{g_t} C_{t-1} + e^{i~_t} k_t^T v_t,   n_t = e^{g_t} n_{t-1} + e^{i~_t} k_t,
  *     h_t = (scale q_t) C_t / max(|(scale q_t) . n_t|, 1).
  * The stabilised recurrence (running max m_t of the log weights, states kept times e^{-m_t}, bound
- * e^{-m_t}) gives the same h_t; here the two sums are gated linear attention passes (values v and a
- * tile of ones) with the input gate e^{i~ - c}, c the head's largest i~, so no gate exceeds 1.
- * p: as for gla_fwd with gate = GLA_GATE_PER_HEAD (g [B,H,L] f32 is the log forget gate); plan as
- *   for gla_fwd (bf16 I/O runs the tensor-core kernels). itil [B,H,L] f32: i~.
+ * e^{-m_t}) gives the same h_t; here both sums use the input gate e^{i~ - c}, c the head's largest
+ * i~, so no gate exceeds 1. The numerator is a gated linear attention pass with values v; the
+ * normaliser n_t (a Dk-vector) is an fp32 recurrence on the CUDA cores, because h divides by
+ * |den| and an error proportional to den's terms would be amplified where |den| is near the bound.
+ * p: as for gla_fwd with gate = GLA_GATE_PER_HEAD (g [B,H,L] f32 is the log forget gate). plan:
+ *   GLA_PLAN_AUTO and GLA_PLAN_SIMT run the numerator on the CUDA cores in fp32 (bf16 inputs are
+ *   converted in the workspace, gradients cast back); GLA_PLAN_TC (bf16 I/O) runs it on the tensor
+ *   cores in bf16: much faster, with the bf16 pass's error carried into h and, where the
+ *   numerator's and normaliser's gradients nearly cancel, amplified in dq and dk.
+ *   itil [B,H,L] f32: i~.
  * gla_mlstm_fwd: h [B,H,L,Dv] (I/O dtype, written).
  * gla_mlstm_bwd: gradients of sum(dh * h): dq, dk [B,H,L,Dk], dv [B,H,L,Dv] (I/O dtype), dg and
  *   ditil [B,H,L] f32 (all written). dh [B,H,L,Dv] I/O dtype.

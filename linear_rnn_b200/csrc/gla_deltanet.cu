@@ -24,7 +24,10 @@
 //      rows sequential; the group splits each dot product and reduces by shuffles);
 //   3. X = T R with R = diag(beta)(V - K S);
 //   4. O = scale (Q S + lower(Q K^T) X) to global memory, and S += K^T X.
+#include <type_traits>
+
 #include "gla_common.cuh"
+#include "gla_plans.h"
 
 namespace gla {
 namespace {
@@ -260,9 +263,12 @@ cudaError_t dn_launch(const gla_problem* p, const void* q, const void* k, const 
     return cudaGetLastError();
 }
 
+// bf16 I/O runs the tensor-core forward (gla_deltanet_tc.cu); fp32 I/O the CUDA-core one above.
 template <typename T>
 cudaError_t dn_launch_dk(const gla_problem* p, const void* q, const void* k, const void* v, const float* beta,
                          const float* h0, void* o, float* hT, float* saved, cudaStream_t st) {
+    if (std::is_same<T, __nv_bfloat16>::value)
+        return tc::deltanet_fwd(p->B, p->H, p->L, p->Dk, p->Dv, p->scale, q, k, v, beta, h0, o, hT, saved, nullptr, st);
     return p->Dk == 64 ? dn_launch<T, 64>(p, q, k, v, beta, h0, o, hT, saved, st)
                        : dn_launch<T, 128>(p, q, k, v, beta, h0, o, hT, saved, st);
 }
@@ -722,7 +728,7 @@ template <typename T, int DK>
 cudaError_t dn_bwd_launch(const gla_problem* p, const void* q, const void* k, const void* v, const float* beta,
                           const float* h0, const void* dO, const float* dhT, void* dq, void* dk, void* dv,
                           float* dbeta, float* dh0, const DnBwdWs& w, cudaStream_t st) {
-    cudaError_t e = dn_launch<T, DK>(p, q, k, v, beta, h0, nullptr, nullptr, w.saved, st);
+    cudaError_t e = dn_launch_dk<T>(p, q, k, v, beta, h0, nullptr, nullptr, w.saved, st);
     if (e != cudaSuccess) return e;
     const int BH = p->B * p->H, NC = (p->L + DN_C - 1) / DN_C;
     auto walk = k_deltanet_bwd_walk<T, DK>;

@@ -1,0 +1,471 @@
+// Chunkwise DeltaNet forward on the tensor cores (tcgen05 / TMEM / TMA), bf16 I/O.
+//
+// The chunk form of the talk summary "Hardware-Efficient Training of Linear Attention Models",
+// sections 22:36 and 31:16 (delta rule with writing strength beta; the WY representation turns
+// the product of a chunk's identity-plus-rank-one transitions into matrix products). In the row
+// form (state S [Dk, Dv], keys and queries rows), for a 64-token chunk entered with S:
+//   T = (I + strict_lower(diag(beta) K K^T))^{-1}      (unit lower triangular)
+//   R = diag(beta) (V - K S),   X = T R
+//   O = scale (Q S + lower(Q K^T) X)                    (lower keeps the diagonal)
+//   S <- S + K^T X
+// One CTA per (batch*head, 64-column value slice): the value columns of the state are
+// independent, so a CTA walks its head's chunks in order with its [Dk, 64] state slice in tensor
+// memory (fp32; the state product accumulates onto it) and a bf16 copy in shared memory as the
+// B operand of K S and Q S. Per chunk:
+//   1. tcgen05: K K^T and Q K^T (M=64 N=64), K S and Q S (M=64 N=64) into tensor memory;
+//   2. CUDA cores: diag(beta) K K^T (strict lower, fp32), P = lower(Q K^T) (bf16), R (bf16);
+//      T by forward substitution in fp32 (rows sequential, columns in parallel), then bf16;
+//   3. tcgen05: X = T R;  4. X to bf16;
+//   5. tcgen05: O = Q S + P X (onto the Q S accumulator), S += K^T X;
+//   6. o = scale O (bf16, TMA store), the state's bf16 copy (and, for the backward, the state
+//      entering the next chunk in fp32).
+// K, Q and V tiles arrive by TMA into a two-stage ring, so the next chunk's loads overlap this
+// chunk's work. Every phase runs on all 8 warps in turn; one elected lane of warp 0 issues the
+// MMAs and the TMA copies.
+#include <cudaTypedefs.h>
+
+#include "gla_common.cuh"
+#include "gla_plans.h"
+#include "gla_tc_common.cuh"
+
+namespace gla {
+namespace tc {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int DT_NT = 256;   // 8 warps: two warpgroups
+constexpr int DT_VT = 64;    // value columns per CTA
+constexpr int DT_TS = 68;    // row stride (floats) of the fp32 T^T used by the substitution
+
+template <int DK>
+struct DtCfg {
+    static constexpr uint32_t KB = TR * DK * 2;   // K tile (bf16, 128-byte swizzled 64-column blocks)
+    static constexpr uint32_t QB = TR * DK * 2;   // Q tile
+    static constexpr uint32_t VB = TR * DT_VT * 2;
+    static constexpr uint32_t STAGE = KB + QB + VB;
+    static constexpr int NS = 2;
+    static constexpr uint32_t SB = DK * DT_VT * 2;        // bf16 state copy (MN-major B: row = key dim)
+    static constexpr uint32_t MB = TR * TR * 2;           // one 64 x 64 bf16 operand (T, P, R, X, O staging)
+    static constexpr uint32_t AF = TR * TR * 4;           // diag(beta) K K^T, fp32 [t][s]
+    static constexpr uint32_t TF = TR * DT_TS * 4;        // T^T, fp32 [c][t]
+    static constexpr uint32_t SMALL = 256 + 4 * TR;
+    static constexpr uint32_t SMEM = NS * STAGE + SB + 5 * MB + AF + TF + SMALL + 1024;
+    // TMEM columns: the state [0, 64) (M = Dk rows), then three M=64 accumulators, each pair in
+    // lanes 0-15 / 16-31 of the same columns: K K^T | Q K^T at 64, K S | Q S (then O) at 128,
+    // X at 192
+    static constexpr uint32_t C_S = 0, C_KK = 64, C_KS = 128, C_X = 192, NCOL = 256;
+    static constexpr int MS = DK == 64 ? 64 : 128;        // M of the state product
+    static_assert(SMEM <= 227 * 1024, "shared memory");
+    static_assert(STAGE % 1024 == 0 && SB % 1024 == 0, "alignment");
+};
+
+struct DtArgs {
+    const float* beta;   // [BH*L]
+    const float* h0;     // [BH, Dk, Dv] or null
+    float* hT;           // [BH, Dk, Dv] or null
+    float* saved;        // [BH, NC, Dk, Dv]: the state entering every chunk, or null
+    int* status;         // device status word (a wait that gave up), or null
+    int L, Dv;
+    float scale;
+};
+
+__device__ __forceinline__ bool dt_wait(uint64_t* bar, uint32_t parity) {
+    const bool ok = mbar_wait(bar, parity);
+    return __syncthreads_and(ok) != 0;
+}
+
+// The CTA's [DK, 64] state slice, row `d` (this thread's TMEM lane), 32 columns from `c`: fp32 to
+// global memory (saved / hT), 128 contiguous bytes per thread.
+__device__ __forceinline__ void dt_put_row(float* dst, const uint32_t* r) {
+#pragma unroll
+    for (int j = 0; j < 32; j += 4)
+        *reinterpret_cast<float4*>(dst + j) =
+            make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                        __uint_as_float(r[j + 3]));
+}
+
+template <int DK, bool OUT>
+__global__ void __launch_bounds__(DT_NT, 1)
+    k_deltanet_tc_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                      const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to, DtArgs A) {
+    using C = DtCfg<DK>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = smem_align1024(smem_raw);
+    uint8_t* sS = sm + C::NS * C::STAGE;
+    uint8_t* sT = sS + C::SB;
+    uint8_t* sP = sT + C::MB;
+    uint8_t* sR = sP + C::MB;
+    uint8_t* sX = sR + C::MB;
+    uint8_t* sO = sX + C::MB;
+    float* sA = reinterpret_cast<float*>(sO + C::MB);
+    float* sTt = sA + TR * TR;
+    uint8_t* small = reinterpret_cast<uint8_t*>(sTt + TR * DT_TS);
+    uint64_t* bar_full = reinterpret_cast<uint64_t*>(small);   // [2]
+    uint64_t* bar_mma = bar_full + 2;
+    uint64_t* bar_drain = bar_full + 3;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 64);
+    float* sB = reinterpret_cast<float*>(small + 256);   // beta of the chunk [64]
+
+    const int bh = blockIdx.x, col0 = blockIdx.y * DT_VT;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2, qd = warp & 3;
+    const int L = A.L, Dv = A.Dv;
+    const int nc = (L + TR - 1) / TR;
+    const long rowbase = (long)bh * L;
+    // state rows: this thread's TMEM lane holds key dim srow (M=64 state: lanes 0-15 only)
+    const bool srow_ok = DK != 64 || lane < 16;
+    const int srow = DK == 64 ? 16 * qd + (lane & 15) : 32 * qd + lane;
+    // M=64 accumulators: lane l < 16 holds row 16 qd + l of the first, l >= 16 of the second
+    const int mrow = 16 * qd + (lane & 15);
+    const bool first = lane < 16;
+
+    if (tid == 0) {
+        mbar_init(&bar_full[0], 1);
+        mbar_init(&bar_full[1], 1);
+        mbar_init(bar_mma, 1);
+        mbar_init(bar_drain, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, C::NCOL);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tq_lane = tbase + ((uint32_t)(32 * qd) << 16);
+
+    auto issue_loads = [&](int c, int s) {
+        uint8_t* st = sm + s * C::STAGE;
+        const int t0 = c * TR;
+        mbar_arrive_expect_tx(&bar_full[s], OUT ? C::STAGE : C::KB + C::VB);
+        for (int cb = 0; cb < DK / 64; ++cb) {
+            tma_load_3d(st + cb * BLK, &tk, cb * 64, t0, bh, &bar_full[s]);
+            if (OUT) tma_load_3d(st + C::KB + cb * BLK, &tq, cb * 64, t0, bh, &bar_full[s]);
+        }
+        tma_load_3d(st + C::KB + C::QB, &tv, col0, t0, bh, &bar_full[s]);
+    };
+    if (tid == 0)
+        for (int c = 0; c < C::NS && c < nc; ++c) issue_loads(c, c);
+
+    // ---- the initial state: TMEM (fp32), its bf16 copy, and the state entering chunk 0
+    {
+        const float* src = A.h0 ? A.h0 + ((long)bh * DK + srow) * Dv + col0 : nullptr;
+        const int c = 32 * wg;
+        float f[32];
+        if (src && srow_ok) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                const float4 x = *reinterpret_cast<const float4*>(src + c + j);
+                f[j] = x.x; f[j + 1] = x.y; f[j + 2] = x.z; f[j + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) f[j] = 0.f;
+        }
+        tmem_st32(tq_lane + C::C_S + c, reinterpret_cast<uint32_t*>(f));
+        if (srow_ok) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) store8_bf16(sS, sw128_off(srow, c + j, DK * 128), f + j);
+            if (A.saved && nc > 0)
+                dt_put_row(A.saved + (((long)bh * nc) * DK + srow) * Dv + col0 + c, reinterpret_cast<uint32_t*>(f));
+        }
+        tmem_wait_st();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    int err = 0, n_mma = 0;
+    for (int c = 0; c < nc; ++c) {
+        const int s = c % C::NS;
+        uint8_t* sk = sm + s * C::STAGE;
+        uint8_t* sq = sk + C::KB;
+        uint8_t* sv = sq + C::QB;
+        const int t0 = c * TR;
+        if (tid < TR) sB[tid] = t0 + tid < L ? A.beta[rowbase + t0 + tid] : 0.f;
+        if (!dt_wait(&bar_full[s], (c / C::NS) & 1)) { err = 1; break; }
+
+        // ---- 1. K K^T, Q K^T, K S, Q S
+        if (warp == 0) {
+            const bool leader = elect_one();
+            tc_fence_after();
+            const uint32_t ka = smem_u32(sk), qa = smem_u32(sq);
+            const uint32_t idAA = idesc_bf16(64, 64, 0, 0), idAS = idesc_bf16(64, DT_VT, 0, 1);
+            const uint64_t dS = sw128_desc(smem_u32(sS), DK * 128, 1024);
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+                if (leader) {
+                    mma_bf16(tbase + C::C_KK, sw128_desc(ka + koff, 16, 1024), sw128_desc(ka + koff, 16, 1024), idAA,
+                             kk > 0);
+                    mma_bf16(tbase + C::C_KS, sw128_desc(ka + koff, 16, 1024), dS + ((kk * 2048) >> 4), idAS, kk > 0);
+                    if (OUT) {
+                        mma_bf16(tbase + C::C_KK + (16u << 16), sw128_desc(qa + koff, 16, 1024),
+                                 sw128_desc(ka + koff, 16, 1024), idAA, kk > 0);
+                        mma_bf16(tbase + C::C_KS + (16u << 16), sw128_desc(qa + koff, 16, 1024), dS + ((kk * 2048) >> 4),
+                                 idAS, kk > 0);
+                    }
+                }
+            }
+            if (leader) mma_commit(bar_mma);
+            __syncwarp();
+        }
+        ++n_mma;
+        if (!dt_wait(bar_mma, (n_mma - 1) & 1)) { err = 1; break; }
+        tc_fence_after();
+
+        // ---- 2a. diag(beta) K K^T (strict lower, fp32) and P = lower(Q K^T) (bf16): one TMEM read,
+        //      K K^T rows in lanes 0-15, Q K^T rows in lanes 16-31; 32 columns per warpgroup
+        {
+            uint32_t r[32];
+            tmem_ld32(tq_lane + C::C_KK + 32 * wg, r);
+            tmem_wait_ld();
+            const int t = mrow;
+            if (first) {
+                const float bt = sB[t];
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    const int sc = 32 * wg + j;
+                    *reinterpret_cast<float4*>(sA + t * TR + sc) =
+                        make_float4(sc < t ? bt * __uint_as_float(r[j]) : 0.f, sc + 1 < t ? bt * __uint_as_float(r[j + 1]) : 0.f,
+                                    sc + 2 < t ? bt * __uint_as_float(r[j + 2]) : 0.f,
+                                    sc + 3 < t ? bt * __uint_as_float(r[j + 3]) : 0.f);
+                }
+            } else if (OUT) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    float f[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int sc = 32 * wg + 8 * u + j;
+                        f[j] = sc <= t ? __uint_as_float(r[8 * u + j]) : 0.f;
+                    }
+                    store8_bf16(sP, sw128_off(t, 32 * wg + 8 * u, BLK), f);
+                }
+            }
+        }
+        // ---- 2b. R = diag(beta) (V - K S) (bf16, laid out like a V tile: the B operand of T R)
+        {
+            uint32_t r[32];
+            tmem_ld32(tq_lane + C::C_KS + 32 * wg, r);
+            tmem_wait_ld();
+            if (first) {
+                const int t = mrow;
+                const float bt = sB[t];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int cc = 32 * wg + 8 * u;
+                    const uint4 vw = *reinterpret_cast<const uint4*>(sv + sw128_off(t, cc, BLK));
+                    const uint32_t* vp = reinterpret_cast<const uint32_t*>(&vw);
+                    float f[8];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vp[j]));
+                        f[2 * j] = bt * (vf.x - __uint_as_float(r[8 * u + 2 * j]));
+                        f[2 * j + 1] = bt * (vf.y - __uint_as_float(r[8 * u + 2 * j + 1]));
+                    }
+                    store8_bf16(sR, sw128_off(t, cc, BLK), f);
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- 2c. T = (I + A)^{-1}: T[t][c] = [t == c] - sum_{c <= i < t} A[t][i] T[i][c], row by row;
+        //      column c = 8 warp + lane / 4, its dot products split over 4 lanes
+        {
+            const int sc = warp * 8 + (lane >> 2), sp = lane & 3;
+            for (int t = 0; t < TR; ++t) {
+                float part = 0.f;
+                for (int i = sc + sp; i < t; i += 4) part = fmaf(sA[t * TR + i], sTt[sc * DT_TS + i], part);
+                part += __shfl_xor_sync(0xffffffffu, part, 1);
+                part += __shfl_xor_sync(0xffffffffu, part, 2);
+                if (sp == 0) sTt[sc * DT_TS + t] = t < sc ? 0.f : t == sc ? 1.f : -part;
+                __syncwarp();
+            }
+        }
+        __syncthreads();
+        // T to bf16, K-major A operand: thread = row t, 16 columns
+        {
+            const int t = tid >> 2, c0 = 16 * (tid & 3);
+            float f[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) f[j] = sTt[(c0 + j) * DT_TS + t];
+            store8_bf16(sT, sw128_off(t, c0, BLK), f);
+            store8_bf16(sT, sw128_off(t, c0 + 8, BLK), f + 8);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ---- 3. X = T R
+        if (warp == 0) {
+            const bool leader = elect_one();
+            const uint32_t idX = idesc_bf16(64, DT_VT, 0, 1);
+            const uint64_t dT = sw128_desc(smem_u32(sT), 16, 1024), dR = sw128_desc(smem_u32(sR), BLK, 1024);
+#pragma unroll
+            for (int ks = 0; ks < TR / 16; ++ks)
+                if (leader) mma_bf16(tbase + C::C_X, dT + ((ks * 32) >> 4), dR + ((ks * 2048) >> 4), idX, ks > 0);
+            if (leader) mma_commit(bar_mma);
+            __syncwarp();
+        }
+        ++n_mma;
+        if (!dt_wait(bar_mma, (n_mma - 1) & 1)) { err = 1; break; }
+        tc_fence_after();
+
+        // ---- 4. X to bf16 (the B operand of P X and K^T X)
+        {
+            uint32_t r[32];
+            tmem_ld32(tq_lane + C::C_X + 32 * wg, r);
+            tmem_wait_ld();
+            if (first)
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    store8_bf16(sX, sw128_off(mrow, 32 * wg + 8 * u, BLK), reinterpret_cast<const float*>(r + 8 * u));
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ---- 5. O = Q S + P X, S += K^T X
+        if (warp == 0) {
+            const bool leader = elect_one();
+            const uint32_t idO = idesc_bf16(64, DT_VT, 0, 1), idS = idesc_bf16(C::MS, DT_VT, 1, 1);
+            const uint64_t dP = sw128_desc(smem_u32(sP), 16, 1024), dX = sw128_desc(smem_u32(sX), BLK, 1024);
+            const uint64_t dKm = sw128_desc(smem_u32(sk), BLK, 1024);
+#pragma unroll
+            for (int ks = 0; ks < TR / 16; ++ks) {
+                if (leader && OUT)
+                    mma_bf16(tbase + C::C_KS + (16u << 16), dP + ((ks * 32) >> 4), dX + ((ks * 2048) >> 4), idO, 1);
+                if (leader) mma_bf16(tbase + C::C_S, dKm + ((ks * 2048) >> 4), dX + ((ks * 2048) >> 4), idS, 1);
+            }
+            if (leader) mma_commit(bar_mma);
+            __syncwarp();
+        }
+        ++n_mma;
+        if (!dt_wait(bar_mma, (n_mma - 1) & 1)) { err = 1; break; }
+        tc_fence_after();
+
+        // ---- 6. o = scale O (bf16 tile -> TMA store); the state's bf16 copy and the state entering
+        //      the next chunk
+        if (OUT) {
+            uint32_t r[32];
+            tmem_ld32(tq_lane + C::C_KS + 32 * wg, r);
+            tmem_wait_ld();
+            if (!first) {
+                float f[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) f[j] = A.scale * __uint_as_float(r[j]);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) store8_bf16(sO, sw128_off(mrow, 32 * wg + 8 * u, BLK), f + 8 * u);
+            }
+        }
+        {
+            uint32_t r[32];
+            tmem_ld32(tq_lane + C::C_S + 32 * wg, r);
+            tmem_wait_ld();
+            if (srow_ok) {
+#pragma unroll
+                for (int j = 0; j < 32; j += 8)
+                    store8_bf16(sS, sw128_off(srow, 32 * wg + j, DK * 128), reinterpret_cast<const float*>(r + j));
+                if (A.saved && c + 1 < nc)
+                    dt_put_row(A.saved + (((long)bh * nc + c + 1) * DK + srow) * Dv + col0 + 32 * wg, r);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0) {
+            if (OUT) {
+                tma_store_3d(&to, sO, col0, t0, bh);
+                bulk_commit();
+            }
+            // every product that read this stage is done: the chunk after next may take it
+            if (c + C::NS < nc) issue_loads(c + C::NS, s);
+            if (OUT) bulk_wait_read<0>();   // the o tile is read before the next chunk rewrites it
+        }
+    }
+
+    if (err) {
+        if (warp == 0) {
+            // every product the issuing lane issued completes before TMEM and shared memory go away
+            const bool leader = elect_one();
+            if (leader) {
+                if (A.status) atomicOr(A.status, kDevStatusTimeout);
+                mma_commit(bar_drain);
+                mbar_wait(bar_drain, 0, 1u << 20);
+            }
+            __syncwarp();
+        }
+    } else if (A.hT) {
+        uint32_t r[32];
+        tmem_ld32(tq_lane + C::C_S + 32 * wg, r);
+        tmem_wait_ld();
+        if (srow_ok) dt_put_row(A.hT + ((long)bh * DK + srow) * Dv + col0 + 32 * wg, r);
+    }
+    if (tid == 0) bulk_wait<0>();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, C::NCOL);
+}
+
+template <int DK, bool OUT>
+cudaError_t dt_launch(int B, int H, int L, int Dv, const CUtensorMap& mq, const CUtensorMap& mk,
+                      const CUtensorMap& mv, const CUtensorMap& mo, const DtArgs& a, cudaStream_t st) {
+    auto kern = k_deltanet_tc_fwd<DK, OUT>;
+    const uint32_t smem = DtCfg<DK>::SMEM;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(B * H, Dv / DT_VT);
+    GLA_LAUNCH(OUT ? "deltanet_fwd" : "deltanet_state", st, (kern<<<grid, DT_NT, smem, st>>>(mq, mk, mv, mo, a)));
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t deltanet_fwd(int B, int H, int L, int Dk, int Dv, float scale, const void* q, const void* k,
+                         const void* v, const float* beta, const float* h0, void* o, float* hT, float* saved,
+                         int* status, cudaStream_t st) {
+    const int BH = B * H;
+    if (BH == 0) return cudaSuccess;
+    if (L == 0) {
+        // no chunk (and no tensor map over an empty sequence): hT = h0 (or zero), nothing else
+        if (hT) {
+            const size_t n = (size_t)BH * Dk * Dv * sizeof(float);
+            return h0 ? cudaMemcpyAsync(hT, h0, n, cudaMemcpyDeviceToDevice, st) : cudaMemsetAsync(hT, 0, n, st);
+        }
+        return cudaSuccess;
+    }
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dk, L, BH, 64, true) ||
+        !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dv, L, BH, 64, true))
+        return cudaErrorInvalidValue;
+    if (o) {
+        if (!make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dk, L, BH, 64, true) ||
+            !make_map(&mo, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dv, L, BH, 64, true))
+            return cudaErrorInvalidValue;
+    } else {
+        mq = mk;
+        mo = mv;
+    }
+    DtArgs a{};
+    a.beta = beta;
+    a.h0 = h0;
+    a.hT = hT;
+    a.saved = saved;
+    a.status = status;
+    a.L = L;
+    a.Dv = Dv;
+    a.scale = scale;
+    if (Dk == 64)
+        return o ? dt_launch<64, true>(B, H, L, Dv, mq, mk, mv, mo, a, st)
+                 : dt_launch<64, false>(B, H, L, Dv, mq, mk, mv, mo, a, st);
+    return o ? dt_launch<128, true>(B, H, L, Dv, mq, mk, mv, mo, a, st)
+             : dt_launch<128, false>(B, H, L, Dv, mq, mk, mv, mo, a, st);
+}
+
+}  // namespace tc
+}  // namespace gla

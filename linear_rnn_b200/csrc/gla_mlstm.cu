@@ -10,14 +10,19 @@
 // (the stabiliser) so that no exp(i~) leaves the floating-point range; the states it keeps
 // are exp(-m_t) times C_t and n_t and its bound exp(-m_t) times 1, so h_t is unchanged.
 //
-// Here num and den are two passes of the gated linear attention kernels (per-head log-decay g,
-// input gate e^{i~ - c}; values v, and a tile of ones whose every output column is den), with
-// c the largest i~ of the head: the same kind of constant shift as the stabiliser, it keeps every
-// input gate <= 1 and turns the bound into e^{-c}. Small kernels then form h, and in the backward
-// the upstream gradients of the two passes,
+// Here num is a pass of the gated linear attention kernels (per-head log-decay g, input gate
+// e^{i~ - c}, values v), with c the largest i~ of the head: the same kind of constant shift as
+// the stabiliser, it keeps every input gate <= 1 and turns the bound into e^{-c}. den is the same
+// sum with a value of one: n_t = e^{g_t} n_{t-1} + e^{i~_t - c} k_t is a Dk-vector recurrence,
+// which runs in fp32 on the CUDA cores (one thread per key dim, the sequence cut into 32-token
+// segments joined by a scan over segment end states), den_t = (scale q_t) . n_t. Small kernels
+// then form h, and in the backward the upstream gradients of the two sums,
 //     dnum = dh / N,   dden = -(dh . h) / N * sign(den) where |den| > e^{-c} (else 0),
 // and, after the two backward passes, the sums of their dq, dk, dg and the chain rule through
-// the input gate, d i~ = (di_num + di_den) e^{i~ - c} (h does not depend on c).
+// the input gate, d i~ = (di_num + di_den) e^{i~ - c} (h does not depend on c). The normaliser's
+// backward is the recurrence's: with dn_t = scale dden_t q_t + e^{g_{t+1}} dn_{t+1},
+//     dq_t = scale dden_t n_t,  dk_t = i_t dn_t,  di_t = k_t . dn_t,  dg_t = (n_t - i_t k_t) . dn_t
+// (i_t the input gate, e^{g_t} n_{t-1} = n_t - i_t k_t).
 #include <math.h>
 #include <stdint.h>
 
@@ -27,6 +32,7 @@ namespace gla {
 namespace {
 
 constexpr int ML_NT = 256;
+constexpr int ML_SL = 32;   // tokens per segment of the normaliser recurrence
 
 template <typename T>
 __device__ __forceinline__ float ld_f(const T* p) { return to_f(*p); }
@@ -50,41 +56,177 @@ __global__ void __launch_bounds__(ML_NT) k_mlstm_prep(const float* __restrict__ 
     for (int t = threadIdx.x; t < L; t += ML_NT) ig[bh * L + t] = expf(x[t] - c);
 }
 
-template <typename T>
-__global__ void k_fill_ones(T* __restrict__ p, long n) {
-    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x)
-        p[i] = from_f<T>(1.f);
-}
-
 template <typename Tin, typename Tout>
 __global__ void k_cast(const Tin* __restrict__ a, Tout* __restrict__ b, long n) {
     for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x)
         b[i] = from_f<Tout>(to_f(a[i]));
 }
 
+// ---- the normaliser recurrence n_t = e^{g_t} n_{t-1} + i_t k_t, fp32, one thread per key dim,
+// grid (segment, batch*head) with blocks of Dk threads
+
+// the segment's end state from zero and its total log-decay
+template <typename T>
+__global__ void k_mlstm_nloc(const T* __restrict__ k, const float* __restrict__ g, const float* __restrict__ ig,
+                             int L, int Dk, int nseg, float* __restrict__ nloc, float* __restrict__ gam) {
+    const long bh = blockIdx.y;
+    const int s = blockIdx.x, d = threadIdx.x;
+    const int t0 = s * ML_SL, t1 = min(L, t0 + ML_SL);
+    float n = 0.f, G = 0.f;
+#pragma unroll 8
+    for (int t = t0; t < t1; ++t) {
+        const float gt = g[bh * L + t];
+        n = __expf(gt) * n + ig[bh * L + t] * to_f(k[(bh * L + t) * Dk + d]);
+        G += gt;
+    }
+    nloc[(bh * nseg + s) * Dk + d] = n;
+    if (d == 0) gam[bh * nseg + s] = G;
+}
+
+// the state entering every segment (grid batch*head, blocks of Dk threads)
+__global__ void k_mlstm_nscan(const float* __restrict__ nloc, const float* __restrict__ gam, int nseg, int Dk,
+                              float* __restrict__ nstart) {
+    const long bh = blockIdx.x;
+    const int d = threadIdx.x;
+    float n = 0.f;
+#pragma unroll 8
+    for (int s = 0; s < nseg; ++s) {
+        const long i = (bh * nseg + s) * Dk + d;
+        nstart[i] = n;
+        n = __expf(gam[bh * nseg + s]) * n + nloc[i];
+    }
+}
+
+// sum over the block's Dk threads of one value per thread, for token slot j: warp sums into part
+template <int NW>
+__device__ __forceinline__ void ml_warp_part(float x, float (*part)[NW], int j) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    if ((threadIdx.x & 31) == 0) part[j][threadIdx.x >> 5] = x;
+}
+
+// den_t = scale q_t . n_t over the segment (den [BH*L] fp32)
+template <typename T>
+__global__ void k_mlstm_den(const T* __restrict__ q, const T* __restrict__ k, const float* __restrict__ g,
+                            const float* __restrict__ ig, const float* __restrict__ nstart, int L, int Dk, int nseg,
+                            float scale, float* __restrict__ den) {
+    __shared__ float part[ML_SL][8];
+    const long bh = blockIdx.y;
+    const int s = blockIdx.x, d = threadIdx.x, nw = Dk / 32;
+    const int t0 = s * ML_SL, cnt = min(L - t0, ML_SL);
+    float n = nstart[(bh * nseg + s) * Dk + d];
+#pragma unroll 4
+    for (int j = 0; j < cnt; ++j) {
+        const long r = bh * L + t0 + j;
+        n = __expf(g[r]) * n + ig[r] * to_f(k[r * Dk + d]);
+        ml_warp_part<8>(to_f(q[r * Dk + d]) * n, part, j);
+    }
+    __syncthreads();
+    if (d < cnt) {
+        float x = 0.f;
+        for (int w = 0; w < nw; ++w) x += part[d][w];
+        den[bh * L + t0 + d] = scale * x;
+    }
+}
+
+// backward, local: the gradient carried out of the segment's start from a zero carry at its end,
+// c = e^{g_t} dn_t with dn_t = scale dden_t q_t + c (walking the segment backwards)
+template <typename T>
+__global__ void k_mlstm_dnloc(const T* __restrict__ q, const float* __restrict__ g, const float* __restrict__ dden,
+                              int L, int Dk, int nseg, float scale, float* __restrict__ cloc) {
+    const long bh = blockIdx.y;
+    const int s = blockIdx.x, d = threadIdx.x;
+    const int t0 = s * ML_SL, t1 = min(L, t0 + ML_SL);
+    float c = 0.f;
+#pragma unroll 8
+    for (int t = t1 - 1; t >= t0; --t) {
+        const long r = bh * L + t;
+        c = __expf(g[r]) * (scale * dden[r] * to_f(q[r * Dk + d]) + c);
+    }
+    cloc[(bh * nseg + s) * Dk + d] = c;
+}
+
+// the carry entering every segment from the segments after it (grid batch*head)
+__global__ void k_mlstm_cscan(const float* __restrict__ cloc, const float* __restrict__ gam, int nseg, int Dk,
+                              float* __restrict__ cin) {
+    const long bh = blockIdx.x;
+    const int d = threadIdx.x;
+    float c = 0.f;
+#pragma unroll 8
+    for (int s = nseg - 1; s >= 0; --s) {
+        const long i = (bh * nseg + s) * Dk + d;
+        cin[i] = c;
+        c = __expf(gam[bh * nseg + s]) * c + cloc[i];
+    }
+}
+
+// the normaliser's gradients over a segment: n_t forward from the segment's start state (kept in
+// shared memory), then dn_t backwards from the carry entering the segment's end
+template <typename T>
+__global__ void k_mlstm_den_bwd(const T* __restrict__ q, const T* __restrict__ k, const float* __restrict__ g,
+                                const float* __restrict__ ig, const float* __restrict__ dden,
+                                const float* __restrict__ nstart, const float* __restrict__ cin, int L, int Dk, int nseg,
+                                float scale, float* __restrict__ dq2, float* __restrict__ dk2, float* __restrict__ dg2,
+                                float* __restrict__ di2) {
+    __shared__ float pi[ML_SL][8], pg[ML_SL][8];
+    __shared__ float nv[ML_SL][256];   // n_t of the segment's tokens, [token][key dim]
+    const long bh = blockIdx.y;
+    const int s = blockIdx.x, d = threadIdx.x, nw = Dk / 32;
+    const int t0 = s * ML_SL, cnt = min(L - t0, ML_SL);
+    const long r0 = bh * L + t0;
+    float n = nstart[(bh * nseg + s) * Dk + d];
+#pragma unroll 8
+    for (int j = 0; j < cnt; ++j) {
+        n = __expf(g[r0 + j]) * n + ig[r0 + j] * to_f(k[(r0 + j) * Dk + d]);
+        nv[j][d] = n;
+    }
+    float c = cin[(bh * nseg + s) * Dk + d];
+#pragma unroll 4
+    for (int j = cnt - 1; j >= 0; --j) {
+        const long r = r0 + j;
+        const float sd = scale * dden[r], it = ig[r], kt = to_f(k[r * Dk + d]), nj = nv[j][d];
+        const float dn = sd * to_f(q[r * Dk + d]) + c;
+        dq2[r * Dk + d] = sd * nj;
+        dk2[r * Dk + d] = it * dn;
+        ml_warp_part<8>(kt * dn, pi, j);
+        ml_warp_part<8>((nj - it * kt) * dn, pg, j);
+        c = __expf(g[r]) * dn;
+    }
+    __syncthreads();
+    if (d < cnt) {
+        float xi = 0.f, xg = 0.f;
+        for (int w = 0; w < nw; ++w) {
+            xi += pi[d][w];
+            xg += pg[d][w];
+        }
+        di2[r0 + d] = xi;
+        dg2[r0 + d] = xg;
+    }
+}
+
 // One warp per token row: N = max(|den|, e^{-c}), h = num / N.
-template <typename Ti, typename To>
-__global__ void __launch_bounds__(ML_NT) k_mlstm_norm(const Ti* __restrict__ num, const Ti* __restrict__ den,
+template <typename Ta, typename To>
+__global__ void __launch_bounds__(ML_NT) k_mlstm_norm(const Ta* __restrict__ num, const float* __restrict__ den,
                                                       const float* __restrict__ cst, To* __restrict__ h, long rows,
-                                                      int L, int Dv, int Dvn) {
+                                                      int L, int Dv) {
     const long row = blockIdx.x * (long)(ML_NT / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
-    const float N = fmaxf(fabsf(ld_f(den + row * Dvn)), expf(-cst[row / L]));
+    const float N = fmaxf(fabsf(den[row]), expf(-cst[row / L]));
     const float inv = 1.f / N;
     for (int e = lane; e < Dv; e += 32) h[row * Dv + e] = from_f<To>(ld_f(num + row * Dv + e) * inv);
 }
 
-// One warp per token row: the upstream gradients of the two passes.
-template <typename Ti, typename To>
-__global__ void __launch_bounds__(ML_NT) k_mlstm_bwd_prep(const Ti* __restrict__ num, const Ti* __restrict__ den,
+// One warp per token row: the upstream gradients of the two sums.
+template <typename Ta, typename To>
+__global__ void __launch_bounds__(ML_NT) k_mlstm_bwd_prep(const Ta* __restrict__ num, const float* __restrict__ den,
                                                           const float* __restrict__ cst, const To* __restrict__ dh,
-                                                          Ti* __restrict__ dnum, Ti* __restrict__ dden, long rows, int L,
-                                                          int Dv, int Dvn) {
+                                                          Ta* __restrict__ dnum, float* __restrict__ dden, long rows,
+                                                          int L, int Dv) {
     const long row = blockIdx.x * (long)(ML_NT / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
-    const float dn = ld_f(den + row * Dvn);
+    const float dn = den[row];
     const float bound = expf(-cst[row / L]);
     const float N = fmaxf(fabsf(dn), bound);
     const float inv = 1.f / N;
@@ -92,28 +234,27 @@ __global__ void __launch_bounds__(ML_NT) k_mlstm_bwd_prep(const Ti* __restrict__
     for (int e = lane; e < Dv; e += 32) {
         const float d = ld_f(dh + row * Dv + e);
         s += d * ld_f(num + row * Dv + e) * inv;
-        dnum[row * Dv + e] = from_f<Ti>(d * inv);
+        dnum[row * Dv + e] = from_f<Ta>(d * inv);
     }
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    const float dd = fabsf(dn) > bound ? -s * inv * (dn > 0.f ? 1.f : -1.f) : 0.f;
-    for (int e = lane; e < Dvn; e += 32) dden[row * Dvn + e] = from_f<Ti>(e == 0 ? dd : 0.f);
+    if (lane == 0) dden[row] = fabsf(dn) > bound ? -s * inv * (dn > 0.f ? 1.f : -1.f) : 0.f;
 }
 
-// dq = dq1 + dq2 and dk = dk1 + dk2 (n_qk elements), dv = dv1 (n_v elements, only when the passes
-// ran in another type than the outputs), dg = dg1 + dg2 and d i~ = (di1 + di2) * e^{i~ - c}
+// dq = dq1 + dq2 and dk = dk1 + dk2 (n_qk elements), dv = dv1 (n_v elements, only when the value
+// pass ran in another type than the outputs), dg += dg2 and d i~ = (di1 + di2) * e^{i~ - c}
 // (n_t tokens). dq1 / dk1 / dv1 may be the outputs themselves.
-template <typename Ti, typename To>
-__global__ void k_mlstm_bwd_final(To* dq, To* dk, To* dv, const Ti* dq1, const Ti* dk1, const Ti* dv1,
-                                  const Ti* __restrict__ dq2, const Ti* __restrict__ dk2, long n_qk, long n_v,
+template <typename Ta, typename To>
+__global__ void k_mlstm_bwd_final(To* dq, To* dk, To* dv, const Ta* dq1, const Ta* dk1, const Ta* dv1,
+                                  const float* __restrict__ dq2, const float* __restrict__ dk2, long n_qk, long n_v,
                                   float* __restrict__ dg, const float* __restrict__ dg2, const float* __restrict__ di1,
                                   const float* __restrict__ di2, const float* __restrict__ ig,
                                   float* __restrict__ ditil, long n_t) {
     const long stride = (long)gridDim.x * blockDim.x;
     const long i0 = blockIdx.x * (long)blockDim.x + threadIdx.x;
     for (long i = i0; i < n_qk; i += stride) {
-        dq[i] = from_f<To>(to_f(dq1[i]) + to_f(dq2[i]));
-        dk[i] = from_f<To>(to_f(dk1[i]) + to_f(dk2[i]));
+        dq[i] = from_f<To>(to_f(dq1[i]) + dq2[i]);
+        dk[i] = from_f<To>(to_f(dk1[i]) + dk2[i]);
     }
     for (long i = i0; i < n_v; i += stride) dv[i] = from_f<To>(to_f(dv1[i]));
     for (long i = i0; i < n_t; i += stride) {
@@ -122,24 +263,19 @@ __global__ void k_mlstm_bwd_final(To* dq, To* dk, To* dv, const Ti* dq1, const T
     }
 }
 
-// The device status word of the second pass joins the first (the one at the workspace start).
-__global__ void k_status_or(int* a, const int* b) { atomicOr(a, *b); }
-
 bool ml_aligned16(const void* x) { return x == nullptr || (reinterpret_cast<uintptr_t>(x) & 15u) == 0; }
 
 struct MlLayout {
-    gla_problem pa, pb;   // value pass, normaliser pass (a tile of Dvn ones)
-    bool f32;             // the passes run with fp32 I/O (converted copies of bf16 inputs)
-    bool cast;            // ... and the I/O is bf16: inputs are converted, gradients cast back
-    size_t wsa, wsb;      // the passes' workspace bytes
-    size_t o_wsb, o_ig, o_c, o_qf, o_kf, o_vf, o_num, o_den, o_ones;
-    size_t o_dnum, o_dden, o_dq1, o_dk1, o_dv1, o_dq2, o_dk2, o_dv2, o_dg2, o_di1, o_di2;
+    gla_problem pa;       // the value pass
+    bool fa;              // the value pass runs with fp32 I/O
+    bool cast_a;          // ... on bf16 I/O: converted copies of q, k, v, and its gradients are
+                          // cast back
+    int nseg;             // 32-token segments of the normaliser recurrence
+    size_t wsa;           // the value pass's workspace bytes
+    size_t o_ig, o_c, o_qf, o_kf, o_vf, o_num, o_den, o_nloc, o_gam, o_nst;
+    size_t o_dnum, o_dden, o_dq1, o_dk1, o_dv1, o_dq2, o_dk2, o_dg2, o_di1, o_di2, o_cloc, o_cin;
     size_t total;
 };
-
-// Width of the normaliser pass's value tile: the smallest head dim whose tensor-core backward
-// runs with this key dim (key dim 256 needs 128).
-int ml_dvn(const gla_problem* p) { return p->Dk > 128 ? 128 : 64; }
 
 gla_status ml_layout(const gla_problem* p, bool bwd, MlLayout* w) {
     if (!p || p->B < 0 || p->H < 0 || p->L < 0) return GLA_ERR_INVALID_ARG;
@@ -147,59 +283,57 @@ gla_status ml_layout(const gla_problem* p, bool bwd, MlLayout* w) {
     if (p->io != GLA_F32 && p->io != GLA_BF16) return GLA_ERR_INVALID_ARG;
     if (p->plan < GLA_PLAN_AUTO || p->plan > GLA_PLAN_TC) return GLA_ERR_INVALID_ARG;
     w->pa = *p;
-    w->pb = *p;
-    w->pb.Dv = ml_dvn(p);
-    // The automatic plan (and GLA_PLAN_SIMT) runs both passes on the CUDA cores with fp32 I/O:
-    // h divides by |den| wherever |den| exceeds the bound, den is a sum of terms of both signs,
-    // and the gradients add the two passes' parts, which can nearly cancel. An error proportional
-    // to the terms (bf16 operands and bf16-rounded partial results) then becomes a large relative
-    // error where |den| sits just above the bound. GLA_PLAN_TC runs the tensor-core passes in the
-    // I/O dtype instead (faster, less accurate there).
-    w->f32 = p->plan != GLA_PLAN_TC;
-    w->cast = w->f32 && p->io == GLA_BF16;
-    if (w->f32) {
-        w->pa.plan = w->pb.plan = GLA_PLAN_SIMT;
-        w->pa.io = w->pb.io = GLA_F32;
-    }
-    auto need = [&](const gla_problem* q) {
-        const size_t f = gla_workspace_bytes(q, 0);
-        const size_t b = bwd ? gla_workspace_bytes(q, 1) : 0;
-        return (f == 0 || (bwd && b == 0)) ? (size_t)0 : (f > b ? f : b);
-    };
-    w->wsa = need(&w->pa);
-    w->wsb = need(&w->pb);
-    if (w->wsa == 0 || w->wsb == 0) return GLA_ERR_UNSUPPORTED;   // the verdict gla_fwd / gla_bwd give
+    // h divides by |den| wherever |den| exceeds the bound, and den is a sum of terms of both
+    // signs: an error proportional to the terms becomes a large relative error of h where |den|
+    // sits just above the bound, and the gradients add the two sums' parts, which can nearly
+    // cancel. So the normaliser always runs as its fp32 recurrence (a Dk-vector state, a small
+    // share of the work). The value pass runs on the CUDA cores in fp32 (the automatic plan and
+    // GLA_PLAN_SIMT; fp32 I/O always), or with GLA_PLAN_TC on the tensor cores in bf16: much
+    // faster, with the bf16 pass's error carried into h and, through the cancellation, into dq
+    // and dk.
+    const bool bf = p->io == GLA_BF16;
+    w->fa = !bf || p->plan != GLA_PLAN_TC;
+    w->cast_a = bf && w->fa;
+    w->pa.plan = w->fa ? GLA_PLAN_SIMT : GLA_PLAN_TC;
+    if (w->fa) w->pa.io = GLA_F32;
+    const size_t f = gla_workspace_bytes(&w->pa, 0);
+    const size_t b = bwd ? gla_workspace_bytes(&w->pa, 1) : 0;
+    w->wsa = (f == 0 || (bwd && b == 0)) ? 0 : (f > b ? f : b);
+    if (w->wsa == 0) return GLA_ERR_UNSUPPORTED;   // the verdict gla_fwd / gla_bwd give
     const size_t BHL = (size_t)p->B * p->H * p->L, BH = (size_t)p->B * p->H;
-    const size_t e = w->f32 ? 4 : 2;   // bytes of the passes' elements
-    const int Dvn = w->pb.Dv;
+    const size_t ea = w->fa ? 4 : 2;   // bytes of the value pass's elements
+    w->nseg = (p->L + ML_SL - 1) / ML_SL;
+    const size_t NS = BH * (size_t)w->nseg;
     size_t off = align_up(w->wsa, 256);
     auto take = [&](size_t bytes) {
         const size_t o = off;
         off = align_up(off + bytes, 256);
         return o;
     };
-    w->o_wsb = take(w->wsb);
     w->o_ig = take(4 * BHL);
     w->o_c = take(4 * BH);
-    if (w->cast) {
+    if (w->cast_a) {
         w->o_qf = take(4 * BHL * p->Dk);
         w->o_kf = take(4 * BHL * p->Dk);
         w->o_vf = take(4 * BHL * p->Dv);
     }
-    w->o_num = take(e * BHL * p->Dv);
-    w->o_den = take(e * BHL * Dvn);
-    w->o_ones = take(e * BHL * Dvn);
+    w->o_num = take(ea * BHL * p->Dv);
+    w->o_den = take(4 * BHL);
+    w->o_nloc = take(4 * NS * p->Dk);
+    w->o_gam = take(4 * NS);
+    w->o_nst = take(4 * NS * p->Dk);
     if (bwd) {
-        w->o_dnum = take(e * BHL * p->Dv);
-        w->o_dden = take(e * BHL * Dvn);
-        if (w->cast) {
+        w->o_dnum = take(ea * BHL * p->Dv);
+        w->o_dden = take(4 * BHL);
+        if (w->cast_a) {
             w->o_dq1 = take(4 * BHL * p->Dk);
             w->o_dk1 = take(4 * BHL * p->Dk);
             w->o_dv1 = take(4 * BHL * p->Dv);
         }
-        w->o_dq2 = take(e * BHL * p->Dk);
-        w->o_dk2 = take(e * BHL * p->Dk);
-        w->o_dv2 = take(e * BHL * Dvn);
+        w->o_dq2 = take(4 * BHL * p->Dk);
+        w->o_dk2 = take(4 * BHL * p->Dk);
+        w->o_cloc = take(4 * NS * p->Dk);
+        w->o_cin = take(4 * NS * p->Dk);
         w->o_dg2 = take(4 * BHL);
         w->o_di1 = take(4 * BHL);
         w->o_di2 = take(4 * BHL);
@@ -213,20 +347,25 @@ unsigned ml_grid(long n, int nt) {
     return (unsigned)(b < 1 ? 1 : b > 148L * 16 ? 148L * 16 : b);
 }
 
+// The inputs the value pass reads (the caller's, or converted fp32 copies in the workspace).
+struct MlInputs {
+    const void *qa, *ka, *va;
+};
+
 // Shared by the forward and the backward: the input gate, fp32 copies of bf16 inputs where the
-// passes run in fp32, the ones tile, and the two forward passes (num, den) in the workspace.
-// q, k, v are replaced by the pointers the passes read.
-template <typename Ti, typename To>
-gla_status ml_forward_passes(const gla_problem* p, const MlLayout& w, const void*& q, const void*& k, const void*& v,
-                             const float* g, const float* itil, char* ws, cudaStream_t st) {
+// value pass runs in fp32, num (the value pass) and den (the normaliser recurrence) in the
+// workspace.
+template <typename Ta, typename To>
+gla_status ml_forward_passes(const gla_problem* p, const MlLayout& w, const void* q, const void* k, const void* v,
+                             const float* g, const float* itil, char* ws, MlInputs* in, cudaStream_t st) {
     const long BH = (long)p->B * p->H, BHL = BH * p->L;
     float* ig = reinterpret_cast<float*>(ws + w.o_ig);
     float* cst = reinterpret_cast<float*>(ws + w.o_c);
-    Ti* ones = reinterpret_cast<Ti*>(ws + w.o_ones);
+    *in = MlInputs{q, k, v};
     GLA_LAUNCH("mlstm_prep", st, k_mlstm_prep<<<(unsigned)BH, ML_NT, 0, st>>>(itil, p->L, ig, cst));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return record_cuda(e, "mLSTM gate launch");
-    if (w.cast) {
+    if (w.cast_a) {
         const long nq = BHL * p->Dk, nv = BHL * p->Dv;
         float* qf = reinterpret_cast<float*>(ws + w.o_qf);
         float* kf = reinterpret_cast<float*>(ws + w.o_kf);
@@ -235,50 +374,54 @@ gla_status ml_forward_passes(const gla_problem* p, const MlLayout& w, const void
         GLA_LAUNCH("mlstm_cast", st, (k_cast<To, float><<<ml_grid(nq, 256), 256, 0, st>>>(static_cast<const To*>(k), kf, nq)));
         GLA_LAUNCH("mlstm_cast", st, (k_cast<To, float><<<ml_grid(nv, 256), 256, 0, st>>>(static_cast<const To*>(v), vf, nv)));
         if ((e = cudaGetLastError()) != cudaSuccess) return record_cuda(e, "mLSTM input conversion launch");
-        q = qf;
-        k = kf;
-        v = vf;
+        *in = MlInputs{qf, kf, vf};
     }
-    const long nones = BHL * w.pb.Dv;
-    GLA_LAUNCH("mlstm_ones", st, k_fill_ones<Ti><<<ml_grid(nones, 256), 256, 0, st>>>(ones, nones));
-    if ((e = cudaGetLastError()) != cudaSuccess) return record_cuda(e, "mLSTM ones launch");
-    gla_status s = gla_fwd(&w.pa, q, k, v, g, ig, nullptr, ws + w.o_num, nullptr, ws, w.wsa, st);
+    gla_status s = gla_fwd(&w.pa, in->qa, in->ka, in->va, g, ig, nullptr, ws + w.o_num, nullptr, ws, w.wsa, st);
     if (s != GLA_OK) return s;
-    return gla_fwd(&w.pb, q, k, ones, g, ig, nullptr, ws + w.o_den, nullptr, ws + w.o_wsb, w.wsb, st);
+    // the normaliser recurrence, reading q and k in the I/O dtype
+    const To* tq = static_cast<const To*>(q);
+    const To* tk = static_cast<const To*>(k);
+    float* nloc = reinterpret_cast<float*>(ws + w.o_nloc);
+    float* gam = reinterpret_cast<float*>(ws + w.o_gam);
+    float* nst = reinterpret_cast<float*>(ws + w.o_nst);
+    const dim3 grid(w.nseg, (unsigned)BH);
+    GLA_LAUNCH("mlstm_nloc", st, k_mlstm_nloc<To><<<grid, p->Dk, 0, st>>>(tk, g, ig, p->L, p->Dk, w.nseg, nloc, gam));
+    GLA_LAUNCH("mlstm_nscan", st, k_mlstm_nscan<<<(unsigned)BH, p->Dk, 0, st>>>(nloc, gam, w.nseg, p->Dk, nst));
+    GLA_LAUNCH("mlstm_den", st,
+               k_mlstm_den<To><<<grid, p->Dk, 0, st>>>(tq, tk, g, ig, nst, p->L, p->Dk, w.nseg, p->scale,
+                                                       reinterpret_cast<float*>(ws + w.o_den)));
+    return record_cuda(cudaGetLastError(), "mLSTM normaliser launch");
 }
 
-template <typename Ti, typename To>
+template <typename Ta, typename To>
 gla_status ml_fwd(const gla_problem* p, const MlLayout& w, const void* q, const void* k, const void* v,
                   const float* g, const float* itil, void* h, char* ws, cudaStream_t st) {
-    gla_status s = ml_forward_passes<Ti, To>(p, w, q, k, v, g, itil, ws, st);
+    MlInputs in;
+    gla_status s = ml_forward_passes<Ta, To>(p, w, q, k, v, g, itil, ws, &in, st);
     if (s != GLA_OK) return s;
     const long rows = (long)p->B * p->H * p->L;
     GLA_LAUNCH("mlstm_norm", st,
-               (k_mlstm_norm<Ti, To><<<(unsigned)((rows + ML_NT / 32 - 1) / (ML_NT / 32)), ML_NT, 0, st>>>(
-                   reinterpret_cast<const Ti*>(ws + w.o_num), reinterpret_cast<const Ti*>(ws + w.o_den),
-                   reinterpret_cast<const float*>(ws + w.o_c), static_cast<To*>(h), rows, p->L, p->Dv, w.pb.Dv)));
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return record_cuda(e, "mLSTM normalise launch");
-    GLA_LAUNCH("mlstm_status", st,
-               k_status_or<<<1, 1, 0, st>>>(reinterpret_cast<int*>(ws), reinterpret_cast<const int*>(ws + w.o_wsb)));
-    return record_cuda(cudaGetLastError(), "mLSTM status launch");
+               (k_mlstm_norm<Ta, To><<<(unsigned)((rows + ML_NT / 32 - 1) / (ML_NT / 32)), ML_NT, 0, st>>>(
+                   reinterpret_cast<const Ta*>(ws + w.o_num), reinterpret_cast<const float*>(ws + w.o_den),
+                   reinterpret_cast<const float*>(ws + w.o_c), static_cast<To*>(h), rows, p->L, p->Dv)));
+    return record_cuda(cudaGetLastError(), "mLSTM normalise launch");
 }
 
-template <typename Ti, typename To>
+template <typename Ta, typename To>
 gla_status ml_bwd(const gla_problem* p, const MlLayout& w, const void* q, const void* k, const void* v,
                   const float* g, const float* itil, const void* dh, void* dq, void* dk, void* dv, float* dg,
                   float* ditil, char* ws, cudaStream_t st) {
-    gla_status s = ml_forward_passes<Ti, To>(p, w, q, k, v, g, itil, ws, st);
+    MlInputs in;
+    gla_status s = ml_forward_passes<Ta, To>(p, w, q, k, v, g, itil, ws, &in, st);
     if (s != GLA_OK) return s;
     const long rows = (long)p->B * p->H * p->L;
-    const int Dvn = w.pb.Dv;
-    Ti* dnum = reinterpret_cast<Ti*>(ws + w.o_dnum);
-    Ti* dden = reinterpret_cast<Ti*>(ws + w.o_dden);
+    Ta* dnum = reinterpret_cast<Ta*>(ws + w.o_dnum);
+    float* dden = reinterpret_cast<float*>(ws + w.o_dden);
     GLA_LAUNCH("mlstm_bwd_prep", st,
-               (k_mlstm_bwd_prep<Ti, To><<<(unsigned)((rows + ML_NT / 32 - 1) / (ML_NT / 32)), ML_NT, 0, st>>>(
-                   reinterpret_cast<const Ti*>(ws + w.o_num), reinterpret_cast<const Ti*>(ws + w.o_den),
+               (k_mlstm_bwd_prep<Ta, To><<<(unsigned)((rows + ML_NT / 32 - 1) / (ML_NT / 32)), ML_NT, 0, st>>>(
+                   reinterpret_cast<const Ta*>(ws + w.o_num), reinterpret_cast<const float*>(ws + w.o_den),
                    reinterpret_cast<const float*>(ws + w.o_c), static_cast<const To*>(dh), dnum, dden, rows, p->L,
-                   p->Dv, Dvn)));
+                   p->Dv)));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return record_cuda(e, "mLSTM backward prep launch");
     const float* ig = reinterpret_cast<const float*>(ws + w.o_ig);
@@ -286,24 +429,39 @@ gla_status ml_bwd(const gla_problem* p, const MlLayout& w, const void* q, const 
     float* di2 = reinterpret_cast<float*>(ws + w.o_di2);
     float* dg2 = reinterpret_cast<float*>(ws + w.o_dg2);
     // the value pass writes its gradients straight into the outputs unless they are cast back
-    void* dq1 = w.cast ? ws + w.o_dq1 : dq;
-    void* dk1 = w.cast ? ws + w.o_dk1 : dk;
-    void* dv1 = w.cast ? ws + w.o_dv1 : dv;
-    s = gla_bwd(&w.pa, q, k, v, g, ig, nullptr, dnum, nullptr, dq1, dk1, dv1, dg, di1, nullptr, ws, w.wsa, st);
+    void* dq1 = w.cast_a ? ws + w.o_dq1 : dq;
+    void* dk1 = w.cast_a ? ws + w.o_dk1 : dk;
+    void* dv1 = w.cast_a ? ws + w.o_dv1 : dv;
+    s = gla_bwd(&w.pa, in.qa, in.ka, in.va, g, ig, nullptr, dnum, nullptr, dq1, dk1, dv1, dg, di1, nullptr, ws, w.wsa,
+                st);
     if (s != GLA_OK) return s;
-    s = gla_bwd(&w.pb, q, k, ws + w.o_ones, g, ig, nullptr, dden, nullptr, ws + w.o_dq2, ws + w.o_dk2,
-                ws + w.o_dv2, dg2, di2, nullptr, ws + w.o_wsb, w.wsb, st);
-    if (s != GLA_OK) return s;
-    const long nqk = rows * p->Dk, nv = w.cast ? rows * p->Dv : 0;
+    // the normaliser recurrence's backward, reading q and k in the I/O dtype
+    {
+        const long BH = (long)p->B * p->H;
+        const To* tq = static_cast<const To*>(q);
+        const To* tk = static_cast<const To*>(k);
+        float* cloc = reinterpret_cast<float*>(ws + w.o_cloc);
+        float* cin = reinterpret_cast<float*>(ws + w.o_cin);
+        const dim3 grid(w.nseg, (unsigned)BH);
+        GLA_LAUNCH("mlstm_dnloc", st,
+                   k_mlstm_dnloc<To><<<grid, p->Dk, 0, st>>>(tq, g, dden, p->L, p->Dk, w.nseg, p->scale, cloc));
+        GLA_LAUNCH("mlstm_cscan", st,
+                   k_mlstm_cscan<<<(unsigned)BH, p->Dk, 0, st>>>(cloc, reinterpret_cast<const float*>(ws + w.o_gam),
+                                                                w.nseg, p->Dk, cin));
+        GLA_LAUNCH("mlstm_den_bwd", st,
+                   k_mlstm_den_bwd<To><<<grid, p->Dk, 0, st>>>(
+                       tq, tk, g, ig, dden, reinterpret_cast<const float*>(ws + w.o_nst), cin, p->L, p->Dk, w.nseg,
+                       p->scale, reinterpret_cast<float*>(ws + w.o_dq2), reinterpret_cast<float*>(ws + w.o_dk2), dg2,
+                       di2));
+        if ((e = cudaGetLastError()) != cudaSuccess) return record_cuda(e, "mLSTM normaliser backward launch");
+    }
+    const long nqk = rows * p->Dk, nv = w.cast_a ? rows * p->Dv : 0;
     GLA_LAUNCH("mlstm_bwd_final", st,
-               (k_mlstm_bwd_final<Ti, To><<<ml_grid(nqk, 256), 256, 0, st>>>(
-                   static_cast<To*>(dq), static_cast<To*>(dk), static_cast<To*>(dv), static_cast<const Ti*>(dq1),
-                   static_cast<const Ti*>(dk1), static_cast<const Ti*>(dv1), reinterpret_cast<const Ti*>(ws + w.o_dq2),
-                   reinterpret_cast<const Ti*>(ws + w.o_dk2), nqk, nv, dg, dg2, di1, di2, ig, ditil, rows)));
-    if ((e = cudaGetLastError()) != cudaSuccess) return record_cuda(e, "mLSTM backward final launch");
-    GLA_LAUNCH("mlstm_status", st,
-               k_status_or<<<1, 1, 0, st>>>(reinterpret_cast<int*>(ws), reinterpret_cast<const int*>(ws + w.o_wsb)));
-    return record_cuda(cudaGetLastError(), "mLSTM status launch");
+               (k_mlstm_bwd_final<Ta, To><<<ml_grid(nqk, 256), 256, 0, st>>>(
+                   static_cast<To*>(dq), static_cast<To*>(dk), static_cast<To*>(dv), static_cast<const Ta*>(dq1),
+                   static_cast<const Ta*>(dk1), static_cast<const Ta*>(dv1), reinterpret_cast<const float*>(ws + w.o_dq2),
+                   reinterpret_cast<const float*>(ws + w.o_dk2), nqk, nv, dg, dg2, di1, di2, ig, ditil, rows)));
+    return record_cuda(cudaGetLastError(), "mLSTM backward final launch");
 }
 
 }  // namespace
@@ -334,9 +492,10 @@ gla_status gla_mlstm_fwd(const gla_problem* p, const void* q, const void* k, con
     if (e != cudaSuccess) return gla::record_cuda(e, "status word reset");
     if (empty) return GLA_OK;
     char* wsb = static_cast<char*>(ws);
+    using bf16 = __nv_bfloat16;
     if (p->io == GLA_F32) return gla::ml_fwd<float, float>(p, w, q, k, v, g, itil, h, wsb, st);
-    return w.f32 ? gla::ml_fwd<float, __nv_bfloat16>(p, w, q, k, v, g, itil, h, wsb, st)
-                 : gla::ml_fwd<__nv_bfloat16, __nv_bfloat16>(p, w, q, k, v, g, itil, h, wsb, st);
+    return w.fa ? gla::ml_fwd<float, bf16>(p, w, q, k, v, g, itil, h, wsb, st)
+                : gla::ml_fwd<bf16, bf16>(p, w, q, k, v, g, itil, h, wsb, st);
 }
 
 gla_status gla_mlstm_bwd(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
@@ -358,10 +517,11 @@ gla_status gla_mlstm_bwd(const gla_problem* p, const void* q, const void* k, con
     if (e != cudaSuccess) return gla::record_cuda(e, "status word reset");
     if (empty) return GLA_OK;
     char* wsb = static_cast<char*>(ws);
-    if (p->io == GLA_F32) return gla::ml_bwd<float, float>(p, w, q, k, v, g, itil, dh, dq, dk, dv, dg, ditil, wsb, st);
-    return w.f32 ? gla::ml_bwd<float, __nv_bfloat16>(p, w, q, k, v, g, itil, dh, dq, dk, dv, dg, ditil, wsb, st)
-                 : gla::ml_bwd<__nv_bfloat16, __nv_bfloat16>(p, w, q, k, v, g, itil, dh, dq, dk, dv, dg, ditil, wsb,
-                                                             st);
+    using bf16 = __nv_bfloat16;
+    if (p->io == GLA_F32)
+        return gla::ml_bwd<float, float>(p, w, q, k, v, g, itil, dh, dq, dk, dv, dg, ditil, wsb, st);
+    return w.fa ? gla::ml_bwd<float, bf16>(p, w, q, k, v, g, itil, dh, dq, dk, dv, dg, ditil, wsb, st)
+                : gla::ml_bwd<bf16, bf16>(p, w, q, k, v, g, itil, dh, dq, dk, dv, dg, ditil, wsb, st);
 }
 
 }  // extern "C"

@@ -40,6 +40,13 @@ cudaError_t seg_scan(const Dims& P, int nseg, const float* seg_state, const floa
 cudaError_t seg_rscan(const Dims& P, int nseg, const float* seg_state, const float* seg_gamma, const float* dhT,
                       float* gend, cudaStream_t st);
 int num_sms();
+// DeltaNet forward on the tensor cores (gla_deltanet_tc.cu): bf16 I/O, Dk 64 or 128, Dv a
+// multiple of 64, chunk 64. o null: the state walk only (the backward's recompute). saved
+// (nullable): [BH, ceil(L/64), Dk, Dv] the state entering every chunk; status (nullable): device
+// status word for a wait that gave up.
+cudaError_t deltanet_fwd(int B, int H, int L, int Dk, int Dv, float scale, const void* q, const void* k,
+                         const void* v, const float* beta, const float* h0, void* o, float* hT, float* saved,
+                         int* status, cudaStream_t st);
 // Backward (gla_tc_bwd.cu)
 bool bwd_supports(const Dims& P);
 size_t bwd_workspace_bytes(const Dims& P);

@@ -3,7 +3,8 @@ with the float64 delta-rule oracle (oracle/deltanet.py: the recurrence and its b
 through time, pinned in test_oracle_deltanet.py), element by element, on seeded inputs: unit-norm keys, beta = sigmoid(N(0,1)). Cases span several 64-token chunks and a ragged
 tail, both key widths, several 64-column value slices, with and without h0, and the edge
 lengths L = 0, 1 and 64. Bound: the max-normalised error, 1e-4 for fp32 I/O and 1e-2 for bf16
-(the fp32 kernel against float64: rounding only; bf16 adds the output's rounding)."""
+(fp32 I/O runs the CUDA-core forward, rounding only; bf16 I/O runs the tensor-core forward, whose
+bf16 operands T, R, X and the state copy add their rounding to the output's)."""
 import numpy as np
 import pytest
 import torch
@@ -30,17 +31,38 @@ def err(got, ref):
     return float(np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-30))
 
 
-def check(B, H, L, Dk, Dv, dtype, h0_std, seed=0):
+def record(case, errs):
+    """Measured errors of a case, appended to the report file GLA_PARITY_REPORT names (if set)."""
+    import json
+    import os
+    path = os.environ.get("GLA_PARITY_REPORT")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": case, "errors": errs}) + "\n")
+
+
+def heads_of(t, heads):
+    if t is None or heads is None:
+        return t
+    B, H = t.shape[0], t.shape[1]
+    return t.reshape((B * H,) + tuple(t.shape[2:]))[heads][None]
+
+
+def check(B, H, L, Dk, Dv, dtype, h0_std, seed=0, heads=None, case=None):
     from linear_rnn_b200 import ops
     x = I.make_deltanet_inputs(B, H, L, Dk, Dv, dtype, seed=seed, h0_std=h0_std)
     xd = {n: (None if t is None else t.cuda()) for n, t in x.items()}
     scale = Dk ** -0.5
     o, hT = ops.gla_deltanet_fwd(xd["q"], xd["k"], xd["v"], xd["beta"], xd["h0"], scale=scale)
     torch.cuda.synchronize()
-    ro, rS = DN.deltanet_fwd(x["q"], x["k"], x["v"], x["beta"], x["h0"], scale)
+    xs = {n: heads_of(t, heads) for n, t in x.items()}
+    ro, rS = DN.deltanet_fwd(xs["q"], xs["k"], xs["v"], xs["beta"], xs["h0"], scale)
+    errs = {"hT": err(f64(heads_of(hT, heads)), rS)}
     if L:
-        assert err(f64(o), ro) <= TOL[dtype]
-    assert err(f64(hT), rS) <= TOL[dtype]
+        errs["o"] = err(f64(heads_of(o, heads)), ro)
+    if case:
+        record(case, errs)
+    assert all(e <= TOL[dtype] for e in errs.values()), errs
     return o, hT
 
 
@@ -58,6 +80,22 @@ def test_parity(B, H, L, Dk, Dv, dtype, h0_std):
 @pytest.mark.parametrize("L", [1, 63, 65])
 def test_edge_lengths(L):
     check(1, 2, L, 64, 64, "f32", 0.5, seed=3)
+
+
+@pytest.mark.parametrize("Dk", [64, 128])
+@pytest.mark.parametrize("L", [1, 63, 64, 65, 129])
+def test_tensor_core_edge_lengths(Dk, L):
+    """bf16 I/O (the tensor-core forward) at chunk edges: a ragged last chunk reads zero rows past
+    the end and stores none."""
+    check(1, 2, L, Dk, 128, "bf16", 0.5, seed=11)
+
+
+def test_tensor_core_full_size():
+    """The DeltaNet workload (B=4 H=16 L=4096 Dk=Dv=128, bf16) on the tensor cores; two heads
+    against the oracle."""
+    c = I.DELTANET
+    check(c["B"], c["H"], c["L"], c["Dk"], c["Dv"], c["dtype"], 0.5, seed=0, heads=[5, 50],
+          case="deltanet full size heads=[5, 50]")
 
 
 def test_empty_sequence_returns_h0():
@@ -88,7 +126,7 @@ def test_deterministic_and_host_round_trip():
     assert oh.device.type == "cpu" and torch.equal(oh, o1.cpu()) and torch.equal(hh, h1.cpu())
 
 
-def check_bwd(B, H, L, Dk, Dv, dtype, h0_std, with_dhT, seed=0):
+def check_bwd(B, H, L, Dk, Dv, dtype, h0_std, with_dhT, seed=0, case=None):
     from linear_rnn_b200 import ops
     x = I.make_deltanet_inputs(B, H, L, Dk, Dv, dtype, seed=seed, h0_std=h0_std)
     gen = torch.Generator().manual_seed(100 + seed)
@@ -100,9 +138,10 @@ def check_bwd(B, H, L, Dk, Dv, dtype, h0_std, with_dhT, seed=0):
                              None if dhT is None else dhT.cuda(), scale=scale)
     torch.cuda.synchronize()
     ref = DN.deltanet_bwd(x["q"], x["k"], x["v"], x["beta"], x["h0"], dO, dhT, scale)
-    for name in ("dq", "dk", "dv", "dbeta", "dh0"):
-        if ref[name].size:
-            assert err(f64(r[name]), ref[name]) <= TOL[dtype], name
+    errs = {name: err(f64(r[name]), ref[name]) for name in ("dq", "dk", "dv", "dbeta", "dh0") if ref[name].size}
+    if case:
+        record(case, errs)
+    assert all(e <= TOL[dtype] for e in errs.values()), errs
     return r
 
 
@@ -124,4 +163,10 @@ def test_backward_edge_lengths(L):
 
 
 def test_backward_long_sequence():
-    check_bwd(1, 2, 2048, 128, 128, "bf16", 0.5, True, seed=8)
+    check_bwd(1, 2, 2048, 128, 128, "bf16", 0.5, True, seed=8, case="deltanet backward L=2048")
+
+
+@pytest.mark.parametrize("L", [1, 64, 65])
+def test_backward_tensor_core_recompute_edges(L):
+    """bf16 I/O: the backward's chunk start states come from the tensor-core state walk."""
+    check_bwd(1, 2, L, 128, 128, "bf16", 0.5, True, seed=12)
