@@ -13,11 +13,13 @@
 // memory (fp32; the state product accumulates onto it) and a bf16 copy in shared memory as the
 // B operand of K S and Q S. Per chunk:
 //   1. tcgen05: K K^T and Q K^T (M=64 N=64), K S and Q S (M=64 N=64) into tensor memory;
-//   2. CUDA cores: diag(beta) K K^T (strict lower, fp32), P = lower(Q K^T) (bf16), R (bf16);
-//      T by forward substitution in fp32 (rows sequential, columns in parallel), then bf16;
-//   3. tcgen05: X = T R;  4. X to bf16;
-//   5. tcgen05: O = Q S + P X (onto the Q S accumulator), S += K^T X;
-//   6. o = scale O (bf16, TMA store), the state's bf16 copy (and, for the backward, the state
+//   2. CUDA cores: A = diag(beta) K K^T (strict lower) and R in fp32, P = lower(Q K^T) in bf16;
+//   3. CUDA cores: X = T R by solving (I + A) X = R in fp32, row by row: once row t of X is
+//      final it is subtracted from every later row (A[u][t] X[t] for u > t), so each row's value
+//      is ready the moment the row before it is; thread = value column x every 4th row, the
+//      rows in registers. X goes to bf16 as the B operand of the next products;
+//   4. tcgen05: O = Q S + P X (onto the Q S accumulator), S += K^T X;
+//   5. o = scale O (bf16, TMA store), the state's bf16 copy (and, for the backward, the state
 //      entering the next chunk in fp32).
 // K, Q and V tiles arrive by TMA into a two-stage ring, so the next chunk's loads overlap this
 // chunk's work. Every phase runs on all 8 warps in turn; one elected lane of warp 0 issues the
@@ -37,7 +39,7 @@ namespace {
 
 constexpr int DT_NT = 256;   // 8 warps: two warpgroups
 constexpr int DT_VT = 64;    // value columns per CTA
-constexpr int DT_TS = 68;    // row stride (floats) of the fp32 T^T used by the substitution
+constexpr int DT_TS = 68;    // row stride (floats) of the fp32 A and R tiles (16-byte rows, spread banks)
 
 template <int DK>
 struct DtCfg {
@@ -47,15 +49,14 @@ struct DtCfg {
     static constexpr uint32_t STAGE = KB + QB + VB;
     static constexpr int NS = 2;
     static constexpr uint32_t SB = DK * DT_VT * 2;        // bf16 state copy (MN-major B: row = key dim)
-    static constexpr uint32_t MB = TR * TR * 2;           // one 64 x 64 bf16 operand (T, P, R, X, O staging)
-    static constexpr uint32_t AF = TR * TR * 4;           // diag(beta) K K^T, fp32 [t][s]
-    static constexpr uint32_t TF = TR * DT_TS * 4;        // T^T, fp32 [c][t]
+    static constexpr uint32_t MB = TR * TR * 2;           // one 64 x 64 bf16 operand (P, X, O staging)
+    static constexpr uint32_t AF = TR * DT_TS * 4;        // diag(beta) K K^T, fp32 [t][s]
+    static constexpr uint32_t RF = TR * DT_TS * 4;        // R, fp32 [t][value column]
     static constexpr uint32_t SMALL = 256 + 4 * TR;
-    static constexpr uint32_t SMEM = NS * STAGE + SB + 5 * MB + AF + TF + SMALL + 1024;
-    // TMEM columns: the state [0, 64) (M = Dk rows), then three M=64 accumulators, each pair in
-    // lanes 0-15 / 16-31 of the same columns: K K^T | Q K^T at 64, K S | Q S (then O) at 128,
-    // X at 192
-    static constexpr uint32_t C_S = 0, C_KK = 64, C_KS = 128, C_X = 192, NCOL = 256;
+    static constexpr uint32_t SMEM = NS * STAGE + SB + 3 * MB + AF + RF + SMALL + 1024;
+    // TMEM columns: the state [0, 64) (M = Dk rows), then two M=64 accumulators, each pair in
+    // lanes 0-15 / 16-31 of the same columns: K K^T | Q K^T at 64, K S | Q S (then O) at 128
+    static constexpr uint32_t C_S = 0, C_KK = 64, C_KS = 128, NCOL = 256;
     static constexpr int MS = DK == 64 ? 64 : 128;        // M of the state product
     static_assert(SMEM <= 227 * 1024, "shared memory");
     static_assert(STAGE % 1024 == 0 && SB % 1024 == 0, "alignment");
@@ -94,14 +95,12 @@ __global__ void __launch_bounds__(DT_NT, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = smem_align1024(smem_raw);
     uint8_t* sS = sm + C::NS * C::STAGE;
-    uint8_t* sT = sS + C::SB;
-    uint8_t* sP = sT + C::MB;
-    uint8_t* sR = sP + C::MB;
-    uint8_t* sX = sR + C::MB;
+    uint8_t* sP = sS + C::SB;
+    uint8_t* sX = sP + C::MB;
     uint8_t* sO = sX + C::MB;
     float* sA = reinterpret_cast<float*>(sO + C::MB);
-    float* sTt = sA + TR * TR;
-    uint8_t* small = reinterpret_cast<uint8_t*>(sTt + TR * DT_TS);
+    float* sRf = sA + TR * DT_TS;
+    uint8_t* small = reinterpret_cast<uint8_t*>(sRf + TR * DT_TS);
     uint64_t* bar_full = reinterpret_cast<uint64_t*>(small);   // [2]
     uint64_t* bar_mma = bar_full + 2;
     uint64_t* bar_drain = bar_full + 3;
@@ -215,8 +214,8 @@ __global__ void __launch_bounds__(DT_NT, 1)
         if (!dt_wait(bar_mma, (n_mma - 1) & 1)) { err = 1; break; }
         tc_fence_after();
 
-        // ---- 2a. diag(beta) K K^T (strict lower, fp32) and P = lower(Q K^T) (bf16): one TMEM read,
-        //      K K^T rows in lanes 0-15, Q K^T rows in lanes 16-31; 32 columns per warpgroup
+        // ---- 2a. A = diag(beta) K K^T (strict lower, fp32) and P = lower(Q K^T) (bf16): one TMEM
+        //      read, K K^T rows in lanes 0-15, Q K^T rows in lanes 16-31; 32 columns per warpgroup
         {
             uint32_t r[32];
             tmem_ld32(tq_lane + C::C_KK + 32 * wg, r);
@@ -227,7 +226,7 @@ __global__ void __launch_bounds__(DT_NT, 1)
 #pragma unroll
                 for (int j = 0; j < 32; j += 4) {
                     const int sc = 32 * wg + j;
-                    *reinterpret_cast<float4*>(sA + t * TR + sc) =
+                    *reinterpret_cast<float4*>(sA + t * DT_TS + sc) =
                         make_float4(sc < t ? bt * __uint_as_float(r[j]) : 0.f, sc + 1 < t ? bt * __uint_as_float(r[j + 1]) : 0.f,
                                     sc + 2 < t ? bt * __uint_as_float(r[j + 2]) : 0.f,
                                     sc + 3 < t ? bt * __uint_as_float(r[j + 3]) : 0.f);
@@ -245,7 +244,7 @@ __global__ void __launch_bounds__(DT_NT, 1)
                 }
             }
         }
-        // ---- 2b. R = diag(beta) (V - K S) (bf16, laid out like a V tile: the B operand of T R)
+        // ---- 2b. R = diag(beta) (V - K S), fp32 [t][value column]
         {
             uint32_t r[32];
             tmem_ld32(tq_lane + C::C_KS + 32 * wg, r);
@@ -265,71 +264,48 @@ __global__ void __launch_bounds__(DT_NT, 1)
                         f[2 * j] = bt * (vf.x - __uint_as_float(r[8 * u + 2 * j]));
                         f[2 * j + 1] = bt * (vf.y - __uint_as_float(r[8 * u + 2 * j + 1]));
                     }
-                    store8_bf16(sR, sw128_off(t, cc, BLK), f);
+                    *reinterpret_cast<float4*>(sRf + t * DT_TS + cc) = make_float4(f[0], f[1], f[2], f[3]);
+                    *reinterpret_cast<float4*>(sRf + t * DT_TS + cc + 4) = make_float4(f[4], f[5], f[6], f[7]);
                 }
             }
         }
         __syncthreads();
 
-        // ---- 2c. T = (I + A)^{-1}: T[t][c] = [t == c] - sum_{c <= i < t} A[t][i] T[i][c], row by row;
-        //      column c = 8 warp + lane / 4, its dot products split over 4 lanes
+        // ---- 3. X = (I + A)^{-1} R in fp32: thread = value column j x rows u = 4 m + sp (m = 0..15),
+        //      their values in registers; row t, once final, is broadcast from its owner and
+        //      subtracted from the thread's later rows. A is read four columns at a time.
         {
-            const int sc = warp * 8 + (lane >> 2), sp = lane & 3;
-            for (int t = 0; t < TR; ++t) {
-                float part = 0.f;
-                for (int i = sc + sp; i < t; i += 4) part = fmaf(sA[t * TR + i], sTt[sc * DT_TS + i], part);
-                part += __shfl_xor_sync(0xffffffffu, part, 1);
-                part += __shfl_xor_sync(0xffffffffu, part, 2);
-                if (sp == 0) sTt[sc * DT_TS + t] = t < sc ? 0.f : t == sc ? 1.f : -part;
-                __syncwarp();
+            const int j = warp * 8 + (lane >> 2), sp = lane & 3;
+            float x[16];
+#pragma unroll
+            for (int m = 0; m < 16; ++m) x[m] = sRf[(4 * m + sp) * DT_TS + j];
+#pragma unroll
+            for (int t4 = 0; t4 < TR; t4 += 4) {
+                float4 a[16];   // A[u][t4 .. t4 + 3] of the thread's rows u >= t4
+#pragma unroll
+                for (int m = t4 / 4; m < 16; ++m) a[m] = *reinterpret_cast<const float4*>(sA + (4 * m + sp) * DT_TS + t4);
+#pragma unroll
+                for (int tt = 0; tt < 4; ++tt) {
+                    const int t = t4 + tt;
+                    const float xt = __shfl_sync(0xffffffffu, x[t >> 2], (lane & ~3) | (t & 3));
+#pragma unroll
+                    for (int m = t4 / 4; m < 16; ++m) {
+                        const float at = tt == 0 ? a[m].x : tt == 1 ? a[m].y : tt == 2 ? a[m].z : a[m].w;
+                        if (4 * m + sp > t) x[m] = fmaf(-at, xt, x[m]);
+                    }
+                }
             }
-        }
-        __syncthreads();
-        // T to bf16, K-major A operand: thread = row t, 16 columns
-        {
-            const int t = tid >> 2, c0 = 16 * (tid & 3);
-            float f[16];
+            // X to bf16, laid out like a V tile (the B operand of P X and K^T X)
 #pragma unroll
-            for (int j = 0; j < 16; ++j) f[j] = sTt[(c0 + j) * DT_TS + t];
-            store8_bf16(sT, sw128_off(t, c0, BLK), f);
-            store8_bf16(sT, sw128_off(t, c0 + 8, BLK), f + 8);
+            for (int m = 0; m < 16; ++m)
+                *reinterpret_cast<__nv_bfloat16*>(sX + sw128_off(4 * m + sp, j, BLK)) = __float2bfloat16_rn(x[m]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
 
-        // ---- 3. X = T R
-        if (warp == 0) {
-            const bool leader = elect_one();
-            const uint32_t idX = idesc_bf16(64, DT_VT, 0, 1);
-            const uint64_t dT = sw128_desc(smem_u32(sT), 16, 1024), dR = sw128_desc(smem_u32(sR), BLK, 1024);
-#pragma unroll
-            for (int ks = 0; ks < TR / 16; ++ks)
-                if (leader) mma_bf16(tbase + C::C_X, dT + ((ks * 32) >> 4), dR + ((ks * 2048) >> 4), idX, ks > 0);
-            if (leader) mma_commit(bar_mma);
-            __syncwarp();
-        }
-        ++n_mma;
-        if (!dt_wait(bar_mma, (n_mma - 1) & 1)) { err = 1; break; }
-        tc_fence_after();
-
-        // ---- 4. X to bf16 (the B operand of P X and K^T X)
-        {
-            uint32_t r[32];
-            tmem_ld32(tq_lane + C::C_X + 32 * wg, r);
-            tmem_wait_ld();
-            if (first)
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    store8_bf16(sX, sw128_off(mrow, 32 * wg + 8 * u, BLK), reinterpret_cast<const float*>(r + 8 * u));
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-
-        // ---- 5. O = Q S + P X, S += K^T X
+        // ---- 4. O = Q S + P X, S += K^T X
         if (warp == 0) {
             const bool leader = elect_one();
             const uint32_t idO = idesc_bf16(64, DT_VT, 0, 1), idS = idesc_bf16(C::MS, DT_VT, 1, 1);
@@ -348,7 +324,7 @@ __global__ void __launch_bounds__(DT_NT, 1)
         if (!dt_wait(bar_mma, (n_mma - 1) & 1)) { err = 1; break; }
         tc_fence_after();
 
-        // ---- 6. o = scale O (bf16 tile -> TMA store); the state's bf16 copy and the state entering
+        // ---- 5. o = scale O (bf16 tile -> TMA store); the state's bf16 copy and the state entering
         //      the next chunk
         if (OUT) {
             uint32_t r[32];
