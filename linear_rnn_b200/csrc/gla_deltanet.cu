@@ -740,11 +740,18 @@ cudaError_t dn_bwd_launch(const gla_problem* p, const void* q, const void* k, co
     const T* tq = static_cast<const T*>(q);
     const T* tk = static_cast<const T*>(k);
     const T* tdo = static_cast<const T*>(dO);
-    GLA_LAUNCH("deltanet_bwd_walk", st,
-               (walk<<<dim3(BH, p->Dv / DN_VT), DN_NT, sw, st>>>(tq, tk, static_cast<const T*>(v), beta, tdo, dhT,
-                                                                 w.saved, w.xw, w.drw, w.dsend, w.db1,
-                                                                 static_cast<T*>(dv), dh0, BH, p->L, p->Dv, p->scale)));
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (std::is_same<T, __nv_bfloat16>::value) {   // bf16 I/O: the tensor-core walk
+        e = tc::deltanet_walk(p->B, p->H, p->L, DK, p->Dv, p->scale, q, k, v, beta, dO, dhT, w.saved, w.xw, w.drw,
+                              w.dsend, w.db1, dv, dh0, st);
+    } else {
+        GLA_LAUNCH("deltanet_bwd_walk", st,
+                   (walk<<<dim3(BH, p->Dv / DN_VT), DN_NT, sw, st>>>(tq, tk, static_cast<const T*>(v), beta, tdo, dhT,
+                                                                     w.saved, w.xw, w.drw, w.dsend, w.db1,
+                                                                     static_cast<T*>(dv), dh0, BH, p->L, p->Dv,
+                                                                     p->scale)));
+        e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) return e;
     if (NC > 0)
         GLA_LAUNCH("deltanet_bwd_grads", st,
                    (grads<<<dim3(NC, BH), DN_NT, sg, st>>>(tq, tk, beta, tdo, w.saved, w.xw, w.drw, w.dsend, w.db1,

@@ -77,6 +77,18 @@ __device__ __forceinline__ bool dt_wait(uint64_t* bar, uint32_t parity) {
     return __syncthreads_and(ok) != 0;
 }
 
+// 16 consecutive values to bf16 in global memory (32-byte aligned)
+__device__ __forceinline__ void dt_store16_bf16(__nv_bfloat16* dst, const float* v) {
+    uint32_t w[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        __nv_bfloat162 p = __floats2bfloat162_rn(v[2 * u], v[2 * u + 1]);
+        w[u] = *reinterpret_cast<uint32_t*>(&p);
+    }
+    reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
 // The CTA's [DK, 64] state slice, row `d` (this thread's TMEM lane), 32 columns from `c`: fp32 to
 // global memory (saved / hT), 128 contiguous bytes per thread.
 __device__ __forceinline__ void dt_put_row(float* dst, const uint32_t* r) {
@@ -400,6 +412,467 @@ cudaError_t dt_launch(int B, int H, int L, int Dv, const CUtensorMap& mq, const 
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ backward walk
+// With U = V - K S, R = diag(beta) U, X = T R, P = lower(Q K^T) and dS' the gradient reaching the
+// chunk's end state, a chunk's reverse step is
+//   dX = scale P^T dO + K dS',   dR = T^T dX,   dV = diag(beta) dR,
+//   dS = dS' + scale Q^T dO - K^T diag(beta) dR       (the gradient at the chunk's start).
+// One CTA per (batch*head, 64-column value slice) walks the chunks in reverse with its dS slice in
+// tensor memory. Per chunk:
+//   1. q is scaled in place (so that Q K^T and Q^T dO carry the output scale); tcgen05: K K^T,
+//      Q K^T, K S (S: the chunk's start state from the forward walk, bf16) and K dS';
+//   2. A = diag(beta) strict_lower(K K^T) and its transpose, U and R (fp32), P = lower(Q K^T)
+//      (bf16); tcgen05: dX = K dS' + P^T dO (onto the K dS' accumulator);
+//   3. X = (I + A)^{-1} R (the forward's substitution) -> global for the gradient kernel;
+//   4. dR = (I + A)^{-T} dX: the same substitution backwards, row 63 first;
+//   5. dR and dV = diag(beta) dR to global, the slice's part of sum_j dR U, -diag(beta) dR (bf16);
+//   6. tcgen05: dS += Q^T dO + K^T (-diag(beta) dR); its bf16 copy for the next chunk.
+template <int DK>
+struct DwCfg {
+    static constexpr uint32_t KB = TR * DK * 2, QB = TR * DK * 2, VB = TR * DT_VT * 2, OB = TR * DT_VT * 2;
+    static constexpr uint32_t STAGE = KB + QB + VB + OB;
+    static constexpr int NS = 2;
+    static constexpr uint32_t SB = DK * DT_VT * 2;   // bf16 copy of the chunk's start state
+    static constexpr uint32_t GB = DK * DT_VT * 2;   // bf16 copy of dS'
+    static constexpr uint32_t MB = TR * TR * 2;      // P; -diag(beta) dR
+    static constexpr uint32_t F = TR * DT_TS * 4;    // fp32 tiles: A, A^T, U, W (R, X, dX, dR in turn)
+    static constexpr uint32_t SMALL = 256 + 4 * TR;
+    static constexpr uint32_t SMEM = NS * STAGE + SB + GB + 2 * MB + 4 * F + SMALL + 1024;
+    static constexpr uint32_t C_S = 0, C_KK = 64, C_KS = 128, NCOL = 256;
+    static constexpr int MS = DK == 64 ? 64 : 128;
+    static_assert(SMEM <= 227 * 1024, "shared memory");
+    static_assert(STAGE % 1024 == 0 && SB % 1024 == 0, "alignment");
+};
+
+struct DwArgs {
+    const float* beta;    // [BH*L]
+    const float* saved;   // [BH, NC, Dk, Dv] the state entering every chunk
+    const float* dhT;     // [BH, Dk, Dv] or null
+    float* xw;            // [BH*L, Dv] X
+    float* drw;           // [BH*L, Dv] dR
+    float* dsend;         // [BH, NC, Dk, Dv] the gradient at every chunk's end
+    float* db1;           // [Dv/64, BH*L] the slice's sum_j dR U
+    __nv_bfloat16* dv;    // [BH*L, Dv]
+    float* dh0;           // [BH, Dk, Dv] or null
+    int BH, L, Dv;
+    float scale;
+};
+
+template <int DK>
+__global__ void __launch_bounds__(DT_NT, 1)
+    k_deltanet_tc_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                       const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo, DwArgs A) {
+    using C = DwCfg<DK>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = smem_align1024(smem_raw);
+    uint8_t* sS = sm + C::NS * C::STAGE;
+    uint8_t* sG = sS + C::SB;
+    uint8_t* sP = sG + C::GB;
+    uint8_t* sBR = sP + C::MB;
+    float* sA = reinterpret_cast<float*>(sBR + C::MB);
+    float* sAT = sA + TR * DT_TS;
+    float* sU = sAT + TR * DT_TS;
+    float* sW = sU + TR * DT_TS;
+    uint8_t* small = reinterpret_cast<uint8_t*>(sW + TR * DT_TS);
+    uint64_t* bar_full = reinterpret_cast<uint64_t*>(small);   // [2]
+    uint64_t* bar_mma = bar_full + 2;
+    uint64_t* bar_drain = bar_full + 3;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 64);
+    float* sB = reinterpret_cast<float*>(small + 256);
+
+    const int bh = blockIdx.x, slice = blockIdx.y, col0 = slice * DT_VT;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2, qd = warp & 3;
+    const int L = A.L, Dv = A.Dv;
+    const int nc = (L + TR - 1) / TR;
+    const long rowbase = (long)bh * L;
+    const bool srow_ok = DK != 64 || lane < 16;
+    const int srow = DK == 64 ? 16 * qd + (lane & 15) : 32 * qd + lane;
+    const int mrow = 16 * qd + (lane & 15);
+    const bool first = lane < 16;
+    // substitution mapping: value column j, rows 4 m + sp
+    const int sj = warp * 8 + (lane >> 2), sp = lane & 3;
+    // row-pass mapping: row rt, columns rc .. rc + 15
+    const int rt = tid >> 2, rc = 16 * (tid & 3);
+
+    if (tid == 0) {
+        mbar_init(&bar_full[0], 1);
+        mbar_init(&bar_full[1], 1);
+        mbar_init(bar_mma, 1);
+        mbar_init(bar_drain, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, C::NCOL);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tq_lane = tbase + ((uint32_t)(32 * qd) << 16);
+
+    auto chunk_at = [&](int i) { return nc - 1 - i; };
+    auto issue_loads = [&](int i, int s) {
+        uint8_t* st = sm + s * C::STAGE;
+        const int t0 = chunk_at(i) * TR;
+        mbar_arrive_expect_tx(&bar_full[s], C::STAGE);
+        for (int cb = 0; cb < DK / 64; ++cb) {
+            tma_load_3d(st + cb * BLK, &tk, cb * 64, t0, bh, &bar_full[s]);
+            tma_load_3d(st + C::KB + cb * BLK, &tq, cb * 64, t0, bh, &bar_full[s]);
+        }
+        tma_load_3d(st + C::KB + C::QB, &tv, col0, t0, bh, &bar_full[s]);
+        tma_load_3d(st + C::KB + C::QB + C::VB, &tdo, col0, t0, bh, &bar_full[s]);
+    };
+    if (tid == 0)
+        for (int i = 0; i < C::NS && i < nc; ++i) issue_loads(i, i);
+
+    // ---- dS' at the sequence's end (dhT or zero): TMEM and its bf16 copy
+    {
+        const float* src = A.dhT ? A.dhT + ((long)bh * DK + srow) * Dv + col0 : nullptr;
+        const int c = 32 * wg;
+        float f[32];
+        if (src && srow_ok) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                const float4 x = *reinterpret_cast<const float4*>(src + c + j);
+                f[j] = x.x; f[j + 1] = x.y; f[j + 2] = x.z; f[j + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) f[j] = 0.f;
+        }
+        tmem_st32(tq_lane + C::C_S + c, reinterpret_cast<uint32_t*>(f));
+        if (srow_ok)
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) store8_bf16(sG, sw128_off(srow, c + j, DK * 128), f + j);
+        tmem_wait_st();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    int err = 0, n_mma = 0;
+    for (int i = 0; i < nc; ++i) {
+        const int s = i % C::NS, ci = chunk_at(i), t0 = ci * TR;
+        uint8_t* sk = sm + s * C::STAGE;
+        uint8_t* sq = sk + C::KB;
+        uint8_t* sv = sq + C::QB;
+        uint8_t* sdo = sv + C::VB;
+        const long cbase = (long)bh * nc + ci;
+        if (tid < TR) sB[tid] = t0 + tid < L ? A.beta[rowbase + t0 + tid] : 0.f;
+        // the gradient at this chunk's end, and the chunk's start state as a bf16 operand
+        {
+            uint32_t r[32];
+            tmem_ld32(tq_lane + C::C_S + 32 * wg, r);
+            tmem_wait_ld();
+            if (srow_ok) {
+                dt_put_row(A.dsend + (cbase * DK + srow) * Dv + col0 + 32 * wg, r);
+                const float* src = A.saved + (cbase * DK + srow) * Dv + col0 + 32 * wg;
+                float f[32];
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 x = __ldg(reinterpret_cast<const float4*>(src + j));
+                    f[j] = x.x; f[j + 1] = x.y; f[j + 2] = x.z; f[j + 3] = x.w;
+                }
+#pragma unroll
+                for (int j = 0; j < 32; j += 8) store8_bf16(sS, sw128_off(srow, 32 * wg + j, DK * 128), f + j);
+            }
+        }
+        if (!dt_wait(&bar_full[s], (i / C::NS) & 1)) { err = 1; break; }
+        // q scaled in place (bf16, layout-blind 16-byte chunks)
+        for (int e = tid; e < (int)(C::QB / 16); e += DT_NT) {
+            uint4 w = *reinterpret_cast<uint4*>(sq + 16 * e);
+            uint32_t* pw = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&pw[u]));
+                __nv_bfloat162 h = __floats2bfloat162_rn(f.x * A.scale, f.y * A.scale);
+                pw[u] = *reinterpret_cast<uint32_t*>(&h);
+            }
+            *reinterpret_cast<uint4*>(sq + 16 * e) = w;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ---- 1. K K^T | Q K^T, K S | K dS'
+        if (warp == 0) {
+            const bool leader = elect_one();
+            const uint32_t ka = smem_u32(sk), qa = smem_u32(sq);
+            const uint32_t idAA = idesc_bf16(64, 64, 0, 0), idAS = idesc_bf16(64, DT_VT, 0, 1);
+            const uint64_t dS = sw128_desc(smem_u32(sS), DK * 128, 1024), dG = sw128_desc(smem_u32(sG), DK * 128, 1024);
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+                if (leader) {
+                    mma_bf16(tbase + C::C_KK, sw128_desc(ka + koff, 16, 1024), sw128_desc(ka + koff, 16, 1024), idAA,
+                             kk > 0);
+                    mma_bf16(tbase + C::C_KK + (16u << 16), sw128_desc(qa + koff, 16, 1024),
+                             sw128_desc(ka + koff, 16, 1024), idAA, kk > 0);
+                    mma_bf16(tbase + C::C_KS, sw128_desc(ka + koff, 16, 1024), dS + ((kk * 2048) >> 4), idAS, kk > 0);
+                    mma_bf16(tbase + C::C_KS + (16u << 16), sw128_desc(ka + koff, 16, 1024), dG + ((kk * 2048) >> 4),
+                             idAS, kk > 0);
+                }
+            }
+            if (leader) mma_commit(bar_mma);
+            __syncwarp();
+        }
+        ++n_mma;
+        if (!dt_wait(bar_mma, (n_mma - 1) & 1)) { err = 1; break; }
+        tc_fence_after();
+
+        // ---- 2. A and A^T (fp32), P (bf16); U and R (fp32)
+        {
+            uint32_t r[32];
+            tmem_ld32(tq_lane + C::C_KK + 32 * wg, r);
+            tmem_wait_ld();
+            const int t = mrow;
+            if (first) {
+                const float bt = sB[t];
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    const int sc = 32 * wg + j;
+                    float a4[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) a4[u] = sc + u < t ? bt * __uint_as_float(r[j + u]) : 0.f;
+                    *reinterpret_cast<float4*>(sA + t * DT_TS + sc) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) sAT[(sc + u) * DT_TS + t] = a4[u];
+                }
+            } else {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    float f[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int sc = 32 * wg + 8 * u + j;
+                        f[j] = sc <= t ? __uint_as_float(r[8 * u + j]) : 0.f;
+                    }
+                    store8_bf16(sP, sw128_off(t, 32 * wg + 8 * u, BLK), f);
+                }
+            }
+        }
+        {
+            uint32_t r[32];
+            tmem_ld32(tq_lane + C::C_KS + 32 * wg, r);
+            tmem_wait_ld();
+            if (first) {
+                const int t = mrow;
+                const float bt = sB[t];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int cc = 32 * wg + 8 * u;
+                    const uint4 vw = *reinterpret_cast<const uint4*>(sv + sw128_off(t, cc, BLK));
+                    const uint32_t* vp = reinterpret_cast<const uint32_t*>(&vw);
+                    float uu[8];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vp[j]));
+                        uu[2 * j] = vf.x - __uint_as_float(r[8 * u + 2 * j]);
+                        uu[2 * j + 1] = vf.y - __uint_as_float(r[8 * u + 2 * j + 1]);
+                    }
+                    *reinterpret_cast<float4*>(sU + t * DT_TS + cc) = make_float4(uu[0], uu[1], uu[2], uu[3]);
+                    *reinterpret_cast<float4*>(sU + t * DT_TS + cc + 4) = make_float4(uu[4], uu[5], uu[6], uu[7]);
+                    *reinterpret_cast<float4*>(sW + t * DT_TS + cc) =
+                        make_float4(bt * uu[0], bt * uu[1], bt * uu[2], bt * uu[3]);
+                    *reinterpret_cast<float4*>(sW + t * DT_TS + cc + 4) =
+                        make_float4(bt * uu[4], bt * uu[5], bt * uu[6], bt * uu[7]);
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // dX = K dS' + P^T dO (P^T: the P tile read as an MN-major A operand)
+        if (warp == 0) {
+            const bool leader = elect_one();
+            const uint32_t idX = idesc_bf16(64, DT_VT, 1, 1);
+            const uint64_t dPt = sw128_desc(smem_u32(sP), BLK, 1024), dO = sw128_desc(smem_u32(sdo), BLK, 1024);
+#pragma unroll
+            for (int ks = 0; ks < TR / 16; ++ks)
+                if (leader)
+                    mma_bf16(tbase + C::C_KS + (16u << 16), dPt + ((ks * 2048) >> 4), dO + ((ks * 2048) >> 4), idX, 1);
+            if (leader) mma_commit(bar_mma);
+            __syncwarp();
+        }
+        ++n_mma;
+
+        // ---- 3. X = (I + A)^{-1} R, as in the forward
+        {
+            float x[16];
+#pragma unroll
+            for (int m = 0; m < 16; ++m) x[m] = sW[(4 * m + sp) * DT_TS + sj];
+#pragma unroll
+            for (int t4 = 0; t4 < TR; t4 += 4) {
+                float4 a[16];
+#pragma unroll
+                for (int m = t4 / 4; m < 16; ++m) a[m] = *reinterpret_cast<const float4*>(sA + (4 * m + sp) * DT_TS + t4);
+#pragma unroll
+                for (int tt = 0; tt < 4; ++tt) {
+                    const int t = t4 + tt;
+                    const float xt = __shfl_sync(0xffffffffu, x[t >> 2], (lane & ~3) | (t & 3));
+#pragma unroll
+                    for (int m = t4 / 4; m < 16; ++m) {
+                        const float at = tt == 0 ? a[m].x : tt == 1 ? a[m].y : tt == 2 ? a[m].z : a[m].w;
+                        if (4 * m + sp > t) x[m] = fmaf(-at, xt, x[m]);
+                    }
+                }
+            }
+            __syncthreads();   // every thread has read its R
+#pragma unroll
+            for (int m = 0; m < 16; ++m) sW[(4 * m + sp) * DT_TS + sj] = x[m];
+        }
+        __syncthreads();
+        if (t0 + rt < L) {
+            float* dst = A.xw + (rowbase + t0 + rt) * Dv + col0 + rc;
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(dst + j) = *reinterpret_cast<const float4*>(sW + rt * DT_TS + rc + j);
+        }
+        if (!dt_wait(bar_mma, (n_mma - 1) & 1)) { err = 1; break; }   // dX (and X's readers above)
+        tc_fence_after();
+        {
+            uint32_t r[32];
+            tmem_ld32(tq_lane + C::C_KS + 32 * wg, r);
+            tmem_wait_ld();
+            if (!first)
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4*>(sW + mrow * DT_TS + 32 * wg + j) =
+                        make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                                    __uint_as_float(r[j + 3]));
+        }
+        __syncthreads();
+
+        // ---- 4. dR = (I + A)^{-T} dX: rows from the last, dR[u] subtracted (A[u][t] dR[u]) from
+        //      every earlier row t; A^T read four columns at a time
+        {
+            float x[16];
+#pragma unroll
+            for (int m = 0; m < 16; ++m) x[m] = sW[(4 * m + sp) * DT_TS + sj];
+#pragma unroll
+            for (int u4 = TR - 4; u4 >= 0; u4 -= 4) {
+                float4 a[16];
+#pragma unroll
+                for (int m = 0; m <= u4 / 4; ++m) a[m] = *reinterpret_cast<const float4*>(sAT + (4 * m + sp) * DT_TS + u4);
+#pragma unroll
+                for (int uu = 3; uu >= 0; --uu) {
+                    const int u = u4 + uu;
+                    const float xu = __shfl_sync(0xffffffffu, x[u >> 2], (lane & ~3) | (u & 3));
+#pragma unroll
+                    for (int m = 0; m <= u4 / 4; ++m) {
+                        const float at = uu == 0 ? a[m].x : uu == 1 ? a[m].y : uu == 2 ? a[m].z : a[m].w;
+                        if (4 * m + sp < u) x[m] = fmaf(-at, xu, x[m]);
+                    }
+                }
+            }
+            __syncthreads();
+#pragma unroll
+            for (int m = 0; m < 16; ++m) sW[(4 * m + sp) * DT_TS + sj] = x[m];
+        }
+        __syncthreads();
+
+        // ---- 5. dR, dV = diag(beta) dR, the slice's part of sum_j dR U, and -diag(beta) dR (bf16)
+        {
+            const float bt = sB[rt];
+            float dr[16], acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) {
+                const float4 x = *reinterpret_cast<const float4*>(sW + rt * DT_TS + rc + j);
+                const float4 u4 = *reinterpret_cast<const float4*>(sU + rt * DT_TS + rc + j);
+                dr[j] = x.x; dr[j + 1] = x.y; dr[j + 2] = x.z; dr[j + 3] = x.w;
+                acc += x.x * u4.x + x.y * u4.y + x.z * u4.z + x.w * u4.w;
+            }
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            if (t0 + rt < L) {
+                const long row = rowbase + t0 + rt;
+                float* dst = A.drw + row * Dv + col0 + rc;
+#pragma unroll
+                for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(dr[j], dr[j + 1], dr[j + 2], dr[j + 3]);
+                float bv[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) bv[j] = bt * dr[j];
+                dt_store16_bf16(A.dv + row * Dv + col0 + rc, bv);
+                if ((tid & 3) == 0) A.db1[(long)slice * A.BH * L + row] = acc;
+            }
+            float nb[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) nb[j] = -bt * dr[j];
+            store8_bf16(sBR, sw128_off(rt, rc, BLK), nb);
+            store8_bf16(sBR, sw128_off(rt, rc + 8, BLK), nb + 8);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ---- 6. dS += Q^T dO + K^T (-diag(beta) dR)
+        if (warp == 0) {
+            const bool leader = elect_one();
+            const uint32_t idS = idesc_bf16(C::MS, DT_VT, 1, 1);
+            const uint64_t dQm = sw128_desc(smem_u32(sq), BLK, 1024), dKm = sw128_desc(smem_u32(sk), BLK, 1024);
+            const uint64_t dO = sw128_desc(smem_u32(sdo), BLK, 1024), dB = sw128_desc(smem_u32(sBR), BLK, 1024);
+#pragma unroll
+            for (int ks = 0; ks < TR / 16; ++ks) {
+                if (leader) {
+                    mma_bf16(tbase + C::C_S, dQm + ((ks * 2048) >> 4), dO + ((ks * 2048) >> 4), idS, 1);
+                    mma_bf16(tbase + C::C_S, dKm + ((ks * 2048) >> 4), dB + ((ks * 2048) >> 4), idS, 1);
+                }
+            }
+            if (leader) mma_commit(bar_mma);
+            __syncwarp();
+        }
+        ++n_mma;
+        if (!dt_wait(bar_mma, (n_mma - 1) & 1)) { err = 1; break; }
+        tc_fence_after();
+        {
+            uint32_t r[32];
+            tmem_ld32(tq_lane + C::C_S + 32 * wg, r);
+            tmem_wait_ld();
+            if (srow_ok)
+#pragma unroll
+                for (int j = 0; j < 32; j += 8)
+                    store8_bf16(sG, sw128_off(srow, 32 * wg + j, DK * 128), reinterpret_cast<const float*>(r + j));
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0 && i + C::NS < nc) issue_loads(i + C::NS, s);
+    }
+
+    if (err) {
+        if (warp == 0) {
+            const bool leader = elect_one();
+            if (leader) {
+                mma_commit(bar_drain);
+                mbar_wait(bar_drain, 0, 1u << 20);
+            }
+            __syncwarp();
+        }
+    } else if (A.dh0) {
+        uint32_t r[32];
+        tmem_ld32(tq_lane + C::C_S + 32 * wg, r);
+        tmem_wait_ld();
+        if (srow_ok) dt_put_row(A.dh0 + ((long)bh * DK + srow) * Dv + col0 + 32 * wg, r);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, C::NCOL);
+}
+
+template <int DK>
+cudaError_t dw_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                      const DwArgs& a, cudaStream_t st) {
+    auto kern = k_deltanet_tc_walk<DK>;
+    const uint32_t smem = DwCfg<DK>::SMEM;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(a.BH, a.Dv / DT_VT);
+    GLA_LAUNCH("deltanet_bwd_walk", st, (kern<<<grid, DT_NT, smem, st>>>(mq, mk, mv, mdo, a)));
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t deltanet_fwd(int B, int H, int L, int Dk, int Dv, float scale, const void* q, const void* k,
@@ -441,6 +914,42 @@ cudaError_t deltanet_fwd(int B, int H, int L, int Dk, int Dv, float scale, const
                  : dt_launch<64, false>(B, H, L, Dv, mq, mk, mv, mo, a, st);
     return o ? dt_launch<128, true>(B, H, L, Dv, mq, mk, mv, mo, a, st)
              : dt_launch<128, false>(B, H, L, Dv, mq, mk, mv, mo, a, st);
+}
+
+
+cudaError_t deltanet_walk(int B, int H, int L, int Dk, int Dv, float scale, const void* q, const void* k,
+                          const void* v, const float* beta, const void* dO, const float* dhT, const float* saved,
+                          float* xw, float* drw, float* dsend, float* db1, void* dv, float* dh0, cudaStream_t st) {
+    const int BH = B * H;
+    if (BH == 0) return cudaSuccess;
+    if (L == 0) {   // no chunk: dh0 = dhT (or zero)
+        if (dh0) {
+            const size_t n = (size_t)BH * Dk * Dv * sizeof(float);
+            return dhT ? cudaMemcpyAsync(dh0, dhT, n, cudaMemcpyDeviceToDevice, st) : cudaMemsetAsync(dh0, 0, n, st);
+        }
+        return cudaSuccess;
+    }
+    CUtensorMap mq, mk, mv, mdo;
+    if (!make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dk, L, BH, 64, true) ||
+        !make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dk, L, BH, 64, true) ||
+        !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dv, L, BH, 64, true) ||
+        !make_map(&mdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dv, L, BH, 64, true))
+        return cudaErrorInvalidValue;
+    DwArgs a{};
+    a.beta = beta;
+    a.saved = saved;
+    a.dhT = dhT;
+    a.xw = xw;
+    a.drw = drw;
+    a.dsend = dsend;
+    a.db1 = db1;
+    a.dv = static_cast<__nv_bfloat16*>(dv);
+    a.dh0 = dh0;
+    a.BH = BH;
+    a.L = L;
+    a.Dv = Dv;
+    a.scale = scale;
+    return Dk == 64 ? dw_launch<64>(mq, mk, mv, mdo, a, st) : dw_launch<128>(mq, mk, mv, mdo, a, st);
 }
 
 }  // namespace tc

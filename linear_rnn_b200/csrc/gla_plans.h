@@ -47,6 +47,12 @@ int num_sms();
 cudaError_t deltanet_fwd(int B, int H, int L, int Dk, int Dv, float scale, const void* q, const void* k,
                          const void* v, const float* beta, const float* h0, void* o, float* hT, float* saved,
                          int* status, cudaStream_t st);
+// The DeltaNet backward's reverse walk on the tensor cores (gla_deltanet_tc.cu), same limits:
+// from the saved chunk start states, writes X and dR ([BH*L, Dv] fp32), the gradient at every
+// chunk's end (as saved), each 64-column slice's sum_j dR U ([Dv/64, BH*L]), dv (bf16) and dh0.
+cudaError_t deltanet_walk(int B, int H, int L, int Dk, int Dv, float scale, const void* q, const void* k,
+                          const void* v, const float* beta, const void* dO, const float* dhT, const float* saved,
+                          float* xw, float* drw, float* dsend, float* db1, void* dv, float* dh0, cudaStream_t st);
 // Backward (gla_tc_bwd.cu)
 bool bwd_supports(const Dims& P);
 size_t bwd_workspace_bytes(const Dims& P);

@@ -162,6 +162,26 @@ def test_backward_edge_lengths(L):
     assert r["dq"].shape == (1, 2, L, 64)
 
 
+def test_backward_full_size():
+    """The DeltaNet workload's backward (B=4 H=16 L=4096 Dk=Dv=128, bf16: the tensor-core state
+    and reverse walks); two heads against the oracle's back-propagation through time."""
+    from linear_rnn_b200 import ops
+    c = I.DELTANET
+    B, H, L, Dk, Dv = c["B"], c["H"], c["L"], c["Dk"], c["Dv"]
+    x = I.make_deltanet_inputs(B, H, L, Dk, Dv, c["dtype"], seed=0, h0_std=0.5)
+    gen = torch.Generator().manual_seed(100)
+    dO = torch.randn(B, H, L, Dv, generator=gen).to(x["q"].dtype)
+    xd = {n: (None if t is None else t.cuda()) for n, t in x.items()}
+    r = ops.gla_deltanet_bwd(xd["q"], xd["k"], xd["v"], xd["beta"], xd["h0"], dO.cuda(), None, scale=Dk ** -0.5)
+    torch.cuda.synchronize()
+    heads = [5, 50]
+    xs = {n: heads_of(t, heads) for n, t in x.items()}
+    ref = DN.deltanet_bwd(xs["q"], xs["k"], xs["v"], xs["beta"], xs["h0"], heads_of(dO, heads), None, Dk ** -0.5)
+    errs = {n: err(f64(heads_of(r[n], heads)), ref[n]) for n in ("dq", "dk", "dv", "dbeta", "dh0")}
+    record("deltanet backward full size heads=[5, 50]", errs)
+    assert all(e <= TOL["bf16"] for e in errs.values()), errs
+
+
 def test_backward_long_sequence():
     check_bwd(1, 2, 2048, 128, 128, "bf16", 0.5, True, seed=8, case="deltanet backward L=2048")
 
