@@ -752,6 +752,9 @@ cudaError_t dn_bwd_launch(const gla_problem* p, const void* q, const void* k, co
         e = cudaGetLastError();
     }
     if (e != cudaSuccess) return e;
+    if (std::is_same<T, __nv_bfloat16>::value)   // bf16 I/O: the tensor-core gradients
+        return tc::deltanet_grads(p->B, p->H, p->L, DK, p->Dv, p->scale, q, k, beta, dO, w.saved, w.xw, w.drw,
+                                  w.dsend, w.db1, dq, dk, dbeta, st);
     if (NC > 0)
         GLA_LAUNCH("deltanet_bwd_grads", st,
                    (grads<<<dim3(NC, BH), DN_NT, sg, st>>>(tq, tk, beta, tdo, w.saved, w.xw, w.drw, w.dsend, w.db1,

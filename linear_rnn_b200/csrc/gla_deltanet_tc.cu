@@ -23,7 +23,8 @@
 //      entering the next chunk in fp32).
 // K, Q and V tiles arrive by TMA into a two-stage ring, so the next chunk's loads overlap this
 // chunk's work. Every phase runs on all 8 warps in turn; one elected lane of warp 0 issues the
-// MMAs and the TMA copies.
+// MMAs and the TMA copies. The backward's reverse walk and its per-chunk gradient kernel follow
+// below in the same style.
 #include <cudaTypedefs.h>
 
 #include "gla_common.cuh"
@@ -873,6 +874,330 @@ cudaError_t dw_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ backward gradients
+// Per chunk, all chunks in parallel, from the walk's X, dR, the chunk's start state S and end
+// gradient dS' (value columns in 64-wide slices, summed in tensor memory):
+//   dP = scale lower(dO X^T),  G = -strict_lower(dR X^T)
+//   dQ = scale dO S^T + dP K
+//   dK = X dS'^T - diag(beta) dR S^T + dP^T Q + diag(beta) (G K) + G^T diag(beta) K
+//   dbeta_t = sum_j dR_tj U_tj (the walk's slice sums) + sum_i k_ti (G K)_ti
+// One CTA per (chunk, batch*head). dO is scaled in place, so dO X^T and dO S^T carry the scale.
+template <int DK>
+struct DgCfg {
+    static constexpr uint32_t KB = TR * DK * 2;   // K, Q tiles (TMA)
+    static constexpr uint32_t MB = TR * TR * 2;   // 64 x 64 bf16: dO, X, dR, -diag(beta) dR, dP, G
+    static constexpr uint32_t SB = DK * DT_VT * 2;   // S and dS' slices, bf16, K-major rows of key dims
+    static constexpr uint32_t SMALL = 256 + 4 * TR + 8 * TR;
+    static constexpr uint32_t SMEM = 3 * KB + 6 * MB + 2 * SB + SMALL + 1024;
+    // TMEM: dO X^T | dR X^T (lanes 0-15 | 16-31) at 0; dQ | dK at 64; G K (lanes 16-31) at 64 + DK
+    static constexpr uint32_t C_PG = 0, C_QK = 64, C_GK = 64 + DK, NCOL = 64 + 2 * DK <= 256 ? 256 : 512;
+    static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+struct DgArgs {
+    const float* beta;    // [BH*L]
+    const float* saved;   // [BH, NC, Dk, Dv]
+    const float* xw;      // [BH*L, Dv]
+    const float* drw;     // [BH*L, Dv]
+    const float* dsend;   // [BH, NC, Dk, Dv]
+    const float* db1;     // [Dv/64, BH*L]
+    __nv_bfloat16* dq;    // [BH*L, Dk]
+    __nv_bfloat16* dk;
+    float* dbeta;         // [BH*L]
+    int BH, L, Dv;
+    float scale;
+};
+
+template <int DK>
+__global__ void __launch_bounds__(DT_NT, 1)
+    k_deltanet_tc_grads(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                        const __grid_constant__ CUtensorMap tdo, DgArgs A) {
+    using C = DgCfg<DK>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = smem_align1024(smem_raw);
+    uint8_t* sK = sm;
+    uint8_t* sQ = sK + C::KB;
+    uint8_t* sBK = sQ + C::KB;      // diag(beta) K
+    uint8_t* sDO = sBK + C::KB;
+    uint8_t* sX = sDO + C::MB;
+    uint8_t* sDR = sX + C::MB;
+    uint8_t* sNB = sDR + C::MB;     // -diag(beta) dR
+    uint8_t* sDP = sNB + C::MB;
+    uint8_t* sGm = sDP + C::MB;
+    uint8_t* sSb = sGm + C::MB;
+    uint8_t* sDS = sSb + C::SB;
+    uint8_t* small = sDS + C::SB;
+    uint64_t* bar_kq = reinterpret_cast<uint64_t*>(small);
+    uint64_t* bar_do = bar_kq + 1;
+    uint64_t* bar_mma = bar_kq + 2;
+    uint64_t* bar_drain = bar_kq + 3;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 64);
+    float* sB = reinterpret_cast<float*>(small + 256);      // beta [64]
+    float* sDB = sB + TR;                                   // [2][64] partial sums of k . (G K)
+
+    const int ci = blockIdx.x, bh = blockIdx.y;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2, qd = warp & 3;
+    const int L = A.L, Dv = A.Dv, nsl = Dv / DT_VT;
+    const int nc = (L + TR - 1) / TR, t0 = ci * TR;
+    const long rowbase = (long)bh * L;
+    const long cbase = (long)bh * nc + ci;
+    const int mrow = 16 * qd + (lane & 15);
+    const bool first = lane < 16;
+    const int rt = tid >> 2, rc = 16 * (tid & 3);   // row pass: token row, 16 value columns
+
+    if (tid == 0) {
+        mbar_init(bar_kq, 1);
+        mbar_init(bar_do, 1);
+        mbar_init(bar_mma, 1);
+        mbar_init(bar_drain, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, C::NCOL);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tq_lane = tbase + ((uint32_t)(32 * qd) << 16);
+    if (tid == 0) {
+        mbar_arrive_expect_tx(bar_kq, 2 * C::KB);
+        for (int cb = 0; cb < DK / 64; ++cb) {
+            tma_load_3d(sK + cb * BLK, &tk, cb * 64, t0, bh, bar_kq);
+            tma_load_3d(sQ + cb * BLK, &tq, cb * 64, t0, bh, bar_kq);
+        }
+    }
+    if (tid < TR) sB[tid] = t0 + tid < L ? A.beta[rowbase + t0 + tid] : 0.f;
+    __syncthreads();   // beta is read by every row pass below
+
+    int err = 0, n_mma = 0, n_do = 0;
+    for (int sl = 0; sl < nsl && !err; ++sl) {
+        const int col0 = sl * DT_VT;
+        if (tid == 0) {
+            mbar_arrive_expect_tx(bar_do, C::MB);
+            tma_load_3d(sDO, &tdo, col0, t0, bh, bar_do);
+        }
+        // X, dR and -diag(beta) dR (bf16, rows of tokens); S and dS' (bf16, rows of key dims)
+        {
+            const bool in = t0 + rt < L;
+            const long off = (rowbase + t0 + rt) * Dv + col0 + rc;
+            const float bt = sB[rt];
+            float x[16], d[16], nb[16];
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) {
+                const float4 a = in ? __ldg(reinterpret_cast<const float4*>(A.xw + off + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float4 b = in ? __ldg(reinterpret_cast<const float4*>(A.drw + off + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                x[j] = a.x; x[j + 1] = a.y; x[j + 2] = a.z; x[j + 3] = a.w;
+                d[j] = b.x; d[j + 1] = b.y; d[j + 2] = b.z; d[j + 3] = b.w;
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) nb[j] = -bt * d[j];
+            store8_bf16(sX, sw128_off(rt, rc, BLK), x);
+            store8_bf16(sX, sw128_off(rt, rc + 8, BLK), x + 8);
+            store8_bf16(sDR, sw128_off(rt, rc, BLK), d);
+            store8_bf16(sDR, sw128_off(rt, rc + 8, BLK), d + 8);
+            store8_bf16(sNB, sw128_off(rt, rc, BLK), nb);
+            store8_bf16(sNB, sw128_off(rt, rc + 8, BLK), nb + 8);
+        }
+        {
+            constexpr int TPR = DT_NT / DK, CPT = DT_VT / TPR;   // threads per key row, columns per thread
+            const int kr = tid / TPR, kc = (tid % TPR) * CPT;
+            const long off = (cbase * DK + kr) * Dv + col0 + kc;
+#pragma unroll
+            for (int j = 0; j < CPT; j += 8) {
+                float s8[8], g8[8];
+#pragma unroll
+                for (int u = 0; u < 8; u += 4) {
+                    const float4 a = __ldg(reinterpret_cast<const float4*>(A.saved + off + j + u));
+                    const float4 b = __ldg(reinterpret_cast<const float4*>(A.dsend + off + j + u));
+                    s8[u] = a.x; s8[u + 1] = a.y; s8[u + 2] = a.z; s8[u + 3] = a.w;
+                    g8[u] = b.x; g8[u + 1] = b.y; g8[u + 2] = b.z; g8[u + 3] = b.w;
+                }
+                store8_bf16(sSb, sw128_off(kr, kc + j, BLK), s8);
+                store8_bf16(sDS, sw128_off(kr, kc + j, BLK), g8);
+            }
+        }
+        ++n_do;
+        if (!dt_wait(bar_do, (n_do - 1) & 1)) { err = 1; break; }
+        // dO scaled in place (the output scale of dO X^T and dO S^T)
+        for (int e = tid; e < (int)(C::MB / 16); e += DT_NT) {
+            uint4 w = *reinterpret_cast<uint4*>(sDO + 16 * e);
+            uint32_t* pw = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&pw[u]));
+                __nv_bfloat162 h = __floats2bfloat162_rn(f.x * A.scale, f.y * A.scale);
+                pw[u] = *reinterpret_cast<uint32_t*>(&h);
+            }
+            *reinterpret_cast<uint4*>(sDO + 16 * e) = w;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (warp == 0) {
+            const bool leader = elect_one();
+            const uint32_t id64 = idesc_bf16(64, 64, 0, 0), idK = idesc_bf16(64, DK, 0, 0);
+            const uint32_t a_do = smem_u32(sDO), a_x = smem_u32(sX), a_dr = smem_u32(sDR), a_nb = smem_u32(sNB);
+            const uint32_t b_s = smem_u32(sSb), b_ds = smem_u32(sDS);
+#pragma unroll
+            for (int kk = 0; kk < DT_VT / 16; ++kk) {
+                const uint32_t ko = kk * 32;
+                const uint32_t acc = (sl > 0 || kk > 0) ? 1u : 0u;
+                if (leader) {
+                    mma_bf16(tbase + C::C_PG, sw128_desc(a_do + ko, 16, 1024), sw128_desc(a_x + ko, 16, 1024), id64, acc);
+                    mma_bf16(tbase + C::C_PG + (16u << 16), sw128_desc(a_dr + ko, 16, 1024), sw128_desc(a_x + ko, 16, 1024),
+                             id64, acc);
+                    mma_bf16(tbase + C::C_QK, sw128_desc(a_do + ko, 16, 1024), sw128_desc(b_s + ko, 16, 1024), idK, acc);
+                    mma_bf16(tbase + C::C_QK + (16u << 16), sw128_desc(a_x + ko, 16, 1024), sw128_desc(b_ds + ko, 16, 1024),
+                             idK, acc);
+                    mma_bf16(tbase + C::C_QK + (16u << 16), sw128_desc(a_nb + ko, 16, 1024), sw128_desc(b_s + ko, 16, 1024),
+                             idK, 1);
+                }
+            }
+            if (leader) mma_commit(bar_mma);
+            __syncwarp();
+        }
+        ++n_mma;
+        if (!dt_wait(bar_mma, (n_mma - 1) & 1)) { err = 1; break; }   // the slice's tiles may be rewritten
+        tc_fence_after();
+    }
+    if (!err && !dt_wait(bar_kq, 0)) err = 1;
+    if (!err) {
+        // dP = lower(dO X^T) (bf16; the scale came with dO) and G = -strict_lower(dR X^T); diag(beta) K
+        {
+            uint32_t r[32];
+            tmem_ld32(tq_lane + C::C_PG + 32 * wg, r);
+            tmem_wait_ld();
+            const int t = mrow;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float f[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int sc = 32 * wg + 8 * u + j;
+                    const float y = __uint_as_float(r[8 * u + j]);
+                    f[j] = first ? (sc <= t ? y : 0.f) : (sc < t ? -y : 0.f);
+                }
+                store8_bf16(first ? sDP : sGm, sw128_off(t, 32 * wg + 8 * u, BLK), f);
+            }
+        }
+        for (int e = tid; e < (int)(C::KB / 16); e += DT_NT) {
+            // 16-byte chunk e of the K tile: row (e % 8 + 8 (e / 64 % 8)) ... the row of a chunk in
+            // the 128-byte-swizzled layout is its byte offset / 128 within its 64-column block
+            const int row = (int)(((uint32_t)e * 16 % BLK) / 128);
+            uint4 w = *reinterpret_cast<const uint4*>(sK + 16 * e);
+            uint32_t* pw = reinterpret_cast<uint32_t*>(&w);
+            const float b = sB[row];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&pw[u]));
+                __nv_bfloat162 h = __floats2bfloat162_rn(f.x * b, f.y * b);
+                pw[u] = *reinterpret_cast<uint32_t*>(&h);
+            }
+            *reinterpret_cast<uint4*>(sBK + 16 * e) = w;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (warp == 0) {
+            const bool leader = elect_one();
+            const uint32_t idKm = idesc_bf16(64, DK, 0, 1), idMM = idesc_bf16(64, DK, 1, 1);
+            const uint64_t dPk = sw128_desc(smem_u32(sDP), 16, 1024), dPm = sw128_desc(smem_u32(sDP), BLK, 1024);
+            const uint64_t dGk = sw128_desc(smem_u32(sGm), 16, 1024), dGm = sw128_desc(smem_u32(sGm), BLK, 1024);
+            const uint64_t dKm = sw128_desc(smem_u32(sK), BLK, 1024), dQm = sw128_desc(smem_u32(sQ), BLK, 1024);
+            const uint64_t dBm = sw128_desc(smem_u32(sBK), BLK, 1024);
+#pragma unroll
+            for (int ks = 0; ks < TR / 16; ++ks) {
+                const uint64_t ka = (ks * 32) >> 4, km = (ks * 2048) >> 4;
+                if (leader) {
+                    mma_bf16(tbase + C::C_QK, dPk + ka, dKm + km, idKm, 1);                      // dQ += dP K
+                    mma_bf16(tbase + C::C_QK + (16u << 16), dPm + km, dQm + km, idMM, 1);        // dK += dP^T Q
+                    mma_bf16(tbase + C::C_QK + (16u << 16), dGm + km, dBm + km, idMM, 1);        // dK += G^T diag(beta) K
+                    mma_bf16(tbase + C::C_GK + (16u << 16), dGk + ka, dKm + km, idKm, ks > 0);   // G K
+                }
+            }
+            if (leader) mma_commit(bar_mma);
+            __syncwarp();
+        }
+        ++n_mma;
+        if (!dt_wait(bar_mma, (n_mma - 1) & 1)) err = 1;
+    }
+    if (!err) {
+        tc_fence_after();
+        // dq (lanes 0-15) and dk = dK + diag(beta) G K (lanes 16-31); k_t . (G K)_t partial sums
+        const int t = mrow;
+        const bool in = t0 + t < L;
+        float dbp = 0.f;
+        for (int cc = 0; cc < DK / 2; cc += 32) {
+            const int c = wg * (DK / 2) + cc;
+            uint32_t r[32], g[32];
+            tmem_ld32(tq_lane + C::C_QK + c, r);
+            tmem_ld32(tq_lane + C::C_GK + c, g);
+            tmem_wait_ld();
+            if (first) {
+                if (in) {
+                    float f[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(r[j]);
+                    dt_store16_bf16(A.dq + (rowbase + t0 + t) * DK + c, f);
+                    dt_store16_bf16(A.dq + (rowbase + t0 + t) * DK + c + 16, f + 16);
+                }
+            } else {
+                const float bt = sB[t];
+                float f[32];
+#pragma unroll
+                for (int j = 0; j < 32; j += 8) {
+                    const uint4 kw = *reinterpret_cast<const uint4*>(sK + sw128_off(t, c + j, BLK));
+                    const uint32_t* kp = reinterpret_cast<const uint32_t*>(&kw);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kp[u]));
+                        const float g0 = __uint_as_float(g[j + 2 * u]), g1 = __uint_as_float(g[j + 2 * u + 1]);
+                        f[j + 2 * u] = __uint_as_float(r[j + 2 * u]) + bt * g0;
+                        f[j + 2 * u + 1] = __uint_as_float(r[j + 2 * u + 1]) + bt * g1;
+                        dbp += kf.x * g0 + kf.y * g1;
+                    }
+                }
+                if (in) {
+                    dt_store16_bf16(A.dk + (rowbase + t0 + t) * DK + c, f);
+                    dt_store16_bf16(A.dk + (rowbase + t0 + t) * DK + c + 16, f + 16);
+                }
+            }
+        }
+        if (!first) sDB[wg * TR + t] = dbp;
+        __syncthreads();
+        if (tid < TR && t0 + tid < L) {
+            float x = sDB[tid] + sDB[TR + tid];
+            for (int s2 = 0; s2 < nsl; ++s2) x += A.db1[(long)s2 * A.BH * L + rowbase + t0 + tid];
+            A.dbeta[rowbase + t0 + tid] = x;
+        }
+    }
+    if (err) {
+        if (warp == 0) {
+            const bool leader = elect_one();
+            if (leader) {
+                mma_commit(bar_drain);
+                mbar_wait(bar_drain, 0, 1u << 20);
+            }
+            __syncwarp();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, C::NCOL);
+}
+
+template <int DK>
+cudaError_t dg_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mdo, const DgArgs& a,
+                      int nc, cudaStream_t st) {
+    auto kern = k_deltanet_tc_grads<DK>;
+    const uint32_t smem = DgCfg<DK>::SMEM;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    GLA_LAUNCH("deltanet_bwd_grads", st, (kern<<<dim3(nc, a.BH), DT_NT, smem, st>>>(mq, mk, mdo, a)));
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t deltanet_fwd(int B, int H, int L, int Dk, int Dv, float scale, const void* q, const void* k,
@@ -950,6 +1275,33 @@ cudaError_t deltanet_walk(int B, int H, int L, int Dk, int Dv, float scale, cons
     a.Dv = Dv;
     a.scale = scale;
     return Dk == 64 ? dw_launch<64>(mq, mk, mv, mdo, a, st) : dw_launch<128>(mq, mk, mv, mdo, a, st);
+}
+
+cudaError_t deltanet_grads(int B, int H, int L, int Dk, int Dv, float scale, const void* q, const void* k,
+                           const float* beta, const void* dO, const float* saved, const float* xw, const float* drw,
+                           const float* dsend, const float* db1, void* dq, void* dk, float* dbeta, cudaStream_t st) {
+    const int BH = B * H, nc = (L + TR - 1) / TR;
+    if (BH == 0 || nc == 0) return cudaSuccess;
+    CUtensorMap mq, mk, mdo;
+    if (!make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dk, L, BH, 64, true) ||
+        !make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dk, L, BH, 64, true) ||
+        !make_map(&mdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dv, L, BH, 64, true))
+        return cudaErrorInvalidValue;
+    DgArgs a{};
+    a.beta = beta;
+    a.saved = saved;
+    a.xw = xw;
+    a.drw = drw;
+    a.dsend = dsend;
+    a.db1 = db1;
+    a.dq = static_cast<__nv_bfloat16*>(dq);
+    a.dk = static_cast<__nv_bfloat16*>(dk);
+    a.dbeta = dbeta;
+    a.BH = BH;
+    a.L = L;
+    a.Dv = Dv;
+    a.scale = scale;
+    return Dk == 64 ? dg_launch<64>(mq, mk, mdo, a, nc, st) : dg_launch<128>(mq, mk, mdo, a, nc, st);
 }
 
 }  // namespace tc

@@ -53,6 +53,11 @@ cudaError_t deltanet_fwd(int B, int H, int L, int Dk, int Dv, float scale, const
 cudaError_t deltanet_walk(int B, int H, int L, int Dk, int Dv, float scale, const void* q, const void* k,
                           const void* v, const float* beta, const void* dO, const float* dhT, const float* saved,
                           float* xw, float* drw, float* dsend, float* db1, void* dv, float* dh0, cudaStream_t st);
+// The DeltaNet backward's per-chunk gradients on the tensor cores (gla_deltanet_tc.cu): dq, dk
+// (bf16) and dbeta from the walk's outputs, one CTA per (chunk, batch*head).
+cudaError_t deltanet_grads(int B, int H, int L, int Dk, int Dv, float scale, const void* q, const void* k,
+                           const float* beta, const void* dO, const float* saved, const float* xw, const float* drw,
+                           const float* dsend, const float* db1, void* dq, void* dk, float* dbeta, cudaStream_t st);
 // Backward (gla_tc_bwd.cu)
 bool bwd_supports(const Dims& P);
 size_t bwd_workspace_bytes(const Dims& P);
