@@ -496,17 +496,21 @@ def run_deltanet(args, world, rank, local):
 
     if rank != 0:
         return
-    peak = deltanet_alu_peak_tflops(clocks.get("sm_max_mhz"))
+    # bf16 I/O runs the chunk products on the tensor cores (against the measured bf16 GEMM peak);
+    # fp32 I/O on the CUDA cores (against the FP32 FMA peak derived from the unit counts)
+    tensor = I.DELTANET["dtype"] == "bf16"
+    peaks, peak_src = load_peaks()
+    peak = peaks["bf16_tflops"] if tensor else deltanet_alu_peak_tflops(clocks.get("sm_max_mhz"))
     roofline = None
     if kprof:
         name, (cnt, ms) = max(kprof.items(), key=lambda kv: kv[1][1])
         avg_s = ms / cnt / 1e3
         fl = deltanet_kernel_flops(name, B, H, L, Dk, Dv)
         ach = fl / avg_s / 1e12
-        roofline = {"bound": "alu", "kernel": name, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                    "frac": ach / peak, "traffic": None,
-                    "peak_source": "nominal, derived (not measured): 148 SMs x 128 FP32 lanes x 2 FLOPs x "
-                                   "the sampled max SM clock",
+        roofline = {"bound": "tensor" if tensor else "alu", "kernel": name, "achieved": ach, "peak": peak,
+                    "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
+                    "peak_source": peak_src if tensor else
+                    "nominal, derived (not measured): 148 SMs x 128 FP32 lanes x 2 FLOPs x the sampled max SM clock",
                     "algorithmic_flops_per_launch": fl, "avg_launch_us": avg_s * 1e6,
                     "share_of_step": ms / sum(v[1] for v in kprof.values())}
     extra = {"e2e": e2e, "gpu_launches": int(launches), "roofline": roofline, "clocks": clocks,
