@@ -158,6 +158,8 @@ MEASURED_TRAFFIC = {
                           "sha": "fab635eb697cc988", "case": "c3"},
     ("tc_bwd_dq", "c5"): {"bytes": 392.6e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
                           "sha": "fab635eb697cc988", "case": "c5"},
+    ("deltanet_bwd_walk", "deltanet"): {"bytes": 1099.9e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_deltanet_tc.cu",
+                                         "sha": "6ca3bafb3ab9258b", "case": "deltanet"},
     ("decode", "decode"): {"bytes": 214.9e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_decode.cu",
                            "sha": "45347f72608393eb", "case": "decode, 1024 heads"},
 }
@@ -508,7 +510,8 @@ def run_deltanet(args, world, rank, local):
         fl = deltanet_kernel_flops(name, B, H, L, Dk, Dv)
         ach = fl / avg_s / 1e12
         roofline = {"bound": "tensor" if tensor else "alu", "kernel": name, "achieved": ach, "peak": peak,
-                    "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
+                    "unit": "TFLOP/s", "frac": ach / peak,
+                    "traffic": measured_traffic(name, "deltanet") if tensor else None,
                     "peak_source": peak_src if tensor else
                     "nominal, derived (not measured): 148 SMs x 128 FP32 lanes x 2 FLOPs x the sampled max SM clock",
                     "algorithmic_flops_per_launch": fl, "avg_launch_us": avg_s * 1e6,
