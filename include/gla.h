@@ -224,10 +224,10 @@ GLA_API gla_status gla_deltanet_fwd(const gla_problem* p, const void* q, const v
  * the gradient at the chunk's end), then per chunk dQ, dK, dbeta from those products.
  * Same p and inputs as gla_deltanet_fwd; dO [B,H,L,Dv] io dtype; dhT [B,H,Dk,Dv] f32 or NULL.
  * Outputs (written): dq, dk [B,H,L,Dk] and dv [B,H,L,Dv] io dtype; dbeta [B,H,L] f32; dh0
- * [B,H,Dk,Dv] f32 or NULL. ws: device workspace of gla_deltanet_bwd_workspace_bytes(p) bytes
- * (the chunk start states, X, dR, the chunk end gradients and per-slice sums), caller-owned.
- * Three launches on `stream` (the forward's state pass, the reverse walk, the per-chunk
- * gradients).
+ * [B,H,Dk,Dv] f32 or NULL. ws: device workspace of gla_deltanet_bwd_workspace_bytes(p) bytes,
+ * caller-owned: the chunk start states and end gradients (bf16 for bf16 I/O, fp32 for fp32 I/O)
+ * and dR; fp32 I/O also X and per-slice sums. Three launches on `stream` (the forward's state
+ * walk, the reverse walk, the per-chunk gradients); bf16 I/O runs them on the tensor cores.
  * Errors: as gla_deltanet_fwd, plus GLA_ERR_WORKSPACE. */
 GLA_API size_t gla_deltanet_bwd_workspace_bytes(const gla_problem* p);
 GLA_API gla_status gla_deltanet_bwd(const gla_problem* p, const void* q, const void* k, const void* v,

@@ -709,16 +709,21 @@ struct DnBwdWs {
     size_t bytes;
 };
 
+// Backward workspace. fp32 I/O (CUDA-core kernels): the chunk start states and end gradients in
+// fp32, X and dR, and each value slice's sum_j dR U. bf16 I/O (tensor-core kernels): the chunk
+// start states and end gradients in bf16 (the precision the products read them in) and dR; the
+// gradient kernel forms X and sum_j dR U itself.
 DnBwdWs dn_bwd_ws(const gla_problem* p, void* base) {
     const size_t BH = (size_t)p->B * p->H, NC = (size_t)((p->L + DN_C - 1) / DN_C);
     const size_t st = BH * NC * p->Dk * p->Dv, tok = BH * p->L * p->Dv, nsl = p->Dv / DN_VT;
-    const size_t sizes[5] = {st, tok, tok, st, nsl * BH * p->L};
+    const bool tc = p->io == GLA_BF16;
+    const size_t bytes[5] = {st * (tc ? 2 : 4), tc ? 0 : tok * 4, tok * 4, st * (tc ? 2 : 4), tc ? 0 : nsl * BH * p->L * 4};
     DnBwdWs w{};
     float** dst[5] = {&w.saved, &w.xw, &w.drw, &w.dsend, &w.db1};
     size_t off = 0;
     for (int i = 0; i < 5; ++i) {
-        *dst[i] = base ? reinterpret_cast<float*>(static_cast<char*>(base) + off) : nullptr;
-        off += (sizes[i] * 4 + 255) / 256 * 256;
+        *dst[i] = (base && bytes[i]) ? reinterpret_cast<float*>(static_cast<char*>(base) + off) : nullptr;
+        off += (bytes[i] + 255) / 256 * 256;
     }
     w.bytes = off > 0 ? off : 256;   // never 0, which the size query reserves for "unsupported"
     return w;
@@ -741,8 +746,8 @@ cudaError_t dn_bwd_launch(const gla_problem* p, const void* q, const void* k, co
     const T* tk = static_cast<const T*>(k);
     const T* tdo = static_cast<const T*>(dO);
     if (std::is_same<T, __nv_bfloat16>::value) {   // bf16 I/O: the tensor-core walk
-        e = tc::deltanet_walk(p->B, p->H, p->L, DK, p->Dv, p->scale, q, k, v, beta, dO, dhT, w.saved, w.xw, w.drw,
-                              w.dsend, w.db1, dv, dh0, st);
+        e = tc::deltanet_walk(p->B, p->H, p->L, DK, p->Dv, p->scale, q, k, beta, dO, dhT, w.drw, w.dsend, dv, dh0,
+                              st);
     } else {
         GLA_LAUNCH("deltanet_bwd_walk", st,
                    (walk<<<dim3(BH, p->Dv / DN_VT), DN_NT, sw, st>>>(tq, tk, static_cast<const T*>(v), beta, tdo, dhT,
@@ -753,8 +758,8 @@ cudaError_t dn_bwd_launch(const gla_problem* p, const void* q, const void* k, co
     }
     if (e != cudaSuccess) return e;
     if (std::is_same<T, __nv_bfloat16>::value)   // bf16 I/O: the tensor-core gradients
-        return tc::deltanet_grads(p->B, p->H, p->L, DK, p->Dv, p->scale, q, k, beta, dO, w.saved, w.xw, w.drw,
-                                  w.dsend, w.db1, dq, dk, dbeta, st);
+        return tc::deltanet_grads(p->B, p->H, p->L, DK, p->Dv, p->scale, q, k, v, beta, dO, w.saved, w.drw,
+                                  w.dsend, dq, dk, dbeta, st);
     if (NC > 0)
         GLA_LAUNCH("deltanet_bwd_grads", st,
                    (grads<<<dim3(NC, BH), DN_NT, sg, st>>>(tq, tk, beta, tdo, w.saved, w.xw, w.drw, w.dsend, w.db1,

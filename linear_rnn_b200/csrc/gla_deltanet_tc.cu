@@ -67,7 +67,8 @@ struct DtArgs {
     const float* beta;   // [BH*L]
     const float* h0;     // [BH, Dk, Dv] or null
     float* hT;           // [BH, Dk, Dv] or null
-    float* saved;        // [BH, NC, Dk, Dv]: the state entering every chunk, or null
+    __nv_bfloat16* saved;   // [BH, NC, Dk, Dv]: the state entering every chunk (bf16, the precision
+                            // the backward's products read it in), or null
     int* status;         // device status word (a wait that gave up), or null
     int L, Dv;
     float scale;
@@ -88,6 +89,12 @@ __device__ __forceinline__ void dt_store16_bf16(__nv_bfloat16* dst, const float*
     }
     reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
     reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+// 32 values to bf16 in global memory (64 contiguous bytes)
+__device__ __forceinline__ void dt_put_row_bf16(__nv_bfloat16* dst, const float* v) {
+    dt_store16_bf16(dst, v);
+    dt_store16_bf16(dst + 16, v + 16);
 }
 
 // The CTA's [DK, 64] state slice, row `d` (this thread's TMEM lane), 32 columns from `c`: fp32 to
@@ -178,8 +185,7 @@ __global__ void __launch_bounds__(DT_NT, 1)
         if (srow_ok) {
 #pragma unroll
             for (int j = 0; j < 32; j += 8) store8_bf16(sS, sw128_off(srow, c + j, DK * 128), f + j);
-            if (A.saved && nc > 0)
-                dt_put_row(A.saved + (((long)bh * nc) * DK + srow) * Dv + col0 + c, reinterpret_cast<uint32_t*>(f));
+            if (A.saved && nc > 0) dt_put_row_bf16(A.saved + (((long)bh * nc) * DK + srow) * Dv + col0 + c, f);
         }
         tmem_wait_st();
     }
@@ -360,7 +366,8 @@ __global__ void __launch_bounds__(DT_NT, 1)
                 for (int j = 0; j < 32; j += 8)
                     store8_bf16(sS, sw128_off(srow, 32 * wg + j, DK * 128), reinterpret_cast<const float*>(r + j));
                 if (A.saved && c + 1 < nc)
-                    dt_put_row(A.saved + (((long)bh * nc + c + 1) * DK + srow) * Dv + col0 + 32 * wg, r);
+                    dt_put_row_bf16(A.saved + (((long)bh * nc + c + 1) * DK + srow) * Dv + col0 + 32 * wg,
+                                    reinterpret_cast<const float*>(r));
             }
         }
         fence_proxy_async_smem();
@@ -418,43 +425,42 @@ cudaError_t dt_launch(int B, int H, int L, int Dv, const CUtensorMap& mq, const 
 // chunk's end state, a chunk's reverse step is
 //   dX = scale P^T dO + K dS',   dR = T^T dX,   dV = diag(beta) dR,
 //   dS = dS' + scale Q^T dO - K^T diag(beta) dR       (the gradient at the chunk's start).
-// One CTA per (batch*head, 64-column value slice) walks the chunks in reverse with its dS slice in
-// tensor memory. Per chunk:
+// Only dS carries across chunks, and none of it needs S, X or U: those belong to the gradient
+// kernel below, which runs all chunks in parallel. One CTA per (batch*head, 64-column value
+// slice) walks the chunks in reverse with its dS slice in tensor memory. Per chunk:
 //   1. q is scaled in place (so that Q K^T and Q^T dO carry the output scale); tcgen05: K K^T,
-//      Q K^T, K S (S: the chunk's start state from the forward walk, bf16) and K dS';
-//   2. A = diag(beta) strict_lower(K K^T) and its transpose, U and R (fp32), P = lower(Q K^T)
-//      (bf16); tcgen05: dX = K dS' + P^T dO (onto the K dS' accumulator);
-//   3. X = (I + A)^{-1} R (the forward's substitution) -> global for the gradient kernel;
-//   4. dR = (I + A)^{-T} dX: the same substitution backwards, row 63 first;
-//   5. dR and dV = diag(beta) dR to global, the slice's part of sum_j dR U, -diag(beta) dR (bf16);
-//   6. tcgen05: dS += Q^T dO + K^T (-diag(beta) dR); its bf16 copy for the next chunk.
+//      Q K^T, K dS';
+//   2. A^T = strict_lower(diag(beta) K K^T)^T (fp32) and P = lower(Q K^T) (bf16); tcgen05:
+//      dX = K dS' + P^T dO (onto the K dS' accumulator; P read as an MN-major A operand);
+//   3. dR = (I + A)^{-T} dX: a right-looking substitution in fp32 from the last row (thread =
+//      value column x every fourth row, the rows in registers; once row u is final it is
+//      broadcast and A[u][t] dR[u] subtracted from every earlier row t);
+//   4. dR (fp32) and dV = diag(beta) dR to global memory, -diag(beta) dR as a bf16 operand;
+//   5. tcgen05: dS += Q^T dO + K^T (-diag(beta) dR); its bf16 copy for the next chunk, and the
+//      gradient at the next chunk's end (bf16, for the gradient kernel).
 template <int DK>
 struct DwCfg {
-    static constexpr uint32_t KB = TR * DK * 2, QB = TR * DK * 2, VB = TR * DT_VT * 2, OB = TR * DT_VT * 2;
-    static constexpr uint32_t STAGE = KB + QB + VB + OB;
+    static constexpr uint32_t KB = TR * DK * 2, QB = TR * DK * 2, OB = TR * DT_VT * 2;
+    static constexpr uint32_t STAGE = KB + QB + OB;
     static constexpr int NS = 2;
-    static constexpr uint32_t SB = DK * DT_VT * 2;   // bf16 copy of the chunk's start state
     static constexpr uint32_t GB = DK * DT_VT * 2;   // bf16 copy of dS'
     static constexpr uint32_t MB = TR * TR * 2;      // P; -diag(beta) dR
-    static constexpr uint32_t F = TR * DT_TS * 4;    // fp32 tiles: A, A^T, U, W (R, X, dX, dR in turn)
+    static constexpr uint32_t F = TR * DT_TS * 4;    // fp32 tiles: A^T, W (dX, then dR)
     static constexpr uint32_t SMALL = 256 + 4 * TR;
-    static constexpr uint32_t SMEM = NS * STAGE + SB + GB + 2 * MB + 4 * F + SMALL + 1024;
-    static constexpr uint32_t C_S = 0, C_KK = 64, C_KS = 128, NCOL = 256;
+    static constexpr uint32_t SMEM = NS * STAGE + GB + 2 * MB + 2 * F + SMALL + 1024;
+    static constexpr uint32_t C_S = 0, C_KK = 64, C_KD = 128, NCOL = 256;
     static constexpr int MS = DK == 64 ? 64 : 128;
     static_assert(SMEM <= 227 * 1024, "shared memory");
-    static_assert(STAGE % 1024 == 0 && SB % 1024 == 0, "alignment");
+    static_assert(STAGE % 1024 == 0 && GB % 1024 == 0, "alignment");
 };
 
 struct DwArgs {
-    const float* beta;    // [BH*L]
-    const float* saved;   // [BH, NC, Dk, Dv] the state entering every chunk
-    const float* dhT;     // [BH, Dk, Dv] or null
-    float* xw;            // [BH*L, Dv] X
-    float* drw;           // [BH*L, Dv] dR
-    float* dsend;         // [BH, NC, Dk, Dv] the gradient at every chunk's end
-    float* db1;           // [Dv/64, BH*L] the slice's sum_j dR U
-    __nv_bfloat16* dv;    // [BH*L, Dv]
-    float* dh0;           // [BH, Dk, Dv] or null
+    const float* beta;      // [BH*L]
+    const float* dhT;       // [BH, Dk, Dv] or null
+    float* drw;             // [BH*L, Dv] dR
+    __nv_bfloat16* dsend;   // [BH, NC, Dk, Dv] the gradient at every chunk's end
+    __nv_bfloat16* dv;      // [BH*L, Dv]
+    float* dh0;             // [BH, Dk, Dv] or null
     int BH, L, Dv;
     float scale;
 };
@@ -462,18 +468,15 @@ struct DwArgs {
 template <int DK>
 __global__ void __launch_bounds__(DT_NT, 1)
     k_deltanet_tc_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                       const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo, DwArgs A) {
+                       const __grid_constant__ CUtensorMap tdo, DwArgs A) {
     using C = DwCfg<DK>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = smem_align1024(smem_raw);
-    uint8_t* sS = sm + C::NS * C::STAGE;
-    uint8_t* sG = sS + C::SB;
+    uint8_t* sG = sm + C::NS * C::STAGE;
     uint8_t* sP = sG + C::GB;
     uint8_t* sBR = sP + C::MB;
-    float* sA = reinterpret_cast<float*>(sBR + C::MB);
-    float* sAT = sA + TR * DT_TS;
-    float* sU = sAT + TR * DT_TS;
-    float* sW = sU + TR * DT_TS;
+    float* sAT = reinterpret_cast<float*>(sBR + C::MB);
+    float* sW = sAT + TR * DT_TS;
     uint8_t* small = reinterpret_cast<uint8_t*>(sW + TR * DT_TS);
     uint64_t* bar_full = reinterpret_cast<uint64_t*>(small);   // [2]
     uint64_t* bar_mma = bar_full + 2;
@@ -481,7 +484,7 @@ __global__ void __launch_bounds__(DT_NT, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 64);
     float* sB = reinterpret_cast<float*>(small + 256);
 
-    const int bh = blockIdx.x, slice = blockIdx.y, col0 = slice * DT_VT;
+    const int bh = blockIdx.x, col0 = blockIdx.y * DT_VT;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2, qd = warp & 3;
     const int L = A.L, Dv = A.Dv;
     const int nc = (L + TR - 1) / TR;
@@ -490,10 +493,8 @@ __global__ void __launch_bounds__(DT_NT, 1)
     const int srow = DK == 64 ? 16 * qd + (lane & 15) : 32 * qd + lane;
     const int mrow = 16 * qd + (lane & 15);
     const bool first = lane < 16;
-    // substitution mapping: value column j, rows 4 m + sp
-    const int sj = warp * 8 + (lane >> 2), sp = lane & 3;
-    // row-pass mapping: row rt, columns rc .. rc + 15
-    const int rt = tid >> 2, rc = 16 * (tid & 3);
+    const int sj = warp * 8 + (lane >> 2), sp = lane & 3;   // substitution: value column, row phase
+    const int rt = tid >> 2, rc = 16 * (tid & 3);           // row pass: token row, 16 value columns
 
     if (tid == 0) {
         mbar_init(&bar_full[0], 1);
@@ -518,8 +519,7 @@ __global__ void __launch_bounds__(DT_NT, 1)
             tma_load_3d(st + cb * BLK, &tk, cb * 64, t0, bh, &bar_full[s]);
             tma_load_3d(st + C::KB + cb * BLK, &tq, cb * 64, t0, bh, &bar_full[s]);
         }
-        tma_load_3d(st + C::KB + C::QB, &tv, col0, t0, bh, &bar_full[s]);
-        tma_load_3d(st + C::KB + C::QB + C::VB, &tdo, col0, t0, bh, &bar_full[s]);
+        tma_load_3d(st + C::KB + C::QB, &tdo, col0, t0, bh, &bar_full[s]);
     };
     if (tid == 0)
         for (int i = 0; i < C::NS && i < nc; ++i) issue_loads(i, i);
@@ -555,27 +555,15 @@ __global__ void __launch_bounds__(DT_NT, 1)
         const int s = i % C::NS, ci = chunk_at(i), t0 = ci * TR;
         uint8_t* sk = sm + s * C::STAGE;
         uint8_t* sq = sk + C::KB;
-        uint8_t* sv = sq + C::QB;
-        uint8_t* sdo = sv + C::VB;
+        uint8_t* sdo = sq + C::QB;
         const long cbase = (long)bh * nc + ci;
         if (tid < TR) sB[tid] = t0 + tid < L ? A.beta[rowbase + t0 + tid] : 0.f;
-        // the gradient at this chunk's end, and the chunk's start state as a bf16 operand
-        {
-            uint32_t r[32];
-            tmem_ld32(tq_lane + C::C_S + 32 * wg, r);
-            tmem_wait_ld();
-            if (srow_ok) {
-                dt_put_row(A.dsend + (cbase * DK + srow) * Dv + col0 + 32 * wg, r);
-                const float* src = A.saved + (cbase * DK + srow) * Dv + col0 + 32 * wg;
-                float f[32];
+        // the gradient at this chunk's end, for the gradient kernel (its bf16 copy is in sG)
+        if (srow_ok) {
 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const float4 x = __ldg(reinterpret_cast<const float4*>(src + j));
-                    f[j] = x.x; f[j + 1] = x.y; f[j + 2] = x.z; f[j + 3] = x.w;
-                }
-#pragma unroll
-                for (int j = 0; j < 32; j += 8) store8_bf16(sS, sw128_off(srow, 32 * wg + j, DK * 128), f + j);
-            }
+            for (int j = 0; j < 32; j += 8)
+                *reinterpret_cast<uint4*>(A.dsend + (cbase * DK + srow) * Dv + col0 + 32 * wg + j) =
+                    *reinterpret_cast<const uint4*>(sG + sw128_off(srow, 32 * wg + j, DK * 128));
         }
         if (!dt_wait(&bar_full[s], (i / C::NS) & 1)) { err = 1; break; }
         // q scaled in place (bf16, layout-blind 16-byte chunks)
@@ -595,12 +583,12 @@ __global__ void __launch_bounds__(DT_NT, 1)
         __syncthreads();
         tc_fence_after();
 
-        // ---- 1. K K^T | Q K^T, K S | K dS'
+        // ---- 1. K K^T | Q K^T, K dS'
         if (warp == 0) {
             const bool leader = elect_one();
             const uint32_t ka = smem_u32(sk), qa = smem_u32(sq);
             const uint32_t idAA = idesc_bf16(64, 64, 0, 0), idAS = idesc_bf16(64, DT_VT, 0, 1);
-            const uint64_t dS = sw128_desc(smem_u32(sS), DK * 128, 1024), dG = sw128_desc(smem_u32(sG), DK * 128, 1024);
+            const uint64_t dG = sw128_desc(smem_u32(sG), DK * 128, 1024);
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
@@ -609,9 +597,7 @@ __global__ void __launch_bounds__(DT_NT, 1)
                              kk > 0);
                     mma_bf16(tbase + C::C_KK + (16u << 16), sw128_desc(qa + koff, 16, 1024),
                              sw128_desc(ka + koff, 16, 1024), idAA, kk > 0);
-                    mma_bf16(tbase + C::C_KS, sw128_desc(ka + koff, 16, 1024), dS + ((kk * 2048) >> 4), idAS, kk > 0);
-                    mma_bf16(tbase + C::C_KS + (16u << 16), sw128_desc(ka + koff, 16, 1024), dG + ((kk * 2048) >> 4),
-                             idAS, kk > 0);
+                    mma_bf16(tbase + C::C_KD, sw128_desc(ka + koff, 16, 1024), dG + ((kk * 2048) >> 4), idAS, kk > 0);
                 }
             }
             if (leader) mma_commit(bar_mma);
@@ -621,7 +607,7 @@ __global__ void __launch_bounds__(DT_NT, 1)
         if (!dt_wait(bar_mma, (n_mma - 1) & 1)) { err = 1; break; }
         tc_fence_after();
 
-        // ---- 2. A and A^T (fp32), P (bf16); U and R (fp32)
+        // ---- 2. A^T (fp32) and P (bf16); dX = K dS' + P^T dO
         {
             uint32_t r[32];
             tmem_ld32(tq_lane + C::C_KK + 32 * wg, r);
@@ -630,14 +616,9 @@ __global__ void __launch_bounds__(DT_NT, 1)
             if (first) {
                 const float bt = sB[t];
 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
+                for (int j = 0; j < 32; ++j) {
                     const int sc = 32 * wg + j;
-                    float a4[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) a4[u] = sc + u < t ? bt * __uint_as_float(r[j + u]) : 0.f;
-                    *reinterpret_cast<float4*>(sA + t * DT_TS + sc) = make_float4(a4[0], a4[1], a4[2], a4[3]);
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) sAT[(sc + u) * DT_TS + t] = a4[u];
+                    sAT[sc * DT_TS + t] = sc < t ? bt * __uint_as_float(r[j]) : 0.f;
                 }
             } else {
 #pragma unroll
@@ -652,90 +633,28 @@ __global__ void __launch_bounds__(DT_NT, 1)
                 }
             }
         }
-        {
-            uint32_t r[32];
-            tmem_ld32(tq_lane + C::C_KS + 32 * wg, r);
-            tmem_wait_ld();
-            if (first) {
-                const int t = mrow;
-                const float bt = sB[t];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int cc = 32 * wg + 8 * u;
-                    const uint4 vw = *reinterpret_cast<const uint4*>(sv + sw128_off(t, cc, BLK));
-                    const uint32_t* vp = reinterpret_cast<const uint32_t*>(&vw);
-                    float uu[8];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float2 vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vp[j]));
-                        uu[2 * j] = vf.x - __uint_as_float(r[8 * u + 2 * j]);
-                        uu[2 * j + 1] = vf.y - __uint_as_float(r[8 * u + 2 * j + 1]);
-                    }
-                    *reinterpret_cast<float4*>(sU + t * DT_TS + cc) = make_float4(uu[0], uu[1], uu[2], uu[3]);
-                    *reinterpret_cast<float4*>(sU + t * DT_TS + cc + 4) = make_float4(uu[4], uu[5], uu[6], uu[7]);
-                    *reinterpret_cast<float4*>(sW + t * DT_TS + cc) =
-                        make_float4(bt * uu[0], bt * uu[1], bt * uu[2], bt * uu[3]);
-                    *reinterpret_cast<float4*>(sW + t * DT_TS + cc + 4) =
-                        make_float4(bt * uu[4], bt * uu[5], bt * uu[6], bt * uu[7]);
-                }
-            }
-        }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        // dX = K dS' + P^T dO (P^T: the P tile read as an MN-major A operand)
         if (warp == 0) {
             const bool leader = elect_one();
             const uint32_t idX = idesc_bf16(64, DT_VT, 1, 1);
             const uint64_t dPt = sw128_desc(smem_u32(sP), BLK, 1024), dO = sw128_desc(smem_u32(sdo), BLK, 1024);
 #pragma unroll
             for (int ks = 0; ks < TR / 16; ++ks)
-                if (leader)
-                    mma_bf16(tbase + C::C_KS + (16u << 16), dPt + ((ks * 2048) >> 4), dO + ((ks * 2048) >> 4), idX, 1);
+                if (leader) mma_bf16(tbase + C::C_KD, dPt + ((ks * 2048) >> 4), dO + ((ks * 2048) >> 4), idX, 1);
             if (leader) mma_commit(bar_mma);
             __syncwarp();
         }
         ++n_mma;
-
-        // ---- 3. X = (I + A)^{-1} R, as in the forward
-        {
-            float x[16];
-#pragma unroll
-            for (int m = 0; m < 16; ++m) x[m] = sW[(4 * m + sp) * DT_TS + sj];
-#pragma unroll
-            for (int t4 = 0; t4 < TR; t4 += 4) {
-                float4 a[16];
-#pragma unroll
-                for (int m = t4 / 4; m < 16; ++m) a[m] = *reinterpret_cast<const float4*>(sA + (4 * m + sp) * DT_TS + t4);
-#pragma unroll
-                for (int tt = 0; tt < 4; ++tt) {
-                    const int t = t4 + tt;
-                    const float xt = __shfl_sync(0xffffffffu, x[t >> 2], (lane & ~3) | (t & 3));
-#pragma unroll
-                    for (int m = t4 / 4; m < 16; ++m) {
-                        const float at = tt == 0 ? a[m].x : tt == 1 ? a[m].y : tt == 2 ? a[m].z : a[m].w;
-                        if (4 * m + sp > t) x[m] = fmaf(-at, xt, x[m]);
-                    }
-                }
-            }
-            __syncthreads();   // every thread has read its R
-#pragma unroll
-            for (int m = 0; m < 16; ++m) sW[(4 * m + sp) * DT_TS + sj] = x[m];
-        }
-        __syncthreads();
-        if (t0 + rt < L) {
-            float* dst = A.xw + (rowbase + t0 + rt) * Dv + col0 + rc;
-#pragma unroll
-            for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(dst + j) = *reinterpret_cast<const float4*>(sW + rt * DT_TS + rc + j);
-        }
-        if (!dt_wait(bar_mma, (n_mma - 1) & 1)) { err = 1; break; }   // dX (and X's readers above)
+        if (!dt_wait(bar_mma, (n_mma - 1) & 1)) { err = 1; break; }
         tc_fence_after();
         {
             uint32_t r[32];
-            tmem_ld32(tq_lane + C::C_KS + 32 * wg, r);
+            tmem_ld32(tq_lane + C::C_KD + 32 * wg, r);
             tmem_wait_ld();
-            if (!first)
+            if (first)
 #pragma unroll
                 for (int j = 0; j < 32; j += 4)
                     *reinterpret_cast<float4*>(sW + mrow * DT_TS + 32 * wg + j) =
@@ -744,8 +663,7 @@ __global__ void __launch_bounds__(DT_NT, 1)
         }
         __syncthreads();
 
-        // ---- 4. dR = (I + A)^{-T} dX: rows from the last, dR[u] subtracted (A[u][t] dR[u]) from
-        //      every earlier row t; A^T read four columns at a time
+        // ---- 3. dR = (I + A)^{-T} dX, rows from the last; A^T read four columns at a time
         {
             float x[16];
 #pragma unroll
@@ -772,19 +690,15 @@ __global__ void __launch_bounds__(DT_NT, 1)
         }
         __syncthreads();
 
-        // ---- 5. dR, dV = diag(beta) dR, the slice's part of sum_j dR U, and -diag(beta) dR (bf16)
+        // ---- 4. dR and dV = diag(beta) dR to global memory, -diag(beta) dR (bf16)
         {
             const float bt = sB[rt];
-            float dr[16], acc = 0.f;
+            float dr[16];
 #pragma unroll
             for (int j = 0; j < 16; j += 4) {
                 const float4 x = *reinterpret_cast<const float4*>(sW + rt * DT_TS + rc + j);
-                const float4 u4 = *reinterpret_cast<const float4*>(sU + rt * DT_TS + rc + j);
                 dr[j] = x.x; dr[j + 1] = x.y; dr[j + 2] = x.z; dr[j + 3] = x.w;
-                acc += x.x * u4.x + x.y * u4.y + x.z * u4.z + x.w * u4.w;
             }
-            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
             if (t0 + rt < L) {
                 const long row = rowbase + t0 + rt;
                 float* dst = A.drw + row * Dv + col0 + rc;
@@ -794,7 +708,6 @@ __global__ void __launch_bounds__(DT_NT, 1)
 #pragma unroll
                 for (int j = 0; j < 16; ++j) bv[j] = bt * dr[j];
                 dt_store16_bf16(A.dv + row * Dv + col0 + rc, bv);
-                if ((tid & 3) == 0) A.db1[(long)slice * A.BH * L + row] = acc;
             }
             float nb[16];
 #pragma unroll
@@ -807,7 +720,7 @@ __global__ void __launch_bounds__(DT_NT, 1)
         __syncthreads();
         tc_fence_after();
 
-        // ---- 6. dS += Q^T dO + K^T (-diag(beta) dR)
+        // ---- 5. dS += Q^T dO + K^T (-diag(beta) dR)
         if (warp == 0) {
             const bool leader = elect_one();
             const uint32_t idS = idesc_bf16(C::MS, DT_VT, 1, 1);
@@ -863,47 +776,52 @@ __global__ void __launch_bounds__(DT_NT, 1)
 }
 
 template <int DK>
-cudaError_t dw_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
-                      const DwArgs& a, cudaStream_t st) {
+cudaError_t dw_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mdo, const DwArgs& a,
+                      cudaStream_t st) {
     auto kern = k_deltanet_tc_walk<DK>;
     const uint32_t smem = DwCfg<DK>::SMEM;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const dim3 grid(a.BH, a.Dv / DT_VT);
-    GLA_LAUNCH("deltanet_bwd_walk", st, (kern<<<grid, DT_NT, smem, st>>>(mq, mk, mv, mdo, a)));
+    GLA_LAUNCH("deltanet_bwd_walk", st, (kern<<<grid, DT_NT, smem, st>>>(mq, mk, mdo, a)));
     return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ backward gradients
-// Per chunk, all chunks in parallel, from the walk's X, dR, the chunk's start state S and end
-// gradient dS' (value columns in 64-wide slices, summed in tensor memory):
+// Per chunk, all chunks in parallel, from the chunk's start state S (saved by the forward's state
+// walk, bf16), the gradient at its end dS' and dR (both from the reverse walk), value columns in
+// 64-wide slices summed in tensor memory:
+//   A = strict_lower(diag(beta) K K^T),  U = V - K S,  X = (I + A)^{-1} diag(beta) U
 //   dP = scale lower(dO X^T),  G = -strict_lower(dR X^T)
 //   dQ = scale dO S^T + dP K
 //   dK = X dS'^T - diag(beta) dR S^T + dP^T Q + diag(beta) (G K) + G^T diag(beta) K
-//   dbeta_t = sum_j dR_tj U_tj (the walk's slice sums) + sum_i k_ti (G K)_ti
+//   dbeta_t = sum_j dR_tj U_tj + sum_i k_ti (G K)_ti
 // One CTA per (chunk, batch*head). dO is scaled in place, so dO X^T and dO S^T carry the scale.
+// X comes from the forward's substitution (fp32, rows in registers), once per value slice.
 template <int DK>
 struct DgCfg {
-    static constexpr uint32_t KB = TR * DK * 2;   // K, Q tiles (TMA)
-    static constexpr uint32_t MB = TR * TR * 2;   // 64 x 64 bf16: dO, X, dR, -diag(beta) dR, dP, G
-    static constexpr uint32_t SB = DK * DT_VT * 2;   // S and dS' slices, bf16, K-major rows of key dims
-    static constexpr uint32_t SMALL = 256 + 4 * TR + 8 * TR;
-    static constexpr uint32_t SMEM = 3 * KB + 6 * MB + 2 * SB + SMALL + 1024;
-    // TMEM: dO X^T | dR X^T (lanes 0-15 | 16-31) at 0; dQ | dK at 64; G K (lanes 16-31) at 64 + DK
-    static constexpr uint32_t C_PG = 0, C_QK = 64, C_GK = 64 + DK, NCOL = 64 + 2 * DK <= 256 ? 256 : 512;
+    static constexpr uint32_t KB = TR * DK * 2;      // K, Q (TMA), diag(beta) K
+    static constexpr uint32_t MB = TR * TR * 2;      // 64 x 64 bf16: dO, V, X, dR, -diag(beta) dR, dP, G
+    static constexpr uint32_t SB = DK * DT_VT * 2;   // S and dS' slices, bf16, rows of key dims
+    static constexpr uint32_t F = TR * DT_TS * 4;    // fp32: A, U, R (then X)
+    static constexpr uint32_t SMALL = 256 + 4 * TR + 8 * TR + 4 * TR;
+    static constexpr uint32_t SMEM = 3 * KB + 7 * MB + 2 * SB + 3 * F + SMALL + 1024;
+    // TMEM: dO X^T | dR X^T (lanes 0-15 | 16-31) at 0; dQ | dK at 64; G K (lanes 16-31) at
+    // 64 + DK; K K^T at 64 + 2 DK; K S at 128 + 2 DK
+    static constexpr uint32_t C_PG = 0, C_QK = 64, C_GK = 64 + DK, C_KK = 64 + 2 * DK, C_KS = 128 + 2 * DK;
+    static constexpr uint32_t NCOL = 512;
+    static_assert(C_KS + 64 <= NCOL, "tensor memory");
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
 struct DgArgs {
-    const float* beta;    // [BH*L]
-    const float* saved;   // [BH, NC, Dk, Dv]
-    const float* xw;      // [BH*L, Dv]
-    const float* drw;     // [BH*L, Dv]
-    const float* dsend;   // [BH, NC, Dk, Dv]
-    const float* db1;     // [Dv/64, BH*L]
-    __nv_bfloat16* dq;    // [BH*L, Dk]
+    const float* beta;            // [BH*L]
+    const __nv_bfloat16* saved;   // [BH, NC, Dk, Dv] the state entering every chunk
+    const float* drw;             // [BH*L, Dv]
+    const __nv_bfloat16* dsend;   // [BH, NC, Dk, Dv] the gradient at every chunk's end
+    __nv_bfloat16* dq;            // [BH*L, Dk]
     __nv_bfloat16* dk;
-    float* dbeta;         // [BH*L]
+    float* dbeta;                 // [BH*L]
     int BH, L, Dv;
     float scale;
 };
@@ -911,7 +829,7 @@ struct DgArgs {
 template <int DK>
 __global__ void __launch_bounds__(DT_NT, 1)
     k_deltanet_tc_grads(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                        const __grid_constant__ CUtensorMap tdo, DgArgs A) {
+                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo, DgArgs A) {
     using C = DgCfg<DK>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = smem_align1024(smem_raw);
@@ -919,14 +837,18 @@ __global__ void __launch_bounds__(DT_NT, 1)
     uint8_t* sQ = sK + C::KB;
     uint8_t* sBK = sQ + C::KB;      // diag(beta) K
     uint8_t* sDO = sBK + C::KB;
-    uint8_t* sX = sDO + C::MB;
+    uint8_t* sV = sDO + C::MB;
+    uint8_t* sX = sV + C::MB;
     uint8_t* sDR = sX + C::MB;
     uint8_t* sNB = sDR + C::MB;     // -diag(beta) dR
     uint8_t* sDP = sNB + C::MB;
     uint8_t* sGm = sDP + C::MB;
     uint8_t* sSb = sGm + C::MB;
     uint8_t* sDS = sSb + C::SB;
-    uint8_t* small = sDS + C::SB;
+    float* sAf = reinterpret_cast<float*>(sDS + C::SB);
+    float* sU = sAf + TR * DT_TS;
+    float* sRf = sU + TR * DT_TS;
+    uint8_t* small = reinterpret_cast<uint8_t*>(sRf + TR * DT_TS);
     uint64_t* bar_kq = reinterpret_cast<uint64_t*>(small);
     uint64_t* bar_do = bar_kq + 1;
     uint64_t* bar_mma = bar_kq + 2;
@@ -934,6 +856,7 @@ __global__ void __launch_bounds__(DT_NT, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(small + 64);
     float* sB = reinterpret_cast<float*>(small + 256);      // beta [64]
     float* sDB = sB + TR;                                   // [2][64] partial sums of k . (G K)
+    float* sDU = sDB + 2 * TR;                              // [64] sum_j dR U over the slices
 
     const int ci = blockIdx.x, bh = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2, qd = warp & 3;
@@ -943,7 +866,8 @@ __global__ void __launch_bounds__(DT_NT, 1)
     const long cbase = (long)bh * nc + ci;
     const int mrow = 16 * qd + (lane & 15);
     const bool first = lane < 16;
-    const int rt = tid >> 2, rc = 16 * (tid & 3);   // row pass: token row, 16 value columns
+    const int rt = tid >> 2, rc = 16 * (tid & 3);           // row pass: token row, 16 value columns
+    const int sj = warp * 8 + (lane >> 2), sp = lane & 3;   // substitution: value column, row phase
 
     if (tid == 0) {
         mbar_init(bar_kq, 1);
@@ -965,54 +889,66 @@ __global__ void __launch_bounds__(DT_NT, 1)
             tma_load_3d(sQ + cb * BLK, &tq, cb * 64, t0, bh, bar_kq);
         }
     }
-    if (tid < TR) sB[tid] = t0 + tid < L ? A.beta[rowbase + t0 + tid] : 0.f;
-    __syncthreads();   // beta is read by every row pass below
-
+    if (tid < TR) {
+        sB[tid] = t0 + tid < L ? A.beta[rowbase + t0 + tid] : 0.f;
+        sDU[tid] = 0.f;
+    }
     int err = 0, n_mma = 0, n_do = 0;
+    // ---- K K^T, then A (fp32)
+    if (!dt_wait(bar_kq, 0)) err = 1;
+    if (!err) {
+        if (warp == 0) {
+            const bool leader = elect_one();
+            tc_fence_after();
+            const uint32_t ka = smem_u32(sK);
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+                if (leader)
+                    mma_bf16(tbase + C::C_KK, sw128_desc(ka + koff, 16, 1024), sw128_desc(ka + koff, 16, 1024),
+                             idesc_bf16(64, 64, 0, 0), kk > 0);
+            }
+            if (leader) mma_commit(bar_mma);
+            __syncwarp();
+        }
+        ++n_mma;
+        if (!dt_wait(bar_mma, (n_mma - 1) & 1)) err = 1;
+    }
+    if (!err) {
+        tc_fence_after();
+        uint32_t r[32];
+        tmem_ld32(tq_lane + C::C_KK + 32 * wg, r);
+        tmem_wait_ld();
+        if (first) {
+            const int t = mrow;
+            const float bt = sB[t];
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                const int sc = 32 * wg + j;
+                *reinterpret_cast<float4*>(sAf + t * DT_TS + sc) =
+                    make_float4(sc < t ? bt * __uint_as_float(r[j]) : 0.f, sc + 1 < t ? bt * __uint_as_float(r[j + 1]) : 0.f,
+                                sc + 2 < t ? bt * __uint_as_float(r[j + 2]) : 0.f,
+                                sc + 3 < t ? bt * __uint_as_float(r[j + 3]) : 0.f);
+            }
+        }
+    }
+
     for (int sl = 0; sl < nsl && !err; ++sl) {
         const int col0 = sl * DT_VT;
         if (tid == 0) {
-            mbar_arrive_expect_tx(bar_do, C::MB);
+            mbar_arrive_expect_tx(bar_do, 2 * C::MB);
             tma_load_3d(sDO, &tdo, col0, t0, bh, bar_do);
+            tma_load_3d(sV, &tv, col0, t0, bh, bar_do);
         }
-        // X, dR and -diag(beta) dR (bf16, rows of tokens); S and dS' (bf16, rows of key dims)
-        {
-            const bool in = t0 + rt < L;
-            const long off = (rowbase + t0 + rt) * Dv + col0 + rc;
-            const float bt = sB[rt];
-            float x[16], d[16], nb[16];
-#pragma unroll
-            for (int j = 0; j < 16; j += 4) {
-                const float4 a = in ? __ldg(reinterpret_cast<const float4*>(A.xw + off + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
-                const float4 b = in ? __ldg(reinterpret_cast<const float4*>(A.drw + off + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
-                x[j] = a.x; x[j + 1] = a.y; x[j + 2] = a.z; x[j + 3] = a.w;
-                d[j] = b.x; d[j + 1] = b.y; d[j + 2] = b.z; d[j + 3] = b.w;
-            }
-#pragma unroll
-            for (int j = 0; j < 16; ++j) nb[j] = -bt * d[j];
-            store8_bf16(sX, sw128_off(rt, rc, BLK), x);
-            store8_bf16(sX, sw128_off(rt, rc + 8, BLK), x + 8);
-            store8_bf16(sDR, sw128_off(rt, rc, BLK), d);
-            store8_bf16(sDR, sw128_off(rt, rc + 8, BLK), d + 8);
-            store8_bf16(sNB, sw128_off(rt, rc, BLK), nb);
-            store8_bf16(sNB, sw128_off(rt, rc + 8, BLK), nb + 8);
-        }
+        // S and dS' slices (bf16, rows of key dims), copied as they are
         {
             constexpr int TPR = DT_NT / DK, CPT = DT_VT / TPR;   // threads per key row, columns per thread
             const int kr = tid / TPR, kc = (tid % TPR) * CPT;
             const long off = (cbase * DK + kr) * Dv + col0 + kc;
 #pragma unroll
             for (int j = 0; j < CPT; j += 8) {
-                float s8[8], g8[8];
-#pragma unroll
-                for (int u = 0; u < 8; u += 4) {
-                    const float4 a = __ldg(reinterpret_cast<const float4*>(A.saved + off + j + u));
-                    const float4 b = __ldg(reinterpret_cast<const float4*>(A.dsend + off + j + u));
-                    s8[u] = a.x; s8[u + 1] = a.y; s8[u + 2] = a.z; s8[u + 3] = a.w;
-                    g8[u] = b.x; g8[u + 1] = b.y; g8[u + 2] = b.z; g8[u + 3] = b.w;
-                }
-                store8_bf16(sSb, sw128_off(kr, kc + j, BLK), s8);
-                store8_bf16(sDS, sw128_off(kr, kc + j, BLK), g8);
+                *reinterpret_cast<uint4*>(sSb + sw128_off(kr, kc + j, BLK)) = __ldg(reinterpret_cast<const uint4*>(A.saved + off + j));
+                *reinterpret_cast<uint4*>(sDS + sw128_off(kr, kc + j, BLK)) = __ldg(reinterpret_cast<const uint4*>(A.dsend + off + j));
             }
         }
         ++n_do;
@@ -1028,6 +964,105 @@ __global__ void __launch_bounds__(DT_NT, 1)
                 pw[u] = *reinterpret_cast<uint32_t*>(&h);
             }
             *reinterpret_cast<uint4*>(sDO + 16 * e) = w;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // K S (the slice's S as an MN-major B operand)
+        if (warp == 0) {
+            const bool leader = elect_one();
+            const uint32_t ka = smem_u32(sK);
+            const uint64_t dS = sw128_desc(smem_u32(sSb), DK * 128, 1024);
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+                if (leader)
+                    mma_bf16(tbase + C::C_KS, sw128_desc(ka + koff, 16, 1024), dS + ((kk * 2048) >> 4),
+                             idesc_bf16(64, DT_VT, 0, 1), kk > 0);
+            }
+            if (leader) mma_commit(bar_mma);
+            __syncwarp();
+        }
+        ++n_mma;
+        if (!dt_wait(bar_mma, (n_mma - 1) & 1)) { err = 1; break; }
+        tc_fence_after();
+        // U = V - K S and R = diag(beta) U (fp32)
+        {
+            uint32_t r[32];
+            tmem_ld32(tq_lane + C::C_KS + 32 * wg, r);
+            tmem_wait_ld();
+            if (first) {
+                const int t = mrow;
+                const float bt = sB[t];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int cc = 32 * wg + 8 * u;
+                    const uint4 vw = *reinterpret_cast<const uint4*>(sV + sw128_off(t, cc, BLK));
+                    const uint32_t* vp = reinterpret_cast<const uint32_t*>(&vw);
+                    float uu[8];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vp[j]));
+                        uu[2 * j] = vf.x - __uint_as_float(r[8 * u + 2 * j]);
+                        uu[2 * j + 1] = vf.y - __uint_as_float(r[8 * u + 2 * j + 1]);
+                    }
+                    *reinterpret_cast<float4*>(sU + t * DT_TS + cc) = make_float4(uu[0], uu[1], uu[2], uu[3]);
+                    *reinterpret_cast<float4*>(sU + t * DT_TS + cc + 4) = make_float4(uu[4], uu[5], uu[6], uu[7]);
+                    *reinterpret_cast<float4*>(sRf + t * DT_TS + cc) = make_float4(bt * uu[0], bt * uu[1], bt * uu[2], bt * uu[3]);
+                    *reinterpret_cast<float4*>(sRf + t * DT_TS + cc + 4) =
+                        make_float4(bt * uu[4], bt * uu[5], bt * uu[6], bt * uu[7]);
+                }
+            }
+        }
+        __syncthreads();
+        // dR (fp32 from the walk): its bf16 operands, and sum_j dR U
+        {
+            const bool in = t0 + rt < L;
+            const long off = (rowbase + t0 + rt) * Dv + col0 + rc;
+            const float bt = sB[rt];
+            float d[16], nb[16], acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) {
+                const float4 b = in ? __ldg(reinterpret_cast<const float4*>(A.drw + off + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float4 u4 = *reinterpret_cast<const float4*>(sU + rt * DT_TS + rc + j);
+                d[j] = b.x; d[j + 1] = b.y; d[j + 2] = b.z; d[j + 3] = b.w;
+                acc += b.x * u4.x + b.y * u4.y + b.z * u4.z + b.w * u4.w;
+            }
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            if ((tid & 3) == 0) sDU[rt] += acc;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) nb[j] = -bt * d[j];
+            store8_bf16(sDR, sw128_off(rt, rc, BLK), d);
+            store8_bf16(sDR, sw128_off(rt, rc + 8, BLK), d + 8);
+            store8_bf16(sNB, sw128_off(rt, rc, BLK), nb);
+            store8_bf16(sNB, sw128_off(rt, rc + 8, BLK), nb + 8);
+        }
+        // X = (I + A)^{-1} R, as in the forward; X to bf16
+        {
+            float x[16];
+#pragma unroll
+            for (int m = 0; m < 16; ++m) x[m] = sRf[(4 * m + sp) * DT_TS + sj];
+#pragma unroll
+            for (int t4 = 0; t4 < TR; t4 += 4) {
+                float4 a[16];
+#pragma unroll
+                for (int m = t4 / 4; m < 16; ++m) a[m] = *reinterpret_cast<const float4*>(sAf + (4 * m + sp) * DT_TS + t4);
+#pragma unroll
+                for (int tt = 0; tt < 4; ++tt) {
+                    const int t = t4 + tt;
+                    const float xt = __shfl_sync(0xffffffffu, x[t >> 2], (lane & ~3) | (t & 3));
+#pragma unroll
+                    for (int m = t4 / 4; m < 16; ++m) {
+                        const float at = tt == 0 ? a[m].x : tt == 1 ? a[m].y : tt == 2 ? a[m].z : a[m].w;
+                        if (4 * m + sp > t) x[m] = fmaf(-at, xt, x[m]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < 16; ++m)
+                *reinterpret_cast<__nv_bfloat16*>(sX + sw128_off(4 * m + sp, sj, BLK)) = __float2bfloat16_rn(x[m]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -1060,7 +1095,7 @@ __global__ void __launch_bounds__(DT_NT, 1)
         if (!dt_wait(bar_mma, (n_mma - 1) & 1)) { err = 1; break; }   // the slice's tiles may be rewritten
         tc_fence_after();
     }
-    if (!err && !dt_wait(bar_kq, 0)) err = 1;
+
     if (!err) {
         // dP = lower(dO X^T) (bf16; the scale came with dO) and G = -strict_lower(dR X^T); diag(beta) K
         {
@@ -1168,7 +1203,7 @@ __global__ void __launch_bounds__(DT_NT, 1)
         __syncthreads();
         if (tid < TR && t0 + tid < L) {
             float x = sDB[tid] + sDB[TR + tid];
-            for (int s2 = 0; s2 < nsl; ++s2) x += A.db1[(long)s2 * A.BH * L + rowbase + t0 + tid];
+            x += sDU[tid];
             A.dbeta[rowbase + t0 + tid] = x;
         }
     }
@@ -1188,20 +1223,20 @@ __global__ void __launch_bounds__(DT_NT, 1)
 }
 
 template <int DK>
-cudaError_t dg_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mdo, const DgArgs& a,
-                      int nc, cudaStream_t st) {
+cudaError_t dg_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                      const DgArgs& a, int nc, cudaStream_t st) {
     auto kern = k_deltanet_tc_grads<DK>;
     const uint32_t smem = DgCfg<DK>::SMEM;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    GLA_LAUNCH("deltanet_bwd_grads", st, (kern<<<dim3(nc, a.BH), DT_NT, smem, st>>>(mq, mk, mdo, a)));
+    GLA_LAUNCH("deltanet_bwd_grads", st, (kern<<<dim3(nc, a.BH), DT_NT, smem, st>>>(mq, mk, mv, mdo, a)));
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t deltanet_fwd(int B, int H, int L, int Dk, int Dv, float scale, const void* q, const void* k,
-                         const void* v, const float* beta, const float* h0, void* o, float* hT, float* saved,
+                         const void* v, const float* beta, const float* h0, void* o, float* hT, void* saved,
                          int* status, cudaStream_t st) {
     const int BH = B * H;
     if (BH == 0) return cudaSuccess;
@@ -1229,7 +1264,7 @@ cudaError_t deltanet_fwd(int B, int H, int L, int Dk, int Dv, float scale, const
     a.beta = beta;
     a.h0 = h0;
     a.hT = hT;
-    a.saved = saved;
+    a.saved = static_cast<__nv_bfloat16*>(saved);
     a.status = status;
     a.L = L;
     a.Dv = Dv;
@@ -1243,8 +1278,8 @@ cudaError_t deltanet_fwd(int B, int H, int L, int Dk, int Dv, float scale, const
 
 
 cudaError_t deltanet_walk(int B, int H, int L, int Dk, int Dv, float scale, const void* q, const void* k,
-                          const void* v, const float* beta, const void* dO, const float* dhT, const float* saved,
-                          float* xw, float* drw, float* dsend, float* db1, void* dv, float* dh0, cudaStream_t st) {
+                          const float* beta, const void* dO, const float* dhT, float* drw, void* dsend, void* dv,
+                          float* dh0, cudaStream_t st) {
     const int BH = B * H;
     if (BH == 0) return cudaSuccess;
     if (L == 0) {   // no chunk: dh0 = dhT (or zero)
@@ -1254,46 +1289,41 @@ cudaError_t deltanet_walk(int B, int H, int L, int Dk, int Dv, float scale, cons
         }
         return cudaSuccess;
     }
-    CUtensorMap mq, mk, mv, mdo;
+    CUtensorMap mq, mk, mdo;
     if (!make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dk, L, BH, 64, true) ||
         !make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dk, L, BH, 64, true) ||
-        !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dv, L, BH, 64, true) ||
         !make_map(&mdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dv, L, BH, 64, true))
         return cudaErrorInvalidValue;
     DwArgs a{};
     a.beta = beta;
-    a.saved = saved;
     a.dhT = dhT;
-    a.xw = xw;
     a.drw = drw;
-    a.dsend = dsend;
-    a.db1 = db1;
+    a.dsend = static_cast<__nv_bfloat16*>(dsend);
     a.dv = static_cast<__nv_bfloat16*>(dv);
     a.dh0 = dh0;
     a.BH = BH;
     a.L = L;
     a.Dv = Dv;
     a.scale = scale;
-    return Dk == 64 ? dw_launch<64>(mq, mk, mv, mdo, a, st) : dw_launch<128>(mq, mk, mv, mdo, a, st);
+    return Dk == 64 ? dw_launch<64>(mq, mk, mdo, a, st) : dw_launch<128>(mq, mk, mdo, a, st);
 }
 
 cudaError_t deltanet_grads(int B, int H, int L, int Dk, int Dv, float scale, const void* q, const void* k,
-                           const float* beta, const void* dO, const float* saved, const float* xw, const float* drw,
-                           const float* dsend, const float* db1, void* dq, void* dk, float* dbeta, cudaStream_t st) {
+                           const void* v, const float* beta, const void* dO, const void* saved, const float* drw,
+                           const void* dsend, void* dq, void* dk, float* dbeta, cudaStream_t st) {
     const int BH = B * H, nc = (L + TR - 1) / TR;
     if (BH == 0 || nc == 0) return cudaSuccess;
-    CUtensorMap mq, mk, mdo;
+    CUtensorMap mq, mk, mv, mdo;
     if (!make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dk, L, BH, 64, true) ||
         !make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dk, L, BH, 64, true) ||
+        !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dv, L, BH, 64, true) ||
         !make_map(&mdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Dv, L, BH, 64, true))
         return cudaErrorInvalidValue;
     DgArgs a{};
     a.beta = beta;
-    a.saved = saved;
-    a.xw = xw;
+    a.saved = static_cast<const __nv_bfloat16*>(saved);
     a.drw = drw;
-    a.dsend = dsend;
-    a.db1 = db1;
+    a.dsend = static_cast<const __nv_bfloat16*>(dsend);
     a.dq = static_cast<__nv_bfloat16*>(dq);
     a.dk = static_cast<__nv_bfloat16*>(dk);
     a.dbeta = dbeta;
@@ -1301,7 +1331,7 @@ cudaError_t deltanet_grads(int B, int H, int L, int Dk, int Dv, float scale, con
     a.L = L;
     a.Dv = Dv;
     a.scale = scale;
-    return Dk == 64 ? dg_launch<64>(mq, mk, mdo, a, nc, st) : dg_launch<128>(mq, mk, mdo, a, nc, st);
+    return Dk == 64 ? dg_launch<64>(mq, mk, mv, mdo, a, nc, st) : dg_launch<128>(mq, mk, mv, mdo, a, nc, st);
 }
 
 }  // namespace tc

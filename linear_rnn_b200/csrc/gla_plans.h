@@ -40,24 +40,23 @@ cudaError_t seg_scan(const Dims& P, int nseg, const float* seg_state, const floa
 cudaError_t seg_rscan(const Dims& P, int nseg, const float* seg_state, const float* seg_gamma, const float* dhT,
                       float* gend, cudaStream_t st);
 int num_sms();
-// DeltaNet forward on the tensor cores (gla_deltanet_tc.cu): bf16 I/O, Dk 64 or 128, Dv a
-// multiple of 64, chunk 64. o null: the state walk only (the backward's recompute). saved
-// (nullable): [BH, ceil(L/64), Dk, Dv] the state entering every chunk; status (nullable): device
-// status word for a wait that gave up.
+// DeltaNet on the tensor cores (gla_deltanet_tc.cu): bf16 I/O, Dk 64 or 128, Dv a multiple of
+// 64, chunk 64. Forward walk; o null: the state walk only (the backward's recompute). saved
+// (nullable): [BH, ceil(L/64), Dk, Dv] bf16, the state entering every chunk; status (nullable):
+// device status word for a wait that gave up.
 cudaError_t deltanet_fwd(int B, int H, int L, int Dk, int Dv, float scale, const void* q, const void* k,
-                         const void* v, const float* beta, const float* h0, void* o, float* hT, float* saved,
+                         const void* v, const float* beta, const float* h0, void* o, float* hT, void* saved,
                          int* status, cudaStream_t st);
-// The DeltaNet backward's reverse walk on the tensor cores (gla_deltanet_tc.cu), same limits:
-// from the saved chunk start states, writes X and dR ([BH*L, Dv] fp32), the gradient at every
-// chunk's end (as saved), each 64-column slice's sum_j dR U ([Dv/64, BH*L]), dv (bf16) and dh0.
+// The backward's reverse walk: dR ([BH*L, Dv] fp32), dv (bf16), dh0, and the gradient at every
+// chunk's end (bf16, laid out as saved).
 cudaError_t deltanet_walk(int B, int H, int L, int Dk, int Dv, float scale, const void* q, const void* k,
-                          const void* v, const float* beta, const void* dO, const float* dhT, const float* saved,
-                          float* xw, float* drw, float* dsend, float* db1, void* dv, float* dh0, cudaStream_t st);
-// The DeltaNet backward's per-chunk gradients on the tensor cores (gla_deltanet_tc.cu): dq, dk
-// (bf16) and dbeta from the walk's outputs, one CTA per (chunk, batch*head).
+                          const float* beta, const void* dO, const float* dhT, float* drw, void* dsend, void* dv,
+                          float* dh0, cudaStream_t st);
+// The backward's per-chunk gradients: dq, dk (bf16) and dbeta from the saved states, the end
+// gradients and dR, one CTA per (chunk, batch*head).
 cudaError_t deltanet_grads(int B, int H, int L, int Dk, int Dv, float scale, const void* q, const void* k,
-                           const float* beta, const void* dO, const float* saved, const float* xw, const float* drw,
-                           const float* dsend, const float* db1, void* dq, void* dk, float* dbeta, cudaStream_t st);
+                           const void* v, const float* beta, const void* dO, const void* saved, const float* drw,
+                           const void* dsend, void* dq, void* dk, float* dbeta, cudaStream_t st);
 // Backward (gla_tc_bwd.cu)
 bool bwd_supports(const Dims& P);
 size_t bwd_workspace_bytes(const Dims& P);
