@@ -18,9 +18,10 @@
 // segments joined by a scan over segment end states), den_t = (scale q_t) . n_t. Small kernels
 // then form h, and in the backward the upstream gradients of the two sums,
 //     dnum = dh / N,   dden = -(dh . h) / N * sign(den) where |den| > e^{-c} (else 0),
-// and, after the two backward passes, the sums of their dq, dk, dg and the chain rule through
-// the input gate, d i~ = (di_num + di_den) e^{i~ - c} (h does not depend on c). The normaliser's
-// backward is the recurrence's: with dn_t = scale dden_t q_t + e^{g_{t+1}} dn_{t+1},
+// and the sums of the two backward parts' dq, dk, dg and the chain rule through the input gate,
+// d i~ = (di_num + di_den) e^{i~ - c} (h does not depend on c), formed by the normaliser's last
+// kernel as it produces its part. The normaliser's backward is the recurrence's: with
+// dn_t = scale dden_t q_t + e^{g_{t+1}} dn_{t+1},
 //     dq_t = scale dden_t n_t,  dk_t = i_t dn_t,  di_t = k_t . dn_t,  dg_t = (n_t - i_t k_t) . dn_t
 // (i_t the input gate, e^{g_t} n_{t-1} = n_t - i_t k_t).
 #include <math.h>
@@ -88,12 +89,22 @@ __global__ void k_mlstm_nscan(const float* __restrict__ nloc, const float* __res
                               float* __restrict__ nstart) {
     const long bh = blockIdx.x;
     const int d = threadIdx.x;
+    // loads of 16 segments at a time go out before the chain that uses them
     float n = 0.f;
-#pragma unroll 8
-    for (int s = 0; s < nseg; ++s) {
-        const long i = (bh * nseg + s) * Dk + d;
-        nstart[i] = n;
-        n = __expf(gam[bh * nseg + s]) * n + nloc[i];
+    for (int s0 = 0; s0 < nseg; s0 += 16) {
+        float nl[16], ga[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+            if (s0 + u < nseg) {
+                nl[u] = nloc[(bh * nseg + s0 + u) * Dk + d];
+                ga[u] = gam[bh * nseg + s0 + u];
+            }
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+            if (s0 + u < nseg) {
+                nstart[(bh * nseg + s0 + u) * Dk + d] = n;
+                n = __expf(ga[u]) * n + nl[u];
+            }
     }
 }
 
@@ -151,23 +162,36 @@ __global__ void k_mlstm_cscan(const float* __restrict__ cloc, const float* __res
                               float* __restrict__ cin) {
     const long bh = blockIdx.x;
     const int d = threadIdx.x;
+    // loads of 16 segments at a time go out before the chain that uses them
     float c = 0.f;
-#pragma unroll 8
-    for (int s = nseg - 1; s >= 0; --s) {
-        const long i = (bh * nseg + s) * Dk + d;
-        cin[i] = c;
-        c = __expf(gam[bh * nseg + s]) * c + cloc[i];
+    for (int s1 = nseg - 1; s1 >= 0; s1 -= 16) {
+        float cl[16], ga[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+            if (s1 - u >= 0) {
+                cl[u] = cloc[(bh * nseg + s1 - u) * Dk + d];
+                ga[u] = gam[bh * nseg + s1 - u];
+            }
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+            if (s1 - u >= 0) {
+                cin[(bh * nseg + s1 - u) * Dk + d] = c;
+                c = __expf(ga[u]) * c + cl[u];
+            }
     }
 }
 
 // the normaliser's gradients over a segment: n_t forward from the segment's start state (kept in
-// shared memory), then dn_t backwards from the carry entering the segment's end
-template <typename T>
+// shared memory), then dn_t backwards from the carry entering the segment's end. They are added
+// to the value pass's in the same step: dq = dq1 + scale dden n_t and dk = dk1 + i_t dn_t in the
+// output dtype (dq1 / dk1 may be the outputs themselves), dg += (n_t - i_t k_t) . dn_t and
+// d i~ = (di1 + k_t . dn_t) i_t.
+template <typename T, typename Ta>
 __global__ void k_mlstm_den_bwd(const T* __restrict__ q, const T* __restrict__ k, const float* __restrict__ g,
                                 const float* __restrict__ ig, const float* __restrict__ dden,
                                 const float* __restrict__ nstart, const float* __restrict__ cin, int L, int Dk, int nseg,
-                                float scale, float* __restrict__ dq2, float* __restrict__ dk2, float* __restrict__ dg2,
-                                float* __restrict__ di2) {
+                                float scale, const Ta* dq1, const Ta* dk1, T* dq, T* dk, float* __restrict__ dg,
+                                const float* __restrict__ di1, float* __restrict__ ditil) {
     __shared__ float pi[ML_SL][8], pg[ML_SL][8];
     __shared__ float nv[ML_SL][256];   // n_t of the segment's tokens, [token][key dim]
     const long bh = blockIdx.y;
@@ -186,8 +210,8 @@ __global__ void k_mlstm_den_bwd(const T* __restrict__ q, const T* __restrict__ k
         const long r = r0 + j;
         const float sd = scale * dden[r], it = ig[r], kt = to_f(k[r * Dk + d]), nj = nv[j][d];
         const float dn = sd * to_f(q[r * Dk + d]) + c;
-        dq2[r * Dk + d] = sd * nj;
-        dk2[r * Dk + d] = it * dn;
+        dq[r * Dk + d] = from_f<T>(to_f(dq1[r * Dk + d]) + sd * nj);
+        dk[r * Dk + d] = from_f<T>(to_f(dk1[r * Dk + d]) + it * dn);
         ml_warp_part<8>(kt * dn, pi, j);
         ml_warp_part<8>((nj - it * kt) * dn, pg, j);
         c = __expf(g[r]) * dn;
@@ -199,8 +223,8 @@ __global__ void k_mlstm_den_bwd(const T* __restrict__ q, const T* __restrict__ k
             xi += pi[d][w];
             xg += pg[d][w];
         }
-        di2[r0 + d] = xi;
-        dg2[r0 + d] = xg;
+        dg[r0 + d] += xg;
+        ditil[r0 + d] = (di1[r0 + d] + xi) * ig[r0 + d];
     }
 }
 
@@ -241,28 +265,6 @@ __global__ void __launch_bounds__(ML_NT) k_mlstm_bwd_prep(const Ta* __restrict__
     if (lane == 0) dden[row] = fabsf(dn) > bound ? -s * inv * (dn > 0.f ? 1.f : -1.f) : 0.f;
 }
 
-// dq = dq1 + dq2 and dk = dk1 + dk2 (n_qk elements), dv = dv1 (n_v elements, only when the value
-// pass ran in another type than the outputs), dg += dg2 and d i~ = (di1 + di2) * e^{i~ - c}
-// (n_t tokens). dq1 / dk1 / dv1 may be the outputs themselves.
-template <typename Ta, typename To>
-__global__ void k_mlstm_bwd_final(To* dq, To* dk, To* dv, const Ta* dq1, const Ta* dk1, const Ta* dv1,
-                                  const float* __restrict__ dq2, const float* __restrict__ dk2, long n_qk, long n_v,
-                                  float* __restrict__ dg, const float* __restrict__ dg2, const float* __restrict__ di1,
-                                  const float* __restrict__ di2, const float* __restrict__ ig,
-                                  float* __restrict__ ditil, long n_t) {
-    const long stride = (long)gridDim.x * blockDim.x;
-    const long i0 = blockIdx.x * (long)blockDim.x + threadIdx.x;
-    for (long i = i0; i < n_qk; i += stride) {
-        dq[i] = from_f<To>(to_f(dq1[i]) + dq2[i]);
-        dk[i] = from_f<To>(to_f(dk1[i]) + dk2[i]);
-    }
-    for (long i = i0; i < n_v; i += stride) dv[i] = from_f<To>(to_f(dv1[i]));
-    for (long i = i0; i < n_t; i += stride) {
-        dg[i] += dg2[i];
-        ditil[i] = (di1[i] + di2[i]) * ig[i];
-    }
-}
-
 bool ml_aligned16(const void* x) { return x == nullptr || (reinterpret_cast<uintptr_t>(x) & 15u) == 0; }
 
 struct MlLayout {
@@ -273,7 +275,7 @@ struct MlLayout {
     int nseg;             // 32-token segments of the normaliser recurrence
     size_t wsa;           // the value pass's workspace bytes
     size_t o_ig, o_c, o_qf, o_kf, o_vf, o_num, o_den, o_nloc, o_gam, o_nst;
-    size_t o_dnum, o_dden, o_dq1, o_dk1, o_dv1, o_dq2, o_dk2, o_dg2, o_di1, o_di2, o_cloc, o_cin;
+    size_t o_dnum, o_dden, o_dq1, o_dk1, o_dv1, o_di1, o_cloc, o_cin;
     size_t total;
 };
 
@@ -330,13 +332,9 @@ gla_status ml_layout(const gla_problem* p, bool bwd, MlLayout* w) {
             w->o_dk1 = take(4 * BHL * p->Dk);
             w->o_dv1 = take(4 * BHL * p->Dv);
         }
-        w->o_dq2 = take(4 * BHL * p->Dk);
-        w->o_dk2 = take(4 * BHL * p->Dk);
         w->o_cloc = take(4 * NS * p->Dk);
         w->o_cin = take(4 * NS * p->Dk);
-        w->o_dg2 = take(4 * BHL);
         w->o_di1 = take(4 * BHL);
-        w->o_di2 = take(4 * BHL);
     }
     w->total = off;
     return GLA_OK;
@@ -426,8 +424,6 @@ gla_status ml_bwd(const gla_problem* p, const MlLayout& w, const void* q, const 
     if (e != cudaSuccess) return record_cuda(e, "mLSTM backward prep launch");
     const float* ig = reinterpret_cast<const float*>(ws + w.o_ig);
     float* di1 = reinterpret_cast<float*>(ws + w.o_di1);
-    float* di2 = reinterpret_cast<float*>(ws + w.o_di2);
-    float* dg2 = reinterpret_cast<float*>(ws + w.o_dg2);
     // the value pass writes its gradients straight into the outputs unless they are cast back
     void* dq1 = w.cast_a ? ws + w.o_dq1 : dq;
     void* dk1 = w.cast_a ? ws + w.o_dk1 : dk;
@@ -449,19 +445,19 @@ gla_status ml_bwd(const gla_problem* p, const MlLayout& w, const void* q, const 
                    k_mlstm_cscan<<<(unsigned)BH, p->Dk, 0, st>>>(cloc, reinterpret_cast<const float*>(ws + w.o_gam),
                                                                 w.nseg, p->Dk, cin));
         GLA_LAUNCH("mlstm_den_bwd", st,
-                   k_mlstm_den_bwd<To><<<grid, p->Dk, 0, st>>>(
+                   (k_mlstm_den_bwd<To, Ta><<<grid, p->Dk, 0, st>>>(
                        tq, tk, g, ig, dden, reinterpret_cast<const float*>(ws + w.o_nst), cin, p->L, p->Dk, w.nseg,
-                       p->scale, reinterpret_cast<float*>(ws + w.o_dq2), reinterpret_cast<float*>(ws + w.o_dk2), dg2,
-                       di2));
+                       p->scale, static_cast<const Ta*>(dq1), static_cast<const Ta*>(dk1), static_cast<To*>(dq),
+                       static_cast<To*>(dk), dg, di1, ditil)));
         if ((e = cudaGetLastError()) != cudaSuccess) return record_cuda(e, "mLSTM normaliser backward launch");
     }
-    const long nqk = rows * p->Dk, nv = w.cast_a ? rows * p->Dv : 0;
-    GLA_LAUNCH("mlstm_bwd_final", st,
-               (k_mlstm_bwd_final<Ta, To><<<ml_grid(nqk, 256), 256, 0, st>>>(
-                   static_cast<To*>(dq), static_cast<To*>(dk), static_cast<To*>(dv), static_cast<const Ta*>(dq1),
-                   static_cast<const Ta*>(dk1), static_cast<const Ta*>(dv1), reinterpret_cast<const float*>(ws + w.o_dq2),
-                   reinterpret_cast<const float*>(ws + w.o_dk2), nqk, nv, dg, dg2, di1, di2, ig, ditil, rows)));
-    return record_cuda(cudaGetLastError(), "mLSTM backward final launch");
+    if (w.cast_a) {   // dv of the fp32 value pass, cast back
+        const long nv = rows * p->Dv;
+        GLA_LAUNCH("mlstm_cast", st,
+                   (k_cast<float, To><<<ml_grid(nv, 256), 256, 0, st>>>(static_cast<const float*>(dv1),
+                                                                        static_cast<To*>(dv), nv)));
+    }
+    return record_cuda(cudaGetLastError(), "mLSTM backward cast launch");
 }
 
 }  // namespace
