@@ -136,7 +136,8 @@ def test_normaliser_bound_active():
 def test_full_size_workload():
     """The mLSTM workload (B=2 H=8 L=8192 Dk=Dv=256, bf16) on the GPU; two heads against the
     oracle."""
-    run(I.MLSTM, seed=0, heads=[1, 14])
+    errs = run(I.MLSTM, seed=0, heads=[1, 14])
+    record("mlstm automatic plan full size heads=[1, 14]", errs)
 
 
 def test_empty_and_deterministic():
