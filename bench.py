@@ -158,8 +158,10 @@ MEASURED_TRAFFIC = {
                           "sha": "fab635eb697cc988", "case": "c3"},
     ("tc_bwd_dq", "c5"): {"bytes": 392.6e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_tc_bwd.cu",
                           "sha": "fab635eb697cc988", "case": "c5"},
-    ("deltanet_bwd_walk", "deltanet"): {"bytes": 1099.9e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_deltanet_tc.cu",
-                                         "sha": "6ca3bafb3ab9258b", "case": "deltanet"},
+    ("deltanet_bwd_walk", "deltanet"): {"bytes": 490.5e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_deltanet_tc.cu",
+                                         "sha": "b19710d35dc88dde", "case": "deltanet"},
+    ("deltanet_bwd_grads", "deltanet"): {"bytes": 793.1e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_deltanet_tc.cu",
+                                          "sha": "b19710d35dc88dde", "case": "deltanet"},
     ("decode", "decode"): {"bytes": 214.9e6, "scale": 1, "src": "linear_rnn_b200/csrc/gla_decode.cu",
                            "sha": "45347f72608393eb", "case": "decode, 1024 heads"},
 }
@@ -335,19 +337,29 @@ DN_C = 64
 
 def deltanet_kernel_flops(name, B, H, L, Dk, Dv):
     """Algorithmic FLOPs of one launch (per token-head, multiplied by B*H*L): causal C x C
-    products count their lower half, K K^T and Q K^T once per head (not per value slice), the
-    chunk's triangular inverse C^2/3 per token."""
+    products count their lower half, K K^T and Q K^T once per head (not per value slice), a
+    chunk's triangular solve C per value column and token (C^2/3 per token for the inverse of the
+    CUDA-core plan). The tensor-core backward splits its work differently from the CUDA-core one
+    (the walk keeps only the dS chain, the gradient kernel forms X and U), so bf16 and fp32 I/O
+    have their own rows."""
     C = DN_C
+    tc = I.DELTANET["dtype"] == "bf16"
     per = {
-        # K K^T, Q K^T; K S, Q S, K^T X; T R, lower(Q K^T) X; the inverse
-        "deltanet_fwd": 2 * C * Dk + 6 * Dk * Dv + 2 * C * Dv + C * C / 3,
-        # the backward's state pass (no output): K K^T; K S, K^T X; T R; the inverse
-        "deltanet_state": C * Dk + 4 * Dk * Dv + C * Dv + C * C / 3,
-        # K K^T, P; K S, K dS', the dS update (2 products); P^T dO, T R, T^T dX; the inverse
-        "deltanet_bwd_walk": 2 * C * Dk + 8 * Dk * Dv + 3 * C * Dv + C * C / 3,
-        # dO X^T, dR X^T; dO S^T, X dS'^T, dR S^T; dP K, dP^T Q, G K, G^T (beta K)
-        "deltanet_bwd_grads": 2 * C * Dv + 6 * Dk * Dv + 4 * C * Dk,
+        # K K^T, Q K^T; K S, Q S, K^T X; the solve for X, lower(Q K^T) X
+        "deltanet_fwd": 2 * C * Dk + 6 * Dk * Dv + 2 * C * Dv + (0 if tc else C * C / 3),
+        # the backward's state pass (no output): K K^T; K S, K^T X; the solve for X
+        "deltanet_state": C * Dk + 4 * Dk * Dv + C * Dv + (0 if tc else C * C / 3),
     }
+    if tc:
+        # K K^T, Q K^T; K dS', Q^T dO, K^T diag(beta) dR; P^T dO; the transposed solve
+        per["deltanet_bwd_walk"] = 2 * C * Dk + 6 * Dk * Dv + 2 * C * Dv
+        # K K^T, K S, the solve for X; dO X^T, dR X^T; dO S^T, X dS'^T, dR S^T; dP K, dP^T Q, G K, G^T K
+        per["deltanet_bwd_grads"] = 5 * C * Dk + 8 * Dk * Dv + 3 * C * Dv
+    else:
+        # K K^T, P; K S, K dS', the dS update (2 products); P^T dO, T R, T^T dX; the inverse
+        per["deltanet_bwd_walk"] = 2 * C * Dk + 8 * Dk * Dv + 3 * C * Dv + C * C / 3
+        # dO X^T, dR X^T; dO S^T, X dS'^T, dR S^T; dP K, dP^T Q, G K, G^T (beta K)
+        per["deltanet_bwd_grads"] = 2 * C * Dv + 6 * Dk * Dv + 4 * C * Dk
     return float(per.get(name, 0.0)) * B * H * L
 
 

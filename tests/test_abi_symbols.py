@@ -243,11 +243,17 @@ def test_deltanet_backward_validates_before_launch():
         return _lib.lib.gla_deltanet_bwd(ctypes.byref(p), *(vp(a[n]) for n in names), a["nbytes"], None)
     dn = lambda **kw: prob(**dict(dict(gate=_lib.GLA_GATE_NONE, Dk=64, Dv=64), **kw))
     need = _lib.lib.gla_deltanet_bwd_workspace_bytes(ctypes.byref(dn()))
-    # chunk start states and end gradients (2 x B*H*5 chunks*Dk*Dv), X and dR (2 x B*H*L*Dv),
-    # per-slice sums (B*H*L), each region rounded up to 256 bytes
+    # each region rounded up to 256 bytes. fp32 I/O (CUDA-core kernels): chunk start states and
+    # end gradients (2 x B*H*5 chunks*Dk*Dv fp32), X and dR (2 x B*H*L*Dv fp32), per-slice sums
+    # (B*H*L fp32). bf16 I/O (tensor-core kernels): the states and end gradients in bf16, dR fp32.
     BH, L = 6, 300
-    parts = [BH * 5 * 64 * 64, BH * L * 64, BH * L * 64, BH * 5 * 64 * 64, BH * L]
-    assert need == sum((4 * n + 255) // 256 * 256 for n in parts)
+    rnd = lambda b: (b + 255) // 256 * 256
+    st, tok = BH * 5 * 64 * 64, BH * L * 64
+    assert _lib.lib.gla_deltanet_bwd_workspace_bytes(ctypes.byref(dn(io=_lib.GLA_F32))) == \
+        sum(rnd(4 * n) for n in (st, tok, tok, st, BH * L))
+    io = dn().io
+    assert need == (rnd(2 * st) + rnd(4 * tok) + rnd(2 * st) if io == _lib.GLA_BF16 else
+                    sum(rnd(4 * n) for n in (st, tok, tok, st, BH * L)))
     assert _lib.lib.gla_deltanet_bwd_workspace_bytes(ctypes.byref(dn(Dk=256))) == 0
     assert _lib.lib.gla_deltanet_bwd_workspace_bytes(ctypes.byref(dn(L=0))) == 256   # empty, still usable
     assert call(dn(), nbytes=need - 1) == _lib.GLA_ERR_WORKSPACE

@@ -83,9 +83,12 @@ def test_deltanet_reference_arm_and_flop_model():
     assert d["config"]["workload"].startswith("deltanet:") and d["e2e"]["d2h_bytes_per_step"] == 0
     sys.path.insert(0, ROOT)
     import bench
-    # per token-head at C = 64, Dk = Dv = 128: 2*64*128 + 6*128^2 + 2*64*128 + 64^2/3
-    per = 2 * 64 * 128 + 6 * 128 * 128 + 2 * 64 * 128 + 64 * 64 / 3
+    # per token-head at C = 64, Dk = Dv = 128 on the tensor-core plan (the bf16 workload): the chunk
+    # products and the substitution, no triangular inverse: 2*64*128 + 6*128^2 + 2*64*128
+    per = 2 * 64 * 128 + 6 * 128 * 128 + 2 * 64 * 128
     assert bench.deltanet_kernel_flops("deltanet_fwd", 1, 2, 10, 128, 128) == per * 20
+    # the gradient kernel: 5 C Dk + 8 Dk Dv + 3 C Dv
+    assert bench.deltanet_kernel_flops("deltanet_bwd_grads", 1, 1, 1, 128, 128) == 5 * 64 * 128 + 8 * 128 * 128 + 3 * 64 * 128
     assert bench.deltanet_kernel_flops("other", 1, 1, 1, 64, 64) == 0.0
     assert abs(bench.deltanet_alu_peak_tflops(1965.0) - 74.45) < 0.01
 
