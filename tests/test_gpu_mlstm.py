@@ -115,6 +115,13 @@ def test_normaliser_segment_edges(L):
     run(I.MLSTM.replace(B=1, H=3, L=L, Dk=64, Dv=64, scale=0.125), seed=9)
 
 
+@pytest.mark.parametrize("L", [1, 33, 257])
+def test_normaliser_segment_edges_fp32(L):
+    """fp32 I/O (both sums on the CUDA cores in fp32) at 1e-4, across segment edges and the
+    segment scans."""
+    run(I.MLSTM.replace(B=2, H=1, L=L, Dk=128, Dv=64, dtype="f32", scale=128 ** -0.5), seed=13)
+
+
 @pytest.mark.parametrize("shift", [60.0, -20.0])
 def test_input_gates_far_from_zero(shift):
     """exp(i~) far outside [e^-20, e^60]: the per-head shift keeps the gates in range and h equals
