@@ -211,7 +211,11 @@ GLA_API gla_status gla_shard_state_grad(const gla_problem* p, const void* q, con
  *   Keys are used as given (unit-norm keys with beta in [0, 1] keep each transition's
  *   eigenvalues in [1 - beta, 1]). All pointers 16-byte aligned, device memory, owned by the
  *   caller; no workspace. L = 0 copies h0 (or zero) to hT.
- * CUDA cores, fp32 arithmetic; asynchronous on `stream`.
+ * bf16 I/O runs on the tensor cores (chunk products as tcgen05 MMAs with fp32 accumulation,
+ * the chunk's triangular solve in fp32); fp32 I/O on the CUDA cores in fp32. Asynchronous on
+ * `stream`. There is no device status word: the tensor-core kernels' waits on their own copies
+ * and products are bounded, and one that gave up (a fault elsewhere on the device) leaves the
+ * outputs unwritten rather than hanging.
  * Errors: GLA_ERR_INVALID_ARG (null or misaligned pointer, bad enum, a gate mode),
  *   GLA_ERR_UNSUPPORTED (head dims, chunk, B*H), GLA_ERR_CUDA (gla_last_error_detail says
  *   which call failed). */
