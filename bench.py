@@ -18,6 +18,7 @@ ranks. `--impl reference` times the float64 CPU oracle on a bounded sample inste
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import math
@@ -441,10 +442,15 @@ def run_deltanet(args, world, rank, local):
     xd = {n: t.to(dev) for n, t in x.items()}
     dOd = dO.to(dev)
     sc = Dk ** -0.5
+    # training pair: the forward leaves the chunk start states the backward reads
+    prob = ops.make_problem(xd["q"], xd["v"], None, scale=sc, chunk=64, plan="auto")
+    saved = torch.empty(max(ops.gla_deltanet_saved_bytes(prob), 16), dtype=torch.uint8, device=dev)
+    ws = torch.empty(_lib.lib.gla_deltanet_bwd_workspace_bytes(ctypes.byref(prob)), dtype=torch.uint8, device=dev)
 
     def step():
-        ops.gla_deltanet_fwd(xd["q"], xd["k"], xd["v"], xd["beta"], xd["h0"], scale=sc)
-        ops.gla_deltanet_bwd(xd["q"], xd["k"], xd["v"], xd["beta"], xd["h0"], dOd, None, scale=sc)
+        ops.gla_deltanet_fwd(xd["q"], xd["k"], xd["v"], xd["beta"], xd["h0"], scale=sc, saved_states=saved)
+        ops.gla_deltanet_bwd(xd["q"], xd["k"], xd["v"], xd["beta"], xd["h0"], dOd, None, scale=sc, workspace=ws,
+                             saved_states=saved)
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     sampler = ClockSampler(local)
@@ -489,8 +495,10 @@ def run_deltanet(args, world, rank, local):
 
         def e2e_step():
             nonlocal d2h
-            o, hT = ops.gla_deltanet_fwd(xh["q"], xh["k"], xh["v"], xh["beta"], xh["h0"], scale=sc)
-            r = ops.gla_deltanet_bwd(xh["q"], xh["k"], xh["v"], xh["beta"], xh["h0"], dOh, None, scale=sc)
+            o, hT = ops.gla_deltanet_fwd(xh["q"], xh["k"], xh["v"], xh["beta"], xh["h0"], scale=sc,
+                                         saved_states=saved)
+            r = ops.gla_deltanet_bwd(xh["q"], xh["k"], xh["v"], xh["beta"], xh["h0"], dOh, None, scale=sc,
+                                     saved_states=saved)
             d2h = sum(t.numel() * t.element_size() for t in [o, hT, *r.values()] if t is not None)
 
         for _ in range(2):
@@ -663,14 +671,16 @@ def run_mlstm(args, world, rank, local):
     xd = {k: v.to(dev) for k, v in x.items()}
     kw = dict(scale=w.scale, chunk=w.chunk, plan=mplan)
     prob = ops.make_problem(xd["q"], xd["v"], xd["g"], scale=w.scale, chunk=w.chunk, plan=mplan)
-    import ctypes
     from linear_rnn_b200 import _lib
     ws = torch.empty(max(_lib.lib.gla_mlstm_workspace_bytes(ctypes.byref(prob), 0),
                          _lib.lib.gla_mlstm_workspace_bytes(ctypes.byref(prob), 1)), dtype=torch.uint8, device=dev)
+    # training pair: the forward keeps its results for the backward
+    saved = torch.empty(max(ops.gla_mlstm_saved_bytes(prob), 16), dtype=torch.uint8, device=dev)
 
     def step():
-        ops.gla_mlstm_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["itil"], workspace=ws, **kw)
-        ops.gla_mlstm_bwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["itil"], xd["dh"], workspace=ws, **kw)
+        ops.gla_mlstm_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["itil"], workspace=ws, saved_states=saved, **kw)
+        ops.gla_mlstm_bwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["itil"], xd["dh"], workspace=ws, saved_states=saved,
+                          **kw)
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     sampler = ClockSampler(local)
@@ -693,8 +703,8 @@ def run_mlstm(args, world, rank, local):
 
         def e2e_step():
             nonlocal d2h
-            h = ops.gla_mlstm_fwd(xh["q"], xh["k"], xh["v"], xh["g"], xh["itil"], **kw)
-            r = ops.gla_mlstm_bwd(xh["q"], xh["k"], xh["v"], xh["g"], xh["itil"], xh["dh"], **kw)
+            h = ops.gla_mlstm_fwd(xh["q"], xh["k"], xh["v"], xh["g"], xh["itil"], saved_states=saved, **kw)
+            r = ops.gla_mlstm_bwd(xh["q"], xh["k"], xh["v"], xh["g"], xh["itil"], xh["dh"], saved_states=saved, **kw)
             d2h = sum(t.numel() * t.element_size() for t in [h, *r.values()])
 
         for _ in range(2):

@@ -239,6 +239,27 @@ GLA_API gla_status gla_deltanet_bwd(const gla_problem* p, const void* q, const v
                                     void* dq, void* dk, void* dv, float* dbeta, float* dh0, void* ws,
                                     size_t ws_bytes, void* stream);
 
+/* DeltaNet training pair without the backward's state walk.
+ * gla_deltanet_saved_bytes: bytes of the buffer in which gla_deltanet_fwd_save leaves the state
+ *   entering every 64-token chunk, layout [B*H][ceil(L/64)][Dk][Dv], bf16 for bf16 I/O and f32
+ *   for f32 I/O (the values the backward's own state walk would write); 0 for an invalid
+ *   problem or L = 0.
+ * gla_deltanet_fwd_save: gla_deltanet_fwd that also writes those states into `saved` (NULL, or
+ *   a caller-owned device buffer of gla_deltanet_saved_bytes(p) bytes, 16-byte aligned).
+ * gla_deltanet_bwd_saved: gla_deltanet_bwd that reads them from `saved` instead of walking the
+ *   forward's recurrence again (two launches instead of three). `saved` must come from
+ *   gla_deltanet_fwd_save with the same problem and the same q, k, v, beta, h0; NULL means
+ *   recompute (the same as gla_deltanet_bwd). The workspace is gla_deltanet_bwd_workspace_bytes.
+ * Other arguments, results and errors as for gla_deltanet_fwd / gla_deltanet_bwd. */
+GLA_API size_t gla_deltanet_saved_bytes(const gla_problem* p);
+GLA_API gla_status gla_deltanet_fwd_save(const gla_problem* p, const void* q, const void* k, const void* v,
+                                         const float* beta, const float* h0, void* o, float* hT, void* saved,
+                                         void* stream);
+GLA_API gla_status gla_deltanet_bwd_saved(const gla_problem* p, const void* q, const void* k, const void* v,
+                                          const float* beta, const float* h0, const void* dO, const float* dhT,
+                                          const void* saved, void* dq, void* dk, void* dv, float* dbeta,
+                                          float* dh0, void* ws, size_t ws_bytes, void* stream);
+
 /* mLSTM cell: matrix memory with an exponential input gate, a normaliser state and a
  * max-stabiliser (named by the Tiled Flash Linear Attention abstract as the xLSTM cell its kernels
  * speed up; the cell is the published xLSTM one). Per (batch, head), with g_t the log forget gate
@@ -269,6 +290,30 @@ GLA_API gla_status gla_mlstm_fwd(const gla_problem* p, const void* q, const void
 GLA_API gla_status gla_mlstm_bwd(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
                                  const float* itil, const void* dh, void* dq, void* dk, void* dv, float* dg,
                                  float* ditil, void* ws, size_t ws_bytes, void* stream);
+
+/* mLSTM training pair without the backward's forward passes.
+ * gla_mlstm_saved_bytes: bytes of the caller-owned device buffer in which gla_mlstm_fwd_save
+ *   leaves, for gla_mlstm_bwd_saved, the forward's results the backward reads: the input gate and
+ *   per-head shift, the numerator and the normaliser term of every token, the normaliser
+ *   recurrence's segment decays and start states, and the value pass's saved states
+ *   (gla_saved_states_bytes of that pass); 0 for an invalid problem or an empty one.
+ * gla_mlstm_fwd_save: gla_mlstm_fwd that keeps those results in `saved` (NULL: in the workspace,
+ *   the same as gla_mlstm_fwd).
+ * gla_mlstm_bwd_saved: gla_mlstm_bwd that reads them from `saved` instead of running the forward
+ *   passes again, and hands the value pass's saved states to gla_bwd_saved. `saved` must come
+ *   from gla_mlstm_fwd_save with the same problem (plan included) and the same q, k, v, g, itil;
+ *   NULL means recompute (the same as gla_mlstm_bwd). The workspace is
+ *   gla_mlstm_workspace_bytes(p, 1) bytes.
+ * `saved` 16-byte aligned; other arguments, results and errors as for gla_mlstm_fwd /
+ * gla_mlstm_bwd. */
+GLA_API size_t gla_mlstm_saved_bytes(const gla_problem* p);
+GLA_API gla_status gla_mlstm_fwd_save(const gla_problem* p, const void* q, const void* k, const void* v,
+                                      const float* g, const float* itil, void* h, void* saved, void* ws,
+                                      size_t ws_bytes, void* stream);
+GLA_API gla_status gla_mlstm_bwd_saved(const gla_problem* p, const void* q, const void* k, const void* v,
+                                       const float* g, const float* itil, const void* dh, const void* saved,
+                                       void* dq, void* dk, void* dv, float* dg, float* ditil, void* ws,
+                                       size_t ws_bytes, void* stream);
 
 /* Static description of a status code (never NULL). */
 GLA_API const char* gla_status_string(gla_status s);

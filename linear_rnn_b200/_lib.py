@@ -23,7 +23,8 @@ EXPORTED = ("gla_workspace_bytes", "gla_fwd", "gla_bwd", "gla_status_string",
             "gla_saved_states_bytes", "gla_fwd_save", "gla_bwd_saved", "gla_debug_wait_timeout",
             "gla_decode", "gla_shard_state", "gla_state_fold", "gla_shard_state_grad", "gla_deltanet_fwd",
             "gla_deltanet_bwd_workspace_bytes", "gla_deltanet_bwd", "gla_mlstm_workspace_bytes", "gla_mlstm_fwd",
-            "gla_mlstm_bwd", "gla_shard_workspace_bytes")
+            "gla_mlstm_bwd", "gla_shard_workspace_bytes", "gla_deltanet_saved_bytes", "gla_deltanet_fwd_save",
+            "gla_deltanet_bwd_saved", "gla_mlstm_saved_bytes", "gla_mlstm_fwd_save", "gla_mlstm_bwd_saved")
 
 
 class GlaProblem(ctypes.Structure):
@@ -90,12 +91,24 @@ def _load():
     lib.gla_deltanet_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.gla_deltanet_bwd.argtypes = [pp] + [ctypes.c_void_p] * 13 + [ctypes.c_size_t, ctypes.c_void_p]
     lib.gla_deltanet_bwd.restype = ctypes.c_int
+    lib.gla_deltanet_saved_bytes.argtypes = [pp]
+    lib.gla_deltanet_saved_bytes.restype = ctypes.c_size_t
+    lib.gla_deltanet_fwd_save.argtypes = [pp] + [ctypes.c_void_p] * 9
+    lib.gla_deltanet_fwd_save.restype = ctypes.c_int
+    lib.gla_deltanet_bwd_saved.argtypes = [pp] + [ctypes.c_void_p] * 14 + [ctypes.c_size_t, ctypes.c_void_p]
+    lib.gla_deltanet_bwd_saved.restype = ctypes.c_int
     lib.gla_mlstm_workspace_bytes.argtypes = [pp, ctypes.c_int]
     lib.gla_mlstm_workspace_bytes.restype = ctypes.c_size_t
     lib.gla_mlstm_fwd.argtypes = [pp] + [ctypes.c_void_p] * 7 + [ctypes.c_size_t, ctypes.c_void_p]
     lib.gla_mlstm_fwd.restype = ctypes.c_int
     lib.gla_mlstm_bwd.argtypes = [pp] + [ctypes.c_void_p] * 12 + [ctypes.c_size_t, ctypes.c_void_p]
     lib.gla_mlstm_bwd.restype = ctypes.c_int
+    lib.gla_mlstm_saved_bytes.argtypes = [pp]
+    lib.gla_mlstm_saved_bytes.restype = ctypes.c_size_t
+    lib.gla_mlstm_fwd_save.argtypes = [pp] + [ctypes.c_void_p] * 8 + [ctypes.c_size_t, ctypes.c_void_p]
+    lib.gla_mlstm_fwd_save.restype = ctypes.c_int
+    lib.gla_mlstm_bwd_saved.argtypes = [pp] + [ctypes.c_void_p] * 13 + [ctypes.c_size_t, ctypes.c_void_p]
+    lib.gla_mlstm_bwd_saved.restype = ctypes.c_int
     lib.gla_state_fold.argtypes = [pp, ctypes.c_int] + [ctypes.c_void_p] * 5
     lib.gla_state_fold.restype = ctypes.c_int
     lib.gla_decode.argtypes = [pp] + [ctypes.c_void_p] * 8

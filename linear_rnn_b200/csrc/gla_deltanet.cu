@@ -729,11 +729,13 @@ DnBwdWs dn_bwd_ws(const gla_problem* p, void* base) {
     return w;
 }
 
+// states_given: w.saved already holds the chunk start states (left by the forward of a training
+// pair), so the forward's state walk is not run again.
 template <typename T, int DK>
 cudaError_t dn_bwd_launch(const gla_problem* p, const void* q, const void* k, const void* v, const float* beta,
                           const float* h0, const void* dO, const float* dhT, void* dq, void* dk, void* dv,
-                          float* dbeta, float* dh0, const DnBwdWs& w, cudaStream_t st) {
-    cudaError_t e = dn_launch_dk<T>(p, q, k, v, beta, h0, nullptr, nullptr, w.saved, st);
+                          float* dbeta, float* dh0, const DnBwdWs& w, bool states_given, cudaStream_t st) {
+    cudaError_t e = states_given ? cudaSuccess : dn_launch_dk<T>(p, q, k, v, beta, h0, nullptr, nullptr, w.saved, st);
     if (e != cudaSuccess) return e;
     const int BH = p->B * p->H, NC = (p->L + DN_C - 1) / DN_C;
     auto walk = k_deltanet_bwd_walk<T, DK>;
@@ -791,20 +793,75 @@ gla_status dn_check(const gla_problem* p) {
 }  // namespace
 }  // namespace gla
 
-extern "C" gla_status gla_deltanet_fwd(const gla_problem* p, const void* q, const void* k, const void* v,
-                                       const float* beta, const float* h0, void* o, float* hT, void* stream) {
-    const gla_status c = gla::dn_check(p);
+namespace gla {
+namespace {
+
+// Bytes of the chunk start states the backward reads: [B*H][chunks][Dk][Dv] in bf16 for bf16 I/O
+// (the precision the tensor-core products read them in), fp32 for fp32 I/O.
+size_t dn_saved_bytes(const gla_problem* p) {
+    const size_t BH = (size_t)p->B * p->H, NC = (size_t)((p->L + DN_C - 1) / DN_C);
+    return BH * NC * p->Dk * p->Dv * (p->io == GLA_BF16 ? 2 : 4);
+}
+
+gla_status dn_fwd_entry(const gla_problem* p, const void* q, const void* k, const void* v, const float* beta,
+                        const float* h0, void* o, float* hT, void* saved, void* stream) {
+    const gla_status c = dn_check(p);
     if (c != GLA_OK) return c;
     if ((size_t)p->B * p->H == 0) return GLA_OK;
     if (p->L > 0 && (!q || !k || !v || !beta || !o)) return GLA_ERR_INVALID_ARG;
-    const void* ptrs[] = {q, k, v, beta, h0, o, hT};
+    const void* ptrs[] = {q, k, v, beta, h0, o, hT, saved};
     for (const void* x : ptrs)
-        if (!gla::dn_aligned16(x)) return GLA_ERR_INVALID_ARG;
+        if (!dn_aligned16(x)) return GLA_ERR_INVALID_ARG;
+    if (dn_saved_bytes(p) == 0) saved = nullptr;
     cudaStream_t st = (cudaStream_t)stream;
-    const cudaError_t e = p->io == GLA_BF16
-                              ? gla::dn_launch_dk<__nv_bfloat16>(p, q, k, v, beta, h0, o, hT, nullptr, st)
-                              : gla::dn_launch_dk<float>(p, q, k, v, beta, h0, o, hT, nullptr, st);
-    return gla::record_cuda(e, "DeltaNet forward launch");
+    float* sv = static_cast<float*>(saved);
+    const cudaError_t e = p->io == GLA_BF16 ? dn_launch_dk<__nv_bfloat16>(p, q, k, v, beta, h0, o, hT, sv, st)
+                                            : dn_launch_dk<float>(p, q, k, v, beta, h0, o, hT, sv, st);
+    return record_cuda(e, "DeltaNet forward launch");
+}
+
+gla_status dn_bwd_entry(const gla_problem* p, const void* q, const void* k, const void* v, const float* beta,
+                        const float* h0, const void* dO, const float* dhT, const void* saved, void* dq, void* dk,
+                        void* dv, float* dbeta, float* dh0, void* ws, size_t ws_bytes, void* stream) {
+    const gla_status c = dn_check(p);
+    if (c != GLA_OK) return c;
+    if ((size_t)p->B * p->H == 0) return GLA_OK;
+    if (p->L > 0 && (!q || !k || !v || !beta || !dO || !dq || !dk || !dv || !dbeta)) return GLA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, beta, h0, dO, dhT, saved, dq, dk, dv, dbeta, dh0, ws};
+    for (const void* x : ptrs)
+        if (!dn_aligned16(x)) return GLA_ERR_INVALID_ARG;
+    DnBwdWs w = dn_bwd_ws(p, ws);
+    if (!ws || ws_bytes < w.bytes) return GLA_ERR_WORKSPACE;
+    const bool given = saved != nullptr && dn_saved_bytes(p) > 0;
+    if (given) w.saved = const_cast<float*>(static_cast<const float*>(saved));   // read only
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e;
+    if (p->io == GLA_BF16)
+        e = p->Dk == 64 ? dn_bwd_launch<__nv_bfloat16, 64>(p, q, k, v, beta, h0, dO, dhT, dq, dk, dv, dbeta, dh0, w, given, st)
+                        : dn_bwd_launch<__nv_bfloat16, 128>(p, q, k, v, beta, h0, dO, dhT, dq, dk, dv, dbeta, dh0, w, given, st);
+    else
+        e = p->Dk == 64 ? dn_bwd_launch<float, 64>(p, q, k, v, beta, h0, dO, dhT, dq, dk, dv, dbeta, dh0, w, given, st)
+                        : dn_bwd_launch<float, 128>(p, q, k, v, beta, h0, dO, dhT, dq, dk, dv, dbeta, dh0, w, given, st);
+    return record_cuda(e, "DeltaNet backward launch");
+}
+
+}  // namespace
+}  // namespace gla
+
+extern "C" gla_status gla_deltanet_fwd(const gla_problem* p, const void* q, const void* k, const void* v,
+                                       const float* beta, const float* h0, void* o, float* hT, void* stream) {
+    return gla::dn_fwd_entry(p, q, k, v, beta, h0, o, hT, nullptr, stream);
+}
+
+extern "C" size_t gla_deltanet_saved_bytes(const gla_problem* p) {
+    if (gla::dn_check(p) != GLA_OK) return 0;
+    return gla::dn_saved_bytes(p);
+}
+
+extern "C" gla_status gla_deltanet_fwd_save(const gla_problem* p, const void* q, const void* k, const void* v,
+                                            const float* beta, const float* h0, void* o, float* hT, void* saved,
+                                            void* stream) {
+    return gla::dn_fwd_entry(p, q, k, v, beta, h0, o, hT, saved, stream);
 }
 
 extern "C" size_t gla_deltanet_bwd_workspace_bytes(const gla_problem* p) {
@@ -816,22 +873,12 @@ extern "C" gla_status gla_deltanet_bwd(const gla_problem* p, const void* q, cons
                                        const float* beta, const float* h0, const void* dO, const float* dhT,
                                        void* dq, void* dk, void* dv, float* dbeta, float* dh0, void* ws,
                                        size_t ws_bytes, void* stream) {
-    const gla_status c = gla::dn_check(p);
-    if (c != GLA_OK) return c;
-    if ((size_t)p->B * p->H == 0) return GLA_OK;
-    if (p->L > 0 && (!q || !k || !v || !beta || !dO || !dq || !dk || !dv || !dbeta)) return GLA_ERR_INVALID_ARG;
-    const void* ptrs[] = {q, k, v, beta, h0, dO, dhT, dq, dk, dv, dbeta, dh0, ws};
-    for (const void* x : ptrs)
-        if (!gla::dn_aligned16(x)) return GLA_ERR_INVALID_ARG;
-    const gla::DnBwdWs w = gla::dn_bwd_ws(p, ws);
-    if (!ws || ws_bytes < w.bytes) return GLA_ERR_WORKSPACE;
-    cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e;
-    if (p->io == GLA_BF16)
-        e = p->Dk == 64 ? gla::dn_bwd_launch<__nv_bfloat16, 64>(p, q, k, v, beta, h0, dO, dhT, dq, dk, dv, dbeta, dh0, w, st)
-                        : gla::dn_bwd_launch<__nv_bfloat16, 128>(p, q, k, v, beta, h0, dO, dhT, dq, dk, dv, dbeta, dh0, w, st);
-    else
-        e = p->Dk == 64 ? gla::dn_bwd_launch<float, 64>(p, q, k, v, beta, h0, dO, dhT, dq, dk, dv, dbeta, dh0, w, st)
-                        : gla::dn_bwd_launch<float, 128>(p, q, k, v, beta, h0, dO, dhT, dq, dk, dv, dbeta, dh0, w, st);
-    return gla::record_cuda(e, "DeltaNet backward launch");
+    return gla::dn_bwd_entry(p, q, k, v, beta, h0, dO, dhT, nullptr, dq, dk, dv, dbeta, dh0, ws, ws_bytes, stream);
+}
+
+extern "C" gla_status gla_deltanet_bwd_saved(const gla_problem* p, const void* q, const void* k, const void* v,
+                                             const float* beta, const float* h0, const void* dO, const float* dhT,
+                                             const void* saved, void* dq, void* dk, void* dv, float* dbeta,
+                                             float* dh0, void* ws, size_t ws_bytes, void* stream) {
+    return gla::dn_bwd_entry(p, q, k, v, beta, h0, dO, dhT, saved, dq, dk, dv, dbeta, dh0, ws, ws_bytes, stream);
 }

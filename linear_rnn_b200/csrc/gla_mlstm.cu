@@ -274,9 +274,14 @@ struct MlLayout {
                           // cast back
     int nseg;             // 32-token segments of the normaliser recurrence
     size_t wsa;           // the value pass's workspace bytes
-    size_t o_ig, o_c, o_qf, o_kf, o_vf, o_num, o_den, o_nloc, o_gam, o_nst;
+    size_t o_qf, o_kf, o_vf, o_nloc;
     size_t o_dnum, o_dden, o_dq1, o_dk1, o_dv1, o_di1, o_cloc, o_cin;
+    size_t o_res;         // the forward's results (MlRes) when they live in the workspace
     size_t total;
+    // The forward's results the backward reads, at offsets from their own base: the input gate,
+    // the per-head shift, num, den, the normaliser's segment decays and start states, and (saved
+    // buffer only) the value pass's saved states for gla_bwd_saved.
+    size_t r_ig, r_c, r_num, r_den, r_gam, r_nst, r_gla, res_bytes, gla_saved, saved_total;
 };
 
 gla_status ml_layout(const gla_problem* p, bool bwd, MlLayout* w) {
@@ -312,18 +317,31 @@ gla_status ml_layout(const gla_problem* p, bool bwd, MlLayout* w) {
         off = align_up(off + bytes, 256);
         return o;
     };
-    w->o_ig = take(4 * BHL);
-    w->o_c = take(4 * BH);
+    {
+        size_t r = 0;
+        auto rtake = [&](size_t bytes) {
+            const size_t o = r;
+            r = align_up(r + bytes, 256);
+            return o;
+        };
+        w->r_ig = rtake(4 * BHL);
+        w->r_c = rtake(4 * BH);
+        w->r_num = rtake(ea * BHL * p->Dv);
+        w->r_den = rtake(4 * BHL);
+        w->r_gam = rtake(4 * NS);
+        w->r_nst = rtake(4 * NS * p->Dk);
+        w->res_bytes = r;
+        w->gla_saved = gla_saved_states_bytes(&w->pa);
+        w->r_gla = w->gla_saved ? rtake(w->gla_saved) : 0;
+        w->saved_total = r;
+    }
+    w->o_res = take(w->res_bytes);
     if (w->cast_a) {
         w->o_qf = take(4 * BHL * p->Dk);
         w->o_kf = take(4 * BHL * p->Dk);
         w->o_vf = take(4 * BHL * p->Dv);
     }
-    w->o_num = take(ea * BHL * p->Dv);
-    w->o_den = take(4 * BHL);
     w->o_nloc = take(4 * NS * p->Dk);
-    w->o_gam = take(4 * NS);
-    w->o_nst = take(4 * NS * p->Dk);
     if (bwd) {
         w->o_dnum = take(ea * BHL * p->Dv);
         w->o_dden = take(4 * BHL);
@@ -350,86 +368,124 @@ struct MlInputs {
     const void *qa, *ka, *va;
 };
 
-// Shared by the forward and the backward: the input gate, fp32 copies of bf16 inputs where the
-// value pass runs in fp32, num (the value pass) and den (the normaliser recurrence) in the
-// workspace.
-template <typename Ta, typename To>
-gla_status ml_forward_passes(const gla_problem* p, const MlLayout& w, const void* q, const void* k, const void* v,
-                             const float* g, const float* itil, char* ws, MlInputs* in, cudaStream_t st) {
-    const long BH = (long)p->B * p->H, BHL = BH * p->L;
-    float* ig = reinterpret_cast<float*>(ws + w.o_ig);
-    float* cst = reinterpret_cast<float*>(ws + w.o_c);
+// Where the forward's results live: in the workspace, or (a training pair) in the caller's
+// saved buffer, which then also takes the value pass's saved states.
+struct MlRes {
+    float* ig;
+    float* c;
+    void* num;
+    float* den;
+    float* gam;
+    float* nst;
+    float* gla;   // value pass's saved states, or null
+};
+
+MlRes ml_res(const MlLayout& w, char* ws, char* saved) {
+    char* b = saved ? saved : ws + w.o_res;
+    MlRes r;
+    r.ig = reinterpret_cast<float*>(b + w.r_ig);
+    r.c = reinterpret_cast<float*>(b + w.r_c);
+    r.num = b + w.r_num;
+    r.den = reinterpret_cast<float*>(b + w.r_den);
+    r.gam = reinterpret_cast<float*>(b + w.r_gam);
+    r.nst = reinterpret_cast<float*>(b + w.r_nst);
+    r.gla = (saved && w.gla_saved) ? reinterpret_cast<float*>(b + w.r_gla) : nullptr;
+    return r;
+}
+
+// fp32 copies of bf16 inputs where the value pass runs in fp32 (else the caller's inputs).
+template <typename To>
+gla_status ml_inputs(const gla_problem* p, const MlLayout& w, const void* q, const void* k, const void* v, char* ws,
+                     MlInputs* in, cudaStream_t st) {
     *in = MlInputs{q, k, v};
-    GLA_LAUNCH("mlstm_prep", st, k_mlstm_prep<<<(unsigned)BH, ML_NT, 0, st>>>(itil, p->L, ig, cst));
+    if (!w.cast_a) return GLA_OK;
+    const long BHL = (long)p->B * p->H * p->L;
+    const long nq = BHL * p->Dk, nv = BHL * p->Dv;
+    float* qf = reinterpret_cast<float*>(ws + w.o_qf);
+    float* kf = reinterpret_cast<float*>(ws + w.o_kf);
+    float* vf = reinterpret_cast<float*>(ws + w.o_vf);
+    GLA_LAUNCH("mlstm_cast", st, (k_cast<To, float><<<ml_grid(nq, 256), 256, 0, st>>>(static_cast<const To*>(q), qf, nq)));
+    GLA_LAUNCH("mlstm_cast", st, (k_cast<To, float><<<ml_grid(nq, 256), 256, 0, st>>>(static_cast<const To*>(k), kf, nq)));
+    GLA_LAUNCH("mlstm_cast", st, (k_cast<To, float><<<ml_grid(nv, 256), 256, 0, st>>>(static_cast<const To*>(v), vf, nv)));
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return record_cuda(e, "mLSTM input conversion launch");
+    *in = MlInputs{qf, kf, vf};
+    return GLA_OK;
+}
+
+// Shared by the forward and the backward (unless the backward reads a training pair's saved
+// results): the input gate, num (the value pass) and den (the normaliser recurrence) into `r`.
+template <typename Ta, typename To>
+gla_status ml_forward_passes(const gla_problem* p, const MlLayout& w, const MlInputs& in, const void* q,
+                             const void* k, const float* g, const float* itil, char* ws, const MlRes& r,
+                             cudaStream_t st) {
+    const long BH = (long)p->B * p->H;
+    GLA_LAUNCH("mlstm_prep", st, k_mlstm_prep<<<(unsigned)BH, ML_NT, 0, st>>>(itil, p->L, r.ig, r.c));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return record_cuda(e, "mLSTM gate launch");
-    if (w.cast_a) {
-        const long nq = BHL * p->Dk, nv = BHL * p->Dv;
-        float* qf = reinterpret_cast<float*>(ws + w.o_qf);
-        float* kf = reinterpret_cast<float*>(ws + w.o_kf);
-        float* vf = reinterpret_cast<float*>(ws + w.o_vf);
-        GLA_LAUNCH("mlstm_cast", st, (k_cast<To, float><<<ml_grid(nq, 256), 256, 0, st>>>(static_cast<const To*>(q), qf, nq)));
-        GLA_LAUNCH("mlstm_cast", st, (k_cast<To, float><<<ml_grid(nq, 256), 256, 0, st>>>(static_cast<const To*>(k), kf, nq)));
-        GLA_LAUNCH("mlstm_cast", st, (k_cast<To, float><<<ml_grid(nv, 256), 256, 0, st>>>(static_cast<const To*>(v), vf, nv)));
-        if ((e = cudaGetLastError()) != cudaSuccess) return record_cuda(e, "mLSTM input conversion launch");
-        *in = MlInputs{qf, kf, vf};
-    }
-    gla_status s = gla_fwd(&w.pa, in->qa, in->ka, in->va, g, ig, nullptr, ws + w.o_num, nullptr, ws, w.wsa, st);
+    gla_status s = gla_fwd_save(&w.pa, in.qa, in.ka, in.va, g, r.ig, nullptr, r.num, nullptr, r.gla, ws, w.wsa, st);
     if (s != GLA_OK) return s;
     // the normaliser recurrence, reading q and k in the I/O dtype
     const To* tq = static_cast<const To*>(q);
     const To* tk = static_cast<const To*>(k);
     float* nloc = reinterpret_cast<float*>(ws + w.o_nloc);
-    float* gam = reinterpret_cast<float*>(ws + w.o_gam);
-    float* nst = reinterpret_cast<float*>(ws + w.o_nst);
     const dim3 grid(w.nseg, (unsigned)BH);
-    GLA_LAUNCH("mlstm_nloc", st, k_mlstm_nloc<To><<<grid, p->Dk, 0, st>>>(tk, g, ig, p->L, p->Dk, w.nseg, nloc, gam));
-    GLA_LAUNCH("mlstm_nscan", st, k_mlstm_nscan<<<(unsigned)BH, p->Dk, 0, st>>>(nloc, gam, w.nseg, p->Dk, nst));
+    GLA_LAUNCH("mlstm_nloc", st, k_mlstm_nloc<To><<<grid, p->Dk, 0, st>>>(tk, g, r.ig, p->L, p->Dk, w.nseg, nloc, r.gam));
+    GLA_LAUNCH("mlstm_nscan", st, k_mlstm_nscan<<<(unsigned)BH, p->Dk, 0, st>>>(nloc, r.gam, w.nseg, p->Dk, r.nst));
     GLA_LAUNCH("mlstm_den", st,
-               k_mlstm_den<To><<<grid, p->Dk, 0, st>>>(tq, tk, g, ig, nst, p->L, p->Dk, w.nseg, p->scale,
-                                                       reinterpret_cast<float*>(ws + w.o_den)));
+               k_mlstm_den<To><<<grid, p->Dk, 0, st>>>(tq, tk, g, r.ig, r.nst, p->L, p->Dk, w.nseg, p->scale, r.den));
     return record_cuda(cudaGetLastError(), "mLSTM normaliser launch");
 }
 
+// saved: a training pair's buffer (gla_mlstm_saved_bytes) that receives the forward's results, or
+// null to keep them in the workspace.
 template <typename Ta, typename To>
 gla_status ml_fwd(const gla_problem* p, const MlLayout& w, const void* q, const void* k, const void* v,
-                  const float* g, const float* itil, void* h, char* ws, cudaStream_t st) {
+                  const float* g, const float* itil, void* h, char* ws, char* saved, cudaStream_t st) {
     MlInputs in;
-    gla_status s = ml_forward_passes<Ta, To>(p, w, q, k, v, g, itil, ws, &in, st);
+    gla_status s = ml_inputs<To>(p, w, q, k, v, ws, &in, st);
+    if (s != GLA_OK) return s;
+    const MlRes r = ml_res(w, ws, saved);
+    s = ml_forward_passes<Ta, To>(p, w, in, q, k, g, itil, ws, r, st);
     if (s != GLA_OK) return s;
     const long rows = (long)p->B * p->H * p->L;
     GLA_LAUNCH("mlstm_norm", st,
                (k_mlstm_norm<Ta, To><<<(unsigned)((rows + ML_NT / 32 - 1) / (ML_NT / 32)), ML_NT, 0, st>>>(
-                   reinterpret_cast<const Ta*>(ws + w.o_num), reinterpret_cast<const float*>(ws + w.o_den),
-                   reinterpret_cast<const float*>(ws + w.o_c), static_cast<To*>(h), rows, p->L, p->Dv)));
+                   static_cast<const Ta*>(r.num), r.den, r.c, static_cast<To*>(h), rows, p->L, p->Dv)));
     return record_cuda(cudaGetLastError(), "mLSTM normalise launch");
 }
 
+// saved: the buffer the forward of a training pair filled (its results are read from there and
+// the forward passes are not run again), or null to run them.
 template <typename Ta, typename To>
 gla_status ml_bwd(const gla_problem* p, const MlLayout& w, const void* q, const void* k, const void* v,
                   const float* g, const float* itil, const void* dh, void* dq, void* dk, void* dv, float* dg,
-                  float* ditil, char* ws, cudaStream_t st) {
+                  float* ditil, char* ws, char* saved, cudaStream_t st) {
     MlInputs in;
-    gla_status s = ml_forward_passes<Ta, To>(p, w, q, k, v, g, itil, ws, &in, st);
+    gla_status s = ml_inputs<To>(p, w, q, k, v, ws, &in, st);
     if (s != GLA_OK) return s;
+    const MlRes r = ml_res(w, ws, saved);
+    if (!saved) {
+        s = ml_forward_passes<Ta, To>(p, w, in, q, k, g, itil, ws, r, st);
+        if (s != GLA_OK) return s;
+    }
     const long rows = (long)p->B * p->H * p->L;
     Ta* dnum = reinterpret_cast<Ta*>(ws + w.o_dnum);
     float* dden = reinterpret_cast<float*>(ws + w.o_dden);
     GLA_LAUNCH("mlstm_bwd_prep", st,
                (k_mlstm_bwd_prep<Ta, To><<<(unsigned)((rows + ML_NT / 32 - 1) / (ML_NT / 32)), ML_NT, 0, st>>>(
-                   reinterpret_cast<const Ta*>(ws + w.o_num), reinterpret_cast<const float*>(ws + w.o_den),
-                   reinterpret_cast<const float*>(ws + w.o_c), static_cast<const To*>(dh), dnum, dden, rows, p->L,
+                   static_cast<const Ta*>(r.num), r.den, r.c, static_cast<const To*>(dh), dnum, dden, rows, p->L,
                    p->Dv)));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return record_cuda(e, "mLSTM backward prep launch");
-    const float* ig = reinterpret_cast<const float*>(ws + w.o_ig);
+    const float* ig = r.ig;
     float* di1 = reinterpret_cast<float*>(ws + w.o_di1);
     // the value pass writes its gradients straight into the outputs unless they are cast back
     void* dq1 = w.cast_a ? ws + w.o_dq1 : dq;
     void* dk1 = w.cast_a ? ws + w.o_dk1 : dk;
     void* dv1 = w.cast_a ? ws + w.o_dv1 : dv;
-    s = gla_bwd(&w.pa, in.qa, in.ka, in.va, g, ig, nullptr, dnum, nullptr, dq1, dk1, dv1, dg, di1, nullptr, ws, w.wsa,
-                st);
+    s = gla_bwd_saved(&w.pa, in.qa, in.ka, in.va, g, ig, nullptr, dnum, nullptr, r.gla, dq1, dk1, dv1, dg, di1,
+                      nullptr, ws, w.wsa, st);
     if (s != GLA_OK) return s;
     // the normaliser recurrence's backward, reading q and k in the I/O dtype
     {
@@ -442,11 +498,10 @@ gla_status ml_bwd(const gla_problem* p, const MlLayout& w, const void* q, const 
         GLA_LAUNCH("mlstm_dnloc", st,
                    k_mlstm_dnloc<To><<<grid, p->Dk, 0, st>>>(tq, g, dden, p->L, p->Dk, w.nseg, p->scale, cloc));
         GLA_LAUNCH("mlstm_cscan", st,
-                   k_mlstm_cscan<<<(unsigned)BH, p->Dk, 0, st>>>(cloc, reinterpret_cast<const float*>(ws + w.o_gam),
-                                                                w.nseg, p->Dk, cin));
+                   k_mlstm_cscan<<<(unsigned)BH, p->Dk, 0, st>>>(cloc, r.gam, w.nseg, p->Dk, cin));
         GLA_LAUNCH("mlstm_den_bwd", st,
                    (k_mlstm_den_bwd<To, Ta><<<grid, p->Dk, 0, st>>>(
-                       tq, tk, g, ig, dden, reinterpret_cast<const float*>(ws + w.o_nst), cin, p->L, p->Dk, w.nseg,
+                       tq, tk, g, ig, dden, r.nst, cin, p->L, p->Dk, w.nseg,
                        p->scale, static_cast<const Ta*>(dq1), static_cast<const Ta*>(dk1), static_cast<To*>(dq),
                        static_cast<To*>(dk), dg, di1, ditil)));
         if ((e = cudaGetLastError()) != cudaSuccess) return record_cuda(e, "mLSTM normaliser backward launch");
@@ -463,6 +518,63 @@ gla_status ml_bwd(const gla_problem* p, const MlLayout& w, const void* q, const 
 }  // namespace
 }  // namespace gla
 
+namespace gla {
+namespace {
+
+gla_status ml_fwd_entry(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
+                        const float* itil, void* h, void* saved, void* ws, size_t ws_bytes, void* stream) {
+    MlLayout w;
+    const gla_status s = ml_layout(p, false, &w);
+    if (s != GLA_OK) return s;
+    const bool empty = (size_t)p->B * p->H * p->L == 0;
+    if (!empty && (!q || !k || !v || !g || !itil || !h)) return GLA_ERR_INVALID_ARG;
+    if (!ws) return GLA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, g, itil, h, saved, ws};
+    for (const void* x : ptrs)
+        if (!ml_aligned16(x)) return GLA_ERR_INVALID_ARG;
+    if (ws_bytes < w.total) return GLA_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    const cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, st);
+    if (e != cudaSuccess) return record_cuda(e, "status word reset");
+    if (empty) return GLA_OK;
+    char* wsb = static_cast<char*>(ws);
+    char* sv = static_cast<char*>(saved);
+    using bf16 = __nv_bfloat16;
+    if (p->io == GLA_F32) return ml_fwd<float, float>(p, w, q, k, v, g, itil, h, wsb, sv, st);
+    return w.fa ? ml_fwd<float, bf16>(p, w, q, k, v, g, itil, h, wsb, sv, st)
+                : ml_fwd<bf16, bf16>(p, w, q, k, v, g, itil, h, wsb, sv, st);
+}
+
+gla_status ml_bwd_entry(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
+                        const float* itil, const void* dh, const void* saved, void* dq, void* dk, void* dv, float* dg,
+                        float* ditil, void* ws, size_t ws_bytes, void* stream) {
+    MlLayout w;
+    const gla_status s = ml_layout(p, true, &w);
+    if (s != GLA_OK) return s;
+    const bool empty = (size_t)p->B * p->H * p->L == 0;
+    if (!empty && (!q || !k || !v || !g || !itil || !dh || !dq || !dk || !dv || !dg || !ditil))
+        return GLA_ERR_INVALID_ARG;
+    if (!ws) return GLA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, g, itil, dh, saved, dq, dk, dv, dg, ditil, ws};
+    for (const void* x : ptrs)
+        if (!ml_aligned16(x)) return GLA_ERR_INVALID_ARG;
+    if (ws_bytes < w.total) return GLA_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    const cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, st);
+    if (e != cudaSuccess) return record_cuda(e, "status word reset");
+    if (empty) return GLA_OK;
+    char* wsb = static_cast<char*>(ws);
+    char* sv = const_cast<char*>(static_cast<const char*>(saved));   // read only
+    using bf16 = __nv_bfloat16;
+    if (p->io == GLA_F32)
+        return ml_bwd<float, float>(p, w, q, k, v, g, itil, dh, dq, dk, dv, dg, ditil, wsb, sv, st);
+    return w.fa ? ml_bwd<float, bf16>(p, w, q, k, v, g, itil, dh, dq, dk, dv, dg, ditil, wsb, sv, st)
+                : ml_bwd<bf16, bf16>(p, w, q, k, v, g, itil, dh, dq, dk, dv, dg, ditil, wsb, sv, st);
+}
+
+}  // namespace
+}  // namespace gla
+
 extern "C" {
 
 size_t gla_mlstm_workspace_bytes(const gla_problem* p, int for_backward) {
@@ -471,53 +583,33 @@ size_t gla_mlstm_workspace_bytes(const gla_problem* p, int for_backward) {
     return w.total;
 }
 
+size_t gla_mlstm_saved_bytes(const gla_problem* p) {
+    gla::MlLayout w;
+    if (gla::ml_layout(p, true, &w) != GLA_OK) return 0;
+    if ((size_t)p->B * p->H * p->L == 0) return 0;
+    return w.saved_total;
+}
+
 gla_status gla_mlstm_fwd(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
                          const float* itil, void* h, void* ws, size_t ws_bytes, void* stream) {
-    gla::MlLayout w;
-    const gla_status s = gla::ml_layout(p, false, &w);
-    if (s != GLA_OK) return s;
-    const bool empty = (size_t)p->B * p->H * p->L == 0;
-    if (!empty && (!q || !k || !v || !g || !itil || !h)) return GLA_ERR_INVALID_ARG;
-    if (!ws) return GLA_ERR_INVALID_ARG;
-    const void* ptrs[] = {q, k, v, g, itil, h, ws};
-    for (const void* x : ptrs)
-        if (!gla::ml_aligned16(x)) return GLA_ERR_INVALID_ARG;
-    if (ws_bytes < w.total) return GLA_ERR_WORKSPACE;
-    cudaStream_t st = (cudaStream_t)stream;
-    const cudaError_t e = cudaMemsetAsync(ws, 0, gla::kStatusBytes, st);
-    if (e != cudaSuccess) return gla::record_cuda(e, "status word reset");
-    if (empty) return GLA_OK;
-    char* wsb = static_cast<char*>(ws);
-    using bf16 = __nv_bfloat16;
-    if (p->io == GLA_F32) return gla::ml_fwd<float, float>(p, w, q, k, v, g, itil, h, wsb, st);
-    return w.fa ? gla::ml_fwd<float, bf16>(p, w, q, k, v, g, itil, h, wsb, st)
-                : gla::ml_fwd<bf16, bf16>(p, w, q, k, v, g, itil, h, wsb, st);
+    return gla::ml_fwd_entry(p, q, k, v, g, itil, h, nullptr, ws, ws_bytes, stream);
+}
+
+gla_status gla_mlstm_fwd_save(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
+                              const float* itil, void* h, void* saved, void* ws, size_t ws_bytes, void* stream) {
+    return gla::ml_fwd_entry(p, q, k, v, g, itil, h, saved, ws, ws_bytes, stream);
 }
 
 gla_status gla_mlstm_bwd(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
                          const float* itil, const void* dh, void* dq, void* dk, void* dv, float* dg, float* ditil,
                          void* ws, size_t ws_bytes, void* stream) {
-    gla::MlLayout w;
-    const gla_status s = gla::ml_layout(p, true, &w);
-    if (s != GLA_OK) return s;
-    const bool empty = (size_t)p->B * p->H * p->L == 0;
-    if (!empty && (!q || !k || !v || !g || !itil || !dh || !dq || !dk || !dv || !dg || !ditil))
-        return GLA_ERR_INVALID_ARG;
-    if (!ws) return GLA_ERR_INVALID_ARG;
-    const void* ptrs[] = {q, k, v, g, itil, dh, dq, dk, dv, dg, ditil, ws};
-    for (const void* x : ptrs)
-        if (!gla::ml_aligned16(x)) return GLA_ERR_INVALID_ARG;
-    if (ws_bytes < w.total) return GLA_ERR_WORKSPACE;
-    cudaStream_t st = (cudaStream_t)stream;
-    const cudaError_t e = cudaMemsetAsync(ws, 0, gla::kStatusBytes, st);
-    if (e != cudaSuccess) return gla::record_cuda(e, "status word reset");
-    if (empty) return GLA_OK;
-    char* wsb = static_cast<char*>(ws);
-    using bf16 = __nv_bfloat16;
-    if (p->io == GLA_F32)
-        return gla::ml_bwd<float, float>(p, w, q, k, v, g, itil, dh, dq, dk, dv, dg, ditil, wsb, st);
-    return w.fa ? gla::ml_bwd<float, bf16>(p, w, q, k, v, g, itil, dh, dq, dk, dv, dg, ditil, wsb, st)
-                : gla::ml_bwd<bf16, bf16>(p, w, q, k, v, g, itil, dh, dq, dk, dv, dg, ditil, wsb, st);
+    return gla::ml_bwd_entry(p, q, k, v, g, itil, dh, nullptr, dq, dk, dv, dg, ditil, ws, ws_bytes, stream);
+}
+
+gla_status gla_mlstm_bwd_saved(const gla_problem* p, const void* q, const void* k, const void* v, const float* g,
+                               const float* itil, const void* dh, const void* saved, void* dq, void* dk, void* dv,
+                               float* dg, float* ditil, void* ws, size_t ws_bytes, void* stream) {
+    return gla::ml_bwd_entry(p, q, k, v, g, itil, dh, saved, dq, dk, dv, dg, ditil, ws, ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -139,10 +139,26 @@ def _mlstm_problem(q, v, g, itil, scale, chunk, plan):
     return make_problem(q, v, g, scale=scale, chunk=chunk, plan=plan)
 
 
+def gla_mlstm_saved_bytes(problem: GlaProblem) -> int:
+    return int(_lib.lib.gla_mlstm_saved_bytes(ctypes.byref(problem)))
+
+
+def _check_ml_saved(saved, prob):
+    if saved is None:
+        return
+    if saved.device.type != "cuda" or not saved.is_contiguous():
+        raise ValueError("saved_states must be a contiguous CUDA tensor")
+    if saved.numel() * saved.element_size() < gla_mlstm_saved_bytes(prob):
+        raise GlaError(_lib.GLA_ERR_WORKSPACE, "saved_states")
+
+
 def gla_mlstm_fwd(q, k, v, g, itil, *, scale: Optional[float] = None, chunk: int = 64, plan: str = "auto",
-                  workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+                  workspace: Optional[torch.Tensor] = None,
+                  saved_states: Optional[torch.Tensor] = None) -> torch.Tensor:
     """mLSTM cell (exponential input gate, normaliser, stabiliser): q, k [B,H,L,Dk], v [B,H,L,Dv],
-    g = log forget gate and itil = log input gate, both fp32 [B,H,L]. Returns h [B,H,L,Dv]."""
+    g = log forget gate and itil = log input gate, both fp32 [B,H,L]. Returns h [B,H,L,Dv].
+    saved_states: optional device buffer (at least gla_mlstm_saved_bytes) that keeps the forward's
+    results for gla_mlstm_bwd(..., saved_states=), which then does not run the forward again."""
     host = q.device.type != "cuda"
     device = torch.device("cuda", torch.cuda.current_device()) if host else q.device
     q, k, v, g, itil = (_to_dev(t, device) for t in (q, k, v, g, itil))
@@ -151,9 +167,11 @@ def gla_mlstm_fwd(q, k, v, g, itil, *, scale: Optional[float] = None, chunk: int
     if nbytes == 0:
         raise GlaError(_lib.GLA_ERR_UNSUPPORTED, "gla_mlstm_workspace_bytes")
     ws = _workspace(nbytes, device, workspace)
+    _check_ml_saved(saved_states, prob)
     h = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=device)
-    st = _lib.lib.gla_mlstm_fwd(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(itil), _ptr(h),
-                                _ptr(ws), ws.numel() * ws.element_size(), _stream_handle(device))
+    st = _lib.lib.gla_mlstm_fwd_save(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(itil), _ptr(h),
+                                     _ptr(saved_states), _ptr(ws), ws.numel() * ws.element_size(),
+                                     _stream_handle(device))
     _check(st, "gla_mlstm_fwd")
     if host:
         (h,) = _to_host([h])
@@ -161,8 +179,11 @@ def gla_mlstm_fwd(q, k, v, g, itil, *, scale: Optional[float] = None, chunk: int
 
 
 def gla_mlstm_bwd(q, k, v, g, itil, dh, *, scale: Optional[float] = None, chunk: int = 64, plan: str = "auto",
-                  workspace: Optional[torch.Tensor] = None) -> Dict[str, torch.Tensor]:
-    """Gradients of sum(dh * h) of gla_mlstm_fwd: dict dq, dk, dv (io dtype), dg, ditil (fp32)."""
+                  workspace: Optional[torch.Tensor] = None,
+                  saved_states: Optional[torch.Tensor] = None) -> Dict[str, torch.Tensor]:
+    """Gradients of sum(dh * h) of gla_mlstm_fwd: dict dq, dk, dv (io dtype), dg, ditil (fp32).
+    saved_states: the buffer a gla_mlstm_fwd with the same inputs and plan filled, or None to
+    run the forward passes again."""
     host = q.device.type != "cuda"
     device = torch.device("cuda", torch.cuda.current_device()) if host else q.device
     q, k, v, g, itil, dh = (_to_dev(t, device) for t in (q, k, v, g, itil, dh))
@@ -171,11 +192,12 @@ def gla_mlstm_bwd(q, k, v, g, itil, dh, *, scale: Optional[float] = None, chunk:
     if nbytes == 0:
         raise GlaError(_lib.GLA_ERR_UNSUPPORTED, "gla_mlstm_workspace_bytes")
     ws = _workspace(nbytes, device, workspace)
+    _check_ml_saved(saved_states, prob)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     dg, ditil = torch.empty_like(g), torch.empty_like(itil)
-    st = _lib.lib.gla_mlstm_bwd(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(itil), _ptr(dh),
-                                _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(ditil), _ptr(ws),
-                                ws.numel() * ws.element_size(), _stream_handle(device))
+    st = _lib.lib.gla_mlstm_bwd_saved(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(itil), _ptr(dh),
+                                      _ptr(saved_states), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(ditil),
+                                      _ptr(ws), ws.numel() * ws.element_size(), _stream_handle(device))
     _check(st, "gla_mlstm_bwd")
     out = {"dq": dq, "dk": dk, "dv": dv, "dg": dg, "ditil": ditil}
     if host:
@@ -201,23 +223,40 @@ def gla_decode(q, k, v, g, igate, state, *, scale: Optional[float] = None) -> to
     return o
 
 
+def gla_deltanet_saved_bytes(problem: GlaProblem) -> int:
+    return int(_lib.lib.gla_deltanet_saved_bytes(ctypes.byref(problem)))
+
+
+def _check_dn_saved(saved, prob):
+    if saved is None:
+        return
+    if saved.device.type != "cuda" or not saved.is_contiguous():
+        raise ValueError("saved_states must be a contiguous CUDA tensor")
+    if saved.numel() * saved.element_size() < gla_deltanet_saved_bytes(prob):
+        raise GlaError(_lib.GLA_ERR_WORKSPACE, "saved_states")
+
+
 def gla_deltanet_fwd(q, k, v, beta, h0=None, *, scale: Optional[float] = None,
-                 output_final_state: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+                     output_final_state: bool = True,
+                     saved_states: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunkwise DeltaNet forward: q, k [B,H,L,Dk], v [B,H,L,Dv] (bf16 or fp32), beta [B,H,L]
     fp32, h0 [B,H,Dk,Dv] fp32 or None. Returns o [B,H,L,Dv] and the final state (fp32, or None
-    when output_final_state is False). Host tensors are copied to the current device and the
-    results back."""
+    when output_final_state is False). saved_states: optional device buffer (at least
+    gla_deltanet_saved_bytes) that receives the chunk start states, which
+    gla_deltanet_bwd(..., saved_states=) then reads instead of walking the recurrence again.
+    Host tensors are copied to the current device and the results back."""
     host = q.device.type != "cuda"
     device = torch.device("cuda", torch.cuda.current_device()) if host else q.device
     q, k, v, beta, h0 = (_to_dev(t, device) for t in (q, k, v, beta, h0))
     if beta is None or beta.dtype != torch.float32 or tuple(beta.shape) != tuple(q.shape[:3]):
         raise ValueError("beta must be float32 [B, H, L]")
     prob = make_problem(q, v, None, scale=scale, chunk=64, plan="auto")
+    _check_dn_saved(saved_states, prob)
     o = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=device)
     hT = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
                      device=device) if output_final_state else None
-    st = _lib.lib.gla_deltanet_fwd(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(h0), _ptr(o),
-                                   _ptr(hT), _stream_handle(device))
+    st = _lib.lib.gla_deltanet_fwd_save(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(h0),
+                                        _ptr(o), _ptr(hT), _ptr(saved_states), _stream_handle(device))
     _check(st, "gla_deltanet_fwd")
     if host:
         o, hT = _to_host([o, hT])
@@ -225,10 +264,12 @@ def gla_deltanet_fwd(q, k, v, beta, h0=None, *, scale: Optional[float] = None,
 
 
 def gla_deltanet_bwd(q, k, v, beta, h0, dO, dhT=None, *, scale: Optional[float] = None,
-                     output_dh0: bool = True) -> Dict[str, Optional[torch.Tensor]]:
+                     output_dh0: bool = True, workspace: Optional[torch.Tensor] = None,
+                     saved_states: Optional[torch.Tensor] = None) -> Dict[str, Optional[torch.Tensor]]:
     """DeltaNet backward: dict dq, dk, dv (io dtype), dbeta (fp32 [B,H,L]) and dh0 (fp32, or
-    None when output_dh0 is False). Host tensors are copied to the current device and the
-    results back."""
+    None when output_dh0 is False). saved_states: the buffer a gla_deltanet_fwd on the same
+    inputs filled, or None to recompute the chunk start states. Host tensors are copied to the
+    current device and the results back."""
     host = q.device.type != "cuda"
     device = torch.device("cuda", torch.cuda.current_device()) if host else q.device
     q, k, v, beta, h0, dO, dhT = (_to_dev(t, device) for t in (q, k, v, beta, h0, dO, dhT))
@@ -238,14 +279,16 @@ def gla_deltanet_bwd(q, k, v, beta, h0, dO, dhT=None, *, scale: Optional[float] 
     nbytes = _lib.lib.gla_deltanet_bwd_workspace_bytes(ctypes.byref(prob))
     if nbytes == 0:
         raise GlaError(_lib.GLA_ERR_UNSUPPORTED, "gla_deltanet_bwd_workspace_bytes")
-    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    ws = _workspace(nbytes, device, workspace)
+    _check_dn_saved(saved_states, prob)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     dbeta = torch.empty_like(beta)
     dh0 = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
                       device=device) if output_dh0 else None
-    st = _lib.lib.gla_deltanet_bwd(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(h0), _ptr(dO),
-                                   _ptr(dhT), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dbeta), _ptr(dh0), _ptr(ws),
-                                   nbytes, _stream_handle(device))
+    st = _lib.lib.gla_deltanet_bwd_saved(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(h0),
+                                         _ptr(dO), _ptr(dhT), _ptr(saved_states), _ptr(dq), _ptr(dk), _ptr(dv),
+                                         _ptr(dbeta), _ptr(dh0), _ptr(ws), ws.numel() * ws.element_size(),
+                                         _stream_handle(device))
     _check(st, "gla_deltanet_bwd")
     out = {"dq": dq, "dk": dk, "dv": dv, "dbeta": dbeta, "dh0": dh0}
     if host:

@@ -267,6 +267,80 @@ def test_deltanet_backward_validates_before_launch():
     assert call(dn(H=0)) == _lib.GLA_OK
 
 
+
+def test_deltanet_training_pair_validates_before_launch():
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    dn = lambda **kw: prob(**dict(dict(gate=_lib.GLA_GATE_NONE, Dk=64, Dv=64), **kw))
+    saved_bytes = lambda p: _lib.lib.gla_deltanet_saved_bytes(ctypes.byref(p))
+    # the chunk start states: B*H x ceil(L/64) x Dk x Dv, bf16 for bf16 I/O and fp32 for fp32 I/O
+    BH, nc = 6, 5
+    assert saved_bytes(dn(io=_lib.GLA_BF16)) == BH * nc * 64 * 64 * 2
+    assert saved_bytes(dn(io=_lib.GLA_F32, Dk=128, Dv=192)) == BH * nc * 128 * 192 * 4
+    assert saved_bytes(dn(L=0)) == 0
+    assert saved_bytes(dn(Dk=256)) == 0 and saved_bytes(dn(gate=_lib.GLA_GATE_PER_KEY)) == 0
+
+    def fwd(p, **kw):
+        a = dict(q=16, k=16, v=16, beta=16, h0=None, o=16, hT=None, saved=16)
+        a.update(kw)
+        return _lib.lib.gla_deltanet_fwd_save(ctypes.byref(p), *(vp(a[n]) for n in ("q", "k", "v", "beta", "h0", "o",
+                                                                                   "hT", "saved")), None)
+    assert fwd(dn(), saved=24) == _lib.GLA_ERR_INVALID_ARG                   # misaligned
+    assert fwd(dn(Dv=96)) == _lib.GLA_ERR_UNSUPPORTED
+    assert fwd(dn(), o=None) == _lib.GLA_ERR_INVALID_ARG
+    assert fwd(dn(B=0)) == _lib.GLA_OK
+
+    names = ("q", "k", "v", "beta", "h0", "dO", "dhT", "saved", "dq", "dk", "dv", "dbeta", "dh0", "ws")
+
+    def bwd(p, **kw):
+        a = dict(q=16, k=16, v=16, beta=16, h0=None, dO=16, dhT=None, saved=16, dq=16, dk=16, dv=16, dbeta=16,
+                 dh0=None, ws=16, nbytes=1 << 40)
+        a.update(kw)
+        return _lib.lib.gla_deltanet_bwd_saved(ctypes.byref(p), *(vp(a[n]) for n in names), a["nbytes"], None)
+    need = _lib.lib.gla_deltanet_bwd_workspace_bytes(ctypes.byref(dn()))
+    assert bwd(dn(), saved=40) == _lib.GLA_ERR_INVALID_ARG                   # misaligned
+    assert bwd(dn(), nbytes=need - 1) == _lib.GLA_ERR_WORKSPACE              # the same workspace as without
+    assert bwd(dn(gate=_lib.GLA_GATE_PER_HEAD)) == _lib.GLA_ERR_INVALID_ARG
+    assert bwd(dn(), dv=None) == _lib.GLA_ERR_INVALID_ARG
+    assert bwd(dn(H=0)) == _lib.GLA_OK
+
+
+def test_mlstm_validates_before_launch():
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    ml = lambda **kw: prob(**dict(dict(gate=_lib.GLA_GATE_PER_HEAD, Dk=128, Dv=128, plan=_lib.GLA_PLAN_TC), **kw))
+    wsb = lambda p, bwd: _lib.lib.gla_mlstm_workspace_bytes(ctypes.byref(p), bwd)
+    saved_bytes = lambda p: _lib.lib.gla_mlstm_saved_bytes(ctypes.byref(p))
+    assert wsb(ml(gate=_lib.GLA_GATE_PER_KEY), 0) == 0                  # per-head forget gate only
+    assert wsb(ml(io=9), 1) == 0
+    assert wsb(ml(), 1) >= wsb(ml(), 0) > 0
+    # the forward's results: gate terms, num, den and the normaliser's segment states, plus the
+    # value pass's saved states (tensor-core plan)
+    BH, L = 6, 300
+    assert saved_bytes(ml()) >= BH * L * 128 * 2 + 2 * BH * L * 4
+    assert saved_bytes(ml(plan=_lib.GLA_PLAN_SIMT)) >= BH * L * 128 * 4   # fp32 numerator
+    assert saved_bytes(ml(L=0)) == 0 and saved_bytes(ml(gate=_lib.GLA_GATE_NONE)) == 0
+
+    def fwd(p, **kw):
+        a = dict(q=16, k=16, v=16, g=16, itil=16, h=16, saved=16, ws=16, nbytes=1 << 40)
+        a.update(kw)
+        return _lib.lib.gla_mlstm_fwd_save(ctypes.byref(p), *(vp(a[n]) for n in ("q", "k", "v", "g", "itil", "h",
+                                                                                "saved", "ws")), a["nbytes"], None)
+    assert fwd(ml(), saved=24) == _lib.GLA_ERR_INVALID_ARG                   # misaligned
+    assert fwd(ml(), ws=None) == _lib.GLA_ERR_INVALID_ARG
+    assert fwd(ml(), nbytes=wsb(ml(), 0) - 1) == _lib.GLA_ERR_WORKSPACE
+    assert fwd(ml(), itil=None) == _lib.GLA_ERR_INVALID_ARG
+
+    names = ("q", "k", "v", "g", "itil", "dh", "saved", "dq", "dk", "dv", "dg", "ditil", "ws")
+
+    def bwd(p, **kw):
+        a = dict(q=16, k=16, v=16, g=16, itil=16, dh=16, saved=16, dq=16, dk=16, dv=16, dg=16, ditil=16, ws=16,
+                 nbytes=1 << 40)
+        a.update(kw)
+        return _lib.lib.gla_mlstm_bwd_saved(ctypes.byref(p), *(vp(a[n]) for n in names), a["nbytes"], None)
+    assert bwd(ml(), saved=40) == _lib.GLA_ERR_INVALID_ARG                   # misaligned
+    assert bwd(ml(), nbytes=wsb(ml(), 1) - 1) == _lib.GLA_ERR_WORKSPACE
+    assert bwd(ml(), ditil=None) == _lib.GLA_ERR_INVALID_ARG
+    assert bwd(ml(gate=_lib.GLA_GATE_NONE)) == _lib.GLA_ERR_INVALID_ARG
+
 def test_debug_wait_timeout_validates_before_launch():
     assert _lib.lib.gla_debug_wait_timeout(None, 100, None) == _lib.GLA_ERR_INVALID_ARG
     assert _lib.lib.gla_debug_wait_timeout(ctypes.c_void_p(24), 100, None) == _lib.GLA_ERR_INVALID_ARG  # misaligned

@@ -190,3 +190,49 @@ def test_backward_long_sequence():
 def test_backward_tensor_core_recompute_edges(L):
     """bf16 I/O: the backward's chunk start states come from the tensor-core state walk."""
     check_bwd(1, 2, L, 128, 128, "bf16", 0.5, True, seed=12)
+
+
+@pytest.mark.parametrize("B,H,L,Dk,Dv,dtype", [
+    (2, 1, 300, 128, 128, "bf16"),
+    (1, 2, 65, 64, 192, "bf16"),
+    (1, 2, 150, 64, 64, "f32"),
+    (1, 1, 1, 128, 64, "f32"),
+])
+def test_training_pair_saved_states(B, H, L, Dk, Dv, dtype):
+    """gla_deltanet_fwd_save -> gla_deltanet_bwd_saved: the forward leaves the chunk start states
+    and the backward reads them instead of walking the recurrence again. The states are the ones
+    the backward's own walk writes, so every gradient is bit-identical to the recomputing
+    backward's; both stay within the bound of the oracle."""
+    from linear_rnn_b200 import ops
+    x = I.make_deltanet_inputs(B, H, L, Dk, Dv, dtype, seed=21, h0_std=0.5)
+    gen = torch.Generator().manual_seed(121)
+    dO = torch.randn(B, H, L, Dv, generator=gen).to(x["q"].dtype)
+    dhT = torch.randn(B, H, Dk, Dv, generator=gen)
+    xd = {n: t.cuda() for n, t in x.items()}
+    scale = Dk ** -0.5
+    prob = ops.make_problem(xd["q"], xd["v"], None, scale=scale, chunk=64, plan="auto")
+    nbytes = ops.gla_deltanet_saved_bytes(prob)
+    esize = 2 if dtype == "bf16" else 4
+    assert nbytes == B * H * ((L + 63) // 64) * Dk * Dv * esize
+    saved = torch.full((nbytes,), 0xFF, dtype=torch.uint8, device="cuda")   # NaN pattern until written
+    o1, h1 = ops.gla_deltanet_fwd(xd["q"], xd["k"], xd["v"], xd["beta"], xd["h0"], scale=scale, saved_states=saved)
+    o0, h0 = ops.gla_deltanet_fwd(xd["q"], xd["k"], xd["v"], xd["beta"], xd["h0"], scale=scale)
+    assert torch.equal(o1, o0) and torch.equal(h1, h0)
+    args = (xd["q"], xd["k"], xd["v"], xd["beta"], xd["h0"], dO.cuda(), dhT.cuda())
+    ra = ops.gla_deltanet_bwd(*args, scale=scale, saved_states=saved)
+    rb = ops.gla_deltanet_bwd(*args, scale=scale)
+    for n in ("dq", "dk", "dv", "dbeta", "dh0"):
+        assert torch.equal(ra[n], rb[n]), n
+    ref = DN.deltanet_bwd(x["q"], x["k"], x["v"], x["beta"], x["h0"], dO, dhT, scale)
+    errs = {n: err(f64(ra[n]), ref[n]) for n in ("dq", "dk", "dv", "dbeta", "dh0")}
+    assert all(e <= TOL[dtype] for e in errs.values()), errs
+
+
+def test_training_pair_rejects_short_saved_buffer():
+    from linear_rnn_b200 import ops
+    from linear_rnn_b200._lib import GlaError
+    x = I.make_deltanet_inputs(1, 1, 128, 64, 64, "bf16", seed=3, h0_std=0.0)
+    xd = {n: (None if t is None else t.cuda()) for n, t in x.items()}
+    short = torch.empty(2 * 64 * 64 * 2 - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(GlaError):
+        ops.gla_deltanet_fwd(xd["q"], xd["k"], xd["v"], xd["beta"], None, saved_states=short)
