@@ -28,6 +28,7 @@
 #include <stdint.h>
 
 #include "gla_common.cuh"
+#include "sm100.cuh"
 
 namespace gla {
 namespace {
@@ -64,24 +65,105 @@ __global__ void k_cast(const Tin* __restrict__ a, Tout* __restrict__ b, long n) 
 }
 
 // ---- the normaliser recurrence n_t = e^{g_t} n_{t-1} + i_t k_t, fp32, one thread per key dim,
-// grid (segment, batch*head) with blocks of Dk threads
+// grid (segment, batch*head) with blocks of Dk threads. A segment's rows of q and k (and of the
+// value pass's dq and dk) are contiguous in memory: one bulk copy each brings them into shared
+// memory (one memory round trip per block), and the chains over the segment's tokens, sequential
+// per key dim, read them there. (Loads issued token by token from global memory left these
+// kernels waiting on memory at about a third of the copy bandwidth.) The first warp stages the
+// per-token scalars e^{g_t}, i_t and scale dden_t.
+
+// sum over the block's threads of one value per thread, for token slot j: warp sums into part
+template <int NW>
+__device__ __forceinline__ void ml_warp_part(float x, float (*part)[NW], int j) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    if ((threadIdx.x & 31) == 0) part[j][threadIdx.x >> 5] = x;
+}
+
+// The first warp stages e^{g_t} (se), and where given i_t (si) and scale dden_t (sd), of the
+// segment's cnt <= 32 tokens from row r0; returns the segment's total log-decay (to every lane of
+// warp 0). The caller synchronises before the others read them.
+__device__ __forceinline__ float ml_stage_scalars(const float* __restrict__ g, const float* __restrict__ ig,
+                                                  const float* __restrict__ dd, float scale, long r0, int cnt,
+                                                  float* se, float* si, float* sd) {
+    const int lane = threadIdx.x;
+    const float gj = lane < cnt ? g[r0 + lane] : 0.f;
+    if (lane < cnt) {
+        se[lane] = __expf(gj);
+        if (si) si[lane] = ig[r0 + lane];
+        if (sd) sd[lane] = scale * dd[r0 + lane];
+    }
+    float G = gj;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) G += __shfl_xor_sync(0xffffffffu, G, off);
+    return G;
+}
+
+// Shared-memory layout of a normaliser block: the mbarrier, the scalars and partial sums, then the
+// row tiles (each ML_SL rows of Dk elements, 16-byte aligned).
+struct MlSmem {
+    static constexpr uint32_t BAR = 0;                   // uint64_t
+    static constexpr uint32_t SE = 16;                   // float[ML_SL] each: se, si, sd
+    static constexpr uint32_t SI = SE + 4 * ML_SL;
+    static constexpr uint32_t SD = SI + 4 * ML_SL;
+    static constexpr uint32_t PI = SD + 4 * ML_SL;       // float[ML_SL][8] each: pi, pg
+    static constexpr uint32_t PG = PI + 4 * ML_SL * 8;
+    static constexpr uint32_t TILES = PG + 4 * ML_SL * 8;
+    static_assert(TILES % 16 == 0, "tile alignment");
+};
+__device__ __forceinline__ uint32_t ml_tile_bytes(int Dk, uint32_t esize) { return (uint32_t)ML_SL * Dk * esize; }
+
+// Thread 0 initialises the block's mbarrier; after the block barrier it expects `bytes` and issues
+// the copies (issue()). Everyone then waits (bounded, with the scalars staged in between by the
+// caller); false when the copies did not complete, after setting the status word's timeout bit.
+template <typename Issue>
+__device__ __forceinline__ void ml_tiles_issue(uint64_t* bar, uint32_t bytes, Issue issue) {
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(bar, 1);
+        sm100::mbar_fence_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        sm100::mbar_arrive_expect_tx(bar, bytes);
+        issue();
+    }
+}
+__device__ __forceinline__ bool ml_tiles_wait(uint64_t* bar, int* status) {
+    const bool ok = sm100::mbar_wait(bar, 0);
+    if (__syncthreads_and(ok)) return true;
+    if (threadIdx.x == 0) atomicOr(status, kDevStatusTimeout);
+    return false;
+}
+template <typename T>
+__device__ __forceinline__ void ml_rows_load(T* dst, const T* src, long r0, int cnt, int Dk, uint64_t* bar) {
+    sm100::bulk_load_1d(dst, src + r0 * Dk, (uint32_t)cnt * Dk * (uint32_t)sizeof(T), bar);
+}
 
 // the segment's end state from zero and its total log-decay
 template <typename T>
-__global__ void k_mlstm_nloc(const T* __restrict__ k, const float* __restrict__ g, const float* __restrict__ ig,
-                             int L, int Dk, int nseg, float* __restrict__ nloc, float* __restrict__ gam) {
+__global__ void __launch_bounds__(256) k_mlstm_nloc(const T* __restrict__ k, const float* __restrict__ g,
+                                                    const float* __restrict__ ig, int L, int Dk, int nseg,
+                                                    float* __restrict__ nloc, float* __restrict__ gam, int* status) {
+    extern __shared__ __align__(128) uint8_t ml_dsm[];
+    uint64_t* bar = reinterpret_cast<uint64_t*>(ml_dsm + MlSmem::BAR);
+    float* se = reinterpret_cast<float*>(ml_dsm + MlSmem::SE);
+    float* si = reinterpret_cast<float*>(ml_dsm + MlSmem::SI);
+    const T* sk = reinterpret_cast<const T*>(ml_dsm + MlSmem::TILES);
     const long bh = blockIdx.y;
     const int s = blockIdx.x, d = threadIdx.x;
-    const int t0 = s * ML_SL, t1 = min(L, t0 + ML_SL);
-    float n = 0.f, G = 0.f;
-#pragma unroll 8
-    for (int t = t0; t < t1; ++t) {
-        const float gt = g[bh * L + t];
-        n = __expf(gt) * n + ig[bh * L + t] * to_f(k[(bh * L + t) * Dk + d]);
-        G += gt;
+    const int t0 = s * ML_SL, cnt = min(L - t0, ML_SL);
+    const long r0 = bh * L + t0;
+    ml_tiles_issue(bar, (uint32_t)cnt * Dk * sizeof(T),
+                   [&] { ml_rows_load(const_cast<T*>(sk), k, r0, cnt, Dk, bar); });
+    if (d < 32) {
+        const float G = ml_stage_scalars(g, ig, nullptr, 0.f, r0, cnt, se, si, nullptr);
+        if (d == 0) gam[bh * nseg + s] = G;
     }
+    if (!ml_tiles_wait(bar, status)) return;
+    float n = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < cnt; ++j) n = se[j] * n + si[j] * to_f(sk[j * Dk + d]);
     nloc[(bh * nseg + s) * Dk + d] = n;
-    if (d == 0) gam[bh * nseg + s] = G;
 }
 
 // the state entering every segment (grid batch*head, blocks of Dk threads)
@@ -108,52 +190,65 @@ __global__ void k_mlstm_nscan(const float* __restrict__ nloc, const float* __res
     }
 }
 
-// sum over the block's Dk threads of one value per thread, for token slot j: warp sums into part
-template <int NW>
-__device__ __forceinline__ void ml_warp_part(float x, float (*part)[NW], int j) {
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-    if ((threadIdx.x & 31) == 0) part[j][threadIdx.x >> 5] = x;
-}
-
 // den_t = scale q_t . n_t over the segment (den [BH*L] fp32)
 template <typename T>
-__global__ void k_mlstm_den(const T* __restrict__ q, const T* __restrict__ k, const float* __restrict__ g,
-                            const float* __restrict__ ig, const float* __restrict__ nstart, int L, int Dk, int nseg,
-                            float scale, float* __restrict__ den) {
-    __shared__ float part[ML_SL][8];
+__global__ void __launch_bounds__(256) k_mlstm_den(const T* __restrict__ q, const T* __restrict__ k,
+                                                   const float* __restrict__ g, const float* __restrict__ ig,
+                                                   const float* __restrict__ nstart, int L, int Dk, int nseg,
+                                                   float scale, float* __restrict__ den, int* status) {
+    extern __shared__ __align__(128) uint8_t ml_dsm[];
+    uint64_t* bar = reinterpret_cast<uint64_t*>(ml_dsm + MlSmem::BAR);
+    float* se = reinterpret_cast<float*>(ml_dsm + MlSmem::SE);
+    float* si = reinterpret_cast<float*>(ml_dsm + MlSmem::SI);
+    float(*part)[8] = reinterpret_cast<float(*)[8]>(ml_dsm + MlSmem::PI);
+    const T* sq = reinterpret_cast<const T*>(ml_dsm + MlSmem::TILES);
+    const T* sk = reinterpret_cast<const T*>(ml_dsm + MlSmem::TILES + ml_tile_bytes(Dk, sizeof(T)));
     const long bh = blockIdx.y;
     const int s = blockIdx.x, d = threadIdx.x, nw = Dk / 32;
     const int t0 = s * ML_SL, cnt = min(L - t0, ML_SL);
+    const long r0 = bh * L + t0;
+    ml_tiles_issue(bar, 2u * cnt * Dk * sizeof(T), [&] {
+        ml_rows_load(const_cast<T*>(sq), q, r0, cnt, Dk, bar);
+        ml_rows_load(const_cast<T*>(sk), k, r0, cnt, Dk, bar);
+    });
+    if (d < 32) ml_stage_scalars(g, ig, nullptr, 0.f, r0, cnt, se, si, nullptr);
     float n = nstart[(bh * nseg + s) * Dk + d];
+    if (!ml_tiles_wait(bar, status)) return;
 #pragma unroll 4
     for (int j = 0; j < cnt; ++j) {
-        const long r = bh * L + t0 + j;
-        n = __expf(g[r]) * n + ig[r] * to_f(k[r * Dk + d]);
-        ml_warp_part<8>(to_f(q[r * Dk + d]) * n, part, j);
+        n = se[j] * n + si[j] * to_f(sk[j * Dk + d]);
+        ml_warp_part<8>(to_f(sq[j * Dk + d]) * n, part, j);
     }
     __syncthreads();
     if (d < cnt) {
         float x = 0.f;
         for (int w = 0; w < nw; ++w) x += part[d][w];
-        den[bh * L + t0 + d] = scale * x;
+        den[r0 + d] = scale * x;
     }
 }
 
 // backward, local: the gradient carried out of the segment's start from a zero carry at its end,
 // c = e^{g_t} dn_t with dn_t = scale dden_t q_t + c (walking the segment backwards)
 template <typename T>
-__global__ void k_mlstm_dnloc(const T* __restrict__ q, const float* __restrict__ g, const float* __restrict__ dden,
-                              int L, int Dk, int nseg, float scale, float* __restrict__ cloc) {
+__global__ void __launch_bounds__(256) k_mlstm_dnloc(const T* __restrict__ q, const float* __restrict__ g,
+                                                     const float* __restrict__ dden, int L, int Dk, int nseg,
+                                                     float scale, float* __restrict__ cloc, int* status) {
+    extern __shared__ __align__(128) uint8_t ml_dsm[];
+    uint64_t* bar = reinterpret_cast<uint64_t*>(ml_dsm + MlSmem::BAR);
+    float* se = reinterpret_cast<float*>(ml_dsm + MlSmem::SE);
+    float* sd = reinterpret_cast<float*>(ml_dsm + MlSmem::SD);
+    const T* sq = reinterpret_cast<const T*>(ml_dsm + MlSmem::TILES);
     const long bh = blockIdx.y;
     const int s = blockIdx.x, d = threadIdx.x;
-    const int t0 = s * ML_SL, t1 = min(L, t0 + ML_SL);
+    const int t0 = s * ML_SL, cnt = min(L - t0, ML_SL);
+    const long r0 = bh * L + t0;
+    ml_tiles_issue(bar, (uint32_t)cnt * Dk * sizeof(T),
+                   [&] { ml_rows_load(const_cast<T*>(sq), q, r0, cnt, Dk, bar); });
+    if (d < 32) ml_stage_scalars(g, nullptr, dden, scale, r0, cnt, se, nullptr, sd);
+    if (!ml_tiles_wait(bar, status)) return;
     float c = 0.f;
 #pragma unroll 8
-    for (int t = t1 - 1; t >= t0; --t) {
-        const long r = bh * L + t;
-        c = __expf(g[r]) * (scale * dden[r] * to_f(q[r * Dk + d]) + c);
-    }
+    for (int j = cnt - 1; j >= 0; --j) c = se[j] * (sd[j] * to_f(sq[j * Dk + d]) + c);
     cloc[(bh * nseg + s) * Dk + d] = c;
 }
 
@@ -184,37 +279,60 @@ __global__ void k_mlstm_cscan(const float* __restrict__ cloc, const float* __res
 // the normaliser's gradients over a segment: n_t forward from the segment's start state (kept in
 // shared memory), then dn_t backwards from the carry entering the segment's end. They are added
 // to the value pass's in the same step: dq = dq1 + scale dden n_t and dk = dk1 + i_t dn_t in the
-// output dtype (dq1 / dk1 may be the outputs themselves), dg += (n_t - i_t k_t) . dn_t and
-// d i~ = (di1 + k_t . dn_t) i_t.
+// output dtype (dq1 / dk1 may be the outputs themselves: each thread reads its element of a row
+// before it writes it), dg += (n_t - i_t k_t) . dn_t and d i~ = (di1 + k_t . dn_t) i_t. The
+// segment's rows of q, k, dq1 and dk1 come into shared memory by bulk copies.
 template <typename T, typename Ta>
-__global__ void k_mlstm_den_bwd(const T* __restrict__ q, const T* __restrict__ k, const float* __restrict__ g,
-                                const float* __restrict__ ig, const float* __restrict__ dden,
-                                const float* __restrict__ nstart, const float* __restrict__ cin, int L, int Dk, int nseg,
-                                float scale, const Ta* dq1, const Ta* dk1, T* dq, T* dk, float* __restrict__ dg,
-                                const float* __restrict__ di1, float* __restrict__ ditil) {
-    __shared__ float pi[ML_SL][8], pg[ML_SL][8];
-    __shared__ float nv[ML_SL][256];   // n_t of the segment's tokens, [token][key dim]
+__global__ void __launch_bounds__(256) k_mlstm_den_bwd(const T* __restrict__ q, const T* __restrict__ k,
+                                                       const float* __restrict__ g, const float* __restrict__ ig,
+                                                       const float* __restrict__ dden,
+                                                       const float* __restrict__ nstart, const float* __restrict__ cin,
+                                                       int L, int Dk, int nseg, float scale, const Ta* dq1,
+                                                       const Ta* dk1, T* dq, T* dk, float* __restrict__ dg,
+                                                       const float* __restrict__ di1, float* __restrict__ ditil,
+                                                       int* status) {
+    extern __shared__ __align__(128) uint8_t ml_dsm[];
+    uint64_t* bar = reinterpret_cast<uint64_t*>(ml_dsm + MlSmem::BAR);
+    float* se = reinterpret_cast<float*>(ml_dsm + MlSmem::SE);
+    float* si = reinterpret_cast<float*>(ml_dsm + MlSmem::SI);
+    float* sd = reinterpret_cast<float*>(ml_dsm + MlSmem::SD);
+    float(*pi)[8] = reinterpret_cast<float(*)[8]>(ml_dsm + MlSmem::PI);
+    float(*pg)[8] = reinterpret_cast<float(*)[8]>(ml_dsm + MlSmem::PG);
+    const uint32_t tb = ml_tile_bytes(Dk, sizeof(T)), ta = ml_tile_bytes(Dk, sizeof(Ta));
+    const T* sq = reinterpret_cast<const T*>(ml_dsm + MlSmem::TILES);
+    const T* sk = reinterpret_cast<const T*>(ml_dsm + MlSmem::TILES + tb);
+    const Ta* sa = reinterpret_cast<const Ta*>(ml_dsm + MlSmem::TILES + 2 * tb);
+    const Ta* sb = reinterpret_cast<const Ta*>(ml_dsm + MlSmem::TILES + 2 * tb + ta);
+    float* nv = reinterpret_cast<float*>(ml_dsm + MlSmem::TILES + 2 * tb + 2 * ta);   // n_t, [token][key dim]
     const long bh = blockIdx.y;
     const int s = blockIdx.x, d = threadIdx.x, nw = Dk / 32;
     const int t0 = s * ML_SL, cnt = min(L - t0, ML_SL);
     const long r0 = bh * L + t0;
+    ml_tiles_issue(bar, 2u * cnt * Dk * (uint32_t)(sizeof(T) + sizeof(Ta)), [&] {
+        ml_rows_load(const_cast<T*>(sq), q, r0, cnt, Dk, bar);
+        ml_rows_load(const_cast<T*>(sk), k, r0, cnt, Dk, bar);
+        ml_rows_load(const_cast<Ta*>(sa), dq1, r0, cnt, Dk, bar);
+        ml_rows_load(const_cast<Ta*>(sb), dk1, r0, cnt, Dk, bar);
+    });
+    if (d < 32) ml_stage_scalars(g, ig, dden, scale, r0, cnt, se, si, sd);
     float n = nstart[(bh * nseg + s) * Dk + d];
+    float c = cin[(bh * nseg + s) * Dk + d];
+    if (!ml_tiles_wait(bar, status)) return;
 #pragma unroll 8
     for (int j = 0; j < cnt; ++j) {
-        n = __expf(g[r0 + j]) * n + ig[r0 + j] * to_f(k[(r0 + j) * Dk + d]);
-        nv[j][d] = n;
+        n = se[j] * n + si[j] * to_f(sk[j * Dk + d]);
+        nv[j * Dk + d] = n;
     }
-    float c = cin[(bh * nseg + s) * Dk + d];
 #pragma unroll 4
     for (int j = cnt - 1; j >= 0; --j) {
-        const long r = r0 + j;
-        const float sd = scale * dden[r], it = ig[r], kt = to_f(k[r * Dk + d]), nj = nv[j][d];
-        const float dn = sd * to_f(q[r * Dk + d]) + c;
-        dq[r * Dk + d] = from_f<T>(to_f(dq1[r * Dk + d]) + sd * nj);
-        dk[r * Dk + d] = from_f<T>(to_f(dk1[r * Dk + d]) + it * dn);
+        const long o = (r0 + j) * Dk + d;
+        const float sdj = sd[j], it = si[j], kt = to_f(sk[j * Dk + d]), nj = nv[j * Dk + d];
+        const float dn = sdj * to_f(sq[j * Dk + d]) + c;
+        dq[o] = from_f<T>(to_f(sa[j * Dk + d]) + sdj * nj);
+        dk[o] = from_f<T>(to_f(sb[j * Dk + d]) + it * dn);
         ml_warp_part<8>(kt * dn, pi, j);
         ml_warp_part<8>((nj - it * kt) * dn, pg, j);
-        c = __expf(g[r]) * dn;
+        c = se[j] * dn;
     }
     __syncthreads();
     if (d < cnt) {
@@ -224,11 +342,50 @@ __global__ void k_mlstm_den_bwd(const T* __restrict__ q, const T* __restrict__ k
             xg += pg[d][w];
         }
         dg[r0 + d] += xg;
-        ditil[r0 + d] = (di1[r0 + d] + xi) * ig[r0 + d];
+        ditil[r0 + d] = (di1[r0 + d] + xi) * si[d];
     }
 }
 
-// One warp per token row: N = max(|den|, e^{-c}), h = num / N.
+// dynamic shared memory of the normaliser kernels: the fixed part and `tiles` row tiles of esize
+// bytes per element (den_bwd: plus its fp32 n_t tile)
+inline size_t ml_smem_bytes(int Dk, size_t tile_elem_bytes) {
+    return MlSmem::TILES + (size_t)ML_SL * Dk * tile_elem_bytes;
+}
+template <typename K>
+inline cudaError_t ml_smem_attr(K kern, size_t bytes) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+// Eight consecutive elements (16 bytes of bf16, 32 of fp32) to / from fp32.
+__device__ __forceinline__ void ld8(const float* p, float* f) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+__device__ __forceinline__ void ld8(const __nv_bfloat16* p, float* f) {
+    const uint4 w = *reinterpret_cast<const uint4*>(p);
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[i]));
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+__device__ __forceinline__ void st8(float* p, const float* f) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(f[0], f[1], f[2], f[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(f[4], f[5], f[6], f[7]);
+}
+__device__ __forceinline__ void st8(__nv_bfloat16* p, const float* f) {
+    uint32_t u[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 x = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+        u[i] = *reinterpret_cast<const uint32_t*>(&x);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(u[0], u[1], u[2], u[3]);
+}
+
+// One warp per token row (eight elements a lane at a time): N = max(|den|, e^{-c}), h = num / N.
 template <typename Ta, typename To>
 __global__ void __launch_bounds__(ML_NT) k_mlstm_norm(const Ta* __restrict__ num, const float* __restrict__ den,
                                                       const float* __restrict__ cst, To* __restrict__ h, long rows,
@@ -238,10 +395,17 @@ __global__ void __launch_bounds__(ML_NT) k_mlstm_norm(const Ta* __restrict__ num
     if (row >= rows) return;
     const float N = fmaxf(fabsf(den[row]), expf(-cst[row / L]));
     const float inv = 1.f / N;
-    for (int e = lane; e < Dv; e += 32) h[row * Dv + e] = from_f<To>(ld_f(num + row * Dv + e) * inv);
+    for (int e = 8 * lane; e < Dv; e += 256) {
+        float f[8];
+        ld8(num + row * Dv + e, f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] *= inv;
+        st8(h + row * Dv + e, f);
+    }
 }
 
-// One warp per token row: the upstream gradients of the two sums.
+// One warp per token row (eight elements a lane at a time): the upstream gradients of the two
+// sums.
 template <typename Ta, typename To>
 __global__ void __launch_bounds__(ML_NT) k_mlstm_bwd_prep(const Ta* __restrict__ num, const float* __restrict__ den,
                                                           const float* __restrict__ cst, const To* __restrict__ dh,
@@ -255,10 +419,16 @@ __global__ void __launch_bounds__(ML_NT) k_mlstm_bwd_prep(const Ta* __restrict__
     const float N = fmaxf(fabsf(dn), bound);
     const float inv = 1.f / N;
     float s = 0.f;   // dh . h
-    for (int e = lane; e < Dv; e += 32) {
-        const float d = ld_f(dh + row * Dv + e);
-        s += d * ld_f(num + row * Dv + e) * inv;
-        dnum[row * Dv + e] = from_f<Ta>(d * inv);
+    for (int e = 8 * lane; e < Dv; e += 256) {
+        float d[8], x[8];
+        ld8(dh + row * Dv + e, d);
+        ld8(num + row * Dv + e, x);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            s += d[i] * x[i] * inv;
+            d[i] *= inv;
+        }
+        st8(dnum + row * Dv + e, d);
     }
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
@@ -430,10 +600,21 @@ gla_status ml_forward_passes(const gla_problem* p, const MlLayout& w, const MlIn
     const To* tk = static_cast<const To*>(k);
     float* nloc = reinterpret_cast<float*>(ws + w.o_nloc);
     const dim3 grid(w.nseg, (unsigned)BH);
-    GLA_LAUNCH("mlstm_nloc", st, k_mlstm_nloc<To><<<grid, p->Dk, 0, st>>>(tk, g, r.ig, p->L, p->Dk, w.nseg, nloc, r.gam));
+    int* status = reinterpret_cast<int*>(ws);
+    const size_t s1 = ml_smem_bytes(p->Dk, sizeof(To)), s2 = ml_smem_bytes(p->Dk, 2 * sizeof(To));
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t ea = ml_smem_attr(k_mlstm_nloc<To>, ml_smem_bytes(256, sizeof(To)));
+        if (ea == cudaSuccess) ea = ml_smem_attr(k_mlstm_den<To>, ml_smem_bytes(256, 2 * sizeof(To)));
+        if (ea != cudaSuccess) return record_cuda(ea, "mLSTM normaliser shared-memory attribute");
+        attr = true;
+    }
+    GLA_LAUNCH("mlstm_nloc", st,
+               k_mlstm_nloc<To><<<grid, p->Dk, s1, st>>>(tk, g, r.ig, p->L, p->Dk, w.nseg, nloc, r.gam, status));
     GLA_LAUNCH("mlstm_nscan", st, k_mlstm_nscan<<<(unsigned)BH, p->Dk, 0, st>>>(nloc, r.gam, w.nseg, p->Dk, r.nst));
     GLA_LAUNCH("mlstm_den", st,
-               k_mlstm_den<To><<<grid, p->Dk, 0, st>>>(tq, tk, g, r.ig, r.nst, p->L, p->Dk, w.nseg, p->scale, r.den));
+               k_mlstm_den<To><<<grid, p->Dk, s2, st>>>(tq, tk, g, r.ig, r.nst, p->L, p->Dk, w.nseg, p->scale, r.den,
+                                                        status));
     return record_cuda(cudaGetLastError(), "mLSTM normaliser launch");
 }
 
@@ -495,15 +676,27 @@ gla_status ml_bwd(const gla_problem* p, const MlLayout& w, const void* q, const 
         float* cloc = reinterpret_cast<float*>(ws + w.o_cloc);
         float* cin = reinterpret_cast<float*>(ws + w.o_cin);
         const dim3 grid(w.nseg, (unsigned)BH);
+        int* status = reinterpret_cast<int*>(ws);
+        const size_t s1 = ml_smem_bytes(p->Dk, sizeof(To));
+        const size_t sb = ml_smem_bytes(p->Dk, 2 * sizeof(To) + 2 * sizeof(Ta) + sizeof(float));
+        static bool attr = false;
+        if (!attr) {
+            cudaError_t ea = ml_smem_attr(k_mlstm_dnloc<To>, ml_smem_bytes(256, sizeof(To)));
+            if (ea == cudaSuccess)
+                ea = ml_smem_attr(k_mlstm_den_bwd<To, Ta>,
+                                  ml_smem_bytes(256, 2 * sizeof(To) + 2 * sizeof(Ta) + sizeof(float)));
+            if (ea != cudaSuccess) return record_cuda(ea, "mLSTM normaliser shared-memory attribute");
+            attr = true;
+        }
         GLA_LAUNCH("mlstm_dnloc", st,
-                   k_mlstm_dnloc<To><<<grid, p->Dk, 0, st>>>(tq, g, dden, p->L, p->Dk, w.nseg, p->scale, cloc));
+                   k_mlstm_dnloc<To><<<grid, p->Dk, s1, st>>>(tq, g, dden, p->L, p->Dk, w.nseg, p->scale, cloc, status));
         GLA_LAUNCH("mlstm_cscan", st,
                    k_mlstm_cscan<<<(unsigned)BH, p->Dk, 0, st>>>(cloc, r.gam, w.nseg, p->Dk, cin));
         GLA_LAUNCH("mlstm_den_bwd", st,
-                   (k_mlstm_den_bwd<To, Ta><<<grid, p->Dk, 0, st>>>(
+                   (k_mlstm_den_bwd<To, Ta><<<grid, p->Dk, sb, st>>>(
                        tq, tk, g, ig, dden, r.nst, cin, p->L, p->Dk, w.nseg,
                        p->scale, static_cast<const Ta*>(dq1), static_cast<const Ta*>(dk1), static_cast<To*>(dq),
-                       static_cast<To*>(dk), dg, di1, ditil)));
+                       static_cast<To*>(dk), dg, di1, ditil, status)));
         if ((e = cudaGetLastError()) != cudaSuccess) return record_cuda(e, "mLSTM normaliser backward launch");
     }
     if (w.cast_a) {   // dv of the fp32 value pass, cast back

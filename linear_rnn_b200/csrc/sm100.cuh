@@ -199,14 +199,22 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c
                  : "memory");
 }
 
-// Tiled TMA store of a shared-memory tile (same box and swizzle as the tensor map) to
-// global memory, tracked as a bulk group of the issuing thread. Rows outside the tensor
-// are not written.
+// Untiled bulk copy of a contiguous global range into this CTA's shared memory (both addresses
+// 16-byte aligned, bytes a multiple of 16; no multicast), completion counted on `bar` in bytes.
+__device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
 // Contiguous global range into L2 (bytes a multiple of 16, address 16-byte aligned).
 __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
                  : "memory");
 }
+// Tiled TMA store of a shared-memory tile (same box and swizzle as the tensor map) to
+// global memory, tracked as a bulk group of the issuing thread. Rows outside the tensor
+// are not written.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
     asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
                      reinterpret_cast<uint64_t>(map)),
