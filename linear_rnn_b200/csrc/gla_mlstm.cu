@@ -166,28 +166,65 @@ __global__ void __launch_bounds__(256) k_mlstm_nloc(const T* __restrict__ k, con
     nloc[(bh * nseg + s) * Dk + d] = n;
 }
 
-// the state entering every segment (grid batch*head, blocks of Dk threads)
-__global__ void k_mlstm_nscan(const float* __restrict__ nloc, const float* __restrict__ gam, int nseg, int Dk,
-                              float* __restrict__ nstart) {
-    const long bh = blockIdx.x;
-    const int d = threadIdx.x;
-    // loads of 16 segments at a time go out before the chain that uses them
-    float n = 0.f;
-    for (int s0 = 0; s0 < nseg; s0 += 16) {
-        float nl[16], ga[16];
+// The two scans over segments run in two levels, groups of ML_SG segments: a first kernel scans
+// every group from zero (all groups in parallel) and leaves its total, a second carries the
+// totals of the groups before (after) each group into it and adds them to its segments. (One
+// block per head walking all segments in order ran only B*H blocks.)
+constexpr int ML_SG = 16;
+
+// the state entering every segment of a group from a zero state at the group's start, and the
+// group's end state and total log-decay (grid (group, batch*head), blocks of Dk threads)
+__global__ void k_mlstm_nscan_local(const float* __restrict__ nloc, const float* __restrict__ gam, int nseg, int Dk,
+                                    float* __restrict__ nstart, float* __restrict__ gst, float* __restrict__ ggam) {
+    const long bh = blockIdx.y;
+    const int gi = blockIdx.x, ng = gridDim.x, d = threadIdx.x;
+    const int s0 = gi * ML_SG, cnt = min(nseg - s0, ML_SG);
+    float nl[ML_SG], ga[ML_SG];
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
-            if (s0 + u < nseg) {
-                nl[u] = nloc[(bh * nseg + s0 + u) * Dk + d];
-                ga[u] = gam[bh * nseg + s0 + u];
+    for (int u = 0; u < ML_SG; ++u)
+        if (u < cnt) {
+            nl[u] = nloc[(bh * nseg + s0 + u) * Dk + d];
+            ga[u] = gam[bh * nseg + s0 + u];
+        }
+    float n = 0.f, G = 0.f;
+#pragma unroll
+    for (int u = 0; u < ML_SG; ++u)
+        if (u < cnt) {
+            nstart[(bh * nseg + s0 + u) * Dk + d] = n;
+            n = __expf(ga[u]) * n + nl[u];
+            G += ga[u];
+        }
+    gst[(bh * ng + gi) * Dk + d] = n;
+    if (d == 0) ggam[bh * ng + gi] = G;
+}
+
+// the state entering group gi from the groups before it, carried into its segments
+__global__ void k_mlstm_nscan_fix(const float* __restrict__ gam, const float* __restrict__ gst,
+                                  const float* __restrict__ ggam, int nseg, int Dk, float* __restrict__ nstart) {
+    const long bh = blockIdx.y;
+    const int gi = blockIdx.x, ng = gridDim.x, d = threadIdx.x;
+    if (gi == 0) return;   // the first group starts from the zero state
+    float e = 0.f;   // groups 0 .. gi-1 in order, their totals loaded ML_SG at a time
+    for (int b0 = 0; b0 < gi; b0 += ML_SG) {
+        float gs[ML_SG], gg[ML_SG];
+#pragma unroll
+        for (int u = 0; u < ML_SG; ++u)
+            if (b0 + u < gi) {
+                gs[u] = gst[(bh * ng + b0 + u) * Dk + d];
+                gg[u] = ggam[bh * ng + b0 + u];
             }
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
-            if (s0 + u < nseg) {
-                nstart[(bh * nseg + s0 + u) * Dk + d] = n;
-                n = __expf(ga[u]) * n + nl[u];
-            }
+        for (int u = 0; u < ML_SG; ++u)
+            if (b0 + u < gi) e = __expf(gg[u]) * e + gs[u];
     }
+    const int s0 = gi * ML_SG, cnt = min(nseg - s0, ML_SG);
+    float D = 1.f;   // decay from the group's start to the segment
+#pragma unroll
+    for (int u = 0; u < ML_SG; ++u)
+        if (u < cnt) {
+            nstart[(bh * nseg + s0 + u) * Dk + d] += D * e;
+            D *= __expf(gam[bh * nseg + s0 + u]);
+        }
 }
 
 // den_t = scale q_t . n_t over the segment (den [BH*L] fp32)
@@ -252,28 +289,59 @@ __global__ void __launch_bounds__(256) k_mlstm_dnloc(const T* __restrict__ q, co
     cloc[(bh * nseg + s) * Dk + d] = c;
 }
 
-// the carry entering every segment from the segments after it (grid batch*head)
-__global__ void k_mlstm_cscan(const float* __restrict__ cloc, const float* __restrict__ gam, int nseg, int Dk,
-                              float* __restrict__ cin) {
-    const long bh = blockIdx.x;
-    const int d = threadIdx.x;
-    // loads of 16 segments at a time go out before the chain that uses them
-    float c = 0.f;
-    for (int s1 = nseg - 1; s1 >= 0; s1 -= 16) {
-        float cl[16], ga[16];
+// the carry entering every segment of a group from a zero carry at the group's end, and the
+// carry out of the group's start and its total log-decay (grid (group, batch*head))
+__global__ void k_mlstm_cscan_local(const float* __restrict__ cloc, const float* __restrict__ gam, int nseg, int Dk,
+                                    float* __restrict__ cin, float* __restrict__ gst, float* __restrict__ ggam) {
+    const long bh = blockIdx.y;
+    const int gi = blockIdx.x, ng = gridDim.x, d = threadIdx.x;
+    const int s0 = gi * ML_SG, cnt = min(nseg - s0, ML_SG);
+    float cl[ML_SG], ga[ML_SG];
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
-            if (s1 - u >= 0) {
-                cl[u] = cloc[(bh * nseg + s1 - u) * Dk + d];
-                ga[u] = gam[bh * nseg + s1 - u];
+    for (int u = 0; u < ML_SG; ++u)
+        if (u < cnt) {
+            cl[u] = cloc[(bh * nseg + s0 + u) * Dk + d];
+            ga[u] = gam[bh * nseg + s0 + u];
+        }
+    float c = 0.f, G = 0.f;
+#pragma unroll
+    for (int u = ML_SG - 1; u >= 0; --u)
+        if (u < cnt) {
+            cin[(bh * nseg + s0 + u) * Dk + d] = c;
+            c = __expf(ga[u]) * c + cl[u];
+            G += ga[u];
+        }
+    gst[(bh * ng + gi) * Dk + d] = c;
+    if (d == 0) ggam[bh * ng + gi] = G;
+}
+
+// the carry entering group gi's end from the groups after it, carried into its segments
+__global__ void k_mlstm_cscan_fix(const float* __restrict__ gam, const float* __restrict__ gst,
+                                  const float* __restrict__ ggam, int nseg, int Dk, float* __restrict__ cin) {
+    const long bh = blockIdx.y;
+    const int gi = blockIdx.x, ng = gridDim.x, d = threadIdx.x;
+    if (gi == ng - 1) return;   // nothing comes after the last group
+    float e = 0.f;   // groups ng-1 .. gi+1 in reverse order, their totals loaded ML_SG at a time
+    for (int b1 = ng - 1; b1 > gi; b1 -= ML_SG) {
+        float gs[ML_SG], gg[ML_SG];
+#pragma unroll
+        for (int u = 0; u < ML_SG; ++u)
+            if (b1 - u > gi) {
+                gs[u] = gst[(bh * ng + b1 - u) * Dk + d];
+                gg[u] = ggam[bh * ng + b1 - u];
             }
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
-            if (s1 - u >= 0) {
-                cin[(bh * nseg + s1 - u) * Dk + d] = c;
-                c = __expf(ga[u]) * c + cl[u];
-            }
+        for (int u = 0; u < ML_SG; ++u)
+            if (b1 - u > gi) e = __expf(gg[u]) * e + gs[u];
     }
+    const int s0 = gi * ML_SG, cnt = min(nseg - s0, ML_SG);
+    float D = 1.f;   // decay from the group's end back to the segment
+#pragma unroll
+    for (int u = ML_SG - 1; u >= 0; --u)
+        if (u < cnt) {
+            cin[(bh * nseg + s0 + u) * Dk + d] += D * e;
+            D *= __expf(gam[bh * nseg + s0 + u]);
+        }
 }
 
 // the normaliser's gradients over a segment: n_t forward from the segment's start state (kept in
@@ -444,7 +512,8 @@ struct MlLayout {
                           // cast back
     int nseg;             // 32-token segments of the normaliser recurrence
     size_t wsa;           // the value pass's workspace bytes
-    size_t o_qf, o_kf, o_vf, o_nloc;
+    int ngrp;             // groups of ML_SG segments of the two-level scans over segments
+    size_t o_qf, o_kf, o_vf, o_nloc, o_gst, o_ggam;
     size_t o_dnum, o_dden, o_dq1, o_dk1, o_dv1, o_di1, o_cloc, o_cin;
     size_t o_res;         // the forward's results (MlRes) when they live in the workspace
     size_t total;
@@ -512,6 +581,9 @@ gla_status ml_layout(const gla_problem* p, bool bwd, MlLayout* w) {
         w->o_vf = take(4 * BHL * p->Dv);
     }
     w->o_nloc = take(4 * NS * p->Dk);
+    w->ngrp = (w->nseg + ML_SG - 1) / ML_SG;
+    w->o_gst = take(4 * BH * (size_t)w->ngrp * p->Dk);
+    w->o_ggam = take(4 * BH * (size_t)w->ngrp);
     if (bwd) {
         w->o_dnum = take(ea * BHL * p->Dv);
         w->o_dden = take(4 * BHL);
@@ -611,7 +683,12 @@ gla_status ml_forward_passes(const gla_problem* p, const MlLayout& w, const MlIn
     }
     GLA_LAUNCH("mlstm_nloc", st,
                k_mlstm_nloc<To><<<grid, p->Dk, s1, st>>>(tk, g, r.ig, p->L, p->Dk, w.nseg, nloc, r.gam, status));
-    GLA_LAUNCH("mlstm_nscan", st, k_mlstm_nscan<<<(unsigned)BH, p->Dk, 0, st>>>(nloc, r.gam, w.nseg, p->Dk, r.nst));
+    float* gst = reinterpret_cast<float*>(ws + w.o_gst);
+    float* ggam = reinterpret_cast<float*>(ws + w.o_ggam);
+    const dim3 ggrid(w.ngrp, (unsigned)BH);
+    GLA_LAUNCH("mlstm_nscan", st,
+               k_mlstm_nscan_local<<<ggrid, p->Dk, 0, st>>>(nloc, r.gam, w.nseg, p->Dk, r.nst, gst, ggam));
+    GLA_LAUNCH("mlstm_nscan", st, k_mlstm_nscan_fix<<<ggrid, p->Dk, 0, st>>>(r.gam, gst, ggam, w.nseg, p->Dk, r.nst));
     GLA_LAUNCH("mlstm_den", st,
                k_mlstm_den<To><<<grid, p->Dk, s2, st>>>(tq, tk, g, r.ig, r.nst, p->L, p->Dk, w.nseg, p->scale, r.den,
                                                         status));
@@ -690,8 +767,13 @@ gla_status ml_bwd(const gla_problem* p, const MlLayout& w, const void* q, const 
         }
         GLA_LAUNCH("mlstm_dnloc", st,
                    k_mlstm_dnloc<To><<<grid, p->Dk, s1, st>>>(tq, g, dden, p->L, p->Dk, w.nseg, p->scale, cloc, status));
+        float* gst = reinterpret_cast<float*>(ws + w.o_gst);
+        float* ggam = reinterpret_cast<float*>(ws + w.o_ggam);
+        const dim3 ggrid(w.ngrp, (unsigned)BH);
         GLA_LAUNCH("mlstm_cscan", st,
-                   k_mlstm_cscan<<<(unsigned)BH, p->Dk, 0, st>>>(cloc, r.gam, w.nseg, p->Dk, cin));
+                   k_mlstm_cscan_local<<<ggrid, p->Dk, 0, st>>>(cloc, r.gam, w.nseg, p->Dk, cin, gst, ggam));
+        GLA_LAUNCH("mlstm_cscan", st,
+                   k_mlstm_cscan_fix<<<ggrid, p->Dk, 0, st>>>(r.gam, gst, ggam, w.nseg, p->Dk, cin));
         GLA_LAUNCH("mlstm_den_bwd", st,
                    (k_mlstm_den_bwd<To, Ta><<<grid, p->Dk, sb, st>>>(
                        tq, tk, g, ig, dden, r.nst, cin, p->L, p->Dk, w.nseg,

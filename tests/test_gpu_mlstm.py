@@ -109,16 +109,17 @@ def test_tensor_core_value_pass_c5_shape(L):
     record(f"mlstm tc plan L={L}", errs)
 
 
-@pytest.mark.parametrize("L", [31, 32, 33, 97])
+@pytest.mark.parametrize("L", [31, 32, 33, 97, 600])
 def test_normaliser_segment_edges(L):
-    """Sequences that end inside, at and just past a 32-token segment of the normaliser recurrence."""
+    """Sequences that end inside, at and just past a 32-token segment of the normaliser recurrence
+    (600 tokens: 19 segments, past a group of 16 in the scans over segments)."""
     run(I.MLSTM.replace(B=1, H=3, L=L, Dk=64, Dv=64, scale=0.125), seed=9)
 
 
-@pytest.mark.parametrize("L", [1, 33, 257])
+@pytest.mark.parametrize("L", [1, 33, 257, 1500])
 def test_normaliser_segment_edges_fp32(L):
     """fp32 I/O (both sums on the CUDA cores in fp32) at 1e-4, across segment edges and the
-    segment scans."""
+    segment scans (1500 tokens: 47 segments, groups of 16, 16 and 15 in the two-level scans)."""
     run(I.MLSTM.replace(B=2, H=1, L=L, Dk=128, Dv=64, dtype="f32", scale=128 ** -0.5), seed=13)
 
 
