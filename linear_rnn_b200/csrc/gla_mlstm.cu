@@ -345,7 +345,7 @@ __global__ void k_mlstm_cscan_fix(const float* __restrict__ gam, const float* __
 }
 
 // the normaliser's gradients over a segment: n_t forward from the segment's start state (kept in
-// shared memory), then dn_t backwards from the carry entering the segment's end. They are added
+// registers), then dn_t backwards from the carry entering the segment's end. They are added
 // to the value pass's in the same step: dq = dq1 + scale dden n_t and dk = dk1 + i_t dn_t in the
 // output dtype (dq1 / dk1 may be the outputs themselves: each thread reads its element of a row
 // before it writes it), dg += (n_t - i_t k_t) . dn_t and d i~ = (di1 + k_t . dn_t) i_t. The
@@ -371,7 +371,6 @@ __global__ void __launch_bounds__(256) k_mlstm_den_bwd(const T* __restrict__ q, 
     const T* sk = reinterpret_cast<const T*>(ml_dsm + MlSmem::TILES + tb);
     const Ta* sa = reinterpret_cast<const Ta*>(ml_dsm + MlSmem::TILES + 2 * tb);
     const Ta* sb = reinterpret_cast<const Ta*>(ml_dsm + MlSmem::TILES + 2 * tb + ta);
-    float* nv = reinterpret_cast<float*>(ml_dsm + MlSmem::TILES + 2 * tb + 2 * ta);   // n_t, [token][key dim]
     const long bh = blockIdx.y;
     const int s = blockIdx.x, d = threadIdx.x, nw = Dk / 32;
     const int t0 = s * ML_SL, cnt = min(L - t0, ML_SL);
@@ -386,22 +385,25 @@ __global__ void __launch_bounds__(256) k_mlstm_den_bwd(const T* __restrict__ q, 
     float n = nstart[(bh * nseg + s) * Dk + d];
     float c = cin[(bh * nseg + s) * Dk + d];
     if (!ml_tiles_wait(bar, status)) return;
-#pragma unroll 8
-    for (int j = 0; j < cnt; ++j) {
-        n = se[j] * n + si[j] * to_f(sk[j * Dk + d]);
-        nv[j * Dk + d] = n;
-    }
-#pragma unroll 4
-    for (int j = cnt - 1; j >= 0; --j) {
-        const long o = (r0 + j) * Dk + d;
-        const float sdj = sd[j], it = si[j], kt = to_f(sk[j * Dk + d]), nj = nv[j * Dk + d];
-        const float dn = sdj * to_f(sq[j * Dk + d]) + c;
-        dq[o] = from_f<T>(to_f(sa[j * Dk + d]) + sdj * nj);
-        dk[o] = from_f<T>(to_f(sb[j * Dk + d]) + it * dn);
-        ml_warp_part<8>(kt * dn, pi, j);
-        ml_warp_part<8>((nj - it * kt) * dn, pg, j);
-        c = se[j] * dn;
-    }
+    float nv[ML_SL];   // n_t of this key dim over the segment (fully unrolled: registers)
+#pragma unroll
+    for (int j = 0; j < ML_SL; ++j)
+        if (j < cnt) {
+            n = se[j] * n + si[j] * to_f(sk[j * Dk + d]);
+            nv[j] = n;
+        }
+#pragma unroll
+    for (int j = ML_SL - 1; j >= 0; --j)
+        if (j < cnt) {
+            const long o = (r0 + j) * Dk + d;
+            const float sdj = sd[j], it = si[j], kt = to_f(sk[j * Dk + d]), nj = nv[j];
+            const float dn = sdj * to_f(sq[j * Dk + d]) + c;
+            dq[o] = from_f<T>(to_f(sa[j * Dk + d]) + sdj * nj);
+            dk[o] = from_f<T>(to_f(sb[j * Dk + d]) + it * dn);
+            ml_warp_part<8>(kt * dn, pi, j);
+            ml_warp_part<8>((nj - it * kt) * dn, pg, j);
+            c = se[j] * dn;
+        }
     __syncthreads();
     if (d < cnt) {
         float xi = 0.f, xg = 0.f;
@@ -755,13 +757,12 @@ gla_status ml_bwd(const gla_problem* p, const MlLayout& w, const void* q, const 
         const dim3 grid(w.nseg, (unsigned)BH);
         int* status = reinterpret_cast<int*>(ws);
         const size_t s1 = ml_smem_bytes(p->Dk, sizeof(To));
-        const size_t sb = ml_smem_bytes(p->Dk, 2 * sizeof(To) + 2 * sizeof(Ta) + sizeof(float));
+        const size_t sb = ml_smem_bytes(p->Dk, 2 * sizeof(To) + 2 * sizeof(Ta));
         static bool attr = false;
         if (!attr) {
             cudaError_t ea = ml_smem_attr(k_mlstm_dnloc<To>, ml_smem_bytes(256, sizeof(To)));
             if (ea == cudaSuccess)
-                ea = ml_smem_attr(k_mlstm_den_bwd<To, Ta>,
-                                  ml_smem_bytes(256, 2 * sizeof(To) + 2 * sizeof(Ta) + sizeof(float)));
+                ea = ml_smem_attr(k_mlstm_den_bwd<To, Ta>, ml_smem_bytes(256, 2 * sizeof(To) + 2 * sizeof(Ta)));
             if (ea != cudaSuccess) return record_cuda(ea, "mLSTM normaliser shared-memory attribute");
             attr = true;
         }
