@@ -36,9 +36,6 @@ namespace {
 constexpr int ML_NT = 256;
 constexpr int ML_SL = 32;   // tokens per segment of the normaliser recurrence
 
-template <typename T>
-__device__ __forceinline__ float ld_f(const T* p) { return to_f(*p); }
-
 // Per head: c = max_t i~_t, and the input gate e^{i~_t - c} (<= 1) for the two passes.
 __global__ void __launch_bounds__(ML_NT) k_mlstm_prep(const float* __restrict__ itil, int L, float* __restrict__ ig,
                                                       float* __restrict__ cst) {
