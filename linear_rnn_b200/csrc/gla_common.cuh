@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/gla.h"
 
 namespace gla {
@@ -35,6 +37,24 @@ constexpr int kDevStatusRange = 2;
 // times O(Dk) products) and down to e^-|Gamma| (q e^b): at |Gamma| = 70 the largest stays about
 // 1e4 below the fp32 / bf16 maximum and the smallest above the smallest normal.
 constexpr float kMinTileLogDecay = -70.f;
+
+// Devices a process may drive, for the per-device host state (launch attributes, streams).
+constexpr int kMaxDevices = 64;
+
+// Raises the dynamic shared-memory limit of `kern` to `bytes` on the current device, once per
+// device and call site (`seen`, one flag per device): the attribute belongs to the device's
+// context, so a process that launches on several devices sets it on each.
+template <typename K>
+inline cudaError_t smem_attr_once(K kern, size_t bytes, std::atomic<bool> (&seen)[kMaxDevices]) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (seen[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) seen[dev].store(true, std::memory_order_release);
+    return e;
+}
 
 // Launch accounting (gla_api.cu): every kernel launch of the library goes through
 // GLA_LAUNCH, which counts it and, while the profiler is enabled, brackets it with CUDA

@@ -418,10 +418,6 @@ __global__ void __launch_bounds__(256) k_mlstm_den_bwd(const T* __restrict__ q, 
 inline size_t ml_smem_bytes(int Dk, size_t tile_elem_bytes) {
     return MlSmem::TILES + (size_t)ML_SL * Dk * tile_elem_bytes;
 }
-template <typename K>
-inline cudaError_t ml_smem_attr(K kern, size_t bytes) {
-    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-}
 
 // Eight consecutive elements (16 bytes of bf16, 32 of fp32) to / from fp32.
 __device__ __forceinline__ void ld8(const float* p, float* f) {
@@ -673,12 +669,11 @@ gla_status ml_forward_passes(const gla_problem* p, const MlLayout& w, const MlIn
     const dim3 grid(w.nseg, (unsigned)BH);
     int* status = reinterpret_cast<int*>(ws);
     const size_t s1 = ml_smem_bytes(p->Dk, sizeof(To)), s2 = ml_smem_bytes(p->Dk, 2 * sizeof(To));
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t ea = ml_smem_attr(k_mlstm_nloc<To>, ml_smem_bytes(256, sizeof(To)));
-        if (ea == cudaSuccess) ea = ml_smem_attr(k_mlstm_den<To>, ml_smem_bytes(256, 2 * sizeof(To)));
+    static std::atomic<bool> attr_nloc[kMaxDevices], attr_den[kMaxDevices];
+    {
+        cudaError_t ea = smem_attr_once(k_mlstm_nloc<To>, ml_smem_bytes(256, sizeof(To)), attr_nloc);
+        if (ea == cudaSuccess) ea = smem_attr_once(k_mlstm_den<To>, ml_smem_bytes(256, 2 * sizeof(To)), attr_den);
         if (ea != cudaSuccess) return record_cuda(ea, "mLSTM normaliser shared-memory attribute");
-        attr = true;
     }
     GLA_LAUNCH("mlstm_nloc", st,
                k_mlstm_nloc<To><<<grid, p->Dk, s1, st>>>(tk, g, r.ig, p->L, p->Dk, w.nseg, nloc, r.gam, status));
@@ -755,13 +750,13 @@ gla_status ml_bwd(const gla_problem* p, const MlLayout& w, const void* q, const 
         int* status = reinterpret_cast<int*>(ws);
         const size_t s1 = ml_smem_bytes(p->Dk, sizeof(To));
         const size_t sb = ml_smem_bytes(p->Dk, 2 * sizeof(To) + 2 * sizeof(Ta));
-        static bool attr = false;
-        if (!attr) {
-            cudaError_t ea = ml_smem_attr(k_mlstm_dnloc<To>, ml_smem_bytes(256, sizeof(To)));
+        static std::atomic<bool> attr_dnloc[kMaxDevices], attr_dbwd[kMaxDevices];
+        {
+            cudaError_t ea = smem_attr_once(k_mlstm_dnloc<To>, ml_smem_bytes(256, sizeof(To)), attr_dnloc);
             if (ea == cudaSuccess)
-                ea = ml_smem_attr(k_mlstm_den_bwd<To, Ta>, ml_smem_bytes(256, 2 * sizeof(To) + 2 * sizeof(Ta)));
+                ea = smem_attr_once(k_mlstm_den_bwd<To, Ta>, ml_smem_bytes(256, 2 * sizeof(To) + 2 * sizeof(Ta)),
+                                    attr_dbwd);
             if (ea != cudaSuccess) return record_cuda(ea, "mLSTM normaliser shared-memory attribute");
-            attr = true;
         }
         GLA_LAUNCH("mlstm_dnloc", st,
                    k_mlstm_dnloc<To><<<grid, p->Dk, s1, st>>>(tq, g, dden, p->L, p->Dk, w.nseg, p->scale, cloc, status));

@@ -27,7 +27,7 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_static_scratch[GLA_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
+using gla::kMaxDevices;
 std::mutex g_mu;
 // Per device: the array's device address and the id of the CUDA context it was looked up in.
 // A device reset (cudaDeviceReset) ends that context and the next one loads the array anew, so

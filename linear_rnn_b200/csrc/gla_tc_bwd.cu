@@ -1408,11 +1408,10 @@ __global__ void __launch_bounds__(NT_B, 1)
 // reverse scan run beside the dq kernel (they do not depend on it): their CTAs fill the SMs the
 // dq kernel's last partial wave leaves idle. nullptr if it cannot be created.
 static cudaStream_t aux_stream() {
-    constexpr int kMaxDev = 64;
-    static std::once_flag once[kMaxDev];
-    static cudaStream_t streams[kMaxDev];
+    static std::once_flag once[kMaxDevices];
+    static cudaStream_t streams[kMaxDevices];
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     std::call_once(once[dev], [dev] {
         if (cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess) streams[dev] = nullptr;
     });
@@ -1505,11 +1504,10 @@ static cudaError_t launch_dq(const Dims& P, const BwdPlan& pl, const CUtensorMap
                              const CUtensorMap& mdq, const BwdArgs& a, cudaStream_t st) {
     using C = QCfg<DKB, DV, GATE>;
     auto kern = k_tc_bwd_dq<DKB, DV, GATE>;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    static std::atomic<bool> attr[kMaxDevices];
+    {
+        const cudaError_t e = smem_attr_once(kern, C::SMEM, attr);
         if (e != cudaSuccess) return e;
-        attr = true;
     }
     dim3 grid(P.B * P.H, P.Dk / DKB, pl.nseg);
     GLA_LAUNCH("tc_bwd_dq", st, kern<<<grid, NT_B, C::SMEM, st>>>(mq, mk, mg, mv, mo, mdq, a, P));
@@ -1523,11 +1521,10 @@ static cudaError_t launch_dkdv(const Dims& P, const BwdPlan& pl, const CUtensorM
                                bool pdl) {
     using C = KVCfg<DK, DV, GATE>;
     auto kern = k_tc_bwd_dkdv<DK, DV, GATE, KS>;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    static std::atomic<bool> attr[kMaxDevices];
+    {
+        const cudaError_t e = smem_attr_once(kern, C::SMEM, attr);
         if (e != cudaSuccess) return e;
-        attr = true;
     }
     // the two key blocks of a (b*h, segment) run as one cluster of two CTAs; with pdl the kernel
     // may start before the kernel ahead of it in the stream (reverse scan or dq) ends, and waits

@@ -929,11 +929,10 @@ static cudaError_t launch_one(const CUtensorMap& mq, const CUtensorMap& mk, cons
                               cudaStream_t st, bool pdl = false) {
     using C = Cfg<DK, DVT, GATE, MODE>;
     auto kern = k_tc_fwd<DK, DVT, GATE, MODE>;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    static std::atomic<bool> attr[kMaxDevices];
+    {
+        const cudaError_t e = smem_attr_once(kern, C::SMEM, attr);
         if (e != cudaSuccess) return e;
-        attr = true;
     }
     dim3 grid(P.B * P.H, P.Dv / DVT, nseg);
     cudaError_t e = cudaSuccess;
